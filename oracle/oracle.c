@@ -1,0 +1,263 @@
+/*
+ * oracle.c -- TEST INFRASTRUCTURE ONLY.  The plain, slow, single-threaded
+ * fp64 CPU statement of what sparse-graph causal attention computes.  Only
+ * tests/, the smoke check and the bench's CPU-baseline leg load it; the
+ * library never does.  It shares no code, header or table with the CUDA path.
+ *
+ * Sources (web pages; section names as printed on them):
+ *  - "SpatialLM-Mini sped up training with a 16K context by 2.47x on an
+ *    RTX 3050", section "How tokens choose whom to listen to": the allowed
+ *    positions of a token are itself, a few nearby predecessors and the
+ *    positions at distance 1, 2, 4, 8, ...; no position ahead; the list is
+ *    fixed in advance.
+ *  - "MiniGPT (Part 6)", section "A mask is not enough", first listing: the
+ *    window keeps key j for query i when j <= i and i - j < w.  Second
+ *    listing (chunked_swa): scores are (q . k) * scale, masked, then softmax
+ *    over the kept keys, then multiplied with V.
+ *  - "Longer Attention Span: Increasing Transformer Context Length with
+ *    Sparse Graph Processing Techniques", Abstract: tokens are graph nodes,
+ *    the mask gives the edges, and only the needed (edge) computations are
+ *    performed.
+ *
+ * Everything is written as the plain definition: per query, loop over its
+ * neighbour list, fp64 arithmetic, no blocking, no reordering.
+ *
+ * Element types of the attention inputs: 0 = bf16 (raw uint16 bits),
+ * 1 = fp32, 2 = fp64.  Conversions to double are exact.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_OK 0
+#define OR_BAD_ROWPTR 1
+#define OR_LOOKAHEAD 2
+#define OR_NEGATIVE 3
+#define OR_BAD_ARG 4
+#define OR_NOMEM 5
+
+/* ---------- element access ---------- */
+
+static double elem(const void *base, int dtype, int64_t idx) {
+    if (dtype == 0) {
+        uint16_t h = ((const uint16_t *)base)[idx];
+        uint32_t bits = ((uint32_t)h) << 16; /* bf16 is the top half of fp32 */
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    if (dtype == 1) return (double)((const float *)base)[idx];
+    return ((const double *)base)[idx];
+}
+
+static int cmp_i32(const void *a, const void *b) {
+    int32_t x = *(const int32_t *)a, y = *(const int32_t *)b;
+    return (x > y) - (x < y);
+}
+
+/* ---------- graph: the fixed neighbour set ---------- */
+
+/* Number of neighbours of query i: the window {i-W+1..i} clipped at 0,
+ * plus the distances 2^k (k from exps[]) that reach a position >= 0 and are
+ * not already inside the window.  Written by listing the set and counting. */
+static int64_t structured_row(int64_t i, int32_t W, const int32_t *exps, int32_t n_exps,
+                              int32_t *buf /* may be NULL */) {
+    int64_t cnt = 0;
+    int64_t lo = i - (int64_t)W + 1;
+    if (lo < 0) lo = 0;
+    for (int64_t j = lo; j <= i; ++j) {
+        if (buf) buf[cnt] = (int32_t)j;
+        ++cnt;
+    }
+    /* distance links; each distinct distance appears once */
+    for (int32_t a = 0; a < n_exps; ++a) {
+        int32_t k = exps[a];
+        if (k < 0 || k > 62) continue;
+        int dup = 0;
+        for (int32_t b = 0; b < a; ++b)
+            if (exps[b] == k) dup = 1;
+        if (dup) continue;
+        int64_t dist = (int64_t)1 << k;
+        int64_t j = i - dist;
+        if (j < 0) continue;          /* no position before the start */
+        if (j >= lo) continue;        /* already in the window */
+        if (buf) buf[cnt] = (int32_t)j;
+        ++cnt;
+    }
+    if (buf) qsort(buf, (size_t)cnt, sizeof(int32_t), cmp_i32);
+    return cnt;
+}
+
+int64_t oracle_graph_structured_nnz(int64_t T, int32_t W, const int32_t *exps, int32_t n_exps) {
+    int64_t nnz = 0;
+    for (int64_t i = 0; i < T; ++i) nnz += structured_row(i, W, exps, n_exps, NULL);
+    return nnz;
+}
+
+/* rowptr[T+1], colidx[nnz]; each row ascending. */
+int oracle_graph_structured(int64_t T, int32_t W, const int32_t *exps, int32_t n_exps,
+                            int64_t *rowptr, int32_t *colidx) {
+    if (T < 0 || W < 1) return OR_BAD_ARG;
+    rowptr[0] = 0;
+    for (int64_t i = 0; i < T; ++i) {
+        int64_t c = structured_row(i, W, exps, n_exps, colidx + rowptr[i]);
+        rowptr[i + 1] = rowptr[i] + c;
+    }
+    return OR_OK;
+}
+
+/* Normalise a caller's neighbour lists: per row sort ascending and drop
+ * repeats; reject a key after the query (no look-ahead), a negative key and
+ * a malformed row pointer.  out_rowptr[T+1], out_colidx[<= nnz_in].
+ * Returns the status; *nnz_out gets the normalised edge count. */
+int oracle_graph_normalize(int64_t T, const int64_t *rowptr, const int32_t *colidx,
+                           int64_t *out_rowptr, int32_t *out_colidx, int64_t *nnz_out) {
+    if (T < 0) return OR_BAD_ARG;
+    if (rowptr[0] != 0) return OR_BAD_ROWPTR;
+    for (int64_t i = 0; i < T; ++i)
+        if (rowptr[i + 1] < rowptr[i]) return OR_BAD_ROWPTR;
+    for (int64_t i = 0; i < T; ++i)
+        for (int64_t e = rowptr[i]; e < rowptr[i + 1]; ++e) {
+            if (colidx[e] < 0) return OR_NEGATIVE;
+            if ((int64_t)colidx[e] > i) return OR_LOOKAHEAD;
+        }
+    int64_t w = 0;
+    out_rowptr[0] = 0;
+    for (int64_t i = 0; i < T; ++i) {
+        int64_t n = rowptr[i + 1] - rowptr[i];
+        int32_t *row = out_colidx + w;
+        memcpy(row, colidx + rowptr[i], (size_t)n * sizeof(int32_t));
+        qsort(row, (size_t)n, sizeof(int32_t), cmp_i32);
+        int64_t u = 0;
+        for (int64_t e = 0; e < n; ++e)
+            if (u == 0 || row[u - 1] != row[e]) row[u++] = row[e];
+        w += u;
+        out_rowptr[i + 1] = w;
+    }
+    *nnz_out = w;
+    return OR_OK;
+}
+
+/* Transpose: for key j, the queries i with j in N(i), ascending in i. */
+int oracle_graph_reverse(int64_t T, const int64_t *rowptr, const int32_t *colidx,
+                         int64_t *rev_rowptr, int32_t *rev_colidx) {
+    int64_t nnz = rowptr[T];
+    int64_t *fill = (int64_t *)calloc((size_t)T + 1, sizeof(int64_t));
+    if (!fill) return OR_NOMEM;
+    for (int64_t e = 0; e < nnz; ++e) fill[colidx[e] + 1] += 1;
+    rev_rowptr[0] = 0;
+    for (int64_t j = 0; j < T; ++j) rev_rowptr[j + 1] = rev_rowptr[j] + fill[j + 1];
+    for (int64_t j = 0; j < T; ++j) fill[j] = rev_rowptr[j];
+    for (int64_t i = 0; i < T; ++i) /* ascending i keeps each list sorted */
+        for (int64_t e = rowptr[i]; e < rowptr[i + 1]; ++e) {
+            int32_t j = colidx[e];
+            rev_colidx[fill[j]++] = (int32_t)i;
+        }
+    free(fill);
+    return OR_OK;
+}
+
+/* ---------- attention over the graph ---------- */
+
+/* One query row: s_j = scale * q.k_j for j in its list; m = max s;
+ * l = sum exp(s_j - m); out = sum exp(s_j - m) v_j / l; lse = m + ln l.
+ * An empty list gives out = 0 and lse = -inf. */
+static void row_forward(int32_t D, int dtype, const void *q, int64_t qrow, const void *k,
+                        const void *v, const int32_t *nbr, int64_t deg, double scale,
+                        double *s /* scratch[deg] */, double *out, double *lse) {
+    for (int32_t d = 0; d < D; ++d) out[d] = 0.0;
+    if (deg == 0) {
+        *lse = -INFINITY;
+        return;
+    }
+    double m = -INFINITY;
+    for (int64_t e = 0; e < deg; ++e) {
+        int64_t j = nbr[e];
+        double dot = 0.0;
+        for (int32_t d = 0; d < D; ++d)
+            dot += elem(q, dtype, qrow * D + d) * elem(k, dtype, j * D + d);
+        s[e] = scale * dot;
+        if (s[e] > m) m = s[e];
+    }
+    double l = 0.0;
+    for (int64_t e = 0; e < deg; ++e) l += exp(s[e] - m);
+    for (int64_t e = 0; e < deg; ++e) {
+        int64_t j = nbr[e];
+        double p = exp(s[e] - m) / l;
+        for (int32_t d = 0; d < D; ++d) out[d] += p * elem(v, dtype, j * D + d);
+    }
+    *lse = m + log(l);
+}
+
+static int64_t max_degree(int64_t nq, const int64_t *rowptr) {
+    int64_t mx = 0;
+    for (int64_t i = 0; i < nq; ++i)
+        if (rowptr[i + 1] - rowptr[i] > mx) mx = rowptr[i + 1] - rowptr[i];
+    return mx;
+}
+
+/* Forward for nq query rows.  Query row r is q[r*D..]; its neighbours are
+ * colidx[rowptr[r]..rowptr[r+1]), indexing rows of k and v.  out[nq*D],
+ * lse[nq] (natural log). */
+int oracle_attn_fwd(int64_t nq, int32_t D, int dtype, const void *q, const void *k,
+                    const void *v, const int64_t *rowptr, const int32_t *colidx, double scale,
+                    double *out, double *lse) {
+    if (nq < 0 || D < 1 || dtype < 0 || dtype > 2) return OR_BAD_ARG;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(max_degree(nq, rowptr) + 1));
+    if (!s) return OR_NOMEM;
+    for (int64_t r = 0; r < nq; ++r)
+        row_forward(D, dtype, q, r, k, v, colidx + rowptr[r], rowptr[r + 1] - rowptr[r], scale, s,
+                    out + r * D, lse + r);
+    free(s);
+    return OR_OK;
+}
+
+/* Backward of the forward above for upstream gradient dout[nq*D].
+ * For each query i (its own fp64 forward recomputed):
+ *   P_ij = exp(s_ij - lse_i), dP_ij = dO_i . v_j, Delta_i = dO_i . out_i,
+ *   dS_ij = P_ij (dP_ij - Delta_i),
+ *   dQ_i += scale * dS_ij k_j,  dK_j += scale * dS_ij q_i,  dV_j += P_ij dO_i.
+ * dq[nq*D]; dk, dv [nk*D] are overwritten (zeroed first).  dK_j and dV_j
+ * are complete for every key whose queries are all among the nq rows. */
+int oracle_attn_bwd(int64_t nq, int64_t nk, int32_t D, int dtype, const void *q, const void *k,
+                    const void *v, const void *dout, const int64_t *rowptr, const int32_t *colidx,
+                    double scale, double *dq, double *dk, double *dv) {
+    if (nq < 0 || nk < 0 || D < 1 || dtype < 0 || dtype > 2) return OR_BAD_ARG;
+    int64_t mdeg = max_degree(nq, rowptr);
+    double *s = (double *)malloc(sizeof(double) * (size_t)(mdeg + 1));
+    double *o = (double *)malloc(sizeof(double) * (size_t)D);
+    if (!s || !o) {
+        free(s);
+        free(o);
+        return OR_NOMEM;
+    }
+    memset(dq, 0, sizeof(double) * (size_t)(nq * D));
+    memset(dk, 0, sizeof(double) * (size_t)(nk * D));
+    memset(dv, 0, sizeof(double) * (size_t)(nk * D));
+    for (int64_t i = 0; i < nq; ++i) {
+        const int32_t *nbr = colidx + rowptr[i];
+        int64_t deg = rowptr[i + 1] - rowptr[i];
+        double lse;
+        row_forward(D, dtype, q, i, k, v, nbr, deg, scale, s, o, &lse);
+        if (deg == 0) continue;
+        double delta = 0.0;
+        for (int32_t d = 0; d < D; ++d) delta += elem(dout, dtype, i * D + d) * o[d];
+        for (int64_t e = 0; e < deg; ++e) {
+            int64_t j = nbr[e];
+            double p = exp(s[e] - lse);
+            double dp = 0.0;
+            for (int32_t d = 0; d < D; ++d)
+                dp += elem(dout, dtype, i * D + d) * elem(v, dtype, j * D + d);
+            double ds = p * (dp - delta);
+            for (int32_t d = 0; d < D; ++d) {
+                dq[i * D + d] += scale * ds * elem(k, dtype, j * D + d);
+                dk[j * D + d] += scale * ds * elem(q, dtype, i * D + d);
+                dv[j * D + d] += p * elem(dout, dtype, i * D + d);
+            }
+        }
+    }
+    free(s);
+    free(o);
+    return OR_OK;
+}

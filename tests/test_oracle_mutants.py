@@ -1,0 +1,54 @@
+"""Plants plausible mistakes in copies of the oracle source (on the CPU) and
+checks that at least one pin catches each: a dropped term, a wrong sign, a
+wrong index, a transposed operand, an off-by-one window, a wrong log base.
+The committed oracle source is never modified."""
+import os
+
+import pytest
+
+import oracle
+import pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTANTS = {
+    "window_off_by_one": ("int64_t lo = i - (int64_t)W + 1;", "int64_t lo = i - (int64_t)W;"),
+    "distance_not_deduplicated": ("if (j >= lo) continue;", "if (j > i) continue;"),
+    "scale_dropped": ("s[e] = scale * dot;", "s[e] = dot;"),
+    "max_not_subtracted": ("for (int64_t e = 0; e < deg; ++e) l += exp(s[e] - m);",
+                           "for (int64_t e = 0; e < deg; ++e) l += exp(s[e]);"),
+    "lse_log2": ("*lse = m + log(l);", "*lse = m + log2(l);"),
+    "delta_sign": ("double ds = p * (dp - delta);", "double ds = p * (dp + delta);"),
+    "dk_transposed_operand": ("dk[j * D + d] += scale * ds * elem(q, dtype, i * D + d);",
+                              "dk[j * D + d] += scale * ds * elem(k, dtype, i * D + d);"),
+    "dq_scale_dropped": ("dq[i * D + d] += scale * ds * elem(k, dtype, j * D + d);",
+                         "dq[i * D + d] += ds * elem(k, dtype, j * D + d);"),
+    "dv_prob_dropped": ("dv[j * D + d] += p * elem(dout, dtype, i * D + d);",
+                        "dv[j * D + d] += elem(dout, dtype, i * D + d);"),
+    "dv_wrong_row": ("dv[j * D + d] += p * elem(dout, dtype, i * D + d);",
+                     "dv[i * D + d] += p * elem(dout, dtype, i * D + d);"),
+    "reverse_stores_key": ("rev_colidx[fill[j]++] = (int32_t)i;",
+                           "rev_colidx[fill[j]++] = (int32_t)j;"),
+    "normalize_keeps_repeats": ("if (u == 0 || row[u - 1] != row[e]) row[u++] = row[e];",
+                                "row[u++] = row[e];"),
+    "lookahead_accepted": ("if ((int64_t)colidx[e] > i) return OR_LOOKAHEAD;",
+                           "if ((int64_t)colidx[e] > i + 1) return OR_LOOKAHEAD;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    before, after = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, "mutation site not found: " + name
+    mpath = tmp_path / "oracle_mutant.c"
+    mpath.write_text(src.replace(before, after))
+    lib = oracle.build(str(mpath), str(tmp_path / "liboracle_mutant.so"))
+    o = oracle.Oracle(lib)
+    caught = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(o)
+        except (AssertionError, oracle.OracleError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, "no pin caught mutant " + name

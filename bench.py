@@ -1,0 +1,394 @@
+"""Benchmark of sparse-graph causal attention on B200.
+
+    python bench.py --gpus N --steps K --warmup W [--workload NAME] [--impl reference]
+
+One step = the whole hot path over one batch of synthetic input: build the
+neighbour graph, forward (out, lse) and backward (dq, dk, dv).  The default
+workload is the 16,384-token layer of "SpatialLM-Mini ..." (B1 H4 T16384 D64
+bf16, window 32 + distance links 2^k, k = 0..13).  The headline value is
+query-key edges per second of fwd+bwd, summed over all ranks; every rank runs
+its own replica (the heads of a batch are independent problems: weak scaling,
+no collective on the data path).
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by its own CUDA
+events on the launching stream, with a 256 MiB buffer written between steps
+so that no step finds its inputs in the 126 MB L2; barrier + synchronize on
+both sides; the max over ranks.  A second pass records per-kernel events for
+the roofline of the dominant kernel; a third measures the same step end to
+end from pinned host buffers (copies inside the timed region).  nvidia-smi
+samples the clocks during the timed region.
+
+``--impl reference`` times the CPU oracle (the plain fp64 statement of the
+method) on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "sparse-attn query-key edges/s (fwd, fwd+bwd) at T=16K and % of roofline"
+
+# Algorithmic (compulsory) bytes of each kernel per (b, h) slice: every input
+# row read once and every output row written once.  es = element size.
+#   fwd                      q, k, v read; out written; lse written
+#   bwd, dQ (+ Delta)        q, k, v, out, dout read; dq written; lse read; Delta written
+#   bwd, dK/dV               q, k, v, dout read; dk, dv written; lse, Delta read
+KERNEL_BYTES = {
+    "fwd": lambda T, D, es: 4 * T * D * es + 4 * T,
+    "bwd_dq": lambda T, D, es: 6 * T * D * es + 8 * T,
+    "bwd_dkdv": lambda T, D, es: 6 * T * D * es + 8 * T,
+}
+
+
+def kernel_class(name: str) -> str:
+    if name.endswith("bwd_dq"):
+        return "bwd_dq"
+    if name.endswith("bwd_dkdv"):
+        return "bwd_dkdv"
+    return "fwd"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def edge_count(w: synth.Workload, g) -> int:
+    return int(g.nnz) * w.B * w.H
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    mhz.append(float(f[1]))
+                    mx = float(f[2])
+                except ValueError:
+                    continue
+                for n, val in zip(names, f[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(n)
+            os.unlink(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def dist_setup(n_gpus):
+    if n_gpus > 1 or "WORLD_SIZE" in os.environ and int(os.environ["WORLD_SIZE"]) > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+        return dist, dist.get_rank(), dist.get_world_size()
+    return None, 0, 1
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def cpu_oracle_run(w: synth.Workload, seconds: float, seed_rows: int = 7):
+    """Time the oracle as it stands on rows of slice 0 of the workload (fwd +
+    bwd), growing the row sample until about `seconds` of CPU work.  Returns
+    (edges/s, edges, seconds, description)."""
+    import oracle
+    o = oracle.get()
+    x = synth.make_qkv(w, device="cpu", with_dout=True)
+    D, T = w.D, w.T
+
+    def host(name, rows):
+        t = x[name].view(w.B * w.H, T, D)[0][torch.as_tensor(rows)]
+        if w.dtype == "bf16":
+            return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+        return t.contiguous().numpy()
+
+    n_rows, done_edges, done_s = 256, 0, 0.0
+    rng = np.random.default_rng(seed_rows)
+    while done_s < seconds and n_rows <= T:
+        rows = np.sort(rng.choice(T, size=n_rows, replace=False)).astype(np.int64)
+        rp, ci = o.structured_rows(rows, w.W, w.exps)
+        keys, local = np.unique(ci, return_inverse=True)
+        q, do = host("q", rows), host("dout", rows)
+        k, v = host("k", keys), host("v", keys)
+        t0 = time.perf_counter()
+        o.fwd(q, k, v, rp, local.astype(np.int32), w.scale, dtype=w.dtype)
+        o.bwd(q, k, v, do, rp, local.astype(np.int32), w.scale, dtype=w.dtype)
+        done_s += time.perf_counter() - t0
+        done_edges += int(rp[-1])
+        n_rows = min(T, n_rows * 2)
+        if n_rows == T and done_s > seconds / 4:
+            break
+    desc = (f"fwd+bwd of {done_edges} edges: random query rows of slice 0 of {w.name}, "
+            f"oracle single-threaded fp64 C")
+    return done_edges / done_s, done_edges, done_s, desc
+
+
+def run_reference(args, dist, rank, world):
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    per_step = max(0.5, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_oracle_run(w, per_step / 4)
+    edges, secs = 0, 0.0
+    for _ in range(args.steps):
+        _, e, s, desc = cpu_oracle_run(w, per_step)
+        edges += e
+        secs += s
+    v = edges / secs
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "edges/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "W": w.W,
+                       "dilation_exps": list(w.exps), "pass": "fwd+bwd",
+                       "parallelism": "replicas"},
+            "cpu_baseline": {"value": v, "unit": "edges/s", "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": "edges/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- GPU arm
+
+def run_gpu(args, dist, rank, world):
+    import sparse_graph_causal_b200 as sa
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    stream = torch.cuda.current_stream()
+    x = synth.make_qkv(w, device=dev, seed=w.seed + 17 * rank)
+    q, k, v, dout = x["q"], x["k"], x["v"], x["dout"]
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    g0 = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+    ws = torch.empty(sa.sparse_attn_bwd_workspace_size(q, g0), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    E = edge_count(w, g0)
+    do_bwd = w.bwd and not args.fwd_only
+
+    def step():
+        g = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+        sa.sparse_attn_fwd(q, k, v, g, w.scale, out=out, lse=lse)
+        if do_bwd:
+            sa.sparse_attn_bwd(q, k, v, out, lse, dout, g, w.scale, dq=dq, dk=dk, dv=dv,
+                               workspace=ws)
+        g.close()
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1)
+        step()
+    sa.sparse_attn_check_device()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, L2 flushed between steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    launches0 = sa.sparse_attn_launch_count()
+    with ClockSampler(local) as clk:
+        barrier(dist)
+        torch.cuda.synchronize()
+        for a, b in evs:
+            flush.fill_(1)
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        barrier(dist)
+    launches = sa.sparse_attn_launch_count() - launches0
+    sa.sparse_attn_check_device()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = max_over_ranks(dist, sum(ms))
+    ms_step = total_ms / args.steps
+    value = E * world / (ms_step * 1e-3)
+
+    # ---- per-kernel event timing (separate pass) for the roofline
+    sa.sparse_attn_profile_begin(True)
+    for _ in range(args.steps):
+        flush.fill_(1)
+        step()
+    prof = sa.sparse_attn_profile_end()
+    kt = {n: (c, t) for n, (c, t) in prof.items() if not n.startswith("graph_")}
+    dom = max(kt, key=lambda n: kt[n][1])
+    cnt, tot = kt[dom]
+    avg_ms = tot / cnt
+    es = 2 if w.dtype == "bf16" else 4
+    alg_bytes = KERNEL_BYTES[kernel_class(dom)](w.T, w.D, es) * w.B * w.H
+    hbm, tflops, src = peaks()
+    achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
+    shares = {n: round(t / sum(tt for _, tt in kt.values()), 4) for n, (_, t) in kt.items()}
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": None, "kernel": dom,
+                "kernel_ms": avg_ms, "algorithmic_bytes": alg_bytes,
+                "peak_source": f"{src} hbm_gbs", "kernel_shares": shares}
+
+    # ---- fwd-only throughput
+    fwd_ms = []
+    for _ in range(min(args.steps, 50)):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        gg = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+        sa.sparse_attn_fwd(q, k, v, gg, w.scale, out=out, lse=lse)
+        b.record(stream)
+        gg.close()
+        fwd_ms.append((a, b))
+    torch.cuda.synchronize()
+    fwd_ms = max_over_ranks(dist, sum(a.elapsed_time(b) for a, b in fwd_ms) / len(fwd_ms))
+
+    # ---- end to end from pinned host memory, through the public API
+    hx = {n: t.cpu().pin_memory() for n, t in x.items()}
+    hout = {n: torch.empty(q.shape, dtype=q.dtype).pin_memory() for n in ("out", "dq", "dk", "dv")}
+    h2d = sum(t.numel() * t.element_size() for n, t in hx.items() if do_bwd or n != "dout")
+    d2h = sum(t.numel() * t.element_size() for n, t in hout.items() if do_bwd or n == "out")
+
+    def e2e_step():
+        for n in ("q", "k", "v") + (("dout",) if do_bwd else ()):
+            x[n].copy_(hx[n], non_blocking=True)
+        step()
+        hout["out"].copy_(out, non_blocking=True)
+        if do_bwd:
+            hout["dq"].copy_(dq, non_blocking=True)
+            hout["dk"].copy_(dk, non_blocking=True)
+            hout["dv"].copy_(dv, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_evs = []
+    n_e2e = min(args.steps, 50)
+    barrier(dist)
+    for _ in range(n_e2e):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        e_evs.append((a, b))
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(dist, sum(a.elapsed_time(b) for a, b in e_evs) / n_e2e)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v_cpu, e_cpu, s_cpu, desc = cpu_oracle_run(w, args.cpu_seconds)
+        cpu = {"value": v_cpu, "unit": "edges/s", "cores": 1, "kind": "oracle",
+               "sample": f"{desc}; {s_cpu:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "W": w.W,
+                       "dilation_exps": list(w.exps), "edges_per_replica": E,
+                       "pass": "fwd+bwd" if do_bwd else "fwd",
+                       "l2": "256 MiB buffer written between timed steps",
+                       "parallelism": f"replicas x{world}"},
+            "fwd_edges_per_s": E * world / (fwd_ms * 1e-3), "fwd_ms": fwd_ms,
+            "tokens_per_s": w.B * w.T * world / (ms_step * 1e-3),
+            "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": E * world / (e2e_ms * 1e-3), "unit": "edges/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches, "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    g0.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="spatiallm_16k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    dist, rank, world = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, dist, rank, world)
+        else:
+            run_gpu(args, dist, rank, world)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -71,6 +71,8 @@ class Oracle:
         L.oracle_graph_structured_nnz.argtypes = [i64, i32, vp, i32]
         L.oracle_graph_structured.restype = ctypes.c_int
         L.oracle_graph_structured.argtypes = [i64, i32, vp, i32, vp, vp]
+        L.oracle_graph_structured_rows.restype = ctypes.c_int
+        L.oracle_graph_structured_rows.argtypes = [i64, vp, i32, vp, i32, vp, vp]
         L.oracle_graph_normalize.restype = ctypes.c_int
         L.oracle_graph_normalize.argtypes = [i64, vp, vp, vp, vp, vp]
         L.oracle_graph_reverse.restype = ctypes.c_int
@@ -96,6 +98,23 @@ class Oracle:
         if st:
             raise OracleError(STATUS[st])
         return rowptr, colidx[:nnz]
+
+    def structured_rows(self, rows, W: int, exps):
+        """Neighbour lists of the given query positions only (any T):
+        (rowptr int64[len(rows)+1], colidx int32[...])."""
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        e = np.ascontiguousarray(np.asarray(list(exps), dtype=np.int32))
+        rowptr = np.zeros(len(rows) + 1, dtype=np.int64)
+        st = self.lib.oracle_graph_structured_rows(len(rows), _ptr(rows), W, _ptr(e), len(e),
+                                                   _ptr(rowptr), None)
+        if st:
+            raise OracleError(STATUS[st])
+        colidx = np.zeros(max(int(rowptr[-1]), 1), dtype=np.int32)
+        st = self.lib.oracle_graph_structured_rows(len(rows), _ptr(rows), W, _ptr(e), len(e),
+                                                   _ptr(rowptr), _ptr(colidx))
+        if st:
+            raise OracleError(STATUS[st])
+        return rowptr, colidx[: int(rowptr[-1])]
 
     def normalize(self, rowptr, colidx):
         """Sort + deduplicate every row; raises OracleError on an invalid graph."""

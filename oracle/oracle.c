@@ -107,6 +107,20 @@ int oracle_graph_structured(int64_t T, int32_t W, const int32_t *exps, int32_t n
     return OR_OK;
 }
 
+/* The lists of selected rows only (for sampled checks of long sequences):
+ * rows[0..n), rowptr[n+1]; pass colidx = NULL to get rowptr alone. */
+int oracle_graph_structured_rows(int64_t n, const int64_t *rows, int32_t W, const int32_t *exps,
+                                 int32_t n_exps, int64_t *rowptr, int32_t *colidx) {
+    if (n < 0 || W < 1) return OR_BAD_ARG;
+    rowptr[0] = 0;
+    for (int64_t r = 0; r < n; ++r) {
+        if (rows[r] < 0) return OR_BAD_ARG;
+        int64_t c = structured_row(rows[r], W, exps, n_exps, colidx ? colidx + rowptr[r] : NULL);
+        rowptr[r + 1] = rowptr[r] + c;
+    }
+    return OR_OK;
+}
+
 /* Normalise a caller's neighbour lists: per row sort ascending and drop
  * repeats; reject a key after the query (no look-ahead), a negative key and
  * a malformed row pointer.  out_rowptr[T+1], out_colidx[<= nnz_in].
@@ -160,11 +174,19 @@ int oracle_graph_reverse(int64_t T, const int64_t *rowptr, const int32_t *colidx
 
 /* ---------- attention over the graph ---------- */
 
+/* Exact copy of n elements of any input type into a new fp64 array. */
+static double *to_f64(const void *base, int dtype, int64_t n) {
+    double *a = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    if (!a) return NULL;
+    for (int64_t x = 0; x < n; ++x) a[x] = elem(base, dtype, x);
+    return a;
+}
+
 /* One query row: s_j = scale * q.k_j for j in its list; m = max s;
  * l = sum exp(s_j - m); out = sum exp(s_j - m) v_j / l; lse = m + ln l.
  * An empty list gives out = 0 and lse = -inf. */
-static void row_forward(int32_t D, int dtype, const void *q, int64_t qrow, const void *k,
-                        const void *v, const int32_t *nbr, int64_t deg, double scale,
+static void row_forward(int32_t D, const double *q, int64_t qrow, const double *k,
+                        const double *v, const int32_t *nbr, int64_t deg, double scale,
                         double *s /* scratch[deg] */, double *out, double *lse) {
     for (int32_t d = 0; d < D; ++d) out[d] = 0.0;
     if (deg == 0) {
@@ -175,8 +197,7 @@ static void row_forward(int32_t D, int dtype, const void *q, int64_t qrow, const
     for (int64_t e = 0; e < deg; ++e) {
         int64_t j = nbr[e];
         double dot = 0.0;
-        for (int32_t d = 0; d < D; ++d)
-            dot += elem(q, dtype, qrow * D + d) * elem(k, dtype, j * D + d);
+        for (int32_t d = 0; d < D; ++d) dot += q[qrow * D + d] * k[j * D + d];
         s[e] = scale * dot;
         if (s[e] > m) m = s[e];
     }
@@ -185,7 +206,7 @@ static void row_forward(int32_t D, int dtype, const void *q, int64_t qrow, const
     for (int64_t e = 0; e < deg; ++e) {
         int64_t j = nbr[e];
         double p = exp(s[e] - m) / l;
-        for (int32_t d = 0; d < D; ++d) out[d] += p * elem(v, dtype, j * D + d);
+        for (int32_t d = 0; d < D; ++d) out[d] += p * v[j * D + d];
     }
     *lse = m + log(l);
 }
@@ -204,13 +225,25 @@ int oracle_attn_fwd(int64_t nq, int32_t D, int dtype, const void *q, const void 
                     const void *v, const int64_t *rowptr, const int32_t *colidx, double scale,
                     double *out, double *lse) {
     if (nq < 0 || D < 1 || dtype < 0 || dtype > 2) return OR_BAD_ARG;
+    int64_t nk = 0; /* key rows referenced: 1 + the largest index */
+    for (int64_t e = 0; e < rowptr[nq]; ++e)
+        if ((int64_t)colidx[e] + 1 > nk) nk = (int64_t)colidx[e] + 1;
     double *s = (double *)malloc(sizeof(double) * (size_t)(max_degree(nq, rowptr) + 1));
-    if (!s) return OR_NOMEM;
-    for (int64_t r = 0; r < nq; ++r)
-        row_forward(D, dtype, q, r, k, v, colidx + rowptr[r], rowptr[r + 1] - rowptr[r], scale, s,
-                    out + r * D, lse + r);
+    double *qd = to_f64(q, dtype, nq * D), *kd = to_f64(k, dtype, nk * D);
+    double *vd = to_f64(v, dtype, nk * D);
+    int st = OR_OK;
+    if (!s || !qd || !kd || !vd) {
+        st = OR_NOMEM;
+    } else {
+        for (int64_t r = 0; r < nq; ++r)
+            row_forward(D, qd, r, kd, vd, colidx + rowptr[r], rowptr[r + 1] - rowptr[r], scale, s,
+                        out + r * D, lse + r);
+    }
     free(s);
-    return OR_OK;
+    free(qd);
+    free(kd);
+    free(vd);
+    return st;
 }
 
 /* Backward of the forward above for upstream gradient dout[nq*D].
@@ -227,10 +260,12 @@ int oracle_attn_bwd(int64_t nq, int64_t nk, int32_t D, int dtype, const void *q,
     int64_t mdeg = max_degree(nq, rowptr);
     double *s = (double *)malloc(sizeof(double) * (size_t)(mdeg + 1));
     double *o = (double *)malloc(sizeof(double) * (size_t)D);
-    if (!s || !o) {
-        free(s);
-        free(o);
-        return OR_NOMEM;
+    double *qd = to_f64(q, dtype, nq * D), *kd = to_f64(k, dtype, nk * D);
+    double *vd = to_f64(v, dtype, nk * D), *dod = to_f64(dout, dtype, nq * D);
+    int st = OR_OK;
+    if (!s || !o || !qd || !kd || !vd || !dod) {
+        st = OR_NOMEM;
+        goto done;
     }
     memset(dq, 0, sizeof(double) * (size_t)(nq * D));
     memset(dk, 0, sizeof(double) * (size_t)(nk * D));
@@ -239,25 +274,29 @@ int oracle_attn_bwd(int64_t nq, int64_t nk, int32_t D, int dtype, const void *q,
         const int32_t *nbr = colidx + rowptr[i];
         int64_t deg = rowptr[i + 1] - rowptr[i];
         double lse;
-        row_forward(D, dtype, q, i, k, v, nbr, deg, scale, s, o, &lse);
+        row_forward(D, qd, i, kd, vd, nbr, deg, scale, s, o, &lse);
         if (deg == 0) continue;
         double delta = 0.0;
-        for (int32_t d = 0; d < D; ++d) delta += elem(dout, dtype, i * D + d) * o[d];
+        for (int32_t d = 0; d < D; ++d) delta += dod[i * D + d] * o[d];
         for (int64_t e = 0; e < deg; ++e) {
             int64_t j = nbr[e];
             double p = exp(s[e] - lse);
             double dp = 0.0;
-            for (int32_t d = 0; d < D; ++d)
-                dp += elem(dout, dtype, i * D + d) * elem(v, dtype, j * D + d);
+            for (int32_t d = 0; d < D; ++d) dp += dod[i * D + d] * vd[j * D + d];
             double ds = p * (dp - delta);
             for (int32_t d = 0; d < D; ++d) {
-                dq[i * D + d] += scale * ds * elem(k, dtype, j * D + d);
-                dk[j * D + d] += scale * ds * elem(q, dtype, i * D + d);
-                dv[j * D + d] += p * elem(dout, dtype, i * D + d);
+                dq[i * D + d] += scale * ds * kd[j * D + d];
+                dk[j * D + d] += scale * ds * qd[i * D + d];
+                dv[j * D + d] += p * dod[i * D + d];
             }
         }
     }
+done:
     free(s);
     free(o);
-    return OR_OK;
+    free(qd);
+    free(kd);
+    free(vd);
+    free(dod);
+    return st;
 }

@@ -1,0 +1,122 @@
+// sa_internal.cuh -- shared internals of libsparse_attn (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sparse_attn.h"
+
+#define SA_MAX_OFFSETS 63
+
+// Library-side graph.  A structured graph is implicit (W + distances); its
+// CSR arrays exist only when materialised.  A CSR graph always holds its
+// normalised lists and their transpose.
+struct sa_graph_s {
+    int64_t T = 0;
+    int kind = 0;           // 0 structured, 1 CSR
+    int32_t W = 0;          // structured: window; CSR: verified band (0 = none)
+    int32_t n_off = 0;      // structured: distances >= W and < T
+    int64_t offs[SA_MAX_OFFSETS] = {0};  // descending
+    int64_t nnz = 0;
+    int materialized = 0;
+    int64_t *rowptr = nullptr;
+    int32_t *colidx = nullptr;
+    int64_t *rev_rowptr = nullptr;
+    int32_t *rev_colidx = nullptr;
+    int32_t max_resid = 0;      // max edges outside the band over rows
+    int32_t max_resid_rev = 0;  // max transpose edges outside the band over keys
+    int device = 0;
+};
+
+// Everything a kernel needs to enumerate N(i) and its transpose.
+struct GraphView {
+    int64_t T;
+    int32_t kind;
+    int32_t W;      // window (structured) or band (CSR)
+    int32_t n_off;
+    int64_t offs[SA_MAX_OFFSETS];  // descending
+    const int64_t *rowptr;
+    const int32_t *colidx;
+    const int64_t *rev_rowptr;
+    const int32_t *rev_colidx;
+};
+
+GraphView make_view(const sa_graph_s *g);
+
+// Launch accounting, optional per-kernel event timing, the device error word.
+void sa_count_launch(int n = 1);
+void sa_prof_begin(const char *kernel, cudaStream_t s);
+void sa_prof_end(cudaStream_t s);
+#define SA_LAUNCH(name, s, ...)        \
+    do {                               \
+        sa_prof_begin(name, s);        \
+        __VA_ARGS__;                   \
+        sa_prof_end(s);                \
+        sa_count_launch();             \
+    } while (0)
+int *sa_device_error_word();  // device address of this device's error word
+
+#define SA_DEVERR_TIMEOUT 1
+#define SA_DEVERR_BOUNDS 2
+
+// Closed forms of the structured graph (host and device).
+__host__ __device__ inline int64_t sg_window_prefix(int64_t i, int64_t W) {
+    // sum_{i' < i} min(i' + 1, W)
+    if (i <= W) return i * (i + 1) / 2;
+    return W * (W + 1) / 2 + (i - W) * W;
+}
+
+__host__ __device__ inline int64_t sg_rowptr(int64_t i, int64_t W, int n_off, const int64_t *offs) {
+    int64_t r = sg_window_prefix(i, W);
+    for (int a = 0; a < n_off; ++a) r += (i > offs[a]) ? (i - offs[a]) : 0;
+    return r;
+}
+
+__host__ __device__ inline int64_t sg_degree(int64_t i, int64_t W, int n_off, const int64_t *offs) {
+    int64_t d = (i + 1 < W) ? i + 1 : W;
+    for (int a = 0; a < n_off; ++a) d += (offs[a] <= i) ? 1 : 0;
+    return d;
+}
+
+__host__ __device__ inline int64_t sg_rev_rowptr(int64_t j, int64_t T, int64_t W, int n_off,
+                                                 const int64_t *offs) {
+    // sum_{j' < j} [ min(T - j', W) + #{o : j' + o < T} ]
+    int64_t lim = T - W + 1;
+    if (lim < 0) lim = 0;
+    int64_t a = j < lim ? j : lim;  // keys j' < a have a full window of queries
+    int64_t r = a * W + (j - a) * T - (a + j - 1) * (j - a) / 2;
+    for (int b = 0; b < n_off; ++b) {
+        int64_t c = T - offs[b];
+        if (c < 0) c = 0;
+        r += j < c ? j : c;
+    }
+    return r;
+}
+
+__host__ __device__ inline int64_t sg_in_degree(int64_t j, int64_t T, int64_t W, int n_off,
+                                                const int64_t *offs) {
+    int64_t d = (T - j < W) ? T - j : W;
+    for (int b = 0; b < n_off; ++b) d += (j + offs[b] < T) ? 1 : 0;
+    return d;
+}
+
+// CUDA error helpers (host)
+#define SA_CUDA_TRY(expr)                                   \
+    do {                                                    \
+        cudaError_t _e = (expr);                            \
+        if (_e != cudaSuccess) return SA_ERR_CUDA;          \
+    } while (0)
+
+// Internal launchers (graph.cu)
+sa_status sa_graph_materialize_structured(sa_graph_s *g, cudaStream_t s);
+sa_status sa_graph_from_csr(sa_graph_s *g, const int64_t *rowptr, const int32_t *colidx,
+                            int64_t nnz, int32_t band, cudaStream_t s);
+
+// Internal launchers (attn_gather.cu): every edge on CUDA cores.
+sa_status sa_gather_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                        const GraphView &gv, float scale, sa_tensor *out, float *lse,
+                        cudaStream_t s);
+sa_status sa_gather_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                        const sa_tensor *out, const float *lse, const sa_tensor *dout,
+                        const GraphView &gv, float scale, sa_tensor *dq, sa_tensor *dk,
+                        sa_tensor *dv, float *delta, cudaStream_t s);

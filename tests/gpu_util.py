@@ -1,0 +1,112 @@
+"""Host-side helpers of the GPU parity tests: moving the exact tensors the
+GPU used to the oracle, building the local neighbour lists of sampled rows,
+and the tolerance checks.  No attention arithmetic lives here.
+
+Tolerances (bf16 inputs, fp32 accumulation): max-abs 2e-2 and mean-abs 2e-3
+on out/lse/dq/dk/dv; fp32 inputs: max-abs 1e-4.  Because some workloads have
+outputs far below 1 (inputs N(0,1)/sqrt(D)), each comparison also bounds the
+error relative to the reference's own range: max-abs <= REL * max|ref| with
+REL = 2^-5 for bf16 (a few bf16 roundings of 2^-9 each, summed over the
+softmax-weighted terms) and 1e-4 for fp32.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+TOL = {"bf16": dict(max_abs=2e-2, mean_abs=2e-3, rel=2.0 ** -5),
+       "fp32": dict(max_abs=1e-4, mean_abs=1e-4, rel=1e-4)}
+
+
+def to_oracle(t: torch.Tensor, dtype: str) -> np.ndarray:
+    """Exact host copy in the oracle's input encoding (bf16 as raw bits)."""
+    t = t.detach().contiguous().cpu()
+    if dtype == "bf16":
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def compare(got, ref: np.ndarray, dtype: str, what: str, scale_floor: float = 1e-6):
+    """got: torch tensor (any float dtype) or ndarray; ref: fp64 ndarray."""
+    if isinstance(got, torch.Tensor):
+        got = got.detach().float().cpu().numpy()
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    fin = np.isfinite(ref)
+    # -inf (empty rows) must match exactly
+    assert np.array_equal(np.isfinite(got), fin), what + ": non-finite pattern differs"
+    assert np.all(got[~fin] == ref[~fin]), what + ": non-finite values differ"
+    if not fin.any():
+        return dict(max_abs=0.0, mean_abs=0.0)
+    err = np.abs(got[fin] - ref[fin])
+    tol = TOL[dtype]
+    mx, mean = float(err.max()), float(err.mean())
+    rng = max(float(np.abs(ref[fin]).max()), scale_floor)
+    assert mx <= tol["max_abs"], f"{what}: max-abs {mx:.3e} > {tol['max_abs']}"
+    assert mean <= tol["mean_abs"], f"{what}: mean-abs {mean:.3e} > {tol['mean_abs']}"
+    assert mx <= tol["rel"] * rng + 1e-7, f"{what}: max-abs {mx:.3e} > {tol['rel']} * {rng:.3e}"
+    return dict(max_abs=mx, mean_abs=mean, range=rng)
+
+
+def local_rows(o, rows, W=None, exps=(), csr=None):
+    """Neighbour lists of sampled query rows: from the oracle's structured
+    graph, or sliced from a (host) CSR (rowptr, colidx) already normalised by
+    the oracle."""
+    rows = np.asarray(rows, dtype=np.int64)
+    if csr is None:
+        return o.structured_rows(rows, W, exps)
+    rp, ci = csr
+    counts = rp[rows + 1] - rp[rows]
+    rowptr = np.zeros(len(rows) + 1, dtype=np.int64)
+    rowptr[1:] = np.cumsum(counts)
+    colidx = np.concatenate([ci[rp[i]:rp[i + 1]] for i in rows]).astype(np.int32) \
+        if len(rows) else np.zeros(0, np.int32)
+    return rowptr, colidx
+
+
+def compact(rowptr, colidx):
+    """Map global key indices of a set of lists to 0..n-1: returns (keys,
+    local colidx)."""
+    keys, inv = np.unique(colidx, return_inverse=True)
+    return keys.astype(np.int64), inv.astype(np.int32)
+
+
+def gather_rows(t: torch.Tensor, bh: int, rows: np.ndarray, dtype: str) -> np.ndarray:
+    """Rows of slice bh of a [B, H, T, D] tensor, copied to the host."""
+    B, H, T, D = t.shape
+    flat = t.view(B * H, T, D)[bh]
+    idx = torch.as_tensor(rows, dtype=torch.int64, device=t.device)
+    return to_oracle(flat.index_select(0, idx), dtype)
+
+
+def oracle_fwd_rows(o, qkv, bh, rows, rowptr, colidx, scale, dtype):
+    keys, local = compact(rowptr, colidx)
+    q = gather_rows(qkv["q"], bh, rows, dtype)
+    k = gather_rows(qkv["k"], bh, keys, dtype)
+    v = gather_rows(qkv["v"], bh, keys, dtype)
+    return o.fwd(q, k, v, rowptr, local, scale, dtype=dtype)
+
+
+def oracle_dq_rows(o, qkv, bh, rows, rowptr, colidx, scale, dtype):
+    keys, local = compact(rowptr, colidx)
+    q = gather_rows(qkv["q"], bh, rows, dtype)
+    do = gather_rows(qkv["dout"], bh, rows, dtype)
+    k = gather_rows(qkv["k"], bh, keys, dtype)
+    v = gather_rows(qkv["v"], bh, keys, dtype)
+    dq, _, _ = o.bwd(q, k, v, do, rowptr, local, scale, dtype=dtype)
+    return dq
+
+
+def oracle_dkdv_keys(o, qkv, bh, key_rows, query_rows, rowptr, colidx, scale, dtype):
+    """dK, dV of key_rows; query_rows must hold every query whose list
+    contains one of them, with (rowptr, colidx) their lists."""
+    keys, local = compact(rowptr, colidx)
+    q = gather_rows(qkv["q"], bh, query_rows, dtype)
+    do = gather_rows(qkv["dout"], bh, query_rows, dtype)
+    k = gather_rows(qkv["k"], bh, keys, dtype)
+    v = gather_rows(qkv["v"], bh, keys, dtype)
+    _, dk, dv = o.bwd(q, k, v, do, rowptr, local, scale, dtype=dtype)
+    pos = np.searchsorted(keys, key_rows)
+    assert np.array_equal(keys[pos], key_rows)
+    return dk[pos], dv[pos]

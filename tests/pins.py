@@ -104,6 +104,16 @@ def pin_graph_closed_forms(o):
     assert o.structured_nnz(16384, 32, range(0, 14)) == 654896
 
 
+def pin_graph_rows_match_full(o):
+    """Selected-row lists equal the same rows of the full graph."""
+    for T, W, exps in GRAPH_CASES:
+        rowptr, colidx = o.structured(T, W, exps)
+        rows = np.array(sorted(set([0, T - 1, T // 2, T // 3])), dtype=np.int64)
+        rr, rc = o.structured_rows(rows, W, exps)
+        for n, i in enumerate(rows):
+            assert np.array_equal(rc[rr[n]:rr[n + 1]], colidx[rowptr[i]:rowptr[i + 1]])
+
+
 def pin_graph_reverse(o):
     for T, W, exps in GRAPH_CASES:
         rowptr, colidx = o.structured(T, W, exps)
@@ -336,7 +346,8 @@ def pin_bwd_invariants(o):
     assert np.allclose(dq2, 0.0, rtol=0, atol=1e-12)
 
 
-ALL_PINS = [pin_graph_golden, pin_graph_bruteforce, pin_graph_closed_forms, pin_graph_reverse,
+ALL_PINS = [pin_graph_golden, pin_graph_bruteforce, pin_graph_closed_forms,
+            pin_graph_rows_match_full, pin_graph_reverse,
             pin_graph_normalize, pin_fwd_golden, pin_fwd_structured_rows_golden,
             pin_fwd_full_causal, pin_fwd_dense, pin_fwd_invariants, pin_fwd_empty_rows,
             pin_bwd_golden, pin_bwd_finite_differences, pin_bwd_dense_autograd,

@@ -1,0 +1,149 @@
+"""GPU forward/backward against the CPU oracle, element by element, on
+sizes the oracle finishes in seconds: several 128-row tiles, ragged tails,
+every supported head size and dtype, structured and CSR graphs, and both
+kernel paths (tcgen05 band tiles + gather, and gather only)."""
+import math
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_util import compare, to_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sa():
+    import sparse_graph_causal_b200 as m
+    return m
+
+
+def _wl(name, B, H, T, D, dtype, W, exps=(), std=1.0, seed=1, csr=None, band=0):
+    w = synth.Workload(name=name, B=B, H=H, T=T, D=D, dtype=dtype, W=W, exps=tuple(exps),
+                       input_std=std, scale=1.0 / math.sqrt(D), seed=seed, band_hint=band,
+                       csr=csr is not None)
+    return w, csr
+
+
+def _random_csr_with_empty(T, seed):
+    rng = np.random.default_rng(seed)
+    rows = []
+    for i in range(T):
+        n = 0 if i % 7 == 3 else int(rng.integers(1, 12))
+        rows.append(list(rng.integers(0, i + 1, size=n)))
+    rp = np.zeros(T + 1, np.int64)
+    rp[1:] = np.cumsum([len(r) for r in rows])
+    return rp, np.array([x for r in rows for x in r], np.int32)
+
+
+CASES = [
+    _wl("tiny", 1, 2, 256, 32, "fp32", 8, range(0, 8), seed=1001),
+    _wl("tiny_full", 1, 2, 256, 32, "fp32", 256, (), seed=1001),
+    _wl("t1", 1, 1, 1, 64, "bf16", 4, range(0, 3)),
+    _wl("d64_ragged", 2, 2, 300, 64, "bf16", 32, range(0, 9)),
+    _wl("d64_self_only", 1, 2, 129, 64, "bf16", 1, (0, 3, 5)),
+    _wl("d64_full", 1, 1, 520, 64, "bf16", 520, ()),
+    _wl("d64_small_values", 1, 4, 700, 64, "bf16", 32, range(0, 10), std=0.125),
+    _wl("d128_w200", 1, 2, 1000, 128, "bf16", 200, (8, 9)),
+    _wl("d128_band", 2, 1, 777, 128, "bf16", 256, ()),
+    _wl("d32_bf16", 1, 2, 200, 32, "bf16", 16, range(0, 8)),
+    _wl("d64_fp32", 1, 2, 333, 64, "fp32", 40, range(0, 9)),
+    _wl("d128_fp32", 1, 1, 150, 128, "fp32", 64, (7,)),
+    _wl("csr_view_3000", 1, 2, 3000, 64, "bf16", 0, (),
+        csr=synth.csr_random_rows(3000, seed=9), band=64),
+    _wl("csr_empty_rows", 1, 2, 400, 64, "bf16", 0, (), csr=_random_csr_with_empty(400, 4)),
+    _wl("csr_d128", 1, 1, 600, 128, "bf16", 0, (), csr=synth.csr_random_rows(600, seed=8), band=64),
+]
+
+
+def build_graph(sa, o, w, csr):
+    if csr is None:
+        g = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+        rp, ci = o.structured(w.T, w.W, w.exps)
+    else:
+        rp_raw, ci_raw = csr
+        g = sa.sparse_attn_graph_build_csr(torch.from_numpy(rp_raw).cuda(),
+                                           torch.from_numpy(ci_raw).cuda(), band_hint=w.band_hint)
+        rp, ci = o.normalize(rp_raw, ci_raw)
+    return g, rp, ci
+
+
+def run_and_check(sa, o, w, csr, path):
+    sa.sparse_attn_set_path(path)
+    try:
+        g, rp, ci = build_graph(sa, o, w, csr)
+        x = synth.make_qkv(w, device="cuda")
+        out, lse = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+        dq, dk, dv = sa.sparse_attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], g, w.scale)
+        sa.sparse_attn_check_device()
+    finally:
+        sa.sparse_attn_set_path(sa.SA_PATH_AUTO)
+    BH = w.B * w.H
+    for bh in range(BH):
+        sl = [to_oracle(x[n].view(BH, w.T, w.D)[bh], w.dtype) for n in ("q", "k", "v", "dout")]
+        rout, rlse = o.fwd(sl[0], sl[1], sl[2], rp, ci, w.scale, dtype=w.dtype)
+        rdq, rdk, rdv = o.bwd(sl[0], sl[1], sl[2], sl[3], rp, ci, w.scale, dtype=w.dtype)
+        tag = f"{w.name}[bh={bh},path={path}]"
+        compare(out.view(BH, w.T, w.D)[bh], rout, w.dtype, tag + " out")
+        compare(lse.view(BH, w.T)[bh], rlse, w.dtype, tag + " lse")
+        compare(dq.view(BH, w.T, w.D)[bh], rdq, w.dtype, tag + " dq")
+        compare(dk.view(BH, w.T, w.D)[bh], rdk, w.dtype, tag + " dk")
+        compare(dv.view(BH, w.T, w.D)[bh], rdv, w.dtype, tag + " dv")
+
+
+@pytest.mark.parametrize("path", [0, 1], ids=["auto", "gather"])
+@pytest.mark.parametrize("case", CASES, ids=lambda c: c[0].name)
+def test_parity_small(sa, oracle_lib, case, path):
+    w, csr = case
+    run_and_check(sa, oracle_lib, w, csr, path)
+
+
+@pytest.mark.parametrize("path", [0, 1], ids=["auto", "gather"])
+def test_causality_bitwise(sa, path):
+    """Changing q/k/v at positions > i leaves rows <= i bitwise unchanged."""
+    w = synth.WORKLOADS["spatiallm_16k"]
+    w = replace(w, T=2000)
+    sa.sparse_attn_set_path(path)
+    try:
+        g = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+        x = synth.make_qkv(w, device="cuda", with_dout=False)
+        out, lse = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+        i0 = 1234
+        for n in ("q", "k", "v"):
+            x[n][:, :, i0 + 1:] = torch.randn_like(x[n][:, :, i0 + 1:])
+        out2, lse2 = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+    finally:
+        sa.sparse_attn_set_path(0)
+    assert torch.equal(out[:, :, : i0 + 1], out2[:, :, : i0 + 1])
+    assert torch.equal(lse[:, :, : i0 + 1], lse2[:, :, : i0 + 1])
+    assert not torch.equal(out[:, :, i0 + 1:], out2[:, :, i0 + 1:])
+
+
+def test_backward_deterministic(sa):
+    w = replace(synth.WORKLOADS["spatiallm_16k"], T=4096)
+    g = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+    x = synth.make_qkv(w, device="cuda")
+    out, lse = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+    r1 = sa.sparse_attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], g, w.scale)
+    r2 = sa.sparse_attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], g, w.scale)
+    for a, b in zip(r1, r2):
+        assert torch.equal(a, b)
+
+
+def test_argument_errors(sa):
+    w = replace(synth.WORKLOADS["spatiallm_16k"], T=256)
+    g = sa.sparse_attn_graph_build_structured(300, w.W, list(w.exps))
+    x = synth.make_qkv(w, device="cuda", with_dout=False)
+    with pytest.raises(sa.SparseAttentionError) as e:     # T mismatch
+        sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+    assert e.value.status == sa.SA_ERR_INVALID_ARG
+    g = sa.sparse_attn_graph_build_structured(256, w.W, list(w.exps))
+    with pytest.raises(sa.SparseAttentionError):           # non-finite scale
+        sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, float("nan"))
+    q48 = torch.zeros(1, 1, 256, 48, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sa.SparseAttentionError) as e:      # head size
+        sa.sparse_attn_fwd(q48, q48, q48, g, 1.0)
+    assert e.value.status == sa.SA_ERR_UNSUPPORTED

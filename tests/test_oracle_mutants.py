@@ -19,14 +19,16 @@ MUTANTS = {
                            "for (int64_t e = 0; e < deg; ++e) l += exp(s[e]);"),
     "lse_log2": ("*lse = m + log(l);", "*lse = m + log2(l);"),
     "delta_sign": ("double ds = p * (dp - delta);", "double ds = p * (dp + delta);"),
-    "dk_transposed_operand": ("dk[j * D + d] += scale * ds * elem(q, dtype, i * D + d);",
-                              "dk[j * D + d] += scale * ds * elem(k, dtype, i * D + d);"),
-    "dq_scale_dropped": ("dq[i * D + d] += scale * ds * elem(k, dtype, j * D + d);",
-                         "dq[i * D + d] += ds * elem(k, dtype, j * D + d);"),
-    "dv_prob_dropped": ("dv[j * D + d] += p * elem(dout, dtype, i * D + d);",
-                        "dv[j * D + d] += elem(dout, dtype, i * D + d);"),
-    "dv_wrong_row": ("dv[j * D + d] += p * elem(dout, dtype, i * D + d);",
-                     "dv[i * D + d] += p * elem(dout, dtype, i * D + d);"),
+    "dk_transposed_operand": ("dk[j * D + d] += scale * ds * qd[i * D + d];",
+                              "dk[j * D + d] += scale * ds * kd[i * D + d];"),
+    "dq_scale_dropped": ("dq[i * D + d] += scale * ds * kd[j * D + d];",
+                         "dq[i * D + d] += ds * kd[j * D + d];"),
+    "dv_prob_dropped": ("dv[j * D + d] += p * dod[i * D + d];",
+                        "dv[j * D + d] += dod[i * D + d];"),
+    "dv_wrong_row": ("dv[j * D + d] += p * dod[i * D + d];",
+                     "dv[i * D + d] += p * dod[i * D + d];"),
+    "delta_from_values": ("delta += dod[i * D + d] * o[d];",
+                          "delta += dod[i * D + d] * vd[i * D + d];"),
     "reverse_stores_key": ("rev_colidx[fill[j]++] = (int32_t)i;",
                            "rev_colidx[fill[j]++] = (int32_t)j;"),
     "normalize_keeps_repeats": ("if (u == 0 || row[u - 1] != row[e]) row[u++] = row[e];",

@@ -1,0 +1,33 @@
+// tmap.cu -- see tmap.cuh.
+#include <mutex>
+
+#include "tmap.cuh"
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_once;
+
+void load_encode() {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+}  // namespace
+
+bool sa_tmap_bf16_3d(CUtensorMap *m, const void *base, uint64_t D, uint64_t T, uint64_t BH,
+                     uint32_t box_rows) {
+    std::call_once(g_once, load_encode);
+    if (!g_encode) return false;
+    cuuint64_t dims[3] = {D, T, BH};
+    cuuint64_t strides[2] = {D * 2, T * D * 2};  // bytes, dims 1 and 2
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}

@@ -4,8 +4,8 @@ Causal attention restricted to a fixed sparse neighbour graph on NVIDIA B200
 (sm_100a).  Every computation runs in the library's CUDA kernels; this module
 only marshals torch tensors (device memory) and the current CUDA stream into
 the C ABI declared in include/sparse_attn.h, under the same names.  There is
-no CPU fallback: importing fails loudly when the library is not built, and
-every call raises when the library reports an error.
+no CPU fallback: the library is loaded on first use and every call raises
+when it is not built or when it reports an error.
 """
 from __future__ import annotations
 
@@ -22,16 +22,14 @@ SA_ERR_OOM, SA_ERR_CUDA, SA_ERR_DEVICE_TIMEOUT = 4, 5, 6
 SA_BF16, SA_FP32 = 0, 1
 SA_PATH_AUTO, SA_PATH_GATHER = 0, 1
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built: run `python -m sparse_graph_causal_b200.build`")
-
-
 class SaTensor(ctypes.Structure):
     _fields_ = [("ptr", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("B", ctypes.c_int64),
                 ("H", ctypes.c_int64), ("T", ctypes.c_int64), ("D", ctypes.c_int64)]
 
 
 def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built: run `python -m sparse_graph_causal_b200.build`")
     lib = ctypes.CDLL(LIB_PATH)
     i64, i32, vp, st = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int
     P = ctypes.POINTER
@@ -60,7 +58,19 @@ def _load():
     return lib
 
 
-_lib = _load()
+class _LazyLib:
+    """The loaded library, opened on first attribute access."""
+
+    def __init__(self):
+        self._lib = None
+
+    def __getattr__(self, name):
+        if self._lib is None:
+            self._lib = _load()
+        return getattr(self._lib, name)
+
+
+_lib = _LazyLib()
 
 
 class SparseAttentionError(RuntimeError):

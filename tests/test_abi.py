@@ -46,6 +46,7 @@ def test_host_side_rejections():
     import sparse_graph_causal_b200 as sa
     lib = sa._lib
     h = ctypes.c_void_p()
+    assert lib.sparse_attn_launch_count() >= 0
     # bad sizes are rejected before any CUDA call
     assert lib.sparse_attn_graph_build_structured(0, 4, None, 0, 0, None, ctypes.byref(h)) == 1
     assert lib.sparse_attn_graph_build_structured(16, 0, None, 0, 0, None, ctypes.byref(h)) == 1

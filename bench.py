@@ -196,7 +196,7 @@ def run_reference(args, dist, rank, world):
     if rank != 0:
         return
     w = synth.WORKLOADS[args.workload]
-    per_step = max(0.5, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = min(args.cpu_seconds, max(0.5, min(3.0, 150.0 / max(1, args.steps + args.warmup))))
     for _ in range(args.warmup):
         cpu_oracle_run(w, per_step / 4)
     edges, secs = 0, 0.0

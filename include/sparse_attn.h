@@ -138,6 +138,27 @@ sa_status sparse_attn_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
                           float scale, sa_tensor *dq, sa_tensor *dk, sa_tensor *dv,
                           void *workspace, size_t ws_bytes, void *stream);
 
+/* Backward that allocates nothing and takes no workspace, for callers that
+ * cannot allocate device memory at the call site: a host running under a
+ * fixed device-memory plan (every byte reserved up front), or code inside an
+ * allocator hook, where allocating again would re-enter the allocator.  The
+ * pages have no counterpart of this call; it is a deployment convenience.
+ * Same arguments and results as sparse_attn_bwd minus the workspace.  Its
+ * scratch (Delta, 4 bytes per query row) is a fixed device array of
+ * SA_NOALLOC_MAX_ROWS floats inside the library: every GPU that loads the
+ * library holds it (4 MiB) until the process exits.  B*H*T above
+ * SA_NOALLOC_MAX_ROWS returns SA_ERR_UNSUPPORTED before anything is enqueued.
+ * Every call on a device shares the array (it keeps the last call's
+ * contents, none of which must start at zero), so calls whose work overlaps
+ * on the GPU race: serialise them (one stream, or events).  The first call
+ * on each device looks up the array's device address; make that first call
+ * before any stream capture. */
+#define SA_NOALLOC_MAX_ROWS (1 << 20)
+sa_status sparse_attn_bwd_noalloc(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                                  const sa_tensor *out, const float *lse, const sa_tensor *dout,
+                                  sa_graph g, float scale, sa_tensor *dq, sa_tensor *dk,
+                                  sa_tensor *dv, void *stream);
+
 /* ------------------------------------------------------------ utilities */
 
 /* Human-readable name of a status. */

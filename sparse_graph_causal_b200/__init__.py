@@ -49,6 +49,9 @@ def _load():
         "sparse_attn_set_path": (st, [i32]),
         "sparse_attn_check_device": (st, [vp]),
         "sparse_attn_launch_count": (i64, []),
+        "sparse_attn_bwd_noalloc": (st, [P(SaTensor), P(SaTensor), P(SaTensor), P(SaTensor), vp,
+                                         P(SaTensor), vp, ctypes.c_float, P(SaTensor),
+                                         P(SaTensor), P(SaTensor), vp]),
         "sparse_attn_profile_begin": (st, [i32]),
         "sparse_attn_profile_end": (i32, [ctypes.c_char_p, i32, P(i32), P(ctypes.c_double), i32]),
     }
@@ -232,6 +235,31 @@ def sparse_attn_bwd(q, k, v, out, lse, dout, g: Graph, scale: float, dq=None, dk
                                 workspace.numel() * workspace.element_size(), _stream(stream)),
            "sparse_attn_bwd")
     return dq, dk, dv
+
+
+def sparse_attn_bwd_noalloc(q, k, v, out, lse, dout, g: Graph, scale: float, dq=None, dk=None,
+                            dv=None, stream=None):
+    """sparse_attn_bwd without a workspace: for callers that cannot allocate
+    device memory when they call it.  The library keeps its scratch in a
+    fixed device array (B*H*T <= SA_NOALLOC_MAX_ROWS); calls that overlap on
+    the GPU race on it.  Output tensors passed in are written, not
+    allocated; the defaults below allocate them here, in Python, for
+    convenience."""
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32")
+    ts = [_tensor(x, n) for x, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout"),
+                                     (dq, "dq"), (dk, "dk"), (dv, "dv"))]
+    r = [ctypes.byref(t) for t in ts]
+    _check(_lib.sparse_attn_bwd_noalloc(r[0], r[1], r[2], r[3], lse.data_ptr(), r[4], g.handle,
+                                        float(scale), r[5], r[6], r[7], _stream(stream)),
+           "sparse_attn_bwd_noalloc")
+    return dq, dk, dv
+
+
+SA_NOALLOC_MAX_ROWS = 1 << 20
 
 
 # ---------------------------------------------------------------- utilities

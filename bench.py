@@ -53,6 +53,11 @@ KERNEL_BYTES = {
     "bwd_dq": lambda T, D, es: 6 * T * D * es + 8 * T,
     "bwd_dkdv": lambda T, D, es: 6 * T * D * es + 8 * T,
 }
+# Algorithmic FLOPs per edge: forward 4D (q.k and p.v); backward 10D split as
+# dQ kernel 6D (S recompute, dP, dQ) and dK/dV kernel 4D (dV, dK); the dK/dV
+# kernel's own recomputation of S and dP is not counted.
+KERNEL_FLOPS_PER_EDGE = {"fwd": lambda D: 4 * D, "bwd_dq": lambda D: 6 * D,
+                         "bwd_dkdv": lambda D: 4 * D}
 
 
 def kernel_class(name: str) -> str:
@@ -285,14 +290,25 @@ def run_gpu(args, dist, rank, world):
     cnt, tot = kt[dom]
     avg_ms = tot / cnt
     es = 2 if w.dtype == "bf16" else 4
-    alg_bytes = KERNEL_BYTES[kernel_class(dom)](w.T, w.D, es) * w.B * w.H
+    kc = kernel_class(dom)
+    alg_bytes = KERNEL_BYTES[kc](w.T, w.D, es) * w.B * w.H
+    alg_flops = KERNEL_FLOPS_PER_EDGE[kc](w.D) * E
     hbm, tflops, src = peaks()
-    achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
     shares = {n: round(t / sum(tt for _, tt in kt.values()), 4) for n, (_, t) in kt.items()}
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": None, "kernel": dom,
-                "kernel_ms": avg_ms, "algorithmic_bytes": alg_bytes,
-                "peak_source": f"{src} hbm_gbs", "kernel_shares": shares}
+    # the kernel's bound: compulsory intensity against the machine balance
+    tensor_bound = alg_flops / alg_bytes > (tflops * 1e12) / (hbm * 1e9) and w.dtype == "bf16"
+    if tensor_bound:
+        achieved = alg_flops / (avg_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": tflops, "unit": "TFLOP/s",
+                    "frac": achieved / tflops, "peak_source": f"{src} bf16_tflops"}
+    else:
+        achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "peak_source": f"{src} hbm_gbs"}
+    roofline.update({"traffic": None, "kernel": dom, "kernel_ms": avg_ms,
+                     "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
+                     "kernel_shares": shares,
+                     "kernel_ms_all": {n: t / c for n, (c, t) in kt.items()}})
 
     # ---- fwd-only throughput
     fwd_ms = []

@@ -589,12 +589,3 @@ sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
     return diag ? launch_band_fwd<128, 1, 1, 1>(q, k, v, g, scale, out, lse, s)
                 : launch_band_fwd<128, 2, 0, 1>(q, k, v, g, scale, out, lse, s);
 }
-
-// The backward on band tiles is not implemented yet: the gather kernels run it.
-bool sa_band_bwd_supported(const sa_tensor *, const sa_graph_s *) { return false; }
-
-sa_status sa_band_bwd(const sa_tensor *, const sa_tensor *, const sa_tensor *, const sa_tensor *,
-                      const float *, const sa_tensor *, const sa_graph_s *, const GraphView &, float,
-                      sa_tensor *, sa_tensor *, sa_tensor *, float *, cudaStream_t) {
-    return SA_ERR_UNSUPPORTED;
-}

@@ -1,0 +1,857 @@
+// attn_band_bwd.cu -- backward on tcgen05 band tiles fused with the gathered
+// edges.  Probabilities are recomputed from lse; two kernels with disjoint
+// outputs and no float atomics, so results are bitwise reproducible:
+//
+//  band_bwd_dq   CTA = 128 queries [q0, q0+128).  Delta_i = dO_i . out_i is
+//                computed per row and written for the second kernel.  Key
+//                blocks of 64 from q0-W+1 (the forward's band in block
+//                coordinates u = 64 b + c, row r keeps r <= u <= r+W-1):
+//                S = Q K^T and dP = dO V^T in TMEM, dS = P (dP - Delta) in
+//                shared memory (bf16), dQ += dS K in TMEM.
+//  band_bwd_dkdv CTA = 128 keys [k0, k0+128).  Query blocks of 64 from k0
+//                (v = i - k0 = 64 b + c, key row r keeps r <= v <= r+W-1):
+//                S^T = K Q^T and dP^T = V dO^T in TMEM, P^T and dS^T in
+//                shared memory, dV += P^T dO and dK += dS^T Q in TMEM.
+//
+// The other edges (2^k distance links or the non-window part of CSR lists)
+// are diagonal blocks as in the forward: row r of a block belongs to query
+// (or key) r; for a distance o the rows are one TMA box, for CSR lists 16-byte
+// cp.async gathers of the row's slot.  They are accumulated on CUDA cores
+// first and initialise the TMEM accumulators, which the band MMAs then add to.
+//
+// Warp roles (256 threads): 0 TMA producer, 1 TMEM allocator + MMA issuer,
+// 2-3 diagonal-block producers, 4-7 compute warpgroup (thread = owned row =
+// TMEM lane).  Waits are bounded as in the forward.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sa_band.cuh"
+#include "tc_common.cuh"
+#include "tmap.cuh"
+
+namespace {
+
+constexpr int BM = 128;  // rows a CTA owns
+constexpr int BB = 64;   // streamed block
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdArgs {
+    int64_t T;
+    int32_t W;
+    int32_t kind;
+    int32_t n_off;
+    int64_t offs[SA_MAX_OFFSETS];  // descending
+    const int64_t *rowptr;
+    const int32_t *colidx;
+    const int64_t *rev_rowptr;
+    const int32_t *rev_colidx;
+    const __nv_bfloat16 *q, *k, *v, *o, *dout;
+    const float *lse;
+    float *delta;
+    __nv_bfloat16 *dq, *dk, *dv;
+    float scale;
+    float scale2;  // scale * log2(e)
+    int *err;
+};
+
+__host__ __device__ constexpr int align1k(int x) { return (x + 1023) & ~1023; }
+
+// ---------------------------------------------------------------- helpers
+
+// Load a 128-row tile (two 64-row boxes per 64-column half) with a box-64 map.
+template <int D>
+__device__ __forceinline__ void tma_tile128(uint32_t dst, const void *map, int64_t row, int64_t bh,
+                                            uint32_t bar) {
+#pragma unroll
+    for (int x = 0; x < D / 64; ++x)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            tc::tma_load_3d(dst + x * (BM * 128) + h * (64 * 128), map, x * 64,
+                            (int32_t)(row + 64 * h), (int32_t)bh, bar);
+}
+
+template <int D>
+__device__ __forceinline__ void tma_block64(uint32_t dst, const void *map, int64_t row, int64_t bh,
+                                            uint32_t bar) {
+#pragma unroll
+    for (int x = 0; x < D / 64; ++x)
+        tc::tma_load_3d(dst + x * (BB * 128), map, x * 64, (int32_t)row, (int32_t)bh, bar);
+}
+
+// 16-byte chunk c of row r in a tile of `rows` rows (64-column halves stacked).
+__device__ __forceinline__ uint32_t tile_off(int rows, int r, int c) {
+    return (uint32_t)((c >> 3) * (rows * 128)) + tc::sw128_off((uint32_t)r, (uint32_t)(c & 7));
+}
+
+template <int D>
+__device__ __forceinline__ void load_row_packed(const uint8_t *tile, int rows, int r, uint32_t *w) {
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 x = *(const uint4 *)(tile + tile_off(rows, r, c));
+        w[4 * c] = x.x;
+        w[4 * c + 1] = x.y;
+        w[4 * c + 2] = x.z;
+        w[4 * c + 3] = x.w;
+    }
+}
+
+template <int D>
+__device__ __forceinline__ float dot_packed(const uint32_t *a, const uint32_t *b) {
+    float s = 0.f;
+#pragma unroll
+    for (int x = 0; x < D / 2; ++x) {
+        s = fmaf(tc::bf16lo(a[x]), tc::bf16lo(b[x]), s);
+        s = fmaf(tc::bf16hi(a[x]), tc::bf16hi(b[x]), s);
+    }
+    return s;
+}
+
+template <int D>
+__device__ __forceinline__ void axpy_packed(float *acc, float a, const uint32_t *x) {
+#pragma unroll
+    for (int e = 0; e < D / 2; ++e) {
+        acc[2 * e] = fmaf(a, tc::bf16lo(x[e]), acc[2 * e]);
+        acc[2 * e + 1] = fmaf(a, tc::bf16hi(x[e]), acc[2 * e + 1]);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void tmem_store_row(uint32_t taddr, const float *acc) {
+#pragma unroll
+    for (int c = 0; c < D; c += 32) {
+        uint32_t w[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) w[x] = __float_as_uint(acc[c + x]);
+        tc::tmem_st32(taddr + c, w);
+    }
+}
+
+// TMEM row (D fp32 columns) * mul -> bf16 row in global memory.
+template <int D>
+__device__ __forceinline__ void tmem_row_to_global(uint32_t taddr, float mul, __nv_bfloat16 *dst,
+                                                   bool store) {
+#pragma unroll
+    for (int c = 0; c < D; c += 32) {
+        uint32_t w[32];
+        tc::tmem_ld32(taddr + c, w);
+        tc::tmem_ld_wait();
+        if (store) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 8) {
+                uint4 o4;
+                o4.x = tc::pack_bf16x2(__uint_as_float(w[x]) * mul, __uint_as_float(w[x + 1]) * mul);
+                o4.y = tc::pack_bf16x2(__uint_as_float(w[x + 2]) * mul,
+                                       __uint_as_float(w[x + 3]) * mul);
+                o4.z = tc::pack_bf16x2(__uint_as_float(w[x + 4]) * mul,
+                                       __uint_as_float(w[x + 5]) * mul);
+                o4.w = tc::pack_bf16x2(__uint_as_float(w[x + 6]) * mul,
+                                       __uint_as_float(w[x + 7]) * mul);
+                *(uint4 *)(dst + c + x) = o4;
+            }
+        }
+    }
+}
+
+// Write 64 bf16 values (from fp32) as row r of a 128 x 64 K-major SW128 tile.
+__device__ __forceinline__ void store_row64_bf16(uint8_t *tile, int r, const float *x) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint4 w;
+        w.x = tc::pack_bf16x2(x[8 * c], x[8 * c + 1]);
+        w.y = tc::pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
+        w.z = tc::pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
+        w.w = tc::pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
+        *(uint4 *)(tile + tc::sw128_off((uint32_t)r, (uint32_t)c)) = w;
+    }
+}
+
+#define WAIT_OR(bar_, par_, action_)                                                   \
+    if (!tc::mbar_wait((bar_), (par_), abort, a.err, SA_DEVERR_TIMEOUT)) {              \
+        action_;                                                                       \
+    }
+
+// =================================================================== dQ
+
+template <int D, int BS, int DS, int PB>
+struct LayoutDQ {
+    static constexpr int kRow = BM * D * 2, kBlk = BB * D * 2, kDSTile = BM * BB * 2;
+    static constexpr int kQ = 0, kDO = kRow, kK = 2 * kRow, kV = kK + BS * kBlk;
+    static constexpr int kDS = kV + BS * kBlk;
+    static constexpr int kDiagK = kDS + PB * kDSTile;
+    static constexpr int kDiagV = kDiagK + DS * kRow;
+    static constexpr int kBars = kDiagV + DS * kRow;
+    static constexpr int DSX = DS > 0 ? DS : 1;
+    static constexpr int bQFull = 0, bBandFull = 1, bBandEmpty = bBandFull + BS;
+    static constexpr int bSFull = bBandEmpty + BS, bSFree = bSFull + 2;
+    static constexpr int bDSFull = bSFree + 2, bDSDone = bDSFull + PB;
+    static constexpr int bInit = bDSDone + PB, bDiagFull = bInit + 1;
+    static constexpr int bDiagEmpty = bDiagFull + DSX, nBars = bDiagEmpty + DSX;
+    static constexpr int kMisc = kBars + nBars * 8;
+    static constexpr int kAlloc = kMisc + 16 + 1024;
+    static constexpr uint32_t tS = 0, tDP = 128, tDQ = 256, kTmemCols = 512;
+};
+
+template <int D, int BS, int DS, int PB>
+__global__ void __launch_bounds__(256, 1)
+band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                   const __grid_constant__ CUtensorMap tv,
+                   const __grid_constant__ CUtensorMap tdo, const BwdArgs a) {
+    using L = LayoutDQ<D, BS, DS, PB>;
+    constexpr int DSX = L::DSX;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = tc::smem_u32(sm);
+    uint32_t *tmem_slot = (uint32_t *)(sm + L::kMisc);
+    volatile int *abort = (volatile int *)(sm + L::kMisc + 4);
+    int *n_diag_s = (int *)(sm + L::kMisc + 8);
+    auto bar = [&](int b) { return sbase + L::kBars + 8u * (uint32_t)b; };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t bh = blockIdx.y, q0 = (int64_t)blockIdx.x * BM, T = a.T;
+    const int32_t W = a.W;
+    const int64_t kb0 = q0 - W + 1;
+    const int64_t last_key = (q0 + BM - 1 < T - 1) ? q0 + BM - 1 : T - 1;
+    const int64_t nblk = (last_key - kb0) / BB + 1;
+    const int64_t need0 = (int64_t)W - 1 - q0;
+    const int64_t b_first = need0 > 0 ? need0 / BB : 0;
+    const int n_band = (int)(nblk - b_first);
+
+    if (tid == 0) {
+        tc::mbar_init(bar(L::bQFull), 1);
+        for (int s = 0; s < BS; ++s) {
+            tc::mbar_init(bar(L::bBandFull + s), 1);
+            tc::mbar_init(bar(L::bBandEmpty + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(bar(L::bSFull + s), 1);
+            tc::mbar_init(bar(L::bSFree + s), 4);
+        }
+        for (int s = 0; s < PB; ++s) {
+            tc::mbar_init(bar(L::bDSFull + s), 4);
+            tc::mbar_init(bar(L::bDSDone + s), 1);
+        }
+        tc::mbar_init(bar(L::bInit), 4);
+        for (int s = 0; s < DSX; ++s) {
+            tc::mbar_init(bar(L::bDiagFull + s), a.kind == 0 ? 1 : 64);
+            tc::mbar_init(bar(L::bDiagEmpty + s), 4);
+        }
+        *abort = 0;
+        *n_diag_s = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), L::kTmemCols);
+    __syncthreads();
+    if (DS > 0 && warp >= 4) {
+        int nd = 0;
+        const int64_t i = q0 + (tid - 128);
+        if (a.kind == 0) {
+            for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last_key) ? 1 : 0;
+        } else if (i < T) {
+            const int64_t deg = a.rowptr[i + 1] - a.rowptr[i];
+            nd = (int)(deg - ((i + 1 < W) ? i + 1 : W));
+        }
+        atomicMax(n_diag_s, nd);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int n_diag = DS > 0 ? *n_diag_s : 0;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tc::mbar_arrive_expect_tx(bar(L::bQFull), 2 * L::kRow);
+            tma_tile128<D>(sbase + L::kQ, &tq, q0, bh, bar(L::bQFull));
+            tma_tile128<D>(sbase + L::kDO, &tdo, q0, bh, bar(L::bQFull));
+            for (int bl = 0; bl < n_band; ++bl) {
+                const int st = bl % BS, use = bl / BS;
+                if (use > 0) WAIT_OR(bar(L::bBandEmpty + st), (use - 1) & 1, break);
+                const int64_t krow = kb0 + (b_first + bl) * BB;
+                tc::mbar_arrive_expect_tx(bar(L::bBandFull + st), 2 * L::kBlk);
+                tma_block64<D>(sbase + L::kK + st * L::kBlk, &tk, krow, bh, bar(L::bBandFull + st));
+                tma_block64<D>(sbase + L::kV + st * L::kBlk, &tv, krow, bh, bar(L::bBandFull + st));
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idS = tc::idesc_bf16(BM, BB, false, false);
+            const uint32_t idQ = tc::idesc_bf16(BM, D, false, true);
+            bool ok = tc::mbar_wait(bar(L::bQFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
+            auto issue = [&](int bl) -> bool {
+                const int st = bl % BS, sb = bl & 1;
+                if (!tc::mbar_wait(bar(L::bBandFull + st), (bl / BS) & 1, abort, a.err,
+                                   SA_DEVERR_TIMEOUT))
+                    return false;
+                if (bl >= 2 && !tc::mbar_wait(bar(L::bSFree + sb), ((bl >> 1) - 1) & 1, abort,
+                                              a.err, SA_DEVERR_TIMEOUT))
+                    return false;
+                tc::tc_fence_after();
+                const uint32_t ka = sbase + L::kK + st * L::kBlk, va = sbase + L::kV + st * L::kBlk;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t offr = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                    const uint32_t offb = (kk >> 2) * (BB * 128) + (kk & 3) * 32;
+                    tc::mma_bf16_ss(tmem + L::tS + sb * BB,
+                                    tc::sdesc_sw128(sbase + L::kQ + offr, 16, 1024),
+                                    tc::sdesc_sw128(ka + offb, 16, 1024), idS, kk > 0);
+                    tc::mma_bf16_ss(tmem + L::tDP + sb * BB,
+                                    tc::sdesc_sw128(sbase + L::kDO + offr, 16, 1024),
+                                    tc::sdesc_sw128(va + offb, 16, 1024), idS, kk > 0);
+                }
+                tc::mma_commit(bar(L::bSFull + sb));
+                return true;
+            };
+            if (ok && n_band > 0) ok = issue(0);
+            for (int bl = 0; ok && bl < n_band; ++bl) {
+                if (BS >= 2 && bl + 1 < n_band && !issue(bl + 1)) break;
+                const int pb = bl % PB, st = bl % BS;
+                if (bl == 0) WAIT_OR(bar(L::bInit), 0, break);
+                WAIT_OR(bar(L::bDSFull + pb), (bl / PB) & 1, break);
+                tc::tc_fence_after();
+                const uint32_t dsa = sbase + L::kDS + pb * L::kDSTile;
+                const uint32_t ka = sbase + L::kK + st * L::kBlk;
+#pragma unroll
+                for (int kk = 0; kk < BB / 16; ++kk)
+                    tc::mma_bf16_ss(tmem + L::tDQ, tc::sdesc_sw128(dsa + kk * 32, 16, 1024),
+                                    tc::sdesc_sw128(ka + kk * 16 * 128, BB * 128, 1024), idQ, 1u);
+                tc::mma_commit(bar(L::bBandEmpty + st));
+                tc::mma_commit(bar(L::bDSDone + pb));
+                if (BS == 1 && bl + 1 < n_band && !issue(bl + 1)) break;
+            }
+        }
+    } else if (warp == 2 || warp == 3) {
+        if (DS > 0) {
+            const int pt = tid - 64;
+            for (int d = 0; d < n_diag; ++d) {
+                const int st = d % DSX, use = d / DSX;
+                const uint32_t kdst = sbase + L::kDiagK + st * L::kRow;
+                const uint32_t vdst = sbase + L::kDiagV + st * L::kRow;
+                if (use > 0) WAIT_OR(bar(L::bDiagEmpty + st), (use - 1) & 1, break);
+                if (a.kind == 0) {
+                    if (pt == 0) {
+                        const int64_t krow = q0 - a.offs[a.n_off - n_diag + d];
+                        tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kRow);
+                        tma_tile128<D>(kdst, &tk, krow, bh, bar(L::bDiagFull + st));
+                        tma_tile128<D>(vdst, &tv, krow, bh, bar(L::bDiagFull + st));
+                    }
+                } else {
+                    constexpr int CH = D / 8;
+                    for (int item = pt; item < BM * CH; item += 64) {
+                        const int r = item / CH, c = item % CH;
+                        const int64_t i = q0 + r;
+                        if (i >= T) continue;
+                        const int64_t rs = a.rowptr[i], deg = a.rowptr[i + 1] - rs;
+                        if (d >= deg - ((i + 1 < W) ? i + 1 : W)) continue;
+                        const int64_t j = a.colidx[rs + d];
+                        const size_t src = ((size_t)bh * (size_t)T + (size_t)j) * D + c * 8;
+                        const uint32_t off = tile_off(BM, r, c);
+                        tc::cp_async_16(kdst + off, a.k + src);
+                        tc::cp_async_16(vdst + off, a.v + src);
+                    }
+                    tc::cp_async_mbar_arrive(bar(L::bDiagFull + st));
+                }
+            }
+        }
+    } else {
+        const int r = tid - 128;
+        const int64_t i = q0 + r;
+        const bool row_ok = i < T;
+        const size_t grow = (size_t)bh * (size_t)T + (size_t)i;
+        const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + L::tS, tDP = tmem + lane_off + L::tDP;
+        const uint32_t tDQ = tmem + lane_off + L::tDQ;
+        const float c2 = a.scale2;
+        const float lse2 = row_ok ? a.lse[grow] * kLog2e : 0.f;
+        bool ok = tc::mbar_wait(bar(L::bQFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
+        float Delta = 0.f;
+        if (ok) {
+            // Delta_i = dO_i . out_i
+            uint32_t dor[D / 2];
+            load_row_packed<D>(sm + L::kDO, BM, r, dor);
+            if (row_ok) {
+                const uint4 *orow = (const uint4 *)(a.o + grow * D);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) {
+                    const uint4 x = __ldg(orow + c);
+                    const uint32_t ow[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        Delta = fmaf(tc::bf16lo(dor[4 * c + e]), tc::bf16lo(ow[e]), Delta);
+                        Delta = fmaf(tc::bf16hi(dor[4 * c + e]), tc::bf16hi(ow[e]), Delta);
+                    }
+                }
+                a.delta[grow] = Delta;
+            }
+            // diagonal blocks
+            float acc[D];
+#pragma unroll
+            for (int x = 0; x < D; ++x) acc[x] = 0.f;
+            if (DS > 0 && n_diag > 0) {
+                uint32_t qr[D / 2];
+                load_row_packed<D>(sm + L::kQ, BM, r, qr);
+                int64_t resid = 0;
+                if (a.kind == 1 && row_ok)
+                    resid = (a.rowptr[i + 1] - a.rowptr[i]) - ((i + 1 < W) ? i + 1 : W);
+                for (int d = 0; d < n_diag; ++d) {
+                    const int st = d % DSX;
+                    WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
+                    const bool valid = row_ok && (a.kind == 0 ? i >= a.offs[a.n_off - n_diag + d]
+                                                              : d < resid);
+                    if (valid) {
+                        uint32_t kr[D / 2], vr[D / 2];
+                        load_row_packed<D>(sm + L::kDiagK + st * L::kRow, BM, r, kr);
+                        load_row_packed<D>(sm + L::kDiagV + st * L::kRow, BM, r, vr);
+                        const float p = tc::ex2(dot_packed<D>(qr, kr) * c2 - lse2);
+                        const float ds = p * (dot_packed<D>(dor, vr) - Delta);
+                        axpy_packed<D>(acc, ds, kr);
+                    }
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                }
+            }
+            tmem_store_row<D>(tDQ, acc);
+            tc::tmem_st_wait();
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar(L::bInit));
+
+        // band blocks
+        for (int bl = 0; ok && bl < n_band; ++bl) {
+            const int sb = bl & 1, pb = bl % PB;
+            const int64_t u0 = (b_first + bl) * BB;
+            WAIT_OR(bar(L::bSFull + sb), (bl >> 1) & 1, ok = false; break);
+            tc::tc_fence_after();
+            float s[BB], dp[BB];
+            tc::tmem_ld32(tS + sb * BB, (uint32_t *)s);
+            tc::tmem_ld32(tS + sb * BB + 32, (uint32_t *)(s + 32));
+            tc::tmem_ld32(tDP + sb * BB, (uint32_t *)dp);
+            tc::tmem_ld32(tDP + sb * BB + 32, (uint32_t *)(dp + 32));
+            tc::tmem_ld_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(L::bSFree + sb));
+            const bool need_mask = (u0 < BM - 1) || (u0 + BB - 1 > (int64_t)W - 1) ||
+                                   (u0 + q0 < (int64_t)W - 1);
+            const int64_t lo = ((int64_t)r > (int64_t)W - 1 - q0) ? r : (int64_t)W - 1 - q0;
+            const int64_t hi = (int64_t)r + W - 1;
+#pragma unroll
+            for (int c = 0; c < BB; ++c) {
+                const bool keep = !need_mask || ((u0 + c >= lo) && (u0 + c <= hi));
+                const float p = keep ? tc::ex2(s[c] * c2 - lse2) : 0.f;
+                s[c] = p * (dp[c] - Delta);  // dS
+            }
+            if (bl >= PB) WAIT_OR(bar(L::bDSDone + pb), ((bl - PB) / PB) & 1, ok = false; break);
+            store_row64_bf16(sm + L::kDS + pb * L::kDSTile, r, s);
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(L::bDSFull + pb));
+        }
+        if (ok && n_band > 0) {
+            const int lb = n_band - 1;
+            ok = tc::mbar_wait(bar(L::bDSDone + lb % PB), (lb / PB) & 1, abort, a.err,
+                               SA_DEVERR_TIMEOUT);
+        }
+        if (ok) {
+            tc::tc_fence_after();
+            tmem_row_to_global<D>(tDQ, a.scale, a.dq + grow * D, row_ok);
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, L::kTmemCols);
+    }
+}
+
+// ================================================================= dK/dV
+
+template <int D, int BS, int DS, int PB>
+struct LayoutDKV {
+    static constexpr int kRow = BM * D * 2, kBlk = BB * D * 2, kPTile = BM * BB * 2;
+    static constexpr int kK = 0, kV = kRow, kQ = 2 * kRow, kDO = kQ + BS * kBlk;
+    static constexpr int kLse = kDO + BS * kBlk, kDel = kLse + BS * 256;
+    static constexpr int kP = align1k(kDel + BS * 256), kDS = kP + PB * kPTile;
+    static constexpr int kDiagQ = kDS + PB * kPTile, kDiagDO = kDiagQ + DS * kRow;
+    static constexpr int kBars = kDiagDO + DS * kRow;
+    static constexpr int DSX = DS > 0 ? DS : 1;
+    static constexpr int bKVFull = 0, bBandFull = 1, bBandEmpty = bBandFull + BS;
+    static constexpr int bSFull = bBandEmpty + BS, bSFree = bSFull + 2;
+    static constexpr int bPFull = bSFree + 2, bPDone = bPFull + PB;
+    static constexpr int bInit = bPDone + PB, bDiagFull = bInit + 1;
+    static constexpr int bDiagEmpty = bDiagFull + DSX, nBars = bDiagEmpty + DSX;
+    static constexpr int kMisc = kBars + nBars * 8;
+    static constexpr int kAlloc = kMisc + 16 + 1024;
+    static constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D, kTmemCols = 512;
+};
+
+template <int D, int BS, int DS, int PB>
+__global__ void __launch_bounds__(256, 1)
+band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv,
+                     const __grid_constant__ CUtensorMap tdo, const BwdArgs a) {
+    using L = LayoutDKV<D, BS, DS, PB>;
+    constexpr int DSX = L::DSX;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = tc::smem_u32(sm);
+    uint32_t *tmem_slot = (uint32_t *)(sm + L::kMisc);
+    volatile int *abort = (volatile int *)(sm + L::kMisc + 4);
+    int *n_diag_s = (int *)(sm + L::kMisc + 8);
+    auto bar = [&](int b) { return sbase + L::kBars + 8u * (uint32_t)b; };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t bh = blockIdx.y, k0 = (int64_t)blockIdx.x * BM, T = a.T;
+    const int32_t W = a.W;
+    // queries k0 .. min(T-1, k0+127+W-1) in blocks of 64 from k0
+    const int64_t vmax_w = (int64_t)BM - 1 + W - 1, vmax_t = T - 1 - k0;
+    const int64_t vmax = vmax_w < vmax_t ? vmax_w : vmax_t;
+    const int n_band = (int)(vmax / BB + 1);
+
+    if (tid == 0) {
+        tc::mbar_init(bar(L::bKVFull), 1);
+        for (int s = 0; s < BS; ++s) {
+            // TMA bytes + the 32 producer lanes that stage lse and Delta
+            tc::mbar_init(bar(L::bBandFull + s), 33);
+            tc::mbar_init(bar(L::bBandEmpty + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(bar(L::bSFull + s), 1);
+            tc::mbar_init(bar(L::bSFree + s), 4);
+        }
+        for (int s = 0; s < PB; ++s) {
+            tc::mbar_init(bar(L::bPFull + s), 4);
+            tc::mbar_init(bar(L::bPDone + s), 1);
+        }
+        tc::mbar_init(bar(L::bInit), 4);
+        for (int s = 0; s < DSX; ++s) {
+            tc::mbar_init(bar(L::bDiagFull + s), a.kind == 0 ? 1 : 64);
+            tc::mbar_init(bar(L::bDiagEmpty + s), 4);
+        }
+        *abort = 0;
+        *n_diag_s = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), L::kTmemCols);
+    __syncthreads();
+    if (DS > 0 && warp >= 4) {
+        int nd = 0;
+        const int64_t j = k0 + (tid - 128);
+        if (a.kind == 0) {
+            for (int x = 0; x < a.n_off; ++x) nd += (k0 + a.offs[x] <= T - 1) ? 1 : 0;
+        } else if (j < T) {
+            const int64_t deg = a.rev_rowptr[j + 1] - a.rev_rowptr[j];
+            nd = (int)(deg - ((T - j < W) ? T - j : W));
+        }
+        atomicMax(n_diag_s, nd);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int n_diag = DS > 0 ? *n_diag_s : 0;
+    // distance list of this tile: the n_diag smallest offsets with k0 + o <= T-1,
+    // taken in descending order (as stored)
+    const int off_first = a.n_off - n_diag;
+
+    if (warp == 0) {
+        // lane 0 issues the TMA copies; all 32 lanes stage lse (base 2) and
+        // Delta of the block's 64 queries (zero past the end of the sequence)
+        if (lane == 0) {
+            tc::mbar_arrive_expect_tx(bar(L::bKVFull), 2 * L::kRow);
+            tma_tile128<D>(sbase + L::kK, &tk, k0, bh, bar(L::bKVFull));
+            tma_tile128<D>(sbase + L::kV, &tv, k0, bh, bar(L::bKVFull));
+        }
+        for (int bl = 0; bl < n_band; ++bl) {
+            const int st = bl % BS, use = bl / BS;
+            if (use > 0) WAIT_OR(bar(L::bBandEmpty + st), (use - 1) & 1, break);
+            const int64_t qrow = k0 + (int64_t)bl * BB;
+            if (lane == 0) {
+                tc::mbar_arrive_expect_tx(bar(L::bBandFull + st), 2 * L::kBlk);
+                tma_block64<D>(sbase + L::kQ + st * L::kBlk, &tq, qrow, bh, bar(L::bBandFull + st));
+                tma_block64<D>(sbase + L::kDO + st * L::kBlk, &tdo, qrow, bh,
+                               bar(L::bBandFull + st));
+            }
+            float *ls = (float *)(sm + L::kLse + st * 256), *dl = (float *)(sm + L::kDel + st * 256);
+            for (int c = lane; c < BB; c += 32) {
+                const int64_t i = qrow + c;
+                const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
+                ls[c] = i < T ? a.lse[gi] * kLog2e : 0.f;
+                dl[c] = i < T ? a.delta[gi] : 0.f;
+            }
+            tc::mbar_arrive(bar(L::bBandFull + st));
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idS = tc::idesc_bf16(BM, BB, false, false);
+            const uint32_t idG = tc::idesc_bf16(BM, D, false, true);
+            bool ok = tc::mbar_wait(bar(L::bKVFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
+            auto issue = [&](int bl) -> bool {
+                const int st = bl % BS, sb = bl & 1;
+                if (!tc::mbar_wait(bar(L::bBandFull + st), (bl / BS) & 1, abort, a.err,
+                                   SA_DEVERR_TIMEOUT))
+                    return false;
+                if (bl >= 2 && !tc::mbar_wait(bar(L::bSFree + sb), ((bl >> 1) - 1) & 1, abort,
+                                              a.err, SA_DEVERR_TIMEOUT))
+                    return false;
+                tc::tc_fence_after();
+                const uint32_t qa = sbase + L::kQ + st * L::kBlk, da = sbase + L::kDO + st * L::kBlk;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t offr = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                    const uint32_t offb = (kk >> 2) * (BB * 128) + (kk & 3) * 32;
+                    tc::mma_bf16_ss(tmem + L::tS + sb * BB,
+                                    tc::sdesc_sw128(sbase + L::kK + offr, 16, 1024),
+                                    tc::sdesc_sw128(qa + offb, 16, 1024), idS, kk > 0);
+                    tc::mma_bf16_ss(tmem + L::tDP + sb * BB,
+                                    tc::sdesc_sw128(sbase + L::kV + offr, 16, 1024),
+                                    tc::sdesc_sw128(da + offb, 16, 1024), idS, kk > 0);
+                }
+                tc::mma_commit(bar(L::bSFull + sb));
+                return true;
+            };
+            if (ok && n_band > 0) ok = issue(0);
+            for (int bl = 0; ok && bl < n_band; ++bl) {
+                if (BS >= 2 && bl + 1 < n_band && !issue(bl + 1)) break;
+                const int pb = bl % PB, st = bl % BS;
+                if (bl == 0) WAIT_OR(bar(L::bInit), 0, break);
+                WAIT_OR(bar(L::bPFull + pb), (bl / PB) & 1, break);
+                tc::tc_fence_after();
+                const uint32_t pa = sbase + L::kP + pb * L::kPTile;
+                const uint32_t dsa = sbase + L::kDS + pb * L::kPTile;
+                const uint32_t qa = sbase + L::kQ + st * L::kBlk, da = sbase + L::kDO + st * L::kBlk;
+#pragma unroll
+                for (int kk = 0; kk < BB / 16; ++kk) {
+                    tc::mma_bf16_ss(tmem + L::tDV, tc::sdesc_sw128(pa + kk * 32, 16, 1024),
+                                    tc::sdesc_sw128(da + kk * 16 * 128, BB * 128, 1024), idG, 1u);
+                    tc::mma_bf16_ss(tmem + L::tDK, tc::sdesc_sw128(dsa + kk * 32, 16, 1024),
+                                    tc::sdesc_sw128(qa + kk * 16 * 128, BB * 128, 1024), idG, 1u);
+                }
+                tc::mma_commit(bar(L::bBandEmpty + st));
+                tc::mma_commit(bar(L::bPDone + pb));
+                if (BS == 1 && bl + 1 < n_band && !issue(bl + 1)) break;
+            }
+        }
+    } else if (warp == 2 || warp == 3) {
+        if (DS > 0) {
+            const int pt = tid - 64;
+            for (int d = 0; d < n_diag; ++d) {
+                const int st = d % DSX, use = d / DSX;
+                const uint32_t qdst = sbase + L::kDiagQ + st * L::kRow;
+                const uint32_t ddst = sbase + L::kDiagDO + st * L::kRow;
+                if (use > 0) WAIT_OR(bar(L::bDiagEmpty + st), (use - 1) & 1, break);
+                if (a.kind == 0) {
+                    if (pt == 0) {
+                        const int64_t qrow = k0 + a.offs[off_first + d];
+                        tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kRow);
+                        tma_tile128<D>(qdst, &tq, qrow, bh, bar(L::bDiagFull + st));
+                        tma_tile128<D>(ddst, &tdo, qrow, bh, bar(L::bDiagFull + st));
+                    }
+                } else {
+                    constexpr int CH = D / 8;
+                    for (int item = pt; item < BM * CH; item += 64) {
+                        const int r = item / CH, c = item % CH;
+                        const int64_t j = k0 + r;
+                        if (j >= T) continue;
+                        const int64_t rs = a.rev_rowptr[j], deg = a.rev_rowptr[j + 1] - rs;
+                        const int64_t nb = (T - j < W) ? T - j : W;
+                        if (d >= deg - nb) continue;
+                        const int64_t i = a.rev_colidx[rs + nb + d];
+                        const size_t src = ((size_t)bh * (size_t)T + (size_t)i) * D + c * 8;
+                        const uint32_t off = tile_off(BM, r, c);
+                        tc::cp_async_16(qdst + off, a.q + src);
+                        tc::cp_async_16(ddst + off, a.dout + src);
+                    }
+                    tc::cp_async_mbar_arrive(bar(L::bDiagFull + st));
+                }
+            }
+        }
+    } else {
+        const int r = tid - 128;
+        const int64_t j = k0 + r;
+        const bool row_ok = j < T;
+        const size_t grow = (size_t)bh * (size_t)T + (size_t)j;
+        const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + L::tS, tDP = tmem + lane_off + L::tDP;
+        const uint32_t tDV = tmem + lane_off + L::tDV, tDK = tmem + lane_off + L::tDK;
+        const float c2 = a.scale2;
+        bool ok = tc::mbar_wait(bar(L::bKVFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
+        if (ok) {
+            float adk[D], adv[D];
+#pragma unroll
+            for (int x = 0; x < D; ++x) adk[x] = adv[x] = 0.f;
+            if (DS > 0 && n_diag > 0) {
+                uint32_t kr[D / 2], vr[D / 2];
+                load_row_packed<D>(sm + L::kK, BM, r, kr);
+                load_row_packed<D>(sm + L::kV, BM, r, vr);
+                int64_t rs = 0, nb = 0, resid = 0;
+                if (a.kind == 1 && row_ok) {
+                    rs = a.rev_rowptr[j];
+                    nb = (T - j < W) ? T - j : W;
+                    resid = a.rev_rowptr[j + 1] - rs - nb;
+                }
+                for (int d = 0; d < n_diag; ++d) {
+                    const int st = d % DSX;
+                    WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
+                    int64_t i = -1;
+                    if (row_ok) {
+                        if (a.kind == 0) {
+                            const int64_t cand = j + a.offs[off_first + d];
+                            if (cand < T) i = cand;
+                        } else if (d < resid) {
+                            i = a.rev_colidx[rs + nb + d];
+                        }
+                    }
+                    if (i >= 0) {
+                        const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
+                        const float lse2 = a.lse[gi] * kLog2e, Dl = a.delta[gi];
+                        uint32_t qr[D / 2], dr[D / 2];
+                        load_row_packed<D>(sm + L::kDiagQ + st * L::kRow, BM, r, qr);
+                        load_row_packed<D>(sm + L::kDiagDO + st * L::kRow, BM, r, dr);
+                        const float p = tc::ex2(dot_packed<D>(qr, kr) * c2 - lse2);
+                        const float ds = p * (dot_packed<D>(dr, vr) - Dl);
+                        axpy_packed<D>(adv, p, dr);
+                        axpy_packed<D>(adk, ds, qr);
+                    }
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                }
+            }
+            tmem_store_row<D>(tDV, adv);
+            tmem_store_row<D>(tDK, adk);
+            tc::tmem_st_wait();
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar(L::bInit));
+
+        for (int bl = 0; ok && bl < n_band; ++bl) {
+            const int sb = bl & 1, pb = bl % PB, st = bl % BS;
+            const int64_t v0 = (int64_t)bl * BB;
+            WAIT_OR(bar(L::bSFull + sb), (bl >> 1) & 1, ok = false; break);
+            tc::tc_fence_after();
+            float s[BB], dp[BB];
+            tc::tmem_ld32(tS + sb * BB, (uint32_t *)s);
+            tc::tmem_ld32(tS + sb * BB + 32, (uint32_t *)(s + 32));
+            tc::tmem_ld32(tDP + sb * BB, (uint32_t *)dp);
+            tc::tmem_ld32(tDP + sb * BB + 32, (uint32_t *)(dp + 32));
+            tc::tmem_ld_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(L::bSFree + sb));
+            const float *lse_s = (const float *)(sm + L::kLse + st * 256);
+            const float *del_s = (const float *)(sm + L::kDel + st * 256);
+            const bool need_mask = (v0 < BM - 1) || (v0 + BB - 1 > (int64_t)W - 1) ||
+                                   (k0 + v0 + BB - 1 > T - 1);
+            const int64_t lo = r, hi = (int64_t)r + W - 1;
+            const int64_t vlim = T - 1 - k0;
+#pragma unroll
+            for (int c = 0; c < BB; ++c) {
+                const int64_t vv = v0 + c;
+                const bool keep = !need_mask || (vv >= lo && vv <= hi && vv <= vlim);
+                const float p = keep ? tc::ex2(s[c] * c2 - lse_s[c]) : 0.f;
+                s[c] = p;
+                dp[c] = p * (dp[c] - del_s[c]);
+            }
+            if (bl >= PB) WAIT_OR(bar(L::bPDone + pb), ((bl - PB) / PB) & 1, ok = false; break);
+            store_row64_bf16(sm + L::kP + pb * L::kPTile, r, s);
+            store_row64_bf16(sm + L::kDS + pb * L::kPTile, r, dp);
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(L::bPFull + pb));
+        }
+        if (ok && n_band > 0) {
+            const int lb = n_band - 1;
+            ok = tc::mbar_wait(bar(L::bPDone + lb % PB), (lb / PB) & 1, abort, a.err,
+                               SA_DEVERR_TIMEOUT);
+        }
+        if (ok) {
+            tc::tc_fence_after();
+            tmem_row_to_global<D>(tDV, 1.f, a.dv + grow * D, row_ok);
+            tmem_row_to_global<D>(tDK, a.scale, a.dk + grow * D, row_ok);
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, L::kTmemCols);
+    }
+}
+
+template <int D, int BS, int DS, int PB>
+sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                          const sa_tensor *o, const float *lse, const sa_tensor *dout,
+                          const sa_graph_s *g, float scale, sa_tensor *dq, sa_tensor *dk,
+                          sa_tensor *dv, float *delta, cudaStream_t s) {
+    using LQ = LayoutDQ<D, BS, DS, PB>;
+    using LK = LayoutDKV<D, BS, DS, PB>;
+    static_assert(LQ::kAlloc <= 232448 && LK::kAlloc <= 232448, "shared memory budget");
+    const int64_t BH = q->B * q->H, T = q->T;
+    CUtensorMap mq, mk, mv, mdo;
+    if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BB) || !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BH, BB) ||
+        !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BH, BB) ||
+        !sa_tmap_bf16_3d(&mdo, dout->ptr, D, T, BH, BB))
+        return SA_ERR_CUDA;
+    BwdArgs a{};
+    a.T = T;
+    a.W = g->W;
+    a.kind = g->kind;
+    a.n_off = g->kind == 0 ? g->n_off : 0;
+    for (int x = 0; x < SA_MAX_OFFSETS; ++x) a.offs[x] = x < a.n_off ? g->offs[x] : 0;
+    a.rowptr = g->rowptr;
+    a.colidx = g->colidx;
+    a.rev_rowptr = g->rev_rowptr;
+    a.rev_colidx = g->rev_colidx;
+    a.q = (const __nv_bfloat16 *)q->ptr;
+    a.k = (const __nv_bfloat16 *)k->ptr;
+    a.v = (const __nv_bfloat16 *)v->ptr;
+    a.o = (const __nv_bfloat16 *)o->ptr;
+    a.dout = (const __nv_bfloat16 *)dout->ptr;
+    a.lse = lse;
+    a.delta = delta;
+    a.dq = (__nv_bfloat16 *)dq->ptr;
+    a.dk = (__nv_bfloat16 *)dk->ptr;
+    a.dv = (__nv_bfloat16 *)dv->ptr;
+    a.scale = scale;
+    a.scale2 = scale * kLog2e;
+    a.err = sa_device_error_word();
+    if (!a.err) return SA_ERR_CUDA;
+    auto kq = band_bwd_dq_kernel<D, BS, DS, PB>;
+    auto kkv = band_bwd_dkdv_kernel<D, BS, DS, PB>;
+    SA_CUDA_TRY(cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, LQ::kAlloc));
+    SA_CUDA_TRY(cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, LK::kAlloc));
+    dim3 grid((unsigned)((T + BM - 1) / BM), (unsigned)BH);
+    SA_LAUNCH("band_bwd_dq", s, kq<<<grid, 256, LQ::kAlloc, s>>>(mq, mk, mv, mdo, a));
+    SA_LAUNCH("band_bwd_dkdv", s, kkv<<<grid, 256, LK::kAlloc, s>>>(mq, mk, mv, mdo, a));
+    SA_CUDA_TRY(cudaGetLastError());
+    return SA_OK;
+}
+
+}  // namespace
+
+bool sa_band_bwd_supported(const sa_tensor *q, const sa_graph_s *g) {
+    if (q->dtype != SA_BF16 || (q->D != 64 && q->D != 128)) return false;
+    if (g->W < 1) return false;
+    if (q->B * q->H > 65535 || q->T >= ((int64_t)1 << 31)) return false;
+    const bool diag = (g->kind == 0) ? g->n_off > 0 : (g->max_resid > 0 || g->max_resid_rev > 0);
+    if (g->kind == 1 && (!g->rowptr || !g->rev_rowptr)) return false;
+    // distance / CSR edges with D = 128 stay on the gather kernels (register budget)
+    if (diag && q->D == 128) return false;
+    return true;
+}
+
+sa_status sa_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                      const sa_tensor *out, const float *lse, const sa_tensor *dout,
+                      const sa_graph_s *g, const GraphView &, float scale, sa_tensor *dq,
+                      sa_tensor *dk, sa_tensor *dv, float *delta, cudaStream_t s) {
+    const bool diag = (g->kind == 0) ? g->n_off > 0 : (g->max_resid > 0 || g->max_resid_rev > 0);
+    if (q->D == 64)
+        return diag ? launch_band_bwd<64, 2, 2, 2>(q, k, v, out, lse, dout, g, scale, dq, dk, dv,
+                                                   delta, s)
+                    : launch_band_bwd<64, 2, 0, 2>(q, k, v, out, lse, dout, g, scale, dq, dk, dv,
+                                                   delta, s);
+    return launch_band_bwd<128, 2, 0, 2>(q, k, v, out, lse, dout, g, scale, dq, dk, dv, delta, s);
+}

@@ -14,6 +14,7 @@ Workloads (shapes from the pages' own experiments, values synthetic):
   band_32k      B4 H32 T32768 D128 bf16, window 4096, no links (the
                 Mistral-style window of "MiniGPT (Part 6)")
   band_4k_full  B4 H32 T4096 D128 bf16, window = T = 4096 (full causal check)
+  band_32k_b1h8 B1 H8 T32768 D128 bf16, window 4096 (profiler-capture size)
   csr_1m        B1 H8 T2^20 D64 bf16, raw CSR rows: window 64 + 16 uniform
                 draws from [0, i) + the first 16 tokens (graph view of
                 "Longer Attention Span ...")
@@ -68,6 +69,9 @@ WORKLOADS = {
                         std=1.0 / math.sqrt(64), seed=1002),
     "band_32k": _w("band_32k", 4, 32, 32768, 128, "bf16", 4096, (), seed=1003),
     "band_4k_full": _w("band_4k_full", 4, 32, 4096, 128, "bf16", 4096, (), seed=1003),
+    # a quarter of band_32k (one batch row, 8 heads): the size used for
+    # detailed profiler captures
+    "band_32k_b1h8": _w("band_32k_b1h8", 1, 8, 32768, 128, "bf16", 4096, (), seed=1003),
     "csr_1m": _w("csr_1m", 1, 8, 1 << 20, 64, "bf16", 0, (), seed=1004, csr=True,
                  band_hint=64, graph_seed=2004, bwd=False),
     "extreme_128m": _w("extreme_128m", 1, 1, 1 << 27, 64, "bf16", 32, range(0, 27), seed=1005,

@@ -408,28 +408,40 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(L::bSFree + sb));
 
-            // mask: r <= u <= r+W-1 and key >= 0, with u = 128 b + c
+            // mask: r <= u <= r+W-1 and key >= 0, with u = 128 b + c, i.e. the
+            // column range [c_lo, c_hi] of this block.  Scores stay raw (the
+            // scale is folded into the exponent's FFMA); a masked raw score is
+            // set to the extreme that the max/min below ignores.
             const int64_t u0 = b * BN;
             const bool need_mask = (u0 < BM - 1) || (u0 + BN - 1 > (int64_t)W - 1) ||
                                    (u0 + q0 < (int64_t)W - 1);
-            float mblk = -INFINITY;
+            const bool pos = c2 >= 0.f;
+            const float ext = pos ? -INFINITY : INFINITY;
             if (need_mask) {
                 const int64_t lo = ((int64_t)r > (int64_t)W - 1 - q0) ? r : (int64_t)W - 1 - q0;
                 const int64_t hi = (int64_t)r + W - 1;
+                const int c_lo = (int)(lo - u0 < 0 ? 0 : (lo - u0 > BN ? BN : lo - u0));
+                const int c_hi = (int)(hi - u0 > BN - 1 ? BN - 1 : (hi - u0 < -1 ? -1 : hi - u0));
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    const int64_t u = u0 + c;
-                    const bool keep = (u >= lo) && (u <= hi);
-                    s[c] = keep ? s[c] * c2 : -INFINITY;
-                    mblk = fmaxf(mblk, s[c]);
-                }
+                for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : ext;
+            }
+            float mr[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) mr[x] = ext;
+            if (pos) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) mr[c & 7] = fmaxf(mr[c & 7], s[c]);
+#pragma unroll
+                for (int x = 4; x > 0; x >>= 1)
+                    for (int y = 0; y < x; ++y) mr[y] = fmaxf(mr[y], mr[y + x]);
             } else {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    s[c] *= c2;
-                    mblk = fmaxf(mblk, s[c]);
-                }
+                for (int c = 0; c < BN; ++c) mr[c & 7] = fminf(mr[c & 7], s[c]);
+#pragma unroll
+                for (int x = 4; x > 0; x >>= 1)
+                    for (int y = 0; y < x; ++y) mr[y] = fminf(mr[y], mr[y + x]);
             }
+            const float mblk = (mr[0] == ext) ? -INFINITY : mr[0] * c2;
             // conditional rescale of O (and l) when the max grows by more than 2^8
             const bool grow = mblk > m_run + kRescaleThreshold;
             if (__any_sync(0xffffffffu, grow)) {
@@ -467,20 +479,38 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             }
             uint8_t *prow = sm + L::kP + pb * L::kPTile;
             const float m_use = (m_run == -INFINITY) ? 0.f : m_run;  // all-masked row: p = 0
-            float lsum = 0.f;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            if (need_mask) {
 #pragma unroll
-            for (int c8 = 0; c8 < BN / 8; ++c8) {
-                uint32_t w[4];
+                for (int c8 = 0; c8 < BN / 8; ++c8) {
+                    uint32_t w[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = tc::ex2(s[8 * c8 + 2 * e] - m_use);
-                    const float p1 = tc::ex2(s[8 * c8 + 2 * e + 1] - m_use);
-                    lsum += p0 + p1;
-                    w[e] = tc::pack_bf16x2(p0, p1);
+                    for (int e = 0; e < 4; ++e) {
+                        const float x0 = s[8 * c8 + 2 * e], x1 = s[8 * c8 + 2 * e + 1];
+                        const float p0 = (x0 != ext) ? tc::ex2(fmaf(x0, c2, -m_use)) : 0.f;
+                        const float p1 = (x1 != ext) ? tc::ex2(fmaf(x1, c2, -m_use)) : 0.f;
+                        ls[e] += p0 + p1;
+                        w[e] = tc::pack_bf16x2(p0, p1);
+                    }
+                    *(uint4 *)(prow + (c8 >> 3) * (BM * 128) + tc::sw128_off(r, c8 & 7)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
                 }
-                *(uint4 *)(prow + (c8 >> 3) * (BM * 128) + tc::sw128_off(r, c8 & 7)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
+            } else {
+#pragma unroll
+                for (int c8 = 0; c8 < BN / 8; ++c8) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float p0 = tc::ex2(fmaf(s[8 * c8 + 2 * e], c2, -m_use));
+                        const float p1 = tc::ex2(fmaf(s[8 * c8 + 2 * e + 1], c2, -m_use));
+                        ls[e] += p0 + p1;
+                        w[e] = tc::pack_bf16x2(p0, p1);
+                    }
+                    *(uint4 *)(prow + (c8 >> 3) * (BM * 128) + tc::sw128_off(r, c8 & 7)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
             }
+            const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
             l_run += lsum;
             tc::fence_proxy_async_smem();
             tc::tmem_st_wait();
@@ -561,7 +591,7 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.err = sa_device_error_word();
     if (!a.err) return SA_ERR_CUDA;
     auto kern = band_fwd_kernel<D, BS, DS, PB>;
-    SA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc));
+    SA_CUDA_TRY(sa_smem_optin((const void *)kern, L::kAlloc));
     dim3 grid((unsigned)((T + BM - 1) / BM), (unsigned)BH);
     SA_LAUNCH("band_fwd", s, kern<<<grid, 256, L::kAlloc, s>>>(mq, mk, mv, a));
     SA_CUDA_TRY(cudaGetLastError());

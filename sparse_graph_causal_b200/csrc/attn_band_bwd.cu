@@ -96,23 +96,56 @@ __device__ __forceinline__ void load_row_packed(const uint8_t *tile, int rows, i
     }
 }
 
+// a . b over one row, a in registers (packed bf16 pairs), b row r of a tile.
 template <int D>
-__device__ __forceinline__ float dot_packed(const uint32_t *a, const uint32_t *b) {
-    float s = 0.f;
+__device__ __forceinline__ float dot_reg_smem(const uint32_t *a, const uint8_t *tile, int rows,
+                                              int r) {
+    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int x = 0; x < D / 2; ++x) {
-        s = fmaf(tc::bf16lo(a[x]), tc::bf16lo(b[x]), s);
-        s = fmaf(tc::bf16hi(a[x]), tc::bf16hi(b[x]), s);
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 x = *(const uint4 *)(tile + tile_off(rows, r, c));
+        const uint32_t b[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            s0 = fmaf(tc::bf16lo(a[4 * c + e]), tc::bf16lo(b[e]), s0);
+            s1 = fmaf(tc::bf16hi(a[4 * c + e]), tc::bf16hi(b[e]), s1);
+        }
     }
-    return s;
+    return s0 + s1;
 }
 
+// a . b with both rows in shared memory (row r of each tile).
 template <int D>
-__device__ __forceinline__ void axpy_packed(float *acc, float a, const uint32_t *x) {
+__device__ __forceinline__ float dot_smem_smem(const uint8_t *ta, const uint8_t *tb, int rows,
+                                               int r) {
+    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int e = 0; e < D / 2; ++e) {
-        acc[2 * e] = fmaf(a, tc::bf16lo(x[e]), acc[2 * e]);
-        acc[2 * e + 1] = fmaf(a, tc::bf16hi(x[e]), acc[2 * e + 1]);
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 x = *(const uint4 *)(ta + tile_off(rows, r, c));
+        const uint4 y = *(const uint4 *)(tb + tile_off(rows, r, c));
+        const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            s0 = fmaf(tc::bf16lo(xa[e]), tc::bf16lo(yb[e]), s0);
+            s1 = fmaf(tc::bf16hi(xa[e]), tc::bf16hi(yb[e]), s1);
+        }
+    }
+    return s0 + s1;
+}
+
+// acc += a * (row r of a tile)
+template <int D>
+__device__ __forceinline__ void axpy_smem(float *acc, float a, const uint8_t *tile, int rows,
+                                          int r) {
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 x = *(const uint4 *)(tile + tile_off(rows, r, c));
+        const uint32_t b[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc[8 * c + 2 * e] = fmaf(a, tc::bf16lo(b[e]), acc[8 * c + 2 * e]);
+            acc[8 * c + 2 * e + 1] = fmaf(a, tc::bf16hi(b[e]), acc[8 * c + 2 * e + 1]);
+        }
     }
 }
 
@@ -399,12 +432,11 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                     const bool valid = row_ok && (a.kind == 0 ? i >= a.offs[a.n_off - n_diag + d]
                                                               : d < resid);
                     if (valid) {
-                        uint32_t kr[D / 2], vr[D / 2];
-                        load_row_packed<D>(sm + L::kDiagK + st * L::kRow, BM, r, kr);
-                        load_row_packed<D>(sm + L::kDiagV + st * L::kRow, BM, r, vr);
-                        const float p = tc::ex2(dot_packed<D>(qr, kr) * c2 - lse2);
-                        const float ds = p * (dot_packed<D>(dor, vr) - Delta);
-                        axpy_packed<D>(acc, ds, kr);
+                        const uint8_t *kt = sm + L::kDiagK + st * L::kRow;
+                        const uint8_t *vt = sm + L::kDiagV + st * L::kRow;
+                        const float p = tc::ex2(fmaf(dot_reg_smem<D>(qr, kt, BM, r), c2, -lse2));
+                        const float ds = p * (dot_reg_smem<D>(dor, vt, BM, r) - Delta);
+                        axpy_smem<D>(acc, ds, kt, BM, r);
                     }
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
@@ -434,13 +466,21 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             if (lane == 0) tc::mbar_arrive(bar(L::bSFree + sb));
             const bool need_mask = (u0 < BM - 1) || (u0 + BB - 1 > (int64_t)W - 1) ||
                                    (u0 + q0 < (int64_t)W - 1);
-            const int64_t lo = ((int64_t)r > (int64_t)W - 1 - q0) ? r : (int64_t)W - 1 - q0;
-            const int64_t hi = (int64_t)r + W - 1;
+            if (need_mask) {
+                // keep columns [c_lo, c_hi]: r <= u <= r+W-1 and key >= 0
+                const int64_t lo = ((int64_t)r > (int64_t)W - 1 - q0) ? r : (int64_t)W - 1 - q0;
+                const int64_t hi = (int64_t)r + W - 1;
+                const int c_lo = (int)(lo - u0 < 0 ? 0 : (lo - u0 > BB ? BB : lo - u0));
+                const int c_hi = (int)(hi - u0 > BB - 1 ? BB - 1 : (hi - u0 < -1 ? -1 : hi - u0));
 #pragma unroll
-            for (int c = 0; c < BB; ++c) {
-                const bool keep = !need_mask || ((u0 + c >= lo) && (u0 + c <= hi));
-                const float p = keep ? tc::ex2(s[c] * c2 - lse2) : 0.f;
-                s[c] = p * (dp[c] - Delta);  // dS
+                for (int c = 0; c < BB; ++c) {
+                    const float p =
+                        (c >= c_lo && c <= c_hi) ? tc::ex2(fmaf(s[c], c2, -lse2)) : 0.f;
+                    s[c] = p * (dp[c] - Delta);  // dS
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < BB; ++c) s[c] = tc::ex2(fmaf(s[c], c2, -lse2)) * (dp[c] - Delta);
             }
             if (bl >= PB) WAIT_OR(bar(L::bDSDone + pb), ((bl - PB) / PB) & 1, ok = false; break);
             store_row64_bf16(sm + L::kDS + pb * L::kDSTile, r, s);
@@ -683,9 +723,6 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
 #pragma unroll
             for (int x = 0; x < D; ++x) adk[x] = adv[x] = 0.f;
             if (DS > 0 && n_diag > 0) {
-                uint32_t kr[D / 2], vr[D / 2];
-                load_row_packed<D>(sm + L::kK, BM, r, kr);
-                load_row_packed<D>(sm + L::kV, BM, r, vr);
                 int64_t rs = 0, nb = 0, resid = 0;
                 if (a.kind == 1 && row_ok) {
                     rs = a.rev_rowptr[j];
@@ -707,13 +744,13 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
                     if (i >= 0) {
                         const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
                         const float lse2 = a.lse[gi] * kLog2e, Dl = a.delta[gi];
-                        uint32_t qr[D / 2], dr[D / 2];
-                        load_row_packed<D>(sm + L::kDiagQ + st * L::kRow, BM, r, qr);
-                        load_row_packed<D>(sm + L::kDiagDO + st * L::kRow, BM, r, dr);
-                        const float p = tc::ex2(dot_packed<D>(qr, kr) * c2 - lse2);
-                        const float ds = p * (dot_packed<D>(dr, vr) - Dl);
-                        axpy_packed<D>(adv, p, dr);
-                        axpy_packed<D>(adk, ds, qr);
+                        const uint8_t *qt = sm + L::kDiagQ + st * L::kRow;
+                        const uint8_t *dt = sm + L::kDiagDO + st * L::kRow;
+                        const float p =
+                            tc::ex2(fmaf(dot_smem_smem<D>(qt, sm + L::kK, BM, r), c2, -lse2));
+                        const float ds = p * (dot_smem_smem<D>(dt, sm + L::kV, BM, r) - Dl);
+                        axpy_smem<D>(adv, p, dt, BM, r);
+                        axpy_smem<D>(adk, ds, qt, BM, r);
                     }
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
@@ -745,15 +782,28 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
             const float *del_s = (const float *)(sm + L::kDel + st * 256);
             const bool need_mask = (v0 < BM - 1) || (v0 + BB - 1 > (int64_t)W - 1) ||
                                    (k0 + v0 + BB - 1 > T - 1);
-            const int64_t lo = r, hi = (int64_t)r + W - 1;
-            const int64_t vlim = T - 1 - k0;
+            if (need_mask) {
+                // keep columns [c_lo, c_hi]: r <= v <= r+W-1 and query < T
+                const int64_t vlim = T - 1 - k0;
+                int64_t hi = (int64_t)r + W - 1;
+                if (hi > vlim) hi = vlim;
+                const int64_t lo = r;
+                const int c_lo = (int)(lo - v0 < 0 ? 0 : (lo - v0 > BB ? BB : lo - v0));
+                const int c_hi = (int)(hi - v0 > BB - 1 ? BB - 1 : (hi - v0 < -1 ? -1 : hi - v0));
 #pragma unroll
-            for (int c = 0; c < BB; ++c) {
-                const int64_t vv = v0 + c;
-                const bool keep = !need_mask || (vv >= lo && vv <= hi && vv <= vlim);
-                const float p = keep ? tc::ex2(s[c] * c2 - lse_s[c]) : 0.f;
-                s[c] = p;
-                dp[c] = p * (dp[c] - del_s[c]);
+                for (int c = 0; c < BB; ++c) {
+                    const float p =
+                        (c >= c_lo && c <= c_hi) ? tc::ex2(fmaf(s[c], c2, -lse_s[c])) : 0.f;
+                    s[c] = p;
+                    dp[c] = p * (dp[c] - del_s[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < BB; ++c) {
+                    const float p = tc::ex2(fmaf(s[c], c2, -lse_s[c]));
+                    s[c] = p;
+                    dp[c] = p * (dp[c] - del_s[c]);
+                }
             }
             if (bl >= PB) WAIT_OR(bar(L::bPDone + pb), ((bl - PB) / PB) & 1, ok = false; break);
             store_row64_bf16(sm + L::kP + pb * L::kPTile, r, s);
@@ -821,8 +871,8 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     if (!a.err) return SA_ERR_CUDA;
     auto kq = band_bwd_dq_kernel<D, BS, DS, PB>;
     auto kkv = band_bwd_dkdv_kernel<D, BS, DS, PB>;
-    SA_CUDA_TRY(cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, LQ::kAlloc));
-    SA_CUDA_TRY(cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, LK::kAlloc));
+    SA_CUDA_TRY(sa_smem_optin((const void *)kq, LQ::kAlloc));
+    SA_CUDA_TRY(sa_smem_optin((const void *)kkv, LK::kAlloc));
     dim3 grid((unsigned)((T + BM - 1) / BM), (unsigned)BH);
     SA_LAUNCH("band_bwd_dq", s, kq<<<grid, 256, LQ::kAlloc, s>>>(mq, mk, mv, mdo, a));
     SA_LAUNCH("band_bwd_dkdv", s, kkv<<<grid, 256, LK::kAlloc, s>>>(mq, mk, mv, mdo, a));

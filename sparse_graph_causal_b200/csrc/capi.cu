@@ -54,6 +54,20 @@ sa_status check_common(const sa_tensor *q, sa_graph g) {
 
 void sa_count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+cudaError_t sa_smem_optin(const void *kernel, int bytes) {
+    static std::mutex mu;
+    static std::vector<std::pair<const void *, int>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
+    for (auto &d : done)
+        if (d.first == kernel && d.second == dev) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.emplace_back(kernel, dev);
+    return e;
+}
+
 namespace {
 struct ProfRecord {
     const char *name;

@@ -122,6 +122,7 @@ def test_extreme_128m_fwd(sa, oracle_lib):
     """B1 H1 T2^27 D64, window 32 + 2^k (k = 0..26), inputs drawn on the
     device: 4096 sampled rows against the oracle."""
     w = synth.WORKLOADS["extreme_128m"]
+    torch.cuda.empty_cache()
     free, _ = torch.cuda.mem_get_info()
     need = 4 * w.T * w.D * 2 + 4 * w.T + (2 << 30)
     if free < need:

@@ -177,6 +177,11 @@ sa_status sparse_attn_set_path(int32_t path);
  * check, SA_ERR_CUDA on a CUDA error, else SA_OK. */
 sa_status sparse_attn_check_device(void *stream);
 
+/* Description of the last CUDA failure this thread saw inside the library
+ * (the failing call and CUDA's error name and string), "" if none.  The
+ * pointer stays valid until the thread's next failing call. */
+const char *sparse_attn_last_error_message(void);
+
 /* Number of kernel launches this library has enqueued on the calling host
  * thread's device since process start (for launch accounting). */
 int64_t sparse_attn_launch_count(void);

@@ -49,6 +49,7 @@ def _load():
         "sparse_attn_set_path": (st, [i32]),
         "sparse_attn_check_device": (st, [vp]),
         "sparse_attn_launch_count": (i64, []),
+        "sparse_attn_last_error_message": (ctypes.c_char_p, []),
         "sparse_attn_bwd_noalloc": (st, [P(SaTensor), P(SaTensor), P(SaTensor), P(SaTensor), vp,
                                          P(SaTensor), vp, ctypes.c_float, P(SaTensor),
                                          P(SaTensor), P(SaTensor), vp]),
@@ -79,7 +80,10 @@ _lib = _LazyLib()
 class SparseAttentionError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {sparse_attn_status_string(status)} (status {status})")
+        detail = ""
+        if status == SA_ERR_CUDA:
+            detail = " [" + sparse_attn_last_error_message() + "]"
+        super().__init__(f"{where}: {sparse_attn_status_string(status)} (status {status}){detail}")
 
 
 def _check(status: int, where: str):
@@ -274,6 +278,10 @@ def sparse_attn_set_path(path: int):
 
 def sparse_attn_check_device(stream=None):
     _check(_lib.sparse_attn_check_device(_stream(stream)), "sparse_attn_check_device")
+
+
+def sparse_attn_last_error_message() -> str:
+    return (_lib.sparse_attn_last_error_message() or b"").decode()
 
 
 def sparse_attn_launch_count() -> int:

@@ -59,22 +59,24 @@ struct FwdArgs {
     int *err;
 };
 
-template <int D, int BS, int DS, int PB>
+template <int D, int KS, int VS, int DS, int PB>
 struct Layout {
     static constexpr int kTile = BM * D * 2;            // 128 rows x D bf16
     static constexpr int kQ = 0;
     static constexpr int kBandK = kQ + kTile;
-    static constexpr int kBandV = kBandK + BS * kTile;
-    static constexpr int kP = kBandV + BS * kTile;
+    static constexpr int kBandV = kBandK + KS * kTile;
+    static constexpr int kP = kBandV + VS * kTile;
     static constexpr int kPTile = BM * BN * 2;
     static constexpr int kDiagK = kP + PB * kPTile;
     static constexpr int kDiagV = kDiagK + DS * kTile;
     static constexpr int kBars = kDiagV + DS * kTile;
     // barriers
     static constexpr int bQFull = 0;
-    static constexpr int bBandFull = 1;
-    static constexpr int bBandEmpty = bBandFull + BS;
-    static constexpr int bSFull = bBandEmpty + BS;
+    static constexpr int bKFull = 1;
+    static constexpr int bKEmpty = bKFull + KS;
+    static constexpr int bVFull = bKEmpty + KS;
+    static constexpr int bVEmpty = bVFull + VS;
+    static constexpr int bSFull = bVEmpty + VS;
     static constexpr int bSFree = bSFull + 2;
     static constexpr int bPFull = bSFree + 2;
     static constexpr int bPVDone = bPFull + PB;
@@ -96,11 +98,12 @@ __device__ __forceinline__ int64_t band_first_block(int64_t q0, int32_t W) {
     return need > 0 ? need / BN : 0;
 }
 
-template <int D, int BS, int DS, int PB>
+template <int D, int KS, int VS, int DS, int PB>
 __global__ void __launch_bounds__(256, 1)
 band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
-    using L = Layout<D, BS, DS, PB>;
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkr,
+                const __grid_constant__ CUtensorMap tvr, const FwdArgs a) {
+    using L = Layout<D, KS, VS, DS, PB>;
     constexpr int DSX = DS > 0 ? DS : 1;  // ring modulus (no diagonal ring when DS == 0)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -124,9 +127,13 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
 
     if (tid == 0) {
         tc::mbar_init(bar(L::bQFull), 1);
-        for (int s = 0; s < BS; ++s) {
-            tc::mbar_init(bar(L::bBandFull + s), 1);
-            tc::mbar_init(bar(L::bBandEmpty + s), 1);
+        for (int s = 0; s < KS; ++s) {
+            tc::mbar_init(bar(L::bKFull + s), 1);
+            tc::mbar_init(bar(L::bKEmpty + s), 1);
+        }
+        for (int s = 0; s < VS; ++s) {
+            tc::mbar_init(bar(L::bVFull + s), 1);
+            tc::mbar_init(bar(L::bVEmpty + s), 1);
         }
         for (int s = 0; s < 2; ++s) {
             tc::mbar_init(bar(L::bSFull + s), 1);
@@ -138,7 +145,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         }
         tc::mbar_init(bar(L::bOInit), 4);
         for (int s = 0; s < DS; ++s) {
-            tc::mbar_init(bar(L::bDiagFull + s), a.kind == 0 ? 1 : 64);
+            tc::mbar_init(bar(L::bDiagFull + s), 1);
             tc::mbar_init(bar(L::bDiagEmpty + s), 4);
         }
         *abort = 0;
@@ -178,20 +185,36 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             for (int x = 0; x < D / 64; ++x)
                 tc::tma_load_3d(sbase + L::kQ + x * (BM * 128), &tq, x * 64, (int32_t)q0,
                                 (int32_t)bh, bar(L::bQFull));
-            for (int bl = 0; bl < n_band; ++bl) {
-                const int st = bl % BS, use = bl / BS;
-                if (use > 0 &&
-                    !tc::mbar_wait(bar(L::bBandEmpty + st), (use - 1) & 1, abort, a.err,
-                                   SA_DEVERR_TIMEOUT))
-                    break;
+            // K runs one block ahead of V: K(b) is released as soon as S(b) is
+            // done, V(b) only after P(b) V(b)
+            auto load_k = [&](int bl) -> bool {
+                const int st = bl % KS, use = bl / KS;
+                if (use > 0 && !tc::mbar_wait(bar(L::bKEmpty + st), (use - 1) & 1, abort, a.err,
+                                              SA_DEVERR_TIMEOUT))
+                    return false;
                 const int32_t krow = (int32_t)(kb0 + (b_first + bl) * BN);
-                tc::mbar_arrive_expect_tx(bar(L::bBandFull + st), 2 * L::kTile);
-                for (int x = 0; x < D / 64; ++x) {
+                tc::mbar_arrive_expect_tx(bar(L::bKFull + st), L::kTile);
+                for (int x = 0; x < D / 64; ++x)
                     tc::tma_load_3d(sbase + L::kBandK + st * L::kTile + x * (BN * 128), &tk,
-                                    x * 64, krow, (int32_t)bh, bar(L::bBandFull + st));
+                                    x * 64, krow, (int32_t)bh, bar(L::bKFull + st));
+                return true;
+            };
+            auto load_v = [&](int bl) -> bool {
+                const int st = bl % VS, use = bl / VS;
+                if (use > 0 && !tc::mbar_wait(bar(L::bVEmpty + st), (use - 1) & 1, abort, a.err,
+                                              SA_DEVERR_TIMEOUT))
+                    return false;
+                const int32_t krow = (int32_t)(kb0 + (b_first + bl) * BN);
+                tc::mbar_arrive_expect_tx(bar(L::bVFull + st), L::kTile);
+                for (int x = 0; x < D / 64; ++x)
                     tc::tma_load_3d(sbase + L::kBandV + st * L::kTile + x * (BN * 128), &tv,
-                                    x * 64, krow, (int32_t)bh, bar(L::bBandFull + st));
-                }
+                                    x * 64, krow, (int32_t)bh, bar(L::bVFull + st));
+                return true;
+            };
+            bool ok = n_band > 0 ? load_k(0) : true;
+            for (int bl = 0; ok && bl < n_band; ++bl) {
+                if (bl + 1 < n_band && !load_k(bl + 1)) break;
+                if (!load_v(bl)) break;
             }
         }
     } else if (warp == 1) {
@@ -201,8 +224,8 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             const uint32_t idO = tc::idesc_bf16(BM, D, false, true);
             bool ok = tc::mbar_wait(bar(L::bQFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
             auto issue_S = [&](int bl) -> bool {
-                const int st = bl % BS, sb = bl & 1;
-                if (!tc::mbar_wait(bar(L::bBandFull + st), (bl / BS) & 1, abort, a.err,
+                const int st = bl % KS, sb = bl & 1;
+                if (!tc::mbar_wait(bar(L::bKFull + st), (bl / KS) & 1, abort, a.err,
                                    SA_DEVERR_TIMEOUT))
                     return false;
                 if (bl >= 2 && !tc::mbar_wait(bar(L::bSFree + sb), ((bl >> 1) - 1) & 1, abort,
@@ -217,25 +240,27 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                                     tc::sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
                 }
                 tc::mma_commit(bar(L::bSFull + sb));
+                tc::mma_commit(bar(L::bKEmpty + st));
                 return true;
             };
             if (ok && n_band > 0) ok = issue_S(0);
             for (int bl = 0; ok && bl < n_band; ++bl) {
-                // with two or more ring stages S of the next block overlaps the
-                // softmax of this one; with one stage its K arrives only after
-                // this block's PV has released the stage
-                if (BS >= 2 && bl + 1 < n_band && !issue_S(bl + 1)) break;
-                const int pb = bl % PB;
+                // S of the next block overlaps the softmax of this one (with a
+                // single K stage its K arrives once S of this block is done)
+                if (bl + 1 < n_band && !issue_S(bl + 1)) break;
+                const int pb = bl % PB, vst = bl % VS;
                 if (bl == 0 &&
                     !tc::mbar_wait(bar(L::bOInit), 0, abort, a.err, SA_DEVERR_TIMEOUT))
                     break;
                 if (!tc::mbar_wait(bar(L::bPFull + pb), (bl / PB) & 1, abort, a.err,
                                    SA_DEVERR_TIMEOUT))
                     break;
+                if (!tc::mbar_wait(bar(L::bVFull + vst), (bl / VS) & 1, abort, a.err,
+                                   SA_DEVERR_TIMEOUT))
+                    break;
                 tc::tc_fence_after();
-                const int st = bl % BS;
                 const uint32_t pa = sbase + L::kP + pb * L::kPTile;
-                const uint32_t va = sbase + L::kBandV + st * L::kTile;
+                const uint32_t va = sbase + L::kBandV + vst * L::kTile;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint32_t offp = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
@@ -243,15 +268,29 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     tc::mma_bf16_ss(tmem + L::tO, tc::sdesc_sw128(pa + offp, 16, 1024),
                                     tc::sdesc_sw128(va + offv, BN * 128, 1024), idO, 1u);
                 }
-                tc::mma_commit(bar(L::bBandEmpty + st));
+                tc::mma_commit(bar(L::bVEmpty + vst));
                 tc::mma_commit(bar(L::bPVDone + pb));
-                if (BS == 1 && bl + 1 < n_band && !issue_S(bl + 1)) break;
             }
         }
     } else if (warp == 2 || warp == 3) {
-        // ---------------- diagonal-block producers
-        if (DS > 0) {
-            const int pt = tid - 64;  // 0..63
+        // warp 2 stages the diagonal blocks; warp 3 has no role
+        // ---------------- diagonal-block producer
+        if (warp == 2 && DS > 0) {
+            // CSR: lane l owns rows 4l .. 4l+3: list start, residual count and
+            // the key of the next slot (fetched one slot ahead)
+            int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
+            int32_t cj[4] = {0, 0, 0, 0};
+            if (a.kind == 1) {
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int64_t i = q0 + 4 * lane + h;
+                    if (i < T) {
+                        cstart[h] = a.rowptr[i];
+                        cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
+                        if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
+                    }
+                }
+            }
             for (int d = 0; d < n_diag; ++d) {
                 const int st = d % DSX, use = d / DSX;
                 const uint32_t kdst = sbase + L::kDiagK + st * L::kTile;
@@ -259,11 +298,11 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 if (use > 0 && !tc::mbar_wait(bar(L::bDiagEmpty + st), (use - 1) & 1, abort,
                                               a.err, SA_DEVERR_TIMEOUT))
                     break;
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kTile);
                 if (a.kind == 0) {
-                    if (pt == 0) {
+                    if (lane == 0) {
                         // distance links: keys q0-o .. q0+127-o, one box each for K and V
                         const int32_t krow = (int32_t)(q0 - a.offs[a.n_off - n_diag + d]);
-                        tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kTile);
                         for (int x = 0; x < D / 64; ++x) {
                             tc::tma_load_3d(kdst + x * (BM * 128), &tk, x * 64, krow, (int32_t)bh,
                                             bar(L::bDiagFull + st));
@@ -272,27 +311,30 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         }
                     }
                 } else {
-                    // CSR slot d of every row: 8 lanes per row, one 16-byte chunk each
-                    constexpr int CH = D / 8;  // 16-byte chunks per row
-                    for (int item = pt; item < BM * CH; item += 64) {
-                        const int r = item / CH, c = item % CH;
-                        const int64_t i = q0 + r;
-                        if (i >= T) continue;
-                        const int64_t rs = a.rowptr[i];
-                        const int64_t deg = a.rowptr[i + 1] - rs;
-                        const int64_t inband = (i + 1 < W) ? i + 1 : W;
-                        if (d >= deg - inband) continue;
-                        const int64_t j = a.colidx[rs + d];
-                        const size_t src = ((size_t)bh * (size_t)T + (size_t)j) * D + c * 8;
-                        const uint32_t off = (c >> 3) * (BM * 128) + tc::sw128_off(r, c & 7);
-                        tc::cp_async_16(kdst + off, a.k + src);
-                        tc::cp_async_16(vdst + off, a.v + src);
+                    // CSR slot d: 4-row TMA gathers of K and V rows (unswizzled);
+                    // a row without slot d loads its own key (masked later)
+                    int32_t rr[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const int64_t i = q0 + 4 * lane + h;
+                        const int64_t j = d < cres[h] ? (int64_t)cj[h] : (i < T ? i : 0);
+                        rr[h] = (int32_t)(bh * T + j);
                     }
-                    tc::cp_async_mbar_arrive(bar(L::bDiagFull + st));
+#pragma unroll
+                    for (int x = 0; x < D / 64; ++x) {
+                        const uint32_t off = x * (BM * 128) + 4 * lane * 128;
+                        tc::tma_gather4(kdst + off, &tkr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                        bar(L::bDiagFull + st));
+                        tc::tma_gather4(vdst + off, &tvr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                        bar(L::bDiagFull + st));
+                    }
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        if (d + 1 < cres[h]) cj[h] = a.colidx[cstart[h] + d + 1];
                 }
             }
         }
-    } else {
+    } else if (warp >= 4 && warp < 8) {
         // ---------------- softmax warpgroup: thread r = query row r = TMEM lane r
         const int r = tid - 128;
         const int64_t i = q0 + r;
@@ -311,10 +353,17 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 ok = tc::mbar_wait(bar(L::bQFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
                 uint32_t qr[D / 2];
                 if (ok) {
+                    // Structured blocks are swizzled like Q: q in logical order.
+                    // CSR gathers are unswizzled: reading them at the swizzled
+                    // address gives chunk c ^ (r & 7), which pairs with the
+                    // physical (unpermuted-address) chunks of the Q row; the
+                    // accumulator is then in that permuted order (undone below).
 #pragma unroll
                     for (int c = 0; c < D / 8; ++c) {
-                        const uint4 w4 = *(const uint4 *)(sm + L::kQ + (c >> 3) * (BM * 128) +
-                                                          tc::sw128_off(r, c & 7));
+                        const uint32_t qoff = (c >> 3) * (BM * 128) +
+                                              (a.kind == 0 ? tc::sw128_off(r, c & 7)
+                                                           : (uint32_t)r * 128u + ((c & 7) << 4));
+                        const uint4 w4 = *(const uint4 *)(sm + L::kQ + qoff);
                         qr[4 * c] = w4.x;
                         qr[4 * c + 1] = w4.y;
                         qr[4 * c + 2] = w4.z;
@@ -374,6 +423,29 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     }
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                }
+                if (a.kind == 1) {
+                    // undo the chunk permutation through the (now idle) first
+                    // diagonal stage: row r of D fp32 at r * 4D bytes
+                    tc::named_barrier(1, 128);
+                    float *scr = (float *)(sm + L::kDiagK) + (size_t)r * D;
+#pragma unroll
+                    for (int t = 0; t < D / 8; ++t) {
+                        const int lc = (t & ~7) | ((t & 7) ^ (r & 7));
+                        *(float4 *)(scr + 8 * lc) =
+                            make_float4(acc[8 * t], acc[8 * t + 1], acc[8 * t + 2], acc[8 * t + 3]);
+                        *(float4 *)(scr + 8 * lc + 4) = make_float4(
+                            acc[8 * t + 4], acc[8 * t + 5], acc[8 * t + 6], acc[8 * t + 7]);
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int t = 0; t < D / 4; ++t) {
+                        const float4 f = *(const float4 *)(scr + 4 * t);
+                        acc[4 * t] = f.x;
+                        acc[4 * t + 1] = f.y;
+                        acc[4 * t + 2] = f.z;
+                        acc[4 * t + 3] = f.w;
+                    }
                 }
             }
             // initialise O (columns tO .. tO+D) with the diagonal part
@@ -564,17 +636,22 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     }
 }
 
-template <int D, int BS, int DS, int PB>
+template <int D, int KS, int VS, int DS, int PB>
 sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_graph_s *g, float scale, sa_tensor *out, float *lse,
                           cudaStream_t s) {
-    using L = Layout<D, BS, DS, PB>;
+    using L = Layout<D, KS, VS, DS, PB>;
     static_assert(L::kAlloc <= 232448, "shared memory budget");
     const int64_t BH = q->B * q->H, T = q->T;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mkr, mvr;
     if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BM) || !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BH, BN) ||
-        !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BH, BN))
+        !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BH, BN) ||
+        !sa_tmap_bf16_rows(&mkr, k->ptr, D, (uint64_t)(BH * T)) ||
+        !sa_tmap_bf16_rows(&mvr, v->ptr, D, (uint64_t)(BH * T)))
+    {
+        sa_record_cuda_error(cudaErrorInvalidValue, "band_fwd: tensor map encoding");
         return SA_ERR_CUDA;
+    }
     FwdArgs a{};
     a.T = T;
     a.W = g->W;
@@ -590,10 +667,10 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.scale2 = scale * kLog2e;
     a.err = sa_device_error_word();
     if (!a.err) return SA_ERR_CUDA;
-    auto kern = band_fwd_kernel<D, BS, DS, PB>;
+    auto kern = band_fwd_kernel<D, KS, VS, DS, PB>;
     SA_CUDA_TRY(sa_smem_optin((const void *)kern, L::kAlloc));
     dim3 grid((unsigned)((T + BM - 1) / BM), (unsigned)BH);
-    SA_LAUNCH("band_fwd", s, kern<<<grid, 256, L::kAlloc, s>>>(mq, mk, mv, a));
+    SA_LAUNCH("band_fwd", s, kern<<<grid, 256, L::kAlloc, s>>>(mq, mk, mv, mkr, mvr, a));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
@@ -612,10 +689,12 @@ sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
                       const sa_graph_s *g, const GraphView &, float scale, sa_tensor *out,
                       float *lse, cudaStream_t s) {
     const bool diag = (g->kind == 0) ? g->n_off > 0 : g->max_resid > 0;
+    // <D, K stages, V stages, diagonal stages, P buffers>, sized to the
+    // 227 KB of shared memory
     if (q->D == 64) {
-        return diag ? launch_band_fwd<64, 2, 2, 2>(q, k, v, g, scale, out, lse, s)
-                    : launch_band_fwd<64, 2, 0, 2>(q, k, v, g, scale, out, lse, s);
+        return diag ? launch_band_fwd<64, 2, 3, 2, 2>(q, k, v, g, scale, out, lse, s)
+                    : launch_band_fwd<64, 2, 3, 0, 2>(q, k, v, g, scale, out, lse, s);
     }
-    return diag ? launch_band_fwd<128, 1, 1, 1>(q, k, v, g, scale, out, lse, s)
-                : launch_band_fwd<128, 2, 0, 1>(q, k, v, g, scale, out, lse, s);
+    return diag ? launch_band_fwd<128, 1, 1, 1, 1>(q, k, v, g, scale, out, lse, s)
+                : launch_band_fwd<128, 2, 3, 0, 1>(q, k, v, g, scale, out, lse, s);
 }

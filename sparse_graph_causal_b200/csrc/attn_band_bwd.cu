@@ -26,6 +26,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "sa_band.cuh"
 #include "tc_common.cuh"
 #include "tmap.cuh"
@@ -96,6 +98,29 @@ __device__ __forceinline__ void load_row_packed(const uint8_t *tile, int rows, i
     }
 }
 
+// acc holds chunk t at logical chunk t ^ (r & 7) (per 64-column half): put it
+// back in logical order through row r of a D-float scratch row in shared memory.
+template <int D>
+__device__ __forceinline__ void unpermute_row(float *acc, float *scr_row, int r) {
+#pragma unroll
+    for (int t = 0; t < D / 8; ++t) {
+        const int lc = (t & ~7) | ((t & 7) ^ (r & 7));
+        *(float4 *)(scr_row + 8 * lc) =
+            make_float4(acc[8 * t], acc[8 * t + 1], acc[8 * t + 2], acc[8 * t + 3]);
+        *(float4 *)(scr_row + 8 * lc + 4) =
+            make_float4(acc[8 * t + 4], acc[8 * t + 5], acc[8 * t + 6], acc[8 * t + 7]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int t = 0; t < D / 4; ++t) {
+        const float4 f = *(const float4 *)(scr_row + 4 * t);
+        acc[4 * t] = f.x;
+        acc[4 * t + 1] = f.y;
+        acc[4 * t + 2] = f.z;
+        acc[4 * t + 3] = f.w;
+    }
+}
+
 // a . b over one row, a in registers (packed bf16 pairs), b row r of a tile.
 template <int D>
 __device__ __forceinline__ float dot_reg_smem(const uint32_t *a, const uint8_t *tile, int rows,
@@ -109,6 +134,27 @@ __device__ __forceinline__ float dot_reg_smem(const uint32_t *a, const uint8_t *
         for (int e = 0; e < 4; ++e) {
             s0 = fmaf(tc::bf16lo(a[4 * c + e]), tc::bf16lo(b[e]), s0);
             s1 = fmaf(tc::bf16hi(a[4 * c + e]), tc::bf16hi(b[e]), s1);
+        }
+    }
+    return s0 + s1;
+}
+
+// a . b, a = row r of a swizzled tile read in physical chunk order, b = row r
+// of an unswizzled gathered tile read at the swizzled address (so both give
+// logical chunk t ^ (r & 7) at step t).
+template <int D>
+__device__ __forceinline__ float dot_phys_gathered(const uint8_t *ta, const uint8_t *tb, int rows,
+                                                   int r) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 x = *(const uint4 *)(ta + (c >> 3) * (rows * 128) + r * 128 + ((c & 7) << 4));
+        const uint4 y = *(const uint4 *)(tb + tile_off(rows, r, c));
+        const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            s0 = fmaf(tc::bf16lo(xa[e]), tc::bf16lo(yb[e]), s0);
+            s1 = fmaf(tc::bf16hi(xa[e]), tc::bf16hi(yb[e]), s1);
         }
     }
     return s0 + s1;
@@ -229,7 +275,9 @@ template <int D, int BS, int DS, int PB>
 __global__ void __launch_bounds__(256, 1)
 band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                    const __grid_constant__ CUtensorMap tv,
-                   const __grid_constant__ CUtensorMap tdo, const BwdArgs a) {
+                   const __grid_constant__ CUtensorMap tdo,
+                   const __grid_constant__ CUtensorMap tkr,
+                   const __grid_constant__ CUtensorMap tvr, const BwdArgs a) {
     using L = LayoutDQ<D, BS, DS, PB>;
     constexpr int DSX = L::DSX;
     extern __shared__ uint8_t smem_raw[];
@@ -266,7 +314,7 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         }
         tc::mbar_init(bar(L::bInit), 4);
         for (int s = 0; s < DSX; ++s) {
-            tc::mbar_init(bar(L::bDiagFull + s), a.kind == 0 ? 1 : 64);
+            tc::mbar_init(bar(L::bDiagFull + s), 1);
             tc::mbar_init(bar(L::bDiagEmpty + s), 4);
         }
         *abort = 0;
@@ -354,39 +402,58 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             }
         }
     } else if (warp == 2 || warp == 3) {
-        if (DS > 0) {
-            const int pt = tid - 64;
+        // warp 2 stages the diagonal blocks; warp 3 has no role
+        if (warp == 2 && DS > 0) {
+            // CSR: lane l owns rows 4l .. 4l+3 (list start, residual count, next key)
+            int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
+            int32_t cj[4] = {0, 0, 0, 0};
+            if (a.kind == 1) {
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int64_t i = q0 + 4 * lane + h;
+                    if (i < T) {
+                        cstart[h] = a.rowptr[i];
+                        cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
+                        if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
+                    }
+                }
+            }
             for (int d = 0; d < n_diag; ++d) {
                 const int st = d % DSX, use = d / DSX;
                 const uint32_t kdst = sbase + L::kDiagK + st * L::kRow;
                 const uint32_t vdst = sbase + L::kDiagV + st * L::kRow;
                 if (use > 0) WAIT_OR(bar(L::bDiagEmpty + st), (use - 1) & 1, break);
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kRow);
                 if (a.kind == 0) {
-                    if (pt == 0) {
+                    if (lane == 0) {
                         const int64_t krow = q0 - a.offs[a.n_off - n_diag + d];
-                        tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kRow);
                         tma_tile128<D>(kdst, &tk, krow, bh, bar(L::bDiagFull + st));
                         tma_tile128<D>(vdst, &tv, krow, bh, bar(L::bDiagFull + st));
                     }
                 } else {
-                    constexpr int CH = D / 8;
-                    for (int item = pt; item < BM * CH; item += 64) {
-                        const int r = item / CH, c = item % CH;
-                        const int64_t i = q0 + r;
-                        if (i >= T) continue;
-                        const int64_t rs = a.rowptr[i], deg = a.rowptr[i + 1] - rs;
-                        if (d >= deg - ((i + 1 < W) ? i + 1 : W)) continue;
-                        const int64_t j = a.colidx[rs + d];
-                        const size_t src = ((size_t)bh * (size_t)T + (size_t)j) * D + c * 8;
-                        const uint32_t off = tile_off(BM, r, c);
-                        tc::cp_async_16(kdst + off, a.k + src);
-                        tc::cp_async_16(vdst + off, a.v + src);
+                    int32_t rr[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const int64_t i = q0 + 4 * lane + h;
+                        const int64_t j = d < cres[h] ? (int64_t)cj[h] : (i < T ? i : 0);
+                        rr[h] = (int32_t)(bh * T + j);
                     }
-                    tc::cp_async_mbar_arrive(bar(L::bDiagFull + st));
+#pragma unroll
+                    for (int x = 0; x < D / 64; ++x) {
+                        const uint32_t off = x * (BM * 128) + 4 * lane * 128;
+                        tc::tma_gather4(kdst + off, &tkr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                        bar(L::bDiagFull + st));
+                        tc::tma_gather4(vdst + off, &tvr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                        bar(L::bDiagFull + st));
+                    }
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        if (d + 1 < cres[h]) cj[h] = a.colidx[cstart[h] + d + 1];
                 }
             }
         }
-    } else {
+    } else if (warp >= 4 && warp < 8) {
+        // compute warpgroup: thread r = owned row r = TMEM lane r
         const int r = tid - 128;
         const int64_t i = q0 + r;
         const bool row_ok = i < T;
@@ -421,25 +488,47 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
 #pragma unroll
             for (int x = 0; x < D; ++x) acc[x] = 0.f;
             if (DS > 0 && n_diag > 0) {
-                uint32_t qr[D / 2];
-                load_row_packed<D>(sm + L::kQ, BM, r, qr);
-                int64_t resid = 0;
-                if (a.kind == 1 && row_ok)
-                    resid = (a.rowptr[i + 1] - a.rowptr[i]) - ((i + 1 < W) ? i + 1 : W);
-                for (int d = 0; d < n_diag; ++d) {
-                    const int st = d % DSX;
-                    WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
-                    const bool valid = row_ok && (a.kind == 0 ? i >= a.offs[a.n_off - n_diag + d]
-                                                              : d < resid);
-                    if (valid) {
-                        const uint8_t *kt = sm + L::kDiagK + st * L::kRow;
-                        const uint8_t *vt = sm + L::kDiagV + st * L::kRow;
-                        const float p = tc::ex2(fmaf(dot_reg_smem<D>(qr, kt, BM, r), c2, -lse2));
-                        const float ds = p * (dot_reg_smem<D>(dor, vt, BM, r) - Delta);
-                        axpy_smem<D>(acc, ds, kt, BM, r);
+                if (a.kind == 0) {
+                    // distance links: swizzled tiles, q in logical chunk order
+                    uint32_t qr[D / 2];
+                    load_row_packed<D>(sm + L::kQ, BM, r, qr);
+                    for (int d = 0; d < n_diag; ++d) {
+                        const int st = d % DSX;
+                        WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
+                        if (row_ok && i >= a.offs[a.n_off - n_diag + d]) {
+                            const uint8_t *kt = sm + L::kDiagK + st * L::kRow;
+                            const uint8_t *vt = sm + L::kDiagV + st * L::kRow;
+                            const float p =
+                                tc::ex2(fmaf(dot_reg_smem<D>(qr, kt, BM, r), c2, -lse2));
+                            const float ds = p * (dot_reg_smem<D>(dor, vt, BM, r) - Delta);
+                            axpy_smem<D>(acc, ds, kt, BM, r);
+                        }
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
                     }
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                } else {
+                    // CSR gathers are unswizzled: pair them with the physical
+                    // chunk order of the swizzled q and dO rows (see the forward)
+                    int64_t resid = 0;
+                    if (row_ok)
+                        resid = (a.rowptr[i + 1] - a.rowptr[i]) - ((i + 1 < W) ? i + 1 : W);
+                    for (int d = 0; d < n_diag; ++d) {
+                        const int st = d % DSX;
+                        WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
+                        if (row_ok && d < resid) {
+                            const uint8_t *kt = sm + L::kDiagK + st * L::kRow;
+                            const uint8_t *vt = sm + L::kDiagV + st * L::kRow;
+                            const float p = tc::ex2(
+                                fmaf(dot_phys_gathered<D>(sm + L::kQ, kt, BM, r), c2, -lse2));
+                            const float ds =
+                                p * (dot_phys_gathered<D>(sm + L::kDO, vt, BM, r) - Delta);
+                            axpy_smem<D>(acc, ds, kt, BM, r);
+                        }
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                    }
+                    tc::named_barrier(1, 128);
+                    unpermute_row<D>(acc, (float *)(sm + L::kDiagK) + (size_t)r * D, r);
                 }
             }
             tmem_store_row<D>(tDQ, acc);
@@ -531,7 +620,9 @@ template <int D, int BS, int DS, int PB>
 __global__ void __launch_bounds__(256, 1)
 band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv,
-                     const __grid_constant__ CUtensorMap tdo, const BwdArgs a) {
+                     const __grid_constant__ CUtensorMap tdo,
+                     const __grid_constant__ CUtensorMap tqr,
+                     const __grid_constant__ CUtensorMap tdor, const BwdArgs a) {
     using L = LayoutDKV<D, BS, DS, PB>;
     constexpr int DSX = L::DSX;
     extern __shared__ uint8_t smem_raw[];
@@ -567,7 +658,7 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         }
         tc::mbar_init(bar(L::bInit), 4);
         for (int s = 0; s < DSX; ++s) {
-            tc::mbar_init(bar(L::bDiagFull + s), a.kind == 0 ? 1 : 64);
+            tc::mbar_init(bar(L::bDiagFull + s), 1);
             tc::mbar_init(bar(L::bDiagEmpty + s), 4);
         }
         *abort = 0;
@@ -675,40 +766,61 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
             }
         }
     } else if (warp == 2 || warp == 3) {
-        if (DS > 0) {
-            const int pt = tid - 64;
+        // warp 2 stages the diagonal blocks; warp 3 has no role
+        if (warp == 2 && DS > 0) {
+            // CSR: lane l owns key rows 4l .. 4l+3: start of the residual part of
+            // their transpose lists (after the band queries j .. j+W-1), its
+            // length, and the next query
+            int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
+            int32_t cj[4] = {0, 0, 0, 0};
+            if (a.kind == 1) {
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int64_t j = k0 + 4 * lane + h;
+                    if (j < T) {
+                        const int64_t nb = (T - j < W) ? T - j : W;
+                        cstart[h] = a.rev_rowptr[j] + nb;
+                        cres[h] = a.rev_rowptr[j + 1] - cstart[h];
+                        if (cres[h] > 0) cj[h] = a.rev_colidx[cstart[h]];
+                    }
+                }
+            }
             for (int d = 0; d < n_diag; ++d) {
                 const int st = d % DSX, use = d / DSX;
                 const uint32_t qdst = sbase + L::kDiagQ + st * L::kRow;
                 const uint32_t ddst = sbase + L::kDiagDO + st * L::kRow;
                 if (use > 0) WAIT_OR(bar(L::bDiagEmpty + st), (use - 1) & 1, break);
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kRow);
                 if (a.kind == 0) {
-                    if (pt == 0) {
+                    if (lane == 0) {
                         const int64_t qrow = k0 + a.offs[off_first + d];
-                        tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kRow);
                         tma_tile128<D>(qdst, &tq, qrow, bh, bar(L::bDiagFull + st));
                         tma_tile128<D>(ddst, &tdo, qrow, bh, bar(L::bDiagFull + st));
                     }
                 } else {
-                    constexpr int CH = D / 8;
-                    for (int item = pt; item < BM * CH; item += 64) {
-                        const int r = item / CH, c = item % CH;
-                        const int64_t j = k0 + r;
-                        if (j >= T) continue;
-                        const int64_t rs = a.rev_rowptr[j], deg = a.rev_rowptr[j + 1] - rs;
-                        const int64_t nb = (T - j < W) ? T - j : W;
-                        if (d >= deg - nb) continue;
-                        const int64_t i = a.rev_colidx[rs + nb + d];
-                        const size_t src = ((size_t)bh * (size_t)T + (size_t)i) * D + c * 8;
-                        const uint32_t off = tile_off(BM, r, c);
-                        tc::cp_async_16(qdst + off, a.q + src);
-                        tc::cp_async_16(ddst + off, a.dout + src);
+                    int32_t rr[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const int64_t j = k0 + 4 * lane + h;
+                        const int64_t i = d < cres[h] ? (int64_t)cj[h] : (j < T ? j : 0);
+                        rr[h] = (int32_t)(bh * T + i);
                     }
-                    tc::cp_async_mbar_arrive(bar(L::bDiagFull + st));
+#pragma unroll
+                    for (int x = 0; x < D / 64; ++x) {
+                        const uint32_t off = x * (BM * 128) + 4 * lane * 128;
+                        tc::tma_gather4(qdst + off, &tqr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                        bar(L::bDiagFull + st));
+                        tc::tma_gather4(ddst + off, &tdor, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                        bar(L::bDiagFull + st));
+                    }
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        if (d + 1 < cres[h]) cj[h] = a.rev_colidx[cstart[h] + d + 1];
                 }
             }
         }
-    } else {
+    } else if (warp >= 4 && warp < 8) {
+        // compute warpgroup: thread r = owned row r = TMEM lane r
         const int r = tid - 128;
         const int64_t j = k0 + r;
         const bool row_ok = j < T;
@@ -723,37 +835,63 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
 #pragma unroll
             for (int x = 0; x < D; ++x) adk[x] = adv[x] = 0.f;
             if (DS > 0 && n_diag > 0) {
-                int64_t rs = 0, nb = 0, resid = 0;
-                if (a.kind == 1 && row_ok) {
-                    rs = a.rev_rowptr[j];
-                    nb = (T - j < W) ? T - j : W;
-                    resid = a.rev_rowptr[j + 1] - rs - nb;
-                }
-                for (int d = 0; d < n_diag; ++d) {
-                    const int st = d % DSX;
-                    WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
-                    int64_t i = -1;
-                    if (row_ok) {
-                        if (a.kind == 0) {
+                if (a.kind == 0) {
+                    // distance links: query j + o, swizzled tiles read in logical order
+                    for (int d = 0; d < n_diag; ++d) {
+                        const int st = d % DSX;
+                        WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
+                        int64_t i = -1;
+                        if (row_ok) {
                             const int64_t cand = j + a.offs[off_first + d];
                             if (cand < T) i = cand;
-                        } else if (d < resid) {
-                            i = a.rev_colidx[rs + nb + d];
                         }
+                        if (i >= 0) {
+                            const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
+                            const float lse2 = a.lse[gi] * kLog2e, Dl = a.delta[gi];
+                            const uint8_t *qt = sm + L::kDiagQ + st * L::kRow;
+                            const uint8_t *dt = sm + L::kDiagDO + st * L::kRow;
+                            const float sdot = dot_smem_smem<D>(qt, sm + L::kK, BM, r);
+                            const float dpdot = dot_smem_smem<D>(dt, sm + L::kV, BM, r);
+                            const float p = tc::ex2(fmaf(sdot, c2, -lse2));
+                            const float ds = p * (dpdot - Dl);
+                            axpy_smem<D>(adv, p, dt, BM, r);
+                            axpy_smem<D>(adk, ds, qt, BM, r);
+                        }
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
                     }
-                    if (i >= 0) {
-                        const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
-                        const float lse2 = a.lse[gi] * kLog2e, Dl = a.delta[gi];
-                        const uint8_t *qt = sm + L::kDiagQ + st * L::kRow;
-                        const uint8_t *dt = sm + L::kDiagDO + st * L::kRow;
-                        const float p =
-                            tc::ex2(fmaf(dot_smem_smem<D>(qt, sm + L::kK, BM, r), c2, -lse2));
-                        const float ds = p * (dot_smem_smem<D>(dt, sm + L::kV, BM, r) - Dl);
-                        axpy_smem<D>(adv, p, dt, BM, r);
-                        axpy_smem<D>(adk, ds, qt, BM, r);
+                } else {
+                    // CSR gathers are unswizzled: the key's k and v rows read in
+                    // physical chunk order pair with them (see the forward)
+                    int64_t rs = 0, nb = 0, resid = 0;
+                    if (row_ok) {
+                        rs = a.rev_rowptr[j];
+                        nb = (T - j < W) ? T - j : W;
+                        resid = a.rev_rowptr[j + 1] - rs - nb;
                     }
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                    for (int d = 0; d < n_diag; ++d) {
+                        const int st = d % DSX;
+                        WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
+                        const int64_t i = (row_ok && d < resid) ? a.rev_colidx[rs + nb + d] : -1;
+                        if (i >= 0) {
+                            const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
+                            const float lse2 = a.lse[gi] * kLog2e, Dl = a.delta[gi];
+                            const uint8_t *qt = sm + L::kDiagQ + st * L::kRow;
+                            const uint8_t *dt = sm + L::kDiagDO + st * L::kRow;
+                            const float sdot = dot_phys_gathered<D>(sm + L::kK, qt, BM, r);
+                            const float dpdot = dot_phys_gathered<D>(sm + L::kV, dt, BM, r);
+                            const float p = tc::ex2(fmaf(sdot, c2, -lse2));
+                            const float ds = p * (dpdot - Dl);
+                            axpy_smem<D>(adv, p, dt, BM, r);
+                            axpy_smem<D>(adk, ds, qt, BM, r);
+                        }
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                    }
+                    tc::named_barrier(1, 128);
+                    float *scr = (float *)(sm + L::kDiagQ);
+                    unpermute_row<D>(adv, scr + (size_t)r * D, r);
+                    unpermute_row<D>(adk, scr + (size_t)(BM + r) * D, r);
                 }
             }
             tmem_store_row<D>(tDV, adv);
@@ -831,20 +969,26 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
     }
 }
 
-template <int D, int BS, int DS, int PB>
+template <int D, int BSQ, int BSK, int DS, int PBQ, int PBK>
 sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_tensor *o, const float *lse, const sa_tensor *dout,
                           const sa_graph_s *g, float scale, sa_tensor *dq, sa_tensor *dk,
                           sa_tensor *dv, float *delta, cudaStream_t s) {
-    using LQ = LayoutDQ<D, BS, DS, PB>;
-    using LK = LayoutDKV<D, BS, DS, PB>;
+    using LQ = LayoutDQ<D, BSQ, DS, PBQ>;
+    using LK = LayoutDKV<D, BSK, DS, PBK>;
     static_assert(LQ::kAlloc <= 232448 && LK::kAlloc <= 232448, "shared memory budget");
     const int64_t BH = q->B * q->H, T = q->T;
-    CUtensorMap mq, mk, mv, mdo;
+    CUtensorMap mq, mk, mv, mdo, mqr, mkr, mvr, mdor;
+    const uint64_t rows = (uint64_t)(BH * T);
     if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BB) || !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BH, BB) ||
         !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BH, BB) ||
-        !sa_tmap_bf16_3d(&mdo, dout->ptr, D, T, BH, BB))
+        !sa_tmap_bf16_3d(&mdo, dout->ptr, D, T, BH, BB) ||
+        !sa_tmap_bf16_rows(&mqr, q->ptr, D, rows) || !sa_tmap_bf16_rows(&mkr, k->ptr, D, rows) ||
+        !sa_tmap_bf16_rows(&mvr, v->ptr, D, rows) || !sa_tmap_bf16_rows(&mdor, dout->ptr, D, rows))
+    {
+        sa_record_cuda_error(cudaErrorInvalidValue, "band_bwd: tensor map encoding");
         return SA_ERR_CUDA;
+    }
     BwdArgs a{};
     a.T = T;
     a.W = g->W;
@@ -869,13 +1013,14 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.scale2 = scale * kLog2e;
     a.err = sa_device_error_word();
     if (!a.err) return SA_ERR_CUDA;
-    auto kq = band_bwd_dq_kernel<D, BS, DS, PB>;
-    auto kkv = band_bwd_dkdv_kernel<D, BS, DS, PB>;
+    auto kq = band_bwd_dq_kernel<D, BSQ, DS, PBQ>;
+    auto kkv = band_bwd_dkdv_kernel<D, BSK, DS, PBK>;
     SA_CUDA_TRY(sa_smem_optin((const void *)kq, LQ::kAlloc));
     SA_CUDA_TRY(sa_smem_optin((const void *)kkv, LK::kAlloc));
     dim3 grid((unsigned)((T + BM - 1) / BM), (unsigned)BH);
-    SA_LAUNCH("band_bwd_dq", s, kq<<<grid, 256, LQ::kAlloc, s>>>(mq, mk, mv, mdo, a));
-    SA_LAUNCH("band_bwd_dkdv", s, kkv<<<grid, 256, LK::kAlloc, s>>>(mq, mk, mv, mdo, a));
+    SA_LAUNCH("band_bwd_dq", s, kq<<<grid, 256, LQ::kAlloc, s>>>(mq, mk, mv, mdo, mkr, mvr, a));
+    SA_LAUNCH("band_bwd_dkdv", s,
+              kkv<<<grid, 256, LK::kAlloc, s>>>(mq, mk, mv, mdo, mqr, mdor, a));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
@@ -898,10 +1043,13 @@ sa_status sa_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
                       const sa_graph_s *g, const GraphView &, float scale, sa_tensor *dq,
                       sa_tensor *dk, sa_tensor *dv, float *delta, cudaStream_t s) {
     const bool diag = (g->kind == 0) ? g->n_off > 0 : (g->max_resid > 0 || g->max_resid_rev > 0);
+    // <D, dQ ring stages, dK/dV ring stages, diagonal stages, dS buffers,
+    //  P^T/dS^T buffers>, sized to the 227 KB of shared memory
     if (q->D == 64)
-        return diag ? launch_band_bwd<64, 2, 2, 2>(q, k, v, out, lse, dout, g, scale, dq, dk, dv,
-                                                   delta, s)
-                    : launch_band_bwd<64, 2, 0, 2>(q, k, v, out, lse, dout, g, scale, dq, dk, dv,
-                                                   delta, s);
-    return launch_band_bwd<128, 2, 0, 2>(q, k, v, out, lse, dout, g, scale, dq, dk, dv, delta, s);
+        return diag ? launch_band_bwd<64, 4, 3, 2, 2, 2>(q, k, v, out, lse, dout, g, scale, dq,
+                                                         dk, dv, delta, s)
+                    : launch_band_bwd<64, 4, 3, 0, 2, 2>(q, k, v, out, lse, dout, g, scale, dq,
+                                                         dk, dv, delta, s);
+    return launch_band_bwd<128, 4, 3, 0, 2, 1>(q, k, v, out, lse, dout, g, scale, dq, dk, dv,
+                                               delta, s);
 }

@@ -54,6 +54,16 @@ sa_status check_common(const sa_tensor *q, sa_graph g) {
 
 void sa_count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+namespace {
+thread_local std::string t_last_error;
+}
+
+void sa_record_cuda_error(cudaError_t e, const char *where) {
+    const char *f = where ? strrchr(where, '/') : nullptr;
+    t_last_error = std::string(f ? f + 1 : (where ? where : "?")) + ": " + cudaGetErrorName(e) +
+                   " (" + cudaGetErrorString(e) + ")";
+}
+
 cudaError_t sa_smem_optin(const void *kernel, int bytes) {
     static std::mutex mu;
     static std::vector<std::pair<const void *, int>> done;
@@ -140,6 +150,8 @@ sa_status sparse_attn_set_path(int32_t path) {
 
 int64_t sparse_attn_launch_count(void) { return g_launches.load(); }
 
+const char *sparse_attn_last_error_message(void) { return t_last_error.c_str(); }
+
 sa_status sparse_attn_profile_begin(int32_t enable) {
     g_prof_on.store(enable ? 1 : 0);
     return SA_OK;
@@ -186,12 +198,12 @@ int32_t sparse_attn_profile_end(char *names, int32_t name_len, int32_t *launches
 
 sa_status sparse_attn_check_device(void *stream) {
     cudaStream_t s = as_stream(stream);
-    if (cudaStreamSynchronize(s) != cudaSuccess) return SA_ERR_CUDA;
+    SA_CUDA_TRY(cudaStreamSynchronize(s));
     int h = 0;
-    if (cudaMemcpyFromSymbol(&h, g_device_error, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
+    SA_CUDA_TRY(cudaMemcpyFromSymbol(&h, g_device_error, sizeof(int)));
     if (h) {
         int z = 0;
-        if (cudaMemcpyToSymbol(g_device_error, &z, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
+        SA_CUDA_TRY(cudaMemcpyToSymbol(g_device_error, &z, sizeof(int)));
         return (h & SA_DEVERR_TIMEOUT) ? SA_ERR_DEVICE_TIMEOUT : SA_ERR_CUDA;
     }
     return SA_OK;

@@ -104,10 +104,18 @@ __host__ __device__ inline int64_t sg_in_degree(int64_t j, int64_t T, int64_t W,
 cudaError_t sa_smem_optin(const void *kernel, int bytes);
 
 // CUDA error helpers (host)
-#define SA_CUDA_TRY(expr)                                   \
-    do {                                                    \
-        cudaError_t _e = (expr);                            \
-        if (_e != cudaSuccess) return SA_ERR_CUDA;          \
+// Record the failing CUDA call (file:line, expression, error string) for
+// sparse_attn_last_error_message().
+void sa_record_cuda_error(cudaError_t e, const char *where);
+#define SA_STR2(x) #x
+#define SA_STR(x) SA_STR2(x)
+#define SA_CUDA_TRY(expr)                                                         \
+    do {                                                                          \
+        cudaError_t _e = (expr);                                                  \
+        if (_e != cudaSuccess) {                                                  \
+            sa_record_cuda_error(_e, __FILE__ ":" SA_STR(__LINE__) ": " #expr);   \
+            return SA_ERR_CUDA;                                                   \
+        }                                                                         \
     } while (0)
 
 // Internal launchers (graph.cu)

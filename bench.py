@@ -68,6 +68,22 @@ def kernel_class(name: str) -> str:
     return "fwd"
 
 
+def ncu_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` at `workload` from the committed ncu
+    summary (profiles/traffic.json), or None when there is none or the
+    kernel's source changed since the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(p))[workload][kernel]
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    except (OSError, KeyError, ValueError):
+        return None
+    if hashlib.sha256(src).hexdigest() != rec["source_sha256"]:
+        return None
+    return rec["bytes"]
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -345,7 +361,7 @@ def run_gpu(args, dist, rank, world):
         achieved = alg_bytes / (avg_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                     "frac": achieved / hbm, "peak_source": f"{src} hbm_gbs"}
-    roofline.update({"traffic": None, "kernel": dom, "kernel_ms": avg_ms,
+    roofline.update({"traffic": ncu_traffic(w.name, dom), "kernel": dom, "kernel_ms": avg_ms,
                      "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
                      "kernel_shares": shares,
                      "kernel_ms_all": {n: t / c for n, (c, t) in kt.items()}})

@@ -20,6 +20,8 @@ Workloads (shapes from the pages' own experiments, values synthetic):
                 "Longer Attention Span ...")
   extreme_128m  B1 H1 T2^27 D64 bf16, window 32 + 2^k links k=0..26, inputs
                 drawn on the device
+  extreme_8m    B1 H1 T2^23 D64 bf16, window 32 + 2^k links k=0..22 (profiler-
+                capture size of extreme_128m)
 """
 from __future__ import annotations
 
@@ -76,6 +78,9 @@ WORKLOADS = {
                  band_hint=64, graph_seed=2004, bwd=False),
     "extreme_128m": _w("extreme_128m", 1, 1, 1 << 27, 64, "bf16", 32, range(0, 27), seed=1005,
                        bwd=False),
+    # a 1/16-length version of extreme_128m: the size used for profiler captures
+    "extreme_8m": _w("extreme_8m", 1, 1, 1 << 23, 64, "bf16", 32, range(0, 23), seed=1005,
+                     bwd=False),
 }
 
 

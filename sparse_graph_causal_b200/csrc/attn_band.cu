@@ -1,6 +1,7 @@
 // attn_band.cu -- forward on tcgen05 band tiles fused with the gathered edges.
 //
-// One CTA owns 128 consecutive queries [q0, q0+128) of one (b, h) slice.
+// A tile is 128 consecutive queries [q0, q0+128) of one (b, h) slice; the
+// kernel is persistent (one CTA per SM walking its share of the tiles).
 //  * Window edges (the band of "MiniGPT (Part 6)", section "A mask is not
 //    enough": keys j <= i with i - j < W) run as dense 128 x 128 tiles on the
 //    tensor cores: keys [q0-W+1, q0+127] are cut into blocks of 128 starting
@@ -45,6 +46,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct FwdArgs {
     int64_t T;
+    int64_t BH;
     int32_t W;          // band width (structured window or verified CSR band)
     int32_t kind;       // 0 structured, 1 CSR
     int32_t n_off;
@@ -59,74 +61,93 @@ struct FwdArgs {
     int *err;
 };
 
-template <int D, int KS, int VS, int DS, int PB>
+template <int D, int KS, int VS, int DS>
 struct Layout {
     static constexpr int kTile = BM * D * 2;            // 128 rows x D bf16
-    static constexpr int kQ = 0;
-    static constexpr int kBandK = kQ + kTile;
+    static constexpr int kQ = 0;                        // two Q buffers
+    static constexpr int kBandK = kQ + 2 * kTile;
     static constexpr int kBandV = kBandK + KS * kTile;
-    static constexpr int kP = kBandV + VS * kTile;
-    static constexpr int kPTile = BM * BN * 2;
-    static constexpr int kDiagK = kP + PB * kPTile;
+    static constexpr int kDiagK = kBandV + VS * kTile;
     static constexpr int kDiagV = kDiagK + DS * kTile;
     static constexpr int kBars = kDiagV + DS * kTile;
-    // barriers
-    static constexpr int bQFull = 0;
-    static constexpr int bKFull = 1;
-    static constexpr int bKEmpty = bKFull + KS;
-    static constexpr int bVFull = bKEmpty + KS;
-    static constexpr int bVEmpty = bVFull + VS;
-    static constexpr int bSFull = bVEmpty + VS;
-    static constexpr int bSFree = bSFull + 2;
-    static constexpr int bPFull = bSFree + 2;
-    static constexpr int bPVDone = bPFull + PB;
-    static constexpr int bOInit = bPVDone + PB;
-    static constexpr int bDiagFull = bOInit + 1;
-    static constexpr int bDiagEmpty = bDiagFull + (DS > 0 ? DS : 1);
-    static constexpr int nBars = bDiagEmpty + (DS > 0 ? DS : 1);
-    static constexpr int kMisc = kBars + nBars * 8;      // tmem slot, abort, n_diag
+    static constexpr int DSX = DS > 0 ? DS : 1;          // ring modulus
+    // barriers (S, P, PVDone per S buffer: P is written over S in TMEM)
+    static constexpr int bQFull = 0, bQEmpty = 2;
+    static constexpr int bKFull = 4, bKEmpty = bKFull + KS;
+    static constexpr int bVFull = bKEmpty + KS, bVEmpty = bVFull + VS;
+    static constexpr int bSFull = bVEmpty + VS, bSFree = bSFull + 2;
+    static constexpr int bPFull = bSFree + 2, bPVDone = bPFull + 2;
+    static constexpr int bOInit = bPVDone + 2;
+    static constexpr int bDiagFull = bOInit + 1, bDiagEmpty = bDiagFull + DSX;
+    static constexpr int bInfoFull = bDiagEmpty + DSX, bInfoEmpty = bInfoFull + 2;
+    static constexpr int bGroup = bInfoEmpty + 2;        // 128-thread softmax barrier
+    static constexpr int nBars = bGroup + 1;
+    static constexpr int kMisc = kBars + nBars * 8;      // tmem slot, abort, info[2]
     static constexpr int kTotal = kMisc + 16;
     static constexpr int kAlloc = kTotal + 1024;         // alignment slack
-    // TMEM columns: S buffers [0,128) and [128,256), O at 256
+    // TMEM columns: S buffers [0,128) and [128,256) (P, bf16, over the first
+    // 64 columns of its S buffer), O at 256
     static constexpr uint32_t tS0 = 0, tO = 256;
     static constexpr uint32_t kTmemCols = 512;
 };
 
-__device__ __forceinline__ int64_t band_first_block(int64_t q0, int32_t W) {
-    // first block holding a key >= 0: u >= W-1-q0
-    int64_t need = (int64_t)W - 1 - q0;
-    return need > 0 ? need / BN : 0;
+// Geometry of query tile t (tiles run over B*H slices, 128 queries each).
+// 32-bit: the band path requires T < 2^31 and W + 127 < 2^31.
+struct TileGeom {
+    int32_t bh, q0, kb0, b_first, n_band;
+};
+
+__device__ __forceinline__ TileGeom tile_geom(int64_t t, int64_t ntq, int64_t T, int32_t W) {
+    TileGeom g;
+    const int64_t bh = t / ntq;
+    g.bh = (int32_t)bh;
+    g.q0 = (int32_t)((t - bh * ntq) * BM);
+    g.kb0 = g.q0 - W + 1;                                             // key of u = 0
+    const int32_t last_key = (g.q0 + BM - 1 < T - 1) ? g.q0 + BM - 1 : (int32_t)(T - 1);
+    const int32_t nblk = (last_key - g.kb0) / BN + 1;                 // blocks up to the last key
+    const int32_t need = W - 1 - g.q0;                                // first block with a key >= 0
+    g.b_first = need > 0 ? need / BN : 0;
+    g.n_band = nblk - g.b_first;
+    return g;
 }
 
-template <int D, int KS, int VS, int DS, int PB>
+// Persistent: each CTA walks the tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+// Every ring (Q, K, V, S, P, diagonal blocks) keeps its phase across tiles, so
+// the loads and MMAs of the next tile proceed while the current one finishes.
+template <int D, int KS, int VS, int DS>
 __global__ void __launch_bounds__(256, 1)
 band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkr,
                 const __grid_constant__ CUtensorMap tvr, const FwdArgs a) {
-    using L = Layout<D, KS, VS, DS, PB>;
-    constexpr int DSX = DS > 0 ? DS : 1;  // ring modulus (no diagonal ring when DS == 0)
+    using L = Layout<D, KS, VS, DS>;
+    constexpr int DSX = L::DSX;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_u32(sm);
-    uint64_t *bars = (uint64_t *)(sm + L::kBars);
     uint32_t *tmem_slot = (uint32_t *)(sm + L::kMisc);
     volatile int *abort = (volatile int *)(sm + L::kMisc + 4);
-    int *n_diag_s = (int *)(sm + L::kMisc + 8);
+    volatile int *info = (volatile int *)(sm + L::kMisc + 8);  // diagonal blocks of tile slot 0/1
     auto bar = [&](int b) { return sbase + L::kBars + 8u * (uint32_t)b; };
+    auto wait = [&](int b, uint32_t parity) {
+        return tc::mbar_wait(bar(b), parity, abort, a.err, SA_DEVERR_TIMEOUT);
+    };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t tile = blockIdx.x, bh = blockIdx.y;
-    const int64_t q0 = tile * BM;
     const int64_t T = a.T;
     const int32_t W = a.W;
-    const int64_t kb0 = q0 - W + 1;                              // key of u = 0
-    const int64_t last_key = (q0 + BM - 1 < T - 1) ? q0 + BM - 1 : T - 1;
-    const int64_t nblk = (last_key - kb0) / BN + 1;              // blocks up to the last key
-    const int64_t b_first = band_first_block(q0, W);
-    const int n_band = (int)(nblk - b_first);
+    const int64_t ntq = (T + BM - 1) / BM, ntiles = ntq * a.BH;
 
     if (tid == 0) {
-        tc::mbar_init(bar(L::bQFull), 1);
+        for (int s = 0; s < 2; ++s) {
+            tc::mbar_init(bar(L::bQFull + s), 1);
+            tc::mbar_init(bar(L::bQEmpty + s), 5);  // last S MMA commit + 4 softmax warps
+            tc::mbar_init(bar(L::bSFull + s), 1);
+            tc::mbar_init(bar(L::bSFree + s), 1);   // P V of the buffer's block done
+            tc::mbar_init(bar(L::bPFull + s), 4);
+            tc::mbar_init(bar(L::bPVDone + s), 1);
+            tc::mbar_init(bar(L::bInfoFull + s), 1);
+            tc::mbar_init(bar(L::bInfoEmpty + s), 4);
+        }
         for (int s = 0; s < KS; ++s) {
             tc::mbar_init(bar(L::bKFull + s), 1);
             tc::mbar_init(bar(L::bKEmpty + s), 1);
@@ -135,469 +156,522 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             tc::mbar_init(bar(L::bVFull + s), 1);
             tc::mbar_init(bar(L::bVEmpty + s), 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            tc::mbar_init(bar(L::bSFull + s), 1);
-            tc::mbar_init(bar(L::bSFree + s), 4);
-        }
-        for (int s = 0; s < PB; ++s) {
-            tc::mbar_init(bar(L::bPFull + s), 4);
-            tc::mbar_init(bar(L::bPVDone + s), 1);
-        }
         tc::mbar_init(bar(L::bOInit), 4);
-        for (int s = 0; s < DS; ++s) {
+        tc::mbar_init(bar(L::bGroup), 128);
+        for (int s = 0; s < DSX; ++s) {
             tc::mbar_init(bar(L::bDiagFull + s), 1);
             tc::mbar_init(bar(L::bDiagEmpty + s), 4);
         }
         *abort = 0;
-        *n_diag_s = 0;
         tc::fence_barrier_init();
     }
     if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), L::kTmemCols);
-    __syncthreads();
-
-    // number of diagonal blocks of this tile
-    if (warp >= 4) {
-        int nd = 0;
-        const int64_t i = q0 + (tid - 128);
-        if (a.kind == 0) {
-            const int64_t last = (q0 + BM - 1 < T - 1) ? q0 + BM - 1 : T - 1;
-            for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last) ? 1 : 0;
-        } else if (i < T) {
-            const int64_t deg = a.rowptr[i + 1] - a.rowptr[i];
-            const int64_t inband = (i + 1 < W) ? i + 1 : W;
-            nd = (int)(deg - inband);
-        }
-        atomicMax(n_diag_s, nd);
-    }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_diag = (DS > 0) ? *n_diag_s : 0;
 
     if (warp == 0) {
-        // ---------------- TMA producer: Q, then the band K/V ring
+        // ---------------- TMA producer: Q of each tile, then its band K/V ring
         if (lane == 0) {
             tc::tma_prefetch_desc(&tq);
             tc::tma_prefetch_desc(&tk);
             tc::tma_prefetch_desc(&tv);
-            tc::mbar_arrive_expect_tx(bar(L::bQFull), L::kTile);
-            for (int x = 0; x < D / 64; ++x)
-                tc::tma_load_3d(sbase + L::kQ + x * (BM * 128), &tq, x * 64, (int32_t)q0,
-                                (int32_t)bh, bar(L::bQFull));
-            // K runs one block ahead of V: K(b) is released as soon as S(b) is
-            // done, V(b) only after P(b) V(b)
-            auto load_k = [&](int bl) -> bool {
-                const int st = bl % KS, use = bl / KS;
-                if (use > 0 && !tc::mbar_wait(bar(L::bKEmpty + st), (use - 1) & 1, abort, a.err,
-                                              SA_DEVERR_TIMEOUT))
-                    return false;
-                const int32_t krow = (int32_t)(kb0 + (b_first + bl) * BN);
-                tc::mbar_arrive_expect_tx(bar(L::bKFull + st), L::kTile);
+            uint32_t kc = 0, vc = 0;  // K and V blocks loaded so far (all tiles)
+            bool ok = true;
+            int64_t lt = 0;
+            for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++lt) {
+                const TileGeom g = tile_geom(t, ntq, T, W);
+                const int qb = (int)(lt & 1);
+                if (lt >= 2 && !wait(L::bQEmpty + qb, (uint32_t)(((lt >> 1) - 1) & 1))) break;
+                tc::mbar_arrive_expect_tx(bar(L::bQFull + qb), L::kTile);
                 for (int x = 0; x < D / 64; ++x)
-                    tc::tma_load_3d(sbase + L::kBandK + st * L::kTile + x * (BN * 128), &tk,
-                                    x * 64, krow, (int32_t)bh, bar(L::bKFull + st));
-                return true;
-            };
-            auto load_v = [&](int bl) -> bool {
-                const int st = bl % VS, use = bl / VS;
-                if (use > 0 && !tc::mbar_wait(bar(L::bVEmpty + st), (use - 1) & 1, abort, a.err,
-                                              SA_DEVERR_TIMEOUT))
-                    return false;
-                const int32_t krow = (int32_t)(kb0 + (b_first + bl) * BN);
-                tc::mbar_arrive_expect_tx(bar(L::bVFull + st), L::kTile);
-                for (int x = 0; x < D / 64; ++x)
-                    tc::tma_load_3d(sbase + L::kBandV + st * L::kTile + x * (BN * 128), &tv,
-                                    x * 64, krow, (int32_t)bh, bar(L::bVFull + st));
-                return true;
-            };
-            bool ok = n_band > 0 ? load_k(0) : true;
-            for (int bl = 0; ok && bl < n_band; ++bl) {
-                if (bl + 1 < n_band && !load_k(bl + 1)) break;
-                if (!load_v(bl)) break;
+                    tc::tma_load_3d(sbase + L::kQ + qb * L::kTile + x * (BM * 128), &tq, x * 64,
+                                    (int32_t)g.q0, (int32_t)g.bh, bar(L::bQFull + qb));
+                // K runs one block ahead of V: K(b) is released as soon as S(b)
+                // is done, V(b) only after P(b) V(b)
+                auto load_k = [&](int bl) -> bool {
+                    const int st = (int)(kc % KS);
+                    const uint32_t use = kc / KS;
+                    if (use > 0 && !wait(L::bKEmpty + st, (use - 1) & 1)) return false;
+                    const int32_t krow = g.kb0 + (g.b_first + bl) * BN;
+                    tc::mbar_arrive_expect_tx(bar(L::bKFull + st), L::kTile);
+                    for (int x = 0; x < D / 64; ++x)
+                        tc::tma_load_3d(sbase + L::kBandK + st * L::kTile + x * (BN * 128), &tk,
+                                        x * 64, krow, (int32_t)g.bh, bar(L::bKFull + st));
+                    ++kc;
+                    return true;
+                };
+                auto load_v = [&](int bl) -> bool {
+                    const int st = (int)(vc % VS);
+                    const uint32_t use = vc / VS;
+                    if (use > 0 && !wait(L::bVEmpty + st, (use - 1) & 1)) return false;
+                    const int32_t krow = g.kb0 + (g.b_first + bl) * BN;
+                    tc::mbar_arrive_expect_tx(bar(L::bVFull + st), L::kTile);
+                    for (int x = 0; x < D / 64; ++x)
+                        tc::tma_load_3d(sbase + L::kBandV + st * L::kTile + x * (BN * 128), &tv,
+                                        x * 64, krow, (int32_t)g.bh, bar(L::bVFull + st));
+                    ++vc;
+                    return true;
+                };
+                ok = load_k(0);
+                for (int bl = 0; ok && bl < g.n_band; ++bl) {
+                    if (bl + 1 < g.n_band && !load_k(bl + 1)) ok = false;
+                    else if (!load_v(bl)) ok = false;
+                }
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer: S of block g, then P V of block g-1
         if (lane == 0) {
             const uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
             const uint32_t idO = tc::idesc_bf16(BM, D, false, true);
-            bool ok = tc::mbar_wait(bar(L::bQFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
-            auto issue_S = [&](int bl) -> bool {
-                const int st = bl % KS, sb = bl & 1;
-                if (!tc::mbar_wait(bar(L::bKFull + st), (bl / KS) & 1, abort, a.err,
-                                   SA_DEVERR_TIMEOUT))
-                    return false;
-                if (bl >= 2 && !tc::mbar_wait(bar(L::bSFree + sb), ((bl >> 1) - 1) & 1, abort,
-                                              a.err, SA_DEVERR_TIMEOUT))
-                    return false;
+            uint32_t kc = 0, gb = 0;  // K stages consumed, band blocks issued (all tiles)
+            bool have_pv = false, pv_first = false, ok = true;
+            uint32_t pv_gb = 0;
+            int64_t pv_lt = 0;
+            auto do_pv = [&]() -> bool {
+                const int sb = (int)(pv_gb & 1), vst = (int)(pv_gb % VS);
+                if (pv_first && !wait(L::bOInit, (uint32_t)(pv_lt & 1))) return false;
+                if (!wait(L::bPFull + sb, (pv_gb >> 1) & 1)) return false;
+                if (!wait(L::bVFull + vst, (pv_gb / VS) & 1)) return false;
                 tc::tc_fence_after();
-                const uint32_t qa = sbase + L::kQ, ka = sbase + L::kBandK + st * L::kTile;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                    tc::mma_bf16_ss(tmem + L::tS0 + sb * BN, tc::sdesc_sw128(qa + off, 16, 1024),
-                                    tc::sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
-                }
-                tc::mma_commit(bar(L::bSFull + sb));
-                tc::mma_commit(bar(L::bKEmpty + st));
-                return true;
-            };
-            if (ok && n_band > 0) ok = issue_S(0);
-            for (int bl = 0; ok && bl < n_band; ++bl) {
-                // S of the next block overlaps the softmax of this one (with a
-                // single K stage its K arrives once S of this block is done)
-                if (bl + 1 < n_band && !issue_S(bl + 1)) break;
-                const int pb = bl % PB, vst = bl % VS;
-                if (bl == 0 &&
-                    !tc::mbar_wait(bar(L::bOInit), 0, abort, a.err, SA_DEVERR_TIMEOUT))
-                    break;
-                if (!tc::mbar_wait(bar(L::bPFull + pb), (bl / PB) & 1, abort, a.err,
-                                   SA_DEVERR_TIMEOUT))
-                    break;
-                if (!tc::mbar_wait(bar(L::bVFull + vst), (bl / VS) & 1, abort, a.err,
-                                   SA_DEVERR_TIMEOUT))
-                    break;
-                tc::tc_fence_after();
-                const uint32_t pa = sbase + L::kP + pb * L::kPTile;
+                // A = P (bf16) in TMEM over the first 64 columns of its S buffer
+                const uint32_t pt = tmem + L::tS0 + sb * BN;
                 const uint32_t va = sbase + L::kBandV + vst * L::kTile;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint32_t offp = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                    const uint32_t offv = kk * 16 * 128;
-                    tc::mma_bf16_ss(tmem + L::tO, tc::sdesc_sw128(pa + offp, 16, 1024),
-                                    tc::sdesc_sw128(va + offv, BN * 128, 1024), idO, 1u);
-                }
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    tc::mma_bf16_ts(tmem + L::tO, pt + kk * 8,
+                                    tc::sdesc_sw128(va + kk * 16 * 128, BN * 128, 1024), idO, 1u);
                 tc::mma_commit(bar(L::bVEmpty + vst));
-                tc::mma_commit(bar(L::bPVDone + pb));
+                tc::mma_commit(bar(L::bPVDone + sb));
+                tc::mma_commit(bar(L::bSFree + sb));
+                return true;
+            };
+            int64_t lt = 0;
+            for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++lt) {
+                const TileGeom g = tile_geom(t, ntq, T, W);
+                const int qb = (int)(lt & 1);
+                if (!wait(L::bQFull + qb, (uint32_t)((lt >> 1) & 1))) break;
+                const uint32_t qa = sbase + L::kQ + qb * L::kTile;
+                for (int bl = 0; bl < g.n_band; ++bl) {
+                    const int st = (int)(kc % KS), sb = (int)(gb & 1);
+                    if (!wait(L::bKFull + st, (kc / KS) & 1) ||
+                        (gb >= 2 && !wait(L::bSFree + sb, ((gb >> 1) - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const uint32_t ka = sbase + L::kBandK + st * L::kTile;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        tc::mma_bf16_ss(tmem + L::tS0 + sb * BN,
+                                        tc::sdesc_sw128(qa + off, 16, 1024),
+                                        tc::sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
+                    }
+                    tc::mma_commit(bar(L::bSFull + sb));
+                    tc::mma_commit(bar(L::bKEmpty + st));
+                    if (bl == g.n_band - 1) tc::mma_commit(bar(L::bQEmpty + qb));
+                    ++kc;
+                    // the softmax of this block overlaps P V of the previous one
+                    if (have_pv && !do_pv()) {
+                        ok = false;
+                        break;
+                    }
+                    have_pv = true;
+                    pv_gb = gb;
+                    pv_first = (bl == 0);
+                    pv_lt = lt;
+                    ++gb;
+                }
             }
+            if (ok && have_pv) do_pv();
         }
     } else if (warp == 2 || warp == 3) {
-        // warp 2 stages the diagonal blocks; warp 3 has no role
-        // ---------------- diagonal-block producer
-        if (warp == 2 && DS > 0) {
-            // CSR: lane l owns rows 4l .. 4l+3: list start, residual count and
-            // the key of the next slot (fetched one slot ahead)
-            int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
-            int32_t cj[4] = {0, 0, 0, 0};
-            if (a.kind == 1) {
+        // ---------------- warp 2: count and stage each tile's diagonal blocks
+        // (warp 3 has no role)
+        if (warp == 2) {
+            uint32_t dc = 0;  // diagonal blocks staged so far (all tiles)
+            int64_t lt = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++lt) {
+                const TileGeom g = tile_geom(t, ntq, T, W);
+                const int64_t last = (g.q0 + BM - 1 < T - 1) ? g.q0 + BM - 1 : T - 1;
+                // CSR: lane l owns rows 4l .. 4l+3 (list start, residual count,
+                // key of the next slot, fetched one slot ahead)
+                int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
+                int32_t cj[4] = {0, 0, 0, 0};
+                int nd = 0;
+                if (DS > 0) {
+                    if (a.kind == 0) {
+                        for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last) ? 1 : 0;
+                    } else {
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int64_t i = q0 + 4 * lane + h;
-                    if (i < T) {
-                        cstart[h] = a.rowptr[i];
-                        cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
-                        if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
-                    }
-                }
-            }
-            for (int d = 0; d < n_diag; ++d) {
-                const int st = d % DSX, use = d / DSX;
-                const uint32_t kdst = sbase + L::kDiagK + st * L::kTile;
-                const uint32_t vdst = sbase + L::kDiagV + st * L::kTile;
-                if (use > 0 && !tc::mbar_wait(bar(L::bDiagEmpty + st), (use - 1) & 1, abort,
-                                              a.err, SA_DEVERR_TIMEOUT))
-                    break;
-                if (lane == 0) tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kTile);
-                if (a.kind == 0) {
-                    if (lane == 0) {
-                        // distance links: keys q0-o .. q0+127-o, one box each for K and V
-                        const int32_t krow = (int32_t)(q0 - a.offs[a.n_off - n_diag + d]);
-                        for (int x = 0; x < D / 64; ++x) {
-                            tc::tma_load_3d(kdst + x * (BM * 128), &tk, x * 64, krow, (int32_t)bh,
-                                            bar(L::bDiagFull + st));
-                            tc::tma_load_3d(vdst + x * (BM * 128), &tv, x * 64, krow, (int32_t)bh,
-                                            bar(L::bDiagFull + st));
+                        for (int h = 0; h < 4; ++h) {
+                            const int64_t i = g.q0 + 4 * lane + h;
+                            if (i < T) {
+                                cstart[h] = a.rowptr[i];
+                                cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
+                                if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
+                                nd = nd > (int)cres[h] ? nd : (int)cres[h];
+                            }
+                        }
+                        for (int o = 16; o > 0; o >>= 1) {
+                            const int x = __shfl_xor_sync(0xffffffffu, nd, o);
+                            nd = nd > x ? nd : x;
                         }
                     }
-                } else {
-                    // CSR slot d: 4-row TMA gathers of K and V rows (unswizzled);
-                    // a row without slot d loads its own key (masked later)
-                    int32_t rr[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int64_t i = q0 + 4 * lane + h;
-                        const int64_t j = d < cres[h] ? (int64_t)cj[h] : (i < T ? i : 0);
-                        rr[h] = (int32_t)(bh * T + j);
+                }
+                const int slot = (int)(lt & 1);
+                if (lt >= 2 && !wait(L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1))) break;
+                if (lane == 0) {
+                    info[slot] = nd;
+                    tc::mbar_arrive(bar(L::bInfoFull + slot));
+                }
+                for (int d = 0; d < nd; ++d) {
+                    const int st = (int)(dc % DSX);
+                    const uint32_t use = dc / DSX;
+                    const uint32_t kdst = sbase + L::kDiagK + st * L::kTile;
+                    const uint32_t vdst = sbase + L::kDiagV + st * L::kTile;
+                    if (use > 0 && !wait(L::bDiagEmpty + st, (use - 1) & 1)) {
+                        ok = false;
+                        break;
                     }
+                    if (lane == 0) tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kTile);
+                    if (a.kind == 0) {
+                        if (lane == 0) {
+                            // distance links: keys q0-o .. q0+127-o, one box each
+                            const int32_t krow = (int32_t)(g.q0 - a.offs[a.n_off - nd + d]);
+                            for (int x = 0; x < D / 64; ++x) {
+                                tc::tma_load_3d(kdst + x * (BM * 128), &tk, x * 64, krow,
+                                                (int32_t)g.bh, bar(L::bDiagFull + st));
+                                tc::tma_load_3d(vdst + x * (BM * 128), &tv, x * 64, krow,
+                                                (int32_t)g.bh, bar(L::bDiagFull + st));
+                            }
+                        }
+                    } else {
+                        // CSR slot d: 4-row TMA gathers of K and V rows
+                        // (unswizzled); a row without slot d loads its own key
+                        int32_t rr[4];
 #pragma unroll
-                    for (int x = 0; x < D / 64; ++x) {
-                        const uint32_t off = x * (BM * 128) + 4 * lane * 128;
-                        tc::tma_gather4(kdst + off, &tkr, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                        bar(L::bDiagFull + st));
-                        tc::tma_gather4(vdst + off, &tvr, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                        bar(L::bDiagFull + st));
+                        for (int h = 0; h < 4; ++h) {
+                            const int64_t i = g.q0 + 4 * lane + h;
+                            const int64_t j = d < cres[h] ? (int64_t)cj[h] : (i < T ? i : 0);
+                            rr[h] = (int32_t)(g.bh * T + j);
+                        }
+#pragma unroll
+                        for (int x = 0; x < D / 64; ++x) {
+                            const uint32_t off = x * (BM * 128) + 4 * lane * 128;
+                            tc::tma_gather4(kdst + off, &tkr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                            bar(L::bDiagFull + st));
+                            tc::tma_gather4(vdst + off, &tvr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                            bar(L::bDiagFull + st));
+                        }
+#pragma unroll
+                        for (int h = 0; h < 4; ++h)
+                            if (d + 1 < cres[h]) cj[h] = a.colidx[cstart[h] + d + 1];
                     }
-#pragma unroll
-                    for (int h = 0; h < 4; ++h)
-                        if (d + 1 < cres[h]) cj[h] = a.colidx[cstart[h] + d + 1];
+                    ++dc;
                 }
             }
         }
     } else if (warp >= 4 && warp < 8) {
         // ---------------- softmax warpgroup: thread r = query row r = TMEM lane r
         const int r = tid - 128;
-        const int64_t i = q0 + r;
         const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
         const uint32_t tS = tmem + lane_off + L::tS0, tO = tmem + lane_off + L::tO;
         const float c2 = a.scale2;
-        float m_run = -INFINITY, l_run = 0.f;
+        uint32_t dc = 0, gb = 0;  // diagonal blocks and band blocks consumed (all tiles)
+        uint32_t group_uses = 0;  // phases of the softmax group barrier
         bool ok = true;
+        int64_t lt = 0;
+        for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++lt) {
+            const TileGeom g = tile_geom(t, ntq, T, W);
+            const int32_t q0 = g.q0, bh = g.bh;
+            const int32_t i = q0 + r;
+            const int slot = (int)(lt & 1), qb = (int)(lt & 1);
+            float m_run = -INFINITY, l_run = 0.f;
+            if (!wait(L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1))) break;
+            const int nd = info[slot];
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(L::bInfoEmpty + slot));
 
-        // --- diagonal blocks: q row from the Q tile, one key/value row per block
-        {
-            float acc[D];
+            // --- diagonal blocks: q row from the Q tile, one key/value row per
+            // block; fp32 pairs (f32x2 FMA), running max rescaled lazily (only
+            // when it grows by more than 2^8, as in the band blocks)
+            {
+                uint64_t acc2[D / 2];
 #pragma unroll
-            for (int x = 0; x < D; ++x) acc[x] = 0.f;
-            if (n_diag > 0) {
-                ok = tc::mbar_wait(bar(L::bQFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
-                uint32_t qr[D / 2];
-                if (ok) {
-                    // Structured blocks are swizzled like Q: q in logical order.
-                    // CSR gathers are unswizzled: reading them at the swizzled
-                    // address gives chunk c ^ (r & 7), which pairs with the
-                    // physical (unpermuted-address) chunks of the Q row; the
+                for (int x = 0; x < D / 2; ++x) acc2[x] = 0ull;
+                if (DS > 0 && nd > 0) {
+                    ok = wait(L::bQFull + qb, (uint32_t)((lt >> 1) & 1));
+                    // Structured blocks are swizzled like Q: q in logical
+                    // order.  CSR gathers are unswizzled: reading them at the
+                    // swizzled address gives chunk c ^ (r & 7), which pairs with
+                    // the physical (unpermuted-address) chunks of the Q row; the
                     // accumulator is then in that permuted order (undone below).
-#pragma unroll
-                    for (int c = 0; c < D / 8; ++c) {
-                        const uint32_t qoff = (c >> 3) * (BM * 128) +
-                                              (a.kind == 0 ? tc::sw128_off(r, c & 7)
-                                                           : (uint32_t)r * 128u + ((c & 7) << 4));
-                        const uint4 w4 = *(const uint4 *)(sm + L::kQ + qoff);
-                        qr[4 * c] = w4.x;
-                        qr[4 * c + 1] = w4.y;
-                        qr[4 * c + 2] = w4.z;
-                        qr[4 * c + 3] = w4.w;
-                    }
-                }
-                int64_t resid = 0;
-                if (a.kind == 1 && i < T) {
-                    const int64_t deg = a.rowptr[i + 1] - a.rowptr[i];
-                    resid = deg - ((i + 1 < W) ? i + 1 : W);
-                }
-                for (int d = 0; ok && d < n_diag; ++d) {
-                    const int st = d % DSX;
-                    if (!tc::mbar_wait(bar(L::bDiagFull + st), (d / DSX) & 1, abort, a.err,
-                                       SA_DEVERR_TIMEOUT)) {
-                        ok = false;
-                        break;
-                    }
-                    bool valid;
-                    if (a.kind == 0)
-                        valid = i < T && i >= a.offs[a.n_off - n_diag + d];
-                    else
-                        valid = d < resid;
-                    if (valid) {
-                        const uint8_t *kr = sm + L::kDiagK + st * L::kTile;
-                        const uint8_t *vr = sm + L::kDiagV + st * L::kTile;
-                        float s = 0.f;
+                    uint64_t q2[D / 2];
+                    if (ok) {
 #pragma unroll
                         for (int c = 0; c < D / 8; ++c) {
-                            const uint4 w4 = *(const uint4 *)(kr + (c >> 3) * (BM * 128) +
-                                                              tc::sw128_off(r, c & 7));
-                            const uint32_t kw[4] = {w4.x, w4.y, w4.z, w4.w};
+                            const uint32_t qoff =
+                                (c >> 3) * (BM * 128) +
+                                (a.kind == 0 ? tc::sw128_off(r, c & 7)
+                                             : (uint32_t)r * 128u + ((c & 7) << 4));
+                            const uint4 w4 = *(const uint4 *)(sm + L::kQ + qb * L::kTile + qoff);
+                            q2[4 * c] = tc::bf2_to_f2(w4.x);
+                            q2[4 * c + 1] = tc::bf2_to_f2(w4.y);
+                            q2[4 * c + 2] = tc::bf2_to_f2(w4.z);
+                            q2[4 * c + 3] = tc::bf2_to_f2(w4.w);
+                        }
+                    }
+                    int32_t resid = 0;
+                    if (a.kind == 1 && i < T) {
+                        const int64_t deg = a.rowptr[i + 1] - a.rowptr[i];
+                        resid = (int32_t)(deg - ((i + 1 < W) ? i + 1 : W));
+                    }
+                    for (int d = 0; ok && d < nd; ++d) {
+                        const int st = (int)(dc % DSX);
+                        if (!wait(L::bDiagFull + st, (dc / DSX) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        bool valid;
+                        if (a.kind == 0)
+                            valid = i < T && i >= a.offs[a.n_off - nd + d];
+                        else
+                            valid = d < resid;
+                        if (valid) {
+                            const uint8_t *kr = sm + L::kDiagK + st * L::kTile;
+                            const uint8_t *vr = sm + L::kDiagV + st * L::kTile;
+                            // four independent partial sums (short dependency chains)
+                            uint64_t sp0 = 0ull, sp1 = 0ull, sp2 = 0ull, sp3 = 0ull;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                s = fmaf(tc::bf16lo(qr[4 * c + e]), tc::bf16lo(kw[e]), s);
-                                s = fmaf(tc::bf16hi(qr[4 * c + e]), tc::bf16hi(kw[e]), s);
+                            for (int c = 0; c < D / 8; ++c) {
+                                const uint4 w4 = *(const uint4 *)(kr + (c >> 3) * (BM * 128) +
+                                                                  tc::sw128_off(r, c & 7));
+                                sp0 = tc::ffma2(q2[4 * c], tc::bf2_to_f2(w4.x), sp0);
+                                sp1 = tc::ffma2(q2[4 * c + 1], tc::bf2_to_f2(w4.y), sp1);
+                                sp2 = tc::ffma2(q2[4 * c + 2], tc::bf2_to_f2(w4.z), sp2);
+                                sp3 = tc::ffma2(q2[4 * c + 3], tc::bf2_to_f2(w4.w), sp3);
+                            }
+                            const float s = ((tc::f2lo(sp0) + tc::f2hi(sp0)) +
+                                             (tc::f2lo(sp1) + tc::f2hi(sp1)) +
+                                             ((tc::f2lo(sp2) + tc::f2hi(sp2)) +
+                                              (tc::f2lo(sp3) + tc::f2hi(sp3)))) *
+                                            c2;
+                            if (s > m_run + kRescaleThreshold) {
+                                const float al = tc::ex2(m_run - s);  // 0 on the first edge
+                                const uint64_t al2 = tc::f2pack(al, al);
+#pragma unroll
+                                for (int x = 0; x < D / 2; ++x) acc2[x] = tc::fmul2(acc2[x], al2);
+                                l_run *= al;
+                                m_run = s;
+                            }
+                            const float p = tc::ex2(s - m_run);
+                            l_run += p;
+                            const uint64_t p2 = tc::f2pack(p, p);
+#pragma unroll
+                            for (int c = 0; c < D / 8; ++c) {
+                                const uint4 w4 = *(const uint4 *)(vr + (c >> 3) * (BM * 128) +
+                                                                  tc::sw128_off(r, c & 7));
+                                acc2[4 * c] = tc::ffma2(p2, tc::bf2_to_f2(w4.x), acc2[4 * c]);
+                                acc2[4 * c + 1] =
+                                    tc::ffma2(p2, tc::bf2_to_f2(w4.y), acc2[4 * c + 1]);
+                                acc2[4 * c + 2] =
+                                    tc::ffma2(p2, tc::bf2_to_f2(w4.z), acc2[4 * c + 2]);
+                                acc2[4 * c + 3] =
+                                    tc::ffma2(p2, tc::bf2_to_f2(w4.w), acc2[4 * c + 3]);
                             }
                         }
-                        s *= c2;
-                        const float mn = fmaxf(m_run, s);
-                        const float al = tc::ex2(m_run - mn), p = tc::ex2(s - mn);
-                        l_run = l_run * al + p;
-#pragma unroll
-                        for (int c = 0; c < D / 8; ++c) {
-                            const uint4 w4 = *(const uint4 *)(vr + (c >> 3) * (BM * 128) +
-                                                              tc::sw128_off(r, c & 7));
-                            const uint32_t vw[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                acc[8 * c + 2 * e] =
-                                    fmaf(p, tc::bf16lo(vw[e]), acc[8 * c + 2 * e] * al);
-                                acc[8 * c + 2 * e + 1] =
-                                    fmaf(p, tc::bf16hi(vw[e]), acc[8 * c + 2 * e + 1] * al);
-                            }
+                        const bool hold = (a.kind == 1) && (d == nd - 1);
+                        if (!hold) {
+                            __syncwarp();
+                            if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
                         }
-                        m_run = mn;
+                        ++dc;
                     }
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                    if (a.kind == 1) {
+                        // undo the chunk permutation (per 64-column half) through
+                        // the last diagonal stage, whose release was held back:
+                        // once every row is done with it, thread r uses 256 bytes
+                        // (rows < 64 in its K half, the others in its V half)
+                        const int st = (int)((dc - 1) % DSX);
+                        // every row is done with the stage (bounded wait)
+                        tc::mbar_arrive(bar(L::bGroup));
+                        if (!wait(L::bGroup, group_uses & 1)) ok = false;
+                        ++group_uses;
+                        uint64_t *scr =
+                            (uint64_t *)(sm + (r < 64 ? L::kDiagK : L::kDiagV) + st * L::kTile) +
+                            (size_t)(r & 63) * 32 * (D / 64);
+#pragma unroll
+                        for (int hh = 0; hh < D / 64; ++hh) {
+#pragma unroll
+                            for (int tt = 0; tt < 8; ++tt) {
+                                const int lc = tt ^ (r & 7);
+                                const uint64_t *src = acc2 + 32 * hh + 4 * tt;
+                                *(ulonglong2 *)(scr + 4 * lc) = make_ulonglong2(src[0], src[1]);
+                                *(ulonglong2 *)(scr + 4 * lc + 2) = make_ulonglong2(src[2], src[3]);
+                            }
+#pragma unroll
+                            for (int tt = 0; tt < 16; ++tt) {
+                                const ulonglong2 f = *(const ulonglong2 *)(scr + 2 * tt);
+                                acc2[32 * hh + 2 * tt] = f.x;
+                                acc2[32 * hh + 2 * tt + 1] = f.y;
+                            }
+                            scr += 32;
+                        }
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                    }
                 }
-                if (a.kind == 1) {
-                    // undo the chunk permutation through the (now idle) first
-                    // diagonal stage: row r of D fp32 at r * 4D bytes
-                    tc::named_barrier(1, 128);
-                    float *scr = (float *)(sm + L::kDiagK) + (size_t)r * D;
-#pragma unroll
-                    for (int t = 0; t < D / 8; ++t) {
-                        const int lc = (t & ~7) | ((t & 7) ^ (r & 7));
-                        *(float4 *)(scr + 8 * lc) =
-                            make_float4(acc[8 * t], acc[8 * t + 1], acc[8 * t + 2], acc[8 * t + 3]);
-                        *(float4 *)(scr + 8 * lc + 4) = make_float4(
-                            acc[8 * t + 4], acc[8 * t + 5], acc[8 * t + 6], acc[8 * t + 7]);
-                    }
-                    __syncwarp();
-#pragma unroll
-                    for (int t = 0; t < D / 4; ++t) {
-                        const float4 f = *(const float4 *)(scr + 4 * t);
-                        acc[4 * t] = f.x;
-                        acc[4 * t + 1] = f.y;
-                        acc[4 * t + 2] = f.z;
-                        acc[4 * t + 3] = f.w;
-                    }
-                }
-            }
-            // initialise O (columns tO .. tO+D) with the diagonal part
-#pragma unroll
-            for (int c = 0; c < D; c += 32) {
-                uint32_t w[32];
-#pragma unroll
-                for (int x = 0; x < 32; ++x) w[x] = __float_as_uint(acc[c + x]);
-                tc::tmem_st32(tO + c, w);
-            }
-            tc::tmem_st_wait();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(L::bOInit));
-        }
-
-        // --- band blocks
-        for (int bl = 0; ok && bl < n_band; ++bl) {
-            const int sb = bl & 1, pb = bl % PB;
-            const int64_t b = b_first + bl;
-            if (!tc::mbar_wait(bar(L::bSFull + sb), (bl >> 1) & 1, abort, a.err,
-                               SA_DEVERR_TIMEOUT)) {
-                ok = false;
-                break;
-            }
-            tc::tc_fence_after();
-            float s[BN];
-#pragma unroll
-            for (int c = 0; c < BN; c += 32) tc::tmem_ld32(tS + sb * BN + c, (uint32_t *)(s + c));
-            tc::tmem_ld_wait();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(L::bSFree + sb));
-
-            // mask: r <= u <= r+W-1 and key >= 0, with u = 128 b + c, i.e. the
-            // column range [c_lo, c_hi] of this block.  Scores stay raw (the
-            // scale is folded into the exponent's FFMA); a masked raw score is
-            // set to the extreme that the max/min below ignores.
-            const int64_t u0 = b * BN;
-            const bool need_mask = (u0 < BM - 1) || (u0 + BN - 1 > (int64_t)W - 1) ||
-                                   (u0 + q0 < (int64_t)W - 1);
-            const bool pos = c2 >= 0.f;
-            const float ext = pos ? -INFINITY : INFINITY;
-            if (need_mask) {
-                const int64_t lo = ((int64_t)r > (int64_t)W - 1 - q0) ? r : (int64_t)W - 1 - q0;
-                const int64_t hi = (int64_t)r + W - 1;
-                const int c_lo = (int)(lo - u0 < 0 ? 0 : (lo - u0 > BN ? BN : lo - u0));
-                const int c_hi = (int)(hi - u0 > BN - 1 ? BN - 1 : (hi - u0 < -1 ? -1 : hi - u0));
-#pragma unroll
-                for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : ext;
-            }
-            float mr[8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) mr[x] = ext;
-            if (pos) {
-#pragma unroll
-                for (int c = 0; c < BN; ++c) mr[c & 7] = fmaxf(mr[c & 7], s[c]);
-#pragma unroll
-                for (int x = 4; x > 0; x >>= 1)
-                    for (int y = 0; y < x; ++y) mr[y] = fmaxf(mr[y], mr[y + x]);
-            } else {
-#pragma unroll
-                for (int c = 0; c < BN; ++c) mr[c & 7] = fminf(mr[c & 7], s[c]);
-#pragma unroll
-                for (int x = 4; x > 0; x >>= 1)
-                    for (int y = 0; y < x; ++y) mr[y] = fminf(mr[y], mr[y + x]);
-            }
-            const float mblk = (mr[0] == ext) ? -INFINITY : mr[0] * c2;
-            // conditional rescale of O (and l) when the max grows by more than 2^8
-            const bool grow = mblk > m_run + kRescaleThreshold;
-            if (__any_sync(0xffffffffu, grow)) {
-                const float m_new = grow ? mblk : m_run;
-                const float alpha = grow ? tc::ex2(m_run - m_new) : 1.f;
-                if (bl > 0) {
-                    const int pp = (bl - 1) % PB;
-                    if (!tc::mbar_wait(bar(L::bPVDone + pp), ((bl - 1) / PB) & 1, abort, a.err,
-                                       SA_DEVERR_TIMEOUT)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::tc_fence_after();
-                }
+                if (!ok) break;
+                // this warp is done reading Q of the tile
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(L::bQEmpty + qb));
+                // initialise O (columns tO .. tO+D) with the diagonal part
 #pragma unroll
                 for (int c = 0; c < D; c += 32) {
                     uint32_t w[32];
-                    tc::tmem_ld32(tO + c, w);
-                    tc::tmem_ld_wait();
 #pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        w[x] = __float_as_uint(__uint_as_float(w[x]) * alpha);
+                    for (int x = 0; x < 16; ++x) {
+                        w[2 * x] = __float_as_uint(tc::f2lo(acc2[c / 2 + x]));
+                        w[2 * x + 1] = __float_as_uint(tc::f2hi(acc2[c / 2 + x]));
+                    }
                     tc::tmem_st32(tO + c, w);
                 }
-                l_run *= alpha;
-                m_run = m_new;
+                tc::tmem_st_wait();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(L::bOInit));
             }
-            // p = 2^(s - m), row sum, bf16 P into the swizzled K-major tile
-            if (bl >= PB) {
-                if (!tc::mbar_wait(bar(L::bPVDone + pb), ((bl - PB) / PB) & 1, abort, a.err,
-                                   SA_DEVERR_TIMEOUT)) {
+
+            // --- band blocks
+            uint32_t gb_last = gb;
+            for (int bl = 0; ok && bl < g.n_band; ++bl, ++gb) {
+                const int sb = (int)(gb & 1);
+                const int32_t b = g.b_first + bl;
+                gb_last = gb;
+                if (!wait(L::bSFull + sb, (gb >> 1) & 1)) {
                     ok = false;
                     break;
                 }
-            }
-            uint8_t *prow = sm + L::kP + pb * L::kPTile;
-            const float m_use = (m_run == -INFINITY) ? 0.f : m_run;  // all-masked row: p = 0
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
-            if (need_mask) {
+                tc::tc_fence_after();
+                float s[BN];
 #pragma unroll
-                for (int c8 = 0; c8 < BN / 8; ++c8) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x0 = s[8 * c8 + 2 * e], x1 = s[8 * c8 + 2 * e + 1];
-                        const float p0 = (x0 != ext) ? tc::ex2(fmaf(x0, c2, -m_use)) : 0.f;
-                        const float p1 = (x1 != ext) ? tc::ex2(fmaf(x1, c2, -m_use)) : 0.f;
-                        ls[e] += p0 + p1;
-                        w[e] = tc::pack_bf16x2(p0, p1);
-                    }
-                    *(uint4 *)(prow + (c8 >> 3) * (BM * 128) + tc::sw128_off(r, c8 & 7)) =
-                        make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            } else {
-#pragma unroll
-                for (int c8 = 0; c8 < BN / 8; ++c8) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float p0 = tc::ex2(fmaf(s[8 * c8 + 2 * e], c2, -m_use));
-                        const float p1 = tc::ex2(fmaf(s[8 * c8 + 2 * e + 1], c2, -m_use));
-                        ls[e] += p0 + p1;
-                        w[e] = tc::pack_bf16x2(p0, p1);
-                    }
-                    *(uint4 *)(prow + (c8 >> 3) * (BM * 128) + tc::sw128_off(r, c8 & 7)) =
-                        make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
-            const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            l_run += lsum;
-            tc::fence_proxy_async_smem();
-            tc::tmem_st_wait();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(L::bPFull + pb));
-        }
+                for (int c = 0; c < BN; c += 32)
+                    tc::tmem_ld32(tS + sb * BN + c, (uint32_t *)(s + c));
+                tc::tmem_ld_wait();
 
-        // --- epilogue
-        if (ok && n_band > 0) {
-            const int lb = n_band - 1;
-            ok = tc::mbar_wait(bar(L::bPVDone + lb % PB), (lb / PB) & 1, abort, a.err,
-                               SA_DEVERR_TIMEOUT);
-        }
-        if (ok) {
+                // mask: r <= u <= r+W-1 and key >= 0, with u = 128 b + c, i.e.
+                // the column range [c_lo, c_hi] of this block.  Scores stay raw
+                // (the scale is folded into the exponent's FFMA); a masked raw
+                // score is set to the extreme that the max/min below ignores.
+                const int32_t u0 = b * BN;
+                const bool need_mask =
+                    (u0 < BM - 1) || (u0 + BN - 1 > W - 1) || (u0 + q0 < W - 1);
+                const bool pos = c2 >= 0.f;
+                const float ext = pos ? -INFINITY : INFINITY;
+                if (need_mask) {
+                    const int32_t lo = (r > W - 1 - q0) ? r : W - 1 - q0;
+                    const int32_t hi = r + W - 1;
+                    const int c_lo = lo - u0 < 0 ? 0 : (lo - u0 > BN ? BN : lo - u0);
+                    const int c_hi = hi - u0 > BN - 1 ? BN - 1 : (hi - u0 < -1 ? -1 : hi - u0);
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : ext;
+                }
+                float mr[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) mr[x] = ext;
+                if (pos) {
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) mr[c & 7] = fmaxf(mr[c & 7], s[c]);
+#pragma unroll
+                    for (int x = 4; x > 0; x >>= 1)
+                        for (int y = 0; y < x; ++y) mr[y] = fmaxf(mr[y], mr[y + x]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) mr[c & 7] = fminf(mr[c & 7], s[c]);
+#pragma unroll
+                    for (int x = 4; x > 0; x >>= 1)
+                        for (int y = 0; y < x; ++y) mr[y] = fminf(mr[y], mr[y + x]);
+                }
+                const float mblk = (mr[0] == ext) ? -INFINITY : mr[0] * c2;
+                // conditional rescale of O (and l) when the max grows by more than 2^8
+                const bool grow = mblk > m_run + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, grow)) {
+                    const float m_new = grow ? mblk : m_run;
+                    const float alpha = grow ? tc::ex2(m_run - m_new) : 1.f;
+                    if (bl > 0) {  // O must hold P V of the previous block of this tile
+                        const uint32_t pg = gb - 1;
+                        if (!wait(L::bPVDone + (int)(pg & 1), (pg >> 1) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::tc_fence_after();
+                    }
+#pragma unroll
+                    for (int c = 0; c < D; c += 32) {
+                        uint32_t w[32];
+                        tc::tmem_ld32(tO + c, w);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x)
+                            w[x] = __float_as_uint(__uint_as_float(w[x]) * alpha);
+                        tc::tmem_st32(tO + c, w);
+                    }
+                    l_run *= alpha;
+                    m_run = m_new;
+                }
+                // p = 2^(s - m), row sum, bf16 P over the first 64 columns of
+                // this S buffer (its scores are already in registers)
+                const float m_use = (m_run == -INFINITY) ? 0.f : m_run;  // all-masked row: p = 0
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t pw[BN / 2];
+                if (need_mask) {
+                    // only 16-column chunks that hold a kept score of some row of
+                    // this warp do exponentials; the rest of P is zero
+#pragma unroll
+                    for (int c16 = 0; c16 < BN / 16; ++c16) {
+                        bool live = false;
+#pragma unroll
+                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) live |= (s[c] != ext);
+                        if (__any_sync(0xffffffffu, live)) {
+#pragma unroll
+                            for (int c = 8 * c16; c < 8 * c16 + 8; ++c) {
+                                const float x0 = s[2 * c], x1 = s[2 * c + 1];
+                                const float p0 = (x0 != ext) ? tc::ex2(fmaf(x0, c2, -m_use)) : 0.f;
+                                const float p1 = (x1 != ext) ? tc::ex2(fmaf(x1, c2, -m_use)) : 0.f;
+                                ls[c & 3] += p0 + p1;
+                                pw[c] = tc::pack_bf16x2(p0, p1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 8 * c16; c < 8 * c16 + 8; ++c) pw[c] = 0u;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BN / 2; ++c) {
+                        const float p0 = tc::ex2(fmaf(s[2 * c], c2, -m_use));
+                        const float p1 = tc::ex2(fmaf(s[2 * c + 1], c2, -m_use));
+                        ls[c & 3] += p0 + p1;
+                        pw[c] = tc::pack_bf16x2(p0, p1);
+                    }
+                }
+                l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+#pragma unroll
+                for (int c = 0; c < BN / 2; c += 32) tc::tmem_st32(tS + sb * BN + c, pw + c);
+                tc::tmem_st_wait();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(L::bPFull + sb));
+            }
+            if (!ok) break;
+
+            // --- epilogue: O / l and lse once the tile's last P V is done
+            if (!wait(L::bPVDone + (int)(gb_last & 1), (gb_last >> 1) & 1)) break;
             tc::tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
             __nv_bfloat16 *orow = a.out + ((size_t)bh * (size_t)T + (size_t)i) * D;
@@ -636,11 +710,11 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     }
 }
 
-template <int D, int KS, int VS, int DS, int PB>
+template <int D, int KS, int VS, int DS>
 sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_graph_s *g, float scale, sa_tensor *out, float *lse,
                           cudaStream_t s) {
-    using L = Layout<D, KS, VS, DS, PB>;
+    using L = Layout<D, KS, VS, DS>;
     static_assert(L::kAlloc <= 232448, "shared memory budget");
     const int64_t BH = q->B * q->H, T = q->T;
     CUtensorMap mq, mk, mv, mkr, mvr;
@@ -654,6 +728,7 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     }
     FwdArgs a{};
     a.T = T;
+    a.BH = BH;
     a.W = g->W;
     a.kind = g->kind;
     a.n_off = g->kind == 0 ? g->n_off : 0;
@@ -667,9 +742,13 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.scale2 = scale * kLog2e;
     a.err = sa_device_error_word();
     if (!a.err) return SA_ERR_CUDA;
-    auto kern = band_fwd_kernel<D, KS, VS, DS, PB>;
+    auto kern = band_fwd_kernel<D, KS, VS, DS>;
     SA_CUDA_TRY(sa_smem_optin((const void *)kern, L::kAlloc));
-    dim3 grid((unsigned)((T + BM - 1) / BM), (unsigned)BH);
+    // persistent: one CTA per SM (shared memory and TMEM allow no more)
+    const int64_t ntiles = ((T + BM - 1) / BM) * BH;
+    int sms = 0;
+    SA_CUDA_TRY(sa_sm_count(&sms));
+    const unsigned grid = (unsigned)(ntiles < sms ? ntiles : sms);
     SA_LAUNCH("band_fwd", s, kern<<<grid, 256, L::kAlloc, s>>>(mq, mk, mv, mkr, mvr, a));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
@@ -689,12 +768,12 @@ sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
                       const sa_graph_s *g, const GraphView &, float scale, sa_tensor *out,
                       float *lse, cudaStream_t s) {
     const bool diag = (g->kind == 0) ? g->n_off > 0 : g->max_resid > 0;
-    // <D, K stages, V stages, diagonal stages, P buffers>, sized to the
-    // 227 KB of shared memory
+    // <D, K stages, V stages, diagonal stages>, sized to the 227 KB of shared
+    // memory (two Q buffers; P lives in TMEM)
     if (q->D == 64) {
-        return diag ? launch_band_fwd<64, 2, 3, 2, 2>(q, k, v, g, scale, out, lse, s)
-                    : launch_band_fwd<64, 2, 3, 0, 2>(q, k, v, g, scale, out, lse, s);
+        return diag ? launch_band_fwd<64, 2, 2, 4>(q, k, v, g, scale, out, lse, s)
+                    : launch_band_fwd<64, 2, 4, 0>(q, k, v, g, scale, out, lse, s);
     }
-    return diag ? launch_band_fwd<128, 1, 1, 1, 1>(q, k, v, g, scale, out, lse, s)
-                : launch_band_fwd<128, 2, 3, 0, 1>(q, k, v, g, scale, out, lse, s);
+    return diag ? launch_band_fwd<128, 1, 1, 1>(q, k, v, g, scale, out, lse, s)
+                : launch_band_fwd<128, 2, 3, 0>(q, k, v, g, scale, out, lse, s);
 }

@@ -125,18 +125,18 @@ __device__ __forceinline__ void unpermute_row(float *acc, float *scr_row, int r)
 template <int D>
 __device__ __forceinline__ float dot_reg_smem(const uint32_t *a, const uint8_t *tile, int rows,
                                               int r) {
-    float s0 = 0.f, s1 = 0.f;
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
         const uint4 x = *(const uint4 *)(tile + tile_off(rows, r, c));
         const uint32_t b[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            s0 = fmaf(tc::bf16lo(a[4 * c + e]), tc::bf16lo(b[e]), s0);
-            s1 = fmaf(tc::bf16hi(a[4 * c + e]), tc::bf16hi(b[e]), s1);
+            sa[e] = fmaf(tc::bf16lo(a[4 * c + e]), tc::bf16lo(b[e]), sa[e]);
+            sb[e] = fmaf(tc::bf16hi(a[4 * c + e]), tc::bf16hi(b[e]), sb[e]);
         }
     }
-    return s0 + s1;
+    return ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
 }
 
 // a . b, a = row r of a swizzled tile read in physical chunk order, b = row r
@@ -145,7 +145,7 @@ __device__ __forceinline__ float dot_reg_smem(const uint32_t *a, const uint8_t *
 template <int D>
 __device__ __forceinline__ float dot_phys_gathered(const uint8_t *ta, const uint8_t *tb, int rows,
                                                    int r) {
-    float s0 = 0.f, s1 = 0.f;
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
         const uint4 x = *(const uint4 *)(ta + (c >> 3) * (rows * 128) + r * 128 + ((c & 7) << 4));
@@ -153,18 +153,18 @@ __device__ __forceinline__ float dot_phys_gathered(const uint8_t *ta, const uint
         const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            s0 = fmaf(tc::bf16lo(xa[e]), tc::bf16lo(yb[e]), s0);
-            s1 = fmaf(tc::bf16hi(xa[e]), tc::bf16hi(yb[e]), s1);
+            sa[e] = fmaf(tc::bf16lo(xa[e]), tc::bf16lo(yb[e]), sa[e]);
+            sb[e] = fmaf(tc::bf16hi(xa[e]), tc::bf16hi(yb[e]), sb[e]);
         }
     }
-    return s0 + s1;
+    return ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
 }
 
 // a . b with both rows in shared memory (row r of each tile).
 template <int D>
 __device__ __forceinline__ float dot_smem_smem(const uint8_t *ta, const uint8_t *tb, int rows,
                                                int r) {
-    float s0 = 0.f, s1 = 0.f;
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
         const uint4 x = *(const uint4 *)(ta + tile_off(rows, r, c));
@@ -172,11 +172,11 @@ __device__ __forceinline__ float dot_smem_smem(const uint8_t *ta, const uint8_t 
         const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            s0 = fmaf(tc::bf16lo(xa[e]), tc::bf16lo(yb[e]), s0);
-            s1 = fmaf(tc::bf16hi(xa[e]), tc::bf16hi(yb[e]), s1);
+            sa[e] = fmaf(tc::bf16lo(xa[e]), tc::bf16lo(yb[e]), sa[e]);
+            sb[e] = fmaf(tc::bf16hi(xa[e]), tc::bf16hi(yb[e]), sb[e]);
         }
     }
-    return s0 + s1;
+    return ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
 }
 
 // acc += a * (row r of a tile)
@@ -265,7 +265,8 @@ struct LayoutDQ {
     static constexpr int bSFull = bBandEmpty + BS, bSFree = bSFull + 2;
     static constexpr int bDSFull = bSFree + 2, bDSDone = bDSFull + PB;
     static constexpr int bInit = bDSDone + PB, bDiagFull = bInit + 1;
-    static constexpr int bDiagEmpty = bDiagFull + DSX, nBars = bDiagEmpty + DSX;
+    static constexpr int bDiagEmpty = bDiagFull + DSX, bGroup = bDiagEmpty + DSX;
+    static constexpr int nBars = bGroup + 1;
     static constexpr int kMisc = kBars + nBars * 8;
     static constexpr int kAlloc = kMisc + 16 + 1024;
     static constexpr uint32_t tS = 0, tDP = 128, tDQ = 256, kTmemCols = 512;
@@ -313,6 +314,7 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             tc::mbar_init(bar(L::bDSDone + s), 1);
         }
         tc::mbar_init(bar(L::bInit), 4);
+        tc::mbar_init(bar(L::bGroup), 128);  // 128-thread compute barrier (bounded)
         for (int s = 0; s < DSX; ++s) {
             tc::mbar_init(bar(L::bDiagFull + s), 1);
             tc::mbar_init(bar(L::bDiagEmpty + s), 4);
@@ -527,7 +529,8 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
                     }
-                    tc::named_barrier(1, 128);
+                    tc::mbar_arrive(bar(L::bGroup));
+                    if (!tc::mbar_wait(bar(L::bGroup), 0, abort, a.err, SA_DEVERR_TIMEOUT)) ok = false;
                     unpermute_row<D>(acc, (float *)(sm + L::kDiagK) + (size_t)r * D, r);
                 }
             }
@@ -561,11 +564,20 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                 const int64_t hi = (int64_t)r + W - 1;
                 const int c_lo = (int)(lo - u0 < 0 ? 0 : (lo - u0 > BB ? BB : lo - u0));
                 const int c_hi = (int)(hi - u0 > BB - 1 ? BB - 1 : (hi - u0 < -1 ? -1 : hi - u0));
+                // 16-column chunks outside every kept range of this warp: dS = 0
 #pragma unroll
-                for (int c = 0; c < BB; ++c) {
-                    const float p =
-                        (c >= c_lo && c <= c_hi) ? tc::ex2(fmaf(s[c], c2, -lse2)) : 0.f;
-                    s[c] = p * (dp[c] - Delta);  // dS
+                for (int c16 = 0; c16 < BB / 16; ++c16) {
+                    if (__any_sync(0xffffffffu, c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16)) {
+#pragma unroll
+                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
+                            const float p =
+                                (c >= c_lo && c <= c_hi) ? tc::ex2(fmaf(s[c], c2, -lse2)) : 0.f;
+                            s[c] = p * (dp[c] - Delta);  // dS
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) s[c] = 0.f;
+                    }
                 }
             } else {
 #pragma unroll
@@ -610,7 +622,8 @@ struct LayoutDKV {
     static constexpr int bSFull = bBandEmpty + BS, bSFree = bSFull + 2;
     static constexpr int bPFull = bSFree + 2, bPDone = bPFull + PB;
     static constexpr int bInit = bPDone + PB, bDiagFull = bInit + 1;
-    static constexpr int bDiagEmpty = bDiagFull + DSX, nBars = bDiagEmpty + DSX;
+    static constexpr int bDiagEmpty = bDiagFull + DSX, bGroup = bDiagEmpty + DSX;
+    static constexpr int nBars = bGroup + 1;
     static constexpr int kMisc = kBars + nBars * 8;
     static constexpr int kAlloc = kMisc + 16 + 1024;
     static constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D, kTmemCols = 512;
@@ -657,6 +670,7 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
             tc::mbar_init(bar(L::bPDone + s), 1);
         }
         tc::mbar_init(bar(L::bInit), 4);
+        tc::mbar_init(bar(L::bGroup), 128);  // 128-thread compute barrier (bounded)
         for (int s = 0; s < DSX; ++s) {
             tc::mbar_init(bar(L::bDiagFull + s), 1);
             tc::mbar_init(bar(L::bDiagEmpty + s), 4);
@@ -888,7 +902,8 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
                     }
-                    tc::named_barrier(1, 128);
+                    tc::mbar_arrive(bar(L::bGroup));
+                    if (!tc::mbar_wait(bar(L::bGroup), 0, abort, a.err, SA_DEVERR_TIMEOUT)) ok = false;
                     float *scr = (float *)(sm + L::kDiagQ);
                     unpermute_row<D>(adv, scr + (size_t)r * D, r);
                     unpermute_row<D>(adk, scr + (size_t)(BM + r) * D, r);
@@ -928,12 +943,22 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
                 const int64_t lo = r;
                 const int c_lo = (int)(lo - v0 < 0 ? 0 : (lo - v0 > BB ? BB : lo - v0));
                 const int c_hi = (int)(hi - v0 > BB - 1 ? BB - 1 : (hi - v0 < -1 ? -1 : hi - v0));
+                // 16-column chunks outside every kept range of this warp: P = dS = 0
 #pragma unroll
-                for (int c = 0; c < BB; ++c) {
-                    const float p =
-                        (c >= c_lo && c <= c_hi) ? tc::ex2(fmaf(s[c], c2, -lse_s[c])) : 0.f;
-                    s[c] = p;
-                    dp[c] = p * (dp[c] - del_s[c]);
+                for (int c16 = 0; c16 < BB / 16; ++c16) {
+                    if (__any_sync(0xffffffffu, c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16)) {
+#pragma unroll
+                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
+                            const float p = (c >= c_lo && c <= c_hi)
+                                                ? tc::ex2(fmaf(s[c], c2, -lse_s[c]))
+                                                : 0.f;
+                            s[c] = p;
+                            dp[c] = p * (dp[c] - del_s[c]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) s[c] = dp[c] = 0.f;
+                    }
                 }
             } else {
 #pragma unroll

@@ -64,6 +64,22 @@ void sa_record_cuda_error(cudaError_t e, const char *where) {
                    " (" + cudaGetErrorString(e) + ")";
 }
 
+cudaError_t sa_sm_count(int *n) {
+    static std::mutex mu;
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) {
+        *n = cached[dev];
+        return cudaSuccess;
+    }
+    e = cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) cached[dev] = *n;
+    return e;
+}
+
 cudaError_t sa_smem_optin(const void *kernel, int bytes) {
     static std::mutex mu;
     static std::vector<std::pair<const void *, int>> done;

@@ -100,6 +100,9 @@ __host__ __device__ inline int64_t sg_in_degree(int64_t j, int64_t T, int64_t W,
     return d;
 }
 
+// Number of SMs of the current device (cached per device).
+cudaError_t sa_sm_count(int *n);
+
 // Opt a kernel into `bytes` of dynamic shared memory, once per (kernel, device).
 cudaError_t sa_smem_optin(const void *kernel, int bytes);
 

@@ -1,30 +1,34 @@
 // attn_band.cu -- forward on tcgen05 band tiles fused with the gathered edges.
 //
-// A tile is 128 consecutive queries [q0, q0+128) of one (b, h) slice; the
-// kernel is persistent (one CTA per SM walking its share of the tiles).
+// A tile is 128 consecutive queries [q0, q0+128) of one (b, h) slice.
 //  * Window edges (the band of "MiniGPT (Part 6)", section "A mask is not
-//    enough": keys j <= i with i - j < W) run as dense 128 x 128 tiles on the
-//    tensor cores: keys [q0-W+1, q0+127] are cut into blocks of 128 starting
-//    at q0-W+1, so in block coordinates u = 128 b + c a query row r keeps
-//    exactly r <= u <= r+W-1 (and j >= 0).  S = Q K^T lands in TMEM, the
-//    softmax warpgroup turns it into P (bf16, shared memory), and O += P V
-//    accumulates in TMEM.
+//    enough": keys j <= i with i - j < W) run as dense 128 x 64 blocks on the
+//    tensor cores: keys [q0-W+1, q0+127] are cut into blocks of 64 starting at
+//    q0-W+1, so in block coordinates u = 64 b + c a query row r keeps exactly
+//    r <= u <= r+W-1 (and j >= 0).  S = Q K^T lands in TMEM, the softmax
+//    warpgroup turns it into P (bf16, written back over S in TMEM), and
+//    O += P V accumulates in TMEM with P read from TMEM by the MMA.
 //  * Every other edge -- the 2^k distance links of "SpatialLM-Mini ...",
 //    section "How tokens choose whom to listen to", or the non-window part of
 //    a CSR list ("Longer Attention Span ...", Abstract) -- is a "diagonal"
 //    block: 128 key rows, row r belonging to query r.  For a distance o the
 //    rows are the contiguous keys q0-o .. q0+127-o (one TMA box); for CSR
-//    lists slot s of every row is gathered with 16-byte cp.async into the
-//    same swizzled layout.  Thread r takes the dot product of its own row.
+//    lists slot s of every row is fetched with 4-row TMA gathers.  Thread r
+//    takes the dot product of its own row on the CUDA cores.
 //  * One online softmax (running max m and sum l per row, base 2) covers both
 //    classes: the diagonal blocks go first, their weighted sum initialises O
 //    in TMEM, then the band blocks rescale O only when a row's max grows by
 //    more than 2^8 (the stale max keeps every p <= 256, exact in fp32).
 //  * Epilogue: out = O / l (bf16, round to nearest even), lse = (m + log2 l) ln 2.
 //
-// Warp roles (256 threads): 0 TMA producer for Q and the band K/V ring,
-// 1 TMEM allocator + MMA issuer, 2-3 producers of the diagonal blocks,
-// 4-7 softmax warpgroup (thread = query row = TMEM lane).
+// The kernel is persistent and runs NP (1 or 2) independent tile pipelines
+// per CTA, each with its own shared-memory rings, TMEM columns (two S
+// buffers and O) and barriers, so that the softmax of one tile overlaps the
+// loads, MMAs and softmax of the other.  Warp roles: warp 2p is the TMA
+// producer of pipeline p (Q, band K/V ring, diagonal blocks), warp 2p+1 its
+// MMA issuer (warp 1 also allocates TMEM), warps 4+4p .. 7+4p its softmax
+// warpgroup (thread = query row = TMEM lane).  With two pipelines the
+// producer warpgroup hands registers to the softmax warpgroups (setmaxnreg).
 // Every mbarrier wait is bounded (2 s); on expiry the CTA records
 // SA_DEVERR_TIMEOUT in the device error word, all roles leave their loops,
 // TMEM is freed and the kernel returns.
@@ -38,11 +42,20 @@
 
 namespace {
 
-constexpr int BM = 128;             // queries per CTA
-constexpr int BN = 128;             // keys per band block
+constexpr int BM = 128;             // queries per tile
+constexpr int BN = 64;              // keys per band block
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Register budgets with two pipelines (384 threads launched at 168 each):
+// the producer warpgroup keeps 56 (72 when it also gathers diagonal blocks),
+// the softmax warpgroups take the rest.
+template <int DS>
+struct Regs {
+    static constexpr int producer = DS > 0 ? 72 : 56;
+    static constexpr int softmax = DS > 0 ? 216 : 224;
+    static_assert(128 * producer + 256 * softmax <= 384 * 168, "register split");
+};
 
 struct FwdArgs {
     int64_t T;
@@ -53,27 +66,29 @@ struct FwdArgs {
     int64_t offs[SA_MAX_OFFSETS];  // distances (structured), descending
     const int64_t *rowptr;         // CSR
     const int32_t *colidx;
-    const __nv_bfloat16 *k;        // CSR gathers read K/V directly
-    const __nv_bfloat16 *v;
     __nv_bfloat16 *out;
     float *lse;
     float scale2;                  // scale * log2(e)
     int *err;
 };
 
-template <int D, int KS, int VS, int DS>
+// Shared memory: NP pipeline regions, then barriers.  All tiles are K-major
+// with 128-byte swizzle, 64 columns (128 bytes) per row and chunk.
+template <int D, int NP, int KS, int VS, int DS>
 struct Layout {
-    static constexpr int kTile = BM * D * 2;            // 128 rows x D bf16
-    static constexpr int kQ = 0;                        // two Q buffers
-    static constexpr int kBandK = kQ + 2 * kTile;
-    static constexpr int kBandV = kBandK + KS * kTile;
-    static constexpr int kDiagK = kBandV + VS * kTile;
-    static constexpr int kDiagV = kDiagK + DS * kTile;
-    static constexpr int kBars = kDiagV + DS * kTile;
-    static constexpr int DSX = DS > 0 ? DS : 1;          // ring modulus
-    // barriers (S, P, PVDone per S buffer: P is written over S in TMEM)
-    static constexpr int bQFull = 0, bQEmpty = 2;
-    static constexpr int bKFull = 4, bKEmpty = bKFull + KS;
+    static constexpr int kQTile = BM * D * 2;          // 128 rows x D
+    static constexpr int kBlk = BN * D * 2;            // 64 rows x D
+    static constexpr int pQ = 0;
+    static constexpr int pK = pQ + kQTile;              // band K ring
+    static constexpr int pV = pK + KS * kBlk;           // band V ring
+    static constexpr int pDK = pV + VS * kBlk;          // diagonal K ring
+    static constexpr int pDV = pDK + DS * kQTile;       // diagonal V ring
+    static constexpr int kPipe = pDV + DS * kQTile;
+    static constexpr int kBars = NP * kPipe;
+    static constexpr int DSX = DS > 0 ? DS : 1;         // ring modulus
+    // barriers of one pipeline (S, P, PVDone per S buffer: P is written over S)
+    static constexpr int bQFull = 0, bQEmpty = 1;
+    static constexpr int bKFull = 2, bKEmpty = bKFull + KS;
     static constexpr int bVFull = bKEmpty + KS, bVEmpty = bVFull + VS;
     static constexpr int bSFull = bVEmpty + VS, bSFree = bSFull + 2;
     static constexpr int bPFull = bSFree + 2, bPVDone = bPFull + 2;
@@ -81,14 +96,16 @@ struct Layout {
     static constexpr int bDiagFull = bOInit + 1, bDiagEmpty = bDiagFull + DSX;
     static constexpr int bInfoFull = bDiagEmpty + DSX, bInfoEmpty = bInfoFull + 2;
     static constexpr int bGroup = bInfoEmpty + 2;        // 128-thread softmax barrier
-    static constexpr int nBars = bGroup + 1;
-    static constexpr int kMisc = kBars + nBars * 8;      // tmem slot, abort, info[2]
-    static constexpr int kTotal = kMisc + 16;
+    static constexpr int nBarsPipe = bGroup + 1;
+    static constexpr int kMisc = kBars + NP * nBarsPipe * 8;  // tmem slot, abort, info[NP][2]
+    static constexpr int kTotal = kMisc + 8 + 8 * NP;
     static constexpr int kAlloc = kTotal + 1024;         // alignment slack
-    // TMEM columns: S buffers [0,128) and [128,256) (P, bf16, over the first
-    // 64 columns of its S buffer), O at 256
-    static constexpr uint32_t tS0 = 0, tO = 256;
+    // TMEM columns of pipeline p start at 256 p: S buffers [0, BN) and
+    // [BN, 2 BN) (P, bf16, over the first BN/2 columns of its S buffer), O at 2 BN
+    static constexpr uint32_t tPipe = 256, tS0 = 0, tO = 2 * BN;
     static constexpr uint32_t kTmemCols = 512;
+    static_assert(2 * BN + D <= 256, "TMEM columns of a pipeline");
+    static_assert(kQTile % 1024 == 0 && kBlk % 1024 == 0, "swizzle atoms");
 };
 
 // Geometry of query tile t (tiles run over B*H slices, 128 queries each).
@@ -111,56 +128,62 @@ __device__ __forceinline__ TileGeom tile_geom(int64_t t, int64_t ntq, int64_t T,
     return g;
 }
 
-// Persistent: each CTA walks the tiles blockIdx.x, blockIdx.x + gridDim.x, ...
-// Every ring (Q, K, V, S, P, diagonal blocks) keeps its phase across tiles, so
-// the loads and MMAs of the next tile proceed while the current one finishes.
-template <int D, int KS, int VS, int DS>
-__global__ void __launch_bounds__(256, 1)
+// Pipeline p of CTA c takes the tiles c NP + p, c NP + p + NP G, ... (G CTAs):
+// the two pipelines of a CTA work on neighbouring tiles.  Every ring keeps its
+// phase across tiles, so the loads and MMAs of the next tile proceed while
+// the current one finishes.
+template <int D, int NP, int KS, int VS, int DS>
+__global__ void __launch_bounds__(128 + 128 * NP, 1)
 band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkr,
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkd,
+                const __grid_constant__ CUtensorMap tvd, const __grid_constant__ CUtensorMap tkr,
                 const __grid_constant__ CUtensorMap tvr, const FwdArgs a) {
-    using L = Layout<D, KS, VS, DS>;
+    using L = Layout<D, NP, KS, VS, DS>;
     constexpr int DSX = L::DSX;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_u32(sm);
     uint32_t *tmem_slot = (uint32_t *)(sm + L::kMisc);
     volatile int *abort = (volatile int *)(sm + L::kMisc + 4);
-    volatile int *info = (volatile int *)(sm + L::kMisc + 8);  // diagonal blocks of tile slot 0/1
-    auto bar = [&](int b) { return sbase + L::kBars + 8u * (uint32_t)b; };
-    auto wait = [&](int b, uint32_t parity) {
-        return tc::mbar_wait(bar(b), parity, abort, a.err, SA_DEVERR_TIMEOUT);
+    auto bar = [&](int p, int b) {
+        return sbase + L::kBars + 8u * (uint32_t)(p * L::nBarsPipe + b);
+    };
+    auto wait = [&](int p, int b, uint32_t parity) {
+        return tc::mbar_wait(bar(p, b), parity, abort, a.err, SA_DEVERR_TIMEOUT);
     };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t T = a.T;
     const int32_t W = a.W;
     const int64_t ntq = (T + BM - 1) / BM, ntiles = ntq * a.BH;
+    const int64_t stride = (int64_t)gridDim.x * NP;
 
     if (tid == 0) {
-        for (int s = 0; s < 2; ++s) {
-            tc::mbar_init(bar(L::bQFull + s), 1);
-            tc::mbar_init(bar(L::bQEmpty + s), 5);  // last S MMA commit + 4 softmax warps
-            tc::mbar_init(bar(L::bSFull + s), 1);
-            tc::mbar_init(bar(L::bSFree + s), 1);   // P V of the buffer's block done
-            tc::mbar_init(bar(L::bPFull + s), 4);
-            tc::mbar_init(bar(L::bPVDone + s), 1);
-            tc::mbar_init(bar(L::bInfoFull + s), 1);
-            tc::mbar_init(bar(L::bInfoEmpty + s), 4);
-        }
-        for (int s = 0; s < KS; ++s) {
-            tc::mbar_init(bar(L::bKFull + s), 1);
-            tc::mbar_init(bar(L::bKEmpty + s), 1);
-        }
-        for (int s = 0; s < VS; ++s) {
-            tc::mbar_init(bar(L::bVFull + s), 1);
-            tc::mbar_init(bar(L::bVEmpty + s), 1);
-        }
-        tc::mbar_init(bar(L::bOInit), 4);
-        tc::mbar_init(bar(L::bGroup), 128);
-        for (int s = 0; s < DSX; ++s) {
-            tc::mbar_init(bar(L::bDiagFull + s), 1);
-            tc::mbar_init(bar(L::bDiagEmpty + s), 4);
+        for (int p = 0; p < NP; ++p) {
+            tc::mbar_init(bar(p, L::bQFull), 1);
+            tc::mbar_init(bar(p, L::bQEmpty), 5);  // last S MMA commit + 4 softmax warps
+            for (int s = 0; s < 2; ++s) {
+                tc::mbar_init(bar(p, L::bSFull + s), 1);
+                tc::mbar_init(bar(p, L::bSFree + s), 1);   // P V of the buffer's block done
+                tc::mbar_init(bar(p, L::bPFull + s), 4);
+                tc::mbar_init(bar(p, L::bPVDone + s), 1);
+                tc::mbar_init(bar(p, L::bInfoFull + s), 1);
+                tc::mbar_init(bar(p, L::bInfoEmpty + s), 4);
+            }
+            for (int s = 0; s < KS; ++s) {
+                tc::mbar_init(bar(p, L::bKFull + s), 1);
+                tc::mbar_init(bar(p, L::bKEmpty + s), 1);
+            }
+            for (int s = 0; s < VS; ++s) {
+                tc::mbar_init(bar(p, L::bVFull + s), 1);
+                tc::mbar_init(bar(p, L::bVEmpty + s), 1);
+            }
+            tc::mbar_init(bar(p, L::bOInit), 4);
+            tc::mbar_init(bar(p, L::bGroup), 128);
+            for (int s = 0; s < DSX; ++s) {
+                tc::mbar_init(bar(p, L::bDiagFull + s), 1);
+                tc::mbar_init(bar(p, L::bDiagEmpty + s), 4);
+            }
         }
         *abort = 0;
         tc::fence_barrier_init();
@@ -171,58 +194,156 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ---------------- TMA producer: Q of each tile, then its band K/V ring
+    if (warp < 4) {
+        // one register budget per warpgroup, set where it dominates the roles
+        if (NP == 2) tc::regs_dec<Regs<DS>::producer>();
+      if ((warp >> 1) < NP && (warp & 1) == 0) {
+        // ---------------- producer of pipeline p: per tile the diagonal-block
+        // count, Q, the first band K/V blocks, the diagonal blocks, the rest
+        const int p = warp >> 1;
+        const uint32_t pb = sbase + (uint32_t)(p * L::kPipe);
+        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
         if (lane == 0) {
             tc::tma_prefetch_desc(&tq);
             tc::tma_prefetch_desc(&tk);
             tc::tma_prefetch_desc(&tv);
-            uint32_t kc = 0, vc = 0;  // K and V blocks loaded so far (all tiles)
-            bool ok = true;
-            int64_t lt = 0;
-            for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++lt) {
-                const TileGeom g = tile_geom(t, ntq, T, W);
-                const int qb = (int)(lt & 1);
-                if (lt >= 2 && !wait(L::bQEmpty + qb, (uint32_t)(((lt >> 1) - 1) & 1))) break;
-                tc::mbar_arrive_expect_tx(bar(L::bQFull + qb), L::kTile);
-                for (int x = 0; x < D / 64; ++x)
-                    tc::tma_load_3d(sbase + L::kQ + qb * L::kTile + x * (BM * 128), &tq, x * 64,
-                                    (int32_t)g.q0, (int32_t)g.bh, bar(L::bQFull + qb));
-                // K runs one block ahead of V: K(b) is released as soon as S(b)
-                // is done, V(b) only after P(b) V(b)
-                auto load_k = [&](int bl) -> bool {
-                    const int st = (int)(kc % KS);
-                    const uint32_t use = kc / KS;
-                    if (use > 0 && !wait(L::bKEmpty + st, (use - 1) & 1)) return false;
-                    const int32_t krow = g.kb0 + (g.b_first + bl) * BN;
-                    tc::mbar_arrive_expect_tx(bar(L::bKFull + st), L::kTile);
-                    for (int x = 0; x < D / 64; ++x)
-                        tc::tma_load_3d(sbase + L::kBandK + st * L::kTile + x * (BN * 128), &tk,
-                                        x * 64, krow, (int32_t)g.bh, bar(L::bKFull + st));
-                    ++kc;
-                    return true;
-                };
-                auto load_v = [&](int bl) -> bool {
-                    const int st = (int)(vc % VS);
-                    const uint32_t use = vc / VS;
-                    if (use > 0 && !wait(L::bVEmpty + st, (use - 1) & 1)) return false;
-                    const int32_t krow = g.kb0 + (g.b_first + bl) * BN;
-                    tc::mbar_arrive_expect_tx(bar(L::bVFull + st), L::kTile);
-                    for (int x = 0; x < D / 64; ++x)
-                        tc::tma_load_3d(sbase + L::kBandV + st * L::kTile + x * (BN * 128), &tv,
-                                        x * 64, krow, (int32_t)g.bh, bar(L::bVFull + st));
-                    ++vc;
-                    return true;
-                };
-                ok = load_k(0);
-                for (int bl = 0; ok && bl < g.n_band; ++bl) {
-                    if (bl + 1 < g.n_band && !load_k(bl + 1)) ok = false;
-                    else if (!load_v(bl)) ok = false;
+        }
+        uint32_t kc = 0, vc = 0, dc = 0;  // K, V and diagonal blocks loaded (all tiles)
+        bool ok = true;
+        int64_t lt = 0;
+        for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
+            const TileGeom g = tile_geom(t, ntq, T, W);
+            const int64_t last = (g.q0 + BM - 1 < T - 1) ? g.q0 + BM - 1 : T - 1;
+            // CSR: lane l owns rows 4l .. 4l+3 (list start, residual count,
+            // key of the next slot, fetched one slot ahead)
+            int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
+            int32_t cj[4] = {0, 0, 0, 0};
+            int nd = 0;
+            if (DS > 0) {
+                if (a.kind == 0) {
+                    for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last) ? 1 : 0;
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const int64_t i = g.q0 + 4 * lane + h;
+                        if (i < T) {
+                            cstart[h] = a.rowptr[i];
+                            cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
+                            if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
+                            nd = nd > (int)cres[h] ? nd : (int)cres[h];
+                        }
+                    }
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const int x = __shfl_xor_sync(0xffffffffu, nd, o);
+                        nd = nd > x ? nd : x;
+                    }
                 }
             }
+            const int slot = (int)(lt & 1);
+            if (lt >= 2 && !wait(p, L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1))) break;
+            if (lane == 0) {
+                info[slot] = nd;
+                tc::mbar_arrive(bar(p, L::bInfoFull + slot));
+            }
+            // band ring loads (lane 0)
+            auto load_k = [&](int bl) -> bool {
+                const int st = (int)(kc % KS);
+                const uint32_t use = kc / KS;
+                if (use > 0 && !wait(p, L::bKEmpty + st, (use - 1) & 1)) return false;
+                const int32_t krow = g.kb0 + (g.b_first + bl) * BN;
+                tc::mbar_arrive_expect_tx(bar(p, L::bKFull + st), L::kBlk);
+                for (int x = 0; x < D / 64; ++x)
+                    tc::tma_load_3d(pb + L::pK + st * L::kBlk + x * (BN * 128), &tk, x * 64, krow,
+                                    (int32_t)g.bh, bar(p, L::bKFull + st));
+                ++kc;
+                return true;
+            };
+            auto load_v = [&](int bl) -> bool {
+                const int st = (int)(vc % VS);
+                const uint32_t use = vc / VS;
+                if (use > 0 && !wait(p, L::bVEmpty + st, (use - 1) & 1)) return false;
+                const int32_t krow = g.kb0 + (g.b_first + bl) * BN;
+                tc::mbar_arrive_expect_tx(bar(p, L::bVFull + st), L::kBlk);
+                for (int x = 0; x < D / 64; ++x)
+                    tc::tma_load_3d(pb + L::pV + st * L::kBlk + x * (BN * 128), &tv, x * 64, krow,
+                                    (int32_t)g.bh, bar(p, L::bVFull + st));
+                ++vc;
+                return true;
+            };
+            // the band blocks that fit the rings go before the diagonal ones
+            const int n_pre = g.n_band < (KS < VS ? KS : VS) ? g.n_band : (KS < VS ? KS : VS);
+            int okl = 1;
+            if (lane == 0) {
+                // Q of this tile once the previous tile's last S MMA and the
+                // softmax warps are done with the buffer
+                if (lt >= 1 && !wait(p, L::bQEmpty, (uint32_t)((lt - 1) & 1))) okl = 0;
+                if (okl) {
+                    tc::mbar_arrive_expect_tx(bar(p, L::bQFull), L::kQTile);
+                    for (int x = 0; x < D / 64; ++x)
+                        tc::tma_load_3d(pb + L::pQ + x * (BM * 128), &tq, x * 64, (int32_t)g.q0,
+                                        (int32_t)g.bh, bar(p, L::bQFull));
+                }
+                for (int bl = 0; okl && bl < n_pre; ++bl)
+                    if (!load_k(bl) || !load_v(bl)) okl = 0;
+            }
+            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+            for (int d = 0; ok && d < nd; ++d) {
+                const int st = (int)(dc % DSX);
+                const uint32_t use = dc / DSX;
+                const uint32_t kdst = pb + L::pDK + st * L::kQTile;
+                const uint32_t vdst = pb + L::pDV + st * L::kQTile;
+                if (use > 0 && !wait(p, L::bDiagEmpty + st, (use - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar(p, L::bDiagFull + st), 2 * L::kQTile);
+                if (a.kind == 0) {
+                    if (lane == 0) {
+                        // distance links: keys q0-o .. q0+127-o, one box each
+                        const int32_t krow = (int32_t)(g.q0 - a.offs[a.n_off - nd + d]);
+                        for (int x = 0; x < D / 64; ++x) {
+                            tc::tma_load_3d(kdst + x * (BM * 128), &tkd, x * 64, krow,
+                                            (int32_t)g.bh, bar(p, L::bDiagFull + st));
+                            tc::tma_load_3d(vdst + x * (BM * 128), &tvd, x * 64, krow,
+                                            (int32_t)g.bh, bar(p, L::bDiagFull + st));
+                        }
+                    }
+                } else {
+                    // CSR slot d: 4-row TMA gathers of K and V rows
+                    // (unswizzled); a row without slot d loads its own key
+                    int32_t rr[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const int64_t i = g.q0 + 4 * lane + h;
+                        const int64_t j = d < cres[h] ? (int64_t)cj[h] : (i < T ? i : 0);
+                        rr[h] = (int32_t)(g.bh * T + j);
+                    }
+#pragma unroll
+                    for (int x = 0; x < D / 64; ++x) {
+                        const uint32_t off = x * (BM * 128) + 4 * lane * 128;
+                        tc::tma_gather4(kdst + off, &tkr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                        bar(p, L::bDiagFull + st));
+                        tc::tma_gather4(vdst + off, &tvr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                                        bar(p, L::bDiagFull + st));
+                    }
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        if (d + 1 < cres[h]) cj[h] = a.colidx[cstart[h] + d + 1];
+                }
+                ++dc;
+            }
+            if (!ok) break;
+            if (lane == 0)
+                for (int bl = n_pre; okl && bl < g.n_band; ++bl)
+                    if (!load_k(bl) || !load_v(bl)) okl = 0;
+            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
         }
-    } else if (warp == 1) {
-        // ---------------- MMA issuer: S of block g, then P V of block g-1
+      } else if ((warp >> 1) < NP) {
+        // ---------------- MMA issuer of pipeline p: S of block g, then P V of
+        // block g-1
+        const int p = warp >> 1;
+        const uint32_t pb = sbase + (uint32_t)(p * L::kPipe);
+        const uint32_t tp = tmem + p * L::tPipe;
         if (lane == 0) {
             const uint32_t idS = tc::idesc_bf16(BM, BN, false, false);
             const uint32_t idO = tc::idesc_bf16(BM, D, false, true);
@@ -232,47 +353,47 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             int64_t pv_lt = 0;
             auto do_pv = [&]() -> bool {
                 const int sb = (int)(pv_gb & 1), vst = (int)(pv_gb % VS);
-                if (pv_first && !wait(L::bOInit, (uint32_t)(pv_lt & 1))) return false;
-                if (!wait(L::bPFull + sb, (pv_gb >> 1) & 1)) return false;
-                if (!wait(L::bVFull + vst, (pv_gb / VS) & 1)) return false;
+                if (pv_first && !wait(p, L::bOInit, (uint32_t)(pv_lt & 1))) return false;
+                if (!wait(p, L::bPFull + sb, (pv_gb >> 1) & 1)) return false;
+                if (!wait(p, L::bVFull + vst, (pv_gb / VS) & 1)) return false;
                 tc::tc_fence_after();
-                // A = P (bf16) in TMEM over the first 64 columns of its S buffer
-                const uint32_t pt = tmem + L::tS0 + sb * BN;
-                const uint32_t va = sbase + L::kBandV + vst * L::kTile;
+                // A = P (bf16) in TMEM over the first BN/2 columns of its S buffer
+                const uint32_t pt = tp + L::tS0 + sb * BN;
+                const uint32_t va = pb + L::pV + vst * L::kBlk;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    tc::mma_bf16_ts(tmem + L::tO, pt + kk * 8,
+                    tc::mma_bf16_ts(tp + L::tO, pt + kk * 8,
                                     tc::sdesc_sw128(va + kk * 16 * 128, BN * 128, 1024), idO, 1u);
-                tc::mma_commit(bar(L::bVEmpty + vst));
-                tc::mma_commit(bar(L::bPVDone + sb));
-                tc::mma_commit(bar(L::bSFree + sb));
+                tc::mma_commit(bar(p, L::bVEmpty + vst));
+                tc::mma_commit(bar(p, L::bPVDone + sb));
+                tc::mma_commit(bar(p, L::bSFree + sb));
                 return true;
             };
             int64_t lt = 0;
-            for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++lt) {
+            for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
                 const TileGeom g = tile_geom(t, ntq, T, W);
-                const int qb = (int)(lt & 1);
-                if (!wait(L::bQFull + qb, (uint32_t)((lt >> 1) & 1))) break;
-                const uint32_t qa = sbase + L::kQ + qb * L::kTile;
+                if (!wait(p, L::bQFull, (uint32_t)(lt & 1))) break;
+                const uint32_t qa = pb + L::pQ;
                 for (int bl = 0; bl < g.n_band; ++bl) {
                     const int st = (int)(kc % KS), sb = (int)(gb & 1);
-                    if (!wait(L::bKFull + st, (kc / KS) & 1) ||
-                        (gb >= 2 && !wait(L::bSFree + sb, ((gb >> 1) - 1) & 1))) {
+                    if (!wait(p, L::bKFull + st, (kc / KS) & 1) ||
+                        (gb >= 2 && !wait(p, L::bSFree + sb, ((gb >> 1) - 1) & 1))) {
                         ok = false;
                         break;
                     }
                     tc::tc_fence_after();
-                    const uint32_t ka = sbase + L::kBandK + st * L::kTile;
+                    const uint32_t ka = pb + L::pK + st * L::kBlk;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                        tc::mma_bf16_ss(tmem + L::tS0 + sb * BN,
-                                        tc::sdesc_sw128(qa + off, 16, 1024),
-                                        tc::sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
+                        const uint32_t in = (kk & 3) * 32;
+                        tc::mma_bf16_ss(tp + L::tS0 + sb * BN,
+                                        tc::sdesc_sw128(qa + (kk >> 2) * (BM * 128) + in, 16, 1024),
+                                        tc::sdesc_sw128(ka + (kk >> 2) * (BN * 128) + in, 16, 1024),
+                                        idS, kk > 0);
                     }
-                    tc::mma_commit(bar(L::bSFull + sb));
-                    tc::mma_commit(bar(L::bKEmpty + st));
-                    if (bl == g.n_band - 1) tc::mma_commit(bar(L::bQEmpty + qb));
+                    tc::mma_commit(bar(p, L::bSFull + sb));
+                    tc::mma_commit(bar(p, L::bKEmpty + st));
+                    if (bl == g.n_band - 1) tc::mma_commit(bar(p, L::bQEmpty));
                     ++kc;
                     // the softmax of this block overlaps P V of the previous one
                     if (have_pv && !do_pv()) {
@@ -288,114 +409,33 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             }
             if (ok && have_pv) do_pv();
         }
-    } else if (warp == 2 || warp == 3) {
-        // ---------------- warp 2: count and stage each tile's diagonal blocks
-        // (warp 3 has no role)
-        if (warp == 2) {
-            uint32_t dc = 0;  // diagonal blocks staged so far (all tiles)
-            int64_t lt = 0;
-            bool ok = true;
-            for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++lt) {
-                const TileGeom g = tile_geom(t, ntq, T, W);
-                const int64_t last = (g.q0 + BM - 1 < T - 1) ? g.q0 + BM - 1 : T - 1;
-                // CSR: lane l owns rows 4l .. 4l+3 (list start, residual count,
-                // key of the next slot, fetched one slot ahead)
-                int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
-                int32_t cj[4] = {0, 0, 0, 0};
-                int nd = 0;
-                if (DS > 0) {
-                    if (a.kind == 0) {
-                        for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last) ? 1 : 0;
-                    } else {
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const int64_t i = g.q0 + 4 * lane + h;
-                            if (i < T) {
-                                cstart[h] = a.rowptr[i];
-                                cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
-                                if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
-                                nd = nd > (int)cres[h] ? nd : (int)cres[h];
-                            }
-                        }
-                        for (int o = 16; o > 0; o >>= 1) {
-                            const int x = __shfl_xor_sync(0xffffffffu, nd, o);
-                            nd = nd > x ? nd : x;
-                        }
-                    }
-                }
-                const int slot = (int)(lt & 1);
-                if (lt >= 2 && !wait(L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1))) break;
-                if (lane == 0) {
-                    info[slot] = nd;
-                    tc::mbar_arrive(bar(L::bInfoFull + slot));
-                }
-                for (int d = 0; d < nd; ++d) {
-                    const int st = (int)(dc % DSX);
-                    const uint32_t use = dc / DSX;
-                    const uint32_t kdst = sbase + L::kDiagK + st * L::kTile;
-                    const uint32_t vdst = sbase + L::kDiagV + st * L::kTile;
-                    if (use > 0 && !wait(L::bDiagEmpty + st, (use - 1) & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    if (lane == 0) tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kTile);
-                    if (a.kind == 0) {
-                        if (lane == 0) {
-                            // distance links: keys q0-o .. q0+127-o, one box each
-                            const int32_t krow = (int32_t)(g.q0 - a.offs[a.n_off - nd + d]);
-                            for (int x = 0; x < D / 64; ++x) {
-                                tc::tma_load_3d(kdst + x * (BM * 128), &tk, x * 64, krow,
-                                                (int32_t)g.bh, bar(L::bDiagFull + st));
-                                tc::tma_load_3d(vdst + x * (BM * 128), &tv, x * 64, krow,
-                                                (int32_t)g.bh, bar(L::bDiagFull + st));
-                            }
-                        }
-                    } else {
-                        // CSR slot d: 4-row TMA gathers of K and V rows
-                        // (unswizzled); a row without slot d loads its own key
-                        int32_t rr[4];
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const int64_t i = g.q0 + 4 * lane + h;
-                            const int64_t j = d < cres[h] ? (int64_t)cj[h] : (i < T ? i : 0);
-                            rr[h] = (int32_t)(g.bh * T + j);
-                        }
-#pragma unroll
-                        for (int x = 0; x < D / 64; ++x) {
-                            const uint32_t off = x * (BM * 128) + 4 * lane * 128;
-                            tc::tma_gather4(kdst + off, &tkr, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                            bar(L::bDiagFull + st));
-                            tc::tma_gather4(vdst + off, &tvr, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                            bar(L::bDiagFull + st));
-                        }
-#pragma unroll
-                        for (int h = 0; h < 4; ++h)
-                            if (d + 1 < cres[h]) cj[h] = a.colidx[cstart[h] + d + 1];
-                    }
-                    ++dc;
-                }
-            }
-        }
-    } else if (warp >= 4 && warp < 8) {
-        // ---------------- softmax warpgroup: thread r = query row r = TMEM lane r
-        const int r = tid - 128;
-        const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
-        const uint32_t tS = tmem + lane_off + L::tS0, tO = tmem + lane_off + L::tO;
+      }
+    } else {
+        // ---------------- softmax warpgroup of pipeline p: thread r = query
+        // row r = TMEM lane r
+        if (NP == 2) tc::regs_inc<Regs<DS>::softmax>();
+        const int p = (warp - 4) >> 2;
+        const int r = tid - 128 - 128 * p;
+        uint8_t *pm = sm + p * L::kPipe;
+        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
+        const uint32_t lane_off = (uint32_t)(((warp - 4) & 3) * 32) << 16;
+        const uint32_t tS = tmem + p * L::tPipe + lane_off + L::tS0;
+        const uint32_t tO = tmem + p * L::tPipe + lane_off + L::tO;
         const float c2 = a.scale2;
         uint32_t dc = 0, gb = 0;  // diagonal blocks and band blocks consumed (all tiles)
         uint32_t group_uses = 0;  // phases of the softmax group barrier
         bool ok = true;
         int64_t lt = 0;
-        for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++lt) {
+        for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
             const TileGeom g = tile_geom(t, ntq, T, W);
             const int32_t q0 = g.q0, bh = g.bh;
             const int32_t i = q0 + r;
-            const int slot = (int)(lt & 1), qb = (int)(lt & 1);
+            const int slot = (int)(lt & 1);
             float m_run = -INFINITY, l_run = 0.f;
-            if (!wait(L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1))) break;
+            if (!wait(p, L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1))) break;
             const int nd = info[slot];
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(L::bInfoEmpty + slot));
+            if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
 
             // --- diagonal blocks: q row from the Q tile, one key/value row per
             // block; fp32 pairs (f32x2 FMA), running max rescaled lazily (only
@@ -405,7 +445,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
 #pragma unroll
                 for (int x = 0; x < D / 2; ++x) acc2[x] = 0ull;
                 if (DS > 0 && nd > 0) {
-                    ok = wait(L::bQFull + qb, (uint32_t)((lt >> 1) & 1));
+                    ok = wait(p, L::bQFull, (uint32_t)(lt & 1));
                     // Structured blocks are swizzled like Q: q in logical
                     // order.  CSR gathers are unswizzled: reading them at the
                     // swizzled address gives chunk c ^ (r & 7), which pairs with
@@ -419,7 +459,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                                 (c >> 3) * (BM * 128) +
                                 (a.kind == 0 ? tc::sw128_off(r, c & 7)
                                              : (uint32_t)r * 128u + ((c & 7) << 4));
-                            const uint4 w4 = *(const uint4 *)(sm + L::kQ + qb * L::kTile + qoff);
+                            const uint4 w4 = *(const uint4 *)(pm + L::pQ + qoff);
                             q2[4 * c] = tc::bf2_to_f2(w4.x);
                             q2[4 * c + 1] = tc::bf2_to_f2(w4.y);
                             q2[4 * c + 2] = tc::bf2_to_f2(w4.z);
@@ -433,7 +473,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     }
                     for (int d = 0; ok && d < nd; ++d) {
                         const int st = (int)(dc % DSX);
-                        if (!wait(L::bDiagFull + st, (dc / DSX) & 1)) {
+                        if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
                             ok = false;
                             break;
                         }
@@ -443,8 +483,8 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         else
                             valid = d < resid;
                         if (valid) {
-                            const uint8_t *kr = sm + L::kDiagK + st * L::kTile;
-                            const uint8_t *vr = sm + L::kDiagV + st * L::kTile;
+                            const uint8_t *kr = pm + L::pDK + st * L::kQTile;
+                            const uint8_t *vr = pm + L::pDV + st * L::kQTile;
                             // four independent partial sums (short dependency chains)
                             uint64_t sp0 = 0ull, sp1 = 0ull, sp2 = 0ull, sp3 = 0ull;
 #pragma unroll
@@ -469,9 +509,9 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                                 l_run *= al;
                                 m_run = s;
                             }
-                            const float p = tc::ex2(s - m_run);
-                            l_run += p;
-                            const uint64_t p2 = tc::f2pack(p, p);
+                            const float pr = tc::ex2(s - m_run);
+                            l_run += pr;
+                            const uint64_t p2 = tc::f2pack(pr, pr);
 #pragma unroll
                             for (int c = 0; c < D / 8; ++c) {
                                 const uint4 w4 = *(const uint4 *)(vr + (c >> 3) * (BM * 128) +
@@ -488,22 +528,21 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         const bool hold = (a.kind == 1) && (d == nd - 1);
                         if (!hold) {
                             __syncwarp();
-                            if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                            if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
                         }
                         ++dc;
                     }
-                    if (a.kind == 1) {
+                    if (ok && a.kind == 1) {
                         // undo the chunk permutation (per 64-column half) through
                         // the last diagonal stage, whose release was held back:
                         // once every row is done with it, thread r uses 256 bytes
                         // (rows < 64 in its K half, the others in its V half)
                         const int st = (int)((dc - 1) % DSX);
-                        // every row is done with the stage (bounded wait)
-                        tc::mbar_arrive(bar(L::bGroup));
-                        if (!wait(L::bGroup, group_uses & 1)) ok = false;
+                        tc::mbar_arrive(bar(p, L::bGroup));
+                        if (!wait(p, L::bGroup, group_uses & 1)) ok = false;
                         ++group_uses;
                         uint64_t *scr =
-                            (uint64_t *)(sm + (r < 64 ? L::kDiagK : L::kDiagV) + st * L::kTile) +
+                            (uint64_t *)(pm + (r < 64 ? L::pDK : L::pDV) + st * L::kQTile) +
                             (size_t)(r & 63) * 32 * (D / 64);
 #pragma unroll
                         for (int hh = 0; hh < D / 64; ++hh) {
@@ -523,13 +562,13 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                             scr += 32;
                         }
                         __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                        if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
                     }
                 }
                 if (!ok) break;
                 // this warp is done reading Q of the tile
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar(L::bQEmpty + qb));
+                if (lane == 0) tc::mbar_arrive(bar(p, L::bQEmpty));
                 // initialise O (columns tO .. tO+D) with the diagonal part
 #pragma unroll
                 for (int c = 0; c < D; c += 32) {
@@ -544,7 +583,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 tc::tmem_st_wait();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar(L::bOInit));
+                if (lane == 0) tc::mbar_arrive(bar(p, L::bOInit));
             }
 
             // --- band blocks
@@ -553,7 +592,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 const int sb = (int)(gb & 1);
                 const int32_t b = g.b_first + bl;
                 gb_last = gb;
-                if (!wait(L::bSFull + sb, (gb >> 1) & 1)) {
+                if (!wait(p, L::bSFull + sb, (gb >> 1) & 1)) {
                     ok = false;
                     break;
                 }
@@ -564,7 +603,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     tc::tmem_ld32(tS + sb * BN + c, (uint32_t *)(s + c));
                 tc::tmem_ld_wait();
 
-                // mask: r <= u <= r+W-1 and key >= 0, with u = 128 b + c, i.e.
+                // mask: r <= u <= r+W-1 and key >= 0, with u = BN b + c, i.e.
                 // the column range [c_lo, c_hi] of this block.  Scores stay raw
                 // (the scale is folded into the exponent's FFMA); a masked raw
                 // score is set to the extreme that the max/min below ignores.
@@ -605,7 +644,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     const float alpha = grow ? tc::ex2(m_run - m_new) : 1.f;
                     if (bl > 0) {  // O must hold P V of the previous block of this tile
                         const uint32_t pg = gb - 1;
-                        if (!wait(L::bPVDone + (int)(pg & 1), (pg >> 1) & 1)) {
+                        if (!wait(p, L::bPVDone + (int)(pg & 1), (pg >> 1) & 1)) {
                             ok = false;
                             break;
                         }
@@ -624,7 +663,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     l_run *= alpha;
                     m_run = m_new;
                 }
-                // p = 2^(s - m), row sum, bf16 P over the first 64 columns of
+                // p = 2^(s - m), row sum, bf16 P over the first BN/2 columns of
                 // this S buffer (its scores are already in registers)
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;  // all-masked row: p = 0
                 float ls[4] = {0.f, 0.f, 0.f, 0.f};
@@ -666,12 +705,12 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 tc::tmem_st_wait();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar(L::bPFull + sb));
+                if (lane == 0) tc::mbar_arrive(bar(p, L::bPFull + sb));
             }
             if (!ok) break;
 
             // --- epilogue: O / l and lse once the tile's last P V is done
-            if (!wait(L::bPVDone + (int)(gb_last & 1), (gb_last >> 1) & 1)) break;
+            if (!wait(p, L::bPVDone + (int)(gb_last & 1), (gb_last >> 1) & 1)) break;
             tc::tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
             __nv_bfloat16 *orow = a.out + ((size_t)bh * (size_t)T + (size_t)i) * D;
@@ -710,19 +749,37 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     }
 }
 
-template <int D, int KS, int VS, int DS>
+template <int D, int NP, int KS, int VS, int DS>
 sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_graph_s *g, float scale, sa_tensor *out, float *lse,
                           cudaStream_t s) {
-    using L = Layout<D, KS, VS, DS>;
+    using L = Layout<D, NP, KS, VS, DS>;
     static_assert(L::kAlloc <= 232448, "shared memory budget");
+    constexpr int kThreads = 128 + 128 * NP;
+    auto kern = band_fwd_kernel<D, NP, KS, VS, DS>;
+    if (NP == 2) {
+        // setmaxnreg.inc waits until the CTA's pool holds the registers it
+        // asks for: the launch must provide the whole split
+        static int regs_ok = -1;
+        if (regs_ok < 0) {
+            cudaFuncAttributes fa;
+            SA_CUDA_TRY(cudaFuncGetAttributes(&fa, (const void *)kern));
+            regs_ok = fa.numRegs * kThreads >= 128 * Regs<DS>::producer + 128 * NP * Regs<DS>::softmax;
+        }
+        if (!regs_ok) {
+            sa_record_cuda_error(cudaErrorInvalidConfiguration,
+                                 "band_fwd: launch registers below the warpgroup split");
+            return SA_ERR_CUDA;
+        }
+    }
     const int64_t BH = q->B * q->H, T = q->T;
-    CUtensorMap mq, mk, mv, mkr, mvr;
+    CUtensorMap mq, mk, mv, mkd, mvd, mkr, mvr;
     if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BM) || !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BH, BN) ||
         !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BH, BN) ||
+        !sa_tmap_bf16_3d(&mkd, k->ptr, D, T, BH, BM) ||
+        !sa_tmap_bf16_3d(&mvd, v->ptr, D, T, BH, BM) ||
         !sa_tmap_bf16_rows(&mkr, k->ptr, D, (uint64_t)(BH * T)) ||
-        !sa_tmap_bf16_rows(&mvr, v->ptr, D, (uint64_t)(BH * T)))
-    {
+        !sa_tmap_bf16_rows(&mvr, v->ptr, D, (uint64_t)(BH * T))) {
         sa_record_cuda_error(cudaErrorInvalidValue, "band_fwd: tensor map encoding");
         return SA_ERR_CUDA;
     }
@@ -735,21 +792,20 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     for (int x = 0; x < SA_MAX_OFFSETS; ++x) a.offs[x] = x < a.n_off ? g->offs[x] : 0;
     a.rowptr = g->rowptr;
     a.colidx = g->colidx;
-    a.k = (const __nv_bfloat16 *)k->ptr;
-    a.v = (const __nv_bfloat16 *)v->ptr;
     a.out = (__nv_bfloat16 *)out->ptr;
     a.lse = lse;
     a.scale2 = scale * kLog2e;
     a.err = sa_device_error_word();
     if (!a.err) return SA_ERR_CUDA;
-    auto kern = band_fwd_kernel<D, KS, VS, DS>;
     SA_CUDA_TRY(sa_smem_optin((const void *)kern, L::kAlloc));
-    // persistent: one CTA per SM (shared memory and TMEM allow no more)
+    // persistent: one CTA per SM, NP tiles in flight in each
     const int64_t ntiles = ((T + BM - 1) / BM) * BH;
+    const int64_t nctas = (ntiles + NP - 1) / NP;
     int sms = 0;
     SA_CUDA_TRY(sa_sm_count(&sms));
-    const unsigned grid = (unsigned)(ntiles < sms ? ntiles : sms);
-    SA_LAUNCH("band_fwd", s, kern<<<grid, 256, L::kAlloc, s>>>(mq, mk, mv, mkr, mvr, a));
+    const unsigned grid = (unsigned)(nctas < sms ? nctas : sms);
+    SA_LAUNCH("band_fwd", s,
+              kern<<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, mkd, mvd, mkr, mvr, a));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
@@ -768,12 +824,12 @@ sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
                       const sa_graph_s *g, const GraphView &, float scale, sa_tensor *out,
                       float *lse, cudaStream_t s) {
     const bool diag = (g->kind == 0) ? g->n_off > 0 : g->max_resid > 0;
-    // <D, K stages, V stages, diagonal stages>, sized to the 227 KB of shared
-    // memory (two Q buffers; P lives in TMEM)
+    // <D, pipelines, K stages, V stages, diagonal stages>, sized to the 227 KB
+    // of shared memory
     if (q->D == 64) {
-        return diag ? launch_band_fwd<64, 2, 2, 4>(q, k, v, g, scale, out, lse, s)
-                    : launch_band_fwd<64, 2, 4, 0>(q, k, v, g, scale, out, lse, s);
+        return diag ? launch_band_fwd<64, 2, 2, 2, 2>(q, k, v, g, scale, out, lse, s)
+                    : launch_band_fwd<64, 2, 4, 4, 0>(q, k, v, g, scale, out, lse, s);
     }
-    return diag ? launch_band_fwd<128, 1, 1, 1>(q, k, v, g, scale, out, lse, s)
-                : launch_band_fwd<128, 2, 3, 0>(q, k, v, g, scale, out, lse, s);
+    return diag ? launch_band_fwd<128, 1, 2, 2, 2>(q, k, v, g, scale, out, lse, s)
+                : launch_band_fwd<128, 2, 3, 2, 0>(q, k, v, g, scale, out, lse, s);
 }

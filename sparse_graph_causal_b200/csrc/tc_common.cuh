@@ -291,6 +291,19 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Per-warpgroup register budgets (all four warps of a warpgroup execute it).
+// `dec` returns registers to the CTA's pool, `inc` waits until the pool holds
+// enough: the launch's registers (threads x registers per thread) must cover
+// the sum of the budgets, which the host checks before launching.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128B-swizzled
 // tile whose rows are 128 bytes (the layout TMA writes with SWIZZLE_128B).
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {

@@ -15,13 +15,14 @@
 //
 // The other edges (2^k distance links or the non-window part of CSR lists)
 // are diagonal blocks as in the forward: row r of a block belongs to query
-// (or key) r; for a distance o the rows are one TMA box, for CSR lists 16-byte
-// cp.async gathers of the row's slot.  They are accumulated on CUDA cores
-// first and initialise the TMEM accumulators, which the band MMAs then add to.
+// (or key) r; for a distance o the rows are one TMA box, for CSR lists 4-row
+// TMA gathers of the row's slot.  They are accumulated on CUDA cores (fp32
+// pairs) first and initialise the TMEM accumulators, which the band MMAs then
+// add to.
 //
 // Warp roles (256 threads): 0 TMA producer, 1 TMEM allocator + MMA issuer,
-// 2-3 diagonal-block producers, 4-7 compute warpgroup (thread = owned row =
-// TMEM lane).  Waits are bounded as in the forward.
+// 2 diagonal-block producer (3 idle), 4-7 compute warpgroup (thread = owned
+// row = TMEM lane).  Waits are bounded as in the forward.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -98,110 +99,127 @@ __device__ __forceinline__ void load_row_packed(const uint8_t *tile, int rows, i
     }
 }
 
-// acc holds chunk t at logical chunk t ^ (r & 7) (per 64-column half): put it
-// back in logical order through row r of a D-float scratch row in shared memory.
-template <int D>
-__device__ __forceinline__ void unpermute_row(float *acc, float *scr_row, int r) {
-#pragma unroll
-    for (int t = 0; t < D / 8; ++t) {
-        const int lc = (t & ~7) | ((t & 7) ^ (r & 7));
-        *(float4 *)(scr_row + 8 * lc) =
-            make_float4(acc[8 * t], acc[8 * t + 1], acc[8 * t + 2], acc[8 * t + 3]);
-        *(float4 *)(scr_row + 8 * lc + 4) =
-            make_float4(acc[8 * t + 4], acc[8 * t + 5], acc[8 * t + 6], acc[8 * t + 7]);
-    }
-    __syncwarp();
-#pragma unroll
-    for (int t = 0; t < D / 4; ++t) {
-        const float4 f = *(const float4 *)(scr_row + 4 * t);
-        acc[4 * t] = f.x;
-        acc[4 * t + 1] = f.y;
-        acc[4 * t + 2] = f.z;
-        acc[4 * t + 3] = f.w;
-    }
+// ---- fp32-pair versions (f32x2 FMA): a row of D values as D/2 pairs
+// (elements 2e, 2e+1), four independent partial sums in the dot products.
+
+__device__ __forceinline__ float sum4_f2(uint64_t s0, uint64_t s1, uint64_t s2, uint64_t s3) {
+    return ((tc::f2lo(s0) + tc::f2hi(s0)) + (tc::f2lo(s1) + tc::f2hi(s1))) +
+           ((tc::f2lo(s2) + tc::f2hi(s2)) + (tc::f2lo(s3) + tc::f2hi(s3)));
 }
 
-// a . b over one row, a in registers (packed bf16 pairs), b row r of a tile.
+// a . b, both rows of swizzled tiles in shared memory (row r of each).
 template <int D>
-__device__ __forceinline__ float dot_reg_smem(const uint32_t *a, const uint8_t *tile, int rows,
-                                              int r) {
-    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        const uint4 x = *(const uint4 *)(tile + tile_off(rows, r, c));
-        const uint32_t b[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            sa[e] = fmaf(tc::bf16lo(a[4 * c + e]), tc::bf16lo(b[e]), sa[e]);
-            sb[e] = fmaf(tc::bf16hi(a[4 * c + e]), tc::bf16hi(b[e]), sb[e]);
-        }
-    }
-    return ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
-}
-
-// a . b, a = row r of a swizzled tile read in physical chunk order, b = row r
-// of an unswizzled gathered tile read at the swizzled address (so both give
-// logical chunk t ^ (r & 7) at step t).
-template <int D>
-__device__ __forceinline__ float dot_phys_gathered(const uint8_t *ta, const uint8_t *tb, int rows,
-                                                   int r) {
-    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        const uint4 x = *(const uint4 *)(ta + (c >> 3) * (rows * 128) + r * 128 + ((c & 7) << 4));
-        const uint4 y = *(const uint4 *)(tb + tile_off(rows, r, c));
-        const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            sa[e] = fmaf(tc::bf16lo(xa[e]), tc::bf16lo(yb[e]), sa[e]);
-            sb[e] = fmaf(tc::bf16hi(xa[e]), tc::bf16hi(yb[e]), sb[e]);
-        }
-    }
-    return ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
-}
-
-// a . b with both rows in shared memory (row r of each tile).
-template <int D>
-__device__ __forceinline__ float dot_smem_smem(const uint8_t *ta, const uint8_t *tb, int rows,
-                                               int r) {
-    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+__device__ __forceinline__ float dot2_smem_smem(const uint8_t *ta, const uint8_t *tb, int rows,
+                                                int r) {
+    uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull, s3 = 0ull;
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
         const uint4 x = *(const uint4 *)(ta + tile_off(rows, r, c));
         const uint4 y = *(const uint4 *)(tb + tile_off(rows, r, c));
-        const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            sa[e] = fmaf(tc::bf16lo(xa[e]), tc::bf16lo(yb[e]), sa[e]);
-            sb[e] = fmaf(tc::bf16hi(xa[e]), tc::bf16hi(yb[e]), sb[e]);
-        }
+        s0 = tc::ffma2(tc::bf2_to_f2(x.x), tc::bf2_to_f2(y.x), s0);
+        s1 = tc::ffma2(tc::bf2_to_f2(x.y), tc::bf2_to_f2(y.y), s1);
+        s2 = tc::ffma2(tc::bf2_to_f2(x.z), tc::bf2_to_f2(y.z), s2);
+        s3 = tc::ffma2(tc::bf2_to_f2(x.w), tc::bf2_to_f2(y.w), s3);
     }
-    return ((sa[0] + sb[0]) + (sa[1] + sb[1])) + ((sa[2] + sb[2]) + (sa[3] + sb[3]));
+    return sum4_f2(s0, s1, s2, s3);
 }
 
-// acc += a * (row r of a tile)
+// a . b, a = row r of a swizzled tile read in physical chunk order, b = row r
+// of an unswizzled gathered tile read at the swizzled address.
 template <int D>
-__device__ __forceinline__ void axpy_smem(float *acc, float a, const uint8_t *tile, int rows,
-                                          int r) {
+__device__ __forceinline__ float dot2_phys_gathered(const uint8_t *ta, const uint8_t *tb, int rows,
+                                                    int r) {
+    uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull, s3 = 0ull;
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
-        const uint4 x = *(const uint4 *)(tile + tile_off(rows, r, c));
-        const uint32_t b[4] = {x.x, x.y, x.z, x.w};
+        const uint4 x = *(const uint4 *)(ta + (c >> 3) * (rows * 128) + r * 128 + ((c & 7) << 4));
+        const uint4 y = *(const uint4 *)(tb + tile_off(rows, r, c));
+        s0 = tc::ffma2(tc::bf2_to_f2(x.x), tc::bf2_to_f2(y.x), s0);
+        s1 = tc::ffma2(tc::bf2_to_f2(x.y), tc::bf2_to_f2(y.y), s1);
+        s2 = tc::ffma2(tc::bf2_to_f2(x.z), tc::bf2_to_f2(y.z), s2);
+        s3 = tc::ffma2(tc::bf2_to_f2(x.w), tc::bf2_to_f2(y.w), s3);
+    }
+    return sum4_f2(s0, s1, s2, s3);
+}
+
+// a . b, a already unpacked to pairs (chunk c in a2[4c .. 4c+3]), b row r of
+// a tile read at the swizzled address.
+template <int D>
+__device__ __forceinline__ float dot2_reg_smem(const uint64_t *a2, const uint8_t *tile, int rows,
+                                               int r) {
+    uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull, s3 = 0ull;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            acc[8 * c + 2 * e] = fmaf(a, tc::bf16lo(b[e]), acc[8 * c + 2 * e]);
-            acc[8 * c + 2 * e + 1] = fmaf(a, tc::bf16hi(b[e]), acc[8 * c + 2 * e + 1]);
-        }
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 y = *(const uint4 *)(tile + tile_off(rows, r, c));
+        s0 = tc::ffma2(a2[4 * c], tc::bf2_to_f2(y.x), s0);
+        s1 = tc::ffma2(a2[4 * c + 1], tc::bf2_to_f2(y.y), s1);
+        s2 = tc::ffma2(a2[4 * c + 2], tc::bf2_to_f2(y.z), s2);
+        s3 = tc::ffma2(a2[4 * c + 3], tc::bf2_to_f2(y.w), s3);
+    }
+    return sum4_f2(s0, s1, s2, s3);
+}
+
+// a . b, a packed bf16 pairs in registers, b row r of a tile.
+template <int D>
+__device__ __forceinline__ float dot2_packed_smem(const uint32_t *a, const uint8_t *tile, int rows,
+                                                  int r) {
+    uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull, s3 = 0ull;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 y = *(const uint4 *)(tile + tile_off(rows, r, c));
+        s0 = tc::ffma2(tc::bf2_to_f2(a[4 * c]), tc::bf2_to_f2(y.x), s0);
+        s1 = tc::ffma2(tc::bf2_to_f2(a[4 * c + 1]), tc::bf2_to_f2(y.y), s1);
+        s2 = tc::ffma2(tc::bf2_to_f2(a[4 * c + 2]), tc::bf2_to_f2(y.z), s2);
+        s3 = tc::ffma2(tc::bf2_to_f2(a[4 * c + 3]), tc::bf2_to_f2(y.w), s3);
+    }
+    return sum4_f2(s0, s1, s2, s3);
+}
+
+// acc2 += a * (row r of a tile), pairs.
+template <int D>
+__device__ __forceinline__ void axpy2_smem(uint64_t *acc2, float a, const uint8_t *tile, int rows,
+                                           int r) {
+    const uint64_t a2 = tc::f2pack(a, a);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 y = *(const uint4 *)(tile + tile_off(rows, r, c));
+        acc2[4 * c] = tc::ffma2(a2, tc::bf2_to_f2(y.x), acc2[4 * c]);
+        acc2[4 * c + 1] = tc::ffma2(a2, tc::bf2_to_f2(y.y), acc2[4 * c + 1]);
+        acc2[4 * c + 2] = tc::ffma2(a2, tc::bf2_to_f2(y.z), acc2[4 * c + 2]);
+        acc2[4 * c + 3] = tc::ffma2(a2, tc::bf2_to_f2(y.w), acc2[4 * c + 3]);
+    }
+}
+
+// acc2 holds chunk t at logical chunk t ^ (r & 7) (per 64-column half): put it
+// back in logical order through a D-float scratch row in shared memory.
+template <int D>
+__device__ __forceinline__ void unpermute_row2(uint64_t *acc2, float *scr_row, int r) {
+    uint64_t *scr = (uint64_t *)scr_row;
+#pragma unroll
+    for (int t = 0; t < D / 8; ++t) {
+        const int lc = (t & ~7) | ((t & 7) ^ (r & 7));
+        *(ulonglong2 *)(scr + 4 * lc) = make_ulonglong2(acc2[4 * t], acc2[4 * t + 1]);
+        *(ulonglong2 *)(scr + 4 * lc + 2) = make_ulonglong2(acc2[4 * t + 2], acc2[4 * t + 3]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int t = 0; t < D / 4; ++t) {
+        const ulonglong2 f = *(const ulonglong2 *)(scr + 2 * t);
+        acc2[2 * t] = f.x;
+        acc2[2 * t + 1] = f.y;
     }
 }
 
 template <int D>
-__device__ __forceinline__ void tmem_store_row(uint32_t taddr, const float *acc) {
+__device__ __forceinline__ void tmem_store_row2(uint32_t taddr, const uint64_t *acc2) {
 #pragma unroll
     for (int c = 0; c < D; c += 32) {
         uint32_t w[32];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) w[x] = __float_as_uint(acc[c + x]);
+        for (int x = 0; x < 16; ++x) {
+            w[2 * x] = __float_as_uint(tc::f2lo(acc2[c / 2 + x]));
+            w[2 * x + 1] = __float_as_uint(tc::f2hi(acc2[c / 2 + x]));
+        }
         tc::tmem_st32(taddr + c, w);
     }
 }
@@ -465,6 +483,11 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         const uint32_t tDQ = tmem + lane_off + L::tDQ;
         const float c2 = a.scale2;
         const float lse2 = row_ok ? a.lse[grow] * kLog2e : 0.f;
+        // the out row for Delta is fetched while Q and dO arrive
+        uint4 orow4[D / 8];
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c)
+            orow4[c] = row_ok ? __ldg((const uint4 *)(a.o + grow * D) + c) : make_uint4(0, 0, 0, 0);
         bool ok = tc::mbar_wait(bar(L::bQFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
         float Delta = 0.f;
         if (ok) {
@@ -472,28 +495,33 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             uint32_t dor[D / 2];
             load_row_packed<D>(sm + L::kDO, BM, r, dor);
             if (row_ok) {
-                const uint4 *orow = (const uint4 *)(a.o + grow * D);
+                uint64_t d0 = 0ull, d1 = 0ull, d2 = 0ull, d3 = 0ull;
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
-                    const uint4 x = __ldg(orow + c);
-                    const uint32_t ow[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        Delta = fmaf(tc::bf16lo(dor[4 * c + e]), tc::bf16lo(ow[e]), Delta);
-                        Delta = fmaf(tc::bf16hi(dor[4 * c + e]), tc::bf16hi(ow[e]), Delta);
-                    }
+                    d0 = tc::ffma2(tc::bf2_to_f2(dor[4 * c]), tc::bf2_to_f2(orow4[c].x), d0);
+                    d1 = tc::ffma2(tc::bf2_to_f2(dor[4 * c + 1]), tc::bf2_to_f2(orow4[c].y), d1);
+                    d2 = tc::ffma2(tc::bf2_to_f2(dor[4 * c + 2]), tc::bf2_to_f2(orow4[c].z), d2);
+                    d3 = tc::ffma2(tc::bf2_to_f2(dor[4 * c + 3]), tc::bf2_to_f2(orow4[c].w), d3);
                 }
+                Delta = sum4_f2(d0, d1, d2, d3);
                 a.delta[grow] = Delta;
             }
-            // diagonal blocks
-            float acc[D];
+            // diagonal blocks (fp32 pairs)
+            uint64_t acc2[D / 2];
 #pragma unroll
-            for (int x = 0; x < D; ++x) acc[x] = 0.f;
+            for (int x = 0; x < D / 2; ++x) acc2[x] = 0ull;
             if (DS > 0 && n_diag > 0) {
                 if (a.kind == 0) {
                     // distance links: swizzled tiles, q in logical chunk order
-                    uint32_t qr[D / 2];
-                    load_row_packed<D>(sm + L::kQ, BM, r, qr);
+                    uint64_t q2[D / 2];
+#pragma unroll
+                    for (int c = 0; c < D / 8; ++c) {
+                        const uint4 x = *(const uint4 *)(sm + L::kQ + tile_off(BM, r, c));
+                        q2[4 * c] = tc::bf2_to_f2(x.x);
+                        q2[4 * c + 1] = tc::bf2_to_f2(x.y);
+                        q2[4 * c + 2] = tc::bf2_to_f2(x.z);
+                        q2[4 * c + 3] = tc::bf2_to_f2(x.w);
+                    }
                     for (int d = 0; d < n_diag; ++d) {
                         const int st = d % DSX;
                         WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
@@ -501,9 +529,9 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                             const uint8_t *kt = sm + L::kDiagK + st * L::kRow;
                             const uint8_t *vt = sm + L::kDiagV + st * L::kRow;
                             const float p =
-                                tc::ex2(fmaf(dot_reg_smem<D>(qr, kt, BM, r), c2, -lse2));
-                            const float ds = p * (dot_reg_smem<D>(dor, vt, BM, r) - Delta);
-                            axpy_smem<D>(acc, ds, kt, BM, r);
+                                tc::ex2(fmaf(dot2_reg_smem<D>(q2, kt, BM, r), c2, -lse2));
+                            const float ds = p * (dot2_packed_smem<D>(dor, vt, BM, r) - Delta);
+                            axpy2_smem<D>(acc2, ds, kt, BM, r);
                         }
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
@@ -521,20 +549,20 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                             const uint8_t *kt = sm + L::kDiagK + st * L::kRow;
                             const uint8_t *vt = sm + L::kDiagV + st * L::kRow;
                             const float p = tc::ex2(
-                                fmaf(dot_phys_gathered<D>(sm + L::kQ, kt, BM, r), c2, -lse2));
+                                fmaf(dot2_phys_gathered<D>(sm + L::kQ, kt, BM, r), c2, -lse2));
                             const float ds =
-                                p * (dot_phys_gathered<D>(sm + L::kDO, vt, BM, r) - Delta);
-                            axpy_smem<D>(acc, ds, kt, BM, r);
+                                p * (dot2_phys_gathered<D>(sm + L::kDO, vt, BM, r) - Delta);
+                            axpy2_smem<D>(acc2, ds, kt, BM, r);
                         }
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
                     }
                     tc::mbar_arrive(bar(L::bGroup));
                     if (!tc::mbar_wait(bar(L::bGroup), 0, abort, a.err, SA_DEVERR_TIMEOUT)) ok = false;
-                    unpermute_row<D>(acc, (float *)(sm + L::kDiagK) + (size_t)r * D, r);
+                    unpermute_row2<D>(acc2, (float *)(sm + L::kDiagK) + (size_t)r * D, r);
                 }
             }
-            tmem_store_row<D>(tDQ, acc);
+            tmem_store_row2<D>(tDQ, acc2);
             tc::tmem_st_wait();
         }
         tc::tc_fence_before();
@@ -845,34 +873,44 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         const float c2 = a.scale2;
         bool ok = tc::mbar_wait(bar(L::bKVFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
         if (ok) {
-            float adk[D], adv[D];
+            // diagonal blocks (fp32 pairs); lse and Delta of the linked query
+            // are loaded one block ahead
+            uint64_t adk2[D / 2], adv2[D / 2];
 #pragma unroll
-            for (int x = 0; x < D; ++x) adk[x] = adv[x] = 0.f;
+            for (int x = 0; x < D / 2; ++x) adk2[x] = adv2[x] = 0ull;
+            const size_t gbh = (size_t)bh * (size_t)T;
             if (DS > 0 && n_diag > 0) {
                 if (a.kind == 0) {
                     // distance links: query j + o, swizzled tiles read in logical order
+                    auto query_of = [&](int d) -> int64_t {
+                        if (!row_ok || d >= n_diag) return -1;
+                        const int64_t cand = j + a.offs[off_first + d];
+                        return cand < T ? cand : -1;
+                    };
+                    int64_t i_cur = query_of(0);
+                    float lse_cur = i_cur >= 0 ? a.lse[gbh + i_cur] : 0.f;
+                    float del_cur = i_cur >= 0 ? a.delta[gbh + i_cur] : 0.f;
                     for (int d = 0; d < n_diag; ++d) {
+                        const int64_t i_nxt = query_of(d + 1);
+                        const float lse_nxt = i_nxt >= 0 ? a.lse[gbh + i_nxt] : 0.f;
+                        const float del_nxt = i_nxt >= 0 ? a.delta[gbh + i_nxt] : 0.f;
                         const int st = d % DSX;
                         WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
-                        int64_t i = -1;
-                        if (row_ok) {
-                            const int64_t cand = j + a.offs[off_first + d];
-                            if (cand < T) i = cand;
-                        }
-                        if (i >= 0) {
-                            const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
-                            const float lse2 = a.lse[gi] * kLog2e, Dl = a.delta[gi];
+                        if (i_cur >= 0) {
                             const uint8_t *qt = sm + L::kDiagQ + st * L::kRow;
                             const uint8_t *dt = sm + L::kDiagDO + st * L::kRow;
-                            const float sdot = dot_smem_smem<D>(qt, sm + L::kK, BM, r);
-                            const float dpdot = dot_smem_smem<D>(dt, sm + L::kV, BM, r);
-                            const float p = tc::ex2(fmaf(sdot, c2, -lse2));
-                            const float ds = p * (dpdot - Dl);
-                            axpy_smem<D>(adv, p, dt, BM, r);
-                            axpy_smem<D>(adk, ds, qt, BM, r);
+                            const float sdot = dot2_smem_smem<D>(qt, sm + L::kK, BM, r);
+                            const float dpdot = dot2_smem_smem<D>(dt, sm + L::kV, BM, r);
+                            const float p = tc::ex2(fmaf(sdot, c2, -lse_cur * kLog2e));
+                            const float ds = p * (dpdot - del_cur);
+                            axpy2_smem<D>(adv2, p, dt, BM, r);
+                            axpy2_smem<D>(adk2, ds, qt, BM, r);
                         }
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                        i_cur = i_nxt;
+                        lse_cur = lse_nxt;
+                        del_cur = del_nxt;
                     }
                 } else {
                     // CSR gathers are unswizzled: the key's k and v rows read in
@@ -883,34 +921,46 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
                         nb = (T - j < W) ? T - j : W;
                         resid = a.rev_rowptr[j + 1] - rs - nb;
                     }
+                    // query of slot d (-1 if none): the list entry two slots
+                    // ahead, lse and Delta one slot ahead
+                    auto query_of = [&](int d) -> int64_t {
+                        return (row_ok && d < resid) ? (int64_t)a.rev_colidx[rs + nb + d] : -1;
+                    };
+                    int64_t i_cur = query_of(0), i_nxt = query_of(1);
+                    float lse_cur = i_cur >= 0 ? a.lse[gbh + i_cur] : 0.f;
+                    float del_cur = i_cur >= 0 ? a.delta[gbh + i_cur] : 0.f;
                     for (int d = 0; d < n_diag; ++d) {
+                        const int64_t i_n2 = query_of(d + 2);
+                        const float lse_nxt = i_nxt >= 0 ? a.lse[gbh + i_nxt] : 0.f;
+                        const float del_nxt = i_nxt >= 0 ? a.delta[gbh + i_nxt] : 0.f;
                         const int st = d % DSX;
                         WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
-                        const int64_t i = (row_ok && d < resid) ? a.rev_colidx[rs + nb + d] : -1;
-                        if (i >= 0) {
-                            const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
-                            const float lse2 = a.lse[gi] * kLog2e, Dl = a.delta[gi];
+                        if (i_cur >= 0) {
                             const uint8_t *qt = sm + L::kDiagQ + st * L::kRow;
                             const uint8_t *dt = sm + L::kDiagDO + st * L::kRow;
-                            const float sdot = dot_phys_gathered<D>(sm + L::kK, qt, BM, r);
-                            const float dpdot = dot_phys_gathered<D>(sm + L::kV, dt, BM, r);
-                            const float p = tc::ex2(fmaf(sdot, c2, -lse2));
-                            const float ds = p * (dpdot - Dl);
-                            axpy_smem<D>(adv, p, dt, BM, r);
-                            axpy_smem<D>(adk, ds, qt, BM, r);
+                            const float sdot = dot2_phys_gathered<D>(sm + L::kK, qt, BM, r);
+                            const float dpdot = dot2_phys_gathered<D>(sm + L::kV, dt, BM, r);
+                            const float p = tc::ex2(fmaf(sdot, c2, -lse_cur * kLog2e));
+                            const float ds = p * (dpdot - del_cur);
+                            axpy2_smem<D>(adv2, p, dt, BM, r);
+                            axpy2_smem<D>(adk2, ds, qt, BM, r);
                         }
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                        i_cur = i_nxt;
+                        i_nxt = i_n2;
+                        lse_cur = lse_nxt;
+                        del_cur = del_nxt;
                     }
                     tc::mbar_arrive(bar(L::bGroup));
                     if (!tc::mbar_wait(bar(L::bGroup), 0, abort, a.err, SA_DEVERR_TIMEOUT)) ok = false;
                     float *scr = (float *)(sm + L::kDiagQ);
-                    unpermute_row<D>(adv, scr + (size_t)r * D, r);
-                    unpermute_row<D>(adk, scr + (size_t)(BM + r) * D, r);
+                    unpermute_row2<D>(adv2, scr + (size_t)r * D, r);
+                    unpermute_row2<D>(adk2, scr + (size_t)(BM + r) * D, r);
                 }
             }
-            tmem_store_row<D>(tDV, adv);
-            tmem_store_row<D>(tDK, adk);
+            tmem_store_row2<D>(tDV, adv2);
+            tmem_store_row2<D>(tDK, adk2);
             tc::tmem_st_wait();
         }
         tc::tc_fence_before();

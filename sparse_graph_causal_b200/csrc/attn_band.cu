@@ -406,8 +406,12 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     pv_lt = lt;
                     ++gb;
                 }
+                // the tile's last P V goes now: its epilogue waits for it
+                if (ok && have_pv) {
+                    ok = do_pv();
+                    have_pv = false;
+                }
             }
-            if (ok && have_pv) do_pv();
         }
       }
     } else {

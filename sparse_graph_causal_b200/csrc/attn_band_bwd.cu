@@ -2,16 +2,17 @@
 // edges.  Probabilities are recomputed from lse; two kernels with disjoint
 // outputs and no float atomics, so results are bitwise reproducible:
 //
-//  band_bwd_dq   CTA = 128 queries [q0, q0+128).  Delta_i = dO_i . out_i is
+//  band_bwd_dq   tile = 128 queries [q0, q0+128).  Delta_i = dO_i . out_i is
 //                computed per row and written for the second kernel.  Key
-//                blocks of 64 from q0-W+1 (the forward's band in block
-//                coordinates u = 64 b + c, row r keeps r <= u <= r+W-1):
-//                S = Q K^T and dP = dO V^T in TMEM, dS = P (dP - Delta) in
-//                shared memory (bf16), dQ += dS K in TMEM.
-//  band_bwd_dkdv CTA = 128 keys [k0, k0+128).  Query blocks of 64 from k0
-//                (v = i - k0 = 64 b + c, key row r keeps r <= v <= r+W-1):
-//                S^T = K Q^T and dP^T = V dO^T in TMEM, P^T and dS^T in
-//                shared memory, dV += P^T dO and dK += dS^T Q in TMEM.
+//                blocks of BB from q0-W+1 (the forward's band in block
+//                coordinates u = BB b + c, row r keeps r <= u <= r+W-1):
+//                S = Q K^T and dP = dO V^T in TMEM, dS = P (dP - Delta)
+//                written back over S in TMEM (bf16), dQ += dS K in TMEM with
+//                dS read from TMEM by the MMA.
+//  band_bwd_dkdv tile = 128 keys [k0, k0+128).  Query blocks of BB from k0
+//                (v = i - k0 = BB b + c, key row r keeps r <= v <= r+W-1):
+//                S^T = K Q^T and dP^T = V dO^T in TMEM, P^T and dS^T written
+//                back over them (bf16), dV += P^T dO and dK += dS^T Q in TMEM.
 //
 // The other edges (2^k distance links or the non-window part of CSR lists)
 // are diagonal blocks as in the forward: row r of a block belongs to query
@@ -20,14 +21,15 @@
 // pairs) first and initialise the TMEM accumulators, which the band MMAs then
 // add to.
 //
-// Warp roles (256 threads): 0 TMA producer, 1 TMEM allocator + MMA issuer,
-// 2 diagonal-block producer (3 idle), 4-7 compute warpgroup (thread = owned
-// row = TMEM lane).  Waits are bounded as in the forward.
+// Both kernels are persistent and run NP (1 or 2) independent tile pipelines
+// per CTA, each with its own shared-memory rings, TMEM columns and barriers.
+// Warp roles: warp 2p is the TMA producer of pipeline p (its tile, the band
+// ring, the diagonal blocks), warp 2p+1 its MMA issuer (warp 1 also allocates
+// TMEM), warps 4+4p .. 7+4p its compute warpgroup (thread = owned row = TMEM
+// lane).  Waits are bounded as in the forward.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
-
-#include <type_traits>
 
 #include "sa_band.cuh"
 #include "tc_common.cuh"
@@ -35,12 +37,12 @@
 
 namespace {
 
-constexpr int BM = 128;  // rows a CTA owns
-constexpr int BB = 64;   // streamed block
+constexpr int BM = 128;  // rows a tile owns
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdArgs {
     int64_t T;
+    int64_t BH;
     int32_t W;
     int32_t kind;
     int32_t n_off;
@@ -49,7 +51,7 @@ struct BwdArgs {
     const int32_t *colidx;
     const int64_t *rev_rowptr;
     const int32_t *rev_colidx;
-    const __nv_bfloat16 *q, *k, *v, *o, *dout;
+    const __nv_bfloat16 *o;        // forward output (Delta)
     const float *lse;
     float *delta;
     __nv_bfloat16 *dq, *dk, *dv;
@@ -58,28 +60,22 @@ struct BwdArgs {
     int *err;
 };
 
-__host__ __device__ constexpr int align1k(int x) { return (x + 1023) & ~1023; }
+// Register budgets with two pipelines (384 threads launched at 168 each).
+struct BwdRegs {
+    static constexpr int producer = 72, compute = 216;
+    static_assert(128 * producer + 256 * compute <= 384 * 168, "register split");
+};
 
 // ---------------------------------------------------------------- helpers
 
-// Load a 128-row tile (two 64-row boxes per 64-column half) with a box-64 map.
-template <int D>
-__device__ __forceinline__ void tma_tile128(uint32_t dst, const void *map, int64_t row, int64_t bh,
-                                            uint32_t bar) {
+// ROWS rows of a [B*H, T, D] tensor (all D/64 column chunks) with a map whose
+// box is ROWS x 64; chunk x lands ROWS * 128 bytes after chunk x-1.
+template <int D, int ROWS>
+__device__ __forceinline__ void tma_rows(uint32_t dst, const void *map, int32_t row, int32_t bh,
+                                         uint32_t bar) {
 #pragma unroll
     for (int x = 0; x < D / 64; ++x)
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-            tc::tma_load_3d(dst + x * (BM * 128) + h * (64 * 128), map, x * 64,
-                            (int32_t)(row + 64 * h), (int32_t)bh, bar);
-}
-
-template <int D>
-__device__ __forceinline__ void tma_block64(uint32_t dst, const void *map, int64_t row, int64_t bh,
-                                            uint32_t bar) {
-#pragma unroll
-    for (int x = 0; x < D / 64; ++x)
-        tc::tma_load_3d(dst + x * (BB * 128), map, x * 64, (int32_t)row, (int32_t)bh, bar);
+        tc::tma_load_3d(dst + x * (ROWS * 128), map, x * 64, row, bh, bar);
 }
 
 // 16-byte chunk c of row r in a tile of `rows` rows (64-column halves stacked).
@@ -250,7 +246,15 @@ __device__ __forceinline__ void tmem_row_to_global(uint32_t taddr, float mul, __
     }
 }
 
-// Write 64 bf16 values (from fp32) as row r of a 128 x 64 K-major SW128 tile.
+// Pack n fp32 values as n/2 bf16 pairs (round to nearest even).
+template <int N>
+__device__ __forceinline__ void pack_bf16_row(const float *x, uint32_t *w) {
+#pragma unroll
+    for (int c = 0; c < N / 2; ++c) w[c] = tc::pack_bf16x2(x[2 * c], x[2 * c + 1]);
+}
+
+// 64 fp32 values as bf16, row r of a 128-row K-major tile with 128-byte
+// swizzle (the layout TMA writes), for a shared-memory MMA operand.
 __device__ __forceinline__ void store_row64_bf16(uint8_t *tile, int r, const float *x) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -263,6 +267,18 @@ __device__ __forceinline__ void store_row64_bf16(uint8_t *tile, int r, const flo
     }
 }
 
+// Tile t of a pipeline: (b*h slice, first row).
+struct TileId {
+    int32_t bh, r0;
+};
+__device__ __forceinline__ TileId tile_id(int64_t t, int64_t ntr) {
+    TileId id;
+    const int64_t bh = t / ntr;
+    id.bh = (int32_t)bh;
+    id.r0 = (int32_t)((t - bh * ntr) * BM);
+    return id;
+}
+
 #define WAIT_OR(bar_, par_, action_)                                                   \
     if (!tc::mbar_wait((bar_), (par_), abort, a.err, SA_DEVERR_TIMEOUT)) {              \
         action_;                                                                       \
@@ -270,185 +286,204 @@ __device__ __forceinline__ void store_row64_bf16(uint8_t *tile, int r, const flo
 
 // =================================================================== dQ
 
-template <int D, int BS, int DS, int PB>
+// PS = 0: dS (bf16) is written over S in TMEM and read from there by the dQ
+// MMA.  PS > 0: dS goes to PS shared-memory tiles instead, which frees the S
+// buffer as soon as the compute warps have read it (for one pipeline).
+template <int D, int NP, int BB, int SB, int BS, int DS, int PS>
 struct LayoutDQ {
     static constexpr int kRow = BM * D * 2, kBlk = BB * D * 2, kDSTile = BM * BB * 2;
-    static constexpr int kQ = 0, kDO = kRow, kK = 2 * kRow, kV = kK + BS * kBlk;
-    static constexpr int kDS = kV + BS * kBlk;
-    static constexpr int kDiagK = kDS + PB * kDSTile;
-    static constexpr int kDiagV = kDiagK + DS * kRow;
-    static constexpr int kBars = kDiagV + DS * kRow;
+    static constexpr int pQ = 0, pDO = kRow, pK = 2 * kRow, pV = pK + BS * kBlk;
+    static constexpr int pDK = pV + BS * kBlk, pDV = pDK + DS * kRow;
+    static constexpr int pDS = pDV + DS * kRow;
+    static constexpr int kPipe = pDS + PS * kDSTile;
+    static constexpr int kBars = NP * kPipe;
     static constexpr int DSX = DS > 0 ? DS : 1;
-    static constexpr int bQFull = 0, bBandFull = 1, bBandEmpty = bBandFull + BS;
-    static constexpr int bSFull = bBandEmpty + BS, bSFree = bSFull + 2;
-    static constexpr int bDSFull = bSFree + 2, bDSDone = bDSFull + PB;
-    static constexpr int bInit = bDSDone + PB, bDiagFull = bInit + 1;
-    static constexpr int bDiagEmpty = bDiagFull + DSX, bGroup = bDiagEmpty + DSX;
-    static constexpr int nBars = bGroup + 1;
-    static constexpr int kMisc = kBars + nBars * 8;
-    static constexpr int kAlloc = kMisc + 16 + 1024;
-    static constexpr uint32_t tS = 0, tDP = 128, tDQ = 256, kTmemCols = 512;
+    // barriers of one pipeline (S and dP share a buffer index sb; dS is
+    // written over S, so a buffer is free once its dQ MMA is done)
+    static constexpr int bQFull = 0, bQEmpty = 1;
+    static constexpr int bKVFull = 2, bKVEmpty = bKVFull + BS;
+    static constexpr int bSFull = bKVEmpty + BS, bSFree = bSFull + SB;
+    static constexpr int bDSFull = bSFree + SB, bDQDone = bDSFull + SB;
+    static constexpr int bInit = bDQDone + SB;
+    static constexpr int bDiagFull = bInit + 1, bDiagEmpty = bDiagFull + DSX;
+    static constexpr int bInfoFull = bDiagEmpty + DSX, bInfoEmpty = bInfoFull + 2;
+    static constexpr int bGroup = bInfoEmpty + 2;
+    static constexpr int bPSDone = bGroup + 1;              // dS tile consumed by its MMA
+    static constexpr int nBarsPipe = bPSDone + (PS > 0 ? PS : 1);
+    static constexpr int kMisc = kBars + NP * nBarsPipe * 8;  // tmem slot, abort, info[NP][2]
+    static constexpr int kTotal = kMisc + 8 + 8 * NP;
+    static constexpr int kAlloc = kTotal + 1024;
+    static_assert(PS == 0 || BB == 64, "shared-memory dS tiles are 64 keys wide");
+    // TMEM columns of pipeline p start at tPipe p: S buffers, dP buffers, dQ
+    static constexpr uint32_t tPipe = 512 / NP, tS = 0, tDP = SB * BB, tDQ = 2 * SB * BB;
+    static constexpr uint32_t kTmemCols = 512;
+    static_assert(2 * SB * BB + D <= (int)tPipe, "TMEM columns of a pipeline");
+    static_assert(kRow % 1024 == 0 && kBlk % 1024 == 0, "swizzle atoms");
 };
 
-template <int D, int BS, int DS, int PB>
-__global__ void __launch_bounds__(256, 1)
-band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                   const __grid_constant__ CUtensorMap tv,
-                   const __grid_constant__ CUtensorMap tdo,
+// Band geometry of a query tile: key blocks of BB from q0-W+1 up to the last key.
+template <int BB>
+struct DQBand {
+    int32_t kb0, b_first, n_band;
+    __device__ __forceinline__ DQBand(int32_t q0, int64_t T, int32_t W) {
+        kb0 = q0 - W + 1;
+        const int32_t last_key = (q0 + BM - 1 < T - 1) ? q0 + BM - 1 : (int32_t)(T - 1);
+        const int32_t nblk = (last_key - kb0) / BB + 1;
+        const int32_t need = W - 1 - q0;
+        b_first = need > 0 ? need / BB : 0;
+        n_band = nblk - b_first;
+    }
+};
+
+template <int D, int NP, int BB, int SB, int BS, int DS, int PS>
+__global__ void __launch_bounds__(128 + 128 * NP, 1)
+band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+                   const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                   const __grid_constant__ CUtensorMap tkd,
+                   const __grid_constant__ CUtensorMap tvd,
                    const __grid_constant__ CUtensorMap tkr,
                    const __grid_constant__ CUtensorMap tvr, const BwdArgs a) {
-    using L = LayoutDQ<D, BS, DS, PB>;
+    using L = LayoutDQ<D, NP, BB, SB, BS, DS, PS>;
     constexpr int DSX = L::DSX;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_u32(sm);
     uint32_t *tmem_slot = (uint32_t *)(sm + L::kMisc);
     volatile int *abort = (volatile int *)(sm + L::kMisc + 4);
-    int *n_diag_s = (int *)(sm + L::kMisc + 8);
-    auto bar = [&](int b) { return sbase + L::kBars + 8u * (uint32_t)b; };
+    auto bar = [&](int p, int b) {
+        return sbase + L::kBars + 8u * (uint32_t)(p * L::nBarsPipe + b);
+    };
+    auto wait = [&](int p, int b, uint32_t parity) {
+        return tc::mbar_wait(bar(p, b), parity, abort, a.err, SA_DEVERR_TIMEOUT);
+    };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t bh = blockIdx.y, q0 = (int64_t)blockIdx.x * BM, T = a.T;
+    const int64_t T = a.T;
     const int32_t W = a.W;
-    const int64_t kb0 = q0 - W + 1;
-    const int64_t last_key = (q0 + BM - 1 < T - 1) ? q0 + BM - 1 : T - 1;
-    const int64_t nblk = (last_key - kb0) / BB + 1;
-    const int64_t need0 = (int64_t)W - 1 - q0;
-    const int64_t b_first = need0 > 0 ? need0 / BB : 0;
-    const int n_band = (int)(nblk - b_first);
+    const int64_t ntr = (T + BM - 1) / BM, ntiles = ntr * a.BH;
+    const int64_t stride = (int64_t)gridDim.x * NP;
 
     if (tid == 0) {
-        tc::mbar_init(bar(L::bQFull), 1);
-        for (int s = 0; s < BS; ++s) {
-            tc::mbar_init(bar(L::bBandFull + s), 1);
-            tc::mbar_init(bar(L::bBandEmpty + s), 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            tc::mbar_init(bar(L::bSFull + s), 1);
-            tc::mbar_init(bar(L::bSFree + s), 4);
-        }
-        for (int s = 0; s < PB; ++s) {
-            tc::mbar_init(bar(L::bDSFull + s), 4);
-            tc::mbar_init(bar(L::bDSDone + s), 1);
-        }
-        tc::mbar_init(bar(L::bInit), 4);
-        tc::mbar_init(bar(L::bGroup), 128);  // 128-thread compute barrier (bounded)
-        for (int s = 0; s < DSX; ++s) {
-            tc::mbar_init(bar(L::bDiagFull + s), 1);
-            tc::mbar_init(bar(L::bDiagEmpty + s), 4);
+        for (int p = 0; p < NP; ++p) {
+            tc::mbar_init(bar(p, L::bQFull), 1);
+            tc::mbar_init(bar(p, L::bQEmpty), 5);  // last S/dP MMA commit + 4 compute warps
+            for (int s = 0; s < BS; ++s) {
+                tc::mbar_init(bar(p, L::bKVFull + s), 1);
+                tc::mbar_init(bar(p, L::bKVEmpty + s), 1);
+            }
+            for (int s = 0; s < SB; ++s) {
+                tc::mbar_init(bar(p, L::bSFull + s), 1);
+                // freed by the dQ MMA (dS in TMEM) or by the compute warps
+                tc::mbar_init(bar(p, L::bSFree + s), PS > 0 ? 4 : 1);
+                tc::mbar_init(bar(p, L::bDSFull + s), 4);
+                tc::mbar_init(bar(p, L::bDQDone + s), 1);
+            }
+            tc::mbar_init(bar(p, L::bInit), 4);
+            for (int s = 0; s < DSX; ++s) {
+                tc::mbar_init(bar(p, L::bDiagFull + s), 1);
+                tc::mbar_init(bar(p, L::bDiagEmpty + s), 4);
+            }
+            for (int s = 0; s < 2; ++s) {
+                tc::mbar_init(bar(p, L::bInfoFull + s), 1);
+                tc::mbar_init(bar(p, L::bInfoEmpty + s), 4);
+            }
+            tc::mbar_init(bar(p, L::bGroup), 128);
+            for (int s = 0; s < PS; ++s) tc::mbar_init(bar(p, L::bPSDone + s), 1);
         }
         *abort = 0;
-        *n_diag_s = 0;
         tc::fence_barrier_init();
     }
     if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), L::kTmemCols);
-    __syncthreads();
-    if (DS > 0 && warp >= 4) {
-        int nd = 0;
-        const int64_t i = q0 + (tid - 128);
-        if (a.kind == 0) {
-            for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last_key) ? 1 : 0;
-        } else if (i < T) {
-            const int64_t deg = a.rowptr[i + 1] - a.rowptr[i];
-            nd = (int)(deg - ((i + 1 < W) ? i + 1 : W));
-        }
-        atomicMax(n_diag_s, nd);
-    }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_diag = DS > 0 ? *n_diag_s : 0;
 
-    if (warp == 0) {
-        if (lane == 0) {
-            tc::mbar_arrive_expect_tx(bar(L::bQFull), 2 * L::kRow);
-            tma_tile128<D>(sbase + L::kQ, &tq, q0, bh, bar(L::bQFull));
-            tma_tile128<D>(sbase + L::kDO, &tdo, q0, bh, bar(L::bQFull));
-            for (int bl = 0; bl < n_band; ++bl) {
-                const int st = bl % BS, use = bl / BS;
-                if (use > 0) WAIT_OR(bar(L::bBandEmpty + st), (use - 1) & 1, break);
-                const int64_t krow = kb0 + (b_first + bl) * BB;
-                tc::mbar_arrive_expect_tx(bar(L::bBandFull + st), 2 * L::kBlk);
-                tma_block64<D>(sbase + L::kK + st * L::kBlk, &tk, krow, bh, bar(L::bBandFull + st));
-                tma_block64<D>(sbase + L::kV + st * L::kBlk, &tv, krow, bh, bar(L::bBandFull + st));
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idS = tc::idesc_bf16(BM, BB, false, false);
-            const uint32_t idQ = tc::idesc_bf16(BM, D, false, true);
-            bool ok = tc::mbar_wait(bar(L::bQFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
-            auto issue = [&](int bl) -> bool {
-                const int st = bl % BS, sb = bl & 1;
-                if (!tc::mbar_wait(bar(L::bBandFull + st), (bl / BS) & 1, abort, a.err,
-                                   SA_DEVERR_TIMEOUT))
-                    return false;
-                if (bl >= 2 && !tc::mbar_wait(bar(L::bSFree + sb), ((bl >> 1) - 1) & 1, abort,
-                                              a.err, SA_DEVERR_TIMEOUT))
-                    return false;
-                tc::tc_fence_after();
-                const uint32_t ka = sbase + L::kK + st * L::kBlk, va = sbase + L::kV + st * L::kBlk;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t offr = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                    const uint32_t offb = (kk >> 2) * (BB * 128) + (kk & 3) * 32;
-                    tc::mma_bf16_ss(tmem + L::tS + sb * BB,
-                                    tc::sdesc_sw128(sbase + L::kQ + offr, 16, 1024),
-                                    tc::sdesc_sw128(ka + offb, 16, 1024), idS, kk > 0);
-                    tc::mma_bf16_ss(tmem + L::tDP + sb * BB,
-                                    tc::sdesc_sw128(sbase + L::kDO + offr, 16, 1024),
-                                    tc::sdesc_sw128(va + offb, 16, 1024), idS, kk > 0);
-                }
-                tc::mma_commit(bar(L::bSFull + sb));
-                return true;
-            };
-            if (ok && n_band > 0) ok = issue(0);
-            for (int bl = 0; ok && bl < n_band; ++bl) {
-                if (BS >= 2 && bl + 1 < n_band && !issue(bl + 1)) break;
-                const int pb = bl % PB, st = bl % BS;
-                if (bl == 0) WAIT_OR(bar(L::bInit), 0, break);
-                WAIT_OR(bar(L::bDSFull + pb), (bl / PB) & 1, break);
-                tc::tc_fence_after();
-                const uint32_t dsa = sbase + L::kDS + pb * L::kDSTile;
-                const uint32_t ka = sbase + L::kK + st * L::kBlk;
-#pragma unroll
-                for (int kk = 0; kk < BB / 16; ++kk)
-                    tc::mma_bf16_ss(tmem + L::tDQ, tc::sdesc_sw128(dsa + kk * 32, 16, 1024),
-                                    tc::sdesc_sw128(ka + kk * 16 * 128, BB * 128, 1024), idQ, 1u);
-                tc::mma_commit(bar(L::bBandEmpty + st));
-                tc::mma_commit(bar(L::bDSDone + pb));
-                if (BS == 1 && bl + 1 < n_band && !issue(bl + 1)) break;
-            }
-        }
-    } else if (warp == 2 || warp == 3) {
-        // warp 2 stages the diagonal blocks; warp 3 has no role
-        if (warp == 2 && DS > 0) {
+    if (warp < 4) {
+        if (NP == 2) tc::regs_dec<BwdRegs::producer>();
+      if ((warp >> 1) < NP && (warp & 1) == 0) {
+        // ---------------- producer of pipeline p: diagonal-block count, Q and
+        // dO of the tile, the first band K/V blocks, the diagonal blocks, the rest
+        const int p = warp >> 1;
+        const uint32_t pb = sbase + (uint32_t)(p * L::kPipe);
+        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
+        uint32_t kvc = 0, dc = 0;
+        bool ok = true;
+        int64_t lt = 0;
+        for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
+            const TileId id = tile_id(t, ntr);
+            const int32_t q0 = id.r0, bh = id.bh;
+            const DQBand<BB> g(q0, T, W);
+            const int64_t last = (q0 + BM - 1 < T - 1) ? q0 + BM - 1 : T - 1;
             // CSR: lane l owns rows 4l .. 4l+3 (list start, residual count, next key)
             int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
             int32_t cj[4] = {0, 0, 0, 0};
-            if (a.kind == 1) {
+            int nd = 0;
+            if (DS > 0) {
+                if (a.kind == 0) {
+                    for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last) ? 1 : 0;
+                } else {
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int64_t i = q0 + 4 * lane + h;
-                    if (i < T) {
-                        cstart[h] = a.rowptr[i];
-                        cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
-                        if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
+                    for (int h = 0; h < 4; ++h) {
+                        const int64_t i = q0 + 4 * lane + h;
+                        if (i < T) {
+                            cstart[h] = a.rowptr[i];
+                            cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
+                            if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
+                            nd = nd > (int)cres[h] ? nd : (int)cres[h];
+                        }
+                    }
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const int x = __shfl_xor_sync(0xffffffffu, nd, o);
+                        nd = nd > x ? nd : x;
                     }
                 }
             }
-            for (int d = 0; d < n_diag; ++d) {
-                const int st = d % DSX, use = d / DSX;
-                const uint32_t kdst = sbase + L::kDiagK + st * L::kRow;
-                const uint32_t vdst = sbase + L::kDiagV + st * L::kRow;
-                if (use > 0) WAIT_OR(bar(L::bDiagEmpty + st), (use - 1) & 1, break);
-                if (lane == 0) tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kRow);
+            const int slot = (int)(lt & 1);
+            if (lt >= 2 && !wait(p, L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1))) break;
+            if (lane == 0) {
+                info[slot] = nd;
+                tc::mbar_arrive(bar(p, L::bInfoFull + slot));
+            }
+            auto load_kv = [&](int bl) -> bool {
+                const int st = (int)(kvc % BS);
+                const uint32_t use = kvc / BS;
+                if (use > 0 && !wait(p, L::bKVEmpty + st, (use - 1) & 1)) return false;
+                const int32_t krow = g.kb0 + (g.b_first + bl) * BB;
+                tc::mbar_arrive_expect_tx(bar(p, L::bKVFull + st), 2 * L::kBlk);
+                tma_rows<D, BB>(pb + L::pK + st * L::kBlk, &tk, krow, bh, bar(p, L::bKVFull + st));
+                tma_rows<D, BB>(pb + L::pV + st * L::kBlk, &tv, krow, bh, bar(p, L::bKVFull + st));
+                ++kvc;
+                return true;
+            };
+            const int n_pre = g.n_band < BS ? g.n_band : BS;
+            int okl = 1;
+            if (lane == 0) {
+                if (lt >= 1 && !wait(p, L::bQEmpty, (uint32_t)((lt - 1) & 1))) okl = 0;
+                if (okl) {
+                    tc::mbar_arrive_expect_tx(bar(p, L::bQFull), 2 * L::kRow);
+                    tma_rows<D, BM>(pb + L::pQ, &tq, q0, bh, bar(p, L::bQFull));
+                    tma_rows<D, BM>(pb + L::pDO, &tdo, q0, bh, bar(p, L::bQFull));
+                }
+                for (int bl = 0; okl && bl < n_pre; ++bl)
+                    if (!load_kv(bl)) okl = 0;
+            }
+            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+            for (int d = 0; ok && d < nd; ++d) {
+                const int st = (int)(dc % DSX);
+                const uint32_t use = dc / DSX;
+                const uint32_t kdst = pb + L::pDK + st * L::kRow;
+                const uint32_t vdst = pb + L::pDV + st * L::kRow;
+                if (use > 0 && !wait(p, L::bDiagEmpty + st, (use - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar(p, L::bDiagFull + st), 2 * L::kRow);
                 if (a.kind == 0) {
                     if (lane == 0) {
-                        const int64_t krow = q0 - a.offs[a.n_off - n_diag + d];
-                        tma_tile128<D>(kdst, &tk, krow, bh, bar(L::bDiagFull + st));
-                        tma_tile128<D>(vdst, &tv, krow, bh, bar(L::bDiagFull + st));
+                        const int32_t krow = (int32_t)(q0 - a.offs[a.n_off - nd + d]);
+                        tma_rows<D, BM>(kdst, &tkd, krow, bh, bar(p, L::bDiagFull + st));
+                        tma_rows<D, BM>(vdst, &tvd, krow, bh, bar(p, L::bDiagFull + st));
                     }
                 } else {
                     int32_t rr[4];
@@ -456,45 +491,163 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                     for (int h = 0; h < 4; ++h) {
                         const int64_t i = q0 + 4 * lane + h;
                         const int64_t j = d < cres[h] ? (int64_t)cj[h] : (i < T ? i : 0);
-                        rr[h] = (int32_t)(bh * T + j);
+                        rr[h] = (int32_t)((int64_t)bh * T + j);
                     }
 #pragma unroll
                     for (int x = 0; x < D / 64; ++x) {
                         const uint32_t off = x * (BM * 128) + 4 * lane * 128;
                         tc::tma_gather4(kdst + off, &tkr, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                        bar(L::bDiagFull + st));
+                                        bar(p, L::bDiagFull + st));
                         tc::tma_gather4(vdst + off, &tvr, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                        bar(L::bDiagFull + st));
+                                        bar(p, L::bDiagFull + st));
                     }
 #pragma unroll
                     for (int h = 0; h < 4; ++h)
                         if (d + 1 < cres[h]) cj[h] = a.colidx[cstart[h] + d + 1];
                 }
+                ++dc;
+            }
+            if (!ok) break;
+            if (lane == 0)
+                for (int bl = n_pre; okl && bl < g.n_band; ++bl)
+                    if (!load_kv(bl)) okl = 0;
+            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+        }
+      } else if ((warp >> 1) < NP) {
+        // ---------------- MMA issuer of pipeline p: S and dP of block g, then
+        // dQ += dS K of block g-1
+        const int p = warp >> 1;
+        const uint32_t pb = sbase + (uint32_t)(p * L::kPipe);
+        const uint32_t tp = tmem + p * L::tPipe;
+        if (lane == 0) {
+            const uint32_t idS = tc::idesc_bf16(BM, BB, false, false);
+            const uint32_t idQ = tc::idesc_bf16(BM, D, false, true);
+            uint32_t gb = 0;  // band blocks issued (all tiles)
+            bool have = false, first = false, ok = true;
+            uint32_t pg = 0;
+            int64_t plt = 0;
+            auto do_dq = [&]() -> bool {
+                const int sb = (int)(pg % SB), st = (int)(pg % BS);
+                if (first && !wait(p, L::bInit, (uint32_t)(plt & 1))) return false;
+                if (!wait(p, L::bDSFull + sb, (pg / SB) & 1)) return false;
+                tc::tc_fence_after();
+                const uint32_t ka = pb + L::pK + st * L::kBlk;
+                if constexpr (PS > 0) {
+                    const int ps = (int)(pg % PS);
+                    const uint32_t dsa = pb + L::pDS + ps * L::kDSTile;
+#pragma unroll
+                    for (int kk = 0; kk < BB / 16; ++kk)
+                        tc::mma_bf16_ss(tp + L::tDQ, tc::sdesc_sw128(dsa + kk * 32, 16, 1024),
+                                        tc::sdesc_sw128(ka + kk * 16 * 128, BB * 128, 1024), idQ,
+                                        1u);
+                    tc::mma_commit(bar(p, L::bKVEmpty + st));
+                    tc::mma_commit(bar(p, L::bPSDone + ps));
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < BB / 16; ++kk)
+                        tc::mma_bf16_ts(tp + L::tDQ, tp + L::tS + sb * BB + kk * 8,
+                                        tc::sdesc_sw128(ka + kk * 16 * 128, BB * 128, 1024), idQ,
+                                        1u);
+                    tc::mma_commit(bar(p, L::bKVEmpty + st));
+                    tc::mma_commit(bar(p, L::bSFree + sb));
+                }
+                tc::mma_commit(bar(p, L::bDQDone + sb));
+                return true;
+            };
+            int64_t lt = 0;
+            for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
+                const TileId id = tile_id(t, ntr);
+                const DQBand<BB> g(id.r0, T, W);
+                if (!wait(p, L::bQFull, (uint32_t)(lt & 1))) break;
+                const uint32_t qa = pb + L::pQ, da = pb + L::pDO;
+                for (int bl = 0; bl < g.n_band; ++bl) {
+                    const int st = (int)(gb % BS), sb = (int)(gb % SB);
+                    // one S buffer: dQ of the previous block frees it first
+                    if (SB == 1 && have) {
+                        if (!do_dq()) {
+                            ok = false;
+                            break;
+                        }
+                        have = false;
+                    }
+                    if (!wait(p, L::bKVFull + st, (gb / BS) & 1) ||
+                        (gb >= SB && !wait(p, L::bSFree + sb, ((gb / SB) - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const uint32_t ka = pb + L::pK + st * L::kBlk, va = pb + L::pV + st * L::kBlk;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t offr = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        const uint32_t offb = (kk >> 2) * (BB * 128) + (kk & 3) * 32;
+                        tc::mma_bf16_ss(tp + L::tS + sb * BB, tc::sdesc_sw128(qa + offr, 16, 1024),
+                                        tc::sdesc_sw128(ka + offb, 16, 1024), idS, kk > 0);
+                        tc::mma_bf16_ss(tp + L::tDP + sb * BB,
+                                        tc::sdesc_sw128(da + offr, 16, 1024),
+                                        tc::sdesc_sw128(va + offb, 16, 1024), idS, kk > 0);
+                    }
+                    tc::mma_commit(bar(p, L::bSFull + sb));
+                    if (bl == g.n_band - 1) tc::mma_commit(bar(p, L::bQEmpty));
+                    // dS of this block is computed while dQ of the previous one runs
+                    if (SB > 1 && have && !do_dq()) {
+                        ok = false;
+                        break;
+                    }
+                    have = true;
+                    pg = gb;
+                    first = (bl == 0);
+                    plt = lt;
+                    ++gb;
+                }
+                // the tile's last dQ MMA goes now: its epilogue waits for it
+                if (ok && have) {
+                    ok = do_dq();
+                    have = false;
+                }
             }
         }
-    } else if (warp >= 4 && warp < 8) {
-        // compute warpgroup: thread r = owned row r = TMEM lane r
-        const int r = tid - 128;
-        const int64_t i = q0 + r;
-        const bool row_ok = i < T;
-        const size_t grow = (size_t)bh * (size_t)T + (size_t)i;
-        const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
-        const uint32_t tS = tmem + lane_off + L::tS, tDP = tmem + lane_off + L::tDP;
-        const uint32_t tDQ = tmem + lane_off + L::tDQ;
+      }
+    } else {
+        // ---------------- compute warpgroup of pipeline p: thread r = query
+        // row r = TMEM lane r
+        if (NP == 2) tc::regs_inc<BwdRegs::compute>();
+        const int p = (warp - 4) >> 2;
+        const int r = tid - 128 - 128 * p;
+        uint8_t *pm = sm + p * L::kPipe;
+        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
+        const uint32_t lane_off = (uint32_t)(((warp - 4) & 3) * 32) << 16;
+        const uint32_t tS = tmem + p * L::tPipe + lane_off + L::tS;
+        const uint32_t tDP = tmem + p * L::tPipe + lane_off + L::tDP;
+        const uint32_t tDQ = tmem + p * L::tPipe + lane_off + L::tDQ;
         const float c2 = a.scale2;
-        const float lse2 = row_ok ? a.lse[grow] * kLog2e : 0.f;
-        // the out row for Delta is fetched while Q and dO arrive
-        uint4 orow4[D / 8];
+        uint32_t dc = 0, gb = 0, group_uses = 0;
+        bool ok = true;
+        int64_t lt = 0;
+        for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
+            const TileId id = tile_id(t, ntr);
+            const int32_t q0 = id.r0, bh = id.bh;
+            const DQBand<BB> g(q0, T, W);
+            const int64_t i = q0 + r;
+            const bool row_ok = i < T;
+            const size_t grow = (size_t)bh * (size_t)T + (size_t)i;
+            const int slot = (int)(lt & 1);
+            if (!wait(p, L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1))) break;
+            const int nd = info[slot];
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
+            const float lse2 = row_ok ? a.lse[grow] * kLog2e : 0.f;
+            // the out row for Delta is fetched while Q and dO arrive
+            uint4 orow4[D / 8];
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-            orow4[c] = row_ok ? __ldg((const uint4 *)(a.o + grow * D) + c) : make_uint4(0, 0, 0, 0);
-        bool ok = tc::mbar_wait(bar(L::bQFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
-        float Delta = 0.f;
-        if (ok) {
+            for (int c = 0; c < D / 8; ++c)
+                orow4[c] = row_ok ? __ldg((const uint4 *)(a.o + grow * D) + c) : make_uint4(0, 0, 0, 0);
+            if (!wait(p, L::bQFull, (uint32_t)(lt & 1))) break;
             // Delta_i = dO_i . out_i
-            uint32_t dor[D / 2];
-            load_row_packed<D>(sm + L::kDO, BM, r, dor);
-            if (row_ok) {
+            float Delta = 0.f;
+            {
+                uint32_t dor[D / 2];
+                load_row_packed<D>(pm + L::pDO, BM, r, dor);
                 uint64_t d0 = 0ull, d1 = 0ull, d2 = 0ull, d3 = 0ull;
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
@@ -504,125 +657,164 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                     d3 = tc::ffma2(tc::bf2_to_f2(dor[4 * c + 3]), tc::bf2_to_f2(orow4[c].w), d3);
                 }
                 Delta = sum4_f2(d0, d1, d2, d3);
-                a.delta[grow] = Delta;
             }
+            if (row_ok) a.delta[grow] = Delta;
             // diagonal blocks (fp32 pairs)
             uint64_t acc2[D / 2];
 #pragma unroll
             for (int x = 0; x < D / 2; ++x) acc2[x] = 0ull;
-            if (DS > 0 && n_diag > 0) {
+            if (DS > 0 && nd > 0) {
                 if (a.kind == 0) {
                     // distance links: swizzled tiles, q in logical chunk order
                     uint64_t q2[D / 2];
 #pragma unroll
                     for (int c = 0; c < D / 8; ++c) {
-                        const uint4 x = *(const uint4 *)(sm + L::kQ + tile_off(BM, r, c));
+                        const uint4 x = *(const uint4 *)(pm + L::pQ + tile_off(BM, r, c));
                         q2[4 * c] = tc::bf2_to_f2(x.x);
                         q2[4 * c + 1] = tc::bf2_to_f2(x.y);
                         q2[4 * c + 2] = tc::bf2_to_f2(x.z);
                         q2[4 * c + 3] = tc::bf2_to_f2(x.w);
                     }
-                    for (int d = 0; d < n_diag; ++d) {
-                        const int st = d % DSX;
-                        WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
-                        if (row_ok && i >= a.offs[a.n_off - n_diag + d]) {
-                            const uint8_t *kt = sm + L::kDiagK + st * L::kRow;
-                            const uint8_t *vt = sm + L::kDiagV + st * L::kRow;
-                            const float p =
+                    for (int d = 0; d < nd; ++d) {
+                        const int st = (int)(dc % DSX);
+                        if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        if (row_ok && i >= a.offs[a.n_off - nd + d]) {
+                            const uint8_t *kt = pm + L::pDK + st * L::kRow;
+                            const uint8_t *vt = pm + L::pDV + st * L::kRow;
+                            const float pr =
                                 tc::ex2(fmaf(dot2_reg_smem<D>(q2, kt, BM, r), c2, -lse2));
-                            const float ds = p * (dot2_packed_smem<D>(dor, vt, BM, r) - Delta);
+                            const float ds =
+                                pr * (dot2_smem_smem<D>(pm + L::pDO, vt, BM, r) - Delta);
                             axpy2_smem<D>(acc2, ds, kt, BM, r);
                         }
                         __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                        if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
+                        ++dc;
                     }
                 } else {
                     // CSR gathers are unswizzled: pair them with the physical
-                    // chunk order of the swizzled q and dO rows (see the forward)
+                    // chunk order of the swizzled q and dO rows (as in the forward)
                     int64_t resid = 0;
                     if (row_ok)
                         resid = (a.rowptr[i + 1] - a.rowptr[i]) - ((i + 1 < W) ? i + 1 : W);
-                    for (int d = 0; d < n_diag; ++d) {
-                        const int st = d % DSX;
-                        WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
+                    for (int d = 0; d < nd; ++d) {
+                        const int st = (int)(dc % DSX);
+                        if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
+                            ok = false;
+                            break;
+                        }
                         if (row_ok && d < resid) {
-                            const uint8_t *kt = sm + L::kDiagK + st * L::kRow;
-                            const uint8_t *vt = sm + L::kDiagV + st * L::kRow;
-                            const float p = tc::ex2(
-                                fmaf(dot2_phys_gathered<D>(sm + L::kQ, kt, BM, r), c2, -lse2));
+                            const uint8_t *kt = pm + L::pDK + st * L::kRow;
+                            const uint8_t *vt = pm + L::pDV + st * L::kRow;
+                            const float pr = tc::ex2(
+                                fmaf(dot2_phys_gathered<D>(pm + L::pQ, kt, BM, r), c2, -lse2));
                             const float ds =
-                                p * (dot2_phys_gathered<D>(sm + L::kDO, vt, BM, r) - Delta);
+                                pr * (dot2_phys_gathered<D>(pm + L::pDO, vt, BM, r) - Delta);
                             axpy2_smem<D>(acc2, ds, kt, BM, r);
                         }
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
+                        if (d < nd - 1) {  // the last stage is released after the unpermute
+                            __syncwarp();
+                            if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
+                        }
+                        ++dc;
                     }
-                    tc::mbar_arrive(bar(L::bGroup));
-                    if (!tc::mbar_wait(bar(L::bGroup), 0, abort, a.err, SA_DEVERR_TIMEOUT)) ok = false;
-                    unpermute_row2<D>(acc2, (float *)(sm + L::kDiagK) + (size_t)r * D, r);
+                    if (ok) {
+                        // once every row is done with the last stage, thread r
+                        // uses D floats of it (rows < 64 in its K half, the
+                        // others in its V half) to restore the logical order
+                        const int st = (int)((dc - 1) % DSX);
+                        tc::mbar_arrive(bar(p, L::bGroup));
+                        if (!wait(p, L::bGroup, group_uses & 1)) ok = false;
+                        ++group_uses;
+                        float *scr = (float *)(pm + (r < 64 ? L::pDK : L::pDV) + st * L::kRow) +
+                                     (size_t)(r & 63) * D;
+                        unpermute_row2<D>(acc2, scr, r);
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
+                    }
                 }
             }
+            if (!ok) break;
+            // this warp is done reading Q and dO of the tile
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(p, L::bQEmpty));
             tmem_store_row2<D>(tDQ, acc2);
             tc::tmem_st_wait();
-        }
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(bar(L::bInit));
-
-        // band blocks
-        for (int bl = 0; ok && bl < n_band; ++bl) {
-            const int sb = bl & 1, pb = bl % PB;
-            const int64_t u0 = (b_first + bl) * BB;
-            WAIT_OR(bar(L::bSFull + sb), (bl >> 1) & 1, ok = false; break);
-            tc::tc_fence_after();
-            float s[BB], dp[BB];
-            tc::tmem_ld32(tS + sb * BB, (uint32_t *)s);
-            tc::tmem_ld32(tS + sb * BB + 32, (uint32_t *)(s + 32));
-            tc::tmem_ld32(tDP + sb * BB, (uint32_t *)dp);
-            tc::tmem_ld32(tDP + sb * BB + 32, (uint32_t *)(dp + 32));
-            tc::tmem_ld_wait();
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(L::bSFree + sb));
-            const bool need_mask = (u0 < BM - 1) || (u0 + BB - 1 > (int64_t)W - 1) ||
-                                   (u0 + q0 < (int64_t)W - 1);
-            if (need_mask) {
-                // keep columns [c_lo, c_hi]: r <= u <= r+W-1 and key >= 0
-                const int64_t lo = ((int64_t)r > (int64_t)W - 1 - q0) ? r : (int64_t)W - 1 - q0;
-                const int64_t hi = (int64_t)r + W - 1;
-                const int c_lo = (int)(lo - u0 < 0 ? 0 : (lo - u0 > BB ? BB : lo - u0));
-                const int c_hi = (int)(hi - u0 > BB - 1 ? BB - 1 : (hi - u0 < -1 ? -1 : hi - u0));
-                // 16-column chunks outside every kept range of this warp: dS = 0
-#pragma unroll
-                for (int c16 = 0; c16 < BB / 16; ++c16) {
-                    if (__any_sync(0xffffffffu, c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16)) {
-#pragma unroll
-                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
-                            const float p =
-                                (c >= c_lo && c <= c_hi) ? tc::ex2(fmaf(s[c], c2, -lse2)) : 0.f;
-                            s[c] = p * (dp[c] - Delta);  // dS
-                        }
-                    } else {
-#pragma unroll
-                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) s[c] = 0.f;
-                    }
+            if (lane == 0) tc::mbar_arrive(bar(p, L::bInit));
+
+            // band blocks: dS = P (dP - Delta), bf16 over S
+            uint32_t gb_last = gb;
+            for (int bl = 0; ok && bl < g.n_band; ++bl, ++gb) {
+                const int sb = (int)(gb % SB);
+                const int32_t u0 = (g.b_first + bl) * BB;
+                gb_last = gb;
+                if (!wait(p, L::bSFull + sb, (gb / SB) & 1)) {
+                    ok = false;
+                    break;
                 }
-            } else {
+                tc::tc_fence_after();
+                float s[BB], dp[BB];
+                tc::tmem_ld_n<BB>(tS + sb * BB, (uint32_t *)s);
+                tc::tmem_ld_n<BB>(tDP + sb * BB, (uint32_t *)dp);
+                tc::tmem_ld_wait();
+                if (PS > 0) {  // S and dP are in registers: the buffer is free
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(p, L::bSFree + sb));
+                }
+                const bool need_mask =
+                    (u0 < BM - 1) || (u0 + BB - 1 > W - 1) || (u0 + q0 < W - 1);
+                if (need_mask) {
+                    // keep columns [c_lo, c_hi]: r <= u <= r+W-1 and key >= 0
+                    const int32_t lo = (r > W - 1 - q0) ? r : W - 1 - q0;
+                    const int32_t hi = r + W - 1;
+                    const int c_lo = lo - u0 < 0 ? 0 : (lo - u0 > BB ? BB : lo - u0);
+                    const int c_hi = hi - u0 > BB - 1 ? BB - 1 : (hi - u0 < -1 ? -1 : hi - u0);
+                    // 16-column chunks outside every kept range of this warp: dS = 0
 #pragma unroll
-                for (int c = 0; c < BB; ++c) s[c] = tc::ex2(fmaf(s[c], c2, -lse2)) * (dp[c] - Delta);
+                    for (int c16 = 0; c16 < BB / 16; ++c16) {
+                        if (__any_sync(0xffffffffu, c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16)) {
+#pragma unroll
+                            for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
+                                const float pr =
+                                    (c >= c_lo && c <= c_hi) ? tc::ex2(fmaf(s[c], c2, -lse2)) : 0.f;
+                                s[c] = pr * (dp[c] - Delta);
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 16 * c16; c < 16 * c16 + 16; ++c) s[c] = 0.f;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BB; ++c)
+                        s[c] = tc::ex2(fmaf(s[c], c2, -lse2)) * (dp[c] - Delta);
+                }
+                if constexpr (PS > 0) {
+                    const int ps = (int)(gb % PS);
+                    if (gb >= PS && !wait(p, L::bPSDone + ps, ((gb / PS) - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    store_row64_bf16(pm + L::pDS + ps * L::kDSTile, r, s);
+                    tc::fence_proxy_async_smem();
+                } else {
+                    uint32_t w[BB / 2];
+                    pack_bf16_row<BB>(s, w);
+                    tc::tmem_st_n<BB / 2>(tS + sb * BB, w);
+                    tc::tmem_st_wait();
+                    tc::tc_fence_before();
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(p, L::bDSFull + sb));
             }
-            if (bl >= PB) WAIT_OR(bar(L::bDSDone + pb), ((bl - PB) / PB) & 1, ok = false; break);
-            store_row64_bf16(sm + L::kDS + pb * L::kDSTile, r, s);
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(L::bDSFull + pb));
-        }
-        if (ok && n_band > 0) {
-            const int lb = n_band - 1;
-            ok = tc::mbar_wait(bar(L::bDSDone + lb % PB), (lb / PB) & 1, abort, a.err,
-                               SA_DEVERR_TIMEOUT);
-        }
-        if (ok) {
+            if (!ok) break;
+            if (!wait(p, L::bDQDone + (int)(gb_last % SB), (gb_last / SB) & 1)) break;
             tc::tc_fence_after();
             tmem_row_to_global<D>(tDQ, a.scale, a.dq + grow * D, row_ok);
         }
@@ -637,207 +829,221 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
 
 // ================================================================= dK/dV
 
-template <int D, int BS, int DS, int PB>
+// PS = 0: P^T and dS^T (bf16) are written over S^T and dP^T in TMEM.  PS > 0:
+// they go to PS pairs of shared-memory tiles, which frees the S^T/dP^T buffer
+// as soon as the compute warps have read it (for one pipeline).
+template <int D, int NP, int BB, int SB, int BS, int DS, int PS>
 struct LayoutDKV {
     static constexpr int kRow = BM * D * 2, kBlk = BB * D * 2, kPTile = BM * BB * 2;
-    static constexpr int kK = 0, kV = kRow, kQ = 2 * kRow, kDO = kQ + BS * kBlk;
-    static constexpr int kLse = kDO + BS * kBlk, kDel = kLse + BS * 256;
-    static constexpr int kP = align1k(kDel + BS * 256), kDS = kP + PB * kPTile;
-    static constexpr int kDiagQ = kDS + PB * kPTile, kDiagDO = kDiagQ + DS * kRow;
-    static constexpr int kBars = kDiagDO + DS * kRow;
+    static constexpr int pK = 0, pV = kRow, pQ = 2 * kRow, pDO = pQ + BS * kBlk;
+    static constexpr int pDQ = pDO + BS * kBlk, pDDO = pDQ + DS * kRow;
+    static constexpr int pP = pDDO + DS * kRow, pDS = pP + PS * kPTile;
+    static constexpr int kPipe = pDS + PS * kPTile;
+    // lse (base 2) and Delta of each band stage's BB queries, after the pipelines
+    static constexpr int kStage = 2 * BB * 4;
+    static constexpr int kLse = NP * kPipe;
+    static constexpr int kBars = kLse + NP * BS * kStage;
     static constexpr int DSX = DS > 0 ? DS : 1;
-    static constexpr int bKVFull = 0, bBandFull = 1, bBandEmpty = bBandFull + BS;
-    static constexpr int bSFull = bBandEmpty + BS, bSFree = bSFull + 2;
-    static constexpr int bPFull = bSFree + 2, bPDone = bPFull + PB;
-    static constexpr int bInit = bPDone + PB, bDiagFull = bInit + 1;
-    static constexpr int bDiagEmpty = bDiagFull + DSX, bGroup = bDiagEmpty + DSX;
-    static constexpr int nBars = bGroup + 1;
-    static constexpr int kMisc = kBars + nBars * 8;
-    static constexpr int kAlloc = kMisc + 16 + 1024;
-    static constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D, kTmemCols = 512;
+    // barriers of one pipeline (S^T and dP^T share a buffer index sb; P^T and
+    // dS^T are written over them, so a buffer is free once its dV/dK MMAs are done)
+    static constexpr int bKVFull = 0, bKVEmpty = 1;
+    static constexpr int bBFull = 2, bBEmpty = bBFull + BS;
+    static constexpr int bSFull = bBEmpty + BS, bSFree = bSFull + SB;
+    static constexpr int bPFull = bSFree + SB, bDKVDone = bPFull + SB;
+    static constexpr int bInit = bDKVDone + SB;
+    static constexpr int bDiagFull = bInit + 1, bDiagEmpty = bDiagFull + DSX;
+    static constexpr int bInfoFull = bDiagEmpty + DSX, bInfoEmpty = bInfoFull + 2;
+    static constexpr int bGroup = bInfoEmpty + 2;
+    static constexpr int bPSDone = bGroup + 1;              // P^T/dS^T tiles consumed
+    static constexpr int nBarsPipe = bPSDone + (PS > 0 ? PS : 1);
+    static constexpr int kMisc = kBars + NP * nBarsPipe * 8;
+    static constexpr int kTotal = kMisc + 8 + 8 * NP;
+    static constexpr int kAlloc = kTotal + 1024;
+    static_assert(PS == 0 || BB == 64, "shared-memory P tiles are 64 queries wide");
+    static constexpr uint32_t tPipe = 512 / NP, tS = 0, tDP = SB * BB, tDV = 2 * SB * BB,
+                              tDK = 2 * SB * BB + D;
+    static constexpr uint32_t kTmemCols = 512;
+    static_assert(2 * SB * BB + 2 * D <= (int)tPipe, "TMEM columns of a pipeline");
+    static_assert(kRow % 1024 == 0 && kBlk % 1024 == 0, "swizzle atoms");
 };
 
-template <int D, int BS, int DS, int PB>
-__global__ void __launch_bounds__(256, 1)
-band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                     const __grid_constant__ CUtensorMap tv,
-                     const __grid_constant__ CUtensorMap tdo,
+// Query blocks of a key tile: BB queries from k0 up to min(k0+127+W-1, T-1).
+template <int BB>
+__device__ __forceinline__ int dkv_n_band(int32_t k0, int64_t T, int32_t W) {
+    const int64_t vmax_w = (int64_t)BM - 1 + W - 1, vmax_t = T - 1 - k0;
+    const int64_t vmax = vmax_w < vmax_t ? vmax_w : vmax_t;
+    return (int)(vmax / BB + 1);
+}
+
+template <int D, int NP, int BB, int SB, int BS, int DS, int PS>
+__global__ void __launch_bounds__(128 + 128 * NP, 1)
+band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
+                     const __grid_constant__ CUtensorMap tvt,
+                     const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+                     const __grid_constant__ CUtensorMap tqd,
+                     const __grid_constant__ CUtensorMap tdod,
                      const __grid_constant__ CUtensorMap tqr,
                      const __grid_constant__ CUtensorMap tdor, const BwdArgs a) {
-    using L = LayoutDKV<D, BS, DS, PB>;
+    using L = LayoutDKV<D, NP, BB, SB, BS, DS, PS>;
     constexpr int DSX = L::DSX;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_u32(sm);
     uint32_t *tmem_slot = (uint32_t *)(sm + L::kMisc);
     volatile int *abort = (volatile int *)(sm + L::kMisc + 4);
-    int *n_diag_s = (int *)(sm + L::kMisc + 8);
-    auto bar = [&](int b) { return sbase + L::kBars + 8u * (uint32_t)b; };
+    auto bar = [&](int p, int b) {
+        return sbase + L::kBars + 8u * (uint32_t)(p * L::nBarsPipe + b);
+    };
+    auto wait = [&](int p, int b, uint32_t parity) {
+        return tc::mbar_wait(bar(p, b), parity, abort, a.err, SA_DEVERR_TIMEOUT);
+    };
+    auto stage_lse = [&](int p, int st) {
+        return (float *)(sm + L::kLse + (p * BS + st) * L::kStage);
+    };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t bh = blockIdx.y, k0 = (int64_t)blockIdx.x * BM, T = a.T;
+    const int64_t T = a.T;
     const int32_t W = a.W;
-    // queries k0 .. min(T-1, k0+127+W-1) in blocks of 64 from k0
-    const int64_t vmax_w = (int64_t)BM - 1 + W - 1, vmax_t = T - 1 - k0;
-    const int64_t vmax = vmax_w < vmax_t ? vmax_w : vmax_t;
-    const int n_band = (int)(vmax / BB + 1);
+    const int64_t ntr = (T + BM - 1) / BM, ntiles = ntr * a.BH;
+    const int64_t stride = (int64_t)gridDim.x * NP;
 
     if (tid == 0) {
-        tc::mbar_init(bar(L::bKVFull), 1);
-        for (int s = 0; s < BS; ++s) {
-            // TMA bytes + the 32 producer lanes that stage lse and Delta
-            tc::mbar_init(bar(L::bBandFull + s), 33);
-            tc::mbar_init(bar(L::bBandEmpty + s), 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            tc::mbar_init(bar(L::bSFull + s), 1);
-            tc::mbar_init(bar(L::bSFree + s), 4);
-        }
-        for (int s = 0; s < PB; ++s) {
-            tc::mbar_init(bar(L::bPFull + s), 4);
-            tc::mbar_init(bar(L::bPDone + s), 1);
-        }
-        tc::mbar_init(bar(L::bInit), 4);
-        tc::mbar_init(bar(L::bGroup), 128);  // 128-thread compute barrier (bounded)
-        for (int s = 0; s < DSX; ++s) {
-            tc::mbar_init(bar(L::bDiagFull + s), 1);
-            tc::mbar_init(bar(L::bDiagEmpty + s), 4);
+        for (int p = 0; p < NP; ++p) {
+            tc::mbar_init(bar(p, L::bKVFull), 1);
+            tc::mbar_init(bar(p, L::bKVEmpty), 5);  // last S^T/dP^T MMA commit + 4 compute warps
+            for (int s = 0; s < BS; ++s) {
+                // TMA bytes + the 32 producer lanes that stage lse and Delta
+                tc::mbar_init(bar(p, L::bBFull + s), 33);
+                tc::mbar_init(bar(p, L::bBEmpty + s), 1);
+            }
+            for (int s = 0; s < SB; ++s) {
+                tc::mbar_init(bar(p, L::bSFull + s), 1);
+                // freed by the dV/dK MMAs (P^T in TMEM) or by the compute warps
+                tc::mbar_init(bar(p, L::bSFree + s), PS > 0 ? 4 : 1);
+                tc::mbar_init(bar(p, L::bPFull + s), 4);
+                tc::mbar_init(bar(p, L::bDKVDone + s), 1);
+            }
+            tc::mbar_init(bar(p, L::bInit), 4);
+            for (int s = 0; s < DSX; ++s) {
+                tc::mbar_init(bar(p, L::bDiagFull + s), 1);
+                tc::mbar_init(bar(p, L::bDiagEmpty + s), 4);
+            }
+            for (int s = 0; s < 2; ++s) {
+                tc::mbar_init(bar(p, L::bInfoFull + s), 1);
+                tc::mbar_init(bar(p, L::bInfoEmpty + s), 4);
+            }
+            tc::mbar_init(bar(p, L::bGroup), 128);
+            for (int s = 0; s < PS; ++s) tc::mbar_init(bar(p, L::bPSDone + s), 1);
         }
         *abort = 0;
-        *n_diag_s = 0;
         tc::fence_barrier_init();
     }
     if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), L::kTmemCols);
-    __syncthreads();
-    if (DS > 0 && warp >= 4) {
-        int nd = 0;
-        const int64_t j = k0 + (tid - 128);
-        if (a.kind == 0) {
-            for (int x = 0; x < a.n_off; ++x) nd += (k0 + a.offs[x] <= T - 1) ? 1 : 0;
-        } else if (j < T) {
-            const int64_t deg = a.rev_rowptr[j + 1] - a.rev_rowptr[j];
-            nd = (int)(deg - ((T - j < W) ? T - j : W));
-        }
-        atomicMax(n_diag_s, nd);
-    }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_diag = DS > 0 ? *n_diag_s : 0;
-    // distance list of this tile: the n_diag smallest offsets with k0 + o <= T-1,
-    // taken in descending order (as stored)
-    const int off_first = a.n_off - n_diag;
 
-    if (warp == 0) {
-        // lane 0 issues the TMA copies; all 32 lanes stage lse (base 2) and
-        // Delta of the block's 64 queries (zero past the end of the sequence)
-        if (lane == 0) {
-            tc::mbar_arrive_expect_tx(bar(L::bKVFull), 2 * L::kRow);
-            tma_tile128<D>(sbase + L::kK, &tk, k0, bh, bar(L::bKVFull));
-            tma_tile128<D>(sbase + L::kV, &tv, k0, bh, bar(L::bKVFull));
-        }
-        for (int bl = 0; bl < n_band; ++bl) {
-            const int st = bl % BS, use = bl / BS;
-            if (use > 0) WAIT_OR(bar(L::bBandEmpty + st), (use - 1) & 1, break);
-            const int64_t qrow = k0 + (int64_t)bl * BB;
-            if (lane == 0) {
-                tc::mbar_arrive_expect_tx(bar(L::bBandFull + st), 2 * L::kBlk);
-                tma_block64<D>(sbase + L::kQ + st * L::kBlk, &tq, qrow, bh, bar(L::bBandFull + st));
-                tma_block64<D>(sbase + L::kDO + st * L::kBlk, &tdo, qrow, bh,
-                               bar(L::bBandFull + st));
-            }
-            float *ls = (float *)(sm + L::kLse + st * 256), *dl = (float *)(sm + L::kDel + st * 256);
-            for (int c = lane; c < BB; c += 32) {
-                const int64_t i = qrow + c;
-                const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
-                ls[c] = i < T ? a.lse[gi] * kLog2e : 0.f;
-                dl[c] = i < T ? a.delta[gi] : 0.f;
-            }
-            tc::mbar_arrive(bar(L::bBandFull + st));
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idS = tc::idesc_bf16(BM, BB, false, false);
-            const uint32_t idG = tc::idesc_bf16(BM, D, false, true);
-            bool ok = tc::mbar_wait(bar(L::bKVFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
-            auto issue = [&](int bl) -> bool {
-                const int st = bl % BS, sb = bl & 1;
-                if (!tc::mbar_wait(bar(L::bBandFull + st), (bl / BS) & 1, abort, a.err,
-                                   SA_DEVERR_TIMEOUT))
-                    return false;
-                if (bl >= 2 && !tc::mbar_wait(bar(L::bSFree + sb), ((bl >> 1) - 1) & 1, abort,
-                                              a.err, SA_DEVERR_TIMEOUT))
-                    return false;
-                tc::tc_fence_after();
-                const uint32_t qa = sbase + L::kQ + st * L::kBlk, da = sbase + L::kDO + st * L::kBlk;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t offr = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                    const uint32_t offb = (kk >> 2) * (BB * 128) + (kk & 3) * 32;
-                    tc::mma_bf16_ss(tmem + L::tS + sb * BB,
-                                    tc::sdesc_sw128(sbase + L::kK + offr, 16, 1024),
-                                    tc::sdesc_sw128(qa + offb, 16, 1024), idS, kk > 0);
-                    tc::mma_bf16_ss(tmem + L::tDP + sb * BB,
-                                    tc::sdesc_sw128(sbase + L::kV + offr, 16, 1024),
-                                    tc::sdesc_sw128(da + offb, 16, 1024), idS, kk > 0);
-                }
-                tc::mma_commit(bar(L::bSFull + sb));
-                return true;
-            };
-            if (ok && n_band > 0) ok = issue(0);
-            for (int bl = 0; ok && bl < n_band; ++bl) {
-                if (BS >= 2 && bl + 1 < n_band && !issue(bl + 1)) break;
-                const int pb = bl % PB, st = bl % BS;
-                if (bl == 0) WAIT_OR(bar(L::bInit), 0, break);
-                WAIT_OR(bar(L::bPFull + pb), (bl / PB) & 1, break);
-                tc::tc_fence_after();
-                const uint32_t pa = sbase + L::kP + pb * L::kPTile;
-                const uint32_t dsa = sbase + L::kDS + pb * L::kPTile;
-                const uint32_t qa = sbase + L::kQ + st * L::kBlk, da = sbase + L::kDO + st * L::kBlk;
-#pragma unroll
-                for (int kk = 0; kk < BB / 16; ++kk) {
-                    tc::mma_bf16_ss(tmem + L::tDV, tc::sdesc_sw128(pa + kk * 32, 16, 1024),
-                                    tc::sdesc_sw128(da + kk * 16 * 128, BB * 128, 1024), idG, 1u);
-                    tc::mma_bf16_ss(tmem + L::tDK, tc::sdesc_sw128(dsa + kk * 32, 16, 1024),
-                                    tc::sdesc_sw128(qa + kk * 16 * 128, BB * 128, 1024), idG, 1u);
-                }
-                tc::mma_commit(bar(L::bBandEmpty + st));
-                tc::mma_commit(bar(L::bPDone + pb));
-                if (BS == 1 && bl + 1 < n_band && !issue(bl + 1)) break;
-            }
-        }
-    } else if (warp == 2 || warp == 3) {
-        // warp 2 stages the diagonal blocks; warp 3 has no role
-        if (warp == 2 && DS > 0) {
+    if (warp < 4) {
+        if (NP == 2) tc::regs_dec<BwdRegs::producer>();
+      if ((warp >> 1) < NP && (warp & 1) == 0) {
+        // ---------------- producer of pipeline p: diagonal-block count, K and V
+        // of the tile, the first band Q/dO blocks (with lse and Delta), the
+        // diagonal blocks, the rest
+        const int p = warp >> 1;
+        const uint32_t pb = sbase + (uint32_t)(p * L::kPipe);
+        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
+        uint32_t bc = 0, dc = 0;
+        bool ok = true;
+        int64_t lt = 0;
+        for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
+            const TileId id = tile_id(t, ntr);
+            const int32_t k0 = id.r0, bh = id.bh;
+            const int n_band = dkv_n_band<BB>(k0, T, W);
             // CSR: lane l owns key rows 4l .. 4l+3: start of the residual part of
             // their transpose lists (after the band queries j .. j+W-1), its
             // length, and the next query
             int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
             int32_t cj[4] = {0, 0, 0, 0};
-            if (a.kind == 1) {
+            int nd = 0;
+            if (DS > 0) {
+                if (a.kind == 0) {
+                    for (int x = 0; x < a.n_off; ++x) nd += (k0 + a.offs[x] <= T - 1) ? 1 : 0;
+                } else {
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int64_t j = k0 + 4 * lane + h;
-                    if (j < T) {
-                        const int64_t nb = (T - j < W) ? T - j : W;
-                        cstart[h] = a.rev_rowptr[j] + nb;
-                        cres[h] = a.rev_rowptr[j + 1] - cstart[h];
-                        if (cres[h] > 0) cj[h] = a.rev_colidx[cstart[h]];
+                    for (int h = 0; h < 4; ++h) {
+                        const int64_t j = k0 + 4 * lane + h;
+                        if (j < T) {
+                            const int64_t nb = (T - j < W) ? T - j : W;
+                            cstart[h] = a.rev_rowptr[j] + nb;
+                            cres[h] = a.rev_rowptr[j + 1] - cstart[h];
+                            if (cres[h] > 0) cj[h] = a.rev_colidx[cstart[h]];
+                            nd = nd > (int)cres[h] ? nd : (int)cres[h];
+                        }
+                    }
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const int x = __shfl_xor_sync(0xffffffffu, nd, o);
+                        nd = nd > x ? nd : x;
                     }
                 }
             }
-            for (int d = 0; d < n_diag; ++d) {
-                const int st = d % DSX, use = d / DSX;
-                const uint32_t qdst = sbase + L::kDiagQ + st * L::kRow;
-                const uint32_t ddst = sbase + L::kDiagDO + st * L::kRow;
-                if (use > 0) WAIT_OR(bar(L::bDiagEmpty + st), (use - 1) & 1, break);
-                if (lane == 0) tc::mbar_arrive_expect_tx(bar(L::bDiagFull + st), 2 * L::kRow);
+            const int slot = (int)(lt & 1);
+            if (lt >= 2 && !wait(p, L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1))) break;
+            if (lane == 0) {
+                info[slot] = nd;
+                tc::mbar_arrive(bar(p, L::bInfoFull + slot));
+            }
+            // band block bl (all lanes): lane 0 the TMA copies, every lane a
+            // share of lse (base 2) and Delta, zero past the end of the sequence
+            auto load_blk = [&](int bl) -> bool {
+                const int st = (int)(bc % BS);
+                const uint32_t use = bc / BS;
+                if (use > 0 && !wait(p, L::bBEmpty + st, (use - 1) & 1)) return false;
+                const int32_t qrow = k0 + bl * BB;
+                if (lane == 0) {
+                    tc::mbar_arrive_expect_tx(bar(p, L::bBFull + st), 2 * L::kBlk);
+                    tma_rows<D, BB>(pb + L::pQ + st * L::kBlk, &tq, qrow, bh, bar(p, L::bBFull + st));
+                    tma_rows<D, BB>(pb + L::pDO + st * L::kBlk, &tdo, qrow, bh,
+                                    bar(p, L::bBFull + st));
+                }
+                float *ls = stage_lse(p, st), *dl = ls + BB;
+                for (int c = lane; c < BB; c += 32) {
+                    const int64_t i = (int64_t)qrow + c;
+                    const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
+                    ls[c] = i < T ? a.lse[gi] * kLog2e : 0.f;
+                    dl[c] = i < T ? a.delta[gi] : 0.f;
+                }
+                tc::mbar_arrive(bar(p, L::bBFull + st));
+                ++bc;
+                return true;
+            };
+            const int n_pre = n_band < BS ? n_band : BS;
+            int okl = 1;
+            if (lane == 0) {
+                if (lt >= 1 && !wait(p, L::bKVEmpty, (uint32_t)((lt - 1) & 1))) okl = 0;
+                if (okl) {
+                    tc::mbar_arrive_expect_tx(bar(p, L::bKVFull), 2 * L::kRow);
+                    tma_rows<D, BM>(pb + L::pK, &tkt, k0, bh, bar(p, L::bKVFull));
+                    tma_rows<D, BM>(pb + L::pV, &tvt, k0, bh, bar(p, L::bKVFull));
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+            for (int bl = 0; ok && bl < n_pre; ++bl) ok = load_blk(bl);
+            for (int d = 0; ok && d < nd; ++d) {
+                const int st = (int)(dc % DSX);
+                const uint32_t use = dc / DSX;
+                const uint32_t qdst = pb + L::pDQ + st * L::kRow;
+                const uint32_t ddst = pb + L::pDDO + st * L::kRow;
+                if (use > 0 && !wait(p, L::bDiagEmpty + st, (use - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar(p, L::bDiagFull + st), 2 * L::kRow);
                 if (a.kind == 0) {
                     if (lane == 0) {
-                        const int64_t qrow = k0 + a.offs[off_first + d];
-                        tma_tile128<D>(qdst, &tq, qrow, bh, bar(L::bDiagFull + st));
-                        tma_tile128<D>(ddst, &tdo, qrow, bh, bar(L::bDiagFull + st));
+                        const int32_t qrow = (int32_t)(k0 + a.offs[a.n_off - nd + d]);
+                        tma_rows<D, BM>(qdst, &tqd, qrow, bh, bar(p, L::bDiagFull + st));
+                        tma_rows<D, BM>(ddst, &tdod, qrow, bh, bar(p, L::bDiagFull + st));
                     }
                 } else {
                     int32_t rr[4];
@@ -845,192 +1051,327 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
                     for (int h = 0; h < 4; ++h) {
                         const int64_t j = k0 + 4 * lane + h;
                         const int64_t i = d < cres[h] ? (int64_t)cj[h] : (j < T ? j : 0);
-                        rr[h] = (int32_t)(bh * T + i);
+                        rr[h] = (int32_t)((int64_t)bh * T + i);
                     }
 #pragma unroll
                     for (int x = 0; x < D / 64; ++x) {
                         const uint32_t off = x * (BM * 128) + 4 * lane * 128;
                         tc::tma_gather4(qdst + off, &tqr, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                        bar(L::bDiagFull + st));
+                                        bar(p, L::bDiagFull + st));
                         tc::tma_gather4(ddst + off, &tdor, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                        bar(L::bDiagFull + st));
+                                        bar(p, L::bDiagFull + st));
                     }
 #pragma unroll
                     for (int h = 0; h < 4; ++h)
                         if (d + 1 < cres[h]) cj[h] = a.rev_colidx[cstart[h] + d + 1];
                 }
+                ++dc;
+            }
+            for (int bl = n_pre; ok && bl < n_band; ++bl) ok = load_blk(bl);
+        }
+      } else if ((warp >> 1) < NP) {
+        // ---------------- MMA issuer of pipeline p: S^T and dP^T of block g,
+        // then dV += P^T dO and dK += dS^T Q of block g-1
+        const int p = warp >> 1;
+        const uint32_t pb = sbase + (uint32_t)(p * L::kPipe);
+        const uint32_t tp = tmem + p * L::tPipe;
+        if (lane == 0) {
+            const uint32_t idS = tc::idesc_bf16(BM, BB, false, false);
+            const uint32_t idG = tc::idesc_bf16(BM, D, false, true);
+            uint32_t gb = 0;
+            bool have = false, first = false, ok = true;
+            uint32_t pg = 0;
+            int64_t plt = 0;
+            auto do_dkv = [&]() -> bool {
+                const int sb = (int)(pg % SB), st = (int)(pg % BS);
+                if (first && !wait(p, L::bInit, (uint32_t)(plt & 1))) return false;
+                if (!wait(p, L::bPFull + sb, (pg / SB) & 1)) return false;
+                tc::tc_fence_after();
+                const uint32_t qa = pb + L::pQ + st * L::kBlk, da = pb + L::pDO + st * L::kBlk;
+                if constexpr (PS > 0) {
+                    const int ps = (int)(pg % PS);
+                    const uint32_t pa = pb + L::pP + ps * L::kPTile;
+                    const uint32_t dsa = pb + L::pDS + ps * L::kPTile;
+#pragma unroll
+                    for (int kk = 0; kk < BB / 16; ++kk) {
+                        tc::mma_bf16_ss(tp + L::tDV, tc::sdesc_sw128(pa + kk * 32, 16, 1024),
+                                        tc::sdesc_sw128(da + kk * 16 * 128, BB * 128, 1024), idG,
+                                        1u);
+                        tc::mma_bf16_ss(tp + L::tDK, tc::sdesc_sw128(dsa + kk * 32, 16, 1024),
+                                        tc::sdesc_sw128(qa + kk * 16 * 128, BB * 128, 1024), idG,
+                                        1u);
+                    }
+                    tc::mma_commit(bar(p, L::bBEmpty + st));
+                    tc::mma_commit(bar(p, L::bPSDone + ps));
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < BB / 16; ++kk) {
+                        tc::mma_bf16_ts(tp + L::tDV, tp + L::tS + sb * BB + kk * 8,
+                                        tc::sdesc_sw128(da + kk * 16 * 128, BB * 128, 1024), idG,
+                                        1u);
+                        tc::mma_bf16_ts(tp + L::tDK, tp + L::tDP + sb * BB + kk * 8,
+                                        tc::sdesc_sw128(qa + kk * 16 * 128, BB * 128, 1024), idG,
+                                        1u);
+                    }
+                    tc::mma_commit(bar(p, L::bBEmpty + st));
+                    tc::mma_commit(bar(p, L::bSFree + sb));
+                }
+                tc::mma_commit(bar(p, L::bDKVDone + sb));
+                return true;
+            };
+            int64_t lt = 0;
+            for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
+                const TileId id = tile_id(t, ntr);
+                const int n_band = dkv_n_band<BB>(id.r0, T, W);
+                if (!wait(p, L::bKVFull, (uint32_t)(lt & 1))) break;
+                const uint32_t ka = pb + L::pK, va = pb + L::pV;
+                for (int bl = 0; bl < n_band; ++bl) {
+                    const int st = (int)(gb % BS), sb = (int)(gb % SB);
+                    // one S^T buffer: dV/dK of the previous block free it first
+                    if (SB == 1 && have) {
+                        if (!do_dkv()) {
+                            ok = false;
+                            break;
+                        }
+                        have = false;
+                    }
+                    if (!wait(p, L::bBFull + st, (gb / BS) & 1) ||
+                        (gb >= SB && !wait(p, L::bSFree + sb, ((gb / SB) - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const uint32_t qa = pb + L::pQ + st * L::kBlk, da = pb + L::pDO + st * L::kBlk;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t offr = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        const uint32_t offb = (kk >> 2) * (BB * 128) + (kk & 3) * 32;
+                        tc::mma_bf16_ss(tp + L::tS + sb * BB, tc::sdesc_sw128(ka + offr, 16, 1024),
+                                        tc::sdesc_sw128(qa + offb, 16, 1024), idS, kk > 0);
+                        tc::mma_bf16_ss(tp + L::tDP + sb * BB,
+                                        tc::sdesc_sw128(va + offr, 16, 1024),
+                                        tc::sdesc_sw128(da + offb, 16, 1024), idS, kk > 0);
+                    }
+                    tc::mma_commit(bar(p, L::bSFull + sb));
+                    if (bl == n_band - 1) tc::mma_commit(bar(p, L::bKVEmpty));
+                    if (SB > 1 && have && !do_dkv()) {
+                        ok = false;
+                        break;
+                    }
+                    have = true;
+                    pg = gb;
+                    first = (bl == 0);
+                    plt = lt;
+                    ++gb;
+                }
+                // the tile's last dV/dK MMAs go now: its epilogue waits for them
+                if (ok && have) {
+                    ok = do_dkv();
+                    have = false;
+                }
             }
         }
-    } else if (warp >= 4 && warp < 8) {
-        // compute warpgroup: thread r = owned row r = TMEM lane r
-        const int r = tid - 128;
-        const int64_t j = k0 + r;
-        const bool row_ok = j < T;
-        const size_t grow = (size_t)bh * (size_t)T + (size_t)j;
-        const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
-        const uint32_t tS = tmem + lane_off + L::tS, tDP = tmem + lane_off + L::tDP;
-        const uint32_t tDV = tmem + lane_off + L::tDV, tDK = tmem + lane_off + L::tDK;
+      }
+    } else {
+        // ---------------- compute warpgroup of pipeline p: thread r = key row
+        // r = TMEM lane r
+        if (NP == 2) tc::regs_inc<BwdRegs::compute>();
+        const int p = (warp - 4) >> 2;
+        const int r = tid - 128 - 128 * p;
+        uint8_t *pm = sm + p * L::kPipe;
+        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
+        const uint32_t lane_off = (uint32_t)(((warp - 4) & 3) * 32) << 16;
+        const uint32_t tbase = tmem + p * L::tPipe + lane_off;
+        const uint32_t tS = tbase + L::tS, tDP = tbase + L::tDP;
+        const uint32_t tDV = tbase + L::tDV, tDK = tbase + L::tDK;
         const float c2 = a.scale2;
-        bool ok = tc::mbar_wait(bar(L::bKVFull), 0, abort, a.err, SA_DEVERR_TIMEOUT);
-        if (ok) {
+        uint32_t dc = 0, gb = 0, group_uses = 0;
+        bool ok = true;
+        int64_t lt = 0;
+        for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
+            const TileId id = tile_id(t, ntr);
+            const int32_t k0 = id.r0, bh = id.bh;
+            const int n_band = dkv_n_band<BB>(k0, T, W);
+            const int64_t j = k0 + r;
+            const bool row_ok = j < T;
+            const size_t gbh = (size_t)bh * (size_t)T;
+            const size_t grow = gbh + (size_t)j;
+            const int slot = (int)(lt & 1);
+            if (!wait(p, L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1))) break;
+            const int nd = info[slot];
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
+            if (!wait(p, L::bKVFull, (uint32_t)(lt & 1))) break;
             // diagonal blocks (fp32 pairs); lse and Delta of the linked query
             // are loaded one block ahead
             uint64_t adk2[D / 2], adv2[D / 2];
 #pragma unroll
             for (int x = 0; x < D / 2; ++x) adk2[x] = adv2[x] = 0ull;
-            const size_t gbh = (size_t)bh * (size_t)T;
-            if (DS > 0 && n_diag > 0) {
-                if (a.kind == 0) {
-                    // distance links: query j + o, swizzled tiles read in logical order
-                    auto query_of = [&](int d) -> int64_t {
-                        if (!row_ok || d >= n_diag) return -1;
+            if (DS > 0 && nd > 0) {
+                const int off_first = a.n_off - nd;
+                int64_t rs = 0, nb = 0, resid = 0;
+                if (a.kind == 1 && row_ok) {
+                    rs = a.rev_rowptr[j];
+                    nb = (T - j < W) ? T - j : W;
+                    resid = a.rev_rowptr[j + 1] - rs - nb;
+                }
+                // query of slot d (-1 if none)
+                auto query_of = [&](int d) -> int64_t {
+                    if (!row_ok || d >= nd) return -1;
+                    if (a.kind == 0) {
                         const int64_t cand = j + a.offs[off_first + d];
                         return cand < T ? cand : -1;
-                    };
-                    int64_t i_cur = query_of(0);
-                    float lse_cur = i_cur >= 0 ? a.lse[gbh + i_cur] : 0.f;
-                    float del_cur = i_cur >= 0 ? a.delta[gbh + i_cur] : 0.f;
-                    for (int d = 0; d < n_diag; ++d) {
-                        const int64_t i_nxt = query_of(d + 1);
-                        const float lse_nxt = i_nxt >= 0 ? a.lse[gbh + i_nxt] : 0.f;
-                        const float del_nxt = i_nxt >= 0 ? a.delta[gbh + i_nxt] : 0.f;
-                        const int st = d % DSX;
-                        WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
-                        if (i_cur >= 0) {
-                            const uint8_t *qt = sm + L::kDiagQ + st * L::kRow;
-                            const uint8_t *dt = sm + L::kDiagDO + st * L::kRow;
-                            const float sdot = dot2_smem_smem<D>(qt, sm + L::kK, BM, r);
-                            const float dpdot = dot2_smem_smem<D>(dt, sm + L::kV, BM, r);
-                            const float p = tc::ex2(fmaf(sdot, c2, -lse_cur * kLog2e));
-                            const float ds = p * (dpdot - del_cur);
-                            axpy2_smem<D>(adv2, p, dt, BM, r);
-                            axpy2_smem<D>(adk2, ds, qt, BM, r);
+                    }
+                    return d < resid ? (int64_t)a.rev_colidx[rs + nb + d] : -1;
+                };
+                int64_t i_cur = query_of(0), i_nxt = query_of(1);
+                float lse_cur = i_cur >= 0 ? a.lse[gbh + i_cur] : 0.f;
+                float del_cur = i_cur >= 0 ? a.delta[gbh + i_cur] : 0.f;
+                for (int d = 0; d < nd; ++d) {
+                    const int64_t i_n2 = query_of(d + 2);
+                    const float lse_nxt = i_nxt >= 0 ? a.lse[gbh + i_nxt] : 0.f;
+                    const float del_nxt = i_nxt >= 0 ? a.delta[gbh + i_nxt] : 0.f;
+                    const int st = (int)(dc % DSX);
+                    if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    if (i_cur >= 0) {
+                        const uint8_t *qt = pm + L::pDQ + st * L::kRow;
+                        const uint8_t *dt = pm + L::pDDO + st * L::kRow;
+                        float sdot, dpdot;
+                        if (a.kind == 0) {
+                            sdot = dot2_smem_smem<D>(qt, pm + L::pK, BM, r);
+                            dpdot = dot2_smem_smem<D>(dt, pm + L::pV, BM, r);
+                        } else {
+                            // CSR gathers are unswizzled: the key's k and v rows
+                            // read in physical chunk order pair with them
+                            sdot = dot2_phys_gathered<D>(pm + L::pK, qt, BM, r);
+                            dpdot = dot2_phys_gathered<D>(pm + L::pV, dt, BM, r);
                         }
+                        const float pr = tc::ex2(fmaf(sdot, c2, -lse_cur * kLog2e));
+                        const float ds = pr * (dpdot - del_cur);
+                        axpy2_smem<D>(adv2, pr, dt, BM, r);
+                        axpy2_smem<D>(adk2, ds, qt, BM, r);
+                    }
+                    if (a.kind == 0 || d < nd - 1) {  // CSR: last stage released below
                         __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
-                        i_cur = i_nxt;
-                        lse_cur = lse_nxt;
-                        del_cur = del_nxt;
+                        if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
                     }
-                } else {
-                    // CSR gathers are unswizzled: the key's k and v rows read in
-                    // physical chunk order pair with them (see the forward)
-                    int64_t rs = 0, nb = 0, resid = 0;
-                    if (row_ok) {
-                        rs = a.rev_rowptr[j];
-                        nb = (T - j < W) ? T - j : W;
-                        resid = a.rev_rowptr[j + 1] - rs - nb;
-                    }
-                    // query of slot d (-1 if none): the list entry two slots
-                    // ahead, lse and Delta one slot ahead
-                    auto query_of = [&](int d) -> int64_t {
-                        return (row_ok && d < resid) ? (int64_t)a.rev_colidx[rs + nb + d] : -1;
-                    };
-                    int64_t i_cur = query_of(0), i_nxt = query_of(1);
-                    float lse_cur = i_cur >= 0 ? a.lse[gbh + i_cur] : 0.f;
-                    float del_cur = i_cur >= 0 ? a.delta[gbh + i_cur] : 0.f;
-                    for (int d = 0; d < n_diag; ++d) {
-                        const int64_t i_n2 = query_of(d + 2);
-                        const float lse_nxt = i_nxt >= 0 ? a.lse[gbh + i_nxt] : 0.f;
-                        const float del_nxt = i_nxt >= 0 ? a.delta[gbh + i_nxt] : 0.f;
-                        const int st = d % DSX;
-                        WAIT_OR(bar(L::bDiagFull + st), (d / DSX) & 1, ok = false; break);
-                        if (i_cur >= 0) {
-                            const uint8_t *qt = sm + L::kDiagQ + st * L::kRow;
-                            const uint8_t *dt = sm + L::kDiagDO + st * L::kRow;
-                            const float sdot = dot2_phys_gathered<D>(sm + L::kK, qt, BM, r);
-                            const float dpdot = dot2_phys_gathered<D>(sm + L::kV, dt, BM, r);
-                            const float p = tc::ex2(fmaf(sdot, c2, -lse_cur * kLog2e));
-                            const float ds = p * (dpdot - del_cur);
-                            axpy2_smem<D>(adv2, p, dt, BM, r);
-                            axpy2_smem<D>(adk2, ds, qt, BM, r);
-                        }
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(bar(L::bDiagEmpty + st));
-                        i_cur = i_nxt;
-                        i_nxt = i_n2;
-                        lse_cur = lse_nxt;
-                        del_cur = del_nxt;
-                    }
-                    tc::mbar_arrive(bar(L::bGroup));
-                    if (!tc::mbar_wait(bar(L::bGroup), 0, abort, a.err, SA_DEVERR_TIMEOUT)) ok = false;
-                    float *scr = (float *)(sm + L::kDiagQ);
-                    unpermute_row2<D>(adv2, scr + (size_t)r * D, r);
-                    unpermute_row2<D>(adk2, scr + (size_t)(BM + r) * D, r);
+                    ++dc;
+                    i_cur = i_nxt;
+                    i_nxt = i_n2;
+                    lse_cur = lse_nxt;
+                    del_cur = del_nxt;
+                }
+                if (ok && a.kind == 1) {
+                    // restore the logical order through the last stage once
+                    // every row is done with it (thread r: D floats, rows < 64
+                    // in its Q half, the others in its dO half)
+                    const int st = (int)((dc - 1) % DSX);
+                    tc::mbar_arrive(bar(p, L::bGroup));
+                    if (!wait(p, L::bGroup, group_uses & 1)) ok = false;
+                    ++group_uses;
+                    float *scr = (float *)(pm + (r < 64 ? L::pDQ : L::pDDO) + st * L::kRow) +
+                                 (size_t)(r & 63) * D;
+                    unpermute_row2<D>(adv2, scr, r);
+                    unpermute_row2<D>(adk2, scr, r);
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
                 }
             }
+            if (!ok) break;
+            // this warp is done reading K and V of the tile
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(p, L::bKVEmpty));
             tmem_store_row2<D>(tDV, adv2);
             tmem_store_row2<D>(tDK, adk2);
             tc::tmem_st_wait();
-        }
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(bar(L::bInit));
-
-        for (int bl = 0; ok && bl < n_band; ++bl) {
-            const int sb = bl & 1, pb = bl % PB, st = bl % BS;
-            const int64_t v0 = (int64_t)bl * BB;
-            WAIT_OR(bar(L::bSFull + sb), (bl >> 1) & 1, ok = false; break);
-            tc::tc_fence_after();
-            float s[BB], dp[BB];
-            tc::tmem_ld32(tS + sb * BB, (uint32_t *)s);
-            tc::tmem_ld32(tS + sb * BB + 32, (uint32_t *)(s + 32));
-            tc::tmem_ld32(tDP + sb * BB, (uint32_t *)dp);
-            tc::tmem_ld32(tDP + sb * BB + 32, (uint32_t *)(dp + 32));
-            tc::tmem_ld_wait();
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(L::bSFree + sb));
-            const float *lse_s = (const float *)(sm + L::kLse + st * 256);
-            const float *del_s = (const float *)(sm + L::kDel + st * 256);
-            const bool need_mask = (v0 < BM - 1) || (v0 + BB - 1 > (int64_t)W - 1) ||
-                                   (k0 + v0 + BB - 1 > T - 1);
-            if (need_mask) {
-                // keep columns [c_lo, c_hi]: r <= v <= r+W-1 and query < T
-                const int64_t vlim = T - 1 - k0;
-                int64_t hi = (int64_t)r + W - 1;
-                if (hi > vlim) hi = vlim;
-                const int64_t lo = r;
-                const int c_lo = (int)(lo - v0 < 0 ? 0 : (lo - v0 > BB ? BB : lo - v0));
-                const int c_hi = (int)(hi - v0 > BB - 1 ? BB - 1 : (hi - v0 < -1 ? -1 : hi - v0));
-                // 16-column chunks outside every kept range of this warp: P = dS = 0
+            if (lane == 0) tc::mbar_arrive(bar(p, L::bInit));
+
+            // band blocks: P^T and dS^T (bf16) over S^T and dP^T
+            uint32_t gb_last = gb;
+            for (int bl = 0; ok && bl < n_band; ++bl, ++gb) {
+                const int sb = (int)(gb % SB), st = (int)(gb % BS);
+                const int32_t v0 = bl * BB;
+                gb_last = gb;
+                if (!wait(p, L::bSFull + sb, (gb / SB) & 1) ||
+                    !wait(p, L::bBFull + st, (gb / BS) & 1)) {  // lse / Delta staged
+                    ok = false;
+                    break;
+                }
+                tc::tc_fence_after();
+                float s[BB], dp[BB];
+                tc::tmem_ld_n<BB>(tS + sb * BB, (uint32_t *)s);
+                tc::tmem_ld_n<BB>(tDP + sb * BB, (uint32_t *)dp);
+                tc::tmem_ld_wait();
+                if (PS > 0) {  // S^T and dP^T are in registers: the buffer is free
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(p, L::bSFree + sb));
+                }
+                const float *lse_s = stage_lse(p, st), *del_s = lse_s + BB;
+                const bool need_mask = (v0 < BM - 1) || (v0 + BB - 1 > W - 1) ||
+                                       ((int64_t)k0 + v0 + BB - 1 > T - 1);
+                if (need_mask) {
+                    // keep columns [c_lo, c_hi]: r <= v <= r+W-1 and query < T
+                    const int64_t vlim = T - 1 - k0;
+                    int64_t hi = (int64_t)r + W - 1;
+                    if (hi > vlim) hi = vlim;
+                    const int64_t lo = r;
+                    const int c_lo = (int)(lo - v0 < 0 ? 0 : (lo - v0 > BB ? BB : lo - v0));
+                    const int c_hi =
+                        (int)(hi - v0 > BB - 1 ? BB - 1 : (hi - v0 < -1 ? -1 : hi - v0));
+                    // 16-column chunks outside every kept range of this warp: P = dS = 0
 #pragma unroll
-                for (int c16 = 0; c16 < BB / 16; ++c16) {
-                    if (__any_sync(0xffffffffu, c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16)) {
+                    for (int c16 = 0; c16 < BB / 16; ++c16) {
+                        if (__any_sync(0xffffffffu, c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16)) {
 #pragma unroll
-                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
-                            const float p = (c >= c_lo && c <= c_hi)
-                                                ? tc::ex2(fmaf(s[c], c2, -lse_s[c]))
-                                                : 0.f;
-                            s[c] = p;
-                            dp[c] = p * (dp[c] - del_s[c]);
+                            for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
+                                const float pr = (c >= c_lo && c <= c_hi)
+                                                     ? tc::ex2(fmaf(s[c], c2, -lse_s[c]))
+                                                     : 0.f;
+                                s[c] = pr;
+                                dp[c] = pr * (dp[c] - del_s[c]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 16 * c16; c < 16 * c16 + 16; ++c) s[c] = dp[c] = 0.f;
                         }
-                    } else {
+                    }
+                } else {
 #pragma unroll
-                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) s[c] = dp[c] = 0.f;
+                    for (int c = 0; c < BB; ++c) {
+                        const float pr = tc::ex2(fmaf(s[c], c2, -lse_s[c]));
+                        s[c] = pr;
+                        dp[c] = pr * (dp[c] - del_s[c]);
                     }
                 }
-            } else {
-#pragma unroll
-                for (int c = 0; c < BB; ++c) {
-                    const float p = tc::ex2(fmaf(s[c], c2, -lse_s[c]));
-                    s[c] = p;
-                    dp[c] = p * (dp[c] - del_s[c]);
+                if constexpr (PS > 0) {
+                    const int ps = (int)(gb % PS);
+                    if (gb >= PS && !wait(p, L::bPSDone + ps, ((gb / PS) - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    store_row64_bf16(pm + L::pP + ps * L::kPTile, r, s);
+                    store_row64_bf16(pm + L::pDS + ps * L::kPTile, r, dp);
+                    tc::fence_proxy_async_smem();
+                } else {
+                    uint32_t w[BB / 2];
+                    pack_bf16_row<BB>(s, w);
+                    tc::tmem_st_n<BB / 2>(tS + sb * BB, w);
+                    pack_bf16_row<BB>(dp, w);
+                    tc::tmem_st_n<BB / 2>(tDP + sb * BB, w);
+                    tc::tmem_st_wait();
+                    tc::tc_fence_before();
                 }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(p, L::bPFull + sb));
             }
-            if (bl >= PB) WAIT_OR(bar(L::bPDone + pb), ((bl - PB) / PB) & 1, ok = false; break);
-            store_row64_bf16(sm + L::kP + pb * L::kPTile, r, s);
-            store_row64_bf16(sm + L::kDS + pb * L::kPTile, r, dp);
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(L::bPFull + pb));
-        }
-        if (ok && n_band > 0) {
-            const int lb = n_band - 1;
-            ok = tc::mbar_wait(bar(L::bPDone + lb % PB), (lb / PB) & 1, abort, a.err,
-                               SA_DEVERR_TIMEOUT);
-        }
-        if (ok) {
+            if (!ok) break;
+            if (!wait(p, L::bDKVDone + (int)(gb_last % SB), (gb_last / SB) & 1)) break;
             tc::tc_fence_after();
             tmem_row_to_global<D>(tDV, 1.f, a.dv + grow * D, row_ok);
             tmem_row_to_global<D>(tDK, a.scale, a.dk + grow * D, row_ok);
@@ -1044,28 +1385,55 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
     }
 }
 
-template <int D, int BSQ, int BSK, int DS, int PBQ, int PBK>
+template <int NP>
+inline bool regs_cover(const void *kern) {
+    // setmaxnreg.inc waits until the CTA's pool holds what it asks for: the
+    // launch must provide the whole warpgroup split
+    if (NP != 2) return true;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
+    return fa.numRegs * (128 + 128 * NP) >= 128 * BwdRegs::producer + 128 * NP * BwdRegs::compute;
+}
+
+template <int D, int NP, int BB, int SB, int BSQ, int BSK, int DS, int PS>
 sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_tensor *o, const float *lse, const sa_tensor *dout,
                           const sa_graph_s *g, float scale, sa_tensor *dq, sa_tensor *dk,
                           sa_tensor *dv, float *delta, cudaStream_t s) {
-    using LQ = LayoutDQ<D, BSQ, DS, PBQ>;
-    using LK = LayoutDKV<D, BSK, DS, PBK>;
+    using LQ = LayoutDQ<D, NP, BB, SB, BSQ, DS, PS>;
+    using LK = LayoutDKV<D, NP, BB, SB, BSK, DS, PS>;
     static_assert(LQ::kAlloc <= 232448 && LK::kAlloc <= 232448, "shared memory budget");
+    constexpr int kThreads = 128 + 128 * NP;
+    auto kq = band_bwd_dq_kernel<D, NP, BB, SB, BSQ, DS, PS>;
+    auto kkv = band_bwd_dkdv_kernel<D, NP, BB, SB, BSK, DS, PS>;
+    static int regs_ok = -1;
+    if (regs_ok < 0)
+        regs_ok = regs_cover<NP>((const void *)kq) && regs_cover<NP>((const void *)kkv);
+    if (!regs_ok) {
+        sa_record_cuda_error(cudaErrorInvalidConfiguration,
+                             "band_bwd: launch registers below the warpgroup split");
+        return SA_ERR_CUDA;
+    }
     const int64_t BH = q->B * q->H, T = q->T;
-    CUtensorMap mq, mk, mv, mdo, mqr, mkr, mvr, mdor;
     const uint64_t rows = (uint64_t)(BH * T);
-    if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BB) || !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BH, BB) ||
-        !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BH, BB) ||
-        !sa_tmap_bf16_3d(&mdo, dout->ptr, D, T, BH, BB) ||
+    // 128-row boxes for the tiles and distance blocks, BB-row boxes for the
+    // band rings, one-row maps for the CSR gathers
+    CUtensorMap mq, mdo, mk, mv, mqb, mdob, mkb, mvb, mqr, mdor, mkr, mvr;
+    if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BM) ||
+        !sa_tmap_bf16_3d(&mdo, dout->ptr, D, T, BH, BM) ||
+        !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BH, BM) || !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BH, BM) ||
+        !sa_tmap_bf16_3d(&mqb, q->ptr, D, T, BH, BB) ||
+        !sa_tmap_bf16_3d(&mdob, dout->ptr, D, T, BH, BB) ||
+        !sa_tmap_bf16_3d(&mkb, k->ptr, D, T, BH, BB) ||
+        !sa_tmap_bf16_3d(&mvb, v->ptr, D, T, BH, BB) ||
         !sa_tmap_bf16_rows(&mqr, q->ptr, D, rows) || !sa_tmap_bf16_rows(&mkr, k->ptr, D, rows) ||
-        !sa_tmap_bf16_rows(&mvr, v->ptr, D, rows) || !sa_tmap_bf16_rows(&mdor, dout->ptr, D, rows))
-    {
+        !sa_tmap_bf16_rows(&mvr, v->ptr, D, rows) || !sa_tmap_bf16_rows(&mdor, dout->ptr, D, rows)) {
         sa_record_cuda_error(cudaErrorInvalidValue, "band_bwd: tensor map encoding");
         return SA_ERR_CUDA;
     }
     BwdArgs a{};
     a.T = T;
+    a.BH = BH;
     a.W = g->W;
     a.kind = g->kind;
     a.n_off = g->kind == 0 ? g->n_off : 0;
@@ -1074,11 +1442,7 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.colidx = g->colidx;
     a.rev_rowptr = g->rev_rowptr;
     a.rev_colidx = g->rev_colidx;
-    a.q = (const __nv_bfloat16 *)q->ptr;
-    a.k = (const __nv_bfloat16 *)k->ptr;
-    a.v = (const __nv_bfloat16 *)v->ptr;
     a.o = (const __nv_bfloat16 *)o->ptr;
-    a.dout = (const __nv_bfloat16 *)dout->ptr;
     a.lse = lse;
     a.delta = delta;
     a.dq = (__nv_bfloat16 *)dq->ptr;
@@ -1088,14 +1452,18 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.scale2 = scale * kLog2e;
     a.err = sa_device_error_word();
     if (!a.err) return SA_ERR_CUDA;
-    auto kq = band_bwd_dq_kernel<D, BSQ, DS, PBQ>;
-    auto kkv = band_bwd_dkdv_kernel<D, BSK, DS, PBK>;
     SA_CUDA_TRY(sa_smem_optin((const void *)kq, LQ::kAlloc));
     SA_CUDA_TRY(sa_smem_optin((const void *)kkv, LK::kAlloc));
-    dim3 grid((unsigned)((T + BM - 1) / BM), (unsigned)BH);
-    SA_LAUNCH("band_bwd_dq", s, kq<<<grid, 256, LQ::kAlloc, s>>>(mq, mk, mv, mdo, mkr, mvr, a));
+    // persistent: one CTA per SM, NP tiles in flight in each
+    const int64_t ntiles = ((T + BM - 1) / BM) * BH;
+    int sms = 0;
+    SA_CUDA_TRY(sa_sm_count(&sms));
+    const int64_t nctas = (ntiles + NP - 1) / NP;
+    const unsigned grid = (unsigned)(nctas < sms ? nctas : sms);
+    SA_LAUNCH("band_bwd_dq", s,
+              kq<<<grid, kThreads, LQ::kAlloc, s>>>(mq, mdo, mkb, mvb, mk, mv, mkr, mvr, a));
     SA_LAUNCH("band_bwd_dkdv", s,
-              kkv<<<grid, 256, LK::kAlloc, s>>>(mq, mk, mv, mdo, mqr, mdor, a));
+              kkv<<<grid, kThreads, LK::kAlloc, s>>>(mk, mv, mqb, mdob, mq, mdo, mqr, mdor, a));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
@@ -1108,7 +1476,7 @@ bool sa_band_bwd_supported(const sa_tensor *q, const sa_graph_s *g) {
     if (q->B * q->H > 65535 || q->T >= ((int64_t)1 << 31)) return false;
     const bool diag = (g->kind == 0) ? g->n_off > 0 : (g->max_resid > 0 || g->max_resid_rev > 0);
     if (g->kind == 1 && (!g->rowptr || !g->rev_rowptr)) return false;
-    // distance / CSR edges with D = 128 stay on the gather kernels (register budget)
+    // distance / CSR edges with D = 128 stay on the gather kernels (shared memory)
     if (diag && q->D == 128) return false;
     return true;
 }
@@ -1118,13 +1486,15 @@ sa_status sa_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
                       const sa_graph_s *g, const GraphView &, float scale, sa_tensor *dq,
                       sa_tensor *dk, sa_tensor *dv, float *delta, cudaStream_t s) {
     const bool diag = (g->kind == 0) ? g->n_off > 0 : (g->max_resid > 0 || g->max_resid_rev > 0);
-    // <D, dQ ring stages, dK/dV ring stages, diagonal stages, dS buffers,
-    //  P^T/dS^T buffers>, sized to the 227 KB of shared memory
+    // <D, pipelines, band block, S buffers, dQ ring stages, dK/dV ring stages,
+    //  diagonal stages, shared-memory P/dS tiles>, sized to the 227 KB of
+    // shared memory and 512 TMEM columns
     if (q->D == 64)
-        return diag ? launch_band_bwd<64, 4, 3, 2, 2, 2>(q, k, v, out, lse, dout, g, scale, dq,
-                                                         dk, dv, delta, s)
-                    : launch_band_bwd<64, 4, 3, 0, 2, 2>(q, k, v, out, lse, dout, g, scale, dq,
-                                                         dk, dv, delta, s);
-    return launch_band_bwd<128, 4, 3, 0, 2, 1>(q, k, v, out, lse, dout, g, scale, dq, dk, dv,
-                                               delta, s);
+        return diag ? launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0>(q, k, v, out, lse, dout, g,
+                                                                scale, dq, dk, dv, delta, s)
+                    : launch_band_bwd<64, 2, 32, 2, 4, 4, 0, 0>(q, k, v, out, lse, dout, g,
+                                                                scale, dq, dk, dv, delta, s);
+    // D = 128: one pipeline, P^T / dS^T and dS in shared memory
+    return launch_band_bwd<128, 1, 64, 2, 3, 3, 0, 1>(q, k, v, out, lse, dout, g, scale, dq, dk,
+                                                      dv, delta, s);
 }

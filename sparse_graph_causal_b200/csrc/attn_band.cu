@@ -442,12 +442,13 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
 
             // --- diagonal blocks: q row from the Q tile, one key/value row per
-            // block; fp32 pairs (f32x2 FMA), running max rescaled lazily (only
-            // when it grows by more than 2^8, as in the band blocks)
+            // block; bf16 x bf16 -> fp32 FMAs (exact products), p rounded to
+            // bf16 for the weighted sum as the band path's P is; running max
+            // rescaled lazily (only when it grows by more than 2^8)
             {
-                uint64_t acc2[D / 2];
+                float acc[D];
 #pragma unroll
-                for (int x = 0; x < D / 2; ++x) acc2[x] = 0ull;
+                for (int x = 0; x < D; ++x) acc[x] = 0.f;
                 if (DS > 0 && nd > 0) {
                     ok = wait(p, L::bQFull, (uint32_t)(lt & 1));
                     // Structured blocks are swizzled like Q: q in logical
@@ -455,7 +456,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     // swizzled address gives chunk c ^ (r & 7), which pairs with
                     // the physical (unpermuted-address) chunks of the Q row; the
                     // accumulator is then in that permuted order (undone below).
-                    uint64_t q2[D / 2];
+                    uint32_t qw[D / 2];
                     if (ok) {
 #pragma unroll
                         for (int c = 0; c < D / 8; ++c) {
@@ -464,10 +465,10 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                                 (a.kind == 0 ? tc::sw128_off(r, c & 7)
                                              : (uint32_t)r * 128u + ((c & 7) << 4));
                             const uint4 w4 = *(const uint4 *)(pm + L::pQ + qoff);
-                            q2[4 * c] = tc::bf2_to_f2(w4.x);
-                            q2[4 * c + 1] = tc::bf2_to_f2(w4.y);
-                            q2[4 * c + 2] = tc::bf2_to_f2(w4.z);
-                            q2[4 * c + 3] = tc::bf2_to_f2(w4.w);
+                            qw[4 * c] = w4.x;
+                            qw[4 * c + 1] = w4.y;
+                            qw[4 * c + 2] = w4.z;
+                            qw[4 * c + 3] = w4.w;
                         }
                     }
                     int32_t resid = 0;
@@ -489,44 +490,47 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         if (valid) {
                             const uint8_t *kr = pm + L::pDK + st * L::kQTile;
                             const uint8_t *vr = pm + L::pDV + st * L::kQTile;
-                            // four independent partial sums (short dependency chains)
-                            uint64_t sp0 = 0ull, sp1 = 0ull, sp2 = 0ull, sp3 = 0ull;
+                            // eight independent partial sums (short dependency chains)
+                            float sp[8];
+#pragma unroll
+                            for (int x = 0; x < 8; ++x) sp[x] = 0.f;
 #pragma unroll
                             for (int c = 0; c < D / 8; ++c) {
                                 const uint4 w4 = *(const uint4 *)(kr + (c >> 3) * (BM * 128) +
                                                                   tc::sw128_off(r, c & 7));
-                                sp0 = tc::ffma2(q2[4 * c], tc::bf2_to_f2(w4.x), sp0);
-                                sp1 = tc::ffma2(q2[4 * c + 1], tc::bf2_to_f2(w4.y), sp1);
-                                sp2 = tc::ffma2(q2[4 * c + 2], tc::bf2_to_f2(w4.z), sp2);
-                                sp3 = tc::ffma2(q2[4 * c + 3], tc::bf2_to_f2(w4.w), sp3);
+                                const uint32_t kw[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    sp[2 * e] = tc::fma_bf_lo(qw[4 * c + e], kw[e], sp[2 * e]);
+                                    sp[2 * e + 1] =
+                                        tc::fma_bf_hi(qw[4 * c + e], kw[e], sp[2 * e + 1]);
+                                }
                             }
-                            const float s = ((tc::f2lo(sp0) + tc::f2hi(sp0)) +
-                                             (tc::f2lo(sp1) + tc::f2hi(sp1)) +
-                                             ((tc::f2lo(sp2) + tc::f2hi(sp2)) +
-                                              (tc::f2lo(sp3) + tc::f2hi(sp3)))) *
+                            const float s = (((sp[0] + sp[1]) + (sp[2] + sp[3])) +
+                                             ((sp[4] + sp[5]) + (sp[6] + sp[7]))) *
                                             c2;
                             if (s > m_run + kRescaleThreshold) {
                                 const float al = tc::ex2(m_run - s);  // 0 on the first edge
-                                const uint64_t al2 = tc::f2pack(al, al);
 #pragma unroll
-                                for (int x = 0; x < D / 2; ++x) acc2[x] = tc::fmul2(acc2[x], al2);
+                                for (int x = 0; x < D; ++x) acc[x] *= al;
                                 l_run *= al;
                                 m_run = s;
                             }
                             const float pr = tc::ex2(s - m_run);
                             l_run += pr;
-                            const uint64_t p2 = tc::f2pack(pr, pr);
+                            const uint32_t p2 = tc::pack_bf16x2(pr, pr);
 #pragma unroll
                             for (int c = 0; c < D / 8; ++c) {
                                 const uint4 w4 = *(const uint4 *)(vr + (c >> 3) * (BM * 128) +
                                                                   tc::sw128_off(r, c & 7));
-                                acc2[4 * c] = tc::ffma2(p2, tc::bf2_to_f2(w4.x), acc2[4 * c]);
-                                acc2[4 * c + 1] =
-                                    tc::ffma2(p2, tc::bf2_to_f2(w4.y), acc2[4 * c + 1]);
-                                acc2[4 * c + 2] =
-                                    tc::ffma2(p2, tc::bf2_to_f2(w4.z), acc2[4 * c + 2]);
-                                acc2[4 * c + 3] =
-                                    tc::ffma2(p2, tc::bf2_to_f2(w4.w), acc2[4 * c + 3]);
+                                const uint32_t vw[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    acc[8 * c + 2 * e] =
+                                        tc::fma_bf_lo(p2, vw[e], acc[8 * c + 2 * e]);
+                                    acc[8 * c + 2 * e + 1] =
+                                        tc::fma_bf_hi(p2, vw[e], acc[8 * c + 2 * e + 1]);
+                                }
                             }
                         }
                         const bool hold = (a.kind == 1) && (d == nd - 1);
@@ -545,25 +549,27 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         tc::mbar_arrive(bar(p, L::bGroup));
                         if (!wait(p, L::bGroup, group_uses & 1)) ok = false;
                         ++group_uses;
-                        uint64_t *scr =
-                            (uint64_t *)(pm + (r < 64 ? L::pDK : L::pDV) + st * L::kQTile) +
-                            (size_t)(r & 63) * 32 * (D / 64);
+                        float *scr = (float *)(pm + (r < 64 ? L::pDK : L::pDV) + st * L::kQTile) +
+                                     (size_t)(r & 63) * D;
 #pragma unroll
                         for (int hh = 0; hh < D / 64; ++hh) {
 #pragma unroll
                             for (int tt = 0; tt < 8; ++tt) {
                                 const int lc = tt ^ (r & 7);
-                                const uint64_t *src = acc2 + 32 * hh + 4 * tt;
-                                *(ulonglong2 *)(scr + 4 * lc) = make_ulonglong2(src[0], src[1]);
-                                *(ulonglong2 *)(scr + 4 * lc + 2) = make_ulonglong2(src[2], src[3]);
+                                const float *src = acc + 64 * hh + 8 * tt;
+                                *(float4 *)(scr + 8 * lc) = make_float4(src[0], src[1], src[2], src[3]);
+                                *(float4 *)(scr + 8 * lc + 4) =
+                                    make_float4(src[4], src[5], src[6], src[7]);
                             }
 #pragma unroll
                             for (int tt = 0; tt < 16; ++tt) {
-                                const ulonglong2 f = *(const ulonglong2 *)(scr + 2 * tt);
-                                acc2[32 * hh + 2 * tt] = f.x;
-                                acc2[32 * hh + 2 * tt + 1] = f.y;
+                                const float4 f = *(const float4 *)(scr + 4 * tt);
+                                acc[64 * hh + 4 * tt] = f.x;
+                                acc[64 * hh + 4 * tt + 1] = f.y;
+                                acc[64 * hh + 4 * tt + 2] = f.z;
+                                acc[64 * hh + 4 * tt + 3] = f.w;
                             }
-                            scr += 32;
+                            scr += 64;
                         }
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
@@ -578,10 +584,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 for (int c = 0; c < D; c += 32) {
                     uint32_t w[32];
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        w[2 * x] = __float_as_uint(tc::f2lo(acc2[c / 2 + x]));
-                        w[2 * x + 1] = __float_as_uint(tc::f2hi(acc2[c / 2 + x]));
-                    }
+                    for (int x = 0; x < 32; ++x) w[x] = __float_as_uint(acc[c + x]);
                     tc::tmem_st32(tO + c, w);
                 }
                 tc::tmem_st_wait();

@@ -95,127 +95,125 @@ __device__ __forceinline__ void load_row_packed(const uint8_t *tile, int rows, i
     }
 }
 
-// ---- fp32-pair versions (f32x2 FMA): a row of D values as D/2 pairs
-// (elements 2e, 2e+1), four independent partial sums in the dot products.
+// ---- bf16 x bf16 -> fp32 FMAs (exact products, one rounding per add):
+// dot products with eight independent partial sums, axpys with the scalar
+// rounded to bf16 (as the band path rounds P and dS for its MMAs).
 
-__device__ __forceinline__ float sum4_f2(uint64_t s0, uint64_t s1, uint64_t s2, uint64_t s3) {
-    return ((tc::f2lo(s0) + tc::f2hi(s0)) + (tc::f2lo(s1) + tc::f2hi(s1))) +
-           ((tc::f2lo(s2) + tc::f2hi(s2)) + (tc::f2lo(s3) + tc::f2hi(s3)));
+__device__ __forceinline__ float sum8(const float *s) {
+    return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
 }
 
 // a . b, both rows of swizzled tiles in shared memory (row r of each).
 template <int D>
-__device__ __forceinline__ float dot2_smem_smem(const uint8_t *ta, const uint8_t *tb, int rows,
-                                                int r) {
-    uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull, s3 = 0ull;
+__device__ __forceinline__ float dot_bf_smem_smem(const uint8_t *ta, const uint8_t *tb, int rows,
+                                                  int r) {
+    float sp[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) sp[x] = 0.f;
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
         const uint4 x = *(const uint4 *)(ta + tile_off(rows, r, c));
         const uint4 y = *(const uint4 *)(tb + tile_off(rows, r, c));
-        s0 = tc::ffma2(tc::bf2_to_f2(x.x), tc::bf2_to_f2(y.x), s0);
-        s1 = tc::ffma2(tc::bf2_to_f2(x.y), tc::bf2_to_f2(y.y), s1);
-        s2 = tc::ffma2(tc::bf2_to_f2(x.z), tc::bf2_to_f2(y.z), s2);
-        s3 = tc::ffma2(tc::bf2_to_f2(x.w), tc::bf2_to_f2(y.w), s3);
+        const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sp[2 * e] = tc::fma_bf_lo(xa[e], yb[e], sp[2 * e]);
+            sp[2 * e + 1] = tc::fma_bf_hi(xa[e], yb[e], sp[2 * e + 1]);
+        }
     }
-    return sum4_f2(s0, s1, s2, s3);
+    return sum8(sp);
 }
 
 // a . b, a = row r of a swizzled tile read in physical chunk order, b = row r
-// of an unswizzled gathered tile read at the swizzled address.
+// of an unswizzled gathered tile read at the swizzled address (both give
+// logical chunk t ^ (r & 7) at step t).
 template <int D>
-__device__ __forceinline__ float dot2_phys_gathered(const uint8_t *ta, const uint8_t *tb, int rows,
-                                                    int r) {
-    uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull, s3 = 0ull;
+__device__ __forceinline__ float dot_bf_phys_gathered(const uint8_t *ta, const uint8_t *tb,
+                                                      int rows, int r) {
+    float sp[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) sp[x] = 0.f;
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
         const uint4 x = *(const uint4 *)(ta + (c >> 3) * (rows * 128) + r * 128 + ((c & 7) << 4));
         const uint4 y = *(const uint4 *)(tb + tile_off(rows, r, c));
-        s0 = tc::ffma2(tc::bf2_to_f2(x.x), tc::bf2_to_f2(y.x), s0);
-        s1 = tc::ffma2(tc::bf2_to_f2(x.y), tc::bf2_to_f2(y.y), s1);
-        s2 = tc::ffma2(tc::bf2_to_f2(x.z), tc::bf2_to_f2(y.z), s2);
-        s3 = tc::ffma2(tc::bf2_to_f2(x.w), tc::bf2_to_f2(y.w), s3);
+        const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sp[2 * e] = tc::fma_bf_lo(xa[e], yb[e], sp[2 * e]);
+            sp[2 * e + 1] = tc::fma_bf_hi(xa[e], yb[e], sp[2 * e + 1]);
+        }
     }
-    return sum4_f2(s0, s1, s2, s3);
+    return sum8(sp);
 }
 
-// a . b, a already unpacked to pairs (chunk c in a2[4c .. 4c+3]), b row r of
-// a tile read at the swizzled address.
+// a . b, a packed bf16 pairs in registers (chunk c in a[4c .. 4c+3]), b row r
+// of a tile read at the swizzled address.
 template <int D>
-__device__ __forceinline__ float dot2_reg_smem(const uint64_t *a2, const uint8_t *tile, int rows,
-                                               int r) {
-    uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull, s3 = 0ull;
+__device__ __forceinline__ float dot_bf_reg_smem(const uint32_t *a, const uint8_t *tile, int rows,
+                                                 int r) {
+    float sp[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) sp[x] = 0.f;
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
         const uint4 y = *(const uint4 *)(tile + tile_off(rows, r, c));
-        s0 = tc::ffma2(a2[4 * c], tc::bf2_to_f2(y.x), s0);
-        s1 = tc::ffma2(a2[4 * c + 1], tc::bf2_to_f2(y.y), s1);
-        s2 = tc::ffma2(a2[4 * c + 2], tc::bf2_to_f2(y.z), s2);
-        s3 = tc::ffma2(a2[4 * c + 3], tc::bf2_to_f2(y.w), s3);
+        const uint32_t yb[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sp[2 * e] = tc::fma_bf_lo(a[4 * c + e], yb[e], sp[2 * e]);
+            sp[2 * e + 1] = tc::fma_bf_hi(a[4 * c + e], yb[e], sp[2 * e + 1]);
+        }
     }
-    return sum4_f2(s0, s1, s2, s3);
+    return sum8(sp);
 }
 
-// a . b, a packed bf16 pairs in registers, b row r of a tile.
+// acc += bf16(a) * (row r of a tile).
 template <int D>
-__device__ __forceinline__ float dot2_packed_smem(const uint32_t *a, const uint8_t *tile, int rows,
-                                                  int r) {
-    uint64_t s0 = 0ull, s1 = 0ull, s2 = 0ull, s3 = 0ull;
+__device__ __forceinline__ void axpy_bf_smem(float *acc, float a, const uint8_t *tile, int rows,
+                                             int r) {
+    const uint32_t a2 = tc::pack_bf16x2(a, a);
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
         const uint4 y = *(const uint4 *)(tile + tile_off(rows, r, c));
-        s0 = tc::ffma2(tc::bf2_to_f2(a[4 * c]), tc::bf2_to_f2(y.x), s0);
-        s1 = tc::ffma2(tc::bf2_to_f2(a[4 * c + 1]), tc::bf2_to_f2(y.y), s1);
-        s2 = tc::ffma2(tc::bf2_to_f2(a[4 * c + 2]), tc::bf2_to_f2(y.z), s2);
-        s3 = tc::ffma2(tc::bf2_to_f2(a[4 * c + 3]), tc::bf2_to_f2(y.w), s3);
-    }
-    return sum4_f2(s0, s1, s2, s3);
-}
-
-// acc2 += a * (row r of a tile), pairs.
-template <int D>
-__device__ __forceinline__ void axpy2_smem(uint64_t *acc2, float a, const uint8_t *tile, int rows,
-                                           int r) {
-    const uint64_t a2 = tc::f2pack(a, a);
+        const uint32_t yb[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        const uint4 y = *(const uint4 *)(tile + tile_off(rows, r, c));
-        acc2[4 * c] = tc::ffma2(a2, tc::bf2_to_f2(y.x), acc2[4 * c]);
-        acc2[4 * c + 1] = tc::ffma2(a2, tc::bf2_to_f2(y.y), acc2[4 * c + 1]);
-        acc2[4 * c + 2] = tc::ffma2(a2, tc::bf2_to_f2(y.z), acc2[4 * c + 2]);
-        acc2[4 * c + 3] = tc::ffma2(a2, tc::bf2_to_f2(y.w), acc2[4 * c + 3]);
+        for (int e = 0; e < 4; ++e) {
+            acc[8 * c + 2 * e] = tc::fma_bf_lo(a2, yb[e], acc[8 * c + 2 * e]);
+            acc[8 * c + 2 * e + 1] = tc::fma_bf_hi(a2, yb[e], acc[8 * c + 2 * e + 1]);
+        }
     }
 }
 
-// acc2 holds chunk t at logical chunk t ^ (r & 7) (per 64-column half): put it
+// acc holds chunk t at logical chunk t ^ (r & 7) (per 64-column half): put it
 // back in logical order through a D-float scratch row in shared memory.
 template <int D>
-__device__ __forceinline__ void unpermute_row2(uint64_t *acc2, float *scr_row, int r) {
-    uint64_t *scr = (uint64_t *)scr_row;
+__device__ __forceinline__ void unpermute_row(float *acc, float *scr_row, int r) {
 #pragma unroll
     for (int t = 0; t < D / 8; ++t) {
         const int lc = (t & ~7) | ((t & 7) ^ (r & 7));
-        *(ulonglong2 *)(scr + 4 * lc) = make_ulonglong2(acc2[4 * t], acc2[4 * t + 1]);
-        *(ulonglong2 *)(scr + 4 * lc + 2) = make_ulonglong2(acc2[4 * t + 2], acc2[4 * t + 3]);
+        *(float4 *)(scr_row + 8 * lc) =
+            make_float4(acc[8 * t], acc[8 * t + 1], acc[8 * t + 2], acc[8 * t + 3]);
+        *(float4 *)(scr_row + 8 * lc + 4) =
+            make_float4(acc[8 * t + 4], acc[8 * t + 5], acc[8 * t + 6], acc[8 * t + 7]);
     }
-    __syncwarp();
 #pragma unroll
     for (int t = 0; t < D / 4; ++t) {
-        const ulonglong2 f = *(const ulonglong2 *)(scr + 2 * t);
-        acc2[2 * t] = f.x;
-        acc2[2 * t + 1] = f.y;
+        const float4 f = *(const float4 *)(scr_row + 4 * t);
+        acc[4 * t] = f.x;
+        acc[4 * t + 1] = f.y;
+        acc[4 * t + 2] = f.z;
+        acc[4 * t + 3] = f.w;
     }
 }
 
 template <int D>
-__device__ __forceinline__ void tmem_store_row2(uint32_t taddr, const uint64_t *acc2) {
+__device__ __forceinline__ void tmem_store_row(uint32_t taddr, const float *acc) {
 #pragma unroll
     for (int c = 0; c < D; c += 32) {
         uint32_t w[32];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-            w[2 * x] = __float_as_uint(tc::f2lo(acc2[c / 2 + x]));
-            w[2 * x + 1] = __float_as_uint(tc::f2hi(acc2[c / 2 + x]));
-        }
+        for (int x = 0; x < 32; ++x) w[x] = __float_as_uint(acc[c + x]);
         tc::tmem_st32(taddr + c, w);
     }
 }
@@ -648,33 +646,30 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             {
                 uint32_t dor[D / 2];
                 load_row_packed<D>(pm + L::pDO, BM, r, dor);
-                uint64_t d0 = 0ull, d1 = 0ull, d2 = 0ull, d3 = 0ull;
+                float sp[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) sp[x] = 0.f;
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
-                    d0 = tc::ffma2(tc::bf2_to_f2(dor[4 * c]), tc::bf2_to_f2(orow4[c].x), d0);
-                    d1 = tc::ffma2(tc::bf2_to_f2(dor[4 * c + 1]), tc::bf2_to_f2(orow4[c].y), d1);
-                    d2 = tc::ffma2(tc::bf2_to_f2(dor[4 * c + 2]), tc::bf2_to_f2(orow4[c].z), d2);
-                    d3 = tc::ffma2(tc::bf2_to_f2(dor[4 * c + 3]), tc::bf2_to_f2(orow4[c].w), d3);
+                    const uint32_t ow[4] = {orow4[c].x, orow4[c].y, orow4[c].z, orow4[c].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        sp[2 * e] = tc::fma_bf_lo(dor[4 * c + e], ow[e], sp[2 * e]);
+                        sp[2 * e + 1] = tc::fma_bf_hi(dor[4 * c + e], ow[e], sp[2 * e + 1]);
+                    }
                 }
-                Delta = sum4_f2(d0, d1, d2, d3);
+                Delta = sum8(sp);
             }
             if (row_ok) a.delta[grow] = Delta;
-            // diagonal blocks (fp32 pairs)
-            uint64_t acc2[D / 2];
+            // diagonal blocks
+            float acc[D];
 #pragma unroll
-            for (int x = 0; x < D / 2; ++x) acc2[x] = 0ull;
+            for (int x = 0; x < D; ++x) acc[x] = 0.f;
             if (DS > 0 && nd > 0) {
                 if (a.kind == 0) {
                     // distance links: swizzled tiles, q in logical chunk order
-                    uint64_t q2[D / 2];
-#pragma unroll
-                    for (int c = 0; c < D / 8; ++c) {
-                        const uint4 x = *(const uint4 *)(pm + L::pQ + tile_off(BM, r, c));
-                        q2[4 * c] = tc::bf2_to_f2(x.x);
-                        q2[4 * c + 1] = tc::bf2_to_f2(x.y);
-                        q2[4 * c + 2] = tc::bf2_to_f2(x.z);
-                        q2[4 * c + 3] = tc::bf2_to_f2(x.w);
-                    }
+                    uint32_t qw[D / 2];
+                    load_row_packed<D>(pm + L::pQ, BM, r, qw);
                     for (int d = 0; d < nd; ++d) {
                         const int st = (int)(dc % DSX);
                         if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
@@ -685,10 +680,10 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                             const uint8_t *kt = pm + L::pDK + st * L::kRow;
                             const uint8_t *vt = pm + L::pDV + st * L::kRow;
                             const float pr =
-                                tc::ex2(fmaf(dot2_reg_smem<D>(q2, kt, BM, r), c2, -lse2));
+                                tc::ex2(fmaf(dot_bf_reg_smem<D>(qw, kt, BM, r), c2, -lse2));
                             const float ds =
-                                pr * (dot2_smem_smem<D>(pm + L::pDO, vt, BM, r) - Delta);
-                            axpy2_smem<D>(acc2, ds, kt, BM, r);
+                                pr * (dot_bf_smem_smem<D>(pm + L::pDO, vt, BM, r) - Delta);
+                            axpy_bf_smem<D>(acc, ds, kt, BM, r);
                         }
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
@@ -710,10 +705,10 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                             const uint8_t *kt = pm + L::pDK + st * L::kRow;
                             const uint8_t *vt = pm + L::pDV + st * L::kRow;
                             const float pr = tc::ex2(
-                                fmaf(dot2_phys_gathered<D>(pm + L::pQ, kt, BM, r), c2, -lse2));
+                                fmaf(dot_bf_phys_gathered<D>(pm + L::pQ, kt, BM, r), c2, -lse2));
                             const float ds =
-                                pr * (dot2_phys_gathered<D>(pm + L::pDO, vt, BM, r) - Delta);
-                            axpy2_smem<D>(acc2, ds, kt, BM, r);
+                                pr * (dot_bf_phys_gathered<D>(pm + L::pDO, vt, BM, r) - Delta);
+                            axpy_bf_smem<D>(acc, ds, kt, BM, r);
                         }
                         if (d < nd - 1) {  // the last stage is released after the unpermute
                             __syncwarp();
@@ -731,7 +726,7 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                         ++group_uses;
                         float *scr = (float *)(pm + (r < 64 ? L::pDK : L::pDV) + st * L::kRow) +
                                      (size_t)(r & 63) * D;
-                        unpermute_row2<D>(acc2, scr, r);
+                        unpermute_row<D>(acc, scr, r);
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
                     }
@@ -741,7 +736,7 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             // this warp is done reading Q and dO of the tile
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(p, L::bQEmpty));
-            tmem_store_row2<D>(tDQ, acc2);
+            tmem_store_row<D>(tDQ, acc);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
@@ -1204,9 +1199,9 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             if (!wait(p, L::bKVFull, (uint32_t)(lt & 1))) break;
             // diagonal blocks (fp32 pairs); lse and Delta of the linked query
             // are loaded one block ahead
-            uint64_t adk2[D / 2], adv2[D / 2];
+            float adk[D], adv[D];
 #pragma unroll
-            for (int x = 0; x < D / 2; ++x) adk2[x] = adv2[x] = 0ull;
+            for (int x = 0; x < D; ++x) adk[x] = adv[x] = 0.f;
             if (DS > 0 && nd > 0) {
                 const int off_first = a.n_off - nd;
                 int64_t rs = 0, nb = 0, resid = 0;
@@ -1241,18 +1236,18 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                         const uint8_t *dt = pm + L::pDDO + st * L::kRow;
                         float sdot, dpdot;
                         if (a.kind == 0) {
-                            sdot = dot2_smem_smem<D>(qt, pm + L::pK, BM, r);
-                            dpdot = dot2_smem_smem<D>(dt, pm + L::pV, BM, r);
+                            sdot = dot_bf_smem_smem<D>(qt, pm + L::pK, BM, r);
+                            dpdot = dot_bf_smem_smem<D>(dt, pm + L::pV, BM, r);
                         } else {
                             // CSR gathers are unswizzled: the key's k and v rows
                             // read in physical chunk order pair with them
-                            sdot = dot2_phys_gathered<D>(pm + L::pK, qt, BM, r);
-                            dpdot = dot2_phys_gathered<D>(pm + L::pV, dt, BM, r);
+                            sdot = dot_bf_phys_gathered<D>(pm + L::pK, qt, BM, r);
+                            dpdot = dot_bf_phys_gathered<D>(pm + L::pV, dt, BM, r);
                         }
                         const float pr = tc::ex2(fmaf(sdot, c2, -lse_cur * kLog2e));
                         const float ds = pr * (dpdot - del_cur);
-                        axpy2_smem<D>(adv2, pr, dt, BM, r);
-                        axpy2_smem<D>(adk2, ds, qt, BM, r);
+                        axpy_bf_smem<D>(adv, pr, dt, BM, r);
+                        axpy_bf_smem<D>(adk, ds, qt, BM, r);
                     }
                     if (a.kind == 0 || d < nd - 1) {  // CSR: last stage released below
                         __syncwarp();
@@ -1274,8 +1269,8 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                     ++group_uses;
                     float *scr = (float *)(pm + (r < 64 ? L::pDQ : L::pDDO) + st * L::kRow) +
                                  (size_t)(r & 63) * D;
-                    unpermute_row2<D>(adv2, scr, r);
-                    unpermute_row2<D>(adk2, scr, r);
+                    unpermute_row<D>(adv, scr, r);
+                    unpermute_row<D>(adk, scr, r);
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
                 }
@@ -1284,8 +1279,8 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             // this warp is done reading K and V of the tile
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(p, L::bKVEmpty));
-            tmem_store_row2<D>(tDV, adv2);
-            tmem_store_row2<D>(tDK, adk2);
+            tmem_store_row<D>(tDV, adv);
+            tmem_store_row<D>(tDK, adk);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();

@@ -328,6 +328,26 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Mixed-precision FMA, d = a * b + c: a and b are the low (lo) or high (hi)
+// bf16 halves of a bf16-pair word, c and d fp32; the product is exact and the
+// sum rounded once, as an fp32 FMA on the converted values would give.
+__device__ __forceinline__ float fma_bf_lo(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float fma_bf_hi(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %3;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+
 // Per-warpgroup register budgets (all four warps of a warpgroup execute it).
 // `dec` returns registers to the CTA's pool, `inc` waits until the pool holds
 // enough: the launch's registers (threads x registers per thread) must cover

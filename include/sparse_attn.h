@@ -124,8 +124,11 @@ sa_status sparse_attn_graph_destroy(sa_graph g);
 sa_status sparse_attn_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v, sa_graph g,
                           float scale, sa_tensor *out, float *lse, void *stream);
 
-/* Bytes of device workspace sparse_attn_bwd needs for these shapes
- * (4 * B * H * T rounded up, for Delta_i = dO_i . out_i in fp32). */
+/* Bytes of device workspace sparse_attn_bwd needs for these shapes and this
+ * graph: 4 * B * H * T (Delta_i = dO_i . out_i in fp32) and, for a
+ * structured graph with n distance links, 8 * n * B * H * T more (the
+ * probability and dS of every distance edge, computed once by the dQ pass and
+ * reused by the dK/dV pass), each part rounded up to 256 bytes. */
 size_t sparse_attn_bwd_workspace_size(const sa_tensor *q, sa_graph g);
 
 /* Backward of sparse_attn_fwd for the upstream gradient dout.  out and lse

@@ -54,6 +54,9 @@ struct BwdArgs {
     const __nv_bfloat16 *o;        // forward output (Delta)
     const float *lse;
     float *delta;
+    // Optional cache of (p, dS) per distance edge, written by dQ, read by
+    // dK/dV: [distance index][b*h][query], fp32 pairs; null to recompute
+    float2 *pds;
     __nv_bfloat16 *dq, *dk, *dv;
     float scale;
     float scale2;  // scale * log2(e)
@@ -683,6 +686,10 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                                 tc::ex2(fmaf(dot_bf_reg_smem<D>(qw, kt, BM, r), c2, -lse2));
                             const float ds =
                                 pr * (dot_bf_smem_smem<D>(pm + L::pDO, vt, BM, r) - Delta);
+                            if (a.pds)
+                                a.pds[((size_t)(a.n_off - nd + d) * (size_t)a.BH + (size_t)bh) *
+                                          (size_t)T +
+                                      (size_t)i] = make_float2(pr, ds);
                             axpy_bf_smem<D>(acc, ds, kt, BM, r);
                         }
                         __syncwarp();
@@ -1197,8 +1204,9 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
             if (!wait(p, L::bKVFull, (uint32_t)(lt & 1))) break;
-            // diagonal blocks (fp32 pairs); lse and Delta of the linked query
-            // are loaded one block ahead
+            // diagonal blocks: (p, dS) of each distance edge from the dQ
+            // kernel's cache, or recomputed from lse and Delta of the linked
+            // query; either pair is loaded one block ahead
             float adk[D], adv[D];
 #pragma unroll
             for (int x = 0; x < D; ++x) adk[x] = adv[x] = 0.f;
@@ -1219,13 +1227,20 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                     }
                     return d < resid ? (int64_t)a.rev_colidx[rs + nb + d] : -1;
                 };
+                const bool cached = a.kind == 0 && a.pds != nullptr;
+                auto edge_vals = [&](int d, int64_t i) -> float2 {
+                    if (i < 0) return make_float2(0.f, 0.f);
+                    if (cached)
+                        return a.pds[((size_t)(off_first + d) * (size_t)a.BH + (size_t)bh) *
+                                         (size_t)T +
+                                     (size_t)i];
+                    return make_float2(a.lse[gbh + i], a.delta[gbh + i]);
+                };
                 int64_t i_cur = query_of(0), i_nxt = query_of(1);
-                float lse_cur = i_cur >= 0 ? a.lse[gbh + i_cur] : 0.f;
-                float del_cur = i_cur >= 0 ? a.delta[gbh + i_cur] : 0.f;
+                float2 v_cur = edge_vals(0, i_cur);
                 for (int d = 0; d < nd; ++d) {
                     const int64_t i_n2 = query_of(d + 2);
-                    const float lse_nxt = i_nxt >= 0 ? a.lse[gbh + i_nxt] : 0.f;
-                    const float del_nxt = i_nxt >= 0 ? a.delta[gbh + i_nxt] : 0.f;
+                    const float2 v_nxt = edge_vals(d + 1, i_nxt);
                     const int st = (int)(dc % DSX);
                     if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
                         ok = false;
@@ -1234,18 +1249,24 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                     if (i_cur >= 0) {
                         const uint8_t *qt = pm + L::pDQ + st * L::kRow;
                         const uint8_t *dt = pm + L::pDDO + st * L::kRow;
-                        float sdot, dpdot;
-                        if (a.kind == 0) {
-                            sdot = dot_bf_smem_smem<D>(qt, pm + L::pK, BM, r);
-                            dpdot = dot_bf_smem_smem<D>(dt, pm + L::pV, BM, r);
+                        float pr, ds;
+                        if (cached) {
+                            pr = v_cur.x;
+                            ds = v_cur.y;
                         } else {
-                            // CSR gathers are unswizzled: the key's k and v rows
-                            // read in physical chunk order pair with them
-                            sdot = dot_bf_phys_gathered<D>(pm + L::pK, qt, BM, r);
-                            dpdot = dot_bf_phys_gathered<D>(pm + L::pV, dt, BM, r);
+                            float sdot, dpdot;
+                            if (a.kind == 0) {
+                                sdot = dot_bf_smem_smem<D>(qt, pm + L::pK, BM, r);
+                                dpdot = dot_bf_smem_smem<D>(dt, pm + L::pV, BM, r);
+                            } else {
+                                // CSR gathers are unswizzled: the key's k and v
+                                // rows read in physical chunk order pair with them
+                                sdot = dot_bf_phys_gathered<D>(pm + L::pK, qt, BM, r);
+                                dpdot = dot_bf_phys_gathered<D>(pm + L::pV, dt, BM, r);
+                            }
+                            pr = tc::ex2(fmaf(sdot, c2, -v_cur.x * kLog2e));
+                            ds = pr * (dpdot - v_cur.y);
                         }
-                        const float pr = tc::ex2(fmaf(sdot, c2, -lse_cur * kLog2e));
-                        const float ds = pr * (dpdot - del_cur);
                         axpy_bf_smem<D>(adv, pr, dt, BM, r);
                         axpy_bf_smem<D>(adk, ds, qt, BM, r);
                     }
@@ -1256,8 +1277,7 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                     ++dc;
                     i_cur = i_nxt;
                     i_nxt = i_n2;
-                    lse_cur = lse_nxt;
-                    del_cur = del_nxt;
+                    v_cur = v_nxt;
                 }
                 if (ok && a.kind == 1) {
                     // restore the logical order through the last stage once
@@ -1394,7 +1414,7 @@ template <int D, int NP, int BB, int SB, int BSQ, int BSK, int DS, int PS>
 sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_tensor *o, const float *lse, const sa_tensor *dout,
                           const sa_graph_s *g, float scale, sa_tensor *dq, sa_tensor *dk,
-                          sa_tensor *dv, float *delta, cudaStream_t s) {
+                          sa_tensor *dv, float *delta, void *pds, cudaStream_t s) {
     using LQ = LayoutDQ<D, NP, BB, SB, BSQ, DS, PS>;
     using LK = LayoutDKV<D, NP, BB, SB, BSK, DS, PS>;
     static_assert(LQ::kAlloc <= 232448 && LK::kAlloc <= 232448, "shared memory budget");
@@ -1440,6 +1460,7 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.o = (const __nv_bfloat16 *)o->ptr;
     a.lse = lse;
     a.delta = delta;
+    a.pds = (g->kind == 0 && g->n_off > 0) ? (float2 *)pds : nullptr;
     a.dq = (__nv_bfloat16 *)dq->ptr;
     a.dk = (__nv_bfloat16 *)dk->ptr;
     a.dv = (__nv_bfloat16 *)dv->ptr;
@@ -1479,17 +1500,17 @@ bool sa_band_bwd_supported(const sa_tensor *q, const sa_graph_s *g) {
 sa_status sa_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                       const sa_tensor *out, const float *lse, const sa_tensor *dout,
                       const sa_graph_s *g, const GraphView &, float scale, sa_tensor *dq,
-                      sa_tensor *dk, sa_tensor *dv, float *delta, cudaStream_t s) {
+                      sa_tensor *dk, sa_tensor *dv, float *delta, void *pds, cudaStream_t s) {
     const bool diag = (g->kind == 0) ? g->n_off > 0 : (g->max_resid > 0 || g->max_resid_rev > 0);
     // <D, pipelines, band block, S buffers, dQ ring stages, dK/dV ring stages,
     //  diagonal stages, shared-memory P/dS tiles>, sized to the 227 KB of
     // shared memory and 512 TMEM columns
     if (q->D == 64)
         return diag ? launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0>(q, k, v, out, lse, dout, g,
-                                                                scale, dq, dk, dv, delta, s)
+                                                                scale, dq, dk, dv, delta, pds, s)
                     : launch_band_bwd<64, 2, 32, 2, 4, 4, 0, 0>(q, k, v, out, lse, dout, g,
-                                                                scale, dq, dk, dv, delta, s);
+                                                                scale, dq, dk, dv, delta, pds, s);
     // D = 128: one pipeline, P^T / dS^T and dS in shared memory
     return launch_band_bwd<128, 1, 64, 2, 3, 3, 0, 1>(q, k, v, out, lse, dout, g, scale, dq, dk,
-                                                      dv, delta, s);
+                                                      dv, delta, pds, s);
 }

@@ -56,7 +56,8 @@ extern "C" sa_status sparse_attn_bwd_noalloc(const sa_tensor *q, const sa_tensor
     sa_status st = noalloc_scratch(&scratch);
     if (st != SA_OK) return st;
     // Delta is written in full by the dQ pass before the dK/dV pass reads it,
-    // so nothing in the array has to start at zero.
-    return sparse_attn_bwd(q, k, v, out, lse, dout, g, scale, dq, dk, dv, scratch,
-                           sizeof(float) * (size_t)SA_NOALLOC_MAX_ROWS, stream);
+    // so nothing in the array has to start at zero.  Without room for the
+    // distance-edge cache the dK/dV pass recomputes p and dS.
+    return sa_bwd_with_scratch(q, k, v, out, lse, dout, g, scale, dq, dk, dv, scratch, nullptr,
+                               stream);
 }

@@ -345,12 +345,46 @@ sa_status sparse_attn_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     return sa_gather_fwd(q, k, v, gv, scale, out, lse, s);
 }
 
-size_t sparse_attn_bwd_workspace_size(const sa_tensor *q, sa_graph g) {
-    (void)g;
-    if (!q || q->B < 1 || q->H < 1 || q->T < 1) return 0;
-    size_t n = sizeof(float) * (size_t)(q->B * q->H * q->T);
+// Workspace layout: Delta (fp32 per query row), then, for a structured graph
+// with distance links, the (p, dS) pair of every distance edge (8 bytes per
+// link per query row), each part 256-byte aligned.
+static size_t delta_bytes(const sa_tensor *q) {
+    const size_t n = sizeof(float) * (size_t)(q->B * q->H * q->T);
     return (n + 255) & ~(size_t)255;
 }
+static size_t edge_cache_bytes(const sa_tensor *q, sa_graph g) {
+    if (!g || g->kind != 0 || g->n_off < 1) return 0;
+    const size_t n = 2 * sizeof(float) * (size_t)g->n_off * (size_t)(q->B * q->H * q->T);
+    return (n + 255) & ~(size_t)255;
+}
+
+size_t sparse_attn_bwd_workspace_size(const sa_tensor *q, sa_graph g) {
+    if (!q || q->B < 1 || q->H < 1 || q->T < 1) return 0;
+    return delta_bytes(q) + edge_cache_bytes(q, g);
+}
+
+}  // extern "C"
+
+// C++ linkage: not part of the C ABI.
+sa_status sa_bwd_with_scratch(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                              const sa_tensor *out, const float *lse, const sa_tensor *dout,
+                              sa_graph g, float scale, sa_tensor *dq, sa_tensor *dk,
+                              sa_tensor *dv, float *delta, void *edge_cache, void *stream) {
+    sa_status st = check_common(q, g);
+    if (st != SA_OK) return st;
+    const sa_tensor *ts[] = {k, v, out, dout, dq, dk, dv};
+    for (const sa_tensor *t : ts)
+        if ((st = check_tensor(t, q)) != SA_OK) return st;
+    if (!lse || !aligned16(lse) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    const GraphView gv = make_view(g);
+    if (g_path.load() == SA_PATH_AUTO && sa_band_bwd_supported(q, g))
+        return sa_band_bwd(q, k, v, out, lse, dout, g, gv, scale, dq, dk, dv, delta, edge_cache,
+                           s);
+    return sa_gather_bwd(q, k, v, out, lse, dout, gv, scale, dq, dk, dv, delta, s);
+}
+
+extern "C" {
 
 sa_status sparse_attn_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_tensor *out, const float *lse, const sa_tensor *dout, sa_graph g,
@@ -358,19 +392,13 @@ sa_status sparse_attn_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
                           void *workspace, size_t ws_bytes, void *stream) {
     sa_status st = check_common(q, g);
     if (st != SA_OK) return st;
-    const sa_tensor *ts[] = {k, v, out, dout, dq, dk, dv};
-    for (const sa_tensor *t : ts)
-        if ((st = check_tensor(t, q)) != SA_OK) return st;
-    if (!lse || !aligned16(lse) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
         ws_bytes < sparse_attn_bwd_workspace_size(q, g))
         return SA_ERR_INVALID_ARG;
-    cudaStream_t s = as_stream(stream);
-    const GraphView gv = make_view(g);
-    float *delta = static_cast<float *>(workspace);
-    if (g_path.load() == SA_PATH_AUTO && sa_band_bwd_supported(q, g))
-        return sa_band_bwd(q, k, v, out, lse, dout, g, gv, scale, dq, dk, dv, delta, s);
-    return sa_gather_bwd(q, k, v, out, lse, dout, gv, scale, dq, dk, dv, delta, s);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *edge_cache = edge_cache_bytes(q, g) ? ws + delta_bytes(q) : nullptr;
+    return sa_bwd_with_scratch(q, k, v, out, lse, dout, g, scale, dq, dk, dv,
+                               reinterpret_cast<float *>(ws), edge_cache, stream);
 }
 
 }  // extern "C"

@@ -11,4 +11,4 @@ sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
 sa_status sa_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                       const sa_tensor *out, const float *lse, const sa_tensor *dout,
                       const sa_graph_s *g, const GraphView &gv, float scale, sa_tensor *dq,
-                      sa_tensor *dk, sa_tensor *dv, float *delta, cudaStream_t s);
+                      sa_tensor *dk, sa_tensor *dv, float *delta, void *pds, cudaStream_t s);

@@ -130,6 +130,12 @@ sa_status sa_graph_from_csr(sa_graph_s *g, const int64_t *rowptr, const int32_t 
 sa_status sa_gather_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                         const GraphView &gv, float scale, sa_tensor *out, float *lse,
                         cudaStream_t s);
+// Backward with caller-placed scratch: Delta (4 bytes per query row) and an
+// optional distance-edge cache (null: recompute); argument checks included.
+sa_status sa_bwd_with_scratch(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                              const sa_tensor *out, const float *lse, const sa_tensor *dout,
+                              sa_graph g, float scale, sa_tensor *dq, sa_tensor *dk,
+                              sa_tensor *dv, float *delta, void *edge_cache, void *stream);
 sa_status sa_gather_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                         const sa_tensor *out, const float *lse, const sa_tensor *dout,
                         const GraphView &gv, float scale, sa_tensor *dq, sa_tensor *dk,

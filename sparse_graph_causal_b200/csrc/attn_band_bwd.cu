@@ -996,7 +996,22 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                 tc::mbar_arrive(bar(p, L::bInfoFull + slot));
             }
             // band block bl (all lanes): lane 0 the TMA copies, every lane a
-            // share of lse (base 2) and Delta, zero past the end of the sequence
+            // share of lse (base 2) and Delta, zero past the end of the
+            // sequence; block bl+1's values are fetched into registers while
+            // the producer waits for the next free stage
+            constexpr int PL = BB / 32;  // values per lane
+            float pf_l[PL], pf_d[PL];
+            auto fetch_vals = [&](int bl) {
+#pragma unroll
+                for (int x = 0; x < PL; ++x) {
+                    const int64_t i = (int64_t)k0 + bl * BB + lane + 32 * x;
+                    const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
+                    const bool in = bl < n_band && i < T;
+                    pf_l[x] = in ? a.lse[gi] : 0.f;
+                    pf_d[x] = in ? a.delta[gi] : 0.f;
+                }
+            };
+            fetch_vals(0);
             auto load_blk = [&](int bl) -> bool {
                 const int st = (int)(bc % BS);
                 const uint32_t use = bc / BS;
@@ -1009,14 +1024,14 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                                     bar(p, L::bBFull + st));
                 }
                 float *ls = stage_lse(p, st), *dl = ls + BB;
-                for (int c = lane; c < BB; c += 32) {
-                    const int64_t i = (int64_t)qrow + c;
-                    const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
-                    ls[c] = i < T ? a.lse[gi] * kLog2e : 0.f;
-                    dl[c] = i < T ? a.delta[gi] : 0.f;
+#pragma unroll
+                for (int x = 0; x < PL; ++x) {
+                    ls[lane + 32 * x] = pf_l[x] * kLog2e;
+                    dl[lane + 32 * x] = pf_d[x];
                 }
                 tc::mbar_arrive(bar(p, L::bBFull + st));
                 ++bc;
+                fetch_vals(bl + 1);
                 return true;
             };
             const int n_pre = n_band < BS ? n_band : BS;

@@ -604,12 +604,6 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     break;
                 }
                 tc::tc_fence_after();
-                float s[BN];
-#pragma unroll
-                for (int c = 0; c < BN; c += 32)
-                    tc::tmem_ld32(tS + sb * BN + c, (uint32_t *)(s + c));
-                tc::tmem_ld_wait();
-
                 // mask: r <= u <= r+W-1 and key >= 0, with u = BN b + c, i.e.
                 // the column range [c_lo, c_hi] of this block.  Scores stay raw
                 // (the scale is folded into the exponent's FFMA); a masked raw
@@ -617,13 +611,33 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 const int32_t u0 = b * BN;
                 const bool need_mask =
                     (u0 < BM - 1) || (u0 + BN - 1 > W - 1) || (u0 + q0 < W - 1);
-                const bool pos = c2 >= 0.f;
-                const float ext = pos ? -INFINITY : INFINITY;
+                int c_lo = 0, c_hi = BN - 1;
                 if (need_mask) {
                     const int32_t lo = (r > W - 1 - q0) ? r : W - 1 - q0;
                     const int32_t hi = r + W - 1;
-                    const int c_lo = lo - u0 < 0 ? 0 : (lo - u0 > BN ? BN : lo - u0);
-                    const int c_hi = hi - u0 > BN - 1 ? BN - 1 : (hi - u0 < -1 ? -1 : hi - u0);
+                    c_lo = lo - u0 < 0 ? 0 : (lo - u0 > BN ? BN : lo - u0);
+                    c_hi = hi - u0 > BN - 1 ? BN - 1 : (hi - u0 < -1 ? -1 : hi - u0);
+                }
+                if (need_mask && __all_sync(0xffffffffu, c_lo > c_hi)) {
+                    // no row of this warp keeps a key of the block: P = 0
+                    uint32_t z[BN / 2];
+#pragma unroll
+                    for (int x = 0; x < BN / 2; ++x) z[x] = 0u;
+                    tc::tmem_st_n<BN / 2>(tS + sb * BN, z);
+                    tc::tmem_st_wait();
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(p, L::bPFull + sb));
+                    continue;
+                }
+                float s[BN];
+#pragma unroll
+                for (int c = 0; c < BN; c += 32)
+                    tc::tmem_ld32(tS + sb * BN + c, (uint32_t *)(s + c));
+                tc::tmem_ld_wait();
+                const bool pos = c2 >= 0.f;
+                const float ext = pos ? -INFINITY : INFINITY;
+                if (need_mask) {
 #pragma unroll
                     for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : ext;
                 }

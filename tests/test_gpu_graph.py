@@ -113,3 +113,24 @@ def test_csr_bad_rowptr_and_band(sa):
     with pytest.raises(sa.SparseAttentionError) as e:
         sa.sparse_attn_graph_build_csr(*a, band_hint=65)
     assert e.value.status == 2
+
+
+def test_bwd_workspace_size(sa):
+    """Delta (4 bytes per query row) plus, for a structured graph with n
+    distance links, the (p, dS) cache of its distance edges (8 n bytes per
+    query row), each part rounded up to 256 bytes; CSR graphs and graphs
+    without links need Delta only."""
+    def up(x):
+        return (x + 255) // 256 * 256
+
+    B, H, T, D = 2, 3, 4097, 64
+    q = torch.empty(B, H, T, D, dtype=torch.bfloat16, device="cuda")
+    rows = B * H * T
+    # window 32: links 2^0 .. 2^4 fall inside it, 2^5 and 2^9 remain
+    g = sa.sparse_attn_graph_build_structured(T, 32, [0, 3, 5, 9])
+    assert sa.sparse_attn_bwd_workspace_size(q, g) == up(4 * rows) + up(8 * 2 * rows)
+    g_band = sa.sparse_attn_graph_build_structured(T, 32, [])
+    assert sa.sparse_attn_bwd_workspace_size(q, g_band) == up(4 * rows)
+    rp, ci = synth.csr_random_rows(T, seed=5, window=16, n_random=2, n_global=2)
+    g_csr = sa.sparse_attn_graph_build_csr(torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda())
+    assert sa.sparse_attn_bwd_workspace_size(q, g_csr) == up(4 * rows)

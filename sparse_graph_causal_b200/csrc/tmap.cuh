@@ -15,6 +15,3 @@ bool sa_tmap_bf16_3d(CUtensorMap *m, const void *base, uint64_t D, uint64_t T, u
 // one-row boxes of 64 values, no swizzle: the map for 4-row TMA gathers.
 bool sa_tmap_bf16_rows(CUtensorMap *m, const void *base, uint64_t D, uint64_t rows);
 
-// fp32 [B*H, T] rows (lse, Delta): 2-D (x = T, y = B*H), box = box_x values of
-// one row, no swizzle, zero fill outside.
-bool sa_tmap_f32_2d(CUtensorMap *m, const void *base, uint64_t T, uint64_t BH, uint32_t box_x);

@@ -47,6 +47,12 @@ constexpr int BN = 64;              // keys per band block
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Distance blocks are prefetched into L2 this many blocks ahead of their
+// loads when K and V do not fit in L2 (long links then miss it, and the
+// two-stage ring alone keeps too few of their DRAM reads in flight); with
+// L2-resident K and V the prefetches are pure overhead and are skipped.
+constexpr int kPrefetchAhead = 4;
+constexpr double kL2ResidentBytes = 64.0 * 1024 * 1024;
 // Register budgets with two pipelines (384 threads launched at 168 each):
 // the producer warpgroup keeps 56 (72 when it also gathers diagonal blocks),
 // the softmax warpgroups take the rest.
@@ -63,6 +69,7 @@ struct FwdArgs {
     int32_t W;          // band width (structured window or verified CSR band)
     int32_t kind;       // 0 structured, 1 CSR
     int32_t n_off;
+    int32_t prefetch;              // distance blocks prefetched into L2 ahead (0: none)
     int64_t offs[SA_MAX_OFFSETS];  // distances (structured), descending
     const int64_t *rowptr;         // CSR
     const int32_t *colidx;
@@ -287,6 +294,15 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     if (!load_k(bl) || !load_v(bl)) okl = 0;
             }
             ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+            auto prefetch_blk = [&](int d) {
+                const int32_t krow = (int32_t)(g.q0 - a.offs[a.n_off - nd + d]);
+                for (int x = 0; x < D / 64; ++x) {
+                    tc::tma_prefetch_3d(&tkd, x * 64, krow, (int32_t)g.bh);
+                    tc::tma_prefetch_3d(&tvd, x * 64, krow, (int32_t)g.bh);
+                }
+            };
+            if (DS > 0 && a.kind == 0 && lane == 0)
+                for (int d = 0; d < nd && d < a.prefetch; ++d) prefetch_blk(d);
             for (int d = 0; ok && d < nd; ++d) {
                 const int st = (int)(dc % DSX);
                 const uint32_t use = dc / DSX;
@@ -307,6 +323,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                             tc::tma_load_3d(vdst + x * (BM * 128), &tvd, x * 64, krow,
                                             (int32_t)g.bh, bar(p, L::bDiagFull + st));
                         }
+                        if (d + a.prefetch < nd && a.prefetch > 0) prefetch_blk(d + a.prefetch);
                     }
                 } else {
                     // CSR slot d: 4-row TMA gathers of K and V rows
@@ -810,6 +827,7 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.W = g->W;
     a.kind = g->kind;
     a.n_off = g->kind == 0 ? g->n_off : 0;
+    a.prefetch = (double)BH * (double)T * D * 2 * 2 > kL2ResidentBytes ? kPrefetchAhead : 0;
     for (int x = 0; x < SA_MAX_OFFSETS; ++x) a.offs[x] = x < a.n_off ? g->offs[x] : 0;
     a.rowptr = g->rowptr;
     a.colidx = g->colidx;

@@ -180,6 +180,14 @@ sa_status sparse_attn_set_path(int32_t path);
  * check, SA_ERR_CUDA on a CUDA error, else SA_OK. */
 sa_status sparse_attn_check_device(void *stream);
 
+/* Diagnostic for the failure path above (the pages have no counterpart):
+ * enqueue on `stream` one warp that waits, with the attention kernels'
+ * bounded wait, on a barrier nothing completes, giving up after limit_ns
+ * (1 ms .. 2 s, else SA_ERR_INVALID_ARG).  It faults nothing: the next
+ * sparse_attn_check_device(stream) returns SA_ERR_DEVICE_TIMEOUT, clears the
+ * word, and the context stays usable. */
+sa_status sparse_attn_selftest_wait_timeout(int64_t limit_ns, void *stream);
+
 /* Description of the last CUDA failure this thread saw inside the library
  * (the failing call and CUDA's error name and string), "" if none.  The
  * pointer stays valid until the thread's next failing call. */

@@ -48,6 +48,7 @@ def _load():
         "sparse_attn_status_string": (ctypes.c_char_p, [st]),
         "sparse_attn_set_path": (st, [i32]),
         "sparse_attn_check_device": (st, [vp]),
+        "sparse_attn_selftest_wait_timeout": (st, [i64, vp]),
         "sparse_attn_launch_count": (i64, []),
         "sparse_attn_last_error_message": (ctypes.c_char_p, []),
         "sparse_attn_bwd_noalloc": (st, [P(SaTensor), P(SaTensor), P(SaTensor), P(SaTensor), vp,
@@ -278,6 +279,14 @@ def sparse_attn_set_path(path: int):
 
 def sparse_attn_check_device(stream=None):
     _check(_lib.sparse_attn_check_device(_stream(stream)), "sparse_attn_check_device")
+
+
+def sparse_attn_selftest_wait_timeout(limit_ns: int = 20_000_000, stream=None):
+    """Enqueue a wait that nothing completes and that gives up after
+    limit_ns; the next sparse_attn_check_device raises with status
+    SA_ERR_DEVICE_TIMEOUT."""
+    _check(_lib.sparse_attn_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "sparse_attn_selftest_wait_timeout")
 
 
 def sparse_attn_last_error_message() -> str:

@@ -14,6 +14,7 @@
 
 #include "sa_internal.cuh"
 #include "sa_band.cuh"
+#include "tc_common.cuh"
 
 namespace {
 
@@ -24,6 +25,21 @@ std::atomic<int> g_path{SA_PATH_AUTO};
 __device__ int g_device_error = 0;
 
 cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// One warp waits on an mbarrier that nothing arrives on, through the same
+// bounded wait the attention kernels use: after limit_ns it records
+// SA_DEVERR_TIMEOUT in the error word and returns.
+__global__ void selftest_wait_kernel(int *err, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t mb;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(tc::smem_u32(&mb), 1);
+        abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    __syncthreads();
+    tc::mbar_wait(tc::smem_u32(&mb), 0, &abort_flag, err, SA_DEVERR_TIMEOUT, limit_ns);
+}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -210,6 +226,16 @@ int32_t sparse_attn_profile_end(char *names, int32_t name_len, int32_t *launches
         if (total_ms) total_ms[k] = ms[k];
     }
     return n;
+}
+
+sa_status sparse_attn_selftest_wait_timeout(int64_t limit_ns, void *stream) {
+    if (limit_ns < 1000000 || limit_ns > 2000000000) return SA_ERR_INVALID_ARG;
+    int *err = sa_device_error_word();
+    if (!err) return SA_ERR_CUDA;
+    cudaStream_t s = as_stream(stream);
+    SA_LAUNCH("selftest_wait", s, selftest_wait_kernel<<<1, 32, 0, s>>>(err, (uint64_t)limit_ns));
+    SA_CUDA_TRY(cudaGetLastError());
+    return SA_OK;
 }
 
 sa_status sparse_attn_check_device(void *stream) {

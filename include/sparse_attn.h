@@ -146,8 +146,11 @@ sa_status sparse_attn_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
  * fixed device-memory plan (every byte reserved up front), or code inside an
  * allocator hook, where allocating again would re-enter the allocator.  The
  * pages have no counterpart of this call; it is a deployment convenience.
- * Same arguments and results as sparse_attn_bwd minus the workspace.  Its
- * scratch (Delta, 4 bytes per query row) is a fixed device array of
+ * Same arguments as sparse_attn_bwd minus the workspace, and the same results
+ * up to rounding: without room for the distance-edge cache its dK/dV pass
+ * recomputes p and dS of the distance links (bitwise reproducible run to run
+ * on its own).  Its scratch (Delta, 4 bytes per query row) is a fixed device
+ * array of
  * SA_NOALLOC_MAX_ROWS floats inside the library: every GPU that loads the
  * library holds it (4 MiB) until the process exits.  B*H*T above
  * SA_NOALLOC_MAX_ROWS returns SA_ERR_UNSUPPORTED before anything is enqueued.

@@ -150,9 +150,8 @@ sa_status sparse_attn_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
  * up to rounding: without room for the distance-edge cache its dK/dV pass
  * recomputes p and dS of the distance links (bitwise reproducible run to run
  * on its own).  Its scratch (Delta, 4 bytes per query row) is a fixed device
- * array of
- * SA_NOALLOC_MAX_ROWS floats inside the library: every GPU that loads the
- * library holds it (4 MiB) until the process exits.  B*H*T above
+ * array of SA_NOALLOC_MAX_ROWS floats inside the library: every GPU that
+ * loads the library holds it (4 MiB) until the process exits.  B*H*T above
  * SA_NOALLOC_MAX_ROWS returns SA_ERR_UNSUPPORTED before anything is enqueued.
  * Every call on a device shares the array (it keeps the last call's
  * contents, none of which must start at zero), so calls whose work overlaps

@@ -26,8 +26,18 @@ def to_oracle(t: torch.Tensor, dtype: str) -> np.ndarray:
     return t.numpy()
 
 
-def compare(got, ref: np.ndarray, dtype: str, what: str, scale_floor: float = 1e-6):
-    """got: torch tensor (any float dtype) or ndarray; ref: fp64 ndarray."""
+def compare(got, ref: np.ndarray, dtype: str, what: str, scale_floor: float = 1e-6,
+            unit_range: float | None = None):
+    """got: torch tensor (any float dtype) or ndarray; ref: fp64 ndarray.
+
+    unit_range: set for inputs far from unit scale.  The fixed max-abs bound
+    then gives way to the relative one (2^-5 of the largest |ref|, checked for
+    every case), and the mean-abs bound grows in proportion to max|ref| beyond
+    unit_range.  Two errors that any bf16-output implementation has grow with
+    the values: a result rounded to bf16 is off by up to 2^-8 of its size
+    (0.03 at |x| = 8), and Delta = dO . out must use the rounded out, which by
+    itself moves dq by 0.016-0.020 at |dq| = 5-6 with scores of standard
+    deviation 2 (fp64 emulation of that step alone)."""
     if isinstance(got, torch.Tensor):
         got = got.detach().float().cpu().numpy()
     got = np.asarray(got, dtype=np.float64)
@@ -43,8 +53,11 @@ def compare(got, ref: np.ndarray, dtype: str, what: str, scale_floor: float = 1e
     tol = TOL[dtype]
     mx, mean = float(err.max()), float(err.mean())
     rng = max(float(np.abs(ref[fin]).max()), scale_floor)
-    assert mx <= tol["max_abs"], f"{what}: max-abs {mx:.3e} > {tol['max_abs']}"
-    assert mean <= tol["mean_abs"], f"{what}: mean-abs {mean:.3e} > {tol['mean_abs']}"
+    grow = max(1.0, rng / unit_range) if unit_range else 1.0
+    if not unit_range:
+        assert mx <= tol["max_abs"], f"{what}: max-abs {mx:.3e} > {tol['max_abs']}"
+    assert mean <= tol["mean_abs"] * grow, \
+        f"{what}: mean-abs {mean:.3e} > {tol['mean_abs']} * {grow:.2f}"
     assert mx <= tol["rel"] * rng + 1e-7, f"{what}: max-abs {mx:.3e} > {tol['rel']} * {rng:.3e}"
     return dict(max_abs=mx, mean_abs=mean, range=rng)
 

@@ -35,6 +35,24 @@ MUTANTS = {
                                 "row[u++] = row[e];"),
     "lookahead_accepted": ("if ((int64_t)colidx[e] > i) return OR_LOOKAHEAD;",
                            "if ((int64_t)colidx[e] > i + 1) return OR_LOOKAHEAD;"),
+    "negative_key_accepted": ("if (colidx[e] < 0) return OR_NEGATIVE;",
+                              "if (colidx[e] < -1) return OR_NEGATIVE;"),
+    "link_before_start_clamped": ("if (j < 0) continue;          /* no position before the start */",
+                                  "if (j < 0) j = 0;"),
+    "repeated_exponent_counted": ("if (dup) continue;", "(void)dup;"),
+    "structured_row_unsorted": ("if (buf) qsort(buf, (size_t)cnt, sizeof(int32_t), cmp_i32);", ""),
+    "normalize_row_unsorted": ("qsort(row, (size_t)n, sizeof(int32_t), cmp_i32);", ""),
+    "reverse_descending": ("for (int64_t i = 0; i < T; ++i) /* ascending i keeps each list sorted */",
+                           "for (int64_t i = T - 1; i >= 0; --i)"),
+    "empty_row_lse_zero": ("*lse = -INFINITY;", "*lse = 0.0;"),
+    "lse_max_dropped": ("*lse = m + log(l);", "*lse = log(l);"),
+    "output_not_normalized": ("double p = exp(s[e] - m) / l;", "double p = exp(s[e] - m);"),
+    "delta_dropped": ("double ds = p * (dp - delta);", "double ds = p * dp;"),
+    "dq_value_for_key": ("dq[i * D + d] += scale * ds * kd[j * D + d];",
+                         "dq[i * D + d] += scale * ds * vd[j * D + d];"),
+    "dk_scale_dropped": ("dk[j * D + d] += scale * ds * qd[i * D + d];",
+                         "dk[j * D + d] += ds * qd[i * D + d];"),
+    "bwd_prob_without_lse": ("double p = exp(s[e] - lse);", "double p = exp(s[e]);"),
 }
 
 

@@ -82,6 +82,12 @@ class Oracle:
         L.oracle_attn_bwd.restype = ctypes.c_int
         L.oracle_attn_bwd.argtypes = [i64, i64, i32, ctypes.c_int, vp, vp, vp, vp, vp, vp, dbl,
                                       vp, vp, vp]
+        L.oracle_dist_fwd.restype = ctypes.c_int
+        L.oracle_dist_fwd.argtypes = [i64, i32, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp,
+                                      dbl, vp, vp]
+        L.oracle_dist_bwd.restype = ctypes.c_int
+        L.oracle_dist_bwd.argtypes = [i64, i64, i32, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp,
+                                      vp, vp, dbl, vp, vp, vp]
 
     # ---------------- graph ----------------
     def structured_nnz(self, T: int, W: int, exps) -> int:
@@ -188,6 +194,56 @@ class Oracle:
         if st:
             raise OracleError(STATUS[st])
         return dq, dk, dv
+
+
+    # ---------------- learned-coordinate (distance) scoring ----------------
+    @staticmethod
+    def _coords(x: np.ndarray, cdtype: str) -> np.ndarray:
+        x = np.ascontiguousarray(x, dtype=np.float32 if cdtype == "fp32" else np.float64)
+        assert x.ndim == 2 and x.shape[1] == 3, "coordinates are [n, 3]"
+        return x
+
+    def dist_fwd(self, a, c, v, rowptr, colidx, scale: float, dtype: str = "f64",
+                 cdtype: str = "f64"):
+        """s_ij = -scale * |a_i - c_j|^2 over the lists.  a [nq, 3] query
+        coordinates; c [nk, 3] key coordinates; v [nk, D].  Returns out
+        [nq, D] and lse [nq] (fp64, natural log)."""
+        a, c = self._coords(a, cdtype), self._coords(c, cdtype)
+        v = self._as_input(v, dtype)
+        nq, D = a.shape[0], v.shape[1]
+        rowptr = np.ascontiguousarray(rowptr, dtype=np.int64)
+        colidx = np.ascontiguousarray(colidx, dtype=np.int32)
+        assert len(rowptr) == nq + 1
+        if len(colidx):
+            assert colidx.min() >= 0 and colidx.max() < c.shape[0] and c.shape[0] == v.shape[0]
+        out = np.zeros((nq, D), dtype=np.float64)
+        lse = np.zeros(nq, dtype=np.float64)
+        st = self.lib.oracle_dist_fwd(nq, D, DTYPE_CODE[cdtype], DTYPE_CODE[dtype], _ptr(a),
+                                      _ptr(c), _ptr(v), _ptr(rowptr), _ptr(colidx), float(scale),
+                                      _ptr(out), _ptr(lse))
+        if st:
+            raise OracleError(STATUS[st])
+        return out, lse
+
+    def dist_bwd(self, a, c, v, dout, rowptr, colidx, scale: float, dtype: str = "f64",
+                 cdtype: str = "f64"):
+        """Gradients of sum(dout * out) w.r.t. a [nq, 3], c [nk, 3], v [nk, D]."""
+        a, c = self._coords(a, cdtype), self._coords(c, cdtype)
+        v, dout = self._as_input(v, dtype), self._as_input(dout, dtype)
+        nq, nk, D = a.shape[0], c.shape[0], v.shape[1]
+        rowptr = np.ascontiguousarray(rowptr, dtype=np.int64)
+        colidx = np.ascontiguousarray(colidx, dtype=np.int32)
+        if len(colidx):
+            assert colidx.min() >= 0 and colidx.max() < nk
+        da = np.zeros((nq, 3), dtype=np.float64)
+        dc = np.zeros((nk, 3), dtype=np.float64)
+        dv = np.zeros((nk, D), dtype=np.float64)
+        st = self.lib.oracle_dist_bwd(nq, nk, D, DTYPE_CODE[cdtype], DTYPE_CODE[dtype], _ptr(a),
+                                      _ptr(c), _ptr(v), _ptr(dout), _ptr(rowptr), _ptr(colidx),
+                                      float(scale), _ptr(da), _ptr(dc), _ptr(dv))
+        if st:
+            raise OracleError(STATUS[st])
+        return da, dc, dv
 
 
 _default: Oracle | None = None

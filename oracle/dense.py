@@ -46,3 +46,21 @@ def attention(q, k, v, mask, scale):
         lse = (m + np.log(l))[:, 0]
     lse = np.where(empty, -np.inf, lse)
     return out, lse
+
+
+def dist_attention(a, c, v, mask, scale):
+    """Learned-coordinate scoring, dense: s_ij = -scale * |a_i - c_j|^2 for
+    kept (i, j) ("SpatialLM-Mini ...", section "How tokens choose whom to
+    listen to": the closer the query and key coordinates, the larger the
+    weight).  a, c: [T, 3]; v: [T, D]; mask [T, T] bool."""
+    diff = a[:, None, :] - c[None, :, :]
+    s = -scale * np.einsum("ijx,ijx->ij", diff, diff)
+    s = np.where(mask, s, -np.inf)
+    empty = ~mask.any(axis=1)
+    m = np.where(empty[:, None], 0.0, s.max(axis=1, keepdims=True))
+    e = np.where(mask, np.exp(s - m), 0.0)
+    l = e.sum(axis=1, keepdims=True)
+    p = np.divide(e, l, out=np.zeros_like(e), where=l > 0)
+    with np.errstate(divide="ignore"):
+        lse = (m + np.log(l))[:, 0]
+    return p @ v, np.where(empty, -np.inf, lse)

@@ -300,3 +300,126 @@ done:
     free(dod);
     return st;
 }
+
+/* ---------- learned-coordinate scoring on the same graph ----------
+ * "SpatialLM-Mini ...", section "How tokens choose whom to listen to": the
+ * hidden state of each token gives a learnable three-dimensional query
+ * coordinate and key coordinate, and the shorter the distance between them,
+ * the higher the weight of the edge; the neighbour list stays fixed.  The
+ * page does not spell out the "additional learnable parameters" that adjust
+ * the weight, so the plainest pinnable form is taken: one positive scale,
+ *     s_ij = -scale * |a_i - c_j|^2      for j in N(i)
+ * (a_i: query coordinate, c_j: key coordinate, both 3 values), softmax over
+ * N(i), out_i = sum_j p_ij v_j, lse_i = ln sum_j exp(s_ij).
+ * Coordinates are read with element type cdtype (1 fp32, 2 fp64), v and dout
+ * with dtype (0 bf16, 1 fp32, 2 fp64).  Loops as in the dot-product
+ * statement above: per query, over its neighbour list, fp64. */
+static void row_forward_dist(int32_t D, const double *a, int64_t qrow, const double *c,
+                             const double *v, const int32_t *nbr, int64_t deg, double scale,
+                             double *w /* scratch[deg] */, double *out, double *lz) {
+    for (int32_t d = 0; d < D; ++d) out[d] = 0.0;
+    if (deg == 0) {
+        *lz = -INFINITY; /* empty list */
+        return;
+    }
+    double mx = -INFINITY;
+    for (int64_t e = 0; e < deg; ++e) {
+        int64_t j = nbr[e];
+        double dist2 = 0.0;
+        for (int x = 0; x < 3; ++x) {
+            double diff = a[qrow * 3 + x] - c[j * 3 + x];
+            dist2 += diff * diff;
+        }
+        w[e] = -scale * dist2;
+        if (w[e] > mx) mx = w[e];
+    }
+    double z = 0.0;
+    for (int64_t e = 0; e < deg; ++e) z += exp(w[e] - mx);
+    for (int64_t e = 0; e < deg; ++e) {
+        int64_t j = nbr[e];
+        double pw = exp(w[e] - mx) / z;
+        for (int32_t d = 0; d < D; ++d) out[d] += pw * v[j * D + d];
+    }
+    *lz = mx + log(z);
+}
+
+/* Forward: a [nq*3], c [nk*3] coordinates; v [nk*D]; out [nq*D], lse [nq]. */
+int oracle_dist_fwd(int64_t nq, int32_t D, int cdtype, int dtype, const void *a, const void *c,
+                    const void *v, const int64_t *rowptr, const int32_t *colidx, double scale,
+                    double *out, double *lse) {
+    if (nq < 0 || D < 1 || cdtype < 1 || cdtype > 2 || dtype < 0 || dtype > 2) return OR_BAD_ARG;
+    int64_t nk = 0;
+    for (int64_t e = 0; e < rowptr[nq]; ++e)
+        if ((int64_t)colidx[e] + 1 > nk) nk = (int64_t)colidx[e] + 1;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(max_degree(nq, rowptr) + 1));
+    double *ad = to_f64(a, cdtype, nq * 3), *cd = to_f64(c, cdtype, nk * 3);
+    double *vd = to_f64(v, dtype, nk * D);
+    int st = OR_OK;
+    if (!s || !ad || !cd || !vd) {
+        st = OR_NOMEM;
+    } else {
+        for (int64_t r = 0; r < nq; ++r)
+            row_forward_dist(D, ad, r, cd, vd, colidx + rowptr[r], rowptr[r + 1] - rowptr[r],
+                             scale, s, out + r * D, lse + r);
+    }
+    free(s);
+    free(ad);
+    free(cd);
+    free(vd);
+    return st;
+}
+
+/* Backward for upstream gradient dout[nq*D].  With the same P, dP, Delta and
+ * dS = P (dP - Delta) as the dot-product statement, and
+ *     d s_ij / d a_i = -2 scale (a_i - c_j),   d s_ij / d c_j = +2 scale (a_i - c_j):
+ *   da_i += dS_ij * (-2 scale (a_i - c_j)),  dc_j -= the same,  dv_j += P_ij dO_i.
+ * da [nq*3], dc [nk*3], dv [nk*D] are overwritten (zeroed first). */
+int oracle_dist_bwd(int64_t nq, int64_t nk, int32_t D, int cdtype, int dtype, const void *a,
+                    const void *c, const void *v, const void *dout, const int64_t *rowptr,
+                    const int32_t *colidx, double scale, double *da, double *dc, double *dv) {
+    if (nq < 0 || nk < 0 || D < 1 || cdtype < 1 || cdtype > 2 || dtype < 0 || dtype > 2)
+        return OR_BAD_ARG;
+    int64_t mdeg = max_degree(nq, rowptr);
+    double *s = (double *)malloc(sizeof(double) * (size_t)(mdeg + 1));
+    double *o = (double *)malloc(sizeof(double) * (size_t)D);
+    double *ad = to_f64(a, cdtype, nq * 3), *cd = to_f64(c, cdtype, nk * 3);
+    double *vd = to_f64(v, dtype, nk * D), *dod = to_f64(dout, dtype, nq * D);
+    int st = OR_OK;
+    if (!s || !o || !ad || !cd || !vd || !dod) {
+        st = OR_NOMEM;
+        goto done;
+    }
+    memset(da, 0, sizeof(double) * (size_t)(nq * 3));
+    memset(dc, 0, sizeof(double) * (size_t)(nk * 3));
+    memset(dv, 0, sizeof(double) * (size_t)(nk * D));
+    for (int64_t i = 0; i < nq; ++i) {
+        const int32_t *nbr = colidx + rowptr[i];
+        int64_t deg = rowptr[i + 1] - rowptr[i];
+        double lz;
+        row_forward_dist(D, ad, i, cd, vd, nbr, deg, scale, s, o, &lz);
+        if (deg == 0) continue;
+        double dlt = 0.0; /* Delta_i */
+        for (int32_t d = 0; d < D; ++d) dlt += dod[i * D + d] * o[d];
+        for (int64_t e = 0; e < deg; ++e) {
+            int64_t j = nbr[e];
+            double pe = exp(s[e] - lz);
+            double dpe = 0.0;
+            for (int32_t d = 0; d < D; ++d) dpe += dod[i * D + d] * vd[j * D + d];
+            double dse = pe * (dpe - dlt);
+            for (int x = 0; x < 3; ++x) {
+                double g = dse * (-2.0 * scale * (ad[i * 3 + x] - cd[j * 3 + x]));
+                da[i * 3 + x] += g;
+                dc[j * 3 + x] -= g;
+            }
+            for (int32_t d = 0; d < D; ++d) dv[j * D + d] += pe * dod[i * D + d];
+        }
+    }
+done:
+    free(s);
+    free(o);
+    free(ad);
+    free(cd);
+    free(vd);
+    free(dod);
+    return st;
+}

@@ -346,9 +346,124 @@ def pin_bwd_invariants(o):
     assert np.allclose(dq2, 0.0, rtol=0, atol=1e-12)
 
 
+# ---------------------------------------------------------------- learned
+# coordinates: s_ij = -scale |a_i - c_j|^2 ("SpatialLM-Mini ...", section
+# "How tokens choose whom to listen to": the closer the coordinates, the
+# larger the weight)
+
+def pin_dist_dense(o):
+    """Equals the dense numpy statement on structured and random CSR graphs."""
+    for n, (T, D) in enumerate([(120, 8), (64, 16)]):
+        a, c = _rand((T, 3), 500 + n), _rand((T, 3), 510 + n)
+        v = _rand((T, D), 520 + n)
+        for rowptr, colidx in (o.structured(T, 5, range(0, 7)), _random_csr(T, 530 + n)):
+            out, lse = o.dist_fwd(a, c, v, rowptr, colidx, 0.8)
+            mask = dense.mask_from_csr(T, rowptr, colidx)
+            r_out, r_lse = dense.dist_attention(a, c, v, mask, 0.8)
+            assert np.allclose(out, r_out, rtol=0, atol=1e-12)
+            fin = np.isfinite(r_lse)
+            assert np.array_equal(np.isfinite(lse), fin)
+            assert np.allclose(lse[fin], r_lse[fin], rtol=0, atol=1e-12)
+
+
+def pin_dist_dot_product_identity(o):
+    """-|a - c|^2 = 2 a.c - |c|^2 - |a|^2 and the last term is the same for
+    every key of a row: with q' = (2a, -1) and k' = (c, |c|^2) the dot-product
+    oracle (pinned on its own) gives the same out, an lse larger by
+    scale |a|^2, and gradients related by the chain rule:
+    da = 2 dq'[:3], dc = dk'[:3] + 2 c dk'[3]."""
+    T, D, W, exps, scale = 150, 8, 6, range(0, 8), 0.45
+    rowptr, colidx = o.structured(T, W, exps)
+    a, c = _rand((T, 3), 540), _rand((T, 3), 541)
+    v, dout = _rand((T, D), 542), _rand((T, D), 543)
+    q2 = np.concatenate([2.0 * a, -np.ones((T, 1))], axis=1)
+    k2 = np.concatenate([c, (c * c).sum(axis=1, keepdims=True)], axis=1)
+    out, lse = o.dist_fwd(a, c, v, rowptr, colidx, scale)
+    # the dot-product oracle's q, k, v share D: pad q' and k' with zeros
+    pad = np.zeros((T, D - 4))
+    qp, kp = np.concatenate([q2, pad], axis=1), np.concatenate([k2, pad], axis=1)
+    r_out, r_lse = o.fwd(qp, kp, v, rowptr, colidx, scale)
+    assert np.allclose(out, r_out, rtol=0, atol=1e-12)
+    assert np.allclose(lse, r_lse - scale * (a * a).sum(axis=1), rtol=0, atol=1e-11)
+    da, dc, dv = o.dist_bwd(a, c, v, dout, rowptr, colidx, scale)
+    dqp, dkp, r_dv = o.bwd(qp, kp, v, dout, rowptr, colidx, scale)
+    assert np.allclose(dv, r_dv, rtol=0, atol=1e-12)
+    assert np.allclose(da, 2.0 * dqp[:, :3], rtol=0, atol=1e-11)
+    assert np.allclose(dc, dkp[:, :3] + 2.0 * c * dkp[:, 3:4], rtol=0, atol=1e-11)
+
+
+def pin_dist_invariants(o):
+    """Moving every coordinate by the same vector changes nothing (distances
+    are unchanged); row 0 sees only itself; constant V gives that constant;
+    the closest key dominates when the scale is large."""
+    T, D, W, exps = 100, 8, 4, range(0, 7)
+    rowptr, colidx = o.structured(T, W, exps)
+    a, c, v = _rand((T, 3), 550), _rand((T, 3), 551), _rand((T, D), 552)
+    dout = _rand((T, D), 553)
+    out, lse = o.dist_fwd(a, c, v, rowptr, colidx, 0.6)
+    u = np.array([0.75, -2.5, 1.25])
+    out2, lse2 = o.dist_fwd(a + u, c + u, v, rowptr, colidx, 0.6)
+    assert np.allclose(out, out2, rtol=0, atol=1e-12)
+    assert np.allclose(lse, lse2, rtol=0, atol=1e-12)
+    g1 = o.dist_bwd(a, c, v, dout, rowptr, colidx, 0.6)
+    g2 = o.dist_bwd(a + u, c + u, v, dout, rowptr, colidx, 0.6)
+    for x, y in zip(g1, g2):
+        assert np.allclose(x, y, rtol=0, atol=1e-11)
+    assert np.allclose(out[0], v[0], rtol=0, atol=1e-15)
+    assert abs(lse[0] + 0.6 * float(((a[0] - c[0]) ** 2).sum())) <= 1e-14
+    cv = np.tile(np.arange(1.0, D + 1.0), (T, 1))
+    out_c, _ = o.dist_fwd(a, c, cv, rowptr, colidx, 0.6)
+    assert np.allclose(out_c, cv, rtol=0, atol=1e-12)
+    # every query placed on its own key, other keys far: out_i -> v_i
+    a3 = np.arange(T, dtype=np.float64)[:, None] * np.array([[10.0, 0.0, 0.0]])
+    out_s, _ = o.dist_fwd(a3, a3.copy(), v, rowptr, colidx, 1.0)
+    assert np.allclose(out_s, v, rtol=0, atol=1e-12)
+    # sum_j dv_j = sum_i dO_i (rows of P sum to one); sum of da + dc is zero
+    # (translation invariance of the loss)
+    da, dc, dv = g1
+    assert np.allclose(dv.sum(axis=0), dout.sum(axis=0), rtol=0, atol=1e-11)
+    assert np.allclose(da.sum(axis=0) + dc.sum(axis=0), 0.0, rtol=0, atol=1e-11)
+
+
+def _dist_loss(o, a, c, v, dout, rowptr, colidx, scale):
+    out, _ = o.dist_fwd(a, c, v, rowptr, colidx, scale)
+    return float(np.sum(out * dout))
+
+
+def pin_dist_finite_differences(o):
+    """Central differences of L = sum(dout * out) along random directions of
+    a, c and v together and separately (h = 1e-6, relative error < 1e-6),
+    and torch autograd through the dense formulation."""
+    T, D, W, exps, scale = 130, 8, 6, range(0, 8), 0.35
+    rowptr, colidx = o.structured(T, W, exps)
+    a, c = _rand((T, 3), 560), _rand((T, 3), 561)
+    v, dout = _rand((T, D), 562), _rand((T, D), 563)
+    da, dc, dv = o.dist_bwd(a, c, v, dout, rowptr, colidx, scale)
+    h = 1e-6
+    rng = np.random.default_rng(6)
+    for which in range(4):
+        ua = rng.standard_normal((T, 3)) * (which in (0, 3))
+        uc = rng.standard_normal((T, 3)) * (which in (1, 3))
+        uv = rng.standard_normal((T, D)) * (which in (2, 3))
+        lp = _dist_loss(o, a + h * ua, c + h * uc, v + h * uv, dout, rowptr, colidx, scale)
+        lm = _dist_loss(o, a - h * ua, c - h * uc, v - h * uv, dout, rowptr, colidx, scale)
+        fd = (lp - lm) / (2 * h)
+        an = float(np.sum(da * ua) + np.sum(dc * uc) + np.sum(dv * uv))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (which, fd, an)
+    mask = torch.from_numpy(dense.structured_mask(T, W, exps))
+    ta, tc, tv = (torch.tensor(x, requires_grad=True) for x in (a, c, v))
+    s = (-scale * ((ta[:, None, :] - tc[None, :, :]) ** 2).sum(-1)).masked_fill(~mask,
+                                                                                float("-inf"))
+    (torch.softmax(s, dim=1) @ tv).backward(torch.from_numpy(dout))
+    assert np.allclose(da, ta.grad.numpy(), rtol=0, atol=1e-12)
+    assert np.allclose(dc, tc.grad.numpy(), rtol=0, atol=1e-12)
+    assert np.allclose(dv, tv.grad.numpy(), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [pin_graph_golden, pin_graph_bruteforce, pin_graph_closed_forms,
             pin_graph_rows_match_full, pin_graph_reverse,
             pin_graph_normalize, pin_fwd_golden, pin_fwd_structured_rows_golden,
             pin_fwd_full_causal, pin_fwd_dense, pin_fwd_invariants, pin_fwd_empty_rows,
             pin_bwd_golden, pin_bwd_finite_differences, pin_bwd_dense_autograd,
-            pin_bwd_invariants]
+            pin_bwd_invariants, pin_dist_dense, pin_dist_dot_product_identity,
+            pin_dist_invariants, pin_dist_finite_differences]

@@ -53,6 +53,14 @@ MUTANTS = {
     "dk_scale_dropped": ("dk[j * D + d] += scale * ds * qd[i * D + d];",
                          "dk[j * D + d] += ds * qd[i * D + d];"),
     "bwd_prob_without_lse": ("double p = exp(s[e] - lse);", "double p = exp(s[e]);"),
+    "dist_sign_flipped": ("w[e] = -scale * dist2;", "w[e] = scale * dist2;"),
+    "dist_not_squared": ("dist2 += diff * diff;", "dist2 += fabs(diff);"),
+    "dist_grad_factor_two_dropped": ("double g = dse * (-2.0 * scale * (ad[i * 3 + x] - cd[j * 3 + x]));",
+                                     "double g = dse * (-scale * (ad[i * 3 + x] - cd[j * 3 + x]));"),
+    "dist_key_grad_sign": ("dc[j * 3 + x] -= g;", "dc[j * 3 + x] += g;"),
+    "dist_key_grad_wrong_row": ("dc[j * 3 + x] -= g;", "dc[i * 3 + x] -= g;"),
+    "dist_delta_dropped": ("double dse = pe * (dpe - dlt);", "double dse = pe * dpe;"),
+    "dist_scale_dropped": ("w[e] = -scale * dist2;", "w[e] = -dist2;"),
 }
 
 

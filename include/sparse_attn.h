@@ -151,18 +151,72 @@ sa_status sparse_attn_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
  * recomputes p and dS of the distance links (bitwise reproducible run to run
  * on its own).  Its scratch (Delta, 4 bytes per query row) is a fixed device
  * array of SA_NOALLOC_MAX_ROWS floats inside the library: every GPU that
- * loads the library holds it (4 MiB) until the process exits.  B*H*T above
- * SA_NOALLOC_MAX_ROWS returns SA_ERR_UNSUPPORTED before anything is enqueued.
- * Every call on a device shares the array (it keeps the last call's
- * contents, none of which must start at zero), so calls whose work overlaps
- * on the GPU race: serialise them (one stream, or events).  The first call
- * on each device looks up the array's device address; make that first call
- * before any stream capture. */
+ * loads the library holds it (4 MiB) until the process exits.  Arguments
+ * are checked as in sparse_attn_bwd (SA_ERR_INVALID_ARG / _UNSUPPORTED);
+ * then B*H*T above SA_NOALLOC_MAX_ROWS returns SA_ERR_UNSUPPORTED.  Either
+ * way nothing is enqueued.  Every call on a device shares the array (it
+ * keeps the last call's contents, none of which must start at zero), so
+ * calls whose work overlaps on the GPU race: serialise them (one stream, or
+ * events).  Every call looks up the array's device address in the current
+ * context (cudaGetSymbolAddress); the first call on a device may also make
+ * the driver load the library's device code, so make that first call before
+ * any stream capture. */
 #define SA_NOALLOC_MAX_ROWS (1 << 20)
 sa_status sparse_attn_bwd_noalloc(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                                   const sa_tensor *out, const float *lse, const sa_tensor *dout,
                                   sa_graph g, float scale, sa_tensor *dq, sa_tensor *dk,
                                   sa_tensor *dv, void *stream);
+
+/* ------------------------------------------------------------------ decode */
+
+/* One new query per batch row and head against a KV cache, over the same
+ * graph (page "SpatialLM-Mini ...", section "What to check before adopting
+ * it in your project", notes the missing KV cache and unmeasured generation
+ * speed).  q and out: [B, H, 1, D]; k_cache, v_cache: [B, Hkv, Tmax, D] with
+ * Hkv dividing H (query head h reads cache head h / (H / Hkv): grouped-query
+ * attention, page "MiniGPT (Part 6)", introduction); same dtype and D as q.
+ * pos: DEVICE int64 [B], the query's position in batch row b -- its own key
+ * and value must already be stored at cache row pos[b].  The query attends
+ * to N(pos[b]) of graph g (g's T >= Tmax), exactly as row pos[b] of
+ * sparse_attn_fwd would.  lse: fp32 [B, H].  A pos[b] outside [0, Tmax)
+ * (only known on the device) gives out = 0, lse = -inf for that row and
+ * flags the device error word (sparse_attn_check_device then reports
+ * SA_ERR_CUDA); nothing faults.  No workspace, no host synchronisation. */
+sa_status sparse_attn_decode(const sa_tensor *q, const sa_tensor *k_cache,
+                             const sa_tensor *v_cache, const int64_t *pos, sa_graph g,
+                             float scale, sa_tensor *out, float *lse, void *stream);
+
+/* -------------------------------------------- learned-coordinate scoring */
+
+/* The same neighbour graph with the edge weight taken from learnable
+ * coordinates instead of a dot product (page "SpatialLM-Mini sped up
+ * training with a 16K context by 2.47x on an RTX 3050", section "How tokens
+ * choose whom to listen to": each token gets a three-dimensional query and
+ * key coordinate, and the shorter their distance the higher the weight).
+ * The page leaves the extra learnable adjustments unspecified; the form
+ * computed is
+ *     s_ij  = -scale * |a_i - c_j|^2            for j in N(i)
+ *     out_i = sum_j softmax_j(s_ij) v_j,   lse_i = ln sum_j exp(s_ij).
+ * a (query coordinates) and c (key coordinates) are fp32 [B, H, T, 3]
+ * (sa_tensor with D = 3, dtype SA_FP32, same B, H, T as v); v and out are
+ * bf16 or fp32 [B, H, T, D], D in {32, 64, 128}; lse fp32 [B, H, T].  Every
+ * edge runs on CUDA cores (a score is three FMAs).  No workspace. */
+sa_status sparse_attn_dist_fwd(const sa_tensor *a, const sa_tensor *c, const sa_tensor *v,
+                               sa_graph g, float scale, sa_tensor *out, float *lse, void *stream);
+
+/* Workspace of sparse_attn_dist_bwd: 4 * B * H * T bytes (Delta), rounded up
+ * to 256 bytes.  `v` gives the shape. */
+size_t sparse_attn_dist_bwd_workspace_size(const sa_tensor *v, sa_graph g);
+
+/* Backward of sparse_attn_dist_fwd for upstream gradient dout: da, dc
+ * (fp32 [B, H, T, 3]) and dv (v's dtype) are written in full.  Recomputes
+ * the probabilities from lse; two kernels with disjoint outputs (da by the
+ * forward lists, dc and dv by the transpose lists), no atomics, bitwise
+ * reproducible.  workspace: caller-owned device memory, 256-byte aligned. */
+sa_status sparse_attn_dist_bwd(const sa_tensor *a, const sa_tensor *c, const sa_tensor *v,
+                               const sa_tensor *out, const float *lse, const sa_tensor *dout,
+                               sa_graph g, float scale, sa_tensor *da, sa_tensor *dc,
+                               sa_tensor *dv, void *workspace, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------ utilities */
 

@@ -54,6 +54,14 @@ def _load():
         "sparse_attn_bwd_noalloc": (st, [P(SaTensor), P(SaTensor), P(SaTensor), P(SaTensor), vp,
                                          P(SaTensor), vp, ctypes.c_float, P(SaTensor),
                                          P(SaTensor), P(SaTensor), vp]),
+        "sparse_attn_decode": (st, [P(SaTensor), P(SaTensor), P(SaTensor), vp, vp,
+                                    ctypes.c_float, P(SaTensor), vp, vp]),
+        "sparse_attn_dist_fwd": (st, [P(SaTensor), P(SaTensor), P(SaTensor), vp,
+                                      ctypes.c_float, P(SaTensor), vp, vp]),
+        "sparse_attn_dist_bwd_workspace_size": (ctypes.c_size_t, [P(SaTensor), vp]),
+        "sparse_attn_dist_bwd": (st, [P(SaTensor), P(SaTensor), P(SaTensor), P(SaTensor), vp,
+                                      P(SaTensor), vp, ctypes.c_float, P(SaTensor),
+                                      P(SaTensor), P(SaTensor), vp, ctypes.c_size_t, vp]),
         "sparse_attn_profile_begin": (st, [i32]),
         "sparse_attn_profile_end": (i32, [ctypes.c_char_p, i32, P(i32), P(ctypes.c_double), i32]),
     }
@@ -267,6 +275,88 @@ def sparse_attn_bwd_noalloc(q, k, v, out, lse, dout, g: Graph, scale: float, dq=
 SA_NOALLOC_MAX_ROWS = 1 << 20
 
 
+# ------------------------------------------------------------------ decode
+
+def sparse_attn_decode(q, k_cache, v_cache, pos, g: Graph, scale: float, out=None, lse=None,
+                       stream=None):
+    """q [B, H, 1, D]; caches [B, Hkv, Tmax, D]; pos: CUDA int64 [B] (the
+    query's own key/value already at cache row pos[b]).  Returns (out
+    [B, H, 1, D], lse fp32 [B, H])."""
+    B, H, _, D = q.shape
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or lse.shape != (B, H):
+        raise ValueError("lse must be a contiguous fp32 [B, H] tensor")
+    if pos.dtype != torch.int64 or not pos.is_cuda or pos.numel() != B:
+        raise ValueError("pos must be a CUDA int64 tensor of B positions")
+    tq, tk, tv, to = (_tensor(x, n) for x, n in ((q, "q"), (k_cache, "k_cache"),
+                                                  (v_cache, "v_cache"), (out, "out")))
+    _check(_lib.sparse_attn_decode(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv),
+                                   pos.data_ptr(), g.handle, float(scale), ctypes.byref(to),
+                                   lse.data_ptr(), _stream(stream)),
+           "sparse_attn_decode")
+    return out, lse
+
+
+# ------------------------------------------------ learned-coordinate scoring
+
+def _coords(t: torch.Tensor, name: str) -> SaTensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32:
+        raise ValueError(f"{name} must be a CUDA fp32 tensor")
+    if t.dim() != 4 or t.shape[3] != 3 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B, H, T, 3] tensor")
+    B, H, T, _ = t.shape
+    return SaTensor(t.data_ptr(), SA_FP32, B, H, T, 3)
+
+
+def sparse_attn_dist_fwd(a, c, v, g: Graph, scale: float, out=None, lse=None, stream=None):
+    """s_ij = -scale |a_i - c_j|^2 over the graph's lists; a, c fp32
+    [B, H, T, 3].  Returns (out [B, H, T, D] in v's dtype, lse fp32 [B, H, T])."""
+    B, H, T, D = v.shape
+    out = torch.empty_like(v) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=v.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or lse.shape != (B, H, T):
+        raise ValueError("lse must be a contiguous fp32 [B, H, T] tensor")
+    ta, tc = _coords(a, "a"), _coords(c, "c")
+    tv, to = _tensor(v, "v"), _tensor(out, "out")
+    _check(_lib.sparse_attn_dist_fwd(ctypes.byref(ta), ctypes.byref(tc), ctypes.byref(tv),
+                                     g.handle, float(scale), ctypes.byref(to), lse.data_ptr(),
+                                     _stream(stream)),
+           "sparse_attn_dist_fwd")
+    return out, lse
+
+
+def sparse_attn_dist_bwd_workspace_size(v, g: Graph) -> int:
+    tv = _tensor(v, "v")
+    return int(_lib.sparse_attn_dist_bwd_workspace_size(ctypes.byref(tv), g.handle))
+
+
+def sparse_attn_dist_bwd(a, c, v, out, lse, dout, g: Graph, scale: float, da=None, dc=None,
+                         dv=None, workspace=None, stream=None):
+    """Returns (da, dc, dv)."""
+    da = torch.empty_like(a) if da is None else da
+    dc = torch.empty_like(c) if dc is None else dc
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(sparse_attn_dist_bwd_workspace_size(v, g), dtype=torch.uint8,
+                                device=v.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32")
+    ta, tc, tda, tdc = _coords(a, "a"), _coords(c, "c"), _coords(da, "da"), _coords(dc, "dc")
+    tv, to, tdo, tdv = (_tensor(x, n) for x, n in ((v, "v"), (out, "out"), (dout, "dout"),
+                                                    (dv, "dv")))
+    _check(_lib.sparse_attn_dist_bwd(ctypes.byref(ta), ctypes.byref(tc), ctypes.byref(tv),
+                                     ctypes.byref(to), lse.data_ptr(), ctypes.byref(tdo),
+                                     g.handle, float(scale), ctypes.byref(tda), ctypes.byref(tdc),
+                                     ctypes.byref(tdv), workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(),
+                                     _stream(stream)),
+           "sparse_attn_dist_bwd")
+    return da, dc, dv
+
+
 # ---------------------------------------------------------------- utilities
 
 def sparse_attn_status_string(status: int) -> str:
@@ -333,6 +423,28 @@ class _SparseAttention(torch.autograd.Function):
         return dq, dk, dv, None, None
 
 
+class _DistAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, a, c, v, graph, scale):
+        out, lse = sparse_attn_dist_fwd(a, c, v, graph, scale)
+        ctx.save_for_backward(a, c, v, out, lse)
+        ctx.graph, ctx.scale = graph, scale
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        a, c, v, out, lse = ctx.saved_tensors
+        da, dc, dv = sparse_attn_dist_bwd(a, c, v, out, lse, dout.contiguous(), ctx.graph,
+                                          ctx.scale)
+        return da, dc, dv, None, None
+
+
+def dist_attention(a, c, v, graph: Graph, scale: float):
+    """Differentiable learned-coordinate attention on the graph:
+    softmax over N(i) of -scale |a_i - c_j|^2, applied to v."""
+    return _DistAttention.apply(a, c, v, graph, scale)
+
+
 def attention(q, k, v, graph: Graph, scale: float):
     """Differentiable sparse-graph causal attention (forward and backward in
     the library's kernels)."""
@@ -340,4 +452,4 @@ def attention(q, k, v, graph: Graph, scale: float):
 
 
 __all__ = [n for n in dir() if n.startswith("sparse_attn_")] + [
-    "Graph", "attention", "SparseAttentionError", "LIB_PATH"]
+    "Graph", "attention", "dist_attention", "SparseAttentionError", "LIB_PATH"]

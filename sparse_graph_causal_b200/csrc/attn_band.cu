@@ -11,10 +11,13 @@
 //  * Every other edge -- the 2^k distance links of "SpatialLM-Mini ...",
 //    section "How tokens choose whom to listen to", or the non-window part of
 //    a CSR list ("Longer Attention Span ...", Abstract) -- is a "diagonal"
-//    block: 128 key rows, row r belonging to query r.  For a distance o the
-//    rows are the contiguous keys q0-o .. q0+127-o (one TMA box); for CSR
-//    lists slot s of every row is fetched with 4-row TMA gathers.  Thread r
-//    takes the dot product of its own row on the CUDA cores.
+//    block: 128 key rows, row r belonging to query r (for a distance o the
+//    keys q0-o .. q0+127-o; for CSR lists slot s of every row's residual
+//    list).  Each softmax warp fetches the K and V rows of its own 32 queries
+//    itself with 16-byte cp.async copies, DS slots ahead (plus L2 prefetches
+//    further ahead when K and V exceed L2), into the band tiles' swizzled
+//    layout; thread r then takes the dot product of its own row on the CUDA
+//    cores.  No other role takes part, so warps progress independently.
 //  * One online softmax (running max m and sum l per row, base 2) covers both
 //    classes: the diagonal blocks go first, their weighted sum initialises O
 //    in TMEM, then the band blocks rescale O only when a row's max grows by
@@ -25,7 +28,7 @@
 // per CTA, each with its own shared-memory rings, TMEM columns (two S
 // buffers and O) and barriers, so that the softmax of one tile overlaps the
 // loads, MMAs and softmax of the other.  Warp roles: warp 2p is the TMA
-// producer of pipeline p (Q, band K/V ring, diagonal blocks), warp 2p+1 its
+// producer of pipeline p (Q and the band K/V ring), warp 2p+1 its
 // MMA issuer (warp 1 also allocates TMEM), warps 4+4p .. 7+4p its softmax
 // warpgroup (thread = query row = TMEM lane).  With two pipelines the
 // producer warpgroup hands registers to the softmax warpgroups (setmaxnreg).
@@ -37,6 +40,7 @@
 #include <stdint.h>
 
 #include "sa_band.cuh"
+#include "sa_rows.cuh"
 #include "tc_common.cuh"
 #include "tmap.cuh"
 
@@ -47,32 +51,44 @@ constexpr int BN = 64;              // keys per band block
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Distance blocks are prefetched into L2 this many blocks ahead of their
-// loads when K and V do not fit in L2 (long links then miss it, and the
-// two-stage ring alone keeps too few of their DRAM reads in flight); with
-// L2-resident K and V the prefetches are pure overhead and are skipped.
-constexpr int kPrefetchAhead = 4;
+// Diagonal rows are prefetched into L2 ahead of their copies when K and V do
+// not fit in L2 (long links and random CSR keys then miss it, and the copy
+// ring alone keeps too few DRAM reads in flight); with L2-resident K and V
+// the prefetches are pure overhead and are skipped.
 constexpr double kL2ResidentBytes = 64.0 * 1024 * 1024;
+// Distance blocks (TMA boxes) are prefetched into L2 this many blocks ahead
+// of their loads under the same condition.
+constexpr int kPrefetchBlocks = 4;
 // Register budgets with two pipelines (384 threads launched at 168 each):
-// the producer warpgroup keeps 56 (72 when it also gathers diagonal blocks),
-// the softmax warpgroups take the rest.
+// the producer warpgroup keeps 56, the softmax warpgroups take the rest.
 template <int DS>
 struct Regs {
-    static constexpr int producer = DS > 0 ? 72 : 56;
-    static constexpr int softmax = DS > 0 ? 216 : 224;
+    static constexpr int producer = 56;
+    static constexpr int softmax = 224;
     static_assert(128 * producer + 256 * softmax <= 384 * 168, "register split");
 };
+
+// Distance links short enough to fall inside the span of key blocks that a
+// tile covers anyway are folded into the band blocks: row r keeps, besides its
+// window, the single key i - o of each folded link o (at most kMaxFold).
+constexpr int kMaxFold = 4;
 
 struct FwdArgs {
     int64_t T;
     int64_t BH;
+    int64_t H, Hkv;                // query and key/value heads (grouped-query attention)
     int32_t W;          // band width (structured window or verified CSR band)
+    int32_t We;         // span of the band blocks: W, or the longest folded link + 1
+    int32_t nf;         // folded links
+    int32_t fold[kMaxFold];
     int32_t kind;       // 0 structured, 1 CSR
+    int32_t gp;         // CSR: every row i holds keys 0 .. min(gp, i + 1) - 1 (0: none)
     int32_t n_off;
-    int32_t prefetch;              // distance blocks prefetched into L2 ahead (0: none)
+    int32_t l2pf;                  // diagonal rows prefetched into L2 ahead of their copies
     int64_t offs[SA_MAX_OFFSETS];  // distances (structured), descending
     const int64_t *rowptr;         // CSR
     const int32_t *colidx;
+    const __nv_bfloat16 *k, *v;    // diagonal rows are copied from here
     __nv_bfloat16 *out;
     float *lse;
     float scale2;                  // scale * log2(e)
@@ -92,7 +108,6 @@ struct Layout {
     static constexpr int pDV = pDK + DS * kQTile;       // diagonal V ring
     static constexpr int kPipe = pDV + DS * kQTile;
     static constexpr int kBars = NP * kPipe;
-    static constexpr int DSX = DS > 0 ? DS : 1;         // ring modulus
     // barriers of one pipeline (S, P, PVDone per S buffer: P is written over S)
     static constexpr int bQFull = 0, bQEmpty = 1;
     static constexpr int bKFull = 2, bKEmpty = bKFull + KS;
@@ -100,10 +115,12 @@ struct Layout {
     static constexpr int bSFull = bVEmpty + VS, bSFree = bSFull + 2;
     static constexpr int bPFull = bSFree + 2, bPVDone = bPFull + 2;
     static constexpr int bOInit = bPVDone + 2;
+    // distance blocks loaded by the producer with TMA (structured graphs): the
+    // ring's barriers and the per-tile block count handed to the softmax warps
+    static constexpr int DSX = DS > 0 ? DS : 1;
     static constexpr int bDiagFull = bOInit + 1, bDiagEmpty = bDiagFull + DSX;
     static constexpr int bInfoFull = bDiagEmpty + DSX, bInfoEmpty = bInfoFull + 2;
-    static constexpr int bGroup = bInfoEmpty + 2;        // 128-thread softmax barrier
-    static constexpr int nBarsPipe = bGroup + 1;
+    static constexpr int nBarsPipe = bInfoEmpty + 2;
     static constexpr int kMisc = kBars + NP * nBarsPipe * 8;  // tmem slot, abort, info[NP][2]
     static constexpr int kTotal = kMisc + 8 + 8 * NP;
     static constexpr int kAlloc = kTotal + 1024;         // alignment slack
@@ -117,14 +134,21 @@ struct Layout {
 
 // Geometry of query tile t (tiles run over B*H slices, 128 queries each).
 // 32-bit: the band path requires T < 2^31 and W + 127 < 2^31.
+// npre = 1 when the tile starts with the shared-prefix block (keys 0 .. 63,
+// kept for row i below min(gp, i - W + 1), i.e. outside its window); the
+// band blocks follow.
 struct TileGeom {
-    int32_t bh, q0, kb0, b_first, n_band;
+    int32_t bh, kvbh, q0, kb0, b_first, n_band, npre;
 };
 
-__device__ __forceinline__ TileGeom tile_geom(int64_t t, int64_t ntq, int64_t T, int32_t W) {
+// kvbh: the key/value slice that query slice bh reads (query head h of batch
+// row b reads key/value head h / (H / Hkv)).
+__device__ __forceinline__ TileGeom tile_geom(int64_t t, int64_t ntq, int64_t T, int32_t W,
+                                              int64_t H, int64_t Hkv, int32_t gp) {
     TileGeom g;
     const int64_t bh = t / ntq;
     g.bh = (int32_t)bh;
+    g.kvbh = (int32_t)((bh / H) * Hkv + (bh % H) / (H / Hkv));
     g.q0 = (int32_t)((t - bh * ntq) * BM);
     g.kb0 = g.q0 - W + 1;                                             // key of u = 0
     const int32_t last_key = (g.q0 + BM - 1 < T - 1) ? g.q0 + BM - 1 : (int32_t)(T - 1);
@@ -132,6 +156,7 @@ __device__ __forceinline__ TileGeom tile_geom(int64_t t, int64_t ntq, int64_t T,
     const int32_t need = W - 1 - g.q0;                                // first block with a key >= 0
     g.b_first = need > 0 ? need / BN : 0;
     g.n_band = nblk - g.b_first;
+    g.npre = (gp > 0 && last_key >= W) ? 1 : 0;  // (no prefix on structured graphs: W = We)
     return g;
 }
 
@@ -139,14 +164,16 @@ __device__ __forceinline__ TileGeom tile_geom(int64_t t, int64_t ntq, int64_t T,
 // the two pipelines of a CTA work on neighbouring tiles.  Every ring keeps its
 // phase across tiles, so the loads and MMAs of the next tile proceed while
 // the current one finishes.
-template <int D, int NP, int KS, int VS, int DS>
+// LDW selects how the diagonal slots are loaded: false -- the producer loads
+// each distance block as TMA boxes (structured graphs: 128 contiguous rows);
+// true -- every softmax warp copies its own rows (CSR lists: one random row
+// per tile row, rows/sa_rows.cuh).
+template <int D, int NP, int KS, int VS, int DS, bool LDW>
 __global__ void __launch_bounds__(128 + 128 * NP, 1)
 band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkd,
-                const __grid_constant__ CUtensorMap tvd, const __grid_constant__ CUtensorMap tkr,
-                const __grid_constant__ CUtensorMap tvr, const FwdArgs a) {
+                const __grid_constant__ CUtensorMap tvd, const FwdArgs a) {
     using L = Layout<D, NP, KS, VS, DS>;
-    constexpr int DSX = L::DSX;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_u32(sm);
@@ -174,8 +201,6 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 tc::mbar_init(bar(p, L::bSFree + s), 1);   // P V of the buffer's block done
                 tc::mbar_init(bar(p, L::bPFull + s), 4);
                 tc::mbar_init(bar(p, L::bPVDone + s), 1);
-                tc::mbar_init(bar(p, L::bInfoFull + s), 1);
-                tc::mbar_init(bar(p, L::bInfoEmpty + s), 4);
             }
             for (int s = 0; s < KS; ++s) {
                 tc::mbar_init(bar(p, L::bKFull + s), 1);
@@ -186,10 +211,13 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 tc::mbar_init(bar(p, L::bVEmpty + s), 1);
             }
             tc::mbar_init(bar(p, L::bOInit), 4);
-            tc::mbar_init(bar(p, L::bGroup), 128);
-            for (int s = 0; s < DSX; ++s) {
+            for (int s = 0; s < L::DSX; ++s) {
                 tc::mbar_init(bar(p, L::bDiagFull + s), 1);
                 tc::mbar_init(bar(p, L::bDiagEmpty + s), 4);
+            }
+            for (int s = 0; s < 2; ++s) {
+                tc::mbar_init(bar(p, L::bInfoFull + s), 1);
+                tc::mbar_init(bar(p, L::bInfoEmpty + s), 4);
             }
         }
         *abort = 0;
@@ -205,8 +233,10 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         // one register budget per warpgroup, set where it dominates the roles
         if (NP == 2) tc::regs_dec<Regs<DS>::producer>();
       if ((warp >> 1) < NP && (warp & 1) == 0) {
-        // ---------------- producer of pipeline p: per tile the diagonal-block
-        // count, Q, the first band K/V blocks, the diagonal blocks, the rest
+        // ---------------- producer of pipeline p (lane 0): per tile Q, the band
+        // K/V blocks through their rings and, for a structured graph, the
+        // distance blocks (the count first, to the softmax warps) after the
+        // band blocks that fit the rings
         const int p = warp >> 1;
         const uint32_t pb = sbase + (uint32_t)(p * L::kPipe);
         volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
@@ -214,146 +244,93 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             tc::tma_prefetch_desc(&tq);
             tc::tma_prefetch_desc(&tk);
             tc::tma_prefetch_desc(&tv);
-        }
-        uint32_t kc = 0, vc = 0, dc = 0;  // K, V and diagonal blocks loaded (all tiles)
-        bool ok = true;
-        int64_t lt = 0;
-        for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
-            const TileGeom g = tile_geom(t, ntq, T, W);
-            const int64_t last = (g.q0 + BM - 1 < T - 1) ? g.q0 + BM - 1 : T - 1;
-            // CSR: lane l owns rows 4l .. 4l+3 (list start, residual count,
-            // key of the next slot, fetched one slot ahead)
-            int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
-            int32_t cj[4] = {0, 0, 0, 0};
-            int nd = 0;
-            if (DS > 0) {
-                if (a.kind == 0) {
+            uint32_t kc = 0, vc = 0, dc = 0;  // K, V and distance blocks loaded (all tiles)
+            bool ok = true;
+            int64_t lt = 0;
+            for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
+                const TileGeom g = tile_geom(t, ntq, T, a.We, a.H, a.Hkv, a.gp);
+                auto load_k = [&](int bl) -> bool {
+                    const int st = (int)(kc % KS);
+                    const uint32_t use = kc / KS;
+                    if (use > 0 && !wait(p, L::bKEmpty + st, (use - 1) & 1)) return false;
+                    const int32_t krow = bl < g.npre ? 0 : g.kb0 + (g.b_first + bl - g.npre) * BN;
+                    tc::mbar_arrive_expect_tx(bar(p, L::bKFull + st), L::kBlk);
+                    for (int x = 0; x < D / 64; ++x)
+                        tc::tma_load_3d(pb + L::pK + st * L::kBlk + x * (BN * 128), &tk, x * 64,
+                                        krow, g.kvbh, bar(p, L::bKFull + st));
+                    ++kc;
+                    return true;
+                };
+                auto load_v = [&](int bl) -> bool {
+                    const int st = (int)(vc % VS);
+                    const uint32_t use = vc / VS;
+                    if (use > 0 && !wait(p, L::bVEmpty + st, (use - 1) & 1)) return false;
+                    const int32_t krow = bl < g.npre ? 0 : g.kb0 + (g.b_first + bl - g.npre) * BN;
+                    tc::mbar_arrive_expect_tx(bar(p, L::bVFull + st), L::kBlk);
+                    for (int x = 0; x < D / 64; ++x)
+                        tc::tma_load_3d(pb + L::pV + st * L::kBlk + x * (BN * 128), &tv, x * 64,
+                                        krow, g.kvbh, bar(p, L::bVFull + st));
+                    ++vc;
+                    return true;
+                };
+                constexpr bool kTmaDiag = DS > 0 && !LDW;
+                int nd = 0;
+                if constexpr (kTmaDiag) {
+                    const int64_t last = (g.q0 + BM - 1 < T - 1) ? g.q0 + BM - 1 : T - 1;
                     for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last) ? 1 : 0;
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int64_t i = g.q0 + 4 * lane + h;
-                        if (i < T) {
-                            cstart[h] = a.rowptr[i];
-                            cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
-                            if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
-                            nd = nd > (int)cres[h] ? nd : (int)cres[h];
-                        }
-                    }
-                    for (int o = 16; o > 0; o >>= 1) {
-                        const int x = __shfl_xor_sync(0xffffffffu, nd, o);
-                        nd = nd > x ? nd : x;
-                    }
+                    const int slot = (int)(lt & 1);
+                    if (lt >= 2 && !wait(p, L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1)))
+                        break;
+                    info[slot] = nd;
+                    tc::mbar_arrive(bar(p, L::bInfoFull + slot));
                 }
-            }
-            const int slot = (int)(lt & 1);
-            if (lt >= 2 && !wait(p, L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1))) break;
-            if (lane == 0) {
-                info[slot] = nd;
-                tc::mbar_arrive(bar(p, L::bInfoFull + slot));
-            }
-            // band ring loads (lane 0)
-            auto load_k = [&](int bl) -> bool {
-                const int st = (int)(kc % KS);
-                const uint32_t use = kc / KS;
-                if (use > 0 && !wait(p, L::bKEmpty + st, (use - 1) & 1)) return false;
-                const int32_t krow = g.kb0 + (g.b_first + bl) * BN;
-                tc::mbar_arrive_expect_tx(bar(p, L::bKFull + st), L::kBlk);
-                for (int x = 0; x < D / 64; ++x)
-                    tc::tma_load_3d(pb + L::pK + st * L::kBlk + x * (BN * 128), &tk, x * 64, krow,
-                                    (int32_t)g.bh, bar(p, L::bKFull + st));
-                ++kc;
-                return true;
-            };
-            auto load_v = [&](int bl) -> bool {
-                const int st = (int)(vc % VS);
-                const uint32_t use = vc / VS;
-                if (use > 0 && !wait(p, L::bVEmpty + st, (use - 1) & 1)) return false;
-                const int32_t krow = g.kb0 + (g.b_first + bl) * BN;
-                tc::mbar_arrive_expect_tx(bar(p, L::bVFull + st), L::kBlk);
-                for (int x = 0; x < D / 64; ++x)
-                    tc::tma_load_3d(pb + L::pV + st * L::kBlk + x * (BN * 128), &tv, x * 64, krow,
-                                    (int32_t)g.bh, bar(p, L::bVFull + st));
-                ++vc;
-                return true;
-            };
-            // the band blocks that fit the rings go before the diagonal ones
-            const int n_pre = g.n_band < (KS < VS ? KS : VS) ? g.n_band : (KS < VS ? KS : VS);
-            int okl = 1;
-            if (lane == 0) {
                 // Q of this tile once the previous tile's last S MMA and the
                 // softmax warps are done with the buffer
-                if (lt >= 1 && !wait(p, L::bQEmpty, (uint32_t)((lt - 1) & 1))) okl = 0;
-                if (okl) {
-                    tc::mbar_arrive_expect_tx(bar(p, L::bQFull), L::kQTile);
-                    for (int x = 0; x < D / 64; ++x)
-                        tc::tma_load_3d(pb + L::pQ + x * (BM * 128), &tq, x * 64, (int32_t)g.q0,
-                                        (int32_t)g.bh, bar(p, L::bQFull));
-                }
-                for (int bl = 0; okl && bl < n_pre; ++bl)
-                    if (!load_k(bl) || !load_v(bl)) okl = 0;
-            }
-            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
-            auto prefetch_blk = [&](int d) {
-                const int32_t krow = (int32_t)(g.q0 - a.offs[a.n_off - nd + d]);
-                for (int x = 0; x < D / 64; ++x) {
-                    tc::tma_prefetch_3d(&tkd, x * 64, krow, (int32_t)g.bh);
-                    tc::tma_prefetch_3d(&tvd, x * 64, krow, (int32_t)g.bh);
-                }
-            };
-            if (DS > 0 && a.kind == 0 && lane == 0)
-                for (int d = 0; d < nd && d < a.prefetch; ++d) prefetch_blk(d);
-            for (int d = 0; ok && d < nd; ++d) {
-                const int st = (int)(dc % DSX);
-                const uint32_t use = dc / DSX;
-                const uint32_t kdst = pb + L::pDK + st * L::kQTile;
-                const uint32_t vdst = pb + L::pDV + st * L::kQTile;
-                if (use > 0 && !wait(p, L::bDiagEmpty + st, (use - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) tc::mbar_arrive_expect_tx(bar(p, L::bDiagFull + st), 2 * L::kQTile);
-                if (a.kind == 0) {
-                    if (lane == 0) {
-                        // distance links: keys q0-o .. q0+127-o, one box each
-                        const int32_t krow = (int32_t)(g.q0 - a.offs[a.n_off - nd + d]);
+                if (lt >= 1 && !wait(p, L::bQEmpty, (uint32_t)((lt - 1) & 1))) break;
+                tc::mbar_arrive_expect_tx(bar(p, L::bQFull), L::kQTile);
+                for (int x = 0; x < D / 64; ++x)
+                    tc::tma_load_3d(pb + L::pQ + x * (BM * 128), &tq, x * 64, (int32_t)g.q0,
+                                    (int32_t)g.bh, bar(p, L::bQFull));
+                const int nblk = g.npre + g.n_band;
+                int bl = 0;
+                if constexpr (kTmaDiag) {
+                    // the band blocks that fit the rings go before the distance blocks
+                    const int n_pre = nblk < (KS < VS ? KS : VS) ? nblk : (KS < VS ? KS : VS);
+                    for (; ok && bl < n_pre; ++bl) ok = load_k(bl) && load_v(bl);
+                    // distance o: keys q0-o .. q0+127-o, one box per 64 columns;
+                    // with K and V beyond L2 the block kPrefetchBlocks ahead is
+                    // prefetched into L2 first
+                    auto krow_of = [&](int d) { return (int32_t)(g.q0 - a.offs[a.n_off - nd + d]); };
+                    auto prefetch_blk = [&](int d) {
                         for (int x = 0; x < D / 64; ++x) {
-                            tc::tma_load_3d(kdst + x * (BM * 128), &tkd, x * 64, krow,
-                                            (int32_t)g.bh, bar(p, L::bDiagFull + st));
-                            tc::tma_load_3d(vdst + x * (BM * 128), &tvd, x * 64, krow,
-                                            (int32_t)g.bh, bar(p, L::bDiagFull + st));
+                            tc::tma_prefetch_3d(&tkd, x * 64, krow_of(d), g.kvbh);
+                            tc::tma_prefetch_3d(&tvd, x * 64, krow_of(d), g.kvbh);
                         }
-                        if (d + a.prefetch < nd && a.prefetch > 0) prefetch_blk(d + a.prefetch);
+                    };
+                    if (a.l2pf)
+                        for (int d = 0; d < nd && d < kPrefetchBlocks; ++d) prefetch_blk(d);
+                    for (int d = 0; ok && d < nd; ++d) {
+                        const int st = (int)(dc % DS);
+                        const uint32_t use = dc / DS;
+                        if (use > 0 && !wait(p, L::bDiagEmpty + st, (use - 1) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t kdst = pb + L::pDK + st * L::kQTile;
+                        const uint32_t vdst = pb + L::pDV + st * L::kQTile;
+                        tc::mbar_arrive_expect_tx(bar(p, L::bDiagFull + st), 2 * L::kQTile);
+                        for (int x = 0; x < D / 64; ++x) {
+                            tc::tma_load_3d(kdst + x * (BM * 128), &tkd, x * 64, krow_of(d), g.kvbh,
+                                            bar(p, L::bDiagFull + st));
+                            tc::tma_load_3d(vdst + x * (BM * 128), &tvd, x * 64, krow_of(d), g.kvbh,
+                                            bar(p, L::bDiagFull + st));
+                        }
+                        if (a.l2pf && d + kPrefetchBlocks < nd) prefetch_blk(d + kPrefetchBlocks);
+                        ++dc;
                     }
-                } else {
-                    // CSR slot d: 4-row TMA gathers of K and V rows
-                    // (unswizzled); a row without slot d loads its own key
-                    int32_t rr[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int64_t i = g.q0 + 4 * lane + h;
-                        const int64_t j = d < cres[h] ? (int64_t)cj[h] : (i < T ? i : 0);
-                        rr[h] = (int32_t)(g.bh * T + j);
-                    }
-#pragma unroll
-                    for (int x = 0; x < D / 64; ++x) {
-                        const uint32_t off = x * (BM * 128) + 4 * lane * 128;
-                        tc::tma_gather4(kdst + off, &tkr, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                        bar(p, L::bDiagFull + st));
-                        tc::tma_gather4(vdst + off, &tvr, x * 64, rr[0], rr[1], rr[2], rr[3],
-                                        bar(p, L::bDiagFull + st));
-                    }
-#pragma unroll
-                    for (int h = 0; h < 4; ++h)
-                        if (d + 1 < cres[h]) cj[h] = a.colidx[cstart[h] + d + 1];
                 }
-                ++dc;
+                for (; ok && bl < nblk; ++bl) ok = load_k(bl) && load_v(bl);
             }
-            if (!ok) break;
-            if (lane == 0)
-                for (int bl = n_pre; okl && bl < g.n_band; ++bl)
-                    if (!load_k(bl) || !load_v(bl)) okl = 0;
-            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
         }
       } else if ((warp >> 1) < NP) {
         // ---------------- MMA issuer of pipeline p: S of block g, then P V of
@@ -388,10 +365,11 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             };
             int64_t lt = 0;
             for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
-                const TileGeom g = tile_geom(t, ntq, T, W);
+                const TileGeom g = tile_geom(t, ntq, T, a.We, a.H, a.Hkv, a.gp);
                 if (!wait(p, L::bQFull, (uint32_t)(lt & 1))) break;
                 const uint32_t qa = pb + L::pQ;
-                for (int bl = 0; bl < g.n_band; ++bl) {
+                const int nblk = g.npre + g.n_band;
+                for (int bl = 0; bl < nblk; ++bl) {
                     const int st = (int)(kc % KS), sb = (int)(gb & 1);
                     if (!wait(p, L::bKFull + st, (kc / KS) & 1) ||
                         (gb >= 2 && !wait(p, L::bSFree + sb, ((gb >> 1) - 1) & 1))) {
@@ -410,7 +388,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     }
                     tc::mma_commit(bar(p, L::bSFull + sb));
                     tc::mma_commit(bar(p, L::bKEmpty + st));
-                    if (bl == g.n_band - 1) tc::mma_commit(bar(p, L::bQEmpty));
+                    if (bl == nblk - 1) tc::mma_commit(bar(p, L::bQEmpty));
                     ++kc;
                     // the softmax of this block overlaps P V of the previous one
                     if (have_pv && !do_pv()) {
@@ -438,158 +416,144 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         const int p = (warp - 4) >> 2;
         const int r = tid - 128 - 128 * p;
         uint8_t *pm = sm + p * L::kPipe;
-        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
         const uint32_t lane_off = (uint32_t)(((warp - 4) & 3) * 32) << 16;
         const uint32_t tS = tmem + p * L::tPipe + lane_off + L::tS0;
         const uint32_t tO = tmem + p * L::tPipe + lane_off + L::tO;
         const float c2 = a.scale2;
-        uint32_t dc = 0, gb = 0;  // diagonal blocks and band blocks consumed (all tiles)
-        uint32_t group_uses = 0;  // phases of the softmax group barrier
+        const int wq = r >> 5;    // warp within the group: rows 32 wq .. 32 wq + 31
+        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
+        uint32_t gb = 0, dc = 0;  // band and TMA distance blocks consumed (all tiles)
         bool ok = true;
         int64_t lt = 0;
         for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
-            const TileGeom g = tile_geom(t, ntq, T, W);
+            const TileGeom g = tile_geom(t, ntq, T, a.We, a.H, a.Hkv, a.gp);
             const int32_t q0 = g.q0, bh = g.bh;
             const int32_t i = q0 + r;
-            const int slot = (int)(lt & 1);
             float m_run = -INFINITY, l_run = 0.f;
-            if (!wait(p, L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1))) break;
-            const int nd = info[slot];
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
 
             // --- diagonal blocks: q row from the Q tile, one key/value row per
-            // block; bf16 x bf16 -> fp32 FMAs (exact products), p rounded to
+            // slot; bf16 x bf16 -> fp32 FMAs (exact products), p rounded to
             // bf16 for the weighted sum as the band path's P is; running max
             // rescaled lazily (only when it grows by more than 2^8)
             {
                 float acc[D];
 #pragma unroll
                 for (int x = 0; x < D; ++x) acc[x] = 0.f;
-                if (DS > 0 && nd > 0) {
-                    ok = wait(p, L::bQFull, (uint32_t)(lt & 1));
-                    // Structured blocks are swizzled like Q: q in logical
-                    // order.  CSR gathers are unswizzled: reading them at the
-                    // swizzled address gives chunk c ^ (r & 7), which pairs with
-                    // the physical (unpermuted-address) chunks of the Q row; the
-                    // accumulator is then in that permuted order (undone below).
+                if constexpr (DS > 0) {
+                    // slots: the tile's distance blocks (count from the
+                    // producer), or, for CSR lists, the longest residual list
+                    // of this warp's rows
+                    int nd = 0;
+                    int64_t cst = 0;
+                    int32_t resid = 0;
+                    if constexpr (!LDW) {
+                        const int slot = (int)(lt & 1);
+                        ok = __all_sync(0xffffffffu,
+                                        wait(p, L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1)));
+                        nd = ok ? info[slot] : 0;
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
+                    } else {
+                        if (i < T) {
+                            // the shared prefix keys outside the window are the
+                            // first entries of the sorted list: the prefix block
+                            // takes them
+                            int32_t gc = i - W + 1 < a.gp ? i - W + 1 : a.gp;
+                            gc = gc > 0 ? gc : 0;
+                            cst = a.rowptr[i] + gc;
+                            resid = (int32_t)(a.rowptr[i + 1] - cst - ((i + 1 < W) ? i + 1 : W));
+                        }
+                        nd = (int)__reduce_max_sync(0xffffffffu, (unsigned)resid);
+                    }
+                    const int dfirst = a.n_off - nd;  // distance index of slot 0 (keys ascending)
+                    // key of this thread's row in slot d, -1 if the row has none
+                    auto key_of = [&](int d) -> int32_t {  // (CSR slots)
+                        return d < resid ? __ldg(a.colidx + cst + d) : -1;
+                    };
+                    const size_t slice = (size_t)g.kvbh * (size_t)T * D;
                     uint32_t qw[D / 2];
-                    if (ok) {
+                    // one slot: dot product with the row's key, online-softmax
+                    // update, p-weighted value row into acc (Q is read on the
+                    // first slot, once its load has landed)
+                    auto body = [&](int d, int st) {
+                        if (d == 0) {
+                            ok = __all_sync(0xffffffffu, wait(p, L::bQFull, (uint32_t)(lt & 1)));
+                            if (ok) {
+#pragma unroll
+                                for (int c = 0; c < D / 8; ++c) {
+                                    const uint4 w4 = *(const uint4 *)(pm + L::pQ +
+                                                                      (c >> 3) * (BM * 128) +
+                                                                      tc::sw128_off(r, c & 7));
+                                    qw[4 * c] = w4.x;
+                                    qw[4 * c + 1] = w4.y;
+                                    qw[4 * c + 2] = w4.z;
+                                    qw[4 * c + 3] = w4.w;
+                                }
+                            }
+                        }
+                        const bool valid = LDW ? (d < resid) : (i < T && i >= a.offs[dfirst + d]);
+                        if (!ok || !valid) return;
+                        const uint8_t *kr = pm + L::pDK + st * L::kQTile;
+                        const uint8_t *vr = pm + L::pDV + st * L::kQTile;
+                        // eight independent partial sums (short dependency chains)
+                        float sp[8];
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) sp[x] = 0.f;
 #pragma unroll
                         for (int c = 0; c < D / 8; ++c) {
-                            const uint32_t qoff =
-                                (c >> 3) * (BM * 128) +
-                                (a.kind == 0 ? tc::sw128_off(r, c & 7)
-                                             : (uint32_t)r * 128u + ((c & 7) << 4));
-                            const uint4 w4 = *(const uint4 *)(pm + L::pQ + qoff);
-                            qw[4 * c] = w4.x;
-                            qw[4 * c + 1] = w4.y;
-                            qw[4 * c + 2] = w4.z;
-                            qw[4 * c + 3] = w4.w;
-                        }
-                    }
-                    int32_t resid = 0;
-                    if (a.kind == 1 && i < T) {
-                        const int64_t deg = a.rowptr[i + 1] - a.rowptr[i];
-                        resid = (int32_t)(deg - ((i + 1 < W) ? i + 1 : W));
-                    }
-                    for (int d = 0; ok && d < nd; ++d) {
-                        const int st = (int)(dc % DSX);
-                        if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
-                            ok = false;
-                            break;
-                        }
-                        bool valid;
-                        if (a.kind == 0)
-                            valid = i < T && i >= a.offs[a.n_off - nd + d];
-                        else
-                            valid = d < resid;
-                        if (valid) {
-                            const uint8_t *kr = pm + L::pDK + st * L::kQTile;
-                            const uint8_t *vr = pm + L::pDV + st * L::kQTile;
-                            // eight independent partial sums (short dependency chains)
-                            float sp[8];
+                            const uint4 w4 = *(const uint4 *)(kr + (c >> 3) * (BM * 128) +
+                                                              tc::sw128_off(r, c & 7));
+                            const uint32_t kw[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                            for (int x = 0; x < 8; ++x) sp[x] = 0.f;
-#pragma unroll
-                            for (int c = 0; c < D / 8; ++c) {
-                                const uint4 w4 = *(const uint4 *)(kr + (c >> 3) * (BM * 128) +
-                                                                  tc::sw128_off(r, c & 7));
-                                const uint32_t kw[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    sp[2 * e] = tc::fma_bf_lo(qw[4 * c + e], kw[e], sp[2 * e]);
-                                    sp[2 * e + 1] =
-                                        tc::fma_bf_hi(qw[4 * c + e], kw[e], sp[2 * e + 1]);
-                                }
-                            }
-                            const float s = (((sp[0] + sp[1]) + (sp[2] + sp[3])) +
-                                             ((sp[4] + sp[5]) + (sp[6] + sp[7]))) *
-                                            c2;
-                            if (s > m_run + kRescaleThreshold) {
-                                const float al = tc::ex2(m_run - s);  // 0 on the first edge
-#pragma unroll
-                                for (int x = 0; x < D; ++x) acc[x] *= al;
-                                l_run *= al;
-                                m_run = s;
-                            }
-                            const float pr = tc::ex2(s - m_run);
-                            l_run += pr;
-                            const uint32_t p2 = tc::pack_bf16x2(pr, pr);
-#pragma unroll
-                            for (int c = 0; c < D / 8; ++c) {
-                                const uint4 w4 = *(const uint4 *)(vr + (c >> 3) * (BM * 128) +
-                                                                  tc::sw128_off(r, c & 7));
-                                const uint32_t vw[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    acc[8 * c + 2 * e] =
-                                        tc::fma_bf_lo(p2, vw[e], acc[8 * c + 2 * e]);
-                                    acc[8 * c + 2 * e + 1] =
-                                        tc::fma_bf_hi(p2, vw[e], acc[8 * c + 2 * e + 1]);
-                                }
+                            for (int e = 0; e < 4; ++e) {
+                                sp[2 * e] = tc::fma_bf_lo(qw[4 * c + e], kw[e], sp[2 * e]);
+                                sp[2 * e + 1] = tc::fma_bf_hi(qw[4 * c + e], kw[e], sp[2 * e + 1]);
                             }
                         }
-                        const bool hold = (a.kind == 1) && (d == nd - 1);
-                        if (!hold) {
+                        const float s = (((sp[0] + sp[1]) + (sp[2] + sp[3])) +
+                                         ((sp[4] + sp[5]) + (sp[6] + sp[7]))) *
+                                        c2;
+                        if (s > m_run + kRescaleThreshold) {
+                            const float al = tc::ex2(m_run - s);  // 0 on the first edge
+#pragma unroll
+                            for (int x = 0; x < D; ++x) acc[x] *= al;
+                            l_run *= al;
+                            m_run = s;
+                        }
+                        const float pr = tc::ex2(s - m_run);
+                        l_run += pr;
+                        const uint32_t p2 = tc::pack_bf16x2(pr, pr);
+#pragma unroll
+                        for (int c = 0; c < D / 8; ++c) {
+                            const uint4 w4 = *(const uint4 *)(vr + (c >> 3) * (BM * 128) +
+                                                              tc::sw128_off(r, c & 7));
+                            const uint32_t vw[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                acc[8 * c + 2 * e] = tc::fma_bf_lo(p2, vw[e], acc[8 * c + 2 * e]);
+                                acc[8 * c + 2 * e + 1] =
+                                    tc::fma_bf_hi(p2, vw[e], acc[8 * c + 2 * e + 1]);
+                            }
+                        }
+                    };
+                    if constexpr (LDW) {
+                        rows::warp_slots<D, DS>(
+                            nd, sbase + (uint32_t)(p * L::kPipe + L::pDK),
+                            sbase + (uint32_t)(p * L::kPipe + L::pDV), (uint32_t)L::kQTile, a.k,
+                            a.v, a.l2pf > 0, lane, wq, [&](int) { return slice; }, key_of, body);
+                    } else {
+                        for (int d = 0; ok && d < nd; ++d) {
+                            const int st = (int)(dc % DS);
+                            if (!__all_sync(0xffffffffu,
+                                            wait(p, L::bDiagFull + st, (dc / DS) & 1))) {
+                                ok = false;
+                                break;
+                            }
+                            body(d, st);
                             __syncwarp();
                             if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
+                            ++dc;
                         }
-                        ++dc;
-                    }
-                    if (ok && a.kind == 1) {
-                        // undo the chunk permutation (per 64-column half) through
-                        // the last diagonal stage, whose release was held back:
-                        // once every row is done with it, thread r uses 256 bytes
-                        // (rows < 64 in its K half, the others in its V half)
-                        const int st = (int)((dc - 1) % DSX);
-                        tc::mbar_arrive(bar(p, L::bGroup));
-                        if (!wait(p, L::bGroup, group_uses & 1)) ok = false;
-                        ++group_uses;
-                        float *scr = (float *)(pm + (r < 64 ? L::pDK : L::pDV) + st * L::kQTile) +
-                                     (size_t)(r & 63) * D;
-#pragma unroll
-                        for (int hh = 0; hh < D / 64; ++hh) {
-#pragma unroll
-                            for (int tt = 0; tt < 8; ++tt) {
-                                const int lc = tt ^ (r & 7);
-                                const float *src = acc + 64 * hh + 8 * tt;
-                                *(float4 *)(scr + 8 * lc) = make_float4(src[0], src[1], src[2], src[3]);
-                                *(float4 *)(scr + 8 * lc + 4) =
-                                    make_float4(src[4], src[5], src[6], src[7]);
-                            }
-#pragma unroll
-                            for (int tt = 0; tt < 16; ++tt) {
-                                const float4 f = *(const float4 *)(scr + 4 * tt);
-                                acc[64 * hh + 4 * tt] = f.x;
-                                acc[64 * hh + 4 * tt + 1] = f.y;
-                                acc[64 * hh + 4 * tt + 2] = f.z;
-                                acc[64 * hh + 4 * tt + 3] = f.w;
-                            }
-                            scr += 64;
-                        }
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
                     }
                 }
                 if (!ok) break;
@@ -612,9 +576,10 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
 
             // --- band blocks
             uint32_t gb_last = gb;
-            for (int bl = 0; ok && bl < g.n_band; ++bl, ++gb) {
+            const int nblk = g.npre + g.n_band;
+            for (int bl = 0; ok && bl < nblk; ++bl, ++gb) {
                 const int sb = (int)(gb & 1);
-                const int32_t b = g.b_first + bl;
+                const int32_t b = g.b_first + bl - g.npre;
                 gb_last = gb;
                 if (!wait(p, L::bSFull + sb, (gb >> 1) & 1)) {
                     ok = false;
@@ -625,17 +590,39 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 // the column range [c_lo, c_hi] of this block.  Scores stay raw
                 // (the scale is folded into the exponent's FFMA); a masked raw
                 // score is set to the extreme that the max/min below ignores.
+                // block coordinates u = BN b + c from key q0 - We + 1: row r
+                // keeps its window u in [r + We - W, r + We - 1], the folded
+                // links u = r + We - 1 - o, and keys >= 0 (u >= We - 1 - q0)
+                const int32_t We = a.We;
                 const int32_t u0 = b * BN;
-                const bool need_mask =
-                    (u0 < BM - 1) || (u0 + BN - 1 > W - 1) || (u0 + q0 < W - 1);
+                const bool pre = bl < g.npre;
+                const bool need_mask = pre || a.nf > 0 || (u0 < BM - 1) ||
+                                       (u0 + BN - 1 > We - 1) || (u0 + q0 < We - 1);
                 int c_lo = 0, c_hi = BN - 1;
-                if (need_mask) {
-                    const int32_t lo = (r > W - 1 - q0) ? r : W - 1 - q0;
-                    const int32_t hi = r + W - 1;
+                int fc[kMaxFold];  // folded-link column of this row in the block, -1 if none
+#pragma unroll
+                for (int x = 0; x < kMaxFold; ++x) fc[x] = -1;
+                bool fany = false;
+                if (pre) {
+                    // shared prefix: keys 0 .. min(gp, i - W + 1) - 1
+                    const int32_t n = i - W + 1 < a.gp ? i - W + 1 : a.gp;
+                    c_hi = n > 0 ? n - 1 : -1;
+                } else if (need_mask) {
+                    const int32_t kmin = We - 1 - q0;  // u of key 0
+                    const int32_t lo = (r + We - W > kmin) ? r + We - W : kmin;
+                    const int32_t hi = r + We - 1;
                     c_lo = lo - u0 < 0 ? 0 : (lo - u0 > BN ? BN : lo - u0);
                     c_hi = hi - u0 > BN - 1 ? BN - 1 : (hi - u0 < -1 ? -1 : hi - u0);
+#pragma unroll
+                    for (int x = 0; x < kMaxFold; ++x) {
+                        const int32_t u = r + We - 1 - a.fold[x];
+                        if (x < a.nf && u >= kmin && u >= u0 && u < u0 + BN) {
+                            fc[x] = u - u0;
+                            fany = true;
+                        }
+                    }
                 }
-                if (need_mask && __all_sync(0xffffffffu, c_lo > c_hi)) {
+                if (need_mask && __all_sync(0xffffffffu, c_lo > c_hi && !fany)) {
                     // no row of this warp keeps a key of the block: P = 0
                     uint32_t z[BN / 2];
 #pragma unroll
@@ -656,7 +643,12 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 const float ext = pos ? -INFINITY : INFINITY;
                 if (need_mask) {
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) s[c] = (c >= c_lo && c <= c_hi) ? s[c] : ext;
+                    for (int c = 0; c < BN; ++c) {
+                        bool keep = c >= c_lo && c <= c_hi;
+#pragma unroll
+                        for (int x = 0; x < kMaxFold; ++x) keep |= (c == fc[x]);
+                        s[c] = keep ? s[c] : ext;
+                    }
                 }
                 float mr[8];
 #pragma unroll
@@ -787,14 +779,14 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     }
 }
 
-template <int D, int NP, int KS, int VS, int DS>
+template <int D, int NP, int KS, int VS, int DS, bool LDW>
 sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_graph_s *g, float scale, sa_tensor *out, float *lse,
                           cudaStream_t s) {
     using L = Layout<D, NP, KS, VS, DS>;
     static_assert(L::kAlloc <= 232448, "shared memory budget");
     constexpr int kThreads = 128 + 128 * NP;
-    auto kern = band_fwd_kernel<D, NP, KS, VS, DS>;
+    auto kern = band_fwd_kernel<D, NP, KS, VS, DS, LDW>;
     if (NP == 2) {
         // setmaxnreg.inc waits until the CTA's pool holds the registers it
         // asks for: the launch must provide the whole split
@@ -810,27 +802,30 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
             return SA_ERR_CUDA;
         }
     }
-    const int64_t BH = q->B * q->H, T = q->T;
-    CUtensorMap mq, mk, mv, mkd, mvd, mkr, mvr;
-    if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BM) || !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BH, BN) ||
-        !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BH, BN) ||
-        !sa_tmap_bf16_3d(&mkd, k->ptr, D, T, BH, BM) ||
-        !sa_tmap_bf16_3d(&mvd, v->ptr, D, T, BH, BM) ||
-        !sa_tmap_bf16_rows(&mkr, k->ptr, D, (uint64_t)(BH * T)) ||
-        !sa_tmap_bf16_rows(&mvr, v->ptr, D, (uint64_t)(BH * T))) {
+    const int64_t BH = q->B * q->H, BHkv = k->B * k->H, T = q->T;
+    CUtensorMap mq, mk, mv, mkd, mvd;  // 64-row band boxes, 128-row distance blocks
+    if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BM) ||
+        !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BHkv, BN) ||
+        !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BHkv, BN) ||
+        !sa_tmap_bf16_3d(&mkd, k->ptr, D, T, BHkv, BM) ||
+        !sa_tmap_bf16_3d(&mvd, v->ptr, D, T, BHkv, BM)) {
         sa_record_cuda_error(cudaErrorInvalidValue, "band_fwd: tensor map encoding");
         return SA_ERR_CUDA;
     }
     FwdArgs a{};
     a.T = T;
     a.BH = BH;
+    a.H = q->H;
+    a.Hkv = k->H;
     a.W = g->W;
     a.kind = g->kind;
-    a.n_off = g->kind == 0 ? g->n_off : 0;
-    a.prefetch = (double)BH * (double)T * D * 2 * 2 > kL2ResidentBytes ? kPrefetchAhead : 0;
-    for (int x = 0; x < SA_MAX_OFFSETS; ++x) a.offs[x] = x < a.n_off ? g->offs[x] : 0;
+    a.gp = g->kind == 1 ? g->gprefix : 0;
+    a.We = sa_fold_links(g, BN, kMaxFold, a.fold, &a.nf, a.offs, &a.n_off);
+    a.l2pf = (double)BHkv * (double)T * D * 2 * 2 > kL2ResidentBytes ? 1 : 0;
     a.rowptr = g->rowptr;
     a.colidx = g->colidx;
+    a.k = (const __nv_bfloat16 *)k->ptr;
+    a.v = (const __nv_bfloat16 *)v->ptr;
     a.out = (__nv_bfloat16 *)out->ptr;
     a.lse = lse;
     a.scale2 = scale * kLog2e;
@@ -844,7 +839,7 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     SA_CUDA_TRY(sa_sm_count(&sms));
     const unsigned grid = (unsigned)(nctas < sms ? nctas : sms);
     SA_LAUNCH("band_fwd", s,
-              kern<<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, mkd, mvd, mkr, mvr, a));
+              kern<<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, mkd, mvd, a));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
@@ -854,7 +849,8 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
 bool sa_band_fwd_supported(const sa_tensor *q, const sa_graph_s *g) {
     if (q->dtype != SA_BF16 || (q->D != 64 && q->D != 128)) return false;
     if (g->W < 1) return false;                       // no band: gather path
-    if (q->B * q->H > 65535 || q->T >= ((int64_t)1 << 31)) return false;
+    // 32-bit tile coordinates (TMA takes int32 row and slice indices)
+    if (q->B * q->H >= ((int64_t)1 << 31) || q->T >= ((int64_t)1 << 31)) return false;
     if (g->kind == 1 && !g->rowptr) return false;
     return true;
 }
@@ -863,12 +859,15 @@ sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
                       const sa_graph_s *g, const GraphView &, float scale, sa_tensor *out,
                       float *lse, cudaStream_t s) {
     const bool diag = (g->kind == 0) ? g->n_off > 0 : g->max_resid > 0;
-    // <D, pipelines, K stages, V stages, diagonal stages>, sized to the 227 KB
-    // of shared memory
+    const bool csr = g->kind == 1;
+    // <D, pipelines, K stages, V stages, diagonal stages, per-warp slots>,
+    // sized to the 227 KB of shared memory
     if (q->D == 64) {
-        return diag ? launch_band_fwd<64, 2, 2, 2, 2>(q, k, v, g, scale, out, lse, s)
-                    : launch_band_fwd<64, 2, 4, 4, 0>(q, k, v, g, scale, out, lse, s);
+        if (!diag) return launch_band_fwd<64, 2, 4, 4, 0, false>(q, k, v, g, scale, out, lse, s);
+        return csr ? launch_band_fwd<64, 2, 2, 2, 2, true>(q, k, v, g, scale, out, lse, s)
+                   : launch_band_fwd<64, 2, 2, 2, 2, false>(q, k, v, g, scale, out, lse, s);
     }
-    return diag ? launch_band_fwd<128, 1, 2, 2, 2>(q, k, v, g, scale, out, lse, s)
-                : launch_band_fwd<128, 2, 3, 2, 0>(q, k, v, g, scale, out, lse, s);
+    if (!diag) return launch_band_fwd<128, 2, 3, 2, 0, false>(q, k, v, g, scale, out, lse, s);
+    return csr ? launch_band_fwd<128, 1, 2, 2, 2, true>(q, k, v, g, scale, out, lse, s)
+               : launch_band_fwd<128, 1, 2, 2, 2, false>(q, k, v, g, scale, out, lse, s);
 }

@@ -32,6 +32,7 @@
 #include <stdint.h>
 
 #include "sa_band.cuh"
+#include "sa_rows.cuh"
 #include "tc_common.cuh"
 #include "tmap.cuh"
 
@@ -40,18 +41,29 @@ namespace {
 constexpr int BM = 128;  // rows a tile owns
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Distance links inside the key span the band blocks of a tile cover anyway
+// are folded into the band blocks (at most kMaxFold; sa_fold_links).
+constexpr int kMaxFold = 4;
+
 struct BwdArgs {
     int64_t T;
-    int64_t BH;
+    int64_t BH;          // query slices B*H
+    int64_t H, Hkv;      // query and key/value heads (grouped-query attention)
     int32_t W;
+    int32_t We;          // span of the band blocks: W, or the longest folded link + 1
+    int32_t nf;          // folded links
+    int32_t fold[kMaxFold];
     int32_t kind;
     int32_t n_off;
+    int32_t l2pf;        // prefetch diagonal rows into L2 (they do not fit in it)
     int64_t offs[SA_MAX_OFFSETS];  // descending
     const int64_t *rowptr;
     const int32_t *colidx;
     const int64_t *rev_rowptr;
     const int32_t *rev_colidx;
     const __nv_bfloat16 *o;        // forward output (Delta)
+    // diagonal rows are copied from these: k, v (dQ pass), q, dout (dK/dV pass)
+    const __nv_bfloat16 *k, *v, *q, *dout;
     const float *lse;
     float *delta;
     // Optional cache of (p, dS) per distance edge, written by dQ, read by
@@ -65,7 +77,7 @@ struct BwdArgs {
 
 // Register budgets with two pipelines (384 threads launched at 168 each).
 struct BwdRegs {
-    static constexpr int producer = 72, compute = 216;
+    static constexpr int producer = 56, compute = 224;
     static_assert(128 * producer + 256 * compute <= 384 * 168, "register split");
 };
 
@@ -127,29 +139,6 @@ __device__ __forceinline__ float dot_bf_smem_smem(const uint8_t *ta, const uint8
     return sum8(sp);
 }
 
-// a . b, a = row r of a swizzled tile read in physical chunk order, b = row r
-// of an unswizzled gathered tile read at the swizzled address (both give
-// logical chunk t ^ (r & 7) at step t).
-template <int D>
-__device__ __forceinline__ float dot_bf_phys_gathered(const uint8_t *ta, const uint8_t *tb,
-                                                      int rows, int r) {
-    float sp[8];
-#pragma unroll
-    for (int x = 0; x < 8; ++x) sp[x] = 0.f;
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        const uint4 x = *(const uint4 *)(ta + (c >> 3) * (rows * 128) + r * 128 + ((c & 7) << 4));
-        const uint4 y = *(const uint4 *)(tb + tile_off(rows, r, c));
-        const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            sp[2 * e] = tc::fma_bf_lo(xa[e], yb[e], sp[2 * e]);
-            sp[2 * e + 1] = tc::fma_bf_hi(xa[e], yb[e], sp[2 * e + 1]);
-        }
-    }
-    return sum8(sp);
-}
-
 // a . b, a packed bf16 pairs in registers (chunk c in a[4c .. 4c+3]), b row r
 // of a tile read at the swizzled address.
 template <int D>
@@ -188,35 +177,41 @@ __device__ __forceinline__ void axpy_bf_smem(float *acc, float a, const uint8_t 
     }
 }
 
-// acc holds chunk t at logical chunk t ^ (r & 7) (per 64-column half): put it
-// back in logical order through a D-float scratch row in shared memory.
+// TMEM row (D fp32 columns) += bf16(a) * (row r of a tile), 32 columns at a
+// time (for D = 128, whose two accumulators do not fit in registers).
 template <int D>
-__device__ __forceinline__ void unpermute_row(float *acc, float *scr_row, int r) {
+__device__ __forceinline__ void tmem_axpy_row(uint32_t taddr, float a, const uint8_t *tile,
+                                              int rows, int r) {
+    const uint32_t a2 = tc::pack_bf16x2(a, a);
 #pragma unroll
-    for (int t = 0; t < D / 8; ++t) {
-        const int lc = (t & ~7) | ((t & 7) ^ (r & 7));
-        *(float4 *)(scr_row + 8 * lc) =
-            make_float4(acc[8 * t], acc[8 * t + 1], acc[8 * t + 2], acc[8 * t + 3]);
-        *(float4 *)(scr_row + 8 * lc + 4) =
-            make_float4(acc[8 * t + 4], acc[8 * t + 5], acc[8 * t + 6], acc[8 * t + 7]);
-    }
+    for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t w[32];
+        tc::tmem_ld32(taddr + c0, w);
+        tc::tmem_ld_wait();
 #pragma unroll
-    for (int t = 0; t < D / 4; ++t) {
-        const float4 f = *(const float4 *)(scr_row + 4 * t);
-        acc[4 * t] = f.x;
-        acc[4 * t + 1] = f.y;
-        acc[4 * t + 2] = f.z;
-        acc[4 * t + 3] = f.w;
+        for (int c = c0 / 8; c < c0 / 8 + 4; ++c) {
+            const uint4 y = *(const uint4 *)(tile + tile_off(rows, r, c));
+            const uint32_t yb[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int x = 8 * c - c0 + 2 * e;
+                w[x] = __float_as_uint(tc::fma_bf_lo(a2, yb[e], __uint_as_float(w[x])));
+                w[x + 1] = __float_as_uint(tc::fma_bf_hi(a2, yb[e], __uint_as_float(w[x + 1])));
+            }
+        }
+        tc::tmem_st32(taddr + c0, w);
+        tc::tmem_st_wait();
     }
 }
 
+// D fp32 values (zeros for acc == nullptr) -> TMEM row.
 template <int D>
 __device__ __forceinline__ void tmem_store_row(uint32_t taddr, const float *acc) {
 #pragma unroll
     for (int c = 0; c < D; c += 32) {
         uint32_t w[32];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) w[x] = __float_as_uint(acc[c + x]);
+        for (int x = 0; x < 32; ++x) w[x] = acc ? __float_as_uint(acc[c + x]) : 0u;
         tc::tmem_st32(taddr + c, w);
     }
 }
@@ -298,7 +293,6 @@ struct LayoutDQ {
     static constexpr int pDS = pDV + DS * kRow;
     static constexpr int kPipe = pDS + PS * kDSTile;
     static constexpr int kBars = NP * kPipe;
-    static constexpr int DSX = DS > 0 ? DS : 1;
     // barriers of one pipeline (S and dP share a buffer index sb; dS is
     // written over S, so a buffer is free once its dQ MMA is done)
     static constexpr int bQFull = 0, bQEmpty = 1;
@@ -306,11 +300,12 @@ struct LayoutDQ {
     static constexpr int bSFull = bKVEmpty + BS, bSFree = bSFull + SB;
     static constexpr int bDSFull = bSFree + SB, bDQDone = bDSFull + SB;
     static constexpr int bInit = bDQDone + SB;
-    static constexpr int bDiagFull = bInit + 1, bDiagEmpty = bDiagFull + DSX;
+    static constexpr int bPSDone = bInit + 1;              // dS tile consumed by its MMA
+    // distance blocks loaded by the producer with TMA (structured graphs)
+    static constexpr int DSX = DS > 0 ? DS : 1;
+    static constexpr int bDiagFull = bPSDone + (PS > 0 ? PS : 1), bDiagEmpty = bDiagFull + DSX;
     static constexpr int bInfoFull = bDiagEmpty + DSX, bInfoEmpty = bInfoFull + 2;
-    static constexpr int bGroup = bInfoEmpty + 2;
-    static constexpr int bPSDone = bGroup + 1;              // dS tile consumed by its MMA
-    static constexpr int nBarsPipe = bPSDone + (PS > 0 ? PS : 1);
+    static constexpr int nBarsPipe = bInfoEmpty + 2;
     static constexpr int kMisc = kBars + NP * nBarsPipe * 8;  // tmem slot, abort, info[NP][2]
     static constexpr int kTotal = kMisc + 8 + 8 * NP;
     static constexpr int kAlloc = kTotal + 1024;
@@ -336,16 +331,15 @@ struct DQBand {
     }
 };
 
-template <int D, int NP, int BB, int SB, int BS, int DS, int PS>
+// LDW: the diagonal slots are copied by each compute warp (CSR lists); else
+// the producer loads each distance block as TMA boxes (structured graphs).
+template <int D, int NP, int BB, int SB, int BS, int DS, int PS, bool LDW>
 __global__ void __launch_bounds__(128 + 128 * NP, 1)
 band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                    const __grid_constant__ CUtensorMap tkd,
-                   const __grid_constant__ CUtensorMap tvd,
-                   const __grid_constant__ CUtensorMap tkr,
-                   const __grid_constant__ CUtensorMap tvr, const BwdArgs a) {
+                   const __grid_constant__ CUtensorMap tvd, const BwdArgs a) {
     using L = LayoutDQ<D, NP, BB, SB, BS, DS, PS>;
-    constexpr int DSX = L::DSX;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_u32(sm);
@@ -380,7 +374,8 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                 tc::mbar_init(bar(p, L::bDQDone + s), 1);
             }
             tc::mbar_init(bar(p, L::bInit), 4);
-            for (int s = 0; s < DSX; ++s) {
+            for (int s = 0; s < PS; ++s) tc::mbar_init(bar(p, L::bPSDone + s), 1);
+            for (int s = 0; s < L::DSX; ++s) {
                 tc::mbar_init(bar(p, L::bDiagFull + s), 1);
                 tc::mbar_init(bar(p, L::bDiagEmpty + s), 4);
             }
@@ -388,8 +383,6 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                 tc::mbar_init(bar(p, L::bInfoFull + s), 1);
                 tc::mbar_init(bar(p, L::bInfoEmpty + s), 4);
             }
-            tc::mbar_init(bar(p, L::bGroup), 128);
-            for (int s = 0; s < PS; ++s) tc::mbar_init(bar(p, L::bPSDone + s), 1);
         }
         *abort = 0;
         tc::fence_barrier_init();
@@ -403,116 +396,73 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     if (warp < 4) {
         if (NP == 2) tc::regs_dec<BwdRegs::producer>();
       if ((warp >> 1) < NP && (warp & 1) == 0) {
-        // ---------------- producer of pipeline p: diagonal-block count, Q and
-        // dO of the tile, the first band K/V blocks, the diagonal blocks, the rest
+        // ---------------- producer of pipeline p (lane 0): Q and dO of the
+        // tile, the band K/V blocks through their ring and, for a structured
+        // graph, the distance blocks (the count first, to the compute warps)
+        // after the band blocks that fit the ring
         const int p = warp >> 1;
         const uint32_t pb = sbase + (uint32_t)(p * L::kPipe);
         volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
-        uint32_t kvc = 0, dc = 0;
-        bool ok = true;
-        int64_t lt = 0;
-        for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
-            const TileId id = tile_id(t, ntr);
-            const int32_t q0 = id.r0, bh = id.bh;
-            const DQBand<BB> g(q0, T, W);
-            const int64_t last = (q0 + BM - 1 < T - 1) ? q0 + BM - 1 : T - 1;
-            // CSR: lane l owns rows 4l .. 4l+3 (list start, residual count, next key)
-            int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
-            int32_t cj[4] = {0, 0, 0, 0};
-            int nd = 0;
-            if (DS > 0) {
-                if (a.kind == 0) {
+        if (lane == 0) {
+            uint32_t kvc = 0, dc = 0;
+            bool ok = true;
+            int64_t lt = 0;
+            for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
+                const TileId id = tile_id(t, ntr);
+                const int32_t q0 = id.r0, bh = id.bh;
+                const int32_t kvbh = (int32_t)((bh / a.H) * a.Hkv + (bh % a.H) / (a.H / a.Hkv));
+                const DQBand<BB> g(q0, T, a.We);
+                constexpr bool kTmaDiag = DS > 0 && !LDW;
+                int nd = 0;
+                if constexpr (kTmaDiag) {
+                    const int64_t last = (q0 + BM - 1 < T - 1) ? q0 + BM - 1 : T - 1;
                     for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last) ? 1 : 0;
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int64_t i = q0 + 4 * lane + h;
-                        if (i < T) {
-                            cstart[h] = a.rowptr[i];
-                            cres[h] = a.rowptr[i + 1] - cstart[h] - ((i + 1 < W) ? i + 1 : W);
-                            if (cres[h] > 0) cj[h] = a.colidx[cstart[h]];
-                            nd = nd > (int)cres[h] ? nd : (int)cres[h];
+                    const int slot = (int)(lt & 1);
+                    if (lt >= 2 && !wait(p, L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1)))
+                        break;
+                    info[slot] = nd;
+                    tc::mbar_arrive(bar(p, L::bInfoFull + slot));
+                }
+                if (lt >= 1 && !wait(p, L::bQEmpty, (uint32_t)((lt - 1) & 1))) break;
+                tc::mbar_arrive_expect_tx(bar(p, L::bQFull), 2 * L::kRow);
+                tma_rows<D, BM>(pb + L::pQ, &tq, q0, bh, bar(p, L::bQFull));
+                tma_rows<D, BM>(pb + L::pDO, &tdo, q0, bh, bar(p, L::bQFull));
+                auto load_kv = [&](int bl) -> bool {
+                    const int st = (int)(kvc % BS);
+                    const uint32_t use = kvc / BS;
+                    if (use > 0 && !wait(p, L::bKVEmpty + st, (use - 1) & 1)) return false;
+                    const int32_t krow = g.kb0 + (g.b_first + bl) * BB;
+                    tc::mbar_arrive_expect_tx(bar(p, L::bKVFull + st), 2 * L::kBlk);
+                    tma_rows<D, BB>(pb + L::pK + st * L::kBlk, &tk, krow, kvbh,
+                                    bar(p, L::bKVFull + st));
+                    tma_rows<D, BB>(pb + L::pV + st * L::kBlk, &tv, krow, kvbh,
+                                    bar(p, L::bKVFull + st));
+                    ++kvc;
+                    return true;
+                };
+                int bl = 0;
+                if constexpr (kTmaDiag) {
+                    const int n_pre = g.n_band < BS ? g.n_band : BS;
+                    for (; ok && bl < n_pre; ++bl) ok = load_kv(bl);
+                    // distance o: keys q0-o .. q0+127-o
+                    for (int d = 0; ok && d < nd; ++d) {
+                        const int st = (int)(dc % DS);
+                        const uint32_t use = dc / DS;
+                        if (use > 0 && !wait(p, L::bDiagEmpty + st, (use - 1) & 1)) {
+                            ok = false;
+                            break;
                         }
-                    }
-                    for (int o = 16; o > 0; o >>= 1) {
-                        const int x = __shfl_xor_sync(0xffffffffu, nd, o);
-                        nd = nd > x ? nd : x;
-                    }
-                }
-            }
-            const int slot = (int)(lt & 1);
-            if (lt >= 2 && !wait(p, L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1))) break;
-            if (lane == 0) {
-                info[slot] = nd;
-                tc::mbar_arrive(bar(p, L::bInfoFull + slot));
-            }
-            auto load_kv = [&](int bl) -> bool {
-                const int st = (int)(kvc % BS);
-                const uint32_t use = kvc / BS;
-                if (use > 0 && !wait(p, L::bKVEmpty + st, (use - 1) & 1)) return false;
-                const int32_t krow = g.kb0 + (g.b_first + bl) * BB;
-                tc::mbar_arrive_expect_tx(bar(p, L::bKVFull + st), 2 * L::kBlk);
-                tma_rows<D, BB>(pb + L::pK + st * L::kBlk, &tk, krow, bh, bar(p, L::bKVFull + st));
-                tma_rows<D, BB>(pb + L::pV + st * L::kBlk, &tv, krow, bh, bar(p, L::bKVFull + st));
-                ++kvc;
-                return true;
-            };
-            const int n_pre = g.n_band < BS ? g.n_band : BS;
-            int okl = 1;
-            if (lane == 0) {
-                if (lt >= 1 && !wait(p, L::bQEmpty, (uint32_t)((lt - 1) & 1))) okl = 0;
-                if (okl) {
-                    tc::mbar_arrive_expect_tx(bar(p, L::bQFull), 2 * L::kRow);
-                    tma_rows<D, BM>(pb + L::pQ, &tq, q0, bh, bar(p, L::bQFull));
-                    tma_rows<D, BM>(pb + L::pDO, &tdo, q0, bh, bar(p, L::bQFull));
-                }
-                for (int bl = 0; okl && bl < n_pre; ++bl)
-                    if (!load_kv(bl)) okl = 0;
-            }
-            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
-            for (int d = 0; ok && d < nd; ++d) {
-                const int st = (int)(dc % DSX);
-                const uint32_t use = dc / DSX;
-                const uint32_t kdst = pb + L::pDK + st * L::kRow;
-                const uint32_t vdst = pb + L::pDV + st * L::kRow;
-                if (use > 0 && !wait(p, L::bDiagEmpty + st, (use - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) tc::mbar_arrive_expect_tx(bar(p, L::bDiagFull + st), 2 * L::kRow);
-                if (a.kind == 0) {
-                    if (lane == 0) {
                         const int32_t krow = (int32_t)(q0 - a.offs[a.n_off - nd + d]);
-                        tma_rows<D, BM>(kdst, &tkd, krow, bh, bar(p, L::bDiagFull + st));
-                        tma_rows<D, BM>(vdst, &tvd, krow, bh, bar(p, L::bDiagFull + st));
-                    }
-                } else {
-                    int32_t rr[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int64_t i = q0 + 4 * lane + h;
-                        const int64_t j = d < cres[h] ? (int64_t)cj[h] : (i < T ? i : 0);
-                        rr[h] = (int32_t)((int64_t)bh * T + j);
-                    }
-#pragma unroll
-                    for (int x = 0; x < D / 64; ++x) {
-                        const uint32_t off = x * (BM * 128) + 4 * lane * 128;
-                        tc::tma_gather4(kdst + off, &tkr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                        tc::mbar_arrive_expect_tx(bar(p, L::bDiagFull + st), 2 * L::kRow);
+                        tma_rows<D, BM>(pb + L::pDK + st * L::kRow, &tkd, krow, kvbh,
                                         bar(p, L::bDiagFull + st));
-                        tc::tma_gather4(vdst + off, &tvr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                        tma_rows<D, BM>(pb + L::pDV + st * L::kRow, &tvd, krow, kvbh,
                                         bar(p, L::bDiagFull + st));
+                        ++dc;
                     }
-#pragma unroll
-                    for (int h = 0; h < 4; ++h)
-                        if (d + 1 < cres[h]) cj[h] = a.colidx[cstart[h] + d + 1];
                 }
-                ++dc;
+                for (; ok && bl < g.n_band; ++bl) ok = load_kv(bl);
             }
-            if (!ok) break;
-            if (lane == 0)
-                for (int bl = n_pre; okl && bl < g.n_band; ++bl)
-                    if (!load_kv(bl)) okl = 0;
-            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
         }
       } else if ((warp >> 1) < NP) {
         // ---------------- MMA issuer of pipeline p: S and dP of block g, then
@@ -558,7 +508,7 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             int64_t lt = 0;
             for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
                 const TileId id = tile_id(t, ntr);
-                const DQBand<BB> g(id.r0, T, W);
+                const DQBand<BB> g(id.r0, T, a.We);
                 if (!wait(p, L::bQFull, (uint32_t)(lt & 1))) break;
                 const uint32_t qa = pb + L::pQ, da = pb + L::pDO;
                 for (int bl = 0; bl < g.n_band; ++bl) {
@@ -616,34 +566,31 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         const int p = (warp - 4) >> 2;
         const int r = tid - 128 - 128 * p;
         uint8_t *pm = sm + p * L::kPipe;
-        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
         const uint32_t lane_off = (uint32_t)(((warp - 4) & 3) * 32) << 16;
         const uint32_t tS = tmem + p * L::tPipe + lane_off + L::tS;
         const uint32_t tDP = tmem + p * L::tPipe + lane_off + L::tDP;
         const uint32_t tDQ = tmem + p * L::tPipe + lane_off + L::tDQ;
         const float c2 = a.scale2;
-        uint32_t dc = 0, gb = 0, group_uses = 0;
+        const int wq = r >> 5;  // warp within the group: rows 32 wq .. 32 wq + 31
+        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
+        uint32_t gb = 0, dc = 0;
         bool ok = true;
         int64_t lt = 0;
         for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
             const TileId id = tile_id(t, ntr);
             const int32_t q0 = id.r0, bh = id.bh;
-            const DQBand<BB> g(q0, T, W);
+            const int64_t kvbh = (bh / a.H) * a.Hkv + (bh % a.H) / (a.H / a.Hkv);
+            const DQBand<BB> g(q0, T, a.We);
             const int64_t i = q0 + r;
             const bool row_ok = i < T;
             const size_t grow = (size_t)bh * (size_t)T + (size_t)i;
-            const int slot = (int)(lt & 1);
-            if (!wait(p, L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1))) break;
-            const int nd = info[slot];
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
             const float lse2 = row_ok ? a.lse[grow] * kLog2e : 0.f;
             // the out row for Delta is fetched while Q and dO arrive
             uint4 orow4[D / 8];
 #pragma unroll
             for (int c = 0; c < D / 8; ++c)
                 orow4[c] = row_ok ? __ldg((const uint4 *)(a.o + grow * D) + c) : make_uint4(0, 0, 0, 0);
-            if (!wait(p, L::bQFull, (uint32_t)(lt & 1))) break;
+            if (!__all_sync(0xffffffffu, wait(p, L::bQFull, (uint32_t)(lt & 1)))) break;
             // Delta_i = dO_i . out_i
             float Delta = 0.f;
             {
@@ -664,78 +611,82 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                 Delta = sum8(sp);
             }
             if (row_ok) a.delta[grow] = Delta;
-            // diagonal blocks
-            float acc[D];
+            // diagonal slots: the K and V rows of this row's distance links (or
+            // CSR residual entries), fetched by this warp itself; their sum is
+            // kept in registers (D = 64) or in the TMEM accumulator (D = 128)
+            constexpr bool kRegAcc = D == 64;
+            float acc[kRegAcc ? D : 1];
 #pragma unroll
-            for (int x = 0; x < D; ++x) acc[x] = 0.f;
-            if (DS > 0 && nd > 0) {
-                if (a.kind == 0) {
-                    // distance links: swizzled tiles, q in logical chunk order
-                    uint32_t qw[D / 2];
-                    load_row_packed<D>(pm + L::pQ, BM, r, qw);
-                    for (int d = 0; d < nd; ++d) {
-                        const int st = (int)(dc % DSX);
-                        if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
-                            ok = false;
-                            break;
-                        }
-                        if (row_ok && i >= a.offs[a.n_off - nd + d]) {
-                            const uint8_t *kt = pm + L::pDK + st * L::kRow;
-                            const uint8_t *vt = pm + L::pDV + st * L::kRow;
-                            const float pr =
-                                tc::ex2(fmaf(dot_bf_reg_smem<D>(qw, kt, BM, r), c2, -lse2));
-                            const float ds =
-                                pr * (dot_bf_smem_smem<D>(pm + L::pDO, vt, BM, r) - Delta);
-                            if (a.pds)
-                                a.pds[((size_t)(a.n_off - nd + d) * (size_t)a.BH + (size_t)bh) *
-                                          (size_t)T +
-                                      (size_t)i] = make_float2(pr, ds);
-                            axpy_bf_smem<D>(acc, ds, kt, BM, r);
-                        }
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
-                        ++dc;
-                    }
+            for (int x = 0; x < (kRegAcc ? D : 1); ++x) acc[x] = 0.f;
+            if constexpr (!kRegAcc) {
+                tmem_store_row<D>(tDQ, nullptr);
+                tc::tmem_st_wait();
+            }
+            if constexpr (DS > 0) {
+                // slots: the tile's distance blocks (count from the producer),
+                // or, for CSR lists, the longest residual list of this warp's rows
+                int nd = 0;
+                int64_t cst = 0;
+                int32_t resid = 0;
+                if constexpr (!LDW) {
+                    const int slot = (int)(lt & 1);
+                    ok = __all_sync(0xffffffffu,
+                                    wait(p, L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1)));
+                    nd = ok ? info[slot] : 0;
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
                 } else {
-                    // CSR gathers are unswizzled: pair them with the physical
-                    // chunk order of the swizzled q and dO rows (as in the forward)
-                    int64_t resid = 0;
-                    if (row_ok)
-                        resid = (a.rowptr[i + 1] - a.rowptr[i]) - ((i + 1 < W) ? i + 1 : W);
-                    for (int d = 0; d < nd; ++d) {
-                        const int st = (int)(dc % DSX);
-                        if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
+                    if (row_ok) {
+                        cst = a.rowptr[i];
+                        resid = (int32_t)(a.rowptr[i + 1] - cst - ((i + 1 < W) ? i + 1 : W));
+                    }
+                    nd = (int)__reduce_max_sync(0xffffffffu, (unsigned)resid);
+                }
+                const int dfirst = a.n_off - nd;  // distance index of slot 0 (keys ascending)
+                auto key_of = [&](int d) -> int32_t {  // (CSR slots)
+                    return d < resid ? __ldg(a.colidx + cst + d) : -1;
+                };
+                // the q row in registers (D = 64) or read from the Q tile (D = 128,
+                // whose accumulator already takes 128 registers)
+                uint32_t qw[D == 64 ? D / 2 : 1];
+                if constexpr (D == 64) load_row_packed<D>(pm + L::pQ, BM, r, qw);
+                auto body = [&](int d, int st) {
+                    const bool valid = LDW ? (d < resid) : (row_ok && i >= a.offs[dfirst + d]);
+                    if (!valid) return;
+                    const uint8_t *kt = pm + L::pDK + st * L::kRow;
+                    const uint8_t *vt = pm + L::pDV + st * L::kRow;
+                    float qk;
+                    if constexpr (D == 64)
+                        qk = dot_bf_reg_smem<D>(qw, kt, BM, r);
+                    else
+                        qk = dot_bf_smem_smem<D>(pm + L::pQ, kt, BM, r);
+                    const float pr = tc::ex2(fmaf(qk, c2, -lse2));
+                    const float ds = pr * (dot_bf_smem_smem<D>(pm + L::pDO, vt, BM, r) - Delta);
+                    if (a.pds)
+                        a.pds[((size_t)(dfirst + d) * (size_t)a.BH + (size_t)bh) * (size_t)T +
+                              (size_t)i] = make_float2(pr, ds);
+                    if constexpr (kRegAcc)
+                        axpy_bf_smem<D>(acc, ds, kt, BM, r);
+                    else
+                        tmem_axpy_row<D>(tDQ, ds, kt, BM, r);
+                };
+                if constexpr (LDW) {
+                    rows::warp_slots<D, DS>(
+                        nd, sbase + (uint32_t)(p * L::kPipe + L::pDK),
+                        sbase + (uint32_t)(p * L::kPipe + L::pDV), (uint32_t)L::kRow, a.k, a.v,
+                        a.l2pf != 0, lane, wq,
+                        [&](int) { return (size_t)kvbh * (size_t)T * D; }, key_of, body);
+                } else {
+                    for (int d = 0; ok && d < nd; ++d) {
+                        const int st = (int)(dc % DS);
+                        if (!__all_sync(0xffffffffu, wait(p, L::bDiagFull + st, (dc / DS) & 1))) {
                             ok = false;
                             break;
                         }
-                        if (row_ok && d < resid) {
-                            const uint8_t *kt = pm + L::pDK + st * L::kRow;
-                            const uint8_t *vt = pm + L::pDV + st * L::kRow;
-                            const float pr = tc::ex2(
-                                fmaf(dot_bf_phys_gathered<D>(pm + L::pQ, kt, BM, r), c2, -lse2));
-                            const float ds =
-                                pr * (dot_bf_phys_gathered<D>(pm + L::pDO, vt, BM, r) - Delta);
-                            axpy_bf_smem<D>(acc, ds, kt, BM, r);
-                        }
-                        if (d < nd - 1) {  // the last stage is released after the unpermute
-                            __syncwarp();
-                            if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
-                        }
-                        ++dc;
-                    }
-                    if (ok) {
-                        // once every row is done with the last stage, thread r
-                        // uses D floats of it (rows < 64 in its K half, the
-                        // others in its V half) to restore the logical order
-                        const int st = (int)((dc - 1) % DSX);
-                        tc::mbar_arrive(bar(p, L::bGroup));
-                        if (!wait(p, L::bGroup, group_uses & 1)) ok = false;
-                        ++group_uses;
-                        float *scr = (float *)(pm + (r < 64 ? L::pDK : L::pDV) + st * L::kRow) +
-                                     (size_t)(r & 63) * D;
-                        unpermute_row<D>(acc, scr, r);
+                        body(d, st);
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
+                        ++dc;
                     }
                 }
             }
@@ -743,7 +694,7 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             // this warp is done reading Q and dO of the tile
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(p, L::bQEmpty));
-            tmem_store_row<D>(tDQ, acc);
+            if constexpr (kRegAcc) tmem_store_row<D>(tDQ, acc);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
@@ -769,22 +720,36 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(bar(p, L::bSFree + sb));
                 }
-                const bool need_mask =
-                    (u0 < BM - 1) || (u0 + BB - 1 > W - 1) || (u0 + q0 < W - 1);
+                const int32_t We = a.We;
+                const bool need_mask = a.nf > 0 || (u0 < BM - 1) || (u0 + BB - 1 > We - 1) ||
+                                       (u0 + q0 < We - 1);
                 if (need_mask) {
-                    // keep columns [c_lo, c_hi]: r <= u <= r+W-1 and key >= 0
-                    const int32_t lo = (r > W - 1 - q0) ? r : W - 1 - q0;
-                    const int32_t hi = r + W - 1;
+                    // keep columns [c_lo, c_hi]: r + We - W <= u <= r + We - 1
+                    // and key >= 0, plus the folded links u = r + We - 1 - o
+                    const int32_t kmin = We - 1 - q0;  // u of key 0
+                    const int32_t lo = (r + We - W > kmin) ? r + We - W : kmin;
+                    const int32_t hi = r + We - 1;
                     const int c_lo = lo - u0 < 0 ? 0 : (lo - u0 > BB ? BB : lo - u0);
                     const int c_hi = hi - u0 > BB - 1 ? BB - 1 : (hi - u0 < -1 ? -1 : hi - u0);
+                    int fc[kMaxFold];
+#pragma unroll
+                    for (int x = 0; x < kMaxFold; ++x) {
+                        const int32_t u = r + We - 1 - a.fold[x];
+                        fc[x] = (x < a.nf && u >= kmin && u >= u0 && u < u0 + BB) ? u - u0 : -1;
+                    }
                     // 16-column chunks outside every kept range of this warp: dS = 0
 #pragma unroll
                     for (int c16 = 0; c16 < BB / 16; ++c16) {
-                        if (__any_sync(0xffffffffu, c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16)) {
+                        bool live = c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16;
+#pragma unroll
+                        for (int x = 0; x < kMaxFold; ++x) live |= (fc[x] >> 4) == c16;
+                        if (__any_sync(0xffffffffu, live)) {
 #pragma unroll
                             for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
-                                const float pr =
-                                    (c >= c_lo && c <= c_hi) ? tc::ex2(fmaf(s[c], c2, -lse2)) : 0.f;
+                                bool keep = c >= c_lo && c <= c_hi;
+#pragma unroll
+                                for (int x = 0; x < kMaxFold; ++x) keep |= (c == fc[x]);
+                                const float pr = keep ? tc::ex2(fmaf(s[c], c2, -lse2)) : 0.f;
                                 s[c] = pr * (dp[c] - Delta);
                             }
                         } else {
@@ -845,20 +810,21 @@ struct LayoutDKV {
     static constexpr int kStage = 2 * BB * 4;
     static constexpr int kLse = NP * kPipe;
     static constexpr int kBars = kLse + NP * BS * kStage;
-    static constexpr int DSX = DS > 0 ? DS : 1;
     // barriers of one pipeline (S^T and dP^T share a buffer index sb; P^T and
-    // dS^T are written over them, so a buffer is free once its dV/dK MMAs are done)
+    // dS^T are written over them, so a buffer is free once its dV/dK MMAs are
+    // done)
     static constexpr int bKVFull = 0, bKVEmpty = 1;
     static constexpr int bBFull = 2, bBEmpty = bBFull + BS;
     static constexpr int bSFull = bBEmpty + BS, bSFree = bSFull + SB;
     static constexpr int bPFull = bSFree + SB, bDKVDone = bPFull + SB;
     static constexpr int bInit = bDKVDone + SB;
-    static constexpr int bDiagFull = bInit + 1, bDiagEmpty = bDiagFull + DSX;
+    static constexpr int bPSDone = bInit + 1;              // P^T/dS^T tiles consumed
+    // distance blocks loaded by the producer with TMA (structured graphs)
+    static constexpr int DSX = DS > 0 ? DS : 1;
+    static constexpr int bDiagFull = bPSDone + (PS > 0 ? PS : 1), bDiagEmpty = bDiagFull + DSX;
     static constexpr int bInfoFull = bDiagEmpty + DSX, bInfoEmpty = bInfoFull + 2;
-    static constexpr int bGroup = bInfoEmpty + 2;
-    static constexpr int bPSDone = bGroup + 1;              // P^T/dS^T tiles consumed
-    static constexpr int nBarsPipe = bPSDone + (PS > 0 ? PS : 1);
-    static constexpr int kMisc = kBars + NP * nBarsPipe * 8;
+    static constexpr int nBarsPipe = bInfoEmpty + 2;
+    static constexpr int kMisc = kBars + NP * nBarsPipe * 8;  // tmem slot, abort, info[NP][2]
     static constexpr int kTotal = kMisc + 8 + 8 * NP;
     static constexpr int kAlloc = kTotal + 1024;
     static_assert(PS == 0 || BB == 64, "shared-memory P tiles are 64 queries wide");
@@ -877,17 +843,16 @@ __device__ __forceinline__ int dkv_n_band(int32_t k0, int64_t T, int32_t W) {
     return (int)(vmax / BB + 1);
 }
 
-template <int D, int NP, int BB, int SB, int BS, int DS, int PS>
+// LDW: the diagonal slots are copied by each compute warp (CSR lists); else
+// the producer loads each distance block as TMA boxes (structured graphs).
+template <int D, int NP, int BB, int SB, int BS, int DS, int PS, bool LDW>
 __global__ void __launch_bounds__(128 + 128 * NP, 1)
 band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                      const __grid_constant__ CUtensorMap tvt,
                      const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
                      const __grid_constant__ CUtensorMap tqd,
-                     const __grid_constant__ CUtensorMap tdod,
-                     const __grid_constant__ CUtensorMap tqr,
-                     const __grid_constant__ CUtensorMap tdor, const BwdArgs a) {
+                     const __grid_constant__ CUtensorMap tdod, const BwdArgs a) {
     using L = LayoutDKV<D, NP, BB, SB, BS, DS, PS>;
-    constexpr int DSX = L::DSX;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_u32(sm);
@@ -906,8 +871,15 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t T = a.T;
     const int32_t W = a.W;
-    const int64_t ntr = (T + BM - 1) / BM, ntiles = ntr * a.BH;
+    // tiles run over key/value slices; each takes the blocks of every query
+    // head of its group (grouped-query attention: GQ = H / Hkv heads)
+    const int64_t BHkv = a.BH / (a.H / a.Hkv);
+    const int GQ = (int)(a.H / a.Hkv);
+    const int64_t ntr = (T + BM - 1) / BM, ntiles = ntr * BHkv;
     const int64_t stride = (int64_t)gridDim.x * NP;
+    auto qslice0 = [&](int32_t kvbh) -> int64_t {  // first query slice of the group
+        return ((int64_t)kvbh / a.Hkv) * a.H + ((int64_t)kvbh % a.Hkv) * GQ;
+    };
 
     if (tid == 0) {
         for (int p = 0; p < NP; ++p) {
@@ -926,7 +898,8 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                 tc::mbar_init(bar(p, L::bDKVDone + s), 1);
             }
             tc::mbar_init(bar(p, L::bInit), 4);
-            for (int s = 0; s < DSX; ++s) {
+            for (int s = 0; s < PS; ++s) tc::mbar_init(bar(p, L::bPSDone + s), 1);
+            for (int s = 0; s < L::DSX; ++s) {
                 tc::mbar_init(bar(p, L::bDiagFull + s), 1);
                 tc::mbar_init(bar(p, L::bDiagEmpty + s), 4);
             }
@@ -934,8 +907,6 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                 tc::mbar_init(bar(p, L::bInfoFull + s), 1);
                 tc::mbar_init(bar(p, L::bInfoEmpty + s), 4);
             }
-            tc::mbar_init(bar(p, L::bGroup), 128);
-            for (int s = 0; s < PS; ++s) tc::mbar_init(bar(p, L::bPSDone + s), 1);
         }
         *abort = 0;
         tc::fence_barrier_init();
@@ -949,51 +920,34 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
     if (warp < 4) {
         if (NP == 2) tc::regs_dec<BwdRegs::producer>();
       if ((warp >> 1) < NP && (warp & 1) == 0) {
-        // ---------------- producer of pipeline p: diagonal-block count, K and V
-        // of the tile, the first band Q/dO blocks (with lse and Delta), the
-        // diagonal blocks, the rest
+        // ---------------- producer of pipeline p: K and V of the tile, then
+        // the band Q/dO blocks of every query head of the group (with lse and
+        // Delta) through their ring and, for a structured graph, the distance
+        // blocks of every head (the count first, to the compute warps) after
+        // the band blocks that fit the ring
         const int p = warp >> 1;
         const uint32_t pb = sbase + (uint32_t)(p * L::kPipe);
         volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
+        constexpr bool kTmaDiag = DS > 0 && !LDW;
         uint32_t bc = 0, dc = 0;
         bool ok = true;
         int64_t lt = 0;
         for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
             const TileId id = tile_id(t, ntr);
-            const int32_t k0 = id.r0, bh = id.bh;
-            const int n_band = dkv_n_band<BB>(k0, T, W);
-            // CSR: lane l owns key rows 4l .. 4l+3: start of the residual part of
-            // their transpose lists (after the band queries j .. j+W-1), its
-            // length, and the next query
-            int64_t cstart[4] = {0, 0, 0, 0}, cres[4] = {0, 0, 0, 0};
-            int32_t cj[4] = {0, 0, 0, 0};
-            int nd = 0;
-            if (DS > 0) {
-                if (a.kind == 0) {
-                    for (int x = 0; x < a.n_off; ++x) nd += (k0 + a.offs[x] <= T - 1) ? 1 : 0;
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int64_t j = k0 + 4 * lane + h;
-                        if (j < T) {
-                            const int64_t nb = (T - j < W) ? T - j : W;
-                            cstart[h] = a.rev_rowptr[j] + nb;
-                            cres[h] = a.rev_rowptr[j + 1] - cstart[h];
-                            if (cres[h] > 0) cj[h] = a.rev_colidx[cstart[h]];
-                            nd = nd > (int)cres[h] ? nd : (int)cres[h];
-                        }
-                    }
-                    for (int o = 16; o > 0; o >>= 1) {
-                        const int x = __shfl_xor_sync(0xffffffffu, nd, o);
-                        nd = nd > x ? nd : x;
-                    }
+            const int32_t k0 = id.r0, kvbh = id.bh;
+            const int64_t qbh0 = qslice0(kvbh);
+            const int n_band = dkv_n_band<BB>(k0, T, a.We);
+            const int NB = GQ * n_band;  // band blocks of all heads of the group
+            int nd = 0;  // distance blocks of one head
+            if constexpr (kTmaDiag) {
+                for (int x = 0; x < a.n_off; ++x) nd += (k0 + a.offs[x] <= T - 1) ? 1 : 0;
+                const int slot = (int)(lt & 1);
+                if (lt >= 2 && !wait(p, L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1)))
+                    break;
+                if (lane == 0) {
+                    info[slot] = nd;
+                    tc::mbar_arrive(bar(p, L::bInfoFull + slot));
                 }
-            }
-            const int slot = (int)(lt & 1);
-            if (lt >= 2 && !wait(p, L::bInfoEmpty + slot, (uint32_t)(((lt >> 1) - 1) & 1))) break;
-            if (lane == 0) {
-                info[slot] = nd;
-                tc::mbar_arrive(bar(p, L::bInfoFull + slot));
             }
             // band block bl (all lanes): lane 0 the TMA copies, every lane a
             // share of lse (base 2) and Delta, zero past the end of the
@@ -1002,11 +956,12 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             constexpr int PL = BB / 32;  // values per lane
             float pf_l[PL], pf_d[PL];
             auto fetch_vals = [&](int bl) {
+                const int hq = bl / n_band, b = bl - hq * n_band;
 #pragma unroll
                 for (int x = 0; x < PL; ++x) {
-                    const int64_t i = (int64_t)k0 + bl * BB + lane + 32 * x;
-                    const size_t gi = (size_t)bh * (size_t)T + (size_t)i;
-                    const bool in = bl < n_band && i < T;
+                    const int64_t i = (int64_t)k0 + b * BB + lane + 32 * x;
+                    const size_t gi = (size_t)(qbh0 + hq) * (size_t)T + (size_t)i;
+                    const bool in = bl < NB && i < T;
                     pf_l[x] = in ? a.lse[gi] : 0.f;
                     pf_d[x] = in ? a.delta[gi] : 0.f;
                 }
@@ -1016,11 +971,13 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                 const int st = (int)(bc % BS);
                 const uint32_t use = bc / BS;
                 if (use > 0 && !wait(p, L::bBEmpty + st, (use - 1) & 1)) return false;
-                const int32_t qrow = k0 + bl * BB;
+                const int hq = bl / n_band;
+                const int32_t qrow = k0 + (bl - hq * n_band) * BB;
+                const int32_t qz = (int32_t)(qbh0 + hq);
                 if (lane == 0) {
                     tc::mbar_arrive_expect_tx(bar(p, L::bBFull + st), 2 * L::kBlk);
-                    tma_rows<D, BB>(pb + L::pQ + st * L::kBlk, &tq, qrow, bh, bar(p, L::bBFull + st));
-                    tma_rows<D, BB>(pb + L::pDO + st * L::kBlk, &tdo, qrow, bh,
+                    tma_rows<D, BB>(pb + L::pQ + st * L::kBlk, &tq, qrow, qz, bar(p, L::bBFull + st));
+                    tma_rows<D, BB>(pb + L::pDO + st * L::kBlk, &tdo, qrow, qz,
                                     bar(p, L::bBFull + st));
                 }
                 float *ls = stage_lse(p, st), *dl = ls + BB;
@@ -1034,57 +991,41 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                 fetch_vals(bl + 1);
                 return true;
             };
-            const int n_pre = n_band < BS ? n_band : BS;
+            const int n_pre = NB < BS ? NB : BS;
             int okl = 1;
             if (lane == 0) {
                 if (lt >= 1 && !wait(p, L::bKVEmpty, (uint32_t)((lt - 1) & 1))) okl = 0;
                 if (okl) {
                     tc::mbar_arrive_expect_tx(bar(p, L::bKVFull), 2 * L::kRow);
-                    tma_rows<D, BM>(pb + L::pK, &tkt, k0, bh, bar(p, L::bKVFull));
-                    tma_rows<D, BM>(pb + L::pV, &tvt, k0, bh, bar(p, L::bKVFull));
+                    tma_rows<D, BM>(pb + L::pK, &tkt, k0, kvbh, bar(p, L::bKVFull));
+                    tma_rows<D, BM>(pb + L::pV, &tvt, k0, kvbh, bar(p, L::bKVFull));
                 }
             }
             ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
             for (int bl = 0; ok && bl < n_pre; ++bl) ok = load_blk(bl);
-            for (int d = 0; ok && d < nd; ++d) {
-                const int st = (int)(dc % DSX);
-                const uint32_t use = dc / DSX;
-                const uint32_t qdst = pb + L::pDQ + st * L::kRow;
-                const uint32_t ddst = pb + L::pDDO + st * L::kRow;
-                if (use > 0 && !wait(p, L::bDiagEmpty + st, (use - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) tc::mbar_arrive_expect_tx(bar(p, L::bDiagFull + st), 2 * L::kRow);
-                if (a.kind == 0) {
+            if constexpr (kTmaDiag) {
+                // distance o of head hq: queries k0+o .. k0+127+o of its slice
+                for (int d = 0; ok && d < GQ * nd; ++d) {
+                    const int hq = d / nd, dd = d - hq * nd;
+                    const int st = (int)(dc % DS);
+                    const uint32_t use = dc / DS;
+                    if (use > 0 && !wait(p, L::bDiagEmpty + st, (use - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
                     if (lane == 0) {
-                        const int32_t qrow = (int32_t)(k0 + a.offs[a.n_off - nd + d]);
-                        tma_rows<D, BM>(qdst, &tqd, qrow, bh, bar(p, L::bDiagFull + st));
-                        tma_rows<D, BM>(ddst, &tdod, qrow, bh, bar(p, L::bDiagFull + st));
-                    }
-                } else {
-                    int32_t rr[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int64_t j = k0 + 4 * lane + h;
-                        const int64_t i = d < cres[h] ? (int64_t)cj[h] : (j < T ? j : 0);
-                        rr[h] = (int32_t)((int64_t)bh * T + i);
-                    }
-#pragma unroll
-                    for (int x = 0; x < D / 64; ++x) {
-                        const uint32_t off = x * (BM * 128) + 4 * lane * 128;
-                        tc::tma_gather4(qdst + off, &tqr, x * 64, rr[0], rr[1], rr[2], rr[3],
+                        const int32_t qrow = (int32_t)(k0 + a.offs[a.n_off - nd + dd]);
+                        const int32_t qz = (int32_t)(qbh0 + hq);
+                        tc::mbar_arrive_expect_tx(bar(p, L::bDiagFull + st), 2 * L::kRow);
+                        tma_rows<D, BM>(pb + L::pDQ + st * L::kRow, &tqd, qrow, qz,
                                         bar(p, L::bDiagFull + st));
-                        tc::tma_gather4(ddst + off, &tdor, x * 64, rr[0], rr[1], rr[2], rr[3],
+                        tma_rows<D, BM>(pb + L::pDDO + st * L::kRow, &tdod, qrow, qz,
                                         bar(p, L::bDiagFull + st));
                     }
-#pragma unroll
-                    for (int h = 0; h < 4; ++h)
-                        if (d + 1 < cres[h]) cj[h] = a.rev_colidx[cstart[h] + d + 1];
+                    ++dc;
                 }
-                ++dc;
             }
-            for (int bl = n_pre; ok && bl < n_band; ++bl) ok = load_blk(bl);
+            for (int bl = n_pre; ok && bl < NB; ++bl) ok = load_blk(bl);
         }
       } else if ((warp >> 1) < NP) {
         // ---------------- MMA issuer of pipeline p: S^T and dP^T of block g,
@@ -1139,10 +1080,10 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             int64_t lt = 0;
             for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
                 const TileId id = tile_id(t, ntr);
-                const int n_band = dkv_n_band<BB>(id.r0, T, W);
+                const int NB = GQ * dkv_n_band<BB>(id.r0, T, a.We);
                 if (!wait(p, L::bKVFull, (uint32_t)(lt & 1))) break;
                 const uint32_t ka = pb + L::pK, va = pb + L::pV;
-                for (int bl = 0; bl < n_band; ++bl) {
+                for (int bl = 0; bl < NB; ++bl) {
                     const int st = (int)(gb % BS), sb = (int)(gb % SB);
                     // one S^T buffer: dV/dK of the previous block free it first
                     if (SB == 1 && have) {
@@ -1170,7 +1111,7 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                                         tc::sdesc_sw128(da + offb, 16, 1024), idS, kk > 0);
                     }
                     tc::mma_commit(bar(p, L::bSFull + sb));
-                    if (bl == n_band - 1) tc::mma_commit(bar(p, L::bKVEmpty));
+                    if (bl == NB - 1) tc::mma_commit(bar(p, L::bKVEmpty));
                     if (SB > 1 && have && !do_dkv()) {
                         ok = false;
                         break;
@@ -1196,71 +1137,91 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
         const int p = (warp - 4) >> 2;
         const int r = tid - 128 - 128 * p;
         uint8_t *pm = sm + p * L::kPipe;
-        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
         const uint32_t lane_off = (uint32_t)(((warp - 4) & 3) * 32) << 16;
         const uint32_t tbase = tmem + p * L::tPipe + lane_off;
         const uint32_t tS = tbase + L::tS, tDP = tbase + L::tDP;
         const uint32_t tDV = tbase + L::tDV, tDK = tbase + L::tDK;
         const float c2 = a.scale2;
-        uint32_t dc = 0, gb = 0, group_uses = 0;
+        const int wq = r >> 5;  // warp within the group: key rows 32 wq .. 32 wq + 31
+        volatile int *info = (volatile int *)(sm + L::kMisc + 8) + 2 * p;
+        uint32_t gb = 0, dc = 0;
         bool ok = true;
         int64_t lt = 0;
         for (int64_t t = (int64_t)blockIdx.x * NP + p; ok && t < ntiles; t += stride, ++lt) {
             const TileId id = tile_id(t, ntr);
-            const int32_t k0 = id.r0, bh = id.bh;
-            const int n_band = dkv_n_band<BB>(k0, T, W);
+            const int32_t k0 = id.r0, kvbh = id.bh;
+            const int64_t qbh0 = qslice0(kvbh);
+            const int n_band = dkv_n_band<BB>(k0, T, a.We);
+            const int NB = GQ * n_band;
             const int64_t j = k0 + r;
             const bool row_ok = j < T;
-            const size_t gbh = (size_t)bh * (size_t)T;
-            const size_t grow = gbh + (size_t)j;
-            const int slot = (int)(lt & 1);
-            if (!wait(p, L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1))) break;
-            const int nd = info[slot];
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
-            if (!wait(p, L::bKVFull, (uint32_t)(lt & 1))) break;
-            // diagonal blocks: (p, dS) of each distance edge from the dQ
-            // kernel's cache, or recomputed from lse and Delta of the linked
-            // query; either pair is loaded one block ahead
-            float adk[D], adv[D];
+            const size_t grow = (size_t)kvbh * (size_t)T + (size_t)j;
+            if (!__all_sync(0xffffffffu, wait(p, L::bKVFull, (uint32_t)(lt & 1)))) break;
+            // diagonal slots: the Q and dO rows of the queries that reach this
+            // key by a distance link (or by a CSR residual entry), for every
+            // query head of the group, fetched by this warp itself; (p, dS) of
+            // each edge comes from the dQ kernel's cache, or is recomputed from
+            // lse and Delta of the query, loaded one slot ahead
+            // D = 64: diagonal sums in registers, stored to TMEM after the
+            // slots; D = 128: summed in TMEM directly (zeroed first)
+            constexpr bool kRegAcc = D == 64;
+            float adk[kRegAcc ? D : 1], adv[kRegAcc ? D : 1];
 #pragma unroll
-            for (int x = 0; x < D; ++x) adk[x] = adv[x] = 0.f;
-            if (DS > 0 && nd > 0) {
-                const int off_first = a.n_off - nd;
+            for (int x = 0; x < (kRegAcc ? D : 1); ++x) adk[x] = adv[x] = 0.f;
+            if constexpr (!kRegAcc) {
+                tmem_store_row<D>(tDV, nullptr);
+                tmem_store_row<D>(tDK, nullptr);
+                tc::tmem_st_wait();
+            }
+            if constexpr (DS > 0) {
+                // slots per head: the tile's distance blocks (count from the
+                // producer), or, for CSR lists, the longest residual transpose
+                // list of this warp's keys
+                int nd = 0;
                 int64_t rs = 0, nb = 0, resid = 0;
-                if (a.kind == 1 && row_ok) {
-                    rs = a.rev_rowptr[j];
-                    nb = (T - j < W) ? T - j : W;
-                    resid = a.rev_rowptr[j + 1] - rs - nb;
-                }
-                // query of slot d (-1 if none)
-                auto query_of = [&](int d) -> int64_t {
-                    if (!row_ok || d >= nd) return -1;
-                    if (a.kind == 0) {
-                        const int64_t cand = j + a.offs[off_first + d];
-                        return cand < T ? cand : -1;
+                if constexpr (!LDW) {
+                    const int slot = (int)(lt & 1);
+                    ok = __all_sync(0xffffffffu,
+                                    wait(p, L::bInfoFull + slot, (uint32_t)((lt >> 1) & 1)));
+                    nd = ok ? info[slot] : 0;
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(p, L::bInfoEmpty + slot));
+                } else {
+                    if (row_ok) {
+                        rs = a.rev_rowptr[j];
+                        nb = (T - j < W) ? T - j : W;
+                        resid = a.rev_rowptr[j + 1] - rs - nb;
                     }
-                    return d < resid ? (int64_t)a.rev_colidx[rs + nb + d] : -1;
+                    nd = (int)__reduce_max_sync(0xffffffffu, (unsigned)resid);
+                }
+                const int off_first = a.n_off - nd;
+                // slot d: link (or residual position) d % nd of query head
+                // d / nd; its query row, -1 if none
+                const int nds = GQ * nd;
+                auto key_of = [&](int d) -> int32_t {
+                    if (!row_ok || d >= nds) return -1;
+                    const int dd = d % nd;
+                    if constexpr (!LDW) {
+                        const int64_t cand = j + a.offs[off_first + dd];
+                        return cand < T ? (int32_t)cand : -1;
+                    }
+                    return dd < resid ? __ldg(a.rev_colidx + rs + nb + dd) : -1;
                 };
                 const bool cached = a.kind == 0 && a.pds != nullptr;
                 auto edge_vals = [&](int d, int64_t i) -> float2 {
                     if (i < 0) return make_float2(0.f, 0.f);
+                    const size_t qbh = (size_t)(qbh0 + d / nd);
                     if (cached)
-                        return a.pds[((size_t)(off_first + d) * (size_t)a.BH + (size_t)bh) *
+                        return a.pds[((size_t)(off_first + d % nd) * (size_t)a.BH + qbh) *
                                          (size_t)T +
                                      (size_t)i];
-                    return make_float2(a.lse[gbh + i], a.delta[gbh + i]);
+                    return make_float2(a.lse[qbh * (size_t)T + i], a.delta[qbh * (size_t)T + i]);
                 };
-                int64_t i_cur = query_of(0), i_nxt = query_of(1);
+                int64_t i_cur = key_of(0), i_nxt = key_of(1);
                 float2 v_cur = edge_vals(0, i_cur);
-                for (int d = 0; d < nd; ++d) {
-                    const int64_t i_n2 = query_of(d + 2);
+                auto body = [&](int d, int st) {
+                    const int64_t i_n2 = key_of(d + 2);
                     const float2 v_nxt = edge_vals(d + 1, i_nxt);
-                    const int st = (int)(dc % DSX);
-                    if (!wait(p, L::bDiagFull + st, (dc / DSX) & 1)) {
-                        ok = false;
-                        break;
-                    }
                     if (i_cur >= 0) {
                         const uint8_t *qt = pm + L::pDQ + st * L::kRow;
                         const uint8_t *dt = pm + L::pDDO + st * L::kRow;
@@ -1269,63 +1230,65 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                             pr = v_cur.x;
                             ds = v_cur.y;
                         } else {
-                            float sdot, dpdot;
-                            if (a.kind == 0) {
-                                sdot = dot_bf_smem_smem<D>(qt, pm + L::pK, BM, r);
-                                dpdot = dot_bf_smem_smem<D>(dt, pm + L::pV, BM, r);
-                            } else {
-                                // CSR gathers are unswizzled: the key's k and v
-                                // rows read in physical chunk order pair with them
-                                sdot = dot_bf_phys_gathered<D>(pm + L::pK, qt, BM, r);
-                                dpdot = dot_bf_phys_gathered<D>(pm + L::pV, dt, BM, r);
-                            }
+                            const float sdot = dot_bf_smem_smem<D>(qt, pm + L::pK, BM, r);
+                            const float dpdot = dot_bf_smem_smem<D>(dt, pm + L::pV, BM, r);
                             pr = tc::ex2(fmaf(sdot, c2, -v_cur.x * kLog2e));
                             ds = pr * (dpdot - v_cur.y);
                         }
-                        axpy_bf_smem<D>(adv, pr, dt, BM, r);
-                        axpy_bf_smem<D>(adk, ds, qt, BM, r);
+                        if constexpr (kRegAcc) {
+                            axpy_bf_smem<D>(adv, pr, dt, BM, r);
+                            axpy_bf_smem<D>(adk, ds, qt, BM, r);
+                        } else {
+                            tmem_axpy_row<D>(tDV, pr, dt, BM, r);
+                            tmem_axpy_row<D>(tDK, ds, qt, BM, r);
+                        }
                     }
-                    if (a.kind == 0 || d < nd - 1) {  // CSR: last stage released below
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
-                    }
-                    ++dc;
                     i_cur = i_nxt;
                     i_nxt = i_n2;
                     v_cur = v_nxt;
-                }
-                if (ok && a.kind == 1) {
-                    // restore the logical order through the last stage once
-                    // every row is done with it (thread r: D floats, rows < 64
-                    // in its Q half, the others in its dO half)
-                    const int st = (int)((dc - 1) % DSX);
-                    tc::mbar_arrive(bar(p, L::bGroup));
-                    if (!wait(p, L::bGroup, group_uses & 1)) ok = false;
-                    ++group_uses;
-                    float *scr = (float *)(pm + (r < 64 ? L::pDQ : L::pDDO) + st * L::kRow) +
-                                 (size_t)(r & 63) * D;
-                    unpermute_row<D>(adv, scr, r);
-                    unpermute_row<D>(adk, scr, r);
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
+                };
+                if constexpr (LDW) {
+                    rows::warp_slots<D, DS>(
+                        nds, sbase + (uint32_t)(p * L::kPipe + L::pDQ),
+                        sbase + (uint32_t)(p * L::kPipe + L::pDDO), (uint32_t)L::kRow, a.q,
+                        a.dout, a.l2pf != 0, lane, wq,
+                        [&](int d) {
+                            return (size_t)(qbh0 + d / (nd > 0 ? nd : 1)) * (size_t)T * D;
+                        },
+                        key_of, body);
+                } else {
+                    for (int d = 0; ok && d < nds; ++d) {
+                        const int st = (int)(dc % DS);
+                        if (!__all_sync(0xffffffffu, wait(p, L::bDiagFull + st, (dc / DS) & 1))) {
+                            ok = false;
+                            break;
+                        }
+                        body(d, st);
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(bar(p, L::bDiagEmpty + st));
+                        ++dc;
+                    }
                 }
             }
             if (!ok) break;
             // this warp is done reading K and V of the tile
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(p, L::bKVEmpty));
-            tmem_store_row<D>(tDV, adv);
-            tmem_store_row<D>(tDK, adk);
+            if constexpr (kRegAcc) {
+                tmem_store_row<D>(tDV, adv);
+                tmem_store_row<D>(tDK, adk);
+            }
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(p, L::bInit));
 
-            // band blocks: P^T and dS^T (bf16) over S^T and dP^T
+            // band blocks of every head of the group: P^T and dS^T (bf16) over
+            // S^T and dP^T
             uint32_t gb_last = gb;
-            for (int bl = 0; ok && bl < n_band; ++bl, ++gb) {
+            for (int bl = 0; ok && bl < NB; ++bl, ++gb) {
                 const int sb = (int)(gb % SB), st = (int)(gb % BS);
-                const int32_t v0 = bl * BB;
+                const int32_t v0 = (bl % n_band) * BB;
                 gb_last = gb;
                 if (!wait(p, L::bSFull + sb, (gb / SB) & 1) ||
                     !wait(p, L::bBFull + st, (gb / BS) & 1)) {  // lse / Delta staged
@@ -1343,10 +1306,11 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                     if (lane == 0) tc::mbar_arrive(bar(p, L::bSFree + sb));
                 }
                 const float *lse_s = stage_lse(p, st), *del_s = lse_s + BB;
-                const bool need_mask = (v0 < BM - 1) || (v0 + BB - 1 > W - 1) ||
+                const bool need_mask = a.nf > 0 || (v0 < BM - 1) || (v0 + BB - 1 > a.We - 1) ||
                                        ((int64_t)k0 + v0 + BB - 1 > T - 1);
                 if (need_mask) {
-                    // keep columns [c_lo, c_hi]: r <= v <= r+W-1 and query < T
+                    // keep columns [c_lo, c_hi]: r <= v <= r+W-1 and query < T,
+                    // plus the folded links v = r + o
                     const int64_t vlim = T - 1 - k0;
                     int64_t hi = (int64_t)r + W - 1;
                     if (hi > vlim) hi = vlim;
@@ -1354,15 +1318,26 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                     const int c_lo = (int)(lo - v0 < 0 ? 0 : (lo - v0 > BB ? BB : lo - v0));
                     const int c_hi =
                         (int)(hi - v0 > BB - 1 ? BB - 1 : (hi - v0 < -1 ? -1 : hi - v0));
+                    int fc[kMaxFold];
+#pragma unroll
+                    for (int x = 0; x < kMaxFold; ++x) {
+                        const int64_t v = (int64_t)r + a.fold[x];
+                        fc[x] = (x < a.nf && v <= vlim && v >= v0 && v < v0 + BB) ? (int)(v - v0)
+                                                                                     : -1;
+                    }
                     // 16-column chunks outside every kept range of this warp: P = dS = 0
 #pragma unroll
                     for (int c16 = 0; c16 < BB / 16; ++c16) {
-                        if (__any_sync(0xffffffffu, c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16)) {
+                        bool live = c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16;
+#pragma unroll
+                        for (int x = 0; x < kMaxFold; ++x) live |= (fc[x] >> 4) == c16;
+                        if (__any_sync(0xffffffffu, live)) {
 #pragma unroll
                             for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
-                                const float pr = (c >= c_lo && c <= c_hi)
-                                                     ? tc::ex2(fmaf(s[c], c2, -lse_s[c]))
-                                                     : 0.f;
+                                bool keep = c >= c_lo && c <= c_hi;
+#pragma unroll
+                                for (int x = 0; x < kMaxFold; ++x) keep |= (c == fc[x]);
+                                const float pr = keep ? tc::ex2(fmaf(s[c], c2, -lse_s[c])) : 0.f;
                                 s[c] = pr;
                                 dp[c] = pr * (dp[c] - del_s[c]);
                             }
@@ -1425,7 +1400,7 @@ inline bool regs_cover(const void *kern) {
     return fa.numRegs * (128 + 128 * NP) >= 128 * BwdRegs::producer + 128 * NP * BwdRegs::compute;
 }
 
-template <int D, int NP, int BB, int SB, int BSQ, int BSK, int DS, int PS>
+template <int D, int NP, int BB, int SB, int BSQ, int BSK, int DS, int PS, bool LDW>
 sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_tensor *o, const float *lse, const sa_tensor *dout,
                           const sa_graph_s *g, float scale, sa_tensor *dq, sa_tensor *dk,
@@ -1434,8 +1409,8 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     using LK = LayoutDKV<D, NP, BB, SB, BSK, DS, PS>;
     static_assert(LQ::kAlloc <= 232448 && LK::kAlloc <= 232448, "shared memory budget");
     constexpr int kThreads = 128 + 128 * NP;
-    auto kq = band_bwd_dq_kernel<D, NP, BB, SB, BSQ, DS, PS>;
-    auto kkv = band_bwd_dkdv_kernel<D, NP, BB, SB, BSK, DS, PS>;
+    auto kq = band_bwd_dq_kernel<D, NP, BB, SB, BSQ, DS, PS, LDW>;
+    auto kkv = band_bwd_dkdv_kernel<D, NP, BB, SB, BSK, DS, PS, LDW>;
     static int regs_ok = -1;
     if (regs_ok < 0)
         regs_ok = regs_cover<NP>((const void *)kq) && regs_cover<NP>((const void *)kkv);
@@ -1444,35 +1419,38 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
                              "band_bwd: launch registers below the warpgroup split");
         return SA_ERR_CUDA;
     }
-    const int64_t BH = q->B * q->H, T = q->T;
-    const uint64_t rows = (uint64_t)(BH * T);
-    // 128-row boxes for the tiles and distance blocks, BB-row boxes for the
-    // band rings, one-row maps for the CSR gathers
-    CUtensorMap mq, mdo, mk, mv, mqb, mdob, mkb, mvb, mqr, mdor, mkr, mvr;
+    const int64_t BH = q->B * q->H, BHkv = k->B * k->H, T = q->T;
+    // 128-row boxes for the tiles, BB-row boxes for the band rings
+    CUtensorMap mq, mdo, mk, mv, mqb, mdob, mkb, mvb;
     if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BM) ||
         !sa_tmap_bf16_3d(&mdo, dout->ptr, D, T, BH, BM) ||
-        !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BH, BM) || !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BH, BM) ||
+        !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BHkv, BM) ||
+        !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BHkv, BM) ||
         !sa_tmap_bf16_3d(&mqb, q->ptr, D, T, BH, BB) ||
         !sa_tmap_bf16_3d(&mdob, dout->ptr, D, T, BH, BB) ||
-        !sa_tmap_bf16_3d(&mkb, k->ptr, D, T, BH, BB) ||
-        !sa_tmap_bf16_3d(&mvb, v->ptr, D, T, BH, BB) ||
-        !sa_tmap_bf16_rows(&mqr, q->ptr, D, rows) || !sa_tmap_bf16_rows(&mkr, k->ptr, D, rows) ||
-        !sa_tmap_bf16_rows(&mvr, v->ptr, D, rows) || !sa_tmap_bf16_rows(&mdor, dout->ptr, D, rows)) {
+        !sa_tmap_bf16_3d(&mkb, k->ptr, D, T, BHkv, BB) ||
+        !sa_tmap_bf16_3d(&mvb, v->ptr, D, T, BHkv, BB)) {
         sa_record_cuda_error(cudaErrorInvalidValue, "band_bwd: tensor map encoding");
         return SA_ERR_CUDA;
     }
     BwdArgs a{};
     a.T = T;
     a.BH = BH;
+    a.H = q->H;
+    a.Hkv = k->H;
+    a.l2pf = (double)BH * (double)T * D * 2 * 2 > 64.0 * 1024 * 1024 ? 1 : 0;
     a.W = g->W;
     a.kind = g->kind;
-    a.n_off = g->kind == 0 ? g->n_off : 0;
-    for (int x = 0; x < SA_MAX_OFFSETS; ++x) a.offs[x] = x < a.n_off ? g->offs[x] : 0;
+    a.We = sa_fold_links(g, BB, kMaxFold, a.fold, &a.nf, a.offs, &a.n_off);
     a.rowptr = g->rowptr;
     a.colidx = g->colidx;
     a.rev_rowptr = g->rev_rowptr;
     a.rev_colidx = g->rev_colidx;
     a.o = (const __nv_bfloat16 *)o->ptr;
+    a.k = (const __nv_bfloat16 *)k->ptr;
+    a.v = (const __nv_bfloat16 *)v->ptr;
+    a.q = (const __nv_bfloat16 *)q->ptr;
+    a.dout = (const __nv_bfloat16 *)dout->ptr;
     a.lse = lse;
     a.delta = delta;
     a.pds = (g->kind == 0 && g->n_off > 0) ? (float2 *)pds : nullptr;
@@ -1485,30 +1463,32 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     if (!a.err) return SA_ERR_CUDA;
     SA_CUDA_TRY(sa_smem_optin((const void *)kq, LQ::kAlloc));
     SA_CUDA_TRY(sa_smem_optin((const void *)kkv, LK::kAlloc));
-    // persistent: one CTA per SM, NP tiles in flight in each
-    const int64_t ntiles = ((T + BM - 1) / BM) * BH;
+    // persistent: one CTA per SM, NP tiles in flight in each; dQ tiles run
+    // over query slices, dK/dV tiles over key/value slices
     int sms = 0;
     SA_CUDA_TRY(sa_sm_count(&sms));
-    const int64_t nctas = (ntiles + NP - 1) / NP;
-    const unsigned grid = (unsigned)(nctas < sms ? nctas : sms);
+    auto grid_for = [&](int64_t slices) {
+        const int64_t nctas = (((T + BM - 1) / BM) * slices + NP - 1) / NP;
+        return (unsigned)(nctas < sms ? nctas : sms);
+    };
     SA_LAUNCH("band_bwd_dq", s,
-              kq<<<grid, kThreads, LQ::kAlloc, s>>>(mq, mdo, mkb, mvb, mk, mv, mkr, mvr, a));
+              kq<<<grid_for(BH), kThreads, LQ::kAlloc, s>>>(mq, mdo, mkb, mvb, mk, mv, a));
     SA_LAUNCH("band_bwd_dkdv", s,
-              kkv<<<grid, kThreads, LK::kAlloc, s>>>(mk, mv, mqb, mdob, mq, mdo, mqr, mdor, a));
+              kkv<<<grid_for(BHkv), kThreads, LK::kAlloc, s>>>(mk, mv, mqb, mdob, mq, mdo, a));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
 
 }  // namespace
 
-bool sa_band_bwd_supported(const sa_tensor *q, const sa_graph_s *g) {
+bool sa_band_bwd_supported(const sa_tensor *q, const sa_tensor *k, const sa_graph_s *g) {
     if (q->dtype != SA_BF16 || (q->D != 64 && q->D != 128)) return false;
     if (g->W < 1) return false;
-    if (q->B * q->H > 65535 || q->T >= ((int64_t)1 << 31)) return false;
-    const bool diag = (g->kind == 0) ? g->n_off > 0 : (g->max_resid > 0 || g->max_resid_rev > 0);
+    // 32-bit tile coordinates; the CSR gathers address rows of all slices
+    // (slice * T + row) as one int32 coordinate
+    if (q->B * q->H >= ((int64_t)1 << 31) || q->T >= ((int64_t)1 << 31)) return false;
+    if (g->kind == 1 && q->B * q->H * q->T >= ((int64_t)1 << 31)) return false;
     if (g->kind == 1 && (!g->rowptr || !g->rev_rowptr)) return false;
-    // distance / CSR edges with D = 128 stay on the gather kernels (shared memory)
-    if (diag && q->D == 128) return false;
     return true;
 }
 
@@ -1520,12 +1500,17 @@ sa_status sa_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
     // <D, pipelines, band block, S buffers, dQ ring stages, dK/dV ring stages,
     //  diagonal stages, shared-memory P/dS tiles>, sized to the 227 KB of
     // shared memory and 512 TMEM columns
-    if (q->D == 64)
-        return diag ? launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0>(q, k, v, out, lse, dout, g,
-                                                                scale, dq, dk, dv, delta, pds, s)
-                    : launch_band_bwd<64, 2, 32, 2, 4, 4, 0, 0>(q, k, v, out, lse, dout, g,
-                                                                scale, dq, dk, dv, delta, pds, s);
-    // D = 128: one pipeline, P^T / dS^T and dS in shared memory
-    return launch_band_bwd<128, 1, 64, 2, 3, 3, 0, 1>(q, k, v, out, lse, dout, g, scale, dq, dk,
-                                                      dv, delta, pds, s);
+    const bool csr = g->kind == 1;
+#define SA_BWD_ARGS q, k, v, out, lse, dout, g, scale, dq, dk, dv, delta, pds, s
+    if (q->D == 64) {
+        if (!diag) return launch_band_bwd<64, 2, 32, 2, 4, 4, 0, 0, false>(SA_BWD_ARGS);
+        return csr ? launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0, true>(SA_BWD_ARGS)
+                   : launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0, false>(SA_BWD_ARGS);
+    }
+    // D = 128: one pipeline, P^T / dS^T and dS in shared memory; with
+    // diagonal edges a one-stage diagonal ring and two-stage band rings
+    if (!diag) return launch_band_bwd<128, 1, 64, 2, 3, 3, 0, 1, false>(SA_BWD_ARGS);
+    return csr ? launch_band_bwd<128, 1, 64, 2, 2, 2, 1, 1, true>(SA_BWD_ARGS)
+               : launch_band_bwd<128, 1, 64, 2, 2, 2, 1, 1, false>(SA_BWD_ARGS);
+#undef SA_BWD_ARGS
 }

@@ -20,143 +20,11 @@
 
 #include "sa_internal.cuh"
 
+#include "gather_common.cuh"
+
 namespace {
 
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr int kWarpsPerBlock = 8;
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ float lg2(float x) {
-    float y;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-template <typename T>
-struct Slice;
-
-template <>
-struct Slice<__nv_bfloat16> {
-    static constexpr int V = 8;
-    __device__ static void load(const __nv_bfloat16 *p, float *f) {
-        uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
-        uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            f[2 * a] = __uint_as_float(w[a] << 16);
-            f[2 * a + 1] = __uint_as_float(w[a] & 0xffff0000u);
-        }
-    }
-    __device__ static void store(__nv_bfloat16 *p, const float *f) {
-        uint32_t w[4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * a], f[2 * a + 1]);
-            w[a] = *reinterpret_cast<uint32_t *>(&h);
-        }
-        *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-};
-
-template <>
-struct Slice<float> {
-    static constexpr int V = 4;
-    __device__ static void load(const float *p, float *f) {
-        float4 u = __ldg(reinterpret_cast<const float4 *>(p));
-        f[0] = u.x;
-        f[1] = u.y;
-        f[2] = u.z;
-        f[3] = u.w;
-    }
-    __device__ static void store(float *p, const float *f) {
-        *reinterpret_cast<float4 *>(p) = make_float4(f[0], f[1], f[2], f[3]);
-    }
-};
-
-// Sum over the L lanes of a group (L a power of two, groups aligned).
-template <int L>
-__device__ __forceinline__ float group_sum(float x) {
-#pragma unroll
-    for (int o = 1; o < L; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
-
-// ---- neighbour enumeration -------------------------------------------------
-
-// Forward list of query i: distance links (keys ascending), then the window.
-struct RowEdges {
-    int64_t deg;
-    int64_t lo;       // window start (structured)
-    int32_t first;    // first distance index with o <= i (structured)
-    int32_t ndil;     // number of distance links (structured)
-    int64_t start;    // CSR start
-};
-
-__device__ __forceinline__ RowEdges row_edges(const GraphView &g, int64_t i) {
-    RowEdges r;
-    if (g.kind == 0) {
-        int32_t first = 0;
-        while (first < g.n_off && g.offs[first] > i) ++first;
-        r.first = first;
-        r.ndil = g.n_off - first;
-        r.lo = i - g.W + 1 < 0 ? 0 : i - g.W + 1;
-        r.deg = r.ndil + (i - r.lo + 1);
-        r.start = 0;
-    } else {
-        r.start = g.rowptr[i];
-        r.deg = g.rowptr[i + 1] - r.start;
-        r.first = r.ndil = 0;
-        r.lo = 0;
-    }
-    return r;
-}
-
-__device__ __forceinline__ int64_t row_edge(const GraphView &g, const RowEdges &r, int64_t i,
-                                            int64_t e) {
-    if (g.kind == 0) {
-        if (e < r.ndil) return i - g.offs[r.first + e];
-        return r.lo + (e - r.ndil);
-    }
-    return g.colidx[r.start + e];
-}
-
-// Transpose list of key j: window queries j .. j+W-1, then j + o ascending.
-struct ColEdges {
-    int64_t deg;
-    int64_t nwin;
-    int64_t start;
-};
-
-__device__ __forceinline__ ColEdges col_edges(const GraphView &g, int64_t j) {
-    ColEdges c;
-    if (g.kind == 0) {
-        c.nwin = g.T - j < g.W ? g.T - j : g.W;
-        int64_t nd = 0;
-        for (int a = 0; a < g.n_off; ++a) nd += (j + g.offs[a] < g.T) ? 1 : 0;
-        c.deg = c.nwin + nd;
-        c.start = 0;
-    } else {
-        c.start = g.rev_rowptr[j];
-        c.deg = g.rev_rowptr[j + 1] - c.start;
-        c.nwin = 0;
-    }
-    return c;
-}
-
-__device__ __forceinline__ int64_t col_edge(const GraphView &g, const ColEdges &c, int64_t j,
-                                            int64_t e) {
-    if (g.kind == 0) {
-        if (e < c.nwin) return j + e;
-        return j + g.offs[g.n_off - 1 - (e - c.nwin)];
-    }
-    return g.rev_colidx[c.start + e];
-}
+using namespace gather;
 
 // ---- kernels ---------------------------------------------------------------
 
@@ -165,7 +33,8 @@ __global__ void __launch_bounds__(256) gather_fwd_kernel(const T *__restrict__ q
                                                          const T *__restrict__ k,
                                                          const T *__restrict__ v, GraphView g,
                                                          float scale2, T *__restrict__ out,
-                                                         float *__restrict__ lse, int64_t ntiles) {
+                                                         float *__restrict__ lse, int64_t ntiles,
+                                                         int64_t H, int64_t Hkv) {
     constexpr int V = Slice<T>::V, L = D / V, G = 32 / L;
     static_assert(L >= 1 && L <= 32 && G * L == 32, "slice layout");
     const int lane = threadIdx.x & 31, grp = lane / L, sub = lane % L;
@@ -173,7 +42,7 @@ __global__ void __launch_bounds__(256) gather_fwd_kernel(const T *__restrict__ q
     const int64_t i = (blockIdx.x % ntiles) * kWarpsPerBlock + (threadIdx.x >> 5);
     const int64_t T_ = g.T;
     if (i >= T_) return;
-    const int64_t base = bh * T_ * D;
+    const int64_t base = bh * T_ * D, kvbase = kv_slice(bh, H, Hkv) * T_ * D;
     float qf[V];
     Slice<T>::load(q + base + i * D + sub * V, qf);
 #pragma unroll
@@ -188,8 +57,8 @@ __global__ void __launch_bounds__(256) gather_fwd_kernel(const T *__restrict__ q
         float kf[V], vf[V];
         if (valid) {
             const int64_t j = row_edge(g, r, i, e);
-            Slice<T>::load(k + base + j * D + sub * V, kf);
-            Slice<T>::load(v + base + j * D + sub * V, vf);
+            Slice<T>::load(k + kvbase + j * D + sub * V, kf);
+            Slice<T>::load(v + kvbase + j * D + sub * V, vf);
         } else {
 #pragma unroll
             for (int a = 0; a < V; ++a) kf[a] = vf[a] = 0.f;
@@ -238,14 +107,15 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) gather_bwd_dq_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const T *__restrict__ o, const float *__restrict__ lse, const T *__restrict__ dout, GraphView g,
-    float scale, T *__restrict__ dq, float *__restrict__ delta, int64_t ntiles) {
+    float scale, T *__restrict__ dq, float *__restrict__ delta, int64_t ntiles, int64_t H,
+    int64_t Hkv) {
     constexpr int V = Slice<T>::V, L = D / V, G = 32 / L;
     const int lane = threadIdx.x & 31, grp = lane / L, sub = lane % L;
     const int64_t bh = blockIdx.x / ntiles;
     const int64_t i = (blockIdx.x % ntiles) * kWarpsPerBlock + (threadIdx.x >> 5);
     const int64_t T_ = g.T;
     if (i >= T_) return;
-    const int64_t base = bh * T_ * D;
+    const int64_t base = bh * T_ * D, kvbase = kv_slice(bh, H, Hkv) * T_ * D;
     const float scale2 = scale * kLog2e;
     float qf[V], df[V], of[V];
     Slice<T>::load(q + base + i * D + sub * V, qf);
@@ -269,8 +139,8 @@ __global__ void __launch_bounds__(256) gather_bwd_dq_kernel(
         float kf[V], vf[V];
         if (valid) {
             const int64_t j = row_edge(g, r, i, e);
-            Slice<T>::load(k + base + j * D + sub * V, kf);
-            Slice<T>::load(v + base + j * D + sub * V, vf);
+            Slice<T>::load(k + kvbase + j * D + sub * V, kf);
+            Slice<T>::load(v + kvbase + j * D + sub * V, vf);
         } else {
 #pragma unroll
             for (int a = 0; a < V; ++a) kf[a] = vf[a] = 0.f;
@@ -306,54 +176,60 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) gather_bwd_dkdv_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const float *__restrict__ lse, const float *__restrict__ delta, const T *__restrict__ dout,
-    GraphView g, float scale, T *__restrict__ dk, T *__restrict__ dv, int64_t ntiles) {
+    GraphView g, float scale, T *__restrict__ dk, T *__restrict__ dv, int64_t ntiles, int64_t H,
+    int64_t Hkv) {
     constexpr int V = Slice<T>::V, L = D / V, G = 32 / L;
     const int lane = threadIdx.x & 31, grp = lane / L, sub = lane % L;
-    const int64_t bh = blockIdx.x / ntiles;
+    const int64_t kvbh = blockIdx.x / ntiles;  // key/value slice
     const int64_t j = (blockIdx.x % ntiles) * kWarpsPerBlock + (threadIdx.x >> 5);
     const int64_t T_ = g.T;
     if (j >= T_) return;
-    const int64_t base = bh * T_ * D;
+    const int64_t kvbase = kvbh * T_ * D;
+    // the query heads that read this key/value head: a group of H / Hkv
+    const int64_t gsize = H / Hkv, qbh0 = (kvbh / Hkv) * H + (kvbh % Hkv) * gsize;
     const float scale2 = scale * kLog2e;
     float kf[V], vf[V];
-    Slice<T>::load(k + base + j * D + sub * V, kf);
-    Slice<T>::load(v + base + j * D + sub * V, vf);
+    Slice<T>::load(k + kvbase + j * D + sub * V, kf);
+    Slice<T>::load(v + kvbase + j * D + sub * V, vf);
 #pragma unroll
     for (int a = 0; a < V; ++a) kf[a] *= scale2;
     const ColEdges c = col_edges(g, j);
     float adk[V], adv[V];
 #pragma unroll
     for (int a = 0; a < V; ++a) adk[a] = adv[a] = 0.f;
-    for (int64_t e0 = 0; e0 < c.deg; e0 += G) {
-        const int64_t e = e0 + grp;
-        const bool valid = e < c.deg;
-        float qf[V], df[V];
-        float lse2 = 0.f, Delta = 0.f;
-        if (valid) {
-            const int64_t i = col_edge(g, c, j, e);
-            Slice<T>::load(q + base + i * D + sub * V, qf);
-            Slice<T>::load(dout + base + i * D + sub * V, df);
-            lse2 = __ldg(lse + bh * T_ + i) * kLog2e;
-            Delta = __ldg(delta + bh * T_ + i);
-        } else {
+    for (int64_t hq = 0; hq < gsize; ++hq) {
+        const int64_t bh = qbh0 + hq, base = bh * T_ * D;
+        for (int64_t e0 = 0; e0 < c.deg; e0 += G) {
+            const int64_t e = e0 + grp;
+            const bool valid = e < c.deg;
+            float qf[V], df[V];
+            float lse2 = 0.f, Delta = 0.f;
+            if (valid) {
+                const int64_t i = col_edge(g, c, j, e);
+                Slice<T>::load(q + base + i * D + sub * V, qf);
+                Slice<T>::load(dout + base + i * D + sub * V, df);
+                lse2 = __ldg(lse + bh * T_ + i) * kLog2e;
+                Delta = __ldg(delta + bh * T_ + i);
+            } else {
 #pragma unroll
-            for (int a = 0; a < V; ++a) qf[a] = df[a] = 0.f;
-        }
-        float s = 0.f, dp = 0.f;
-#pragma unroll
-        for (int a = 0; a < V; ++a) {
-            s = fmaf(qf[a], kf[a], s);
-            dp = fmaf(df[a], vf[a], dp);
-        }
-        s = group_sum<L>(s);
-        dp = group_sum<L>(dp);
-        if (valid) {
-            const float p = ex2(s - lse2);
-            const float ds = p * (dp - Delta);
+                for (int a = 0; a < V; ++a) qf[a] = df[a] = 0.f;
+            }
+            float s = 0.f, dp = 0.f;
 #pragma unroll
             for (int a = 0; a < V; ++a) {
-                adv[a] = fmaf(p, df[a], adv[a]);
-                adk[a] = fmaf(ds, qf[a], adk[a]);
+                s = fmaf(qf[a], kf[a], s);
+                dp = fmaf(df[a], vf[a], dp);
+            }
+            s = group_sum<L>(s);
+            dp = group_sum<L>(dp);
+            if (valid) {
+                const float p = ex2(s - lse2);
+                const float ds = p * (dp - Delta);
+#pragma unroll
+                for (int a = 0; a < V; ++a) {
+                    adv[a] = fmaf(p, df[a], adv[a]);
+                    adk[a] = fmaf(ds, qf[a], adk[a]);
+                }
             }
         }
     }
@@ -367,8 +243,8 @@ __global__ void __launch_bounds__(256) gather_bwd_dkdv_kernel(
     if (grp == 0) {
 #pragma unroll
         for (int a = 0; a < V; ++a) adk[a] *= scale;
-        Slice<T>::store(dk + base + j * D + sub * V, adk);
-        Slice<T>::store(dv + base + j * D + sub * V, adv);
+        Slice<T>::store(dk + kvbase + j * D + sub * V, adk);
+        Slice<T>::store(dv + kvbase + j * D + sub * V, adv);
     }
 }
 
@@ -383,7 +259,7 @@ sa_status launch_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
     SA_LAUNCH("gather_fwd", s,
               gather_fwd_kernel<T, D><<<(unsigned)nblocks, 256, 0, s>>>(
                   (const T *)q->ptr, (const T *)k->ptr, (const T *)v->ptr, g, scale * kLog2e,
-                  (T *)out->ptr, lse, ntiles));
+                  (T *)out->ptr, lse, ntiles, q->H, k->H));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
@@ -401,11 +277,13 @@ sa_status launch_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
     SA_LAUNCH("gather_bwd_dq", s,
               gather_bwd_dq_kernel<T, D><<<(unsigned)nblocks, 256, 0, s>>>(
                   (const T *)q->ptr, (const T *)k->ptr, (const T *)v->ptr, (const T *)o->ptr, lse,
-                  (const T *)dout->ptr, g, scale, (T *)dq->ptr, delta, ntiles));
+                  (const T *)dout->ptr, g, scale, (T *)dq->ptr, delta, ntiles, q->H, k->H));
+    const int64_t nblocks_kv = ntiles * (k->B * k->H);
     SA_LAUNCH("gather_bwd_dkdv", s,
-              gather_bwd_dkdv_kernel<T, D><<<(unsigned)nblocks, 256, 0, s>>>(
+              gather_bwd_dkdv_kernel<T, D><<<(unsigned)nblocks_kv, 256, 0, s>>>(
                   (const T *)q->ptr, (const T *)k->ptr, (const T *)v->ptr, lse, delta,
-                  (const T *)dout->ptr, g, scale, (T *)dk->ptr, (T *)dv->ptr, ntiles));
+                  (const T *)dout->ptr, g, scale, (T *)dk->ptr, (T *)dv->ptr, ntiles, q->H,
+                  k->H));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }

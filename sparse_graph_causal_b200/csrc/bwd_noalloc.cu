@@ -14,32 +14,26 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include <mutex>
-
 #include "sa_internal.cuh"
 
 namespace {
 
 __device__ __align__(256) float g_noalloc_delta[SA_NOALLOC_MAX_ROWS];
 
-constexpr int kMaxDevices = 64;
-float *g_noalloc_ptr[kMaxDevices] = {};
-std::mutex g_noalloc_mu;
-
-// Device address of the array on the current device.  In host code the
+// Device address of the array in the current context.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// with the device current.  It is looked up again on every call (cheap once
+// the module is loaded) rather than cached, so that a reset device or a
+// different context never receives a stale address.
 sa_status noalloc_scratch(float **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return SA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_delta) != cudaSuccess || !p) return SA_ERR_CUDA;
-        g_noalloc_ptr[dev] = static_cast<float *>(p);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_delta);
+    if (e != cudaSuccess || !p) {
+        sa_record_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
+                             "bwd_noalloc: cudaGetSymbolAddress");
+        return SA_ERR_CUDA;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = static_cast<float *>(p);
     return SA_OK;
 }
 
@@ -50,14 +44,20 @@ extern "C" sa_status sparse_attn_bwd_noalloc(const sa_tensor *q, const sa_tensor
                                              const float *lse, const sa_tensor *dout, sa_graph g,
                                              float scale, sa_tensor *dq, sa_tensor *dk,
                                              sa_tensor *dv, void *stream) {
-    if (!q || q->B < 1 || q->H < 1 || q->T < 1) return SA_ERR_INVALID_ARG;
-    if (q->B * q->H * q->T > (int64_t)SA_NOALLOC_MAX_ROWS) return SA_ERR_UNSUPPORTED;
-    float *scratch = nullptr;
-    sa_status st = noalloc_scratch(&scratch);
+    // every argument is checked first (a bad one is SA_ERR_INVALID_ARG
+    // whatever its size), then the size against the array
+    sa_status st = sa_bwd_check_args(q, k, v, out, lse, dout, g, scale, dq, dk, dv);
     if (st != SA_OK) return st;
-    // Delta is written in full by the dQ pass before the dK/dV pass reads it,
-    // so nothing in the array has to start at zero.  Without room for the
-    // distance-edge cache the dK/dV pass recomputes p and dS.
+    // rows = B * H * T, compared step by step so that no product overflows
+    const int64_t kMax = SA_NOALLOC_MAX_ROWS;
+    if (q->B > kMax || q->H > kMax / q->B || q->T > kMax / (q->B * q->H))
+        return SA_ERR_UNSUPPORTED;
+    float *scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != SA_OK) return st;
+    // Delta is written in full by the dQ pass before the dK/dV pass
+    // reads it, so nothing in the array has to start at zero.  Without room
+    // for the distance-edge cache the dK/dV pass recomputes p and dS.
     return sa_bwd_with_scratch(q, k, v, out, lse, dout, g, scale, dq, dk, dv, scratch, nullptr,
                                stream);
 }

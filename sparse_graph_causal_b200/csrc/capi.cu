@@ -54,6 +54,18 @@ sa_status check_tensor(const sa_tensor *t, const sa_tensor *ref) {
     return SA_OK;
 }
 
+// k (and v, dk, dv): q's B, T, D and dtype, with a head count that divides
+// q's (grouped-query attention: query head h reads key/value head
+// h / (H / Hkv)).
+sa_status check_kv(const sa_tensor *t, const sa_tensor *q) {
+    sa_status st = check_tensor(t, nullptr);
+    if (st != SA_OK) return st;
+    if (t->B != q->B || t->T != q->T || t->D != q->D || t->dtype != q->dtype)
+        return SA_ERR_INVALID_ARG;
+    if (q->H % t->H != 0) return SA_ERR_INVALID_ARG;
+    return SA_OK;
+}
+
 sa_status check_common(const sa_tensor *q, sa_graph g) {
     if (!g) return SA_ERR_INVALID_ARG;
     sa_status st = check_tensor(q, nullptr);
@@ -360,7 +372,7 @@ sa_status sparse_attn_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
                           float scale, sa_tensor *out, float *lse, void *stream) {
     sa_status st = check_common(q, g);
     if (st != SA_OK) return st;
-    if ((st = check_tensor(k, q)) != SA_OK || (st = check_tensor(v, q)) != SA_OK ||
+    if ((st = check_kv(k, q)) != SA_OK || (st = check_tensor(v, k)) != SA_OK ||
         (st = check_tensor(out, q)) != SA_OK)
         return st;
     if (!lse || !aligned16(lse) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
@@ -392,19 +404,32 @@ size_t sparse_attn_bwd_workspace_size(const sa_tensor *q, sa_graph g) {
 }  // extern "C"
 
 // C++ linkage: not part of the C ABI.
+sa_status sa_bwd_check_args(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                            const sa_tensor *out, const float *lse, const sa_tensor *dout,
+                            sa_graph g, float scale, const sa_tensor *dq, const sa_tensor *dk,
+                            const sa_tensor *dv) {
+    sa_status st = check_common(q, g);
+    if (st != SA_OK) return st;
+    if ((st = check_kv(k, q)) != SA_OK) return st;
+    const sa_tensor *qs[] = {out, dout, dq};
+    for (const sa_tensor *t : qs)
+        if ((st = check_tensor(t, q)) != SA_OK) return st;
+    const sa_tensor *ks[] = {v, dk, dv};
+    for (const sa_tensor *t : ks)
+        if ((st = check_tensor(t, k)) != SA_OK) return st;
+    if (!lse || !aligned16(lse) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
+    return SA_OK;
+}
+
 sa_status sa_bwd_with_scratch(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                               const sa_tensor *out, const float *lse, const sa_tensor *dout,
                               sa_graph g, float scale, sa_tensor *dq, sa_tensor *dk,
                               sa_tensor *dv, float *delta, void *edge_cache, void *stream) {
-    sa_status st = check_common(q, g);
+    sa_status st = sa_bwd_check_args(q, k, v, out, lse, dout, g, scale, dq, dk, dv);
     if (st != SA_OK) return st;
-    const sa_tensor *ts[] = {k, v, out, dout, dq, dk, dv};
-    for (const sa_tensor *t : ts)
-        if ((st = check_tensor(t, q)) != SA_OK) return st;
-    if (!lse || !aligned16(lse) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
     cudaStream_t s = as_stream(stream);
     const GraphView gv = make_view(g);
-    if (g_path.load() == SA_PATH_AUTO && sa_band_bwd_supported(q, g))
+    if (g_path.load() == SA_PATH_AUTO && sa_band_bwd_supported(q, k, g))
         return sa_band_bwd(q, k, v, out, lse, dout, g, gv, scale, dq, dk, dv, delta, edge_cache,
                            s);
     return sa_gather_bwd(q, k, v, out, lse, dout, gv, scale, dq, dk, dv, delta, s);
@@ -428,3 +453,87 @@ sa_status sparse_attn_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ learned-coordinate scoring
+
+namespace {
+
+// a, c: fp32 [B, H, T, 3] with v's B, H, T; v: bf16/fp32 [B, H, T, D].
+sa_status check_dist(const sa_tensor *a, const sa_tensor *c, const sa_tensor *v, sa_graph g) {
+    sa_status st = check_common(v, g);
+    if (st != SA_OK) return st;
+    if ((st = check_tensor(a, nullptr)) != SA_OK || (st = check_tensor(c, a)) != SA_OK) return st;
+    if (a->dtype != SA_FP32 || a->D != 3) return SA_ERR_INVALID_ARG;
+    if (a->B != v->B || a->H != v->H || a->T != v->T) return SA_ERR_INVALID_ARG;
+    return SA_OK;
+}
+
+size_t dist_delta_bytes(const sa_tensor *v) {
+    const size_t n = sizeof(float) * (size_t)(v->B * v->H * v->T);
+    return (n + 255) & ~(size_t)255;
+}
+
+}  // namespace
+
+extern "C" {
+
+sa_status sparse_attn_dist_fwd(const sa_tensor *a, const sa_tensor *c, const sa_tensor *v,
+                               sa_graph g, float scale, sa_tensor *out, float *lse,
+                               void *stream) {
+    sa_status st = check_dist(a, c, v, g);
+    if (st != SA_OK) return st;
+    if ((st = check_tensor(out, v)) != SA_OK) return st;
+    if (!lse || !aligned16(lse) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
+    return sa_dist_fwd(a, c, v, make_view(g), scale, out, lse, as_stream(stream));
+}
+
+size_t sparse_attn_dist_bwd_workspace_size(const sa_tensor *v, sa_graph) {
+    if (!v || v->B < 1 || v->H < 1 || v->T < 1) return 0;
+    return dist_delta_bytes(v);
+}
+
+sa_status sparse_attn_dist_bwd(const sa_tensor *a, const sa_tensor *c, const sa_tensor *v,
+                               const sa_tensor *out, const float *lse, const sa_tensor *dout,
+                               sa_graph g, float scale, sa_tensor *da, sa_tensor *dc,
+                               sa_tensor *dv, void *workspace, size_t ws_bytes, void *stream) {
+    sa_status st = check_dist(a, c, v, g);
+    if (st != SA_OK) return st;
+    if ((st = check_tensor(out, v)) != SA_OK || (st = check_tensor(dout, v)) != SA_OK ||
+        (st = check_tensor(dv, v)) != SA_OK || (st = check_tensor(da, a)) != SA_OK ||
+        (st = check_tensor(dc, a)) != SA_OK)
+        return st;
+    if (!lse || !aligned16(lse) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+        ws_bytes < dist_delta_bytes(v))
+        return SA_ERR_INVALID_ARG;
+    return sa_dist_bwd(a, c, v, out, lse, dout, make_view(g), scale, da, dc, dv,
+                       static_cast<float *>(workspace), as_stream(stream));
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ decode
+
+extern "C" sa_status sparse_attn_decode(const sa_tensor *q, const sa_tensor *k_cache,
+                                        const sa_tensor *v_cache, const int64_t *pos,
+                                        sa_graph g, float scale, sa_tensor *out, float *lse,
+                                        void *stream) {
+    if (!g) return SA_ERR_INVALID_ARG;
+    sa_status st = check_tensor(q, nullptr);
+    if (st != SA_OK) return st;
+    if ((st = check_tensor(k_cache, nullptr)) != SA_OK ||
+        (st = check_tensor(v_cache, k_cache)) != SA_OK || (st = check_tensor(out, q)) != SA_OK)
+        return st;
+    if (q->T != 1) return SA_ERR_INVALID_ARG;
+    if (k_cache->B != q->B || k_cache->D != q->D || k_cache->dtype != q->dtype)
+        return SA_ERR_INVALID_ARG;
+    if (q->H % k_cache->H != 0) return SA_ERR_INVALID_ARG;
+    if (k_cache->T > g->T) return SA_ERR_INVALID_ARG;
+    if (q->D != 32 && q->D != 64 && q->D != 128) return SA_ERR_UNSUPPORTED;
+    if (!pos || (reinterpret_cast<uintptr_t>(pos) & 7u) != 0) return SA_ERR_INVALID_ARG;
+    if (!lse || !aligned16(lse) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+    if (dev != g->device) return SA_ERR_INVALID_ARG;
+    return sa_decode(q, k_cache, v_cache, pos, make_view(g), scale, out, lse, as_stream(stream));
+}

@@ -21,6 +21,8 @@
 namespace {
 
 constexpr int kThreads = 256;
+// Longest shared key prefix looked for: one 64-key block of the forward.
+const int kPrefixCap = 64;
 
 // ------------------------------------------------------------------ scan
 
@@ -338,6 +340,21 @@ __global__ void csr_band_check(int64_t T, const int64_t *rowptr, const int32_t *
     atomicMax(max_resid, (int)(r > 0x7fffffff ? 0x7fffffff : r));
 }
 
+// Shared key prefix: the largest G <= cap such that every row i holds the
+// keys 0 .. min(G, i + 1) - 1 (global tokens every query sees).  Row i holds
+// them when its sorted list starts 0, 1, ..., so each row that does not hold
+// all of 0 .. i bounds G by the length of its run of leading keys 0, 1, ...
+// (*g_min starts at cap).
+__global__ void csr_key_prefix(int64_t T, const int64_t *rowptr, const int32_t *colidx, int cap,
+                               int *g_min) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= T) return;
+    const int64_t s = rowptr[i], deg = rowptr[i + 1] - s;
+    int run = 0;
+    while (run < cap && run < deg && colidx[s + run] == run) ++run;
+    if (run < cap && (int64_t)run < i + 1) atomicMin(g_min, run);
+}
+
 __global__ void csr_rev_counts(const int32_t *colidx, int64_t nnz, int32_t *indeg) {
     int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e < nnz) atomicAdd(&indeg[colidx[e]], 1);
@@ -412,13 +429,13 @@ sa_status sa_graph_from_csr(sa_graph_s *g, const int64_t *rowptr, const int32_t 
     uint32_t *rows = nullptr, *keys = nullptr;
     int32_t *keep = nullptr, *indeg = nullptr;
     int64_t *pos = nullptr;
-    int *flags = nullptr;  // [0] errors, [1] max resid, [2] max resid rev
+    int *flags = nullptr;  // [0] errors, [1] max resid, [2] max resid rev, [3] key prefix
     SortBuffers sb;
     int64_t n = nnz;
     int64_t ntiles = (n + kRsTile - 1) / kRsTile;
     int64_t nc = 256 * (ntiles < 1 ? 1 : ntiles);
     int64_t scan_n = std::max<int64_t>(std::max<int64_t>(n + 1, T + 1), nc);
-    int host_flags[3] = {0, 0, 0};
+    int host_flags[4] = {0, 0, 0, 0};
     int kbits = bits_for(T > 0 ? T - 1 : 0);
 
 #define TRY(...)                        \
@@ -488,6 +505,12 @@ sa_status sa_graph_from_csr(sa_graph_s *g, const int64_t *rowptr, const int32_t 
     SA_LAUNCH("graph_csr_band", s,
               csr_band_check<<<blocks_for(T), kThreads, 0, s>>>(T, g->rowptr, g->colidx, band,
                                                                  flags, flags + 1));
+    // shared key prefix (at most one 64-key block), for the forward's dense
+    // prefix block
+    CTRY(cudaMemcpyAsync(flags + 3, &kPrefixCap, sizeof(int), cudaMemcpyHostToDevice, s));
+    SA_LAUNCH("graph_csr_prefix", s,
+              csr_key_prefix<<<blocks_for(T), kThreads, 0, s>>>(T, g->rowptr, g->colidx,
+                                                                 kPrefixCap, flags + 3));
     // 5. transpose: stable sort of (key, row) pairs of the normalised lists by key
     CTRY(cudaMemsetAsync(indeg, 0, sizeof(int32_t) * (size_t)(T + 1), s));
     if (new_nnz > 0) {
@@ -508,7 +531,7 @@ sa_status sa_graph_from_csr(sa_graph_s *g, const int64_t *rowptr, const int32_t 
     SA_LAUNCH("graph_csr_rev_resid", s,
               csr_rev_resid<<<blocks_for(T), kThreads, 0, s>>>(T, g->rev_rowptr, band, flags + 2));
     CTRY(cudaGetLastError());
-    CTRY(cudaMemcpyAsync(host_flags, flags, 3 * sizeof(int), cudaMemcpyDeviceToHost, s));
+    CTRY(cudaMemcpyAsync(host_flags, flags, 4 * sizeof(int), cudaMemcpyDeviceToHost, s));
     CTRY(cudaStreamSynchronize(s));
     if (host_flags[0]) {
         st = SA_ERR_INVALID_GRAPH;
@@ -517,6 +540,7 @@ sa_status sa_graph_from_csr(sa_graph_s *g, const int64_t *rowptr, const int32_t 
     g->W = band;
     g->max_resid = host_flags[1];
     g->max_resid_rev = host_flags[2];
+    g->gprefix = host_flags[3];
     g->materialized = 1;
 
 cleanup:

@@ -4,7 +4,7 @@
 #include "sa_internal.cuh"
 
 bool sa_band_fwd_supported(const sa_tensor *q, const sa_graph_s *g);
-bool sa_band_bwd_supported(const sa_tensor *q, const sa_graph_s *g);
+bool sa_band_bwd_supported(const sa_tensor *q, const sa_tensor *k, const sa_graph_s *g);
 sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                       const sa_graph_s *g, const GraphView &gv, float scale, sa_tensor *out,
                       float *lse, cudaStream_t s);

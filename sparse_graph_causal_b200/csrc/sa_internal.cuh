@@ -24,6 +24,7 @@ struct sa_graph_s {
     int64_t *rev_rowptr = nullptr;
     int32_t *rev_colidx = nullptr;
     int32_t max_resid = 0;      // max edges outside the band over rows
+    int32_t gprefix = 0;        // CSR: every row i holds keys 0 .. min(gprefix, i + 1) - 1
     int32_t max_resid_rev = 0;  // max transpose edges outside the band over keys
     int device = 0;
 };
@@ -100,6 +101,35 @@ __host__ __device__ inline int64_t sg_in_degree(int64_t j, int64_t T, int64_t W,
     return d;
 }
 
+// Distance links of a structured graph that fall inside the span of keys the
+// band blocks of a 128-row tile cover anyway (ceil((W + 127) / blk) blocks of
+// blk keys starting at the first window key): such a link o is one more kept
+// key per row inside those blocks, and is taken out of the gathered links.
+// Writes the folded links (ascending, at most max_fold) to fold[], the others
+// (descending) to rest[] and returns the span of the band blocks, We = W or
+// the longest folded link + 1 (the blocks then start at key i - We + 1).
+inline int32_t sa_fold_links(const sa_graph_s *g, int blk, int max_fold, int32_t *fold,
+                             int *n_fold, int64_t *rest, int *n_rest) {
+    *n_fold = 0;
+    *n_rest = 0;
+    int32_t We = g->W;
+    const int64_t span = (int64_t)blk * ((g->W + 127 + blk - 1) / blk) - 127;
+    for (int x = g->n_off - 1; x >= 0; --x) {  // ascending
+        const int64_t o = g->offs[x];
+        if (g->kind == 0 && o < span && *n_fold < max_fold) {
+            fold[(*n_fold)++] = (int32_t)o;
+            We = (int32_t)o + 1;
+        }
+    }
+    for (int x = 0; x < g->n_off; ++x) {
+        const int64_t o = g->offs[x];
+        bool folded = false;
+        for (int y = 0; y < *n_fold; ++y) folded |= (fold[y] == o);
+        if (!folded) rest[(*n_rest)++] = o;
+    }
+    return We;
+}
+
 // Number of SMs of the current device (cached per device).
 cudaError_t sa_sm_count(int *n);
 
@@ -130,6 +160,11 @@ sa_status sa_graph_from_csr(sa_graph_s *g, const int64_t *rowptr, const int32_t 
 sa_status sa_gather_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                         const GraphView &gv, float scale, sa_tensor *out, float *lse,
                         cudaStream_t s);
+// Every argument check of the backward (nothing is launched).
+sa_status sa_bwd_check_args(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                            const sa_tensor *out, const float *lse, const sa_tensor *dout,
+                            sa_graph g, float scale, const sa_tensor *dq, const sa_tensor *dk,
+                            const sa_tensor *dv);
 // Backward with caller-placed scratch: Delta (4 bytes per query row) and an
 // optional distance-edge cache (null: recompute); argument checks included.
 sa_status sa_bwd_with_scratch(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
@@ -140,3 +175,19 @@ sa_status sa_gather_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor 
                         const sa_tensor *out, const float *lse, const sa_tensor *dout,
                         const GraphView &gv, float scale, sa_tensor *dq, sa_tensor *dk,
                         sa_tensor *dv, float *delta, cudaStream_t s);
+
+// Internal launchers (attn_dist.cu): learned-coordinate scoring, every edge
+// on CUDA cores.  a, c: fp32 [B, H, T, 3]; v, out, dout, dv: [B, H, T, D].
+sa_status sa_dist_fwd(const sa_tensor *a, const sa_tensor *c, const sa_tensor *v,
+                      const GraphView &g, float scale, sa_tensor *out, float *lse,
+                      cudaStream_t s);
+sa_status sa_dist_bwd(const sa_tensor *a, const sa_tensor *c, const sa_tensor *v,
+                      const sa_tensor *o, const float *lse, const sa_tensor *dout,
+                      const GraphView &g, float scale, sa_tensor *da, sa_tensor *dc,
+                      sa_tensor *dv, float *delta, cudaStream_t s);
+
+// Internal launcher (attn_decode.cu): one query per (b, h) against a cache.
+// q, out: [B, H, 1, D]; k, v: [B, Hkv, Tmax, D]; pos: device int64 [B].
+sa_status sa_decode(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                    const int64_t *pos, const GraphView &g, float scale, sa_tensor *out,
+                    float *lse, cudaStream_t s);

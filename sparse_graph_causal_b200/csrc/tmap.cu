@@ -32,17 +32,3 @@ bool sa_tmap_bf16_3d(CUtensorMap *m, const void *base, uint64_t D, uint64_t T, u
     return r == CUDA_SUCCESS;
 }
 
-
-bool sa_tmap_bf16_rows(CUtensorMap *m, const void *base, uint64_t D, uint64_t rows) {
-    std::call_once(g_once, load_encode);
-    if (!g_encode) return false;
-    cuuint64_t dims[2] = {D, rows};
-    cuuint64_t strides[1] = {D * 2};
-    cuuint32_t box[2] = {64, 1};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}

@@ -11,7 +11,3 @@
 bool sa_tmap_bf16_3d(CUtensorMap *m, const void *base, uint64_t D, uint64_t T, uint64_t BH,
                      uint32_t box_rows);
 
-// The same bf16 tensor as B*H*T rows of D values (2-D: x = D, y = row),
-// one-row boxes of 64 values, no swizzle: the map for 4-row TMA gathers.
-bool sa_tmap_bf16_rows(CUtensorMap *m, const void *base, uint64_t D, uint64_t rows);
-

@@ -119,6 +119,21 @@ def make_qkv(w: Workload, device="cpu", seed: int | None = None, with_dout: bool
     return out
 
 
+def make_coords(w: Workload, device="cpu", seed: int | None = None, std: float = 1.0):
+    """Query and key coordinates a, c of shape [B, H, T, 3], fp32,
+    N(0, std^2), drawn on ``device`` from a torch.Generator (seed: the
+    workload's + 7)."""
+    seed = (w.seed + 7) if seed is None else seed
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    a = torch.empty((w.B, w.H, w.T, 3), dtype=torch.float32, device=dev).normal_(0.0, std,
+                                                                                generator=g)
+    c = torch.empty((w.B, w.H, w.T, 3), dtype=torch.float32, device=dev).normal_(0.0, std,
+                                                                                generator=g)
+    return a, c
+
+
 def csr_random_rows(T: int, seed: int, window: int = 64, n_random: int = 16,
                     n_global: int = 16):
     """Raw neighbour lists, one row per query i, in this order and unsorted:

@@ -7,7 +7,8 @@ on out/lse/dq/dk/dv; fp32 inputs: max-abs 1e-4.  Because some workloads have
 outputs far below 1 (inputs N(0,1)/sqrt(D)), each comparison also bounds the
 error relative to the reference's own range: max-abs <= REL * max|ref| with
 REL = 2^-5 for bf16 (a few bf16 roundings of 2^-9 each, summed over the
-softmax-weighted terms) and 1e-4 for fp32.
+softmax-weighted terms) and 1e-4 for fp32.  Results far from unit scale
+use the STRESS bounds below instead.
 """
 from __future__ import annotations
 
@@ -16,6 +17,14 @@ import torch
 
 TOL = {"bf16": dict(max_abs=2e-2, mean_abs=2e-3, rel=2.0 ** -5),
        "fp32": dict(max_abs=1e-4, mean_abs=1e-4, rel=1e-4)}
+
+# Results far from unit scale (the sharp-softmax stress cases, gradients of
+# up to |x| ~ 8): the fixed bounds give way to bounds relative to max|ref|,
+# set at about twice the largest errors observed on B200 over every stress
+# case, both kernel paths and all of out/lse/dq/dk/dv (max-abs 0.0079 and
+# mean-abs 0.00023 of max|ref|).
+STRESS = {"bf16": dict(rel=2.0 ** -6, rel_mean=5e-4),
+          "fp32": dict(rel=1e-4, rel_mean=1e-5)}
 
 
 def to_oracle(t: torch.Tensor, dtype: str) -> np.ndarray:
@@ -30,14 +39,14 @@ def compare(got, ref: np.ndarray, dtype: str, what: str, scale_floor: float = 1e
             unit_range: float | None = None):
     """got: torch tensor (any float dtype) or ndarray; ref: fp64 ndarray.
 
-    unit_range: set for inputs far from unit scale.  The fixed max-abs bound
-    then gives way to the relative one (2^-5 of the largest |ref|, checked for
-    every case), and the mean-abs bound grows in proportion to max|ref| beyond
-    unit_range.  Two errors that any bf16-output implementation has grow with
-    the values: a result rounded to bf16 is off by up to 2^-8 of its size
-    (0.03 at |x| = 8), and Delta = dO . out must use the rounded out, which by
-    itself moves dq by 0.016-0.020 at |dq| = 5-6 with scores of standard
-    deviation 2 (fp64 emulation of that step alone)."""
+    unit_range: set for results far from unit scale.  The fixed max-abs bound
+    then gives way to the STRESS bounds (max-abs and mean-abs relative to the
+    largest |ref|), both about twice the errors observed on B200.
+    Two errors that any bf16-output implementation has grow with the values:
+    a result rounded to bf16 is off by up to 2^-8 of its size (0.03 at
+    |x| = 8), and Delta = dO . out must use the rounded out, which by itself
+    moves dq by 0.016-0.020 at |dq| = 5-6 with scores of standard deviation 2
+    (fp64 emulation of that step alone)."""
     if isinstance(got, torch.Tensor):
         got = got.detach().float().cpu().numpy()
     got = np.asarray(got, dtype=np.float64)
@@ -50,14 +59,15 @@ def compare(got, ref: np.ndarray, dtype: str, what: str, scale_floor: float = 1e
     if not fin.any():
         return dict(max_abs=0.0, mean_abs=0.0)
     err = np.abs(got[fin] - ref[fin])
-    tol = TOL[dtype]
+    tol = STRESS[dtype] if unit_range else TOL[dtype]
     mx, mean = float(err.max()), float(err.mean())
     rng = max(float(np.abs(ref[fin]).max()), scale_floor)
-    grow = max(1.0, rng / unit_range) if unit_range else 1.0
-    if not unit_range:
+    if unit_range:
+        assert mean <= tol["rel_mean"] * rng + 1e-7, \
+            f"{what}: mean-abs {mean:.3e} > {tol['rel_mean']} * {rng:.3e}"
+    else:
         assert mx <= tol["max_abs"], f"{what}: max-abs {mx:.3e} > {tol['max_abs']}"
-    assert mean <= tol["mean_abs"] * grow, \
-        f"{what}: mean-abs {mean:.3e} > {tol['mean_abs']} * {grow:.2f}"
+        assert mean <= tol["mean_abs"], f"{what}: mean-abs {mean:.3e} > {tol['mean_abs']}"
     assert mx <= tol["rel"] * rng + 1e-7, f"{what}: max-abs {mx:.3e} > {tol['rel']} * {rng:.3e}"
     return dict(max_abs=mx, mean_abs=mean, range=rng)
 

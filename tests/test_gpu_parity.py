@@ -56,6 +56,12 @@ CASES = [
         csr=synth.csr_random_rows(3000, seed=9), band=64),
     _wl("csr_empty_rows", 1, 2, 400, 64, "bf16", 0, (), csr=_random_csr_with_empty(400, 4)),
     _wl("csr_d128", 1, 1, 600, 128, "bf16", 0, (), csr=synth.csr_random_rows(600, seed=8), band=64),
+    # CSR rows with a band but no shared key prefix, and with a prefix longer
+    # than the band (the forward's dense prefix block: none, and 40 keys)
+    _wl("csr_no_prefix", 1, 2, 2000, 64, "bf16", 0, (),
+        csr=synth.csr_random_rows(2000, seed=41, n_global=0), band=64),
+    _wl("csr_prefix40_band16", 1, 2, 1500, 64, "bf16", 0, (),
+        csr=synth.csr_random_rows(1500, seed=42, window=16, n_global=40), band=16),
 ]
 
 
@@ -175,3 +181,29 @@ def test_argument_errors(sa):
     with pytest.raises(sa.SparseAttentionError) as e:      # head size
         sa.sparse_attn_fwd(q48, q48, q48, g, 1.0)
     assert e.value.status == sa.SA_ERR_UNSUPPORTED
+
+
+def test_many_slices_on_tensor_cores(sa, oracle_lib):
+    """B*H above 65,535 (short sequences, many heads) runs on the band
+    kernels too: fwd and bwd of sampled slices against the oracle."""
+    w = _wl("many_slices", 2, 32800, 130, 64, "bf16", 32, range(0, 8), seed=9)[0]
+    o = oracle_lib
+    g = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+    rp, ci = o.structured(w.T, w.W, w.exps)
+    x = synth.make_qkv(w, device="cuda")
+    n0 = sa.sparse_attn_launch_count()
+    sa.sparse_attn_profile_begin(True)
+    out, lse = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+    dq, dk, dv = sa.sparse_attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], g, w.scale)
+    prof = sa.sparse_attn_profile_end()
+    sa.sparse_attn_check_device()
+    assert set(prof) == {"band_fwd", "band_bwd_dq", "band_bwd_dkdv"}, prof
+    assert sa.sparse_attn_launch_count() - n0 == 3
+    BH = w.B * w.H
+    for bh in (0, 1, 40000, BH - 1):
+        sl = [to_oracle(x[n].view(BH, w.T, w.D)[bh], w.dtype) for n in ("q", "k", "v", "dout")]
+        rout, rlse = o.fwd(sl[0], sl[1], sl[2], rp, ci, w.scale, dtype=w.dtype)
+        rdq, rdk, rdv = o.bwd(*sl, rp, ci, w.scale, dtype=w.dtype)
+        for got, ref, n in ((out, rout, "out"), (dq, rdq, "dq"), (dk, rdk, "dk"), (dv, rdv, "dv")):
+            compare(got.view(BH, w.T, w.D)[bh], ref, w.dtype, f"many_slices[{bh}] {n}")
+        compare(lse.view(BH, w.T)[bh], rlse, w.dtype, f"many_slices[{bh}] lse")

@@ -2,13 +2,16 @@
 
     python bench.py --gpus N --steps K --warmup W [--workload NAME] [--impl reference]
 
-One step = the whole hot path over one batch of synthetic input: build the
-neighbour graph, forward (out, lse) and backward (dq, dk, dv).  The default
+One step = the whole hot path over one batch of synthetic input on its fixed
+neighbour graph: forward (out, lse) and backward (dq, dk, dv).  The default
 workload is the 16,384-token layer of "SpatialLM-Mini ..." (B1 H4 T16384 D64
-bf16, window 32 + distance links 2^k, k = 0..13).  The headline value is
-query-key edges per second of fwd+bwd, summed over all ranks; every rank runs
-its own replica (the heads of a batch are independent problems: weak scaling,
-no collective on the data path).
+bf16, window 32 + distance links 2^k, k = 0..13); its structured graph is
+built once before the timed region (it has no device work: the kernels
+enumerate it from the window and the distances), and the end-to-end pass
+rebuilds it every step.  The headline value is query-key edges per second of
+fwd+bwd, summed over all ranks; every rank runs its own replica (the heads of
+a batch are independent problems: weak scaling, no collective on the data
+path).
 
 Timing: W untimed warm-up steps; then K steps, each bracketed by its own CUDA
 events on the launching stream, with a 256 MiB buffer written between steps
@@ -17,6 +20,11 @@ both sides; the max over ranks.  A second pass records per-kernel events for
 the roofline of the dominant kernel; a third measures the same step end to
 end from pinned host buffers (copies inside the timed region).  nvidia-smi
 samples the clocks during the timed region.
+
+The same line also carries, under "workloads", the other named workloads at
+a few steps each (same timing rules, own roofline and clocks): the W = 4096
+band (fwd+bwd), the graph-view CSR mask at T = 2^20 (fwd, with the timed
+CSR normalise + transpose build) and the T = 2^27 sequence (fwd).
 
 ``--impl reference`` times the CPU oracle (the plain fp64 statement of the
 method) on a bounded sample of the same workload instead.
@@ -234,7 +242,7 @@ def run_reference(args, dist, rank, world):
                        "dilation_exps": list(w.exps), "pass": "fwd+bwd",
                        "parallelism": "replicas"},
             "cpu_baseline": {"value": v, "unit": "edges/s", "cores": 1, "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, **host_info()},
             "e2e": {"value": v, "unit": "edges/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -242,39 +250,97 @@ def run_reference(args, dist, rank, world):
 
 # ------------------------------------------------------------- GPU arm
 
-def run_gpu(args, dist, rank, world):
+# Workloads timed besides the headline one (few steps each): name -> pass.
+EXTRA_WORKLOADS = ("band_32k", "csr_1m", "extreme_128m")
+
+
+def host_info():
+    """CPU model and logical core count of this host (for the CPU baseline)."""
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+def gather_model_bytes(w: synth.Workload, g, dev) -> tuple:
+    """Bytes a forward must move from HBM when the gathered rows that cannot
+    stay in L2 miss it: the compulsory bytes plus one K and one V row per such
+    edge, plus the CSR lists.  CSR workload: the edges outside the window and
+    the 16 global keys (random keys drawn from the whole history).  Structured
+    graph: the distance links o whose rows were last streamed more than an
+    L2 ago (o * 4 D es > L2 bytes).  Returns (bytes per replica, description)."""
+    es = w.elem_size
+    comp = KERNEL_BYTES["fwd"](w.T, w.D, es) * w.B * w.H
+    row2 = 2 * w.D * es
+    if w.csr:
+        rp, ci, _, _ = sa_export(g)
+        deg = rp[1:] - rp[:-1]
+        rows = torch.repeat_interleave(torch.arange(w.T, device=rp.device), deg)
+        far = (ci.long() >= 16) & (ci.long() <= rows - w.band_hint)
+        n_far = int(far.sum())
+        del rp, ci, rows, far
+        lists = 8 * (w.T + 1) + 4 * int(g.nnz)
+        return (comp + lists + row2 * n_far * w.B * w.H,
+                f"compulsory + CSR lists + {row2} B per edge outside the window and the 16 "
+                f"global keys ({n_far} per slice)")
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_far = sum(w.T - (1 << e) for e in w.exps
+                if (1 << e) >= w.W and (1 << e) < w.T and (1 << e) * 4 * w.D * es > l2)
+    return (comp + row2 * n_far * w.B * w.H,
+            f"compulsory + {row2} B per distance-link edge reaching back more than "
+            f"L2 ({l2} B) / {4 * w.D * es} B per row ({n_far} per slice)")
+
+
+def sa_export(g):
     import sparse_graph_causal_b200 as sa
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    w = synth.WORKLOADS[args.workload]
+    return sa.sparse_attn_graph_export(g)
+
+
+def time_workload(sa, w: synth.Workload, dev, rank, world, dist, steps, warmup, fwd_only,
+                  use_graph=True, want_e2e=False, args=None):
+    """Time one workload: K steps with CUDA events (L2 flushed between steps),
+    per-kernel events for the roofline, a fwd-only pass, optionally the
+    end-to-end pass.  Returns a dict of results (rank-max times)."""
     stream = torch.cuda.current_stream()
-    x = synth.make_qkv(w, device=dev, seed=w.seed + 17 * rank)
-    q, k, v, dout = x["q"], x["k"], x["v"], x["dout"]
+    x = synth.make_qkv(w, device=dev, seed=w.seed + 17 * rank, with_dout=w.bwd and not fwd_only)
+    q, k, v = x["q"], x["k"], x["v"]
+    dout = x.get("dout")
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    do_bwd = w.bwd and not fwd_only
+    dq = torch.empty_like(q) if do_bwd else None
+    dk = torch.empty_like(k) if do_bwd else None
+    dv = torch.empty_like(v) if do_bwd else None
     graph_build_ms = None
     if w.csr:
         # graph view: raw CSR rows -> normalised lists + transpose, timed alone
         rp_h, ci_h = synth.csr_random_rows(w.T, seed=w.graph_seed)
         rp_d, ci_d = torch.from_numpy(rp_h).to(dev), torch.from_numpy(ci_h).to(dev)
+        del rp_h, ci_h
         builds = []
+        g0 = None
         for _ in range(3):
+            if g0 is not None:
+                g0.close()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             g0 = sa.sparse_attn_graph_build_csr(rp_d, ci_d, band_hint=w.band_hint)
             b.record(stream)
             torch.cuda.synchronize()
             builds.append(a.elapsed_time(b))
-        graph_build_ms = min(builds)
+        graph_build_ms = max_over_ranks(dist, min(builds))
         del rp_d, ci_d
     else:
         g0 = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
-    ws = torch.empty(sa.sparse_attn_bwd_workspace_size(q, g0), dtype=torch.uint8, device=dev)
+    ws = (torch.empty(sa.sparse_attn_bwd_workspace_size(q, g0), dtype=torch.uint8, device=dev)
+          if do_bwd else None)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     E = edge_count(w, g0)
-    do_bwd = w.bwd and not args.fwd_only
 
     def eager_step():
         sa.sparse_attn_fwd(q, k, v, g0, w.scale, out=out, lse=lse)
@@ -282,18 +348,17 @@ def run_gpu(args, dist, rank, world):
             sa.sparse_attn_bwd(q, k, v, out, lse, dout, g0, w.scale, dq=dq, dk=dk, dv=dv,
                                workspace=ws)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         flush.fill_(1)
         eager_step()
     sa.sparse_attn_check_device()
     torch.cuda.synchronize()
 
-    # The timed step replays fwd + bwd captured once in a CUDA graph (the
-    # neighbour graph is fixed in advance; the structured graph is enumerated
-    # inside the kernels, so it has no device work of its own).
+    # The timed step replays fwd (+ bwd) captured once in a CUDA graph (the
+    # neighbour graph is fixed in advance and built outside the step).
     cuda_graph = None
     launches_per_step = None
-    if not args.no_graph:
+    if use_graph:
         cuda_graph = torch.cuda.CUDAGraph()
         n0 = sa.sparse_attn_launch_count()
         with torch.cuda.graph(cuda_graph):
@@ -314,9 +379,9 @@ def run_gpu(args, dist, rank, world):
 
     # ---- timed region: K steps, L2 flushed between steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+           for _ in range(steps)]
     launches0 = sa.sparse_attn_launch_count()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index or 0) as clk:
         barrier(dist)
         torch.cuda.synchronize()
         for a, b in evs:
@@ -328,24 +393,22 @@ def run_gpu(args, dist, rank, world):
         barrier(dist)
     launches = sa.sparse_attn_launch_count() - launches0
     if cuda_graph is not None:
-        launches = launches_per_step * args.steps
+        launches = launches_per_step * steps
     sa.sparse_attn_check_device()
     ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = max_over_ranks(dist, sum(ms))
-    ms_step = total_ms / args.steps
-    value = E * world / (ms_step * 1e-3)
+    ms_step = max_over_ranks(dist, sum(ms)) / steps
 
     # ---- per-kernel event timing (separate pass) for the roofline
     sa.sparse_attn_profile_begin(True)
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush.fill_(1)
         eager_step()
     prof = sa.sparse_attn_profile_end()
     kt = {n: (c, t) for n, (c, t) in prof.items() if not n.startswith("graph_")}
     dom = max(kt, key=lambda n: kt[n][1])
     cnt, tot = kt[dom]
-    avg_ms = tot / cnt
-    es = 2 if w.dtype == "bf16" else 4
+    avg_ms = max_over_ranks(dist, tot / cnt)
+    es = w.elem_size
     kc = kernel_class(dom)
     alg_bytes = KERNEL_BYTES[kc](w.T, w.D, es) * w.B * w.H
     alg_flops = KERNEL_FLOPS_PER_EDGE[kc](w.D) * E
@@ -365,80 +428,138 @@ def run_gpu(args, dist, rank, world):
                      "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
                      "kernel_shares": shares,
                      "kernel_ms_all": {n: t / c for n, (c, t) in kt.items()}})
+    if not tensor_bound and kc == "fwd" and (w.csr or any((1 << e) >= w.W for e in w.exps)):
+        mb, desc = gather_model_bytes(w, g0, dev)
+        roofline["gather_model"] = {"bytes": mb, "achieved": mb / (avg_ms * 1e-3) / 1e9,
+                                    "frac": mb / (avg_ms * 1e-3) / 1e9 / hbm, "model": desc}
 
     # ---- fwd-only throughput
-    fwd_ms = []
-    for _ in range(min(args.steps, 50)):
+    fwd_ev = []
+    for _ in range(min(steps, 50)):
         flush.fill_(1)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         sa.sparse_attn_fwd(q, k, v, g0, w.scale, out=out, lse=lse)
         b.record(stream)
-        fwd_ms.append((a, b))
+        fwd_ev.append((a, b))
     torch.cuda.synchronize()
-    fwd_ms = max_over_ranks(dist, sum(a.elapsed_time(b) for a, b in fwd_ms) / len(fwd_ms))
+    fwd_ms = max_over_ranks(dist, sum(a.elapsed_time(b) for a, b in fwd_ev) / len(fwd_ev))
 
     e2e = None
-    if not args.no_e2e:
+    if want_e2e:
         e2e = measure_e2e(sa, w, x, out, lse, dq, dk, dv, ws, g0, flush, stream, do_bwd, E,
                           world, dist, args)
+    res = {
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "W": w.W,
+                   "dilation_exps": list(w.exps), "csr": w.csr, "edges_per_replica": E,
+                   "pass": "fwd+bwd" if do_bwd else "fwd",
+                   "l2": "256 MiB buffer written between timed steps",
+                   "timed_step": ("CUDA-graph replay of " if cuda_graph is not None else
+                                  "eager ") + ("fwd+bwd" if do_bwd else "fwd"),
+                   "parallelism": f"replicas x{world}"},
+        "steps": steps, "ms_per_step": ms_step, "edges_per_s": E * world / (ms_step * 1e-3),
+        "fwd_ms": fwd_ms, "fwd_edges_per_s": E * world / (fwd_ms * 1e-3),
+        "tokens_per_s": w.B * w.T * world / (ms_step * 1e-3), "graph_build_ms": graph_build_ms,
+        "roofline": roofline, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
+    }
+    del cuda_graph
+    g0.close()
+    return res
+
+
+def run_gpu(args, dist, rank, world):
+    import sparse_graph_causal_b200 as sa
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    r = time_workload(sa, w, dev, rank, world, dist, args.steps, args.warmup, args.fwd_only,
+                      use_graph=not args.no_graph, want_e2e=not args.no_e2e, args=args)
+    torch.cuda.empty_cache()
+
+    extra = {}
+    if not args.no_extra:
+        for name in EXTRA_WORKLOADS:
+            if name == w.name:
+                continue
+            extra[name] = time_workload(sa, synth.WORKLOADS[name], dev, rank, world, dist,
+                                        args.extra_steps, 3, False)
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu and not w.csr:
         v_cpu, e_cpu, s_cpu, desc = cpu_oracle_run(w, args.cpu_seconds)
         cpu = {"value": v_cpu, "unit": "edges/s", "cores": 1, "kind": "oracle",
-               "sample": f"{desc}; {s_cpu:.1f} s"}
+               "sample": f"{desc}; {s_cpu:.1f} s", **host_info()}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "metric": METRIC, "value": r["edges_per_s"], "unit": "edges/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "W": w.W,
-                       "dilation_exps": list(w.exps), "csr": w.csr, "edges_per_replica": E,
-                       "pass": "fwd+bwd" if do_bwd else "fwd",
-                       "l2": "256 MiB buffer written between timed steps",
-                       "timed_step": "CUDA-graph replay of fwd+bwd" if cuda_graph is not None
-                       else "eager fwd+bwd calls",
-                       "parallelism": f"replicas x{world}"},
-            "fwd_edges_per_s": E * world / (fwd_ms * 1e-3), "fwd_ms": fwd_ms,
-            "tokens_per_s": w.B * w.T * world / (ms_step * 1e-3),
-            "graph_build_ms": graph_build_ms,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clk.summary(),
+            "dtype": w.dtype, "data": "synthetic", "config": r["config"],
+            "fwd_edges_per_s": r["fwd_edges_per_s"], "fwd_ms": r["fwd_ms"],
+            "tokens_per_s": r["tokens_per_s"], "graph_build_ms": r["graph_build_ms"],
+            "roofline": r["roofline"], "cpu_baseline": cpu, "e2e": r["e2e"],
+            "gpu_launches": r["gpu_launches"], "clocks": r["clocks"],
+            "workloads": extra,
         }
         print(json.dumps(line), flush=True)
-    del cuda_graph
-    g0.close()
 
 
 def measure_e2e(sa, w, x, out, lse, dq, dk, dv, ws, g0, flush, stream, do_bwd, E, world, dist,
                 args):
     """Same step through the public API from pinned host memory: H2D of the
-    inputs and D2H of the results inside the timed region."""
-    q, k, v, dout = x["q"], x["k"], x["v"], x.get("dout")
-    hx = {n: t.cpu().pin_memory() for n, t in x.items()}
-    hout = {n: torch.empty(q.shape, dtype=q.dtype).pin_memory() for n in ("out", "dq", "dk", "dv")}
-    h2d = sum(t.numel() * t.element_size() for n, t in hx.items() if do_bwd or n != "dout")
-    d2h = sum(t.numel() * t.element_size() for n, t in hout.items() if do_bwd or n == "out")
+    inputs and D2H of the results inside the timed region.  The (b, h) slices
+    are independent problems on the same graph, so the step runs slice by
+    slice on two streams: the copies of one slice overlap the kernels of the
+    next (and uploads overlap downloads), as a user streaming heads from host
+    memory would run it."""
+    BH, T, D = w.B * w.H, w.T, w.D
+    names_in = ("q", "k", "v") + (("dout",) if do_bwd else ())
+    names_out = ("out",) + (("dq", "dk", "dv") if do_bwd else ())
+    dev_out = {"out": out, "dq": dq, "dk": dk, "dv": dv}
+    hx = {n: x[n].cpu().pin_memory() for n in names_in}
+    hout = {n: torch.empty(x["q"].shape, dtype=x["q"].dtype).pin_memory() for n in names_out}
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = sum(t.numel() * t.element_size() for t in hout.values())
 
-    def e2e_step():
-        for n in ("q", "k", "v") + (("dout",) if do_bwd else ()):
-            x[n].copy_(hx[n], non_blocking=True)
+    def sl(t, c):  # slice c of a [B, H, T, D] tensor as a contiguous [1, 1, T, D] view
+        return t.view(BH, T, D)[c].view(1, 1, T, D)
+
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    ws_s = [torch.empty(sa.sparse_attn_bwd_workspace_size(sl(x["q"], 0), g0), dtype=torch.uint8,
+                        device=x["q"].device) for _ in streams] if do_bwd else [None, None]
+    lse2 = lse.view(BH, T)
+
+    def e2e_step(start):
         g = g0 if w.csr else sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
-        sa.sparse_attn_fwd(q, k, v, g, w.scale, out=out, lse=lse)
-        if do_bwd:
-            sa.sparse_attn_bwd(q, k, v, out, lse, dout, g, w.scale, dq=dq, dk=dk, dv=dv,
-                               workspace=ws)
-        hout["out"].copy_(out, non_blocking=True)
-        if do_bwd:
-            hout["dq"].copy_(dq, non_blocking=True)
-            hout["dk"].copy_(dk, non_blocking=True)
-            hout["dv"].copy_(dv, non_blocking=True)
+        for c in range(BH):
+            si = c % 2
+            s = streams[si]
+            s.wait_event(start)
+            with torch.cuda.stream(s):
+                for n in names_in:
+                    sl(x[n], c).copy_(sl(hx[n], c), non_blocking=True)
+                qc, kc, vc = sl(x["q"], c), sl(x["k"], c), sl(x["v"], c)
+                oc, lc = sl(out, c), lse2[c].view(1, 1, T)
+                sa.sparse_attn_fwd(qc, kc, vc, g, w.scale, out=oc, lse=lc, stream=s)
+                if do_bwd:
+                    sa.sparse_attn_bwd(qc, kc, vc, oc, lc, sl(x["dout"], c), g, w.scale,
+                                       dq=sl(dq, c), dk=sl(dk, c), dv=sl(dv, c),
+                                       workspace=ws_s[si], stream=s)
+                for n in names_out:
+                    sl(hout[n], c).copy_(sl(dev_out[n], c), non_blocking=True)
+        done = torch.cuda.Event()
+        for s in streams:
+            done.record(s)
+            stream.wait_event(done)
+            done = torch.cuda.Event()
 
     for _ in range(3):
-        e2e_step()
+        st = torch.cuda.Event()
+        st.record(stream)
+        e2e_step(st)
     torch.cuda.synchronize()
     e_evs = []
     n_e2e = min(args.steps, 50)
@@ -447,14 +568,16 @@ def measure_e2e(sa, w, x, out, lse, dq, dk, dv, ws, g0, flush, stream, do_bwd, E
         flush.fill_(1)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        e2e_step()
+        e2e_step(a)
         b.record(stream)
         e_evs.append((a, b))
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(dist, sum(a.elapsed_time(b) for a, b in e_evs) / n_e2e)
     return {"value": E * world / (e2e_ms * 1e-3), "unit": "edges/s", "ms_per_step": e2e_ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "graph": "built per step" if not w.csr else "CSR graph built once"}
+            "graph": "built per step" if not w.csr else "CSR graph built once",
+            "pipelining": f"{BH} slices on 2 streams (copies of one slice overlap the kernels "
+                          "of the next)"}
 
 
 def main():
@@ -469,6 +592,10 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="time eager calls, no CUDA graph")
     ap.add_argument("--no-e2e", action="store_true", help="skip the pinned-host end-to-end pass")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only --workload, not the other named workloads")
+    ap.add_argument("--extra-steps", type=int, default=5,
+                    help="timed steps of each of the other named workloads")
     args = ap.parse_args()
     dist, rank, world = dist_setup(args.gpus)
     try:

@@ -61,6 +61,15 @@ KERNEL_BYTES = {
     "bwd_dq": lambda T, D, es: 6 * T * D * es + 8 * T,
     "bwd_dkdv": lambda T, D, es: 6 * T * D * es + 8 * T,
 }
+
+
+def kernel_bytes(kc: str, w) -> int:
+    """KERNEL_BYTES over the whole job, with k, v, dk, dv on the key/value heads
+    (grouped-query attention: Hkv <= H)."""
+    B, H, Hk, T, D, es = w.B, w.H, w.kv_heads, w.T, w.D, w.elem_size
+    rows = {"fwd": (2 * H + 2 * Hk, 4 * H), "bwd_dq": (4 * H + 2 * Hk, 8 * H),
+            "bwd_dkdv": (2 * H + 4 * Hk, 8 * H)}[kc]
+    return B * T * (rows[0] * D * es + rows[1])
 # Algorithmic FLOPs per edge: forward 4D (q.k and p.v); backward 10D split as
 # dQ kernel 6D (S recompute, dP, dQ) and dK/dV kernel 4D (dV, dK); the dK/dV
 # kernel's own recomputation of S and dP is not counted.
@@ -251,7 +260,7 @@ def run_reference(args, dist, rank, world):
 # ------------------------------------------------------------- GPU arm
 
 # Workloads timed besides the headline one (few steps each): name -> pass.
-EXTRA_WORKLOADS = ("band_32k", "csr_1m", "extreme_128m")
+EXTRA_WORKLOADS = ("band_32k", "csr_1m", "extreme_128m", "gqa_16k", "dist_16k", "decode_16k")
 
 
 def host_info():
@@ -275,7 +284,7 @@ def gather_model_bytes(w: synth.Workload, g, dev) -> tuple:
     graph: the distance links o whose rows were last streamed more than an
     L2 ago (o * 4 D es > L2 bytes).  Returns (bytes per replica, description)."""
     es = w.elem_size
-    comp = KERNEL_BYTES["fwd"](w.T, w.D, es) * w.B * w.H
+    comp = kernel_bytes("fwd", w)
     row2 = 2 * w.D * es
     if w.csr:
         rp, ci, _, _ = sa_export(g)
@@ -410,7 +419,7 @@ def time_workload(sa, w: synth.Workload, dev, rank, world, dist, steps, warmup, 
     avg_ms = max_over_ranks(dist, tot / cnt)
     es = w.elem_size
     kc = kernel_class(dom)
-    alg_bytes = KERNEL_BYTES[kc](w.T, w.D, es) * w.B * w.H
+    alg_bytes = kernel_bytes(kc, w)
     alg_flops = KERNEL_FLOPS_PER_EDGE[kc](w.D) * E
     hbm, tflops, src = peaks()
     shares = {n: round(t / sum(tt for _, tt in kt.values()), 4) for n, (_, t) in kt.items()}
@@ -467,6 +476,146 @@ def time_workload(sa, w: synth.Workload, dev, rank, world, dist, steps, warmup, 
     return res
 
 
+def _timed_steps(step, steps, flush, stream, dist, dev):
+    """K steps bracketed by CUDA events, L2 flushed between steps; returns
+    (rank-max mean ms, clocks)."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    with ClockSampler(dev.index or 0) as clk:
+        barrier(dist)
+        torch.cuda.synchronize()
+        for a, b in evs:
+            flush.fill_(1)
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        barrier(dist)
+    return max_over_ranks(dist, sum(a.elapsed_time(b) for a, b in evs)) / steps, clk.summary()
+
+
+def _roofline_bytes(sa, step, steps, flush, kernel_bytes_of, dist):
+    """Per-kernel events of `steps` eager steps; the dominant kernel against
+    the measured HBM bandwidth with its compulsory bytes."""
+    sa.sparse_attn_profile_begin(True)
+    for _ in range(steps):
+        flush.fill_(1)
+        step()
+    prof = sa.sparse_attn_profile_end()
+    dom = max(prof, key=lambda n: prof[n][1])
+    cnt, tot = prof[dom]
+    avg_ms = max_over_ranks(dist, tot / cnt)
+    hbm, _, src = peaks()
+    b = kernel_bytes_of(dom)
+    achieved = b / (avg_ms * 1e-3) / 1e9
+    tot_all = sum(t for _, t in prof.values())
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "peak_source": f"{src} hbm_gbs", "traffic": None,
+            "kernel": dom, "kernel_ms": avg_ms, "algorithmic_bytes": b,
+            "kernel_shares": {n: round(t / tot_all, 4) for n, (_, t) in prof.items()},
+            "kernel_ms_all": {n: t / c for n, (c, t) in prof.items()}}
+
+
+def time_dist(sa, w, dev, rank, world, dist, steps, warmup, fwd_only, **_):
+    """Learned-coordinate scoring (s = -scale |a_i - c_j|^2) on the workload's
+    graph, fwd+bwd, CUDA-graph replay."""
+    stream = torch.cuda.current_stream()
+    x = synth.make_qkv(w, device=dev, seed=w.seed + 17 * rank)
+    v, dout = x["v"], x["dout"]
+    a_, c_ = synth.make_coords(w, device=dev, seed=w.seed + 7 + 17 * rank)
+    g0 = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+    out = torch.empty_like(v)
+    lse = torch.empty(v.shape[:3], dtype=torch.float32, device=dev)
+    da, dc, dv = torch.empty_like(a_), torch.empty_like(c_), torch.empty_like(v)
+    ws = torch.empty(sa.sparse_attn_dist_bwd_workspace_size(v, g0), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    E = edge_count(w, g0)
+
+    def eager():
+        sa.sparse_attn_dist_fwd(a_, c_, v, g0, w.scale, out=out, lse=lse)
+        sa.sparse_attn_dist_bwd(a_, c_, v, out, lse, dout, g0, w.scale, da=da, dc=dc, dv=dv,
+                                workspace=ws)
+
+    for _ in range(max(3, warmup)):
+        eager()
+    sa.sparse_attn_check_device()
+    cg = torch.cuda.CUDAGraph()
+    n0 = sa.sparse_attn_launch_count()
+    with torch.cuda.graph(cg):
+        eager()
+    per_step = sa.sparse_attn_launch_count() - n0
+    for _ in range(3):
+        cg.replay()
+    ms, clk = _timed_steps(cg.replay, steps, flush, stream, dist, dev)
+    sa.sparse_attn_check_device()
+    B, H, T, D, es = w.B, w.H, w.T, w.D, w.elem_size
+    # compulsory bytes per kernel: value rows, coordinates (12 B per row),
+    # lse / Delta (4 B per row), outputs
+    kb = {"dist_fwd": B * H * T * (2 * D * es + 24 + 4),
+          "dist_bwd_da": B * H * T * (3 * D * es + 24 + 12 + 8),
+          "dist_bwd_dcdv": B * H * T * (3 * D * es + 24 + 12 + 8)}
+    roof = _roofline_bytes(sa, eager, steps, flush, lambda n: kb[n], dist)
+    del cg
+    g0.close()
+    return {"config": {"workload": w.name, "B": B, "H": H, "T": T, "D": D, "W": w.W,
+                       "dilation_exps": list(w.exps), "scale": w.scale, "pass": "fwd+bwd",
+                       "score": "-scale |a_i - c_j|^2, 3-D coordinates",
+                       "l2": "256 MiB buffer written between timed steps",
+                       "timed_step": "CUDA-graph replay of fwd+bwd",
+                       "parallelism": f"replicas x{world}"},
+            "steps": steps, "ms_per_step": ms, "edges_per_s": E * world / (ms * 1e-3),
+            "tokens_per_s": B * T * world / (ms * 1e-3), "roofline": roof,
+            "gpu_launches": per_step * steps, "clocks": clk}
+
+
+def time_decode(sa, w, dev, rank, world, dist, steps, warmup, fwd_only, **_):
+    """One new token per sequence (B sequences, H query heads over Hkv cache
+    heads, caches of T rows) at positions drawn in [T/2, T)."""
+    stream = torch.cuda.current_stream()
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 17 * rank)
+    B, H, Hk, T, D = w.B, w.H, w.kv_heads, w.T, w.D
+    q = torch.empty((B, H, 1, D), dtype=torch.float32, device=dev).normal_(
+        generator=g).to(w.torch_dtype)
+    kc = torch.empty((B, Hk, T, D), dtype=torch.float32, device=dev).normal_(
+        generator=g).to(w.torch_dtype)
+    vc = torch.empty((B, Hk, T, D), dtype=torch.float32, device=dev).normal_(
+        generator=g).to(w.torch_dtype)
+    pos = torch.randint(T // 2, T, (B,), generator=g, device=dev, dtype=torch.int64)
+    g0 = sa.sparse_attn_graph_build_structured(T, w.W, list(w.exps))
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def eager():
+        sa.sparse_attn_decode(q, kc, vc, pos, g0, w.scale, out=out, lse=lse)
+
+    for _ in range(max(3, warmup)):
+        eager()
+    sa.sparse_attn_check_device()
+    ms, clk = _timed_steps(eager, steps, flush, stream, dist, dev)
+    sa.sparse_attn_check_device()
+    # neighbours per query: min(p + 1, W) + #{2^k : W <= 2^k <= p}
+    ps = pos.cpu().tolist()
+    offs = sorted({1 << e for e in w.exps if (1 << e) >= w.W})
+    deg = [min(p + 1, w.W) + sum(1 for o in offs if o <= p) for p in ps]
+    edges = sum(deg) * H
+    es = w.elem_size
+    # compulsory bytes: q and out rows, lse, one K and one V row per edge of
+    # each query head (rows shared by the heads of a group are counted once)
+    bytes_ = B * H * (2 * D * es + 4) + sum(deg) * Hk * 2 * D * es
+    roof = _roofline_bytes(sa, eager, steps, flush, lambda n: bytes_, dist)
+    g0.close()
+    return {"config": {"workload": w.name, "B": B, "H": H, "Hkv": Hk, "T_cache": T, "D": D,
+                       "W": w.W, "dilation_exps": list(w.exps), "positions": "uniform in [T/2, T)",
+                       "pass": "decode (one query per sequence and head)",
+                       "l2": "256 MiB buffer written between timed steps",
+                       "parallelism": f"replicas x{world}"},
+            "steps": steps, "ms_per_step": ms, "edges_per_s": edges * world / (ms * 1e-3),
+            "queries_per_s": B * H * world / (ms * 1e-3), "roofline": roof,
+            "gpu_launches": steps, "clocks": clk}
+
+
 def run_gpu(args, dist, rank, world):
     import sparse_graph_causal_b200 as sa
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -482,8 +631,9 @@ def run_gpu(args, dist, rank, world):
         for name in EXTRA_WORKLOADS:
             if name == w.name:
                 continue
-            extra[name] = time_workload(sa, synth.WORKLOADS[name], dev, rank, world, dist,
-                                        args.extra_steps, 3, False)
+            wx = synth.WORKLOADS[name]
+            timer = {"attn": time_workload, "dist": time_dist, "decode": time_decode}[wx.kind]
+            extra[name] = timer(sa, wx, dev, rank, world, dist, args.extra_steps, 3, False)
             torch.cuda.empty_cache()
 
     cpu = None

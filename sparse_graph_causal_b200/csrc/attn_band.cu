@@ -228,6 +228,11 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // the set-up above overlaps the previous kernel's last tiles; its results
+    // (the forward's out and lse, the dQ pass's Delta) are read only after
+    // this point, and the next kernel may be scheduled from here on
+    tc::wait_prior_grid();
+    tc::allow_dependents();
 
     if (warp < 4) {
         // one register budget per warpgroup, set where it dominates the roles
@@ -838,9 +843,10 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     int sms = 0;
     SA_CUDA_TRY(sa_sm_count(&sms));
     const unsigned grid = (unsigned)(nctas < sms ? nctas : sms);
+    cudaError_t le = cudaSuccess;
     SA_LAUNCH("band_fwd", s,
-              kern<<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, mkd, mvd, a));
-    SA_CUDA_TRY(cudaGetLastError());
+              le = sa_launch_pdl(kern, grid, kThreads, L::kAlloc, s, mq, mk, mv, mkd, mvd, a));
+    SA_CUDA_TRY(le);
     return SA_OK;
 }
 

@@ -392,6 +392,11 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // the set-up above overlaps the previous kernel's last tiles; its results
+    // (the forward's out and lse, the dQ pass's Delta) are read only after
+    // this point, and the next kernel may be scheduled from here on
+    tc::wait_prior_grid();
+    tc::allow_dependents();
 
     if (warp < 4) {
         if (NP == 2) tc::regs_dec<BwdRegs::producer>();
@@ -916,6 +921,11 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // the set-up above overlaps the previous kernel's last tiles; its results
+    // (the forward's out and lse, the dQ pass's Delta) are read only after
+    // this point, and the next kernel may be scheduled from here on
+    tc::wait_prior_grid();
+    tc::allow_dependents();
 
     if (warp < 4) {
         if (NP == 2) tc::regs_dec<BwdRegs::producer>();
@@ -1471,11 +1481,15 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
         const int64_t nctas = (((T + BM - 1) / BM) * slices + NP - 1) / NP;
         return (unsigned)(nctas < sms ? nctas : sms);
     };
+    cudaError_t le = cudaSuccess;
     SA_LAUNCH("band_bwd_dq", s,
-              kq<<<grid_for(BH), kThreads, LQ::kAlloc, s>>>(mq, mdo, mkb, mvb, mk, mv, a));
+              le = sa_launch_pdl(kq, grid_for(BH), kThreads, LQ::kAlloc, s, mq, mdo, mkb, mvb, mk,
+                                 mv, a));
+    SA_CUDA_TRY(le);
     SA_LAUNCH("band_bwd_dkdv", s,
-              kkv<<<grid_for(BHkv), kThreads, LK::kAlloc, s>>>(mk, mv, mqb, mdob, mq, mdo, a));
-    SA_CUDA_TRY(cudaGetLastError());
+              le = sa_launch_pdl(kkv, grid_for(BHkv), kThreads, LK::kAlloc, s, mk, mv, mqb, mdob,
+                                 mq, mdo, a));
+    SA_CUDA_TRY(le);
     return SA_OK;
 }
 

@@ -38,6 +38,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
+// Programmatic dependent launch: a grid launched with programmatic stream
+// serialization may start while the previous kernel in the stream drains;
+// wait_prior_grid() blocks until that kernel has completed and its memory is
+// visible (a no-op for a normally launched grid), and allow_dependents()
+// lets the next such grid be scheduled once every CTA of this one has issued
+// it (or exited).
+__device__ __forceinline__ void wait_prior_grid() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

@@ -49,6 +49,12 @@ class Workload:
     seed: int = 0
     graph_seed: int = 0
     bwd: bool = True
+    Hkv: int = 0          # key/value heads (grouped-query attention); 0: H
+    kind: str = "attn"    # "attn", "dist" (learned coordinates) or "decode"
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv or self.H
 
     @property
     def torch_dtype(self):
@@ -81,12 +87,24 @@ WORKLOADS = {
     # a 1/16-length version of extreme_128m: the size used for profiler captures
     "extreme_8m": _w("extreme_8m", 1, 1, 1 << 23, 64, "bf16", 32, range(0, 23), seed=1005,
                      bwd=False),
+    # the 16K layer with grouped-query attention: 8 query heads over 2 key/value heads
+    "gqa_16k": _w("gqa_16k", 1, 8, 16384, 64, "bf16", 32, range(0, 14), std=1.0 / math.sqrt(64),
+                  seed=1006, Hkv=2),
+    # the 16K layer with learned-coordinate weights (coordinates N(0,1), scale 0.5)
+    "dist_16k": Workload(name="dist_16k", B=1, H=4, T=16384, D=64, dtype="bf16", W=32,
+                         exps=tuple(range(0, 14)), input_std=1.0, scale=0.5, seed=1007,
+                         kind="dist"),
+    # decode: one new token per sequence for 64 sequences against 16K caches
+    # (8 query heads over 2 cache heads), positions drawn in [T/2, T)
+    "decode_16k": _w("decode_16k", 64, 8, 16384, 64, "bf16", 32, range(0, 14), seed=1008,
+                     Hkv=2, kind="decode", bwd=False),
 }
 
 
 def make_qkv(w: Workload, device="cpu", seed: int | None = None, with_dout: bool = True,
              std: float | None = None):
-    """q, k, v (and dout) of shape [B, H, T, D], contiguous, N(0, std^2), drawn
+    """q, k, v (and dout) of shape [B, H, T, D] (k and v: [B, Hkv, T, D]),
+    contiguous, N(0, std^2), drawn
     on ``device`` from a torch.Generator seeded with ``seed`` (default: the
     workload's).  Values are drawn in fp32 and rounded to the workload dtype."""
     seed = w.seed if seed is None else seed
@@ -94,10 +112,10 @@ def make_qkv(w: Workload, device="cpu", seed: int | None = None, with_dout: bool
     dev = torch.device(device)
     g = torch.Generator(device=dev)
     g.manual_seed(seed)
-    shape = (w.B, w.H, w.T, w.D)
     names = ["q", "k", "v"] + (["dout"] if with_dout else [])
     out = {}
     for n in names:
+        shape = (w.B, w.kv_heads if n in ("k", "v") else w.H, w.T, w.D)
         t = torch.empty(shape, dtype=w.torch_dtype, device=dev)
         if w.torch_dtype == torch.float32:
             t.normal_(0.0, 1.0, generator=g)

@@ -177,11 +177,13 @@ __device__ __forceinline__ void axpy_bf_smem(float *acc, float a, const uint8_t 
     }
 }
 
-// TMEM row (D fp32 columns) += bf16(a) * (row r of a tile), 32 columns at a
-// time (for D = 128, whose two accumulators do not fit in registers).
+// TMEM row (D fp32 columns) += bf16(a) * (row r of a tile) where `on`, 32
+// columns at a time (for D = 128, whose two accumulators do not fit in
+// registers).  Every lane of the warp must call it (the TMEM loads and stores
+// are warp-collective); a lane with on == false stores its row back unchanged.
 template <int D>
-__device__ __forceinline__ void tmem_axpy_row(uint32_t taddr, float a, const uint8_t *tile,
-                                              int rows, int r) {
+__device__ __forceinline__ void tmem_axpy_row(uint32_t taddr, float a, bool on,
+                                              const uint8_t *tile, int rows, int r) {
     const uint32_t a2 = tc::pack_bf16x2(a, a);
 #pragma unroll
     for (int c0 = 0; c0 < D; c0 += 32) {
@@ -195,8 +197,10 @@ __device__ __forceinline__ void tmem_axpy_row(uint32_t taddr, float a, const uin
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int x = 8 * c - c0 + 2 * e;
-                w[x] = __float_as_uint(tc::fma_bf_lo(a2, yb[e], __uint_as_float(w[x])));
-                w[x + 1] = __float_as_uint(tc::fma_bf_hi(a2, yb[e], __uint_as_float(w[x + 1])));
+                const float lo = tc::fma_bf_lo(a2, yb[e], __uint_as_float(w[x]));
+                const float hi = tc::fma_bf_hi(a2, yb[e], __uint_as_float(w[x + 1]));
+                w[x] = on ? __float_as_uint(lo) : w[x];
+                w[x + 1] = on ? __float_as_uint(hi) : w[x + 1];
             }
         }
         tc::tmem_st32(taddr + c0, w);
@@ -657,23 +661,25 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                 if constexpr (D == 64) load_row_packed<D>(pm + L::pQ, BM, r, qw);
                 auto body = [&](int d, int st) {
                     const bool valid = LDW ? (d < resid) : (row_ok && i >= a.offs[dfirst + d]);
-                    if (!valid) return;
                     const uint8_t *kt = pm + L::pDK + st * L::kRow;
                     const uint8_t *vt = pm + L::pDV + st * L::kRow;
-                    float qk;
-                    if constexpr (D == 64)
-                        qk = dot_bf_reg_smem<D>(qw, kt, BM, r);
-                    else
-                        qk = dot_bf_smem_smem<D>(pm + L::pQ, kt, BM, r);
-                    const float pr = tc::ex2(fmaf(qk, c2, -lse2));
-                    const float ds = pr * (dot_bf_smem_smem<D>(pm + L::pDO, vt, BM, r) - Delta);
-                    if (a.pds)
-                        a.pds[((size_t)(dfirst + d) * (size_t)a.BH + (size_t)bh) * (size_t)T +
-                              (size_t)i] = make_float2(pr, ds);
-                    if constexpr (kRegAcc)
-                        axpy_bf_smem<D>(acc, ds, kt, BM, r);
-                    else
-                        tmem_axpy_row<D>(tDQ, ds, kt, BM, r);
+                    float ds = 0.f;
+                    if (valid) {
+                        float qk;
+                        if constexpr (D == 64)
+                            qk = dot_bf_reg_smem<D>(qw, kt, BM, r);
+                        else
+                            qk = dot_bf_smem_smem<D>(pm + L::pQ, kt, BM, r);
+                        const float pr = tc::ex2(fmaf(qk, c2, -lse2));
+                        ds = pr * (dot_bf_smem_smem<D>(pm + L::pDO, vt, BM, r) - Delta);
+                        if (a.pds)
+                            a.pds[((size_t)(dfirst + d) * (size_t)a.BH + (size_t)bh) *
+                                      (size_t)T +
+                                  (size_t)i] = make_float2(pr, ds);
+                        if constexpr (kRegAcc) axpy_bf_smem<D>(acc, ds, kt, BM, r);
+                    }
+                    // (warp-collective: every lane, whether or not its row has the slot)
+                    if constexpr (!kRegAcc) tmem_axpy_row<D>(tDQ, ds, valid, kt, BM, r);
                 };
                 if constexpr (LDW) {
                     rows::warp_slots<D, DS>(
@@ -1232,10 +1238,10 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                 auto body = [&](int d, int st) {
                     const int64_t i_n2 = key_of(d + 2);
                     const float2 v_nxt = edge_vals(d + 1, i_nxt);
+                    const uint8_t *qt = pm + L::pDQ + st * L::kRow;
+                    const uint8_t *dt = pm + L::pDDO + st * L::kRow;
+                    float pr = 0.f, ds = 0.f;
                     if (i_cur >= 0) {
-                        const uint8_t *qt = pm + L::pDQ + st * L::kRow;
-                        const uint8_t *dt = pm + L::pDDO + st * L::kRow;
-                        float pr, ds;
                         if (cached) {
                             pr = v_cur.x;
                             ds = v_cur.y;
@@ -1248,10 +1254,12 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                         if constexpr (kRegAcc) {
                             axpy_bf_smem<D>(adv, pr, dt, BM, r);
                             axpy_bf_smem<D>(adk, ds, qt, BM, r);
-                        } else {
-                            tmem_axpy_row<D>(tDV, pr, dt, BM, r);
-                            tmem_axpy_row<D>(tDK, ds, qt, BM, r);
                         }
+                    }
+                    // (warp-collective: every lane, whether or not its key has the slot)
+                    if constexpr (!kRegAcc) {
+                        tmem_axpy_row<D>(tDV, pr, i_cur >= 0, dt, BM, r);
+                        tmem_axpy_row<D>(tDK, ds, i_cur >= 0, qt, BM, r);
                     }
                     i_cur = i_nxt;
                     i_nxt = i_n2;

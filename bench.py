@@ -662,9 +662,9 @@ def measure_e2e(sa, w, x, out, lse, dq, dk, dv, ws, g0, flush, stream, do_bwd, E
     """Same step through the public API from pinned host memory: H2D of the
     inputs and D2H of the results inside the timed region.  The (b, h) slices
     are independent problems on the same graph, so the step runs slice by
-    slice on two streams: the copies of one slice overlap the kernels of the
-    next (and uploads overlap downloads), as a user streaming heads from host
-    memory would run it."""
+    slice through an upload, a kernel and a download stream: the copies of
+    one slice overlap the kernels of another (and uploads overlap downloads),
+    as a user streaming heads from host memory would run it."""
     BH, T, D = w.B * w.H, w.T, w.D
     names_in = ("q", "k", "v") + (("dout",) if do_bwd else ())
     names_out = ("out",) + (("dq", "dk", "dv") if do_bwd else ())
@@ -677,34 +677,43 @@ def measure_e2e(sa, w, x, out, lse, dq, dk, dv, ws, g0, flush, stream, do_bwd, E
     def sl(t, c):  # slice c of a [B, H, T, D] tensor as a contiguous [1, 1, T, D] view
         return t.view(BH, T, D)[c].view(1, 1, T, D)
 
-    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
-    ws_s = [torch.empty(sa.sparse_attn_bwd_workspace_size(sl(x["q"], 0), g0), dtype=torch.uint8,
-                        device=x["q"].device) for _ in streams] if do_bwd else [None, None]
+    # three streams: uploads, kernels, downloads; slice c's kernels wait for
+    # its upload and its download for its kernels, so the copy engines stream
+    # continuously in both directions while the kernels run in between
+    up, comp, down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ws_c = (torch.empty(sa.sparse_attn_bwd_workspace_size(sl(x["q"], 0), g0), dtype=torch.uint8,
+                        device=x["q"].device) if do_bwd else None)
     lse2 = lse.view(BH, T)
 
     def e2e_step(start):
         g = g0 if w.csr else sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+        for s_ in (up, comp, down):
+            s_.wait_event(start)
         for c in range(BH):
-            si = c % 2
-            s = streams[si]
-            s.wait_event(start)
-            with torch.cuda.stream(s):
+            with torch.cuda.stream(up):
                 for n in names_in:
                     sl(x[n], c).copy_(sl(hx[n], c), non_blocking=True)
+                uploaded = torch.cuda.Event()
+                uploaded.record(up)
+            comp.wait_event(uploaded)
+            with torch.cuda.stream(comp):
                 qc, kc, vc = sl(x["q"], c), sl(x["k"], c), sl(x["v"], c)
                 oc, lc = sl(out, c), lse2[c].view(1, 1, T)
-                sa.sparse_attn_fwd(qc, kc, vc, g, w.scale, out=oc, lse=lc, stream=s)
+                sa.sparse_attn_fwd(qc, kc, vc, g, w.scale, out=oc, lse=lc, stream=comp)
                 if do_bwd:
                     sa.sparse_attn_bwd(qc, kc, vc, oc, lc, sl(x["dout"], c), g, w.scale,
-                                       dq=sl(dq, c), dk=sl(dk, c), dv=sl(dv, c),
-                                       workspace=ws_s[si], stream=s)
+                                       dq=sl(dq, c), dk=sl(dk, c), dv=sl(dv, c), workspace=ws_c,
+                                       stream=comp)
+                computed = torch.cuda.Event()
+                computed.record(comp)
+            down.wait_event(computed)
+            with torch.cuda.stream(down):
                 for n in names_out:
                     sl(hout[n], c).copy_(sl(dev_out[n], c), non_blocking=True)
-        done = torch.cuda.Event()
-        for s in streams:
-            done.record(s)
-            stream.wait_event(done)
+        for s_ in (up, comp, down):
             done = torch.cuda.Event()
+            done.record(s_)
+            stream.wait_event(done)
 
     for _ in range(3):
         st = torch.cuda.Event()
@@ -726,8 +735,8 @@ def measure_e2e(sa, w, x, out, lse, dq, dk, dv, ws, g0, flush, stream, do_bwd, E
     return {"value": E * world / (e2e_ms * 1e-3), "unit": "edges/s", "ms_per_step": e2e_ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "graph": "built per step" if not w.csr else "CSR graph built once",
-            "pipelining": f"{BH} slices on 2 streams (copies of one slice overlap the kernels "
-                          "of the next)"}
+            "pipelining": f"{BH} slices through upload, kernel and download streams (the "
+                          "copies of one slice overlap the kernels of another)"}
 
 
 def main():

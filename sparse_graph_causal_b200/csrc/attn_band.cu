@@ -228,11 +228,6 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // the set-up above overlaps the previous kernel's last tiles; its results
-    // (the forward's out and lse, the dQ pass's Delta) are read only after
-    // this point, and the next kernel may be scheduled from here on
-    tc::wait_prior_grid();
-    tc::allow_dependents();
 
     if (warp < 4) {
         // one register budget per warpgroup, set where it dominates the roles
@@ -603,31 +598,28 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 const bool pre = bl < g.npre;
                 const bool need_mask = pre || a.nf > 0 || (u0 < BM - 1) ||
                                        (u0 + BN - 1 > We - 1) || (u0 + q0 < We - 1);
-                int c_lo = 0, c_hi = BN - 1;
-                int fc[kMaxFold];  // folded-link column of this row in the block, -1 if none
-#pragma unroll
-                for (int x = 0; x < kMaxFold; ++x) fc[x] = -1;
-                bool fany = false;
+                uint64_t keep = ~0ull;  // bit c: this row keeps column c of the block
                 if (pre) {
                     // shared prefix: keys 0 .. min(gp, i - W + 1) - 1
                     const int32_t n = i - W + 1 < a.gp ? i - W + 1 : a.gp;
-                    c_hi = n > 0 ? n - 1 : -1;
+                    keep = tc::bits_range(0, n - 1);
                 } else if (need_mask) {
                     const int32_t kmin = We - 1 - q0;  // u of key 0
                     const int32_t lo = (r + We - W > kmin) ? r + We - W : kmin;
                     const int32_t hi = r + We - 1;
-                    c_lo = lo - u0 < 0 ? 0 : (lo - u0 > BN ? BN : lo - u0);
-                    c_hi = hi - u0 > BN - 1 ? BN - 1 : (hi - u0 < -1 ? -1 : hi - u0);
+                    const int c_lo = lo - u0 < 0 ? 0 : (lo - u0 > BN ? BN : lo - u0);
+                    const int c_hi = hi - u0 > BN - 1 ? BN - 1 : (hi - u0 < -1 ? -1 : hi - u0);
+                    keep = tc::bits_range(c_lo, c_hi);
+                    if (a.nf > 0) {
 #pragma unroll
-                    for (int x = 0; x < kMaxFold; ++x) {
-                        const int32_t u = r + We - 1 - a.fold[x];
-                        if (x < a.nf && u >= kmin && u >= u0 && u < u0 + BN) {
-                            fc[x] = u - u0;
-                            fany = true;
+                        for (int x = 0; x < kMaxFold; ++x) {
+                            const int32_t u = r + We - 1 - a.fold[x];
+                            if (x < a.nf && u >= kmin && u >= u0 && u < u0 + BN)
+                                keep |= 1ull << (u - u0);
                         }
                     }
                 }
-                if (need_mask && __all_sync(0xffffffffu, c_lo > c_hi && !fany)) {
+                if (need_mask && __all_sync(0xffffffffu, keep == 0ull)) {
                     // no row of this warp keeps a key of the block: P = 0
                     uint32_t z[BN / 2];
 #pragma unroll
@@ -648,12 +640,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 const float ext = pos ? -INFINITY : INFINITY;
                 if (need_mask) {
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) {
-                        bool keep = c >= c_lo && c <= c_hi;
-#pragma unroll
-                        for (int x = 0; x < kMaxFold; ++x) keep |= (c == fc[x]);
-                        s[c] = keep ? s[c] : ext;
-                    }
+                    for (int c = 0; c < BN; ++c) s[c] = ((keep >> c) & 1ull) ? s[c] : ext;
                 }
                 float mr[8];
 #pragma unroll
@@ -843,10 +830,9 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     int sms = 0;
     SA_CUDA_TRY(sa_sm_count(&sms));
     const unsigned grid = (unsigned)(nctas < sms ? nctas : sms);
-    cudaError_t le = cudaSuccess;
     SA_LAUNCH("band_fwd", s,
-              le = sa_launch_pdl(kern, grid, kThreads, L::kAlloc, s, mq, mk, mv, mkd, mvd, a));
-    SA_CUDA_TRY(le);
+              kern<<<grid, kThreads, L::kAlloc, s>>>(mq, mk, mv, mkd, mvd, a));
+    SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
 

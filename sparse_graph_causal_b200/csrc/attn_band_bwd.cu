@@ -396,11 +396,6 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // the set-up above overlaps the previous kernel's last tiles; its results
-    // (the forward's out and lse, the dQ pass's Delta) are read only after
-    // this point, and the next kernel may be scheduled from here on
-    tc::wait_prior_grid();
-    tc::allow_dependents();
 
     if (warp < 4) {
         if (NP == 2) tc::regs_dec<BwdRegs::producer>();
@@ -742,25 +737,23 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                     const int32_t hi = r + We - 1;
                     const int c_lo = lo - u0 < 0 ? 0 : (lo - u0 > BB ? BB : lo - u0);
                     const int c_hi = hi - u0 > BB - 1 ? BB - 1 : (hi - u0 < -1 ? -1 : hi - u0);
-                    int fc[kMaxFold];
+                    uint64_t keep = tc::bits_range(c_lo, c_hi);  // bit c: column c kept
+                    if (a.nf > 0) {
 #pragma unroll
-                    for (int x = 0; x < kMaxFold; ++x) {
-                        const int32_t u = r + We - 1 - a.fold[x];
-                        fc[x] = (x < a.nf && u >= kmin && u >= u0 && u < u0 + BB) ? u - u0 : -1;
+                        for (int x = 0; x < kMaxFold; ++x) {
+                            const int32_t u = r + We - 1 - a.fold[x];
+                            if (x < a.nf && u >= kmin && u >= u0 && u < u0 + BB)
+                                keep |= 1ull << (u - u0);
+                        }
                     }
                     // 16-column chunks outside every kept range of this warp: dS = 0
 #pragma unroll
                     for (int c16 = 0; c16 < BB / 16; ++c16) {
-                        bool live = c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16;
-#pragma unroll
-                        for (int x = 0; x < kMaxFold; ++x) live |= (fc[x] >> 4) == c16;
-                        if (__any_sync(0xffffffffu, live)) {
+                        if (__any_sync(0xffffffffu, ((keep >> (16 * c16)) & 0xffffull) != 0ull)) {
 #pragma unroll
                             for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
-                                bool keep = c >= c_lo && c <= c_hi;
-#pragma unroll
-                                for (int x = 0; x < kMaxFold; ++x) keep |= (c == fc[x]);
-                                const float pr = keep ? tc::ex2(fmaf(s[c], c2, -lse2)) : 0.f;
+                                const float pr =
+                                    ((keep >> c) & 1ull) ? tc::ex2(fmaf(s[c], c2, -lse2)) : 0.f;
                                 s[c] = pr * (dp[c] - Delta);
                             }
                         } else {
@@ -927,11 +920,6 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // the set-up above overlaps the previous kernel's last tiles; its results
-    // (the forward's out and lse, the dQ pass's Delta) are read only after
-    // this point, and the next kernel may be scheduled from here on
-    tc::wait_prior_grid();
-    tc::allow_dependents();
 
     if (warp < 4) {
         if (NP == 2) tc::regs_dec<BwdRegs::producer>();
@@ -1214,9 +1202,13 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                 // slot d: link (or residual position) d % nd of query head
                 // d / nd; its query row, -1 if none
                 const int nds = GQ * nd;
+                // slot d -> (query head d / nd, link d % nd); no division
+                // without grouped heads
+                auto link_of = [&](int d) { return GQ == 1 ? d : d % nd; };
+                auto head_of = [&](int d) { return GQ == 1 ? 0 : d / nd; };
                 auto key_of = [&](int d) -> int32_t {
                     if (!row_ok || d >= nds) return -1;
-                    const int dd = d % nd;
+                    const int dd = link_of(d);
                     if constexpr (!LDW) {
                         const int64_t cand = j + a.offs[off_first + dd];
                         return cand < T ? (int32_t)cand : -1;
@@ -1226,9 +1218,9 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                 const bool cached = a.kind == 0 && a.pds != nullptr;
                 auto edge_vals = [&](int d, int64_t i) -> float2 {
                     if (i < 0) return make_float2(0.f, 0.f);
-                    const size_t qbh = (size_t)(qbh0 + d / nd);
+                    const size_t qbh = (size_t)(qbh0 + head_of(d));
                     if (cached)
-                        return a.pds[((size_t)(off_first + d % nd) * (size_t)a.BH + qbh) *
+                        return a.pds[((size_t)(off_first + link_of(d)) * (size_t)a.BH + qbh) *
                                          (size_t)T +
                                      (size_t)i];
                     return make_float2(a.lse[qbh * (size_t)T + i], a.delta[qbh * (size_t)T + i]);
@@ -1271,7 +1263,7 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                         sbase + (uint32_t)(p * L::kPipe + L::pDDO), (uint32_t)L::kRow, a.q,
                         a.dout, a.l2pf != 0, lane, wq,
                         [&](int d) {
-                            return (size_t)(qbh0 + d / (nd > 0 ? nd : 1)) * (size_t)T * D;
+                            return (size_t)(qbh0 + (nd > 0 ? head_of(d) : 0)) * (size_t)T * D;
                         },
                         key_of, body);
                 } else {
@@ -1306,7 +1298,7 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             uint32_t gb_last = gb;
             for (int bl = 0; ok && bl < NB; ++bl, ++gb) {
                 const int sb = (int)(gb % SB), st = (int)(gb % BS);
-                const int32_t v0 = (bl % n_band) * BB;
+                const int32_t v0 = (GQ == 1 ? bl : bl % n_band) * BB;
                 gb_last = gb;
                 if (!wait(p, L::bSFull + sb, (gb / SB) & 1) ||
                     !wait(p, L::bBFull + st, (gb / BS) & 1)) {  // lse / Delta staged
@@ -1336,26 +1328,23 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                     const int c_lo = (int)(lo - v0 < 0 ? 0 : (lo - v0 > BB ? BB : lo - v0));
                     const int c_hi =
                         (int)(hi - v0 > BB - 1 ? BB - 1 : (hi - v0 < -1 ? -1 : hi - v0));
-                    int fc[kMaxFold];
+                    uint64_t keep = tc::bits_range(c_lo, c_hi);  // bit c: column c kept
+                    if (a.nf > 0) {
 #pragma unroll
-                    for (int x = 0; x < kMaxFold; ++x) {
-                        const int64_t v = (int64_t)r + a.fold[x];
-                        fc[x] = (x < a.nf && v <= vlim && v >= v0 && v < v0 + BB) ? (int)(v - v0)
-                                                                                     : -1;
+                        for (int x = 0; x < kMaxFold; ++x) {
+                            const int64_t v = (int64_t)r + a.fold[x];
+                            if (x < a.nf && v <= vlim && v >= v0 && v < v0 + BB)
+                                keep |= 1ull << (int)(v - v0);
+                        }
                     }
                     // 16-column chunks outside every kept range of this warp: P = dS = 0
 #pragma unroll
                     for (int c16 = 0; c16 < BB / 16; ++c16) {
-                        bool live = c_lo <= 16 * c16 + 15 && c_hi >= 16 * c16;
-#pragma unroll
-                        for (int x = 0; x < kMaxFold; ++x) live |= (fc[x] >> 4) == c16;
-                        if (__any_sync(0xffffffffu, live)) {
+                        if (__any_sync(0xffffffffu, ((keep >> (16 * c16)) & 0xffffull) != 0ull)) {
 #pragma unroll
                             for (int c = 16 * c16; c < 16 * c16 + 16; ++c) {
-                                bool keep = c >= c_lo && c <= c_hi;
-#pragma unroll
-                                for (int x = 0; x < kMaxFold; ++x) keep |= (c == fc[x]);
-                                const float pr = keep ? tc::ex2(fmaf(s[c], c2, -lse_s[c])) : 0.f;
+                                const float pr =
+                                    ((keep >> c) & 1ull) ? tc::ex2(fmaf(s[c], c2, -lse_s[c])) : 0.f;
                                 s[c] = pr;
                                 dp[c] = pr * (dp[c] - del_s[c]);
                             }
@@ -1489,15 +1478,11 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
         const int64_t nctas = (((T + BM - 1) / BM) * slices + NP - 1) / NP;
         return (unsigned)(nctas < sms ? nctas : sms);
     };
-    cudaError_t le = cudaSuccess;
     SA_LAUNCH("band_bwd_dq", s,
-              le = sa_launch_pdl(kq, grid_for(BH), kThreads, LQ::kAlloc, s, mq, mdo, mkb, mvb, mk,
-                                 mv, a));
-    SA_CUDA_TRY(le);
+              kq<<<grid_for(BH), kThreads, LQ::kAlloc, s>>>(mq, mdo, mkb, mvb, mk, mv, a));
     SA_LAUNCH("band_bwd_dkdv", s,
-              le = sa_launch_pdl(kkv, grid_for(BHkv), kThreads, LK::kAlloc, s, mk, mv, mqb, mdob,
-                                 mq, mdo, a));
-    SA_CUDA_TRY(le);
+              kkv<<<grid_for(BHkv), kThreads, LK::kAlloc, s>>>(mk, mv, mqb, mdob, mq, mdo, a));
+    SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
 

@@ -57,25 +57,6 @@ void sa_prof_end(cudaStream_t s);
     } while (0)
 int *sa_device_error_word();  // device address of this device's error word
 
-// Launch with programmatic stream serialization: the kernel may be scheduled
-// while the previous kernel of the stream drains, and must call
-// griddepcontrol.wait (tc::wait_prior_grid) before it touches memory that
-// kernel writes or reads.
-template <typename... KArgs, typename... Args>
-cudaError_t sa_launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
-                          cudaStream_t s, Args &&...args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
-}
 
 #define SA_DEVERR_TIMEOUT 1
 #define SA_DEVERR_BOUNDS 2

@@ -38,19 +38,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
-// Programmatic dependent launch: a grid launched with programmatic stream
-// serialization may start while the previous kernel in the stream drains;
-// wait_prior_grid() blocks until that kernel has completed and its memory is
-// visible (a no-op for a normally launched grid), and allow_dependents()
-// lets the next such grid be scheduled once every CTA of this one has issued
-// it (or exited).
-__device__ __forceinline__ void wait_prior_grid() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void allow_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // ------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -338,6 +325,11 @@ __device__ __forceinline__ void regs_dec() {
 template <uint32_t N>
 __device__ __forceinline__ void regs_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Bits lo .. hi of a 64-bit word (0 when hi < lo); needs lo >= 0, hi <= 63.
+__device__ __forceinline__ uint64_t bits_range(int lo, int hi) {
+    return hi < lo ? 0ull : (~0ull >> (63 - hi)) & (~0ull << lo);
 }
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128B-swizzled

@@ -18,6 +18,8 @@ Workloads (shapes from the pages' own experiments, values synthetic):
   csr_1m        B1 H8 T2^20 D64 bf16, raw CSR rows: window 64 + 16 uniform
                 draws from [0, i) + the first 16 tokens (graph view of
                 "Longer Attention Span ...")
+  csr_256k      B1 H4 T2^18 D64 bf16, the same rows (profiler-capture size of
+                csr_1m: K and V still 256 MB, beyond L2)
   extreme_128m  B1 H1 T2^27 D64 bf16, window 32 + 2^k links k=0..26, inputs
                 drawn on the device
   extreme_8m    B1 H1 T2^23 D64 bf16, window 32 + 2^k links k=0..22 (profiler-
@@ -82,6 +84,10 @@ WORKLOADS = {
     "band_32k_b1h8": _w("band_32k_b1h8", 1, 8, 32768, 128, "bf16", 4096, (), seed=1003),
     "csr_1m": _w("csr_1m", 1, 8, 1 << 20, 64, "bf16", 0, (), seed=1004, csr=True,
                  band_hint=64, graph_seed=2004, bwd=False),
+    # a smaller csr_1m (a quarter of the rows, half the heads): the size used
+    # for detailed profiler captures
+    "csr_256k": _w("csr_256k", 1, 4, 1 << 18, 64, "bf16", 0, (), seed=1004, csr=True,
+                   band_hint=64, graph_seed=2004, bwd=False),
     "extreme_128m": _w("extreme_128m", 1, 1, 1 << 27, 64, "bf16", 32, range(0, 27), seed=1005,
                        bwd=False),
     # a 1/16-length version of extreme_128m: the size used for profiler captures

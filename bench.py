@@ -24,7 +24,10 @@ samples the clocks during the timed region.
 The same line also carries, under "workloads", the other named workloads at
 a few steps each (same timing rules, own roofline and clocks): the W = 4096
 band (fwd+bwd), the graph-view CSR mask at T = 2^20 (fwd, with the timed
-CSR normalise + transpose build) and the T = 2^27 sequence (fwd).
+CSR normalise + transpose build), the T = 2^27 sequence (fwd), the 16K layer
+with grouped-query attention and with learned-coordinate scores (fwd+bwd),
+and decode against 16K caches.  The end-to-end pass streams the (b, h)
+slices through separate upload, kernel and download streams.
 
 ``--impl reference`` times the CPU oracle (the plain fp64 statement of the
 method) on a bounded sample of the same workload instead.

@@ -13,11 +13,18 @@
 //    a CSR list ("Longer Attention Span ...", Abstract) -- is a "diagonal"
 //    block: 128 key rows, row r belonging to query r (for a distance o the
 //    keys q0-o .. q0+127-o; for CSR lists slot s of every row's residual
-//    list).  Each softmax warp fetches the K and V rows of its own 32 queries
-//    itself with 16-byte cp.async copies, DS slots ahead (plus L2 prefetches
-//    further ahead when K and V exceed L2), into the band tiles' swizzled
-//    layout; thread r then takes the dot product of its own row on the CUDA
-//    cores.  No other role takes part, so warps progress independently.
+//    list).  For a distance link the block is 128 contiguous rows: the
+//    producer loads it as TMA boxes into a DS-stage ring (with an L2
+//    prefetch a few blocks ahead when K and V exceed L2).  For CSR lists
+//    each softmax warp copies the K and V rows of its own 32 queries itself
+//    with 16-byte cp.async copies, DS slots ahead, into the same swizzled
+//    layout (sa_rows.cuh).  Thread r then takes the dot product of its own
+//    row on the CUDA cores.
+//  * Links short enough to fall inside the key span that the band blocks
+//    cover anyway (at most kMaxFold) are folded into the band blocks as
+//    extra kept columns; a CSR graph whose rows all start with the same key
+//    prefix (global tokens) gets one more band block holding keys 0 .. 63.
+//    Each row's kept columns of a block are one 64-bit mask.
 //  * One online softmax (running max m and sum l per row, base 2) covers both
 //    classes: the diagonal blocks go first, their weighted sum initialises O
 //    in TMEM, then the band blocks rescale O only when a row's max grows by
@@ -28,7 +35,8 @@
 // per CTA, each with its own shared-memory rings, TMEM columns (two S
 // buffers and O) and barriers, so that the softmax of one tile overlaps the
 // loads, MMAs and softmax of the other.  Warp roles: warp 2p is the TMA
-// producer of pipeline p (Q and the band K/V ring), warp 2p+1 its
+// producer of pipeline p (Q, the band K/V ring and the distance blocks),
+// warp 2p+1 its
 // MMA issuer (warp 1 also allocates TMEM), warps 4+4p .. 7+4p its softmax
 // warpgroup (thread = query row = TMEM lane).  With two pipelines the
 // producer warpgroup hands registers to the softmax warpgroups (setmaxnreg).

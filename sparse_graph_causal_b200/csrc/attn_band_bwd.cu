@@ -16,10 +16,15 @@
 //
 // The other edges (2^k distance links or the non-window part of CSR lists)
 // are diagonal blocks as in the forward: row r of a block belongs to query
-// (or key) r; for a distance o the rows are one TMA box, for CSR lists 4-row
-// TMA gathers of the row's slot.  They are accumulated on CUDA cores (fp32
-// pairs) first and initialise the TMEM accumulators, which the band MMAs then
-// add to.
+// (or key) r; for a distance o the rows are one TMA box loaded by the
+// producer, for CSR lists each compute warp copies its own rows with
+// cp.async (sa_rows.cuh).  They are accumulated on the CUDA cores first
+// (in registers at D = 64, directly in TMEM at D = 128) and initialise the
+// TMEM accumulators, which the band MMAs then add to.  On a structured graph
+// band_bwd_dq stores (p, dS) of every distance edge in a cache that
+// band_bwd_dkdv reads instead of recomputing them.  With grouped-query
+// attention a dK/dV tile covers one key/value head and loops over the query
+// heads of its group.
 //
 // Both kernels are persistent and run NP (1 or 2) independent tile pipelines
 // per CTA, each with its own shared-memory rings, TMEM columns and barriers.

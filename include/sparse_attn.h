@@ -224,8 +224,10 @@ sa_status sparse_attn_dist_bwd(const sa_tensor *a, const sa_tensor *c, const sa_
 const char *sparse_attn_status_string(sa_status s);
 
 /* Kernel selection for fwd/bwd (process-wide; default SA_PATH_AUTO):
- *  SA_PATH_AUTO   bf16 with D in {64, 128} runs the tcgen05 band tiles for the
- *                 window part plus the gather path for the other edges;
+ *  SA_PATH_AUTO   bf16 with D in {32, 64, 128} and a band (W >= 1) runs the
+ *                 tcgen05 band kernels: the window on the tensor cores, the
+ *                 other edges as diagonal blocks on the CUDA cores of the same
+ *                 kernels (D = 32 on the D = 64 tiles, rows zero-extended);
  *                 everything else runs the gather kernels alone.
  *  SA_PATH_GATHER every edge on the gather kernels (CUDA cores). */
 typedef enum { SA_PATH_AUTO = 0, SA_PATH_GATHER = 1 } sa_path;

@@ -176,7 +176,11 @@ __device__ __forceinline__ TileGeom tile_geom(int64_t t, int64_t ntq, int64_t T,
 // each distance block as TMA boxes (structured graphs: 128 contiguous rows);
 // true -- every softmax warp copies its own rows (CSR lists: one random row
 // per tile row, rows/sa_rows.cuh).
-template <int D, int NP, int KS, int VS, int DS, bool LDW>
+// DG: the row length of q, k, v and out in global memory; D the width of the
+// tiles in shared memory and TMEM.  DG = 32 runs on the D = 64 tiles: the TMA
+// boxes read 64 columns, the 32 beyond each row come back as zeros (out of
+// bounds of the tensor map) and add nothing to any product.
+template <int D, int NP, int KS, int VS, int DS, bool LDW, int DG>
 __global__ void __launch_bounds__(128 + 128 * NP, 1)
 band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkd,
@@ -230,6 +234,13 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         }
         *abort = 0;
         tc::fence_barrier_init();
+    }
+    if constexpr (LDW && DG < D) {
+        // the per-warp copies fill DG columns of each diagonal row: the rest
+        // of the rings stays zero
+        for (int p = 0; p < NP; ++p)
+            for (int o = L::pDK + 16 * tid; o < L::kPipe; o += 16 * blockDim.x)
+                *(uint4 *)(sm + p * L::kPipe + o) = make_uint4(0, 0, 0, 0);
     }
     if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), L::kTmemCols);
     tc::tc_fence_before();
@@ -478,7 +489,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     auto key_of = [&](int d) -> int32_t {  // (CSR slots)
                         return d < resid ? __ldg(a.colidx + cst + d) : -1;
                     };
-                    const size_t slice = (size_t)g.kvbh * (size_t)T * D;
+                    const size_t slice = (size_t)g.kvbh * (size_t)T * DG;
                     uint32_t qw[D / 2];
                     // one slot: dot product with the row's key, online-softmax
                     // update, p-weighted value row into acc (Q is read on the
@@ -488,7 +499,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                             ok = __all_sync(0xffffffffu, wait(p, L::bQFull, (uint32_t)(lt & 1)));
                             if (ok) {
 #pragma unroll
-                                for (int c = 0; c < D / 8; ++c) {
+                                for (int c = 0; c < DG / 8; ++c) {
                                     const uint4 w4 = *(const uint4 *)(pm + L::pQ +
                                                                       (c >> 3) * (BM * 128) +
                                                                       tc::sw128_off(r, c & 7));
@@ -508,7 +519,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
 #pragma unroll
                         for (int x = 0; x < 8; ++x) sp[x] = 0.f;
 #pragma unroll
-                        for (int c = 0; c < D / 8; ++c) {
+                        for (int c = 0; c < DG / 8; ++c) {
                             const uint4 w4 = *(const uint4 *)(kr + (c >> 3) * (BM * 128) +
                                                               tc::sw128_off(r, c & 7));
                             const uint32_t kw[4] = {w4.x, w4.y, w4.z, w4.w};
@@ -532,7 +543,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         l_run += pr;
                         const uint32_t p2 = tc::pack_bf16x2(pr, pr);
 #pragma unroll
-                        for (int c = 0; c < D / 8; ++c) {
+                        for (int c = 0; c < DG / 8; ++c) {
                             const uint4 w4 = *(const uint4 *)(vr + (c >> 3) * (BM * 128) +
                                                               tc::sw128_off(r, c & 7));
                             const uint32_t vw[4] = {w4.x, w4.y, w4.z, w4.w};
@@ -545,7 +556,7 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         }
                     };
                     if constexpr (LDW) {
-                        rows::warp_slots<D, DS>(
+                        rows::warp_slots<DG, DS>(
                             nd, sbase + (uint32_t)(p * L::kPipe + L::pDK),
                             sbase + (uint32_t)(p * L::kPipe + L::pDV), (uint32_t)L::kQTile, a.k,
                             a.v, a.l2pf > 0, lane, wq, [&](int) { return slice; }, key_of, body);
@@ -743,9 +754,9 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             if (!wait(p, L::bPVDone + (int)(gb_last & 1), (gb_last >> 1) & 1)) break;
             tc::tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            __nv_bfloat16 *orow = a.out + ((size_t)bh * (size_t)T + (size_t)i) * D;
+            __nv_bfloat16 *orow = a.out + ((size_t)bh * (size_t)T + (size_t)i) * DG;
 #pragma unroll
-            for (int c = 0; c < D; c += 32) {
+            for (int c = 0; c < DG; c += 32) {
                 uint32_t w[32];
                 tc::tmem_ld32(tO + c, w);
                 tc::tmem_ld_wait();
@@ -779,14 +790,15 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     }
 }
 
-template <int D, int NP, int KS, int VS, int DS, bool LDW>
+template <int D, int NP, int KS, int VS, int DS, bool LDW, int DG>
 sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_graph_s *g, float scale, sa_tensor *out, float *lse,
                           cudaStream_t s) {
     using L = Layout<D, NP, KS, VS, DS>;
     static_assert(L::kAlloc <= 232448, "shared memory budget");
     constexpr int kThreads = 128 + 128 * NP;
-    auto kern = band_fwd_kernel<D, NP, KS, VS, DS, LDW>;
+    static_assert(DG == D || (D == 64 && DG == 32), "row length");
+    auto kern = band_fwd_kernel<D, NP, KS, VS, DS, LDW, DG>;
     if (NP == 2) {
         // setmaxnreg.inc waits until the CTA's pool holds the registers it
         // asks for: the launch must provide the whole split
@@ -804,11 +816,11 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     }
     const int64_t BH = q->B * q->H, BHkv = k->B * k->H, T = q->T;
     CUtensorMap mq, mk, mv, mkd, mvd;  // 64-row band boxes, 128-row distance blocks
-    if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BM) ||
-        !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BHkv, BN) ||
-        !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BHkv, BN) ||
-        !sa_tmap_bf16_3d(&mkd, k->ptr, D, T, BHkv, BM) ||
-        !sa_tmap_bf16_3d(&mvd, v->ptr, D, T, BHkv, BM)) {
+    if (!sa_tmap_bf16_3d(&mq, q->ptr, DG, T, BH, BM) ||
+        !sa_tmap_bf16_3d(&mk, k->ptr, DG, T, BHkv, BN) ||
+        !sa_tmap_bf16_3d(&mv, v->ptr, DG, T, BHkv, BN) ||
+        !sa_tmap_bf16_3d(&mkd, k->ptr, DG, T, BHkv, BM) ||
+        !sa_tmap_bf16_3d(&mvd, v->ptr, DG, T, BHkv, BM)) {
         sa_record_cuda_error(cudaErrorInvalidValue, "band_fwd: tensor map encoding");
         return SA_ERR_CUDA;
     }
@@ -821,7 +833,7 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.kind = g->kind;
     a.gp = g->kind == 1 ? g->gprefix : 0;
     a.We = sa_fold_links(g, BN, kMaxFold, a.fold, &a.nf, a.offs, &a.n_off);
-    a.l2pf = (double)BHkv * (double)T * D * 2 * 2 > kL2ResidentBytes ? 1 : 0;
+    a.l2pf = (double)BHkv * (double)T * DG * 2 * 2 > kL2ResidentBytes ? 1 : 0;
     a.rowptr = g->rowptr;
     a.colidx = g->colidx;
     a.k = (const __nv_bfloat16 *)k->ptr;
@@ -847,7 +859,7 @@ sa_status launch_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
 }  // namespace
 
 bool sa_band_fwd_supported(const sa_tensor *q, const sa_graph_s *g) {
-    if (q->dtype != SA_BF16 || (q->D != 64 && q->D != 128)) return false;
+    if (q->dtype != SA_BF16 || (q->D != 32 && q->D != 64 && q->D != 128)) return false;
     if (g->W < 1) return false;                       // no band: gather path
     // 32-bit tile coordinates (TMA takes int32 row and slice indices)
     if (q->B * q->H >= ((int64_t)1 << 31) || q->T >= ((int64_t)1 << 31)) return false;
@@ -862,12 +874,18 @@ sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
     const bool csr = g->kind == 1;
     // <D, pipelines, K stages, V stages, diagonal stages, per-warp slots>,
     // sized to the 227 KB of shared memory
-    if (q->D == 64) {
-        if (!diag) return launch_band_fwd<64, 2, 4, 4, 0, false>(q, k, v, g, scale, out, lse, s);
-        return csr ? launch_band_fwd<64, 2, 2, 2, 2, true>(q, k, v, g, scale, out, lse, s)
-                   : launch_band_fwd<64, 2, 2, 2, 2, false>(q, k, v, g, scale, out, lse, s);
+    // (D = 32 runs on the D = 64 tiles, its rows zero-extended)
+    if (q->D == 32) {
+        if (!diag) return launch_band_fwd<64, 2, 4, 4, 0, false, 32>(q, k, v, g, scale, out, lse, s);
+        return csr ? launch_band_fwd<64, 2, 2, 2, 2, true, 32>(q, k, v, g, scale, out, lse, s)
+                   : launch_band_fwd<64, 2, 2, 2, 2, false, 32>(q, k, v, g, scale, out, lse, s);
     }
-    if (!diag) return launch_band_fwd<128, 2, 3, 2, 0, false>(q, k, v, g, scale, out, lse, s);
-    return csr ? launch_band_fwd<128, 1, 2, 2, 2, true>(q, k, v, g, scale, out, lse, s)
-               : launch_band_fwd<128, 1, 2, 2, 2, false>(q, k, v, g, scale, out, lse, s);
+    if (q->D == 64) {
+        if (!diag) return launch_band_fwd<64, 2, 4, 4, 0, false, 64>(q, k, v, g, scale, out, lse, s);
+        return csr ? launch_band_fwd<64, 2, 2, 2, 2, true, 64>(q, k, v, g, scale, out, lse, s)
+                   : launch_band_fwd<64, 2, 2, 2, 2, false, 64>(q, k, v, g, scale, out, lse, s);
+    }
+    if (!diag) return launch_band_fwd<128, 2, 3, 2, 0, false, 128>(q, k, v, g, scale, out, lse, s);
+    return csr ? launch_band_fwd<128, 1, 2, 2, 2, true, 128>(q, k, v, g, scale, out, lse, s)
+               : launch_band_fwd<128, 1, 2, 2, 2, false, 128>(q, k, v, g, scale, out, lse, s);
 }

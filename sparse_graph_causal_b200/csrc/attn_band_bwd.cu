@@ -342,7 +342,7 @@ struct DQBand {
 
 // LDW: the diagonal slots are copied by each compute warp (CSR lists); else
 // the producer loads each distance block as TMA boxes (structured graphs).
-template <int D, int NP, int BB, int SB, int BS, int DS, int PS, bool LDW>
+template <int D, int NP, int BB, int SB, int BS, int DS, int PS, bool LDW, int DG>
 __global__ void __launch_bounds__(128 + 128 * NP, 1)
 band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -395,6 +395,13 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         }
         *abort = 0;
         tc::fence_barrier_init();
+    }
+    if constexpr (LDW && DG < D) {
+        // the per-warp copies fill DG columns of each diagonal row: the rest
+        // of the rings stays zero
+        for (int p = 0; p < NP; ++p)
+            for (int o = L::pDK + 16 * tid; o < L::pDS; o += 16 * blockDim.x)
+                *(uint4 *)(sm + p * L::kPipe + o) = make_uint4(0, 0, 0, 0);
     }
     if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), L::kTmemCols);
     tc::tc_fence_before();
@@ -595,21 +602,21 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             const size_t grow = (size_t)bh * (size_t)T + (size_t)i;
             const float lse2 = row_ok ? a.lse[grow] * kLog2e : 0.f;
             // the out row for Delta is fetched while Q and dO arrive
-            uint4 orow4[D / 8];
+            uint4 orow4[DG / 8];
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c)
-                orow4[c] = row_ok ? __ldg((const uint4 *)(a.o + grow * D) + c) : make_uint4(0, 0, 0, 0);
+            for (int c = 0; c < DG / 8; ++c)
+                orow4[c] = row_ok ? __ldg((const uint4 *)(a.o + grow * DG) + c) : make_uint4(0, 0, 0, 0);
             if (!__all_sync(0xffffffffu, wait(p, L::bQFull, (uint32_t)(lt & 1)))) break;
             // Delta_i = dO_i . out_i
             float Delta = 0.f;
             {
-                uint32_t dor[D / 2];
-                load_row_packed<D>(pm + L::pDO, BM, r, dor);
+                uint32_t dor[DG / 2];
+                load_row_packed<DG>(pm + L::pDO, BM, r, dor);
                 float sp[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) sp[x] = 0.f;
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
+                for (int c = 0; c < DG / 8; ++c) {
                     const uint32_t ow[4] = {orow4[c].x, orow4[c].y, orow4[c].z, orow4[c].w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -657,8 +664,8 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                 };
                 // the q row in registers (D = 64) or read from the Q tile (D = 128,
                 // whose accumulator already takes 128 registers)
-                uint32_t qw[D == 64 ? D / 2 : 1];
-                if constexpr (D == 64) load_row_packed<D>(pm + L::pQ, BM, r, qw);
+                uint32_t qw[D == 64 ? DG / 2 : 1];
+                if constexpr (D == 64) load_row_packed<DG>(pm + L::pQ, BM, r, qw);
                 auto body = [&](int d, int st) {
                     const bool valid = LDW ? (d < resid) : (row_ok && i >= a.offs[dfirst + d]);
                     const uint8_t *kt = pm + L::pDK + st * L::kRow;
@@ -667,26 +674,26 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                     if (valid) {
                         float qk;
                         if constexpr (D == 64)
-                            qk = dot_bf_reg_smem<D>(qw, kt, BM, r);
+                            qk = dot_bf_reg_smem<DG>(qw, kt, BM, r);
                         else
-                            qk = dot_bf_smem_smem<D>(pm + L::pQ, kt, BM, r);
+                            qk = dot_bf_smem_smem<DG>(pm + L::pQ, kt, BM, r);
                         const float pr = tc::ex2(fmaf(qk, c2, -lse2));
-                        ds = pr * (dot_bf_smem_smem<D>(pm + L::pDO, vt, BM, r) - Delta);
+                        ds = pr * (dot_bf_smem_smem<DG>(pm + L::pDO, vt, BM, r) - Delta);
                         if (a.pds)
                             a.pds[((size_t)(dfirst + d) * (size_t)a.BH + (size_t)bh) *
                                       (size_t)T +
                                   (size_t)i] = make_float2(pr, ds);
-                        if constexpr (kRegAcc) axpy_bf_smem<D>(acc, ds, kt, BM, r);
+                        if constexpr (kRegAcc) axpy_bf_smem<DG>(acc, ds, kt, BM, r);
                     }
                     // (warp-collective: every lane, whether or not its row has the slot)
                     if constexpr (!kRegAcc) tmem_axpy_row<D>(tDQ, ds, valid, kt, BM, r);
                 };
                 if constexpr (LDW) {
-                    rows::warp_slots<D, DS>(
+                    rows::warp_slots<DG, DS>(
                         nd, sbase + (uint32_t)(p * L::kPipe + L::pDK),
                         sbase + (uint32_t)(p * L::kPipe + L::pDV), (uint32_t)L::kRow, a.k, a.v,
                         a.l2pf != 0, lane, wq,
-                        [&](int) { return (size_t)kvbh * (size_t)T * D; }, key_of, body);
+                        [&](int) { return (size_t)kvbh * (size_t)T * DG; }, key_of, body);
                 } else {
                     for (int d = 0; ok && d < nd; ++d) {
                         const int st = (int)(dc % DS);
@@ -792,7 +799,7 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             if (!ok) break;
             if (!wait(p, L::bDQDone + (int)(gb_last % SB), (gb_last / SB) & 1)) break;
             tc::tc_fence_after();
-            tmem_row_to_global<D>(tDQ, a.scale, a.dq + grow * D, row_ok);
+            tmem_row_to_global<DG>(tDQ, a.scale, a.dq + grow * DG, row_ok);
         }
     }
     tc::tc_fence_before();
@@ -854,7 +861,7 @@ __device__ __forceinline__ int dkv_n_band(int32_t k0, int64_t T, int32_t W) {
 
 // LDW: the diagonal slots are copied by each compute warp (CSR lists); else
 // the producer loads each distance block as TMA boxes (structured graphs).
-template <int D, int NP, int BB, int SB, int BS, int DS, int PS, bool LDW>
+template <int D, int NP, int BB, int SB, int BS, int DS, int PS, bool LDW, int DG>
 __global__ void __launch_bounds__(128 + 128 * NP, 1)
 band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                      const __grid_constant__ CUtensorMap tvt,
@@ -919,6 +926,13 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
         }
         *abort = 0;
         tc::fence_barrier_init();
+    }
+    if constexpr (LDW && DG < D) {
+        // the per-warp copies fill DG columns of each diagonal row: the rest
+        // of the rings stays zero
+        for (int p = 0; p < NP; ++p)
+            for (int o = L::pDQ + 16 * tid; o < L::pP; o += 16 * blockDim.x)
+                *(uint4 *)(sm + p * L::kPipe + o) = make_uint4(0, 0, 0, 0);
     }
     if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), L::kTmemCols);
     tc::tc_fence_before();
@@ -1243,14 +1257,14 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                             pr = v_cur.x;
                             ds = v_cur.y;
                         } else {
-                            const float sdot = dot_bf_smem_smem<D>(qt, pm + L::pK, BM, r);
-                            const float dpdot = dot_bf_smem_smem<D>(dt, pm + L::pV, BM, r);
+                            const float sdot = dot_bf_smem_smem<DG>(qt, pm + L::pK, BM, r);
+                            const float dpdot = dot_bf_smem_smem<DG>(dt, pm + L::pV, BM, r);
                             pr = tc::ex2(fmaf(sdot, c2, -v_cur.x * kLog2e));
                             ds = pr * (dpdot - v_cur.y);
                         }
                         if constexpr (kRegAcc) {
-                            axpy_bf_smem<D>(adv, pr, dt, BM, r);
-                            axpy_bf_smem<D>(adk, ds, qt, BM, r);
+                            axpy_bf_smem<DG>(adv, pr, dt, BM, r);
+                            axpy_bf_smem<DG>(adk, ds, qt, BM, r);
                         }
                     }
                     // (warp-collective: every lane, whether or not its key has the slot)
@@ -1263,12 +1277,12 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                     v_cur = v_nxt;
                 };
                 if constexpr (LDW) {
-                    rows::warp_slots<D, DS>(
+                    rows::warp_slots<DG, DS>(
                         nds, sbase + (uint32_t)(p * L::kPipe + L::pDQ),
                         sbase + (uint32_t)(p * L::kPipe + L::pDDO), (uint32_t)L::kRow, a.q,
                         a.dout, a.l2pf != 0, lane, wq,
                         [&](int d) {
-                            return (size_t)(qbh0 + (nd > 0 ? head_of(d) : 0)) * (size_t)T * D;
+                            return (size_t)(qbh0 + (nd > 0 ? head_of(d) : 0)) * (size_t)T * DG;
                         },
                         key_of, body);
                 } else {
@@ -1390,8 +1404,8 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             if (!ok) break;
             if (!wait(p, L::bDKVDone + (int)(gb_last % SB), (gb_last / SB) & 1)) break;
             tc::tc_fence_after();
-            tmem_row_to_global<D>(tDV, 1.f, a.dv + grow * D, row_ok);
-            tmem_row_to_global<D>(tDK, a.scale, a.dk + grow * D, row_ok);
+            tmem_row_to_global<DG>(tDV, 1.f, a.dv + grow * DG, row_ok);
+            tmem_row_to_global<DG>(tDK, a.scale, a.dk + grow * DG, row_ok);
         }
     }
     tc::tc_fence_before();
@@ -1412,7 +1426,7 @@ inline bool regs_cover(const void *kern) {
     return fa.numRegs * (128 + 128 * NP) >= 128 * BwdRegs::producer + 128 * NP * BwdRegs::compute;
 }
 
-template <int D, int NP, int BB, int SB, int BSQ, int BSK, int DS, int PS, bool LDW>
+template <int D, int NP, int BB, int SB, int BSQ, int BSK, int DS, int PS, bool LDW, int DG>
 sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
                           const sa_tensor *o, const float *lse, const sa_tensor *dout,
                           const sa_graph_s *g, float scale, sa_tensor *dq, sa_tensor *dk,
@@ -1421,8 +1435,9 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     using LK = LayoutDKV<D, NP, BB, SB, BSK, DS, PS>;
     static_assert(LQ::kAlloc <= 232448 && LK::kAlloc <= 232448, "shared memory budget");
     constexpr int kThreads = 128 + 128 * NP;
-    auto kq = band_bwd_dq_kernel<D, NP, BB, SB, BSQ, DS, PS, LDW>;
-    auto kkv = band_bwd_dkdv_kernel<D, NP, BB, SB, BSK, DS, PS, LDW>;
+    static_assert(DG == D || (D == 64 && DG == 32), "row length");
+    auto kq = band_bwd_dq_kernel<D, NP, BB, SB, BSQ, DS, PS, LDW, DG>;
+    auto kkv = band_bwd_dkdv_kernel<D, NP, BB, SB, BSK, DS, PS, LDW, DG>;
     static int regs_ok = -1;
     if (regs_ok < 0)
         regs_ok = regs_cover<NP>((const void *)kq) && regs_cover<NP>((const void *)kkv);
@@ -1434,14 +1449,14 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     const int64_t BH = q->B * q->H, BHkv = k->B * k->H, T = q->T;
     // 128-row boxes for the tiles, BB-row boxes for the band rings
     CUtensorMap mq, mdo, mk, mv, mqb, mdob, mkb, mvb;
-    if (!sa_tmap_bf16_3d(&mq, q->ptr, D, T, BH, BM) ||
-        !sa_tmap_bf16_3d(&mdo, dout->ptr, D, T, BH, BM) ||
-        !sa_tmap_bf16_3d(&mk, k->ptr, D, T, BHkv, BM) ||
-        !sa_tmap_bf16_3d(&mv, v->ptr, D, T, BHkv, BM) ||
-        !sa_tmap_bf16_3d(&mqb, q->ptr, D, T, BH, BB) ||
-        !sa_tmap_bf16_3d(&mdob, dout->ptr, D, T, BH, BB) ||
-        !sa_tmap_bf16_3d(&mkb, k->ptr, D, T, BHkv, BB) ||
-        !sa_tmap_bf16_3d(&mvb, v->ptr, D, T, BHkv, BB)) {
+    if (!sa_tmap_bf16_3d(&mq, q->ptr, DG, T, BH, BM) ||
+        !sa_tmap_bf16_3d(&mdo, dout->ptr, DG, T, BH, BM) ||
+        !sa_tmap_bf16_3d(&mk, k->ptr, DG, T, BHkv, BM) ||
+        !sa_tmap_bf16_3d(&mv, v->ptr, DG, T, BHkv, BM) ||
+        !sa_tmap_bf16_3d(&mqb, q->ptr, DG, T, BH, BB) ||
+        !sa_tmap_bf16_3d(&mdob, dout->ptr, DG, T, BH, BB) ||
+        !sa_tmap_bf16_3d(&mkb, k->ptr, DG, T, BHkv, BB) ||
+        !sa_tmap_bf16_3d(&mvb, v->ptr, DG, T, BHkv, BB)) {
         sa_record_cuda_error(cudaErrorInvalidValue, "band_bwd: tensor map encoding");
         return SA_ERR_CUDA;
     }
@@ -1450,7 +1465,7 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     a.BH = BH;
     a.H = q->H;
     a.Hkv = k->H;
-    a.l2pf = (double)BH * (double)T * D * 2 * 2 > 64.0 * 1024 * 1024 ? 1 : 0;
+    a.l2pf = (double)BH * (double)T * DG * 2 * 2 > 64.0 * 1024 * 1024 ? 1 : 0;
     a.W = g->W;
     a.kind = g->kind;
     a.We = sa_fold_links(g, BB, kMaxFold, a.fold, &a.nf, a.offs, &a.n_off);
@@ -1494,7 +1509,7 @@ sa_status launch_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
 }  // namespace
 
 bool sa_band_bwd_supported(const sa_tensor *q, const sa_tensor *k, const sa_graph_s *g) {
-    if (q->dtype != SA_BF16 || (q->D != 64 && q->D != 128)) return false;
+    if (q->dtype != SA_BF16 || (q->D != 32 && q->D != 64 && q->D != 128)) return false;
     if (g->W < 1) return false;
     // 32-bit tile coordinates; the CSR gathers address rows of all slices
     // (slice * T + row) as one int32 coordinate
@@ -1514,15 +1529,21 @@ sa_status sa_band_bwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
     // shared memory and 512 TMEM columns
     const bool csr = g->kind == 1;
 #define SA_BWD_ARGS q, k, v, out, lse, dout, g, scale, dq, dk, dv, delta, pds, s
+    // (D = 32 runs on the D = 64 tiles, its rows zero-extended)
+    if (q->D == 32) {
+        if (!diag) return launch_band_bwd<64, 2, 32, 2, 4, 4, 0, 0, false, 32>(SA_BWD_ARGS);
+        return csr ? launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0, true, 32>(SA_BWD_ARGS)
+                   : launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0, false, 32>(SA_BWD_ARGS);
+    }
     if (q->D == 64) {
-        if (!diag) return launch_band_bwd<64, 2, 32, 2, 4, 4, 0, 0, false>(SA_BWD_ARGS);
-        return csr ? launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0, true>(SA_BWD_ARGS)
-                   : launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0, false>(SA_BWD_ARGS);
+        if (!diag) return launch_band_bwd<64, 2, 32, 2, 4, 4, 0, 0, false, 64>(SA_BWD_ARGS);
+        return csr ? launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0, true, 64>(SA_BWD_ARGS)
+                   : launch_band_bwd<64, 2, 32, 2, 2, 2, 2, 0, false, 64>(SA_BWD_ARGS);
     }
     // D = 128: one pipeline, P^T / dS^T and dS in shared memory; with
     // diagonal edges a one-stage diagonal ring and two-stage band rings
-    if (!diag) return launch_band_bwd<128, 1, 64, 2, 3, 3, 0, 1, false>(SA_BWD_ARGS);
-    return csr ? launch_band_bwd<128, 1, 64, 2, 2, 2, 1, 1, true>(SA_BWD_ARGS)
-               : launch_band_bwd<128, 1, 64, 2, 2, 2, 1, 1, false>(SA_BWD_ARGS);
+    if (!diag) return launch_band_bwd<128, 1, 64, 2, 3, 3, 0, 1, false, 128>(SA_BWD_ARGS);
+    return csr ? launch_band_bwd<128, 1, 64, 2, 2, 2, 1, 1, true, 128>(SA_BWD_ARGS)
+               : launch_band_bwd<128, 1, 64, 2, 2, 2, 1, 1, false, 128>(SA_BWD_ARGS);
 #undef SA_BWD_ARGS
 }

@@ -67,7 +67,7 @@ __device__ __forceinline__ void warp_slots(int nd, uint32_t ring_a, uint32_t rin
         if (key >= 0) {
             const size_t src = (size_t)slot_base(d) + (size_t)key * D;
 #pragma unroll
-            for (int x = 0; x < D / 64; ++x) {
+            for (int x = 0; x < (D + 63) / 64; ++x) {
                 tc::prefetch_l2(src_a + src + 64 * x);
                 tc::prefetch_l2(src_b + src + 64 * x);
             }

@@ -50,6 +50,11 @@ CASES = [
     _wl("d128_w200", 1, 2, 1000, 128, "bf16", 200, (8, 9)),
     _wl("d128_band", 2, 1, 777, 128, "bf16", 256, ()),
     _wl("d32_bf16", 1, 2, 200, 32, "bf16", 16, range(0, 8)),
+    # bf16 D = 32 runs on the D = 64 tensor-core tiles with zero-extended rows
+    _wl("d32_links_ragged", 2, 2, 389, 32, "bf16", 32, range(0, 9)),
+    _wl("d32_band_only", 1, 2, 600, 32, "bf16", 300, ()),
+    _wl("csr_d32", 1, 2, 1500, 32, "bf16", 0, (), csr=synth.csr_random_rows(1500, seed=43),
+        band=64),
     _wl("d64_fp32", 1, 2, 333, 64, "fp32", 40, range(0, 9)),
     _wl("d128_fp32", 1, 1, 150, 128, "fp32", 64, (7,)),
     _wl("csr_view_3000", 1, 2, 3000, 64, "bf16", 0, (),
@@ -207,3 +212,30 @@ def test_many_slices_on_tensor_cores(sa, oracle_lib):
         for got, ref, n in ((out, rout, "out"), (dq, rdq, "dq"), (dk, rdk, "dk"), (dv, rdv, "dv")):
             compare(got.view(BH, w.T, w.D)[bh], ref, w.dtype, f"many_slices[{bh}] {n}")
         compare(lse.view(BH, w.T)[bh], rlse, w.dtype, f"many_slices[{bh}] lse")
+
+
+@pytest.mark.parametrize("kind", ["links", "band", "csr"])
+def test_d32_bf16_on_tensor_cores(sa, oracle_lib, kind):
+    """bf16 with D = 32 takes the tcgen05 band kernels (not the gather
+    kernels) for every graph kind, and matches the oracle there."""
+    w, csr = {"links": _wl("d32_tc_links", 1, 2, 700, 32, "bf16", 32, range(0, 10), seed=5),
+              "band": _wl("d32_tc_band", 1, 2, 700, 32, "bf16", 256, (), seed=6),
+              "csr": _wl("d32_tc_csr", 1, 2, 900, 32, "bf16", 0, (),
+                         csr=synth.csr_random_rows(900, seed=44), band=64)}[kind]
+    o = oracle_lib
+    g, rp, ci = build_graph(sa, o, w, csr)
+    x = synth.make_qkv(w, device="cuda")
+    sa.sparse_attn_profile_begin(True)
+    out, lse = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+    dq, dk, dv = sa.sparse_attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], g, w.scale)
+    prof = sa.sparse_attn_profile_end()
+    sa.sparse_attn_check_device()
+    assert set(prof) == {"band_fwd", "band_bwd_dq", "band_bwd_dkdv"}, prof
+    BH = w.B * w.H
+    for bh in range(BH):
+        sl = [to_oracle(x[n].view(BH, w.T, w.D)[bh], w.dtype) for n in ("q", "k", "v", "dout")]
+        rout, rlse = o.fwd(sl[0], sl[1], sl[2], rp, ci, w.scale, dtype=w.dtype)
+        rdq, rdk, rdv = o.bwd(*sl, rp, ci, w.scale, dtype=w.dtype)
+        for got, ref, n in ((out, rout, "out"), (dq, rdq, "dq"), (dk, rdk, "dk"), (dv, rdv, "dv")):
+            compare(got.view(BH, w.T, w.D)[bh], ref, w.dtype, f"{w.name}[{bh}] {n}")
+        compare(lse.view(BH, w.T)[bh], rlse, w.dtype, f"{w.name}[{bh}] lse")

@@ -233,6 +233,22 @@ const char *sparse_attn_status_string(sa_status s);
 typedef enum { SA_PATH_AUTO = 0, SA_PATH_GATHER = 1 } sa_path;
 sa_status sparse_attn_set_path(int32_t path);
 
+/* Long distance links of a structured graph (process-wide; default
+ * SA_LINKS_AUTO).  The band-kernel forward can take the links of at least
+ * 2^15 rows (when all such links are multiples of 2^15, e.g. powers of two)
+ * in a second pass that runs the tiles in an order keeping their K/V rows in
+ * L2 ("Longer Attention Span ...", Abstract: single-GPU sequences of 160 M
+ * tokens), merged into out and lse by the online-softmax rule.  Results are
+ * the same up to rounding (pass 1's out is read back in the input dtype).
+ *  SA_LINKS_AUTO     two passes when K and V together hold 8 GiB or more and
+ *                    at least three such links exist (below that one pass was
+ *                    measured faster on B200)
+ *  SA_LINKS_SPLIT    two passes whenever such a link exists
+ *  SA_LINKS_ONE_PASS never
+ * Returns SA_ERR_INVALID_ARG for any other value. */
+typedef enum { SA_LINKS_AUTO = 0, SA_LINKS_SPLIT = 1, SA_LINKS_ONE_PASS = 2 } sa_links_mode;
+sa_status sparse_attn_set_link_pass(int32_t mode);
+
 /* Synchronise `stream`, then read and clear the library's device error word:
  * SA_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the last
  * check, SA_ERR_CUDA on a CUDA error, else SA_OK. */

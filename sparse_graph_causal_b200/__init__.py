@@ -21,6 +21,7 @@ SA_OK, SA_ERR_INVALID_ARG, SA_ERR_INVALID_GRAPH, SA_ERR_UNSUPPORTED = 0, 1, 2, 3
 SA_ERR_OOM, SA_ERR_CUDA, SA_ERR_DEVICE_TIMEOUT = 4, 5, 6
 SA_BF16, SA_FP32 = 0, 1
 SA_PATH_AUTO, SA_PATH_GATHER = 0, 1
+SA_LINKS_AUTO, SA_LINKS_SPLIT, SA_LINKS_ONE_PASS = 0, 1, 2
 
 class SaTensor(ctypes.Structure):
     _fields_ = [("ptr", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("B", ctypes.c_int64),
@@ -47,6 +48,7 @@ def _load():
                                  P(SaTensor), vp, ctypes.c_size_t, vp]),
         "sparse_attn_status_string": (ctypes.c_char_p, [st]),
         "sparse_attn_set_path": (st, [i32]),
+        "sparse_attn_set_link_pass": (st, [i32]),
         "sparse_attn_check_device": (st, [vp]),
         "sparse_attn_selftest_wait_timeout": (st, [i64, vp]),
         "sparse_attn_launch_count": (i64, []),
@@ -365,6 +367,10 @@ def sparse_attn_status_string(status: int) -> str:
 
 def sparse_attn_set_path(path: int):
     _check(_lib.sparse_attn_set_path(int(path)), "sparse_attn_set_path")
+
+
+def sparse_attn_set_link_pass(mode: int):
+    _check(_lib.sparse_attn_set_link_pass(int(mode)), "sparse_attn_set_link_pass")
 
 
 def sparse_attn_check_device(stream=None):

@@ -867,9 +867,65 @@ bool sa_band_fwd_supported(const sa_tensor *q, const sa_graph_s *g) {
     return true;
 }
 
+namespace {
+
+// Links of at least kLongSpan rows, all multiples of kLongSpan, can go to a
+// second pass (attn_links.cu): in sequence order their rows have left L2 by
+// the time a link reads them (the sweep reads ~6 KB of K/V per row of
+// progress, so rows 2^15 back are ~200 MB old), while the second pass runs
+// the tiles in an order that keeps them there.  The second pass re-reads q,
+// out and lse and its per-edge cost is about that of the band kernel's
+// distance blocks when they hit L2, so it pays only when many long links miss:
+// on B200 one pass was faster at T = 2^23 (K and V 2 GiB: 4.8 vs 5.1 ms) and
+// two passes at 2^25 (22.8 vs 22.1 ms), 2^26 (49.8 vs 47.0) and 2^27 (114 vs
+// 101), with window 32 and links 2^k.
+constexpr int64_t kLongSpan = (int64_t)1 << 15;
+constexpr int kMinLong = 3;
+constexpr double kTwoPassBytes = 8.0 * 1024 * 1024 * 1024;  // K and V together
+
+int long_links(const sa_tensor *k, const sa_graph_s *g) {
+    const int mode = sa_link_pass_mode();
+    if (g->kind != 0 || mode == SA_LINKS_ONE_PASS) return 0;
+    int n = 0;
+    while (n < g->n_off && g->offs[n] >= kLongSpan) {  // descending
+        if (g->offs[n] % kLongSpan != 0) return 0;
+        ++n;
+    }
+    if (mode == SA_LINKS_SPLIT) return n;
+    const double kv = (double)k->B * (double)k->H * (double)k->T * k->D * 2 * 2;
+    return (kv >= kTwoPassBytes && n >= kMinLong) ? n : 0;
+}
+
+sa_status band_fwd_dispatch(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                            const sa_graph_s *g, float scale, sa_tensor *out, float *lse,
+                            cudaStream_t s);
+
+}  // namespace
+
 sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
-                      const sa_graph_s *g, const GraphView &, float scale, sa_tensor *out,
+                      const sa_graph_s *g_in, const GraphView &, float scale, sa_tensor *out,
                       float *lse, cudaStream_t s) {
+    // the first pass takes the window and the links shorter than kLongSpan
+    const int n_long = long_links(k, g_in);
+    sa_graph_s g_short;
+    const sa_graph_s *g = g_in;
+    if (n_long > 0) {
+        g_short = *g_in;
+        g_short.n_off = g_in->n_off - n_long;
+        for (int x = 0; x < SA_MAX_OFFSETS; ++x)
+            g_short.offs[x] = x < g_short.n_off ? g_in->offs[x + n_long] : 0;
+        g = &g_short;
+    }
+    const sa_status st = band_fwd_dispatch(q, k, v, g, scale, out, lse, s);
+    if (st != SA_OK || n_long == 0) return st;
+    return sa_link_pass(q, k, v, g_in->offs, n_long, kLongSpan, scale, out, lse, s);
+}
+
+namespace {
+
+sa_status band_fwd_dispatch(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,
+                            const sa_graph_s *g, float scale, sa_tensor *out, float *lse,
+                            cudaStream_t s) {
     const bool diag = (g->kind == 0) ? g->n_off > 0 : g->max_resid > 0;
     const bool csr = g->kind == 1;
     // <D, pipelines, K stages, V stages, diagonal stages, per-warp slots>,
@@ -889,3 +945,5 @@ sa_status sa_band_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v
     return csr ? launch_band_fwd<128, 1, 2, 2, 2, true, 128>(q, k, v, g, scale, out, lse, s)
                : launch_band_fwd<128, 1, 2, 2, 2, false, 128>(q, k, v, g, scale, out, lse, s);
 }
+
+}  // namespace

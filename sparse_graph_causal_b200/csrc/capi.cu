@@ -20,6 +20,7 @@ namespace {
 
 std::atomic<int64_t> g_launches{0};
 std::atomic<int> g_path{SA_PATH_AUTO};
+std::atomic<int> g_links{SA_LINKS_AUTO};
 
 // One error word per device, written by kernels whose waits are bounded.
 __device__ int g_device_error = 0;
@@ -171,6 +172,8 @@ GraphView make_view(const sa_graph_s *g) {
     return v;
 }
 
+int sa_link_pass_mode() { return g_links.load(); }
+
 extern "C" {
 
 const char *sparse_attn_status_string(sa_status s) {
@@ -189,6 +192,13 @@ const char *sparse_attn_status_string(sa_status s) {
 sa_status sparse_attn_set_path(int32_t path) {
     if (path != SA_PATH_AUTO && path != SA_PATH_GATHER) return SA_ERR_INVALID_ARG;
     g_path.store(path);
+    return SA_OK;
+}
+
+sa_status sparse_attn_set_link_pass(int32_t mode) {
+    if (mode != SA_LINKS_AUTO && mode != SA_LINKS_SPLIT && mode != SA_LINKS_ONE_PASS)
+        return SA_ERR_INVALID_ARG;
+    g_links.store(mode);
     return SA_OK;
 }
 

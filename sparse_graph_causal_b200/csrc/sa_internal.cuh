@@ -56,6 +56,7 @@ void sa_prof_end(cudaStream_t s);
         sa_count_launch();             \
     } while (0)
 int *sa_device_error_word();  // device address of this device's error word
+int sa_link_pass_mode();      // sparse_attn_set_link_pass's setting
 
 
 #define SA_DEVERR_TIMEOUT 1

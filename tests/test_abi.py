@@ -55,6 +55,7 @@ def test_host_side_rejections():
     assert lib.sparse_attn_graph_build_csr(0, None, None, 0, 0, None, ctypes.byref(h)) == 1
     assert lib.sparse_attn_fwd(None, None, None, None, 1.0, None, None, None) == 1
     assert lib.sparse_attn_set_path(7) == 1
+    assert lib.sparse_attn_set_link_pass(3) == 1 and lib.sparse_attn_set_link_pass(-1) == 1
     assert sa.sparse_attn_status_string(2) == "invalid graph"
 
 

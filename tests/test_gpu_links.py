@@ -1,0 +1,89 @@
+"""The forward's second pass over the long distance links of a structured
+graph: the band kernel takes the window and the links shorter than 2^15
+rows, the link pass the rest, class by class, and merges them into out and
+lse.  The automatic choice takes it only when K and V hold 8 GiB or more
+(the extreme-length workload); here SA_LINKS_SPLIT forces it on sizes whose
+K and V exceed L2.  Checked against the gather kernels (every edge in one
+pass) on every row, against the one-pass band kernel, and against the oracle
+on sampled rows, for D = 32, 64, 128 and grouped heads."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_util import compact, compare, gather_rows, local_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def _wl(name, H, Hkv, T, D, kmax, seed):
+    return synth.Workload(name=name, B=1, H=H, T=T, D=D, dtype="bf16", W=32,
+                          exps=tuple(range(0, kmax + 1)), input_std=1.0,
+                          scale=1.0 / math.sqrt(D), seed=seed, Hkv=Hkv, bwd=False)
+
+
+CASES = [
+    _wl("links_d64", 1, 1, 1 << 19, 64, 18, 71),
+    _wl("links_gqa", 2, 1, 1 << 19, 64, 18, 72),
+    _wl("links_d32", 1, 1, 1 << 20, 32, 19, 73),
+    _wl("links_d128", 1, 1, 1 << 18, 128, 17, 74),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_link_pass_matches_one_pass_and_oracle(oracle_lib, w):
+    import sparse_graph_causal_b200 as sa
+    o = oracle_lib
+    g = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+    x = synth.make_qkv(w, device="cuda", with_dout=False)
+    sa.sparse_attn_set_link_pass(sa.SA_LINKS_SPLIT)
+    try:
+        sa.sparse_attn_profile_begin(True)
+        out, lse = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+        prof = sa.sparse_attn_profile_end()
+        sa.sparse_attn_check_device()
+        assert set(prof) == {"band_fwd", "link_pass"}, prof
+        # one pass (the automatic choice at this size)
+        sa.sparse_attn_set_link_pass(sa.SA_LINKS_AUTO)
+        sa.sparse_attn_profile_begin(True)
+        out2, lse2 = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+        prof = sa.sparse_attn_profile_end()
+        sa.sparse_attn_check_device()
+        assert set(prof) == {"band_fwd"}, prof
+    finally:
+        sa.sparse_attn_set_link_pass(sa.SA_LINKS_AUTO)
+    compare(out, out2.double().cpu().numpy(), w.dtype, f"{w.name} out vs band one pass")
+    compare(lse, lse2.double().cpu().numpy(), w.dtype, f"{w.name} lse vs band one pass")
+    del out2, lse2
+    # every edge in one pass, on the gather kernels
+    sa.sparse_attn_set_path(sa.SA_PATH_GATHER)
+    try:
+        out1, lse1 = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+        sa.sparse_attn_check_device()
+    finally:
+        sa.sparse_attn_set_path(sa.SA_PATH_AUTO)
+    compare(out, out1.double().cpu().numpy(), w.dtype, f"{w.name} out vs one pass")
+    compare(lse, lse1.double().cpu().numpy(), w.dtype, f"{w.name} lse vs one pass")
+    # the oracle on sampled rows: random ones, the rows around the first long
+    # link (2^15) and around the class boundaries of the second pass
+    span = 1 << 15
+    extra = [span - 1, span, span + 1, span + 127, span + 128, 2 * span - 1, 2 * span + 200,
+             w.T - 129, w.T - 128]
+    rows = np.unique(np.concatenate([synth.sample_rows(w.T, 768, seed=w.seed), extra]))
+    rp, ci = local_rows(o, rows, w.W, w.exps)
+    keys, local = compact(rp, ci)
+    G = w.H // w.kv_heads
+    for bh in range(w.H):
+        kvbh = bh // G
+        q = gather_rows(x["q"], bh, rows, w.dtype)
+        k = gather_rows(x["k"], kvbh, keys, w.dtype)
+        v = gather_rows(x["v"], kvbh, keys, w.dtype)
+        rout, rlse = o.fwd(q, k, v, rp, local, w.scale, dtype=w.dtype)
+        idx = torch.as_tensor(rows, device="cuda")
+        compare(out[0, bh].index_select(0, idx), rout, w.dtype, f"{w.name}[{bh}] out")
+        compare(lse[0, bh].index_select(0, idx), rlse, w.dtype, f"{w.name}[{bh}] lse")
+    del x, out, lse, out1, lse1
+    g.close()
+    torch.cuda.empty_cache()

@@ -468,6 +468,7 @@ def time_workload(sa, w: synth.Workload, dev, rank, world, dist, steps, warmup, 
                    "l2": "256 MiB buffer written between timed steps",
                    "timed_step": ("CUDA-graph replay of " if cuda_graph is not None else
                                   "eager ") + ("fwd+bwd" if do_bwd else "fwd"),
+                   "link_pass": args.link_pass if args is not None else "auto",
                    "parallelism": f"replicas x{world}"},
         "steps": steps, "ms_per_step": ms_step, "edges_per_s": E * world / (ms_step * 1e-3),
         "fwd_ms": fwd_ms, "fwd_edges_per_s": E * world / (fwd_ms * 1e-3),
@@ -625,6 +626,8 @@ def run_gpu(args, dist, rank, world):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = synth.WORKLOADS[args.workload]
+    sa.sparse_attn_set_link_pass({"auto": sa.SA_LINKS_AUTO, "split": sa.SA_LINKS_SPLIT,
+                                  "one": sa.SA_LINKS_ONE_PASS}[args.link_pass])
     r = time_workload(sa, w, dev, rank, world, dist, args.steps, args.warmup, args.fwd_only,
                       use_graph=not args.no_graph, want_e2e=not args.no_e2e, args=args)
     torch.cuda.empty_cache()
@@ -636,7 +639,8 @@ def run_gpu(args, dist, rank, world):
                 continue
             wx = synth.WORKLOADS[name]
             timer = {"attn": time_workload, "dist": time_dist, "decode": time_decode}[wx.kind]
-            extra[name] = timer(sa, wx, dev, rank, world, dist, args.extra_steps, 3, False)
+            extra[name] = timer(sa, wx, dev, rank, world, dist, args.extra_steps, 3, False,
+                                args=args)
             torch.cuda.empty_cache()
 
     cpu = None
@@ -758,6 +762,9 @@ def main():
                     help="time only --workload, not the other named workloads")
     ap.add_argument("--extra-steps", type=int, default=5,
                     help="timed steps of each of the other named workloads")
+    ap.add_argument("--link-pass", default="auto", choices=["auto", "split", "one"],
+                    help="long distance links in a second forward pass: the library's "
+                         "automatic choice, always, or never (sparse_attn_set_link_pass)")
     args = ap.parse_args()
     dist, rank, world = dist_setup(args.gpus)
     try:

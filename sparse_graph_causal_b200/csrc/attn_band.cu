@@ -657,22 +657,46 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 tc::tmem_ld_wait();
                 const bool pos = c2 >= 0.f;
                 const float ext = pos ? -INFINITY : INFINITY;
+                // 16-column chunks holding a kept key of some row of this warp;
+                // the others get no masking, max or exponentials (P = 0 there)
+                uint32_t live = (1u << (BN / 16)) - 1u;
                 if (need_mask) {
+                    live = 0u;
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) s[c] = ((keep >> c) & 1ull) ? s[c] : ext;
+                    for (int c16 = 0; c16 < BN / 16; ++c16)
+                        if (__any_sync(0xffffffffu, ((keep >> (16 * c16)) & 0xffffull) != 0ull))
+                            live |= 1u << c16;
+#pragma unroll
+                    for (int c16 = 0; c16 < BN / 16; ++c16) {
+                        if ((live >> c16) & 1u) {
+#pragma unroll
+                            for (int c = 16 * c16; c < 16 * c16 + 16; ++c)
+                                s[c] = ((keep >> c) & 1ull) ? s[c] : ext;
+                        }
+                    }
                 }
                 float mr[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) mr[x] = ext;
-                if (pos) {
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) mr[c & 7] = fmaxf(mr[c & 7], s[c]);
+                for (int c16 = 0; c16 < BN / 16; ++c16) {
+                    if ((live >> c16) & 1u) {
+                        if (pos) {
+#pragma unroll
+                            for (int c = 16 * c16; c < 16 * c16 + 16; ++c)
+                                mr[c & 7] = fmaxf(mr[c & 7], s[c]);
+                        } else {
+#pragma unroll
+                            for (int c = 16 * c16; c < 16 * c16 + 16; ++c)
+                                mr[c & 7] = fminf(mr[c & 7], s[c]);
+                        }
+                    }
+                }
+                if (pos) {
 #pragma unroll
                     for (int x = 4; x > 0; x >>= 1)
                         for (int y = 0; y < x; ++y) mr[y] = fmaxf(mr[y], mr[y + x]);
                 } else {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) mr[c & 7] = fminf(mr[c & 7], s[c]);
 #pragma unroll
                     for (int x = 4; x > 0; x >>= 1)
                         for (int y = 0; y < x; ++y) mr[y] = fminf(mr[y], mr[y + x]);
@@ -710,19 +734,15 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 float ls[4] = {0.f, 0.f, 0.f, 0.f};
                 uint32_t pw[BN / 2];
                 if (need_mask) {
-                    // only 16-column chunks that hold a kept score of some row of
-                    // this warp do exponentials; the rest of P is zero
+                    // a masked score is the extreme whose scaled value is -inf
+                    // (the scale is nonzero on this path), so its p is 0
 #pragma unroll
                     for (int c16 = 0; c16 < BN / 16; ++c16) {
-                        bool live = false;
-#pragma unroll
-                        for (int c = 16 * c16; c < 16 * c16 + 16; ++c) live |= (s[c] != ext);
-                        if (__any_sync(0xffffffffu, live)) {
+                        if ((live >> c16) & 1u) {
 #pragma unroll
                             for (int c = 8 * c16; c < 8 * c16 + 8; ++c) {
-                                const float x0 = s[2 * c], x1 = s[2 * c + 1];
-                                const float p0 = (x0 != ext) ? tc::ex2(fmaf(x0, c2, -m_use)) : 0.f;
-                                const float p1 = (x1 != ext) ? tc::ex2(fmaf(x1, c2, -m_use)) : 0.f;
+                                const float p0 = tc::ex2(fmaf(s[2 * c], c2, -m_use));
+                                const float p1 = tc::ex2(fmaf(s[2 * c + 1], c2, -m_use));
                                 ls[c & 3] += p0 + p1;
                                 pw[c] = tc::pack_bf16x2(p0, p1);
                             }

@@ -388,7 +388,9 @@ sa_status sparse_attn_fwd(const sa_tensor *q, const sa_tensor *k, const sa_tenso
     if (!lse || !aligned16(lse) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
     cudaStream_t s = as_stream(stream);
     const GraphView gv = make_view(g);
-    if (g_path.load() == SA_PATH_AUTO && sa_band_fwd_supported(q, g))
+    // (the band forward masks through the scale's sign: a zero scale, which
+    // makes every kept score 0, takes the gather kernels)
+    if (g_path.load() == SA_PATH_AUTO && scale != 0.f && sa_band_fwd_supported(q, g))
         return sa_band_fwd(q, k, v, g, gv, scale, out, lse, s);
     return sa_gather_fwd(q, k, v, gv, scale, out, lse, s);
 }

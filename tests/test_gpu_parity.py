@@ -47,6 +47,8 @@ CASES = [
     _wl("d64_self_only", 1, 2, 129, 64, "bf16", 1, (0, 3, 5)),
     _wl("d64_full", 1, 1, 520, 64, "bf16", 520, ()),
     _wl("d64_small_values", 1, 4, 700, 64, "bf16", 32, range(0, 10), std=0.125),
+    # scale 0: every kept score is 0 (uniform weights over each row's keys)
+    _wl("d64_zero_scale", 1, 2, 300, 64, "bf16", 32, range(0, 9), mult=0.0),
     _wl("d128_w200", 1, 2, 1000, 128, "bf16", 200, (8, 9)),
     _wl("d128_band", 2, 1, 777, 128, "bf16", 256, ()),
     _wl("d32_bf16", 1, 2, 200, 32, "bf16", 16, range(0, 8)),

@@ -774,25 +774,45 @@ band_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             if (!wait(p, L::bPVDone + (int)(gb_last & 1), (gb_last >> 1) & 1)) break;
             tc::tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            __nv_bfloat16 *orow = a.out + ((size_t)bh * (size_t)T + (size_t)i) * DG;
+            if constexpr (DG % 64 == 0) {
+                // the warp's 32 rows in whole sectors, staged in O's first
+                // columns (O is read out first)
+                uint32_t pk[DG / 2];
 #pragma unroll
-            for (int c = 0; c < DG; c += 32) {
-                uint32_t w[32];
-                tc::tmem_ld32(tO + c, w);
-                tc::tmem_ld_wait();
-                if (i < T) {
+                for (int c = 0; c < DG; c += 32) {
+                    uint32_t w[32];
+                    tc::tmem_ld32(tO + c, w);
+                    tc::tmem_ld_wait();
 #pragma unroll
-                    for (int x = 0; x < 32; x += 8) {
-                        uint4 o4;
-                        o4.x = tc::pack_bf16x2(__uint_as_float(w[x]) * inv,
-                                               __uint_as_float(w[x + 1]) * inv);
-                        o4.y = tc::pack_bf16x2(__uint_as_float(w[x + 2]) * inv,
-                                               __uint_as_float(w[x + 3]) * inv);
-                        o4.z = tc::pack_bf16x2(__uint_as_float(w[x + 4]) * inv,
-                                               __uint_as_float(w[x + 5]) * inv);
-                        o4.w = tc::pack_bf16x2(__uint_as_float(w[x + 6]) * inv,
-                                               __uint_as_float(w[x + 7]) * inv);
-                        *(uint4 *)(orow + c + x) = o4;
+                    for (int x = 0; x < 32; x += 2)
+                        pk[(c + x) / 2] = tc::pack_bf16x2(__uint_as_float(w[x]) * inv,
+                                                          __uint_as_float(w[x + 1]) * inv);
+                }
+                const int64_t row0 = (int64_t)q0 + 32 * wq;
+                const int64_t nr = T - row0;
+                tc::tmem_rows_store<DG / 2>(tO, pk, a.out + ((size_t)bh * (size_t)T + row0) * DG, DG,
+                                            nr < 0 ? 0 : (nr > 32 ? 32 : (int)nr), lane);
+            } else {
+                __nv_bfloat16 *orow = a.out + ((size_t)bh * (size_t)T + (size_t)i) * DG;
+    #pragma unroll
+                for (int c = 0; c < DG; c += 32) {
+                    uint32_t w[32];
+                    tc::tmem_ld32(tO + c, w);
+                    tc::tmem_ld_wait();
+                    if (i < T) {
+    #pragma unroll
+                        for (int x = 0; x < 32; x += 8) {
+                            uint4 o4;
+                            o4.x = tc::pack_bf16x2(__uint_as_float(w[x]) * inv,
+                                                   __uint_as_float(w[x + 1]) * inv);
+                            o4.y = tc::pack_bf16x2(__uint_as_float(w[x + 2]) * inv,
+                                                   __uint_as_float(w[x + 3]) * inv);
+                            o4.z = tc::pack_bf16x2(__uint_as_float(w[x + 4]) * inv,
+                                                   __uint_as_float(w[x + 5]) * inv);
+                            o4.w = tc::pack_bf16x2(__uint_as_float(w[x + 6]) * inv,
+                                                   __uint_as_float(w[x + 7]) * inv);
+                            *(uint4 *)(orow + c + x) = o4;
+                        }
                     }
                 }
             }

@@ -252,6 +252,32 @@ __device__ __forceinline__ void tmem_row_to_global(uint32_t taddr, float mul, __
 }
 
 // Pack n fp32 values as n/2 bf16 pairs (round to nearest even).
+// TMEM rows (D fp32 columns, this warp's 32 lanes from taddr) times `mul` as
+// bf16 to global memory, DG columns per row: in whole sectors through the
+// accumulator's own first columns (tc::tmem_rows_store) when DG is a multiple
+// of 64, else row by row.  dst: the warp's row 0; rows >= nrows not written.
+template <int DG>
+__device__ __forceinline__ void tmem_rows_to_global(uint32_t taddr, float mul, __nv_bfloat16 *dst,
+                                                    int64_t nrows_in, int lane) {
+    const int nrows = nrows_in < 0 ? 0 : (nrows_in > 32 ? 32 : (int)nrows_in);
+    if constexpr (DG % 64 == 0) {
+        uint32_t pk[DG / 2];
+#pragma unroll
+        for (int c = 0; c < DG; c += 32) {
+            uint32_t w[32];
+            tc::tmem_ld32(taddr + c, w);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; x += 2)
+                pk[(c + x) / 2] =
+                    tc::pack_bf16x2(__uint_as_float(w[x]) * mul, __uint_as_float(w[x + 1]) * mul);
+        }
+        tc::tmem_rows_store<DG / 2>(taddr, pk, dst, DG, nrows, lane);
+    } else {
+        tmem_row_to_global<DG>(taddr, mul, dst + (size_t)lane * DG, lane < nrows);
+    }
+}
+
 template <int N>
 __device__ __forceinline__ void pack_bf16_row(const float *x, uint32_t *w) {
 #pragma unroll
@@ -799,7 +825,9 @@ band_bwd_dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             if (!ok) break;
             if (!wait(p, L::bDQDone + (int)(gb_last % SB), (gb_last / SB) & 1)) break;
             tc::tc_fence_after();
-            tmem_row_to_global<DG>(tDQ, a.scale, a.dq + grow * DG, row_ok);
+            tmem_rows_to_global<DG>(tDQ, a.scale,
+                                    a.dq + ((size_t)bh * (size_t)T + (size_t)(q0 + 32 * wq)) * DG,
+                                    T - (q0 + 32 * wq), lane);
         }
     }
     tc::tc_fence_before();
@@ -1404,8 +1432,9 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             if (!ok) break;
             if (!wait(p, L::bDKVDone + (int)(gb_last % SB), (gb_last / SB) & 1)) break;
             tc::tc_fence_after();
-            tmem_row_to_global<DG>(tDV, 1.f, a.dv + grow * DG, row_ok);
-            tmem_row_to_global<DG>(tDK, a.scale, a.dk + grow * DG, row_ok);
+            const size_t wrow = (size_t)kvbh * (size_t)T + (size_t)(k0 + 32 * wq);
+            tmem_rows_to_global<DG>(tDV, 1.f, a.dv + wrow * DG, T - (k0 + 32 * wq), lane);
+            tmem_rows_to_global<DG>(tDK, a.scale, a.dk + wrow * DG, T - (k0 + 32 * wq), lane);
         }
     }
     tc::tc_fence_before();

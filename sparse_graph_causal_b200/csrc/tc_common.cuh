@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace tc {
@@ -236,6 +237,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
         : "r"(taddr));
 }
 
+// Shape 16x256b, .x4: 16 TMEM lanes from taddr's lane, 32 columns.  Thread t
+// receives, for repetition j = 0..3 (columns 8j .. 8j+7): r[4j], r[4j+1] =
+// lane t/4, columns 8j + 2(t%4) and 8j + 2(t%4) + 1; r[4j+2], r[4j+3] = lane
+// 8 + t/4, the same columns.
+__device__ __forceinline__ void tmem_ld16x256_x4(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -288,6 +303,40 @@ __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t *r) {
 #pragma unroll
     for (int c = 0; c + 32 <= N; c += 32) tmem_st32(taddr + c, r + c);
     if (N % 32 == 16) tmem_st16(taddr + (N - 16), r + (N - 16));
+}
+
+// The rows of a warp's 32 TMEM lanes to global memory in whole 32-byte
+// sectors.  w: this thread's row (TMEM lane 32 w + lane) as N bf16 pairs (N a
+// multiple of 32); it is staged in N columns at taddr (lane 0 of the warp's
+// lanes; columns the caller no longer needs) and read back in the 16x256b
+// layout, in which 4 lanes hold 32 contiguous bytes of one row, so each
+// store instruction writes 8 rows x 32 bytes instead of 32 rows x 16 bytes.
+// dst: the warp's row 0; pitch in elements; rows >= nrows are not written.
+template <int N>
+__device__ __forceinline__ void tmem_rows_store(uint32_t taddr, const uint32_t *w,
+                                                __nv_bfloat16 *dst, int64_t pitch, int nrows,
+                                                int lane) {
+    tmem_st_n<N>(taddr, w);
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int q = 0; q < N / 32; ++q) {
+            uint32_t r[16];
+            tmem_ld16x256_x4(taddr + ((uint32_t)(16 * h) << 16) + 32 * q, r);
+            tmem_ld_wait();
+            const int row0 = 16 * h + (lane >> 2), row1 = row0 + 8;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int word = 32 * q + 8 * j + 2 * (lane & 3);
+                if (row0 < nrows)
+                    *(uint2 *)(dst + (int64_t)row0 * pitch + 2 * word) = make_uint2(r[4 * j], r[4 * j + 1]);
+                if (row1 < nrows)
+                    *(uint2 *)(dst + (int64_t)row1 * pitch + 2 * word) =
+                        make_uint2(r[4 * j + 2], r[4 * j + 3]);
+            }
+        }
+    }
 }
 
 __device__ __forceinline__ void tmem_st_wait() {

@@ -305,12 +305,15 @@ __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t *r) {
     if (N % 32 == 16) tmem_st16(taddr + (N - 16), r + (N - 16));
 }
 
-// The rows of a warp's 32 TMEM lanes to global memory in whole 32-byte
-// sectors.  w: this thread's row (TMEM lane 32 w + lane) as N bf16 pairs (N a
-// multiple of 32); it is staged in N columns at taddr (lane 0 of the warp's
-// lanes; columns the caller no longer needs) and read back in the 16x256b
-// layout, in which 4 lanes hold 32 contiguous bytes of one row, so each
-// store instruction writes 8 rows x 32 bytes instead of 32 rows x 16 bytes.
+// The rows of a warp's 32 TMEM lanes to global memory in 64-byte runs.  w:
+// this thread's row (TMEM lane 32 w + lane) as N bf16 pairs (N a multiple of
+// 32); it is staged in N columns at taddr (lane 0 of the warp's lanes;
+// columns the caller no longer needs) and read back in the 16x256b layout, in
+// which the 4 lanes of a quad hold 32 contiguous bytes of one row per
+// repetition; neighbouring lanes then swap one 8-byte half, so that for two
+// repetitions the even lanes hold the first's 16-byte quarters and the odd
+// lanes the second's, and each store instruction writes 8 rows x 64 bytes
+// (instead of 32 rows x 16 bytes from the row-per-thread layout).
 // dst: the warp's row 0; pitch in elements; rows >= nrows are not written.
 template <int N>
 __device__ __forceinline__ void tmem_rows_store(uint32_t taddr, const uint32_t *w,
@@ -325,15 +328,22 @@ __device__ __forceinline__ void tmem_rows_store(uint32_t taddr, const uint32_t *
             uint32_t r[16];
             tmem_ld16x256_x4(taddr + ((uint32_t)(16 * h) << 16) + 32 * q, r);
             tmem_ld_wait();
-            const int row0 = 16 * h + (lane >> 2), row1 = row0 + 8;
+            const bool odd = lane & 1;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int word = 32 * q + 8 * j + 2 * (lane & 3);
-                if (row0 < nrows)
-                    *(uint2 *)(dst + (int64_t)row0 * pitch + 2 * word) = make_uint2(r[4 * j], r[4 * j + 1]);
-                if (row1 < nrows)
-                    *(uint2 *)(dst + (int64_t)row1 * pitch + 2 * word) =
-                        make_uint2(r[4 * j + 2], r[4 * j + 3]);
+            for (int jp = 0; jp < 4; jp += 2) {
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {  // row lane/4 or lane/4 + 8
+                    const uint32_t a0 = r[4 * jp + 2 * hr], a1 = r[4 * jp + 2 * hr + 1];
+                    const uint32_t b0 = r[4 * jp + 4 + 2 * hr], b1 = r[4 * jp + 4 + 2 * hr + 1];
+                    // even lanes keep repetition jp and take the odd
+                    // neighbour's pair of it; odd lanes the other way round
+                    const uint32_t g0 = __shfl_xor_sync(0xffffffffu, odd ? a0 : b0, 1);
+                    const uint32_t g1 = __shfl_xor_sync(0xffffffffu, odd ? a1 : b1, 1);
+                    const uint4 v = odd ? make_uint4(g0, g1, b0, b1) : make_uint4(a0, a1, g0, g1);
+                    const int word = 32 * q + 8 * (jp + (odd ? 1 : 0)) + 2 * (lane & 2);
+                    const int row = 16 * h + (lane >> 2) + 8 * hr;
+                    if (row < nrows) *(uint4 *)(dst + (int64_t)row * pitch + 2 * word) = v;
+                }
             }
         }
     }

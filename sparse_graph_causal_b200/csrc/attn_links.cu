@@ -34,7 +34,8 @@
 namespace {
 
 constexpr int BM = 128;    // queries per tile
-constexpr int kDS = 3;     // ring stages per warp
+constexpr int kDS = 3;         // ring stages per warp
+constexpr int kMinBlocks = 2;  // CTAs per SM the register budget must allow
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units, as in the band kernel
@@ -82,8 +83,8 @@ struct LinkLayout {
 // accumulated).  A link's K and V rows for the 16 queries of a warp are 16
 // contiguous rows of each tensor (keys i - o), copied with 16-byte cp.async
 // copies into the warp's DS-stage ring, DS links ahead of their use.
-template <int D, int DS>
-__global__ void __launch_bounds__(256) link_pass_kernel(const LinkArgs a) {
+template <int D, int DS, int MINB>
+__global__ void __launch_bounds__(256, MINB) link_pass_kernel(const LinkArgs a) {
     using L = LinkLayout<D, DS>;
     constexpr int H2 = D / 2;              // columns per lane
     constexpr int NCH = H2 / 8;            // 16-byte chunks per lane and row
@@ -91,14 +92,15 @@ __global__ void __launch_bounds__(256) link_pass_kernel(const LinkArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
 
     // this CTA's tile: slices in order, then class by class inside a slice
-    const int64_t per_slice = a.C * a.G;
-    const int64_t bh = (int64_t)blockIdx.x / per_slice;
-    const int64_t rem = (int64_t)blockIdx.x - bh * per_slice;
-    const int64_t cls = rem / a.G, jt = rem - cls * a.G;
-    const int64_t t = jt * a.C + cls;
-    if (t >= a.nt) return;
-    const int64_t q0 = t * BM;
-    const int64_t last = (q0 + BM - 1 < a.T - 1) ? q0 + BM - 1 : a.T - 1;
+    // (32-bit: the launcher keeps the block count and T below 2^31)
+    const uint32_t C = (uint32_t)a.C, G = (uint32_t)a.G, per_slice = C * G;
+    const uint32_t bh = blockIdx.x / per_slice, rem = blockIdx.x - bh * per_slice;
+    const uint32_t cls = rem / G, jt = rem - cls * G;
+    const uint32_t t = jt * C + cls;
+    if (t >= (uint32_t)a.nt) return;
+    const int32_t T = (int32_t)a.T;
+    const int32_t q0 = (int32_t)t * BM;
+    const int32_t last = (q0 + BM - 1 < T - 1) ? q0 + BM - 1 : T - 1;
     // the links this tile's rows reach (the longest first: keys ascending)
     int nd = 0;
     for (int x = 0; x < a.n_off; ++x) nd += (a.offs[x] <= last) ? 1 : 0;
@@ -107,12 +109,13 @@ __global__ void __launch_bounds__(256) link_pass_kernel(const LinkArgs a) {
 
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int x = lane >> 1, hf = lane & 1;
-    const int64_t i0 = q0 + 16 * w, i = i0 + x;
-    const bool row_ok = i < a.T;
-    const int64_t kvbh = (bh / a.H) * a.Hkv + (bh % a.H) / (a.H / a.Hkv);
-    const __nv_bfloat16 *kslice = a.k + (size_t)kvbh * (size_t)a.T * D;
-    const __nv_bfloat16 *vslice = a.v + (size_t)kvbh * (size_t)a.T * D;
-    const size_t grow = (size_t)bh * (size_t)a.T + (size_t)i;
+    const int32_t i0 = q0 + 16 * w, i = i0 + x;
+    const bool row_ok = i < T;
+    const uint32_t H = (uint32_t)a.H, Hkv = (uint32_t)a.Hkv;
+    const uint32_t kvbh = (bh / H) * Hkv + (bh % H) / (H / Hkv);
+    const __nv_bfloat16 *kslice = a.k + (size_t)kvbh * (size_t)T * D;
+    const __nv_bfloat16 *vslice = a.v + (size_t)kvbh * (size_t)T * D;
+    const size_t grow = (size_t)bh * (size_t)T + (size_t)i;
     uint8_t *ring = smem_raw + w * L::kWarpRing;
     const uint32_t ring_s = tc::smem_u32(ring);
 
@@ -128,21 +131,32 @@ __global__ void __launch_bounds__(256) link_pass_kernel(const LinkArgs a) {
         qw[4 * c + 3] = w4.w;
     }
 
+    // this lane's copies of a slot, the same for every slot: row xr of the
+    // warp's 16, chunk kc; the destination in the stage and the source offset
+    // from the slot's first key row
+    int xr[NIT];
+    uint32_t doff[NIT], soff[NIT];
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) {
+        const int b = (it * 32 + lane) * 16;
+        xr[it] = b / L::kRowBytes;
+        const int kc = (b % L::kRowBytes) / 16;
+        doff[it] = L::off(xr[it], kc);
+        soff[it] = (uint32_t)(xr[it] * D + 8 * kc);
+    }
     // copies of slot d into stage st (nothing past the last slot, or for rows
     // before the link's reach or past the sequence); one commit group each
     auto issue = [&](int st, int d) {
         if (d < nd) {
-            const int64_t kb = i0 - a.offs[dfirst + d];  // key of the warp's first query
+            const int32_t kb = i0 - a.offs[dfirst + d];  // key of the warp's first query
+            const int64_t kbd = (int64_t)kb * D;
             const uint32_t sk = ring_s + st * L::kStage, sv = sk + L::kPart;
 #pragma unroll
             for (int it = 0; it < NIT; ++it) {
-                const int b = (it * 32 + lane) * 16;
-                const int xr = b / L::kRowBytes, kc = (b % L::kRowBytes) / 16;
-                const int64_t key = kb + xr;
-                if (key >= 0 && i0 + xr < a.T) {
-                    const size_t src = (size_t)key * D + 8 * kc;
-                    tc::cp_async16(sk + L::off(xr, kc), kslice + src);
-                    tc::cp_async16(sv + L::off(xr, kc), vslice + src);
+                if (kb + xr[it] >= 0 && i0 + xr[it] < T) {
+                    const int64_t src = kbd + soff[it];
+                    tc::cp_async16(sk + doff[it], kslice + src);
+                    tc::cp_async16(sv + doff[it], vslice + src);
                 }
             }
         }
@@ -228,14 +242,14 @@ __global__ void __launch_bounds__(256) link_pass_kernel(const LinkArgs a) {
     if (hf == 0) a.lse[grow] = (M + tc::lg2(den)) * kLn2;
 }
 
-template <int D, int DS>
+template <int D, int DS, int MINB>
 sa_status launch_link_pass(const LinkArgs &a, int64_t BH, cudaStream_t s) {
     using L = LinkLayout<D, DS>;
     const int64_t blocks = BH * a.C * a.G;
-    if (blocks > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
-    SA_CUDA_TRY(sa_smem_optin((const void *)link_pass_kernel<D, DS>, L::kAlloc));
+    if (blocks > 0x7fffffffLL || a.T >= ((int64_t)1 << 31)) return SA_ERR_UNSUPPORTED;
+    SA_CUDA_TRY(sa_smem_optin((const void *)link_pass_kernel<D, DS, MINB>, L::kAlloc));
     SA_LAUNCH("link_pass", s,
-              link_pass_kernel<D, DS><<<(unsigned)blocks, 32 * L::kWarps, L::kAlloc, s>>>(a));
+              link_pass_kernel<D, DS, MINB><<<(unsigned)blocks, 32 * L::kWarps, L::kAlloc, s>>>(a));
     SA_CUDA_TRY(cudaGetLastError());
     return SA_OK;
 }
@@ -268,9 +282,9 @@ sa_status sa_link_pass(const sa_tensor *q, const sa_tensor *k, const sa_tensor *
     a.scale2 = scale * kLog2e;
     const int64_t BH = q->B * q->H;
     switch (q->D) {
-        case 32: return launch_link_pass<32, kDS>(a, BH, s);
-        case 64: return launch_link_pass<64, kDS>(a, BH, s);
-        case 128: return launch_link_pass<128, kDS>(a, BH, s);
+        case 32: return launch_link_pass<32, kDS, kMinBlocks>(a, BH, s);
+        case 64: return launch_link_pass<64, kDS, kMinBlocks>(a, BH, s);
+        case 128: return launch_link_pass<128, kDS, 1>(a, BH, s);
     }
     return SA_ERR_UNSUPPORTED;
 }

@@ -29,6 +29,8 @@ CASES = [
     _wl("links_gqa", 2, 1, 1 << 19, 64, 18, 72),
     _wl("links_d32", 1, 1, 1 << 20, 32, 19, 73),
     _wl("links_d128", 1, 1, 1 << 18, 128, 17, 74),
+    # ragged: the last tile partial, the last class one tile short
+    _wl("links_ragged", 1, 1, (1 << 19) + 77, 64, 18, 75),
 ]
 
 

@@ -33,7 +33,7 @@
 
 namespace {
 
-constexpr int BM = 128;    // queries per tile
+constexpr int BM = 128;        // queries per tile
 constexpr int kDS = 3;         // ring stages per warp
 constexpr int kMinBlocks = 2;  // CTAs per SM the register budget must allow
 constexpr float kLog2e = 1.4426950408889634f;

@@ -306,7 +306,7 @@ __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t *r) {
 }
 
 // The rows of a warp's 32 TMEM lanes to global memory in 64-byte runs.  w:
-// this thread's row (TMEM lane 32 w + lane) as N bf16 pairs (N a multiple of
+// this thread's row (TMEM lane 32 x warp + lane) as N bf16 pairs (N a multiple of
 // 32); it is staged in N columns at taddr (lane 0 of the warp's lanes;
 // columns the caller no longer needs) and read back in the 16x256b layout, in
 // which the 4 lanes of a quad hold 32 contiguous bytes of one row per

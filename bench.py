@@ -310,10 +310,10 @@ def gather_model_bytes(w: synth.Workload, g, dev) -> tuple:
 
 def two_pass_model_bytes(w: synth.Workload) -> tuple:
     """Bytes of the two-pass forward (band kernel, then the link pass over the
-    links of at least 2^15 rows in class order, which keeps their rows in
+    links of at least 2^13 rows in class order, which keeps their rows in
     L2): the compulsory bytes, plus the link pass's own q read, out and lse
     read and written, and one more read of K and V (each class's rows once).
-    The first pass's links are all shorter than 2^15 rows and hit L2."""
+    The first pass's links are all shorter than 2^13 rows and hit L2."""
     es = w.elem_size
     BH, BHkv = w.B * w.H, w.B * w.kv_heads
     extra = BH * (3 * w.T * w.D * es + 8 * w.T) + BHkv * 2 * w.T * w.D * es

@@ -235,12 +235,12 @@ sa_status sparse_attn_set_path(int32_t path);
 
 /* Long distance links of a structured graph (process-wide; default
  * SA_LINKS_AUTO).  The band-kernel forward can take the links of at least
- * 2^15 rows (when all such links are multiples of 2^15, e.g. powers of two)
+ * 2^13 rows (when all such links are multiples of 2^13, e.g. powers of two)
  * in a second pass that runs the tiles in an order keeping their K/V rows in
  * L2 ("Longer Attention Span ...", Abstract: single-GPU sequences of 160 M
  * tokens), merged into out and lse by the online-softmax rule.  Results are
  * the same up to rounding (pass 1's out is read back in the input dtype).
- *  SA_LINKS_AUTO     two passes when K and V together hold 8 GiB or more and
+ *  SA_LINKS_AUTO     two passes when K and V together hold 2 GiB or more and
  *                    at least three such links exist (below that one pass was
  *                    measured faster on B200)
  *  SA_LINKS_SPLIT    two passes whenever such a link exists

@@ -910,18 +910,19 @@ bool sa_band_fwd_supported(const sa_tensor *q, const sa_graph_s *g) {
 namespace {
 
 // Links of at least kLongSpan rows, all multiples of kLongSpan, can go to a
-// second pass (attn_links.cu): in sequence order their rows have left L2 by
+// second pass (attn_links.cu): in sequence order their rows are old in L2 by
 // the time a link reads them (the sweep reads ~6 KB of K/V per row of
-// progress, so rows 2^15 back are ~200 MB old), while the second pass runs
-// the tiles in an order that keeps them there.  The second pass re-reads q,
-// out and lse and its per-edge cost is about that of the band kernel's
-// distance blocks when they hit L2, so it pays only when many long links miss:
-// on B200 one pass was faster at T = 2^23 (K and V 2 GiB: 4.8 vs 5.1 ms) and
-// two passes at 2^25 (22.8 vs 22.1 ms), 2^26 (49.8 vs 47.0) and 2^27 (114 vs
-// 101), with window 32 and links 2^k.
-constexpr int64_t kLongSpan = (int64_t)1 << 15;
+// progress, so rows 2^13 back are ~50 MB old, 2^15 back ~200 MB), while the
+// second pass runs the tiles in an order that keeps them there.  The second
+// pass re-reads q, out and lse, so it pays only on long sequences.  Measured
+// on B200 with window 32 and links 2^k: at T = 2^27 the split at 2^13 took
+// 84.7-86.2 ms, at 2^10 89.0, 2^11 85.8, 2^12 85.5, 2^14 88.1, 2^15 89.4-90.1,
+// 2^16 95.6; with the split at 2^13 two passes beat one from T = 2^23 (K and
+// V 2 GiB: 4.36 vs 4.60 ms; 2^24 8.99 vs 10.22; 2^25 18.3 vs 22.7; 2^26 39.7
+// vs 50.4) and lose at 2^22 (2.16 vs 2.06) and below.
+constexpr int64_t kLongSpan = (int64_t)1 << 13;
 constexpr int kMinLong = 3;
-constexpr double kTwoPassBytes = 8.0 * 1024 * 1024 * 1024;  // K and V together
+constexpr double kTwoPassBytes = 2.0 * 1024 * 1024 * 1024;  // K and V together
 
 int long_links(const sa_tensor *k, const sa_graph_s *g) {
     const int mode = sa_link_pass_mode();

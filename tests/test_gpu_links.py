@@ -1,9 +1,9 @@
 """The forward's second pass over the long distance links of a structured
-graph: the band kernel takes the window and the links shorter than 2^15
+graph: the band kernel takes the window and the links shorter than 2^13
 rows, the link pass the rest, class by class, and merges them into out and
-lse.  The automatic choice takes it only when K and V hold 8 GiB or more
-(the extreme-length workload); here SA_LINKS_SPLIT forces it on sizes whose
-K and V exceed L2.  Checked against the gather kernels (every edge in one
+lse.  The automatic choice takes it only when K and V hold 2 GiB or more
+(the extreme-length workloads); here SA_LINKS_SPLIT forces it on sizes
+whose K and V are below that.  Checked against the gather kernels (every edge in one
 pass) on every row, against the one-pass band kernel, and against the oracle
 on sampled rows, for D = 32, 64, 128 and grouped heads."""
 import math
@@ -69,8 +69,8 @@ def test_link_pass_matches_one_pass_and_oracle(oracle_lib, w):
     compare(out, out1.double().cpu().numpy(), w.dtype, f"{w.name} out vs one pass")
     compare(lse, lse1.double().cpu().numpy(), w.dtype, f"{w.name} lse vs one pass")
     # the oracle on sampled rows: random ones, the rows around the first long
-    # link (2^15) and around the class boundaries of the second pass
-    span = 1 << 15
+    # link (2^13) and around the class boundaries of the second pass
+    span = 1 << 13
     extra = [span - 1, span, span + 1, span + 127, span + 128, 2 * span - 1, 2 * span + 200,
              w.T - 129, w.T - 128]
     rows = np.unique(np.concatenate([synth.sample_rows(w.T, 768, seed=w.seed), extra]))

@@ -1212,7 +1212,7 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             // key by a distance link (or by a CSR residual entry), for every
             // query head of the group, fetched by this warp itself; (p, dS) of
             // each edge comes from the dQ kernel's cache, or is recomputed from
-            // lse and Delta of the query, loaded one slot ahead
+            // lse and Delta of the query, loaded three slots ahead
             // D = 64: diagonal sums in registers, stored to TMEM after the
             // slots; D = 128: summed in TMEM directly (zeroed first)
             constexpr bool kRegAcc = D == 64;
@@ -1272,11 +1272,11 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                                      (size_t)i];
                     return make_float2(a.lse[qbh * (size_t)T + i], a.delta[qbh * (size_t)T + i]);
                 };
-                int64_t i_cur = key_of(0), i_nxt = key_of(1);
-                float2 v_cur = edge_vals(0, i_cur);
+                int64_t i_cur = key_of(0), i_nxt = key_of(1), i_n2 = key_of(2), i_n3 = key_of(3);
+                float2 v_cur = edge_vals(0, i_cur), v_nxt = edge_vals(1, i_nxt), v_n2 = edge_vals(2, i_n2);
                 auto body = [&](int d, int st) {
-                    const int64_t i_n2 = key_of(d + 2);
-                    const float2 v_nxt = edge_vals(d + 1, i_nxt);
+                    const int64_t i_n4 = key_of(d + 4);
+                    const float2 v_n3 = edge_vals(d + 3, i_n3);
                     const uint8_t *qt = pm + L::pDQ + st * L::kRow;
                     const uint8_t *dt = pm + L::pDDO + st * L::kRow;
                     float pr = 0.f, ds = 0.f;
@@ -1302,7 +1302,11 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
                     }
                     i_cur = i_nxt;
                     i_nxt = i_n2;
+                    i_n2 = i_n3;
+                    i_n3 = i_n4;
                     v_cur = v_nxt;
+                    v_nxt = v_n2;
+                    v_n2 = v_n3;
                 };
                 if constexpr (LDW) {
                     rows::warp_slots<DG, DS>(

@@ -14,6 +14,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "sa_internal.cuh"
@@ -388,6 +389,54 @@ __global__ void csr_rev_resid(int64_t T, const int64_t *rev_rowptr, int32_t Wb, 
     atomicMax(max_resid, (int)(r > 0x7fffffff ? 0x7fffffff : r));
 }
 
+// The CSR build's temporaries (28 bytes per input entry: 2.8 GB for 10^8
+// entries) come from one memory pool per device that keeps up to
+// kTmpKeep bytes between builds; from the default pool they went back to the
+// driver at every synchronisation, and mapping them again cost as much as the
+// sorts.  Null when no pool could be made (then the default pool serves).
+constexpr uint64_t kTmpKeep = (uint64_t)4 << 30;
+cudaMemPool_t tmp_pool() {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    static bool tried[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    if (!tried[dev]) {
+        tried[dev] = true;
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p = nullptr;
+        if (cudaMemPoolCreate(&p, &props) == cudaSuccess) {
+            uint64_t keep = kTmpKeep;
+            cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+            pools[dev] = p;
+        } else {
+            cudaGetLastError();
+        }
+    }
+    return pools[dev];
+}
+
+template <typename T>
+sa_status dtmp(T **p, int64_t n, cudaStream_t s) {
+    if (n < 1) n = 1;
+    cudaMemPool_t pool = tmp_pool();
+    cudaError_t e = pool ? cudaMallocFromPoolAsync((void **)p, sizeof(T) * (size_t)n, pool, s)
+                         : cudaMallocAsync((void **)p, sizeof(T) * (size_t)n, s);
+    if (e != cudaSuccess) {
+        *p = nullptr;
+        cudaGetLastError();
+        return SA_ERR_OOM;
+    }
+    return SA_OK;
+}
+
 template <typename T>
 sa_status dalloc(T **p, int64_t n, cudaStream_t s) {
     if (n < 1) n = 1;
@@ -451,17 +500,17 @@ sa_status sa_graph_from_csr(sa_graph_s *g, const int64_t *rowptr, const int32_t 
         }                                         \
     } while (0)
 
-    TRY(dalloc(&rows, n, s));
-    TRY(dalloc(&keys, n, s));
-    TRY(dalloc(&keep, n + 1, s));
-    TRY(dalloc(&pos, n + 1, s));
-    TRY(dalloc(&flags, 4, s));
-    TRY(dalloc(&sb.k2, n, s));
-    TRY(dalloc(&sb.v2, n, s));
-    TRY(dalloc(&sb.counts, nc, s));
-    TRY(dalloc(&sb.offs, nc, s));
-    TRY(dalloc(&sb.tmp, scan_tmp_elems(scan_n), s));
-    TRY(dalloc(&sb.total, 1, s));
+    TRY(dtmp(&rows, n, s));
+    TRY(dtmp(&keys, n, s));
+    TRY(dtmp(&keep, n + 1, s));
+    TRY(dtmp(&pos, n + 1, s));
+    TRY(dtmp(&flags, 4, s));
+    TRY(dtmp(&sb.k2, n, s));
+    TRY(dtmp(&sb.v2, n, s));
+    TRY(dtmp(&sb.counts, nc, s));
+    TRY(dtmp(&sb.offs, nc, s));
+    TRY(dtmp(&sb.tmp, scan_tmp_elems(scan_n), s));
+    TRY(dtmp(&sb.total, 1, s));
     CTRY(cudaMemsetAsync(flags, 0, 4 * sizeof(int), s));
 
     // 1. validate, expand (row, key) pairs
@@ -492,7 +541,7 @@ sa_status sa_graph_from_csr(sa_graph_s *g, const int64_t *rowptr, const int32_t 
     TRY(dalloc(&g->colidx, new_nnz, s));
     TRY(dalloc(&g->rev_rowptr, T + 1, s));
     TRY(dalloc(&g->rev_colidx, new_nnz, s));
-    TRY(dalloc(&indeg, T + 1, s));
+    TRY(dtmp(&indeg, T + 1, s));
     if (n > 0) {
         SA_LAUNCH("graph_csr_compact", s,
                   csr_compact<<<blocks_for(n), kThreads, 0, s>>>(keys, keep, pos, n, g->colidx));

@@ -243,7 +243,8 @@ sa_status sparse_attn_set_path(int32_t path);
  * L2 ("Longer Attention Span ...", Abstract: single-GPU sequences of 160 M
  * tokens), merged into out and lse by the online-softmax rule.  Results are
  * the same up to rounding (pass 1's out is read back in the input dtype).
- *  SA_LINKS_AUTO     two passes when K and V together hold 2 GiB or more and
+ *  SA_LINKS_AUTO     two passes when K and V hold 2 GiB or more in total and
+ *                    1 GiB or more per (batch, head) slice, and
  *                    at least three such links exist (below that one pass was
  *                    measured faster on B200)
  *  SA_LINKS_SPLIT    two passes whenever such a link exists

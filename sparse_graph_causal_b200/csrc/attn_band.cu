@@ -919,9 +919,13 @@ namespace {
 // 84.7-86.2 ms, at 2^10 89.0, 2^11 85.8, 2^12 85.5, 2^14 88.1, 2^15 89.4-90.1,
 // 2^16 95.6; with the split at 2^13 two passes beat one from T = 2^23 (K and
 // V 2 GiB: 4.36 vs 4.60 ms; 2^24 8.99 vs 10.22; 2^25 18.3 vs 22.7; 2^26 39.7
-// vs 50.4) and lose at 2^22 (2.16 vs 2.06) and below.
+// vs 50.4) and lose at 2^22 (2.16 vs 2.06) and below.  What counts is the
+// length of one slice's sweep, not the job's size: with 4 slices of 2^22 two
+// passes won (8.56 vs 8.98 ms), with 16 slices of 2^20 (7.77 vs 8.23 ms one
+// pass) and 64 of 2^17 (3.18 vs 3.72) one pass did.
 constexpr int64_t kLongSpan = (int64_t)1 << 13;
 constexpr int kMinLong = 3;
+constexpr double kTwoPassSlice = 1.0 * 1024 * 1024 * 1024;  // K and V of one slice
 constexpr double kTwoPassBytes = 2.0 * 1024 * 1024 * 1024;  // K and V together
 
 int long_links(const sa_tensor *k, const sa_graph_s *g) {
@@ -933,8 +937,9 @@ int long_links(const sa_tensor *k, const sa_graph_s *g) {
         ++n;
     }
     if (mode == SA_LINKS_SPLIT) return n;
-    const double kv = (double)k->B * (double)k->H * (double)k->T * k->D * 2 * 2;
-    return (kv >= kTwoPassBytes && n >= kMinLong) ? n : 0;
+    const double slice = (double)k->T * k->D * 2 * 2;  // bf16 K and V rows of one slice
+    const double kv = slice * (double)k->B * (double)k->H;
+    return (slice >= kTwoPassSlice && kv >= kTwoPassBytes && n >= kMinLong) ? n : 0;
 }
 
 sa_status band_fwd_dispatch(const sa_tensor *q, const sa_tensor *k, const sa_tensor *v,

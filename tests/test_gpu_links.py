@@ -1,9 +1,9 @@
 """The forward's second pass over the long distance links of a structured
 graph: the band kernel takes the window and the links shorter than 2^13
 rows, the link pass the rest, class by class, and merges them into out and
-lse.  The automatic choice takes it only when K and V hold 2 GiB or more
-(the extreme-length workloads); here SA_LINKS_SPLIT forces it on sizes
-whose K and V are below that.  Checked against the gather kernels (every edge in one
+lse.  The automatic choice takes it only when K and V hold 2 GiB or more,
+1 GiB or more per slice (the extreme-length workloads); here SA_LINKS_SPLIT
+forces it on sizes whose K and V are below that.  Checked against the gather kernels (every edge in one
 pass) on every row, against the one-pass band kernel, and against the oracle
 on sampled rows, for D = 32, 64, 128 and grouped heads."""
 import math

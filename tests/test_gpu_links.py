@@ -89,3 +89,31 @@ def test_link_pass_matches_one_pass_and_oracle(oracle_lib, w):
     del x, out, lse, out1, lse1
     g.close()
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("H,lg,expect", [(16, 20, {"band_fwd"}), (4, 22, {"band_fwd", "link_pass"})],
+                         ids=["16x2^20_one_pass", "4x2^22_two_passes"])
+def test_link_pass_automatic_choice(H, lg, expect):
+    """The automatic choice follows the length of one slice, not the job's
+    size: 16 slices of 2^20 rows (K and V 4 GiB in all, 256 MiB a slice) run
+    one pass, 4 slices of 2^22 (4 GiB, 1 GiB a slice) two.  Checked by the
+    kernels that ran; the output rows are finite and lse holds at least the
+    row's own score (every row keeps itself)."""
+    import sparse_graph_causal_b200 as sa
+    w = _wl(f"auto_{H}x{lg}", H, H, 1 << lg, 64, lg - 1, 76)
+    g = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+    x = synth.make_qkv(w, device="cuda", with_dout=False)
+    sa.sparse_attn_set_link_pass(sa.SA_LINKS_AUTO)
+    sa.sparse_attn_profile_begin(True)
+    out, lse = sa.sparse_attn_fwd(x["q"], x["k"], x["v"], g, w.scale)
+    prof = sa.sparse_attn_profile_end()
+    sa.sparse_attn_check_device()
+    assert set(prof) == expect, prof
+    rows = torch.as_tensor(synth.sample_rows(w.T, 256, seed=w.seed), device="cuda")
+    o = out[0].index_select(1, rows).float()
+    assert torch.isfinite(o).all()
+    self_score = (x["q"][0].index_select(1, rows).float() * x["k"][0].index_select(1, rows).float()).sum(-1) * w.scale
+    assert (lse[0].index_select(1, rows) >= self_score - 1e-2).all()
+    del x, out, lse
+    g.close()
+    torch.cuda.empty_cache()

@@ -718,25 +718,32 @@ def measure_e2e(sa, w, x, out, lse, dq, dk, dv, ws, g0, flush, stream, do_bwd, E
         for s_ in (up, comp, down):
             s_.wait_event(start)
         for c in range(BH):
+            # the forward's inputs first, dout after them; out leaves as soon
+            # as the forward is done, the gradients after the backward
+            ev = {}
             with torch.cuda.stream(up):
                 for n in names_in:
                     sl(x[n], c).copy_(sl(hx[n], c), non_blocking=True)
-                uploaded = torch.cuda.Event()
-                uploaded.record(up)
-            comp.wait_event(uploaded)
+                    if n in ("v", "dout"):
+                        ev[n] = torch.cuda.Event()
+                        ev[n].record(up)
+            comp.wait_event(ev["v"])
             with torch.cuda.stream(comp):
                 qc, kc, vc = sl(x["q"], c), sl(x["k"], c), sl(x["v"], c)
                 oc, lc = sl(out, c), lse2[c].view(1, 1, T)
                 sa.sparse_attn_fwd(qc, kc, vc, g, w.scale, out=oc, lse=lc, stream=comp)
+                ev["fwd"] = torch.cuda.Event()
+                ev["fwd"].record(comp)
                 if do_bwd:
+                    comp.wait_event(ev["dout"])
                     sa.sparse_attn_bwd(qc, kc, vc, oc, lc, sl(x["dout"], c), g, w.scale,
                                        dq=sl(dq, c), dk=sl(dk, c), dv=sl(dv, c), workspace=ws_c,
                                        stream=comp)
-                computed = torch.cuda.Event()
-                computed.record(comp)
-            down.wait_event(computed)
+                    ev["bwd"] = torch.cuda.Event()
+                    ev["bwd"].record(comp)
             with torch.cuda.stream(down):
                 for n in names_out:
+                    down.wait_event(ev["fwd" if n == "out" else "bwd"])
                     sl(hout[n], c).copy_(sl(dev_out[n], c), non_blocking=True)
         for s_ in (up, comp, down):
             done = torch.cuda.Event()

@@ -343,21 +343,23 @@ def time_workload(sa, w: synth.Workload, dev, rank, world, dist, steps, warmup, 
     dk = torch.empty_like(k) if do_bwd else None
     dv = torch.empty_like(v) if do_bwd else None
     graph_build_ms = None
+    builds, builds_host = [], []
     if w.csr:
         # graph view: raw CSR rows -> normalised lists + transpose, timed alone
         rp_h, ci_h = synth.csr_random_rows(w.T, seed=w.graph_seed)
         rp_d, ci_d = torch.from_numpy(rp_h).to(dev), torch.from_numpy(ci_h).to(dev)
         del rp_h, ci_h
-        builds = []
         g0 = None
         for _ in range(3):
             if g0 is not None:
                 g0.close()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0 = time.perf_counter()
             a.record(stream)
             g0 = sa.sparse_attn_graph_build_csr(rp_d, ci_d, band_hint=w.band_hint)
             b.record(stream)
             torch.cuda.synchronize()
+            builds_host.append(1e3 * (time.perf_counter() - t0))
             builds.append(a.elapsed_time(b))
         graph_build_ms = max_over_ranks(dist, min(builds))
         del rp_d, ci_d
@@ -494,6 +496,8 @@ def time_workload(sa, w: synth.Workload, dev, rank, world, dist, steps, warmup, 
         "steps": steps, "ms_per_step": ms_step, "edges_per_s": E * world / (ms_step * 1e-3),
         "fwd_ms": fwd_ms, "fwd_edges_per_s": E * world / (fwd_ms * 1e-3),
         "tokens_per_s": w.B * w.T * world / (ms_step * 1e-3), "graph_build_ms": graph_build_ms,
+        "graph_build_ms_each": [round(b, 3) for b in builds] if builds else None,
+        "graph_build_host_ms_each": [round(b, 3) for b in builds_host] if builds else None,
         "roofline": roofline, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
     }
     del cuda_graph
@@ -618,7 +622,16 @@ def time_decode(sa, w, dev, rank, world, dist, steps, warmup, fwd_only, **_):
     for _ in range(max(3, warmup)):
         eager()
     sa.sparse_attn_check_device()
-    ms, clk = _timed_steps(eager, steps, flush, stream, dist, dev)
+    # the timed step replays the decode call captured once in a CUDA graph,
+    # as a serving loop would run it (eager, the host's launch path shows up
+    # in a kernel of ~10 us)
+    cg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(cg):
+        eager()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        cg.replay()
+    ms, clk = _timed_steps(cg.replay, steps, flush, stream, dist, dev)
     sa.sparse_attn_check_device()
     # neighbours per query: min(p + 1, W) + #{2^k : W <= 2^k <= p}
     ps = pos.cpu().tolist()
@@ -634,6 +647,7 @@ def time_decode(sa, w, dev, rank, world, dist, steps, warmup, fwd_only, **_):
     return {"config": {"workload": w.name, "B": B, "H": H, "Hkv": Hk, "T_cache": T, "D": D,
                        "W": w.W, "dilation_exps": list(w.exps), "positions": "uniform in [T/2, T)",
                        "pass": "decode (one query per sequence and head)",
+                       "timed_step": "CUDA-graph replay of the decode call",
                        "l2": "256 MiB buffer written between timed steps",
                        "parallelism": f"replicas x{world}"},
             "steps": steps, "ms_per_step": ms, "edges_per_s": edges * world / (ms * 1e-3),
@@ -678,6 +692,8 @@ def run_gpu(args, dist, rank, world):
             "dtype": w.dtype, "data": "synthetic", "config": r["config"],
             "fwd_edges_per_s": r["fwd_edges_per_s"], "fwd_ms": r["fwd_ms"],
             "tokens_per_s": r["tokens_per_s"], "graph_build_ms": r["graph_build_ms"],
+            "graph_build_ms_each": r["graph_build_ms_each"],
+            "graph_build_host_ms_each": r["graph_build_host_ms_each"],
             "roofline": r["roofline"], "cpu_baseline": cpu, "e2e": r["e2e"],
             "gpu_launches": r["gpu_launches"], "clocks": r["clocks"],
             "workloads": extra,

@@ -98,9 +98,10 @@ sa_status sparse_attn_graph_build_structured(int64_t T, int32_t W, const int32_t
  * queries ascending).  The caller's arrays are only read and may be freed
  * after the call returns.  Synchronises `stream` three times (to read the
  * validation result, the deduplicated entry count and the final checks).
- * Its temporaries (28 bytes per input entry) come from a library-owned
- * stream-ordered memory pool per device that keeps up to 4 GiB between
- * builds.  T < 2^31, nnz < 2^31. */
+ * Its temporaries (28 bytes per input entry) and the graph's lists come from
+ * a library-owned stream-ordered memory pool per device that keeps up to
+ * 4 GiB between builds (the first build in a process maps it).  T < 2^31,
+ * nnz < 2^31. */
 sa_status sparse_attn_graph_build_csr(int64_t T, const int64_t *rowptr, const int32_t *colidx,
                                       int64_t nnz, int32_t band_hint, void *stream,
                                       sa_graph *out);

@@ -1206,7 +1206,6 @@ band_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tkt,
             const int NB = GQ * n_band;
             const int64_t j = k0 + r;
             const bool row_ok = j < T;
-            const size_t grow = (size_t)kvbh * (size_t)T + (size_t)j;
             if (!__all_sync(0xffffffffu, wait(p, L::bKVFull, (uint32_t)(lt & 1)))) break;
             // diagonal slots: the Q and dO rows of the queries that reach this
             // key by a distance link (or by a CSR residual entry), for every

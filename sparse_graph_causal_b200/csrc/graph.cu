@@ -389,11 +389,12 @@ __global__ void csr_rev_resid(int64_t T, const int64_t *rev_rowptr, int32_t Wb, 
     atomicMax(max_resid, (int)(r > 0x7fffffff ? 0x7fffffff : r));
 }
 
-// The CSR build's temporaries (28 bytes per input entry: 2.8 GB for 10^8
-// entries) come from one memory pool per device that keeps up to
-// kTmpKeep bytes between builds; from the default pool they went back to the
-// driver at every synchronisation, and mapping them again cost as much as the
-// sorts.  Null when no pool could be made (then the default pool serves).
+// The graph builds' device memory (the CSR build's temporaries, 28 bytes per
+// input entry: 2.8 GB for 10^8 entries, and the graph's own lists) comes
+// from one memory pool per device that keeps up to kTmpKeep bytes between
+// builds; from the default pool it went back to the driver at every
+// synchronisation (or graph release), and mapping it again cost more than
+// the sorts.  Null when no pool could be made (then the default pool serves).
 constexpr uint64_t kTmpKeep = (uint64_t)4 << 30;
 cudaMemPool_t tmp_pool() {
     static std::mutex mu;
@@ -437,16 +438,11 @@ sa_status dtmp(T **p, int64_t n, cudaStream_t s) {
     return SA_OK;
 }
 
+// The graph's own lists (released by sparse_attn_graph_destroy, whose
+// cudaFree returns them to the pool).
 template <typename T>
 sa_status dalloc(T **p, int64_t n, cudaStream_t s) {
-    if (n < 1) n = 1;
-    cudaError_t e = cudaMallocAsync((void **)p, sizeof(T) * (size_t)n, s);
-    if (e != cudaSuccess) {
-        *p = nullptr;
-        cudaGetLastError();
-        return SA_ERR_OOM;
-    }
-    return SA_OK;
+    return dtmp(p, n, s);
 }
 
 }  // namespace

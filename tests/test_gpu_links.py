@@ -18,8 +18,8 @@ from gpu_util import compact, compare, gather_rows, local_rows
 pytestmark = pytest.mark.gpu
 
 
-def _wl(name, H, Hkv, T, D, kmax, seed):
-    return synth.Workload(name=name, B=1, H=H, T=T, D=D, dtype="bf16", W=32,
+def _wl(name, H, Hkv, T, D, kmax, seed, B=1):
+    return synth.Workload(name=name, B=B, H=H, T=T, D=D, dtype="bf16", W=32,
                           exps=tuple(range(0, kmax + 1)), input_std=1.0,
                           scale=1.0 / math.sqrt(D), seed=seed, Hkv=Hkv, bwd=False)
 
@@ -31,6 +31,9 @@ CASES = [
     _wl("links_d128", 1, 1, 1 << 18, 128, 17, 74),
     # ragged: the last tile partial, the last class one tile short
     _wl("links_ragged", 1, 1, (1 << 19) + 77, 64, 18, 75),
+    # two batch rows of grouped heads: slice b * H + h reads K/V slice
+    # b * Hkv + h / (H / Hkv)
+    _wl("links_b2_gqa", 4, 2, 1 << 18, 64, 17, 77, B=2),
 ]
 
 
@@ -77,15 +80,18 @@ def test_link_pass_matches_one_pass_and_oracle(oracle_lib, w):
     rp, ci = local_rows(o, rows, w.W, w.exps)
     keys, local = compact(rp, ci)
     G = w.H // w.kv_heads
-    for bh in range(w.H):
-        kvbh = bh // G
+    BH = w.B * w.H
+    for bh in range(BH):
+        kvbh = (bh // w.H) * w.kv_heads + (bh % w.H) // G
         q = gather_rows(x["q"], bh, rows, w.dtype)
         k = gather_rows(x["k"], kvbh, keys, w.dtype)
         v = gather_rows(x["v"], kvbh, keys, w.dtype)
         rout, rlse = o.fwd(q, k, v, rp, local, w.scale, dtype=w.dtype)
         idx = torch.as_tensor(rows, device="cuda")
-        compare(out[0, bh].index_select(0, idx), rout, w.dtype, f"{w.name}[{bh}] out")
-        compare(lse[0, bh].index_select(0, idx), rlse, w.dtype, f"{w.name}[{bh}] lse")
+        compare(out.view(BH, w.T, w.D)[bh].index_select(0, idx), rout, w.dtype,
+                f"{w.name}[{bh}] out")
+        compare(lse.view(BH, w.T)[bh].index_select(0, idx), rlse, w.dtype,
+                f"{w.name}[{bh}] lse")
     del x, out, lse, out1, lse1
     g.close()
     torch.cuda.empty_cache()

@@ -10,12 +10,20 @@
 //     out_i = sum_j softmax_j(s_ij) v_j,   lse_i = ln sum_j exp(s_ij).
 // A score costs three differences and three FMAs, so there is no contraction
 // for the tensor cores: these are gather kernels.  A warp owns one query
-// (forward, da) or one key (dc, dv); its lanes form G groups of L lanes, a
-// group holds one neighbour's value row (16 bytes per lane) and computes that
-// neighbour's score itself from the coordinates (every lane of the group
-// reads the same 12 bytes: one broadcast load), so no shuffle is needed for
-// the score.  Each group keeps its own online-softmax state; the groups are
-// merged at the end.  Base-2 arithmetic inside: s2 = log2(e) s.
+// (forward, da) or one key (dc, dv) and walks its list 32 edges at a time in
+// two phases:
+//  1. lane t takes edge t of the chunk: its key (or query) index, the
+//     coordinates, the score and the probability -- once per edge, not once
+//     per lane that touches the edge's row;
+//  2. the 32 lanes form G groups of L lanes (16 bytes of a row per lane); group
+//     g takes edges g, g + G, ... of the chunk, their index and probability
+//     fetched from the owning lanes by shuffles, and reads the value (or dO)
+//     rows.  Per-edge row dot products (dp) go back to the owning lane.
+// The forward's running max is warp-wide (one per chunk), so the groups'
+// partial sums merge by plain addition at the end.  Base-2 arithmetic
+// inside: s2 = log2(e) s.  Every kernel is bounded to 64 registers, so that
+// four 256-thread blocks share an SM: these kernels wait on L2, and the extra
+// resident warps hide more of it than the few spilled registers cost.
 //
 // Backward, probabilities recomputed from lse:
 //   Delta_i = dO_i . out_i,   p = exp(s_ij - lse_i),   dp = dO_i . v_j,
@@ -47,14 +55,59 @@ __device__ __forceinline__ float dist_score(const Coord &a, const Coord &c, floa
     return nscale2 * fmaf(dx, dx, fmaf(dy, dy, dz * dz));
 }
 
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// The structured graph's distances in shared memory, so that the lanes of
+// phase 1 read theirs without indexing the kernel parameters per lane.
+// Every thread of the block must call it (one barrier).
+__device__ __forceinline__ void stage_offsets(const GraphView &g, int64_t *s_offs) {
+    if (g.kind == 0 && (int)threadIdx.x < g.n_off) s_offs[threadIdx.x] = g.offs[threadIdx.x];
+    __syncthreads();
+}
+
+// Key of edge e (< deg) of query i's forward list: as row_edge.
+__device__ __forceinline__ int64_t fwd_key(const GraphView &g, const RowEdges &r,
+                                           const int64_t *s_offs, int64_t i, int64_t e) {
+    if (g.kind == 0) return e < r.ndil ? i - s_offs[r.first + e] : r.lo + (e - r.ndil);
+    return g.colidx[r.start + e];
+}
+
+// Query of edge e (< deg) of key j's transpose list: as col_edge.
+__device__ __forceinline__ int64_t col_query(const GraphView &g, const ColEdges &c,
+                                             const int64_t *s_offs, int64_t j, int64_t e) {
+    if (g.kind == 0) return e < c.nwin ? j + e : j + s_offs[g.n_off - 1 - (e - c.nwin)];
+    return g.rev_colidx[c.start + e];
+}
+
+// Phase 2's hand-back of the per-edge dot products: in the step that starts
+// at chunk edge u0, group x holds dp of edge u0 + x (all L lanes alike); lane
+// t = u0 + x keeps it.  Every lane must call it.
+template <int L, int G>
+__device__ __forceinline__ void take_dp(float dp, int u0, int lane, float &dpt) {
+    const float got = __shfl_sync(0xffffffffu, dp, ((lane - u0) & (G - 1)) * L);
+    if (lane >= u0 && lane < u0 + G) dpt = got;
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256) dist_fwd_kernel(const float *__restrict__ qa,
+__global__ void __launch_bounds__(256, 4) dist_fwd_kernel(const float *__restrict__ qa,
                                                        const float *__restrict__ kc,
                                                        const T *__restrict__ v, GraphView g,
                                                        float nscale2, T *__restrict__ out,
                                                        float *__restrict__ lse, int64_t ntiles) {
     constexpr int V = Slice<T>::V, L = D / V, G = 32 / L;
     static_assert(L >= 1 && L <= 32 && G * L == 32, "slice layout");
+    __shared__ int64_t s_offs[SA_MAX_OFFSETS];
+    stage_offsets(g, s_offs);
     const int lane = threadIdx.x & 31, grp = lane / L, sub = lane % L;
     const int64_t bh = blockIdx.x / ntiles;
     const int64_t i = (blockIdx.x % ntiles) * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -63,41 +116,46 @@ __global__ void __launch_bounds__(256) dist_fwd_kernel(const float *__restrict__
     const int64_t rbase = bh * T_;
     const Coord a = load_coord(qa, rbase + i);
     const RowEdges r = row_edges(g, i);
-    float m = -INFINITY, l = 0.f, acc[V];
+    float m = -INFINITY, lpart = 0.f, acc[V];  // lpart: this lane's edges' share of l
 #pragma unroll
     for (int x = 0; x < V; ++x) acc[x] = 0.f;
-    for (int64_t e0 = 0; e0 < r.deg; e0 += G) {
-        const int64_t e = e0 + grp;
+    for (int64_t e0 = 0; e0 < r.deg; e0 += 32) {
+        // phase 1: lane t scores edge e0 + t (lanes past the list: row i, p = 0)
+        const int64_t e = e0 + lane;
+        int64_t j = i;
+        float s = -INFINITY;
         if (e < r.deg) {
-            const int64_t j = row_edge(g, r, i, e);
-            const float s = dist_score(a, load_coord(kc, rbase + j), nscale2);
-            float vf[V];
-            Slice<T>::load(v + (rbase + j) * D + sub * V, vf);
-            const float mn = fmaxf(m, s);
-            const float al = ex2(m - mn), p = ex2(s - mn);
-            l = l * al + p;
+            j = fwd_key(g, r, s_offs, i, e);
+            s = dist_score(a, load_coord(kc, rbase + j), nscale2);
+        }
+        const float mn = fmaxf(m, warp_max(s));  // finite: lane 0 holds an edge
+        const float al = ex2(m - mn);            // 0 on the first chunk
+        lpart *= al;
 #pragma unroll
-            for (int x = 0; x < V; ++x) acc[x] = fmaf(p, vf[x], acc[x] * al);
-            m = mn;
+        for (int x = 0; x < V; ++x) acc[x] *= al;
+        m = mn;
+        const float p = ex2(s - mn);
+        lpart += p;
+        // phase 2: group grp weighs the value rows of edges u0 + grp
+        const int n = r.deg - e0 < 32 ? (int)(r.deg - e0) : 32;
+#pragma unroll 4
+        for (int u0 = 0; u0 < n; u0 += G) {
+            const int u = u0 + grp;
+            const int64_t ju = __shfl_sync(0xffffffffu, j, u);
+            const float pu = __shfl_sync(0xffffffffu, p, u);
+            float vf[V];
+            Slice<T>::load(v + (rbase + ju) * D + sub * V, vf);
+#pragma unroll
+            for (int x = 0; x < V; ++x) acc[x] = fmaf(pu, vf[x], acc[x]);
         }
     }
-    // merge the G group states
+    // the groups share the running max: their sums add
 #pragma unroll
     for (int o = L; o < 32; o <<= 1) {
-        const float mo = __shfl_xor_sync(0xffffffffu, m, o);
-        const float lo = __shfl_xor_sync(0xffffffffu, l, o);
-        float ao[V];
 #pragma unroll
-        for (int x = 0; x < V; ++x) ao[x] = __shfl_xor_sync(0xffffffffu, acc[x], o);
-        const float mn = fmaxf(m, mo);
-        if (mn != -INFINITY) {
-            const float p0 = ex2(m - mn), p1 = ex2(mo - mn);
-            l = l * p0 + lo * p1;
-#pragma unroll
-            for (int x = 0; x < V; ++x) acc[x] = acc[x] * p0 + ao[x] * p1;
-            m = mn;
-        }
+        for (int x = 0; x < V; ++x) acc[x] += __shfl_xor_sync(0xffffffffu, acc[x], o);
     }
+    const float l = warp_sum(lpart);
     if (grp == 0) {
         float o_[V];
         const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -110,11 +168,13 @@ __global__ void __launch_bounds__(256) dist_fwd_kernel(const float *__restrict__
 
 // da_i (and Delta_i for the second kernel) by the forward lists.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) dist_bwd_da_kernel(
+__global__ void __launch_bounds__(256, 4) dist_bwd_da_kernel(
     const float *__restrict__ qa, const float *__restrict__ kc, const T *__restrict__ v,
     const T *__restrict__ o, const float *__restrict__ lse, const T *__restrict__ dout, GraphView g,
     float scale, float *__restrict__ da, float *__restrict__ delta, int64_t ntiles) {
     constexpr int V = Slice<T>::V, L = D / V, G = 32 / L;
+    __shared__ int64_t s_offs[SA_MAX_OFFSETS];
+    stage_offsets(g, s_offs);
     const int lane = threadIdx.x & 31, grp = lane / L, sub = lane % L;
     const int64_t bh = blockIdx.x / ntiles;
     const int64_t i = (blockIdx.x % ntiles) * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -122,7 +182,7 @@ __global__ void __launch_bounds__(256) dist_bwd_da_kernel(
     if (i >= T_) return;
     const int64_t rbase = bh * T_;
     const float nscale2 = -scale * kLog2e;
-    float df[V], of[V];
+    float df[V], of[V];  // every group holds the whole dO row
     Slice<T>::load(dout + (rbase + i) * D + sub * V, df);
     Slice<T>::load(o + (rbase + i) * D + sub * V, of);
     float dl = 0.f;
@@ -132,39 +192,40 @@ __global__ void __launch_bounds__(256) dist_bwd_da_kernel(
     const float lse2 = lse[rbase + i] * kLog2e;
     const Coord a = load_coord(qa, rbase + i);
     const RowEdges r = row_edges(g, i);
-    float gx = 0.f, gy = 0.f, gz = 0.f;  // sum over this group's edges of dS (a - c)
-    for (int64_t e0 = 0; e0 < r.deg; e0 += G) {
-        const int64_t e = e0 + grp;
+    float gx = 0.f, gy = 0.f, gz = 0.f;  // this lane's edges' dS (a - c)
+    for (int64_t e0 = 0; e0 < r.deg; e0 += 32) {
+        const int64_t e = e0 + lane;
         const bool valid = e < r.deg;
-        float vf[V];
+        int64_t j = i;
         Coord c{0.f, 0.f, 0.f};
+        float p = 0.f;
         if (valid) {
-            const int64_t j = row_edge(g, r, i, e);
+            j = fwd_key(g, r, s_offs, i, e);
             c = load_coord(kc, rbase + j);
-            Slice<T>::load(v + (rbase + j) * D + sub * V, vf);
-        } else {
-#pragma unroll
-            for (int x = 0; x < V; ++x) vf[x] = 0.f;
+            p = ex2(dist_score(a, c, nscale2) - lse2);
         }
-        float dp = 0.f;
+        const int n = r.deg - e0 < 32 ? (int)(r.deg - e0) : 32;
+        float dpt = 0.f;  // dp of this lane's edge
+#pragma unroll 4
+        for (int u0 = 0; u0 < n; u0 += G) {
+            const int64_t ju = __shfl_sync(0xffffffffu, j, u0 + grp);
+            float vf[V];
+            Slice<T>::load(v + (rbase + ju) * D + sub * V, vf);
+            float dp = 0.f;
 #pragma unroll
-        for (int x = 0; x < V; ++x) dp = fmaf(df[x], vf[x], dp);
-        dp = group_sum<L>(dp);
+            for (int x = 0; x < V; ++x) dp = fmaf(df[x], vf[x], dp);
+            take_dp<L, G>(group_sum<L>(dp), u0, lane, dpt);
+        }
         if (valid) {
-            const float p = ex2(dist_score(a, c, nscale2) - lse2);
-            const float ds = p * (dp - Delta);
+            const float ds = p * (dpt - Delta);
             gx = fmaf(ds, a.x - c.x, gx);
             gy = fmaf(ds, a.y - c.y, gy);
             gz = fmaf(ds, a.z - c.z, gz);
         }
     }
-    // every lane of a group holds the same sums: add one lane per group
-#pragma unroll
-    for (int off = L; off < 32; off <<= 1) {
-        gx += __shfl_xor_sync(0xffffffffu, gx, off);
-        gy += __shfl_xor_sync(0xffffffffu, gy, off);
-        gz += __shfl_xor_sync(0xffffffffu, gz, off);
-    }
+    gx = warp_sum(gx);
+    gy = warp_sum(gy);
+    gz = warp_sum(gz);
     if (lane == 0) {
         const float f = -2.f * scale;
         float *dst = da + (rbase + i) * 3;
@@ -177,11 +238,13 @@ __global__ void __launch_bounds__(256) dist_bwd_da_kernel(
 
 // dc_j and dv_j by the transpose lists.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) dist_bwd_dcdv_kernel(
+__global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_kernel(
     const float *__restrict__ qa, const float *__restrict__ kc, const float *__restrict__ lse,
     const float *__restrict__ delta, const T *__restrict__ v, const T *__restrict__ dout,
     GraphView g, float scale, float *__restrict__ dc, T *__restrict__ dv, int64_t ntiles) {
     constexpr int V = Slice<T>::V, L = D / V, G = 32 / L;
+    __shared__ int64_t s_offs[SA_MAX_OFFSETS];
+    stage_offsets(g, s_offs);
     const int lane = threadIdx.x & 31, grp = lane / L, sub = lane % L;
     const int64_t bh = blockIdx.x / ntiles;
     const int64_t j = (blockIdx.x % ntiles) * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -190,38 +253,44 @@ __global__ void __launch_bounds__(256) dist_bwd_dcdv_kernel(
     const int64_t rbase = bh * T_;
     const float nscale2 = -scale * kLog2e;
     const Coord c = load_coord(kc, rbase + j);
-    float vf[V];
+    float vf[V];  // every group holds the whole value row
     Slice<T>::load(v + (rbase + j) * D + sub * V, vf);
     const ColEdges ce = col_edges(g, j);
-    float adv[V];
+    float adv[V];  // this group's edges' p dO
 #pragma unroll
     for (int x = 0; x < V; ++x) adv[x] = 0.f;
-    float gx = 0.f, gy = 0.f, gz = 0.f;
-    for (int64_t e0 = 0; e0 < ce.deg; e0 += G) {
-        const int64_t e = e0 + grp;
+    float gx = 0.f, gy = 0.f, gz = 0.f;  // this lane's edges' dS (a - c)
+    for (int64_t e0 = 0; e0 < ce.deg; e0 += 32) {
+        const int64_t e = e0 + lane;
         const bool valid = e < ce.deg;
-        float df[V];
+        int64_t i = j;
         Coord a{0.f, 0.f, 0.f};
-        float lse2 = 0.f, Delta = 0.f;
+        float p = 0.f, Delta = 0.f;
         if (valid) {
-            const int64_t i = col_edge(g, ce, j, e);
+            i = col_query(g, ce, s_offs, j, e);
             a = load_coord(qa, rbase + i);
-            Slice<T>::load(dout + (rbase + i) * D + sub * V, df);
-            lse2 = __ldg(lse + rbase + i) * kLog2e;
+            p = ex2(dist_score(a, c, nscale2) - __ldg(lse + rbase + i) * kLog2e);
             Delta = __ldg(delta + rbase + i);
-        } else {
-#pragma unroll
-            for (int x = 0; x < V; ++x) df[x] = 0.f;
         }
-        float dp = 0.f;
+        const int n = ce.deg - e0 < 32 ? (int)(ce.deg - e0) : 32;
+        float dpt = 0.f;
+#pragma unroll 4
+        for (int u0 = 0; u0 < n; u0 += G) {
+            const int u = u0 + grp;
+            const int64_t iu = __shfl_sync(0xffffffffu, i, u);
+            const float pu = __shfl_sync(0xffffffffu, p, u);
+            float df[V];
+            Slice<T>::load(dout + (rbase + iu) * D + sub * V, df);
+            float dp = 0.f;
 #pragma unroll
-        for (int x = 0; x < V; ++x) dp = fmaf(df[x], vf[x], dp);
-        dp = group_sum<L>(dp);
+            for (int x = 0; x < V; ++x) {
+                dp = fmaf(df[x], vf[x], dp);
+                adv[x] = fmaf(pu, df[x], adv[x]);
+            }
+            take_dp<L, G>(group_sum<L>(dp), u0, lane, dpt);
+        }
         if (valid) {
-            const float p = ex2(dist_score(a, c, nscale2) - lse2);
-            const float ds = p * (dp - Delta);
-#pragma unroll
-            for (int x = 0; x < V; ++x) adv[x] = fmaf(p, df[x], adv[x]);
+            const float ds = p * (dpt - Delta);
             gx = fmaf(ds, a.x - c.x, gx);
             gy = fmaf(ds, a.y - c.y, gy);
             gz = fmaf(ds, a.z - c.z, gz);
@@ -231,10 +300,10 @@ __global__ void __launch_bounds__(256) dist_bwd_dcdv_kernel(
     for (int off = L; off < 32; off <<= 1) {
 #pragma unroll
         for (int x = 0; x < V; ++x) adv[x] += __shfl_xor_sync(0xffffffffu, adv[x], off);
-        gx += __shfl_xor_sync(0xffffffffu, gx, off);
-        gy += __shfl_xor_sync(0xffffffffu, gy, off);
-        gz += __shfl_xor_sync(0xffffffffu, gz, off);
     }
+    gx = warp_sum(gx);
+    gy = warp_sum(gy);
+    gz = warp_sum(gz);
     if (grp == 0) Slice<T>::store(dv + (rbase + j) * D + sub * V, adv);
     if (lane == 0) {
         const float f = 2.f * scale;  // d s / d c = +2 scale (a - c)

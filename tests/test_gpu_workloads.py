@@ -7,8 +7,8 @@ import pytest
 import torch
 
 import synth
-from gpu_util import (compare, local_rows, oracle_dkdv_keys, oracle_dq_rows, oracle_fwd_rows,
-                      to_oracle)
+from gpu_util import (compact, compare, local_rows, oracle_dkdv_keys, oracle_dq_rows,
+                      oracle_fwd_rows, to_oracle)
 
 pytestmark = pytest.mark.gpu
 
@@ -138,3 +138,96 @@ def test_extreme_128m_fwd(sa, oracle_lib):
     compare(lse.view(w.T).index_select(0, idx), rlse, w.dtype, "lse")
     del x, out, lse
     torch.cuda.empty_cache()
+
+
+def test_gqa_16k_full(sa, oracle_lib):
+    """B1 H8 over 2 key/value heads, T16384 D64 bf16, window 32 + 2^k
+    (k = 0..13): every element.  out, lse and dq per query head from the
+    oracle on its key/value head; dk and dv of a key/value head are the sums
+    of the oracle's gradients over the 4 query heads of its group."""
+    w = synth.WORKLOADS["gqa_16k"]
+    g = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+    x = synth.make_qkv(w, device="cuda")
+    out, lse, (dq, dk, dv) = _fwd_bwd(sa, w, g, x)
+    rp, ci = oracle_lib.structured(w.T, w.W, w.exps)
+    G = w.H // w.kv_heads
+    for hk in range(w.kv_heads):
+        kh, vh = to_oracle(x["k"][0, hk], w.dtype), to_oracle(x["v"][0, hk], w.dtype)
+        sdk, sdv = np.zeros((w.T, w.D)), np.zeros((w.T, w.D))
+        for h in range(hk * G, (hk + 1) * G):
+            qh, doh = to_oracle(x["q"][0, h], w.dtype), to_oracle(x["dout"][0, h], w.dtype)
+            rout, rlse = oracle_lib.fwd(qh, kh, vh, rp, ci, w.scale, dtype=w.dtype)
+            rdq, rdk, rdv = oracle_lib.bwd(qh, kh, vh, doh, rp, ci, w.scale, dtype=w.dtype)
+            compare(out[0, h], rout, w.dtype, f"out[h={h}]")
+            compare(lse[0, h], rlse, w.dtype, f"lse[h={h}]")
+            compare(dq[0, h], rdq, w.dtype, f"dq[h={h}]")
+            sdk += rdk
+            sdv += rdv
+        compare(dk[0, hk], sdk, w.dtype, f"dk[kv head {hk}] (group sum)")
+        compare(dv[0, hk], sdv, w.dtype, f"dv[kv head {hk}] (group sum)")
+
+
+def test_dist_16k_full(sa, oracle_lib):
+    """Learned-coordinate scores, B1 H4 T16384 D64 bf16 over the window 32 +
+    2^k graph, coordinates N(0, 1), scale 0.5: every element of out, lse, da,
+    dc and dv (da and dc carry the coordinates' scale and are bounded against
+    their own range, as in the small learned-coordinate cases)."""
+    w = synth.WORKLOADS["dist_16k"]
+    g = sa.sparse_attn_graph_build_structured(w.T, w.W, list(w.exps))
+    a, c = synth.make_coords(w, device="cuda")
+    x = synth.make_qkv(w, device="cuda")
+    v, dout = x["v"], x["dout"]
+    out, lse = sa.sparse_attn_dist_fwd(a, c, v, g, w.scale)
+    da, dc, dv = sa.sparse_attn_dist_bwd(a, c, v, out, lse, dout, g, w.scale)
+    sa.sparse_attn_check_device()
+    rp, ci = oracle_lib.structured(w.T, w.W, w.exps)
+    BH = w.B * w.H
+    for bh in range(BH):
+        ah = a.view(BH, w.T, 3)[bh].cpu().numpy()
+        ch = c.view(BH, w.T, 3)[bh].cpu().numpy()
+        vh = to_oracle(v.view(BH, w.T, w.D)[bh], w.dtype)
+        doh = to_oracle(dout.view(BH, w.T, w.D)[bh], w.dtype)
+        rout, rlse = oracle_lib.dist_fwd(ah, ch, vh, rp, ci, w.scale, dtype=w.dtype,
+                                         cdtype="fp32")
+        rda, rdc, rdv = oracle_lib.dist_bwd(ah, ch, vh, doh, rp, ci, w.scale, dtype=w.dtype,
+                                            cdtype="fp32")
+        tag = f"dist_16k[bh={bh}]"
+        compare(out.view(BH, w.T, w.D)[bh], rout, w.dtype, tag + " out")
+        compare(lse.view(BH, w.T)[bh], rlse, w.dtype, tag + " lse")
+        compare(da.view(BH, w.T, 3)[bh], rda, w.dtype, tag + " da", unit_range=1.0)
+        compare(dc.view(BH, w.T, 3)[bh], rdc, w.dtype, tag + " dc", unit_range=1.0)
+        compare(dv.view(BH, w.T, w.D)[bh], rdv, w.dtype, tag + " dv")
+
+
+def test_decode_16k_full(sa, oracle_lib):
+    """Decode as the bench times it: 64 sequences, 8 query heads over 2 cache
+    heads, caches of 16384 rows (D64 bf16), positions drawn in [T/2, T), the
+    window 32 + 2^k graph: every query against the oracle on its row p of
+    the graph."""
+    w = synth.WORKLOADS["decode_16k"]
+    B, H, Hk, T, D = w.B, w.H, w.kv_heads, w.T, w.D
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(w.seed + 17)
+    q = torch.empty((B, H, 1, D), dtype=torch.float32, device="cuda").normal_(
+        generator=gen).to(w.torch_dtype)
+    kc = torch.empty((B, Hk, T, D), dtype=torch.float32, device="cuda").normal_(
+        generator=gen).to(w.torch_dtype)
+    vc = torch.empty((B, Hk, T, D), dtype=torch.float32, device="cuda").normal_(
+        generator=gen).to(w.torch_dtype)
+    pos = torch.randint(T // 2, T, (B,), generator=gen, device="cuda", dtype=torch.int64)
+    g = sa.sparse_attn_graph_build_structured(T, w.W, list(w.exps))
+    out, lse = sa.sparse_attn_decode(q, kc, vc, pos, g, w.scale)
+    sa.sparse_attn_check_device()
+    grp = H // Hk
+    for b, p in enumerate(pos.cpu().tolist()):
+        rp, ci = oracle_lib.structured_rows(np.array([p]), w.W, w.exps)
+        keys, local = compact(rp, ci)
+        kidx = torch.as_tensor(keys, device="cuda")
+        for hk in range(Hk):
+            kh = to_oracle(kc[b, hk].index_select(0, kidx), w.dtype)
+            vh = to_oracle(vc[b, hk].index_select(0, kidx), w.dtype)
+            for h in range(hk * grp, (hk + 1) * grp):
+                rout, rlse = oracle_lib.fwd(to_oracle(q[b, h], w.dtype), kh, vh, rp, local,
+                                            w.scale, dtype=w.dtype)
+                compare(out[b, h], rout, w.dtype, f"decode_16k[b={b},h={h},pos={p}] out")
+                compare(lse[b, h:h + 1], rlse, w.dtype, f"decode_16k[b={b},h={h},pos={p}] lse")

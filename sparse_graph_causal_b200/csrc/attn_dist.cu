@@ -35,6 +35,7 @@
 #include <stdint.h>
 
 #include "gather_common.cuh"
+#include "tc_common.cuh"
 
 namespace {
 
@@ -314,10 +315,367 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_kernel(
     }
 }
 
+
+// ---- structured graphs: the gathered rows of a block staged in shared memory
+//
+// On a structured graph the lists of QB consecutive rows b0 .. b0+QB-1 read
+// few distinct rows: the forward lists read the keys of one window span
+// (b0 - W + 1 .. b0 + QB - 1) and, per distance o, the QB keys b0 - o ..
+// b0 - o + QB - 1; the transpose lists read the queries b0 .. b0 + QB + W - 2
+// and b0 + o .. b0 + o + QB - 1.  A block of 8 warps stages those rows
+// (value rows and key coordinates for the forward and da; dO rows, query
+// coordinates, lse and Delta for dc and dv) once with coalesced copies, then
+// each warp takes rows b0 + w, b0 + w + 8, ... as above with its phase-1
+// scores and phase-2 rows read from shared memory: per 32 rows about 350
+// staged rows instead of ~1,300 row reads from L2 (window 32 + 9 links).
+
+constexpr int QB = 32;                  // rows per block
+constexpr int kMaxStageBytes = 52 * 1024;  // four blocks per SM
+
+// staged rows of a block: the window span, then one QB-row block per distance
+__host__ __device__ __forceinline__ int staged_rows(int W, int n_off) {
+    return W + QB - 1 + QB * n_off;
+}
+
+template <typename T, int D>
+__host__ __device__ __forceinline__ size_t stage_bytes(int W, int n_off, bool with_rowvals) {
+    const size_t R = (size_t)staged_rows(W, n_off);
+    return R * D * sizeof(T) + R * 3 * sizeof(float) + (with_rowvals ? R * 2 * sizeof(float) : 0);
+}
+
+// Source row of staged row r: DIR = -1 for the forward lists' keys, +1 for
+// the transpose lists' queries.
+template <int DIR>
+__device__ __forceinline__ int64_t staged_src(const GraphView &g, const int64_t *s_offs, int64_t b0,
+                                              int r) {
+    const int WB = g.W + QB - 1;
+    if (r < WB) return DIR < 0 ? b0 - g.W + 1 + r : b0 + r;
+    const int x = (r - WB) / QB, t = (r - WB) % QB;
+    return DIR < 0 ? b0 - s_offs[x] + t : b0 + s_offs[x] + t;
+}
+
+// Stage the block's rows of src (D columns), their coordinates and, for the
+// transpose lists, lse (base 2) and Delta.  Rows outside 0 .. T-1 are not
+// written (no list reads them).  Every thread of the block must call it.
+template <typename T, int D, int DIR>
+__device__ __forceinline__ void stage_block(const GraphView &g, const int64_t *s_offs,
+                                            int64_t rbase, int64_t b0, const T *src,
+                                            const float *crd_src, const float *lse,
+                                            const float *dl, T *rows, float *crd, float *slse,
+                                            float *sdl) {
+    constexpr int CPR = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
+    const int R = staged_rows(g.W, g.n_off);
+    for (int c = threadIdx.x; c < R * CPR; c += blockDim.x) {
+        const int r = c / CPR, k = c % CPR;
+        const int64_t sr = staged_src<DIR>(g, s_offs, b0, r);
+        if (sr >= 0 && sr < g.T)
+            tc::cp_async16(tc::smem_u32(rows + (size_t)r * D) + 16 * k,
+                           src + (rbase + sr) * D + k * (16 / (int)sizeof(T)));
+    }
+    tc::cp_async_commit();
+    for (int f = threadIdx.x; f < R * 3; f += blockDim.x) {
+        const int64_t sr = staged_src<DIR>(g, s_offs, b0, f / 3);
+        if (sr >= 0 && sr < g.T) crd[f] = __ldg(crd_src + (rbase + sr) * 3 + f % 3);
+    }
+    if (slse) {
+        for (int r = threadIdx.x; r < R; r += blockDim.x) {
+            const int64_t sr = staged_src<DIR>(g, s_offs, b0, r);
+            if (sr >= 0 && sr < g.T) {
+                slse[r] = __ldg(lse + rbase + sr) * kLog2e;
+                sdl[r] = __ldg(dl + rbase + sr);
+            }
+        }
+    }
+    tc::cp_async_wait<0>();
+    __syncthreads();
+}
+
+// A row slice from shared memory (Slice<T>::load reads global memory).
+template <typename T>
+__device__ __forceinline__ void load_staged(const T *p, float *f);
+
+template <>
+__device__ __forceinline__ void load_staged<__nv_bfloat16>(const __nv_bfloat16 *p, float *f) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        f[2 * a] = __uint_as_float(w[a] << 16);
+        f[2 * a + 1] = __uint_as_float(w[a] & 0xffff0000u);
+    }
+}
+
+template <>
+__device__ __forceinline__ void load_staged<float>(const float *p, float *f) {
+    const float4 u = *reinterpret_cast<const float4 *>(p);
+    f[0] = u.x;
+    f[1] = u.y;
+    f[2] = u.z;
+    f[3] = u.w;
+}
+
+// Staged row of edge e of query i = b0 + t (forward list).
+__device__ __forceinline__ int fwd_srow(const GraphView &g, const RowEdges &r, int64_t b0, int t,
+                                        int64_t e) {
+    if (e < r.ndil) return g.W + QB - 1 + QB * (r.first + (int)e) + t;
+    return (int)(r.lo + (e - r.ndil) - (b0 - g.W + 1));
+}
+
+// Staged row of edge e of key j = b0 + t (transpose list).
+__device__ __forceinline__ int col_srow(const GraphView &g, const ColEdges &c, int t, int64_t e) {
+    if (e < c.nwin) return t + (int)e;
+    return g.W + QB - 1 + QB * (g.n_off - 1 - (int)(e - c.nwin)) + t;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 4) dist_fwd_staged_kernel(
+    const float *__restrict__ qa, const float *__restrict__ kc, const T *__restrict__ v,
+    GraphView g, float nscale2, T *__restrict__ out, float *__restrict__ lse, int64_t nblk) {
+    constexpr int V = Slice<T>::V, L = D / V, G = 32 / L;
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ int64_t s_offs[SA_MAX_OFFSETS];
+    stage_offsets(g, s_offs);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, grp = lane / L, sub = lane % L;
+    const int64_t bh = blockIdx.x / nblk, b0 = (blockIdx.x % nblk) * QB, T_ = g.T;
+    const int64_t rbase = bh * T_;
+    const int R = staged_rows(g.W, g.n_off);
+    T *rows = reinterpret_cast<T *>(dsm);
+    float *crd = reinterpret_cast<float *>(dsm + (size_t)R * D * sizeof(T));
+    stage_block<T, D, -1>(g, s_offs, rbase, b0, v, kc, nullptr, nullptr, rows, crd, nullptr,
+                          nullptr);
+    for (int t = warp; t < QB; t += kWarpsPerBlock) {
+        const int64_t i = b0 + t;
+        if (i >= T_) break;
+        const Coord a = load_coord(qa, rbase + i);
+        const RowEdges r = row_edges(g, i);
+        float m = -INFINITY, lpart = 0.f, acc[V];
+#pragma unroll
+        for (int x = 0; x < V; ++x) acc[x] = 0.f;
+        for (int64_t e0 = 0; e0 < r.deg; e0 += 32) {
+            const int64_t e = e0 + lane;
+            int sr = t + g.W - 1;  // lanes past the list: key i's own row (written), p = 0
+            float s = -INFINITY;
+            if (e < r.deg) {
+                sr = fwd_srow(g, r, b0, t, e);
+                s = dist_score(a, Coord{crd[3 * sr], crd[3 * sr + 1], crd[3 * sr + 2]}, nscale2);
+            }
+            const float mn = fmaxf(m, warp_max(s));
+            const float al = ex2(m - mn);
+            lpart *= al;
+#pragma unroll
+            for (int x = 0; x < V; ++x) acc[x] *= al;
+            m = mn;
+            const float p = ex2(s - mn);
+            lpart += p;
+            const int n = r.deg - e0 < 32 ? (int)(r.deg - e0) : 32;
+#pragma unroll 4
+            for (int u0 = 0; u0 < n; u0 += G) {
+                const int u = u0 + grp;
+                const int su = __shfl_sync(0xffffffffu, sr, u);
+                const float pu = __shfl_sync(0xffffffffu, p, u);
+                float vf[V];
+                load_staged<T>(rows + (size_t)su * D + sub * V, vf);
+#pragma unroll
+                for (int x = 0; x < V; ++x) acc[x] = fmaf(pu, vf[x], acc[x]);
+            }
+        }
+#pragma unroll
+        for (int o = L; o < 32; o <<= 1) {
+#pragma unroll
+            for (int x = 0; x < V; ++x) acc[x] += __shfl_xor_sync(0xffffffffu, acc[x], o);
+        }
+        const float l = warp_sum(lpart);
+        if (grp == 0) {
+            float o_[V];
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+            for (int x = 0; x < V; ++x) o_[x] = acc[x] * inv;
+            Slice<T>::store(out + (rbase + i) * D + sub * V, o_);
+            if (sub == 0) lse[rbase + i] = l > 0.f ? (m + lg2(l)) * kLn2 : -INFINITY;
+        }
+    }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 4) dist_bwd_da_staged_kernel(
+    const float *__restrict__ qa, const float *__restrict__ kc, const T *__restrict__ v,
+    const T *__restrict__ o, const float *__restrict__ lse, const T *__restrict__ dout, GraphView g,
+    float scale, float *__restrict__ da, float *__restrict__ delta, int64_t nblk) {
+    constexpr int V = Slice<T>::V, L = D / V, G = 32 / L;
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ int64_t s_offs[SA_MAX_OFFSETS];
+    stage_offsets(g, s_offs);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, grp = lane / L, sub = lane % L;
+    const int64_t bh = blockIdx.x / nblk, b0 = (blockIdx.x % nblk) * QB, T_ = g.T;
+    const int64_t rbase = bh * T_;
+    const float nscale2 = -scale * kLog2e;
+    const int R = staged_rows(g.W, g.n_off);
+    T *rows = reinterpret_cast<T *>(dsm);
+    float *crd = reinterpret_cast<float *>(dsm + (size_t)R * D * sizeof(T));
+    stage_block<T, D, -1>(g, s_offs, rbase, b0, v, kc, nullptr, nullptr, rows, crd, nullptr,
+                          nullptr);
+    for (int t = warp; t < QB; t += kWarpsPerBlock) {
+        const int64_t i = b0 + t;
+        if (i >= T_) break;
+        float df[V], of[V];
+        Slice<T>::load(dout + (rbase + i) * D + sub * V, df);
+        Slice<T>::load(o + (rbase + i) * D + sub * V, of);
+        float dl = 0.f;
+#pragma unroll
+        for (int x = 0; x < V; ++x) dl = fmaf(df[x], of[x], dl);
+        const float Delta = group_sum<L>(dl);
+        const float lse2 = lse[rbase + i] * kLog2e;
+        const Coord a = load_coord(qa, rbase + i);
+        const RowEdges r = row_edges(g, i);
+        float gx = 0.f, gy = 0.f, gz = 0.f;
+        for (int64_t e0 = 0; e0 < r.deg; e0 += 32) {
+            const int64_t e = e0 + lane;
+            int sr = t + g.W - 1;  // lanes past the list: key i's own row (written), p = 0
+            Coord c{0.f, 0.f, 0.f};
+            float p = 0.f;
+            if (e < r.deg) {
+                sr = fwd_srow(g, r, b0, t, e);
+                c = Coord{crd[3 * sr], crd[3 * sr + 1], crd[3 * sr + 2]};
+                p = ex2(dist_score(a, c, nscale2) - lse2);
+            }
+            const int n = r.deg - e0 < 32 ? (int)(r.deg - e0) : 32;
+            float dpt = 0.f;
+#pragma unroll 4
+            for (int u0 = 0; u0 < n; u0 += G) {
+                const int su = __shfl_sync(0xffffffffu, sr, u0 + grp);
+                float vf[V];
+                load_staged<T>(rows + (size_t)su * D + sub * V, vf);
+                float dp = 0.f;
+#pragma unroll
+                for (int x = 0; x < V; ++x) dp = fmaf(df[x], vf[x], dp);
+                take_dp<L, G>(group_sum<L>(dp), u0, lane, dpt);
+            }
+            const float ds = p * (dpt - Delta);  // p = 0 past the list
+            gx = fmaf(ds, a.x - c.x, gx);
+            gy = fmaf(ds, a.y - c.y, gy);
+            gz = fmaf(ds, a.z - c.z, gz);
+        }
+        gx = warp_sum(gx);
+        gy = warp_sum(gy);
+        gz = warp_sum(gz);
+        if (lane == 0) {
+            const float f = -2.f * scale;
+            float *dst = da + (rbase + i) * 3;
+            dst[0] = f * gx;
+            dst[1] = f * gy;
+            dst[2] = f * gz;
+            delta[rbase + i] = Delta;
+        }
+    }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_staged_kernel(
+    const float *__restrict__ qa, const float *__restrict__ kc, const float *__restrict__ lse,
+    const float *__restrict__ delta, const T *__restrict__ v, const T *__restrict__ dout,
+    GraphView g, float scale, float *__restrict__ dc, T *__restrict__ dv, int64_t nblk) {
+    constexpr int V = Slice<T>::V, L = D / V, G = 32 / L;
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ int64_t s_offs[SA_MAX_OFFSETS];
+    stage_offsets(g, s_offs);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, grp = lane / L, sub = lane % L;
+    const int64_t bh = blockIdx.x / nblk, b0 = (blockIdx.x % nblk) * QB, T_ = g.T;
+    const int64_t rbase = bh * T_;
+    const float nscale2 = -scale * kLog2e;
+    const int R = staged_rows(g.W, g.n_off);
+    T *rows = reinterpret_cast<T *>(dsm);
+    float *crd = reinterpret_cast<float *>(dsm + (size_t)R * D * sizeof(T));
+    float *slse = crd + 3 * R, *sdl = slse + R;
+    stage_block<T, D, +1>(g, s_offs, rbase, b0, dout, qa, lse, delta, rows, crd, slse, sdl);
+    for (int t = warp; t < QB; t += kWarpsPerBlock) {
+        const int64_t j = b0 + t;
+        if (j >= T_) break;
+        const Coord c = load_coord(kc, rbase + j);
+        float vf[V];
+        Slice<T>::load(v + (rbase + j) * D + sub * V, vf);
+        const ColEdges ce = col_edges(g, j);
+        float adv[V];
+#pragma unroll
+        for (int x = 0; x < V; ++x) adv[x] = 0.f;
+        float gx = 0.f, gy = 0.f, gz = 0.f;
+        for (int64_t e0 = 0; e0 < ce.deg; e0 += 32) {
+            const int64_t e = e0 + lane;
+            int sr = t;  // lanes past the list: query j's own row (written), p = 0
+            Coord a{0.f, 0.f, 0.f};
+            float p = 0.f, Delta = 0.f;
+            if (e < ce.deg) {
+                sr = col_srow(g, ce, t, e);
+                a = Coord{crd[3 * sr], crd[3 * sr + 1], crd[3 * sr + 2]};
+                p = ex2(dist_score(a, c, nscale2) - slse[sr]);
+                Delta = sdl[sr];
+            }
+            const int n = ce.deg - e0 < 32 ? (int)(ce.deg - e0) : 32;
+            float dpt = 0.f;
+#pragma unroll 4
+            for (int u0 = 0; u0 < n; u0 += G) {
+                const int u = u0 + grp;
+                const int su = __shfl_sync(0xffffffffu, sr, u);
+                const float pu = __shfl_sync(0xffffffffu, p, u);
+                float df[V];
+                load_staged<T>(rows + (size_t)su * D + sub * V, df);
+                float dp = 0.f;
+#pragma unroll
+                for (int x = 0; x < V; ++x) {
+                    dp = fmaf(df[x], vf[x], dp);
+                    adv[x] = fmaf(pu, df[x], adv[x]);
+                }
+                take_dp<L, G>(group_sum<L>(dp), u0, lane, dpt);
+            }
+            const float ds = p * (dpt - Delta);  // p = 0 past the list
+            gx = fmaf(ds, a.x - c.x, gx);
+            gy = fmaf(ds, a.y - c.y, gy);
+            gz = fmaf(ds, a.z - c.z, gz);
+        }
+#pragma unroll
+        for (int off = L; off < 32; off <<= 1) {
+#pragma unroll
+            for (int x = 0; x < V; ++x) adv[x] += __shfl_xor_sync(0xffffffffu, adv[x], off);
+        }
+        gx = warp_sum(gx);
+        gy = warp_sum(gy);
+        gz = warp_sum(gz);
+        if (grp == 0) Slice<T>::store(dv + (rbase + j) * D + sub * V, adv);
+        if (lane == 0) {
+            const float f = 2.f * scale;
+            float *dst = dc + (rbase + j) * 3;
+            dst[0] = f * gx;
+            dst[1] = f * gy;
+            dst[2] = f * gz;
+        }
+    }
+}
+
+// Structured graphs whose staged rows fit kMaxStageBytes take the staged
+// kernels (the window and distance spans of a block are 32-bit offsets).
+// The size varies with the graph, so the kernels are opted in once for the
+// largest.
+template <typename T, int D>
+bool use_staged(const GraphView &g, bool with_rowvals) {
+    return g.kind == 0 && g.W <= (1 << 20) &&
+           stage_bytes<T, D>(g.W, g.n_off, with_rowvals) <= (size_t)kMaxStageBytes;
+}
+
 template <typename T, int D>
 sa_status launch_fwd(const sa_tensor *a, const sa_tensor *c, const sa_tensor *v,
                      const GraphView &g, float scale, sa_tensor *out, float *lse, cudaStream_t s) {
     const int64_t BH = v->B * v->H;
+    if (use_staged<T, D>(g, false)) {
+        const int64_t nblk = (g.T + QB - 1) / QB;
+        if (nblk * BH > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+        const int bytes = (int)stage_bytes<T, D>(g.W, g.n_off, false);
+        SA_CUDA_TRY(sa_smem_optin((const void *)dist_fwd_staged_kernel<T, D>, kMaxStageBytes));
+        SA_LAUNCH("dist_fwd", s,
+                  dist_fwd_staged_kernel<T, D><<<(unsigned)(nblk * BH), 256, bytes, s>>>(
+                      (const float *)a->ptr, (const float *)c->ptr, (const T *)v->ptr, g,
+                      -scale * kLog2e, (T *)out->ptr, lse, nblk));
+        SA_CUDA_TRY(cudaGetLastError());
+        return SA_OK;
+    }
     const int64_t ntiles = (g.T + kWarpsPerBlock - 1) / kWarpsPerBlock;
     const int64_t nblocks = ntiles * BH;
     if (nblocks > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
@@ -335,6 +693,26 @@ sa_status launch_bwd(const sa_tensor *a, const sa_tensor *c, const sa_tensor *v,
                      const GraphView &g, float scale, sa_tensor *da, sa_tensor *dc, sa_tensor *dv,
                      float *delta, cudaStream_t s) {
     const int64_t BH = v->B * v->H;
+    if (use_staged<T, D>(g, true)) {
+        const int64_t nblk = (g.T + QB - 1) / QB;
+        if (nblk * BH > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+        const int b_da = (int)stage_bytes<T, D>(g.W, g.n_off, false);
+        const int b_dc = (int)stage_bytes<T, D>(g.W, g.n_off, true);
+        SA_CUDA_TRY(sa_smem_optin((const void *)dist_bwd_da_staged_kernel<T, D>, kMaxStageBytes));
+        SA_CUDA_TRY(sa_smem_optin((const void *)dist_bwd_dcdv_staged_kernel<T, D>, kMaxStageBytes));
+        SA_LAUNCH("dist_bwd_da", s,
+                  dist_bwd_da_staged_kernel<T, D><<<(unsigned)(nblk * BH), 256, b_da, s>>>(
+                      (const float *)a->ptr, (const float *)c->ptr, (const T *)v->ptr,
+                      (const T *)o->ptr, lse, (const T *)dout->ptr, g, scale, (float *)da->ptr,
+                      delta, nblk));
+        SA_LAUNCH("dist_bwd_dcdv", s,
+                  dist_bwd_dcdv_staged_kernel<T, D><<<(unsigned)(nblk * BH), 256, b_dc, s>>>(
+                      (const float *)a->ptr, (const float *)c->ptr, lse, delta,
+                      (const T *)v->ptr, (const T *)dout->ptr, g, scale, (float *)dc->ptr,
+                      (T *)dv->ptr, nblk));
+        SA_CUDA_TRY(cudaGetLastError());
+        return SA_OK;
+    }
     const int64_t ntiles = (g.T + kWarpsPerBlock - 1) / kWarpsPerBlock;
     const int64_t nblocks = ntiles * BH;
     if (nblocks > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;

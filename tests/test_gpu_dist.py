@@ -2,7 +2,9 @@
 against the CPU oracle, element by element: s_ij = -scale |a_i - c_j|^2 over
 the same neighbour lists ("SpatialLM-Mini ...", section "How tokens choose
 whom to listen to").  Structured and CSR graphs (with empty rows), bf16 and
-fp32 values, every supported head size, ragged tails."""
+fp32 values, every supported head size, ragged tails; structured graphs
+through the kernels that stage a block's rows in shared memory and, when
+those do not fit, through the per-row kernels."""
 import math
 
 import numpy as np
@@ -35,6 +37,9 @@ CASES = [
     (_wl("dist_d64_bf16", 1, 2, 1000, 64, "bf16", 32, range(0, 10)), None),
     (_wl("dist_d32_fp32", 1, 2, 300, 32, "fp32", 8, range(0, 9)), None),
     (_wl("dist_d128_bf16", 2, 1, 333, 128, "bf16", 16, (4, 6, 8)), None),
+    # a structured graph whose staged rows exceed the staged kernels' shared
+    # memory (fp32, D = 128): the per-row kernels
+    (_wl("dist_d128_fp32_unstaged", 1, 2, 700, 128, "fp32", 64, range(6, 10)), None),
     (_wl("dist_csr_empty_rows", 1, 2, 400, 64, "bf16", 0, csr=True), _csr_with_empty(400, 3)),
     (_wl("dist_csr_view", 1, 1, 1500, 64, "fp32", 0, csr=True, band=64),
      synth.csr_random_rows(1500, seed=5)),

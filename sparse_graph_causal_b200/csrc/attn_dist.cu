@@ -343,20 +343,13 @@ __host__ __device__ __forceinline__ size_t stage_bytes(int W, int n_off, bool wi
     return R * D * sizeof(T) + R * 3 * sizeof(float) + (with_rowvals ? R * 2 * sizeof(float) : 0);
 }
 
-// Source row of staged row r: DIR = -1 for the forward lists' keys, +1 for
-// the transpose lists' queries.
-template <int DIR>
-__device__ __forceinline__ int64_t staged_src(const GraphView &g, const int64_t *s_offs, int64_t b0,
-                                              int r) {
-    const int WB = g.W + QB - 1;
-    if (r < WB) return DIR < 0 ? b0 - g.W + 1 + r : b0 + r;
-    const int x = (r - WB) / QB, t = (r - WB) % QB;
-    return DIR < 0 ? b0 - s_offs[x] + t : b0 + s_offs[x] + t;
-}
-
 // Stage the block's rows of src (D columns), their coordinates and, for the
-// transpose lists, lse (base 2) and Delta.  Rows outside 0 .. T-1 are not
-// written (no list reads them).  Every thread of the block must call it.
+// transpose lists, lse (base 2) and Delta: segment 0 is the window span (W +
+// QB - 1 rows), segment 1 + x the QB rows of distance offs[x]; each segment's
+// source rows are contiguous (DIR = -1: keys b0 - W + 1 .. and b0 - o ..;
+// DIR = +1: queries b0 .. and b0 + o ..), so it is one flat copy.  Rows
+// outside 0 .. T-1 are not written (no list reads them).  Every thread of
+// the block must call it.
 template <typename T, int D, int DIR>
 __device__ __forceinline__ void stage_block(const GraphView &g, const int64_t *s_offs,
                                             int64_t rbase, int64_t b0, const T *src,
@@ -364,55 +357,92 @@ __device__ __forceinline__ void stage_block(const GraphView &g, const int64_t *s
                                             const float *dl, T *rows, float *crd, float *slse,
                                             float *sdl) {
     constexpr int CPR = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
-    const int R = staged_rows(g.W, g.n_off);
-    for (int c = threadIdx.x; c < R * CPR; c += blockDim.x) {
-        const int r = c / CPR, k = c % CPR;
-        const int64_t sr = staged_src<DIR>(g, s_offs, b0, r);
-        if (sr >= 0 && sr < g.T)
-            tc::cp_async16(tc::smem_u32(rows + (size_t)r * D) + 16 * k,
-                           src + (rbase + sr) * D + k * (16 / (int)sizeof(T)));
-    }
-    tc::cp_async_commit();
-    for (int f = threadIdx.x; f < R * 3; f += blockDim.x) {
-        const int64_t sr = staged_src<DIR>(g, s_offs, b0, f / 3);
-        if (sr >= 0 && sr < g.T) crd[f] = __ldg(crd_src + (rbase + sr) * 3 + f % 3);
-    }
-    if (slse) {
-        for (int r = threadIdx.x; r < R; r += blockDim.x) {
-            const int64_t sr = staged_src<DIR>(g, s_offs, b0, r);
-            if (sr >= 0 && sr < g.T) {
-                slse[r] = __ldg(lse + rbase + sr) * kLog2e;
-                sdl[r] = __ldg(dl + rbase + sr);
+    constexpr int EPC = 16 / (int)sizeof(T);      // elements per chunk
+    for (int sg = 0; sg <= g.n_off; ++sg) {
+        const int n = sg == 0 ? g.W + QB - 1 : QB;
+        const int r0 = sg == 0 ? 0 : g.W + QB - 1 + QB * (sg - 1);
+        int64_t s0 = sg == 0 ? (DIR < 0 ? b0 - g.W + 1 : b0)
+                             : (DIR < 0 ? b0 - s_offs[sg - 1] : b0 + s_offs[sg - 1]);
+        // the rows of the segment inside 0 .. T-1
+        const int lo = s0 < 0 ? (int)(-s0 < n ? -s0 : n) : 0;
+        const int hi = s0 + n > g.T ? (int)(g.T - s0 > lo ? g.T - s0 : lo) : n;
+        if (hi <= lo) continue;
+        const T *gsrc = src + (rbase + s0 + lo) * D;
+        const uint32_t sdst = tc::smem_u32(rows + (size_t)(r0 + lo) * D);
+        for (int c = threadIdx.x; c < (hi - lo) * CPR; c += blockDim.x)
+            tc::cp_async16(sdst + 16 * c, gsrc + (size_t)c * EPC);
+        const float *csrc = crd_src + (rbase + s0 + lo) * 3;
+        float *cdst = crd + 3 * (r0 + lo);
+        for (int f = threadIdx.x; f < (hi - lo) * 3; f += blockDim.x) cdst[f] = __ldg(csrc + f);
+        if (slse) {
+            for (int r = threadIdx.x; r < hi - lo; r += blockDim.x) {
+                slse[r0 + lo + r] = __ldg(lse + rbase + s0 + lo + r) * kLog2e;
+                sdl[r0 + lo + r] = __ldg(dl + rbase + s0 + lo + r);
             }
         }
     }
+    tc::cp_async_commit();
     tc::cp_async_wait<0>();
     __syncthreads();
 }
 
-// A row slice from shared memory (Slice<T>::load reads global memory).
+// A lane's slice of a row held in registers (bf16: 4 words of bf16 pairs;
+// fp32: 4 floats), with the two row operations of phase 2 against a staged
+// slice: the partial dot product and p * row added to an accumulator.  bf16
+// products are exact (fma.rn.f32.bf16); p is rounded to bf16 for the sum, as
+// the band kernels round P for their P V products.
 template <typename T>
-__device__ __forceinline__ void load_staged(const T *p, float *f);
+struct StagedRow;
 
 template <>
-__device__ __forceinline__ void load_staged<__nv_bfloat16>(const __nv_bfloat16 *p, float *f) {
-    const uint4 u = *reinterpret_cast<const uint4 *>(p);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        f[2 * a] = __uint_as_float(w[a] << 16);
-        f[2 * a + 1] = __uint_as_float(w[a] & 0xffff0000u);
+struct StagedRow<__nv_bfloat16> {
+    uint32_t w[4];
+    __device__ __forceinline__ void hold(const __nv_bfloat16 *p) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+        w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
     }
-}
+    __device__ __forceinline__ void stage(const __nv_bfloat16 *p) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(p);
+        w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
+    }
+    __device__ __forceinline__ float dot(const StagedRow &o) const {
+        float a = 0.f, b = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            a = tc::fma_bf_lo(w[k], o.w[k], a);
+            b = tc::fma_bf_hi(w[k], o.w[k], b);
+        }
+        return a + b;
+    }
+    __device__ __forceinline__ void axpy(float p, float *acc) const {  // acc += p * this
+        const uint32_t p2 = tc::pack_bf16x2(p, p);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            acc[2 * k] = tc::fma_bf_lo(p2, w[k], acc[2 * k]);
+            acc[2 * k + 1] = tc::fma_bf_hi(p2, w[k], acc[2 * k + 1]);
+        }
+    }
+};
 
 template <>
-__device__ __forceinline__ void load_staged<float>(const float *p, float *f) {
-    const float4 u = *reinterpret_cast<const float4 *>(p);
-    f[0] = u.x;
-    f[1] = u.y;
-    f[2] = u.z;
-    f[3] = u.w;
-}
+struct StagedRow<float> {
+    float f[4];
+    __device__ __forceinline__ void hold(const float *p) {
+        const float4 u = __ldg(reinterpret_cast<const float4 *>(p));
+        f[0] = u.x, f[1] = u.y, f[2] = u.z, f[3] = u.w;
+    }
+    __device__ __forceinline__ void stage(const float *p) {
+        const float4 u = *reinterpret_cast<const float4 *>(p);
+        f[0] = u.x, f[1] = u.y, f[2] = u.z, f[3] = u.w;
+    }
+    __device__ __forceinline__ float dot(const StagedRow &o) const {
+        return fmaf(f[0], o.f[0], fmaf(f[1], o.f[1], fmaf(f[2], o.f[2], f[3] * o.f[3])));
+    }
+    __device__ __forceinline__ void axpy(float p, float *acc) const {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[k] = fmaf(p, f[k], acc[k]);
+    }
+};
 
 // Staged row of edge e of query i = b0 + t (forward list).
 __device__ __forceinline__ int fwd_srow(const GraphView &g, const RowEdges &r, int64_t b0, int t,
@@ -473,10 +503,9 @@ __global__ void __launch_bounds__(256, 4) dist_fwd_staged_kernel(
                 const int u = u0 + grp;
                 const int su = __shfl_sync(0xffffffffu, sr, u);
                 const float pu = __shfl_sync(0xffffffffu, p, u);
-                float vf[V];
-                load_staged<T>(rows + (size_t)su * D + sub * V, vf);
-#pragma unroll
-                for (int x = 0; x < V; ++x) acc[x] = fmaf(pu, vf[x], acc[x]);
+                StagedRow<T> vr;
+                vr.stage(rows + (size_t)su * D + sub * V);
+                vr.axpy(pu, acc);
             }
         }
 #pragma unroll
@@ -517,13 +546,10 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_da_staged_kernel(
     for (int t = warp; t < QB; t += kWarpsPerBlock) {
         const int64_t i = b0 + t;
         if (i >= T_) break;
-        float df[V], of[V];
-        Slice<T>::load(dout + (rbase + i) * D + sub * V, df);
-        Slice<T>::load(o + (rbase + i) * D + sub * V, of);
-        float dl = 0.f;
-#pragma unroll
-        for (int x = 0; x < V; ++x) dl = fmaf(df[x], of[x], dl);
-        const float Delta = group_sum<L>(dl);
+        StagedRow<T> dh, oh;  // this lane's slices of the dO and out rows
+        dh.hold(dout + (rbase + i) * D + sub * V);
+        oh.hold(o + (rbase + i) * D + sub * V);
+        const float Delta = group_sum<L>(dh.dot(oh));
         const float lse2 = lse[rbase + i] * kLog2e;
         const Coord a = load_coord(qa, rbase + i);
         const RowEdges r = row_edges(g, i);
@@ -543,12 +569,9 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_da_staged_kernel(
 #pragma unroll 4
             for (int u0 = 0; u0 < n; u0 += G) {
                 const int su = __shfl_sync(0xffffffffu, sr, u0 + grp);
-                float vf[V];
-                load_staged<T>(rows + (size_t)su * D + sub * V, vf);
-                float dp = 0.f;
-#pragma unroll
-                for (int x = 0; x < V; ++x) dp = fmaf(df[x], vf[x], dp);
-                take_dp<L, G>(group_sum<L>(dp), u0, lane, dpt);
+                StagedRow<T> vr;
+                vr.stage(rows + (size_t)su * D + sub * V);
+                take_dp<L, G>(group_sum<L>(dh.dot(vr)), u0, lane, dpt);
             }
             const float ds = p * (dpt - Delta);  // p = 0 past the list
             gx = fmaf(ds, a.x - c.x, gx);
@@ -591,8 +614,8 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_staged_kernel(
         const int64_t j = b0 + t;
         if (j >= T_) break;
         const Coord c = load_coord(kc, rbase + j);
-        float vf[V];
-        Slice<T>::load(v + (rbase + j) * D + sub * V, vf);
+        StagedRow<T> vh;  // this lane's slice of the value row
+        vh.hold(v + (rbase + j) * D + sub * V);
         const ColEdges ce = col_edges(g, j);
         float adv[V];
 #pragma unroll
@@ -616,15 +639,10 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_staged_kernel(
                 const int u = u0 + grp;
                 const int su = __shfl_sync(0xffffffffu, sr, u);
                 const float pu = __shfl_sync(0xffffffffu, p, u);
-                float df[V];
-                load_staged<T>(rows + (size_t)su * D + sub * V, df);
-                float dp = 0.f;
-#pragma unroll
-                for (int x = 0; x < V; ++x) {
-                    dp = fmaf(df[x], vf[x], dp);
-                    adv[x] = fmaf(pu, df[x], adv[x]);
-                }
-                take_dp<L, G>(group_sum<L>(dp), u0, lane, dpt);
+                StagedRow<T> dr;
+                dr.stage(rows + (size_t)su * D + sub * V);
+                dr.axpy(pu, adv);
+                take_dp<L, G>(group_sum<L>(vh.dot(dr)), u0, lane, dpt);
             }
             const float ds = p * (dpt - Delta);  // p = 0 past the list
             gx = fmaf(ds, a.x - c.x, gx);

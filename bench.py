@@ -669,8 +669,12 @@ def run_gpu(args, dist, rank, world):
 
     extra = {}
     if not args.no_extra:
+        chosen = set(filter(None, args.extra.split(",")))
+        unknown = chosen - set(EXTRA_WORKLOADS)
+        if unknown:
+            raise SystemExit(f"--extra: unknown workloads {sorted(unknown)}")
         for name in EXTRA_WORKLOADS:
-            if name == w.name:
+            if name == w.name or name not in chosen:
                 continue
             wx = synth.WORKLOADS[name]
             timer = {"attn": time_workload, "dist": time_dist, "decode": time_decode}[wx.kind]
@@ -796,7 +800,10 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="spatiallm_16k", choices=sorted(synth.WORKLOADS))
+    # the main line times a dot-product workload; the learned-coordinate and
+    # decode workloads are timed under "workloads"
+    ap.add_argument("--workload", default="spatiallm_16k",
+                    choices=sorted(n for n, x in synth.WORKLOADS.items() if x.kind == "attn"))
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls, no CUDA graph")
@@ -804,6 +811,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-extra", action="store_true",
                     help="time only --workload, not the other named workloads")
+    ap.add_argument("--extra", default=",".join(EXTRA_WORKLOADS),
+                    help="comma-separated subset of the other named workloads to time")
     ap.add_argument("--extra-steps", type=int, default=5,
                     help="timed steps of each of the other named workloads")
     ap.add_argument("--link-pass", default="auto", choices=["auto", "split", "one"],

@@ -444,17 +444,39 @@ struct StagedRow<float> {
     }
 };
 
-// Staged row of edge e of query i = b0 + t (forward list).
-__device__ __forceinline__ int fwd_srow(const GraphView &g, const RowEdges &r, int64_t b0, int t,
-                                        int64_t e) {
-    if (e < r.ndil) return g.W + QB - 1 + QB * (r.first + (int)e) + t;
-    return (int)(r.lo + (e - r.ndil) - (b0 - g.W + 1));
+// Staged rows of a list in 32-bit arithmetic, set up once per row: edge e
+// < nsplit is staged row a + sa * e, later edges row b + sb * e.  Forward list of
+// query i = b0 + t: the links (row t of distance block first + e), then the
+// window (key lo + e - ndil).  Transpose list of key j = b0 + t: the window
+// (query j + e), then the links in ascending distance (block n_off - 1 -
+// (e - nwin)).
+struct StagedList {
+    int deg, nsplit, a, sa, b, sb;
+    __device__ __forceinline__ int row(int e) const { return e < nsplit ? a + sa * e : b + sb * e; }
+};
+
+__device__ __forceinline__ StagedList fwd_list(const GraphView &g, const RowEdges &r, int64_t b0,
+                                               int t) {
+    StagedList l;
+    l.deg = (int)r.deg;
+    l.nsplit = r.ndil;
+    l.a = g.W + QB - 1 + QB * r.first + t;
+    l.sa = QB;
+    l.b = (int)(r.lo - (b0 - g.W + 1)) - r.ndil;
+    l.sb = 1;
+    return l;
 }
 
-// Staged row of edge e of key j = b0 + t (transpose list).
-__device__ __forceinline__ int col_srow(const GraphView &g, const ColEdges &c, int t, int64_t e) {
-    if (e < c.nwin) return t + (int)e;
-    return g.W + QB - 1 + QB * (g.n_off - 1 - (int)(e - c.nwin)) + t;
+__device__ __forceinline__ StagedList col_list(const GraphView &g, const ColEdges &c, int t) {
+    StagedList l;
+    l.deg = (int)c.deg;
+    l.nsplit = (int)c.nwin;
+    l.a = t;
+    l.sa = 1;
+    // link e - nwin sits in block n_off - 1 - (e - nwin)
+    l.b = g.W + QB - 1 + QB * (g.n_off - 1) + t + QB * l.nsplit;
+    l.sb = -QB;
+    return l;
 }
 
 template <typename T, int D>
@@ -477,16 +499,16 @@ __global__ void __launch_bounds__(256, 4) dist_fwd_staged_kernel(
         const int64_t i = b0 + t;
         if (i >= T_) break;
         const Coord a = load_coord(qa, rbase + i);
-        const RowEdges r = row_edges(g, i);
+        const StagedList sl = fwd_list(g, row_edges(g, i), b0, t);
         float m = -INFINITY, lpart = 0.f, acc[V];
 #pragma unroll
         for (int x = 0; x < V; ++x) acc[x] = 0.f;
-        for (int64_t e0 = 0; e0 < r.deg; e0 += 32) {
-            const int64_t e = e0 + lane;
+        for (int e0 = 0; e0 < sl.deg; e0 += 32) {
+            const int e = e0 + lane;
             int sr = t + g.W - 1;  // lanes past the list: key i's own row (written), p = 0
             float s = -INFINITY;
-            if (e < r.deg) {
-                sr = fwd_srow(g, r, b0, t, e);
+            if (e < sl.deg) {
+                sr = sl.row(e);
                 s = dist_score(a, Coord{crd[3 * sr], crd[3 * sr + 1], crd[3 * sr + 2]}, nscale2);
             }
             const float mn = fmaxf(m, warp_max(s));
@@ -497,7 +519,7 @@ __global__ void __launch_bounds__(256, 4) dist_fwd_staged_kernel(
             m = mn;
             const float p = ex2(s - mn);
             lpart += p;
-            const int n = r.deg - e0 < 32 ? (int)(r.deg - e0) : 32;
+            const int n = sl.deg - e0 < 32 ? sl.deg - e0 : 32;
 #pragma unroll 4
             for (int u0 = 0; u0 < n; u0 += G) {
                 const int u = u0 + grp;
@@ -552,19 +574,19 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_da_staged_kernel(
         const float Delta = group_sum<L>(dh.dot(oh));
         const float lse2 = lse[rbase + i] * kLog2e;
         const Coord a = load_coord(qa, rbase + i);
-        const RowEdges r = row_edges(g, i);
+        const StagedList sl = fwd_list(g, row_edges(g, i), b0, t);
         float gx = 0.f, gy = 0.f, gz = 0.f;
-        for (int64_t e0 = 0; e0 < r.deg; e0 += 32) {
-            const int64_t e = e0 + lane;
+        for (int e0 = 0; e0 < sl.deg; e0 += 32) {
+            const int e = e0 + lane;
             int sr = t + g.W - 1;  // lanes past the list: key i's own row (written), p = 0
             Coord c{0.f, 0.f, 0.f};
             float p = 0.f;
-            if (e < r.deg) {
-                sr = fwd_srow(g, r, b0, t, e);
+            if (e < sl.deg) {
+                sr = sl.row(e);
                 c = Coord{crd[3 * sr], crd[3 * sr + 1], crd[3 * sr + 2]};
                 p = ex2(dist_score(a, c, nscale2) - lse2);
             }
-            const int n = r.deg - e0 < 32 ? (int)(r.deg - e0) : 32;
+            const int n = sl.deg - e0 < 32 ? sl.deg - e0 : 32;
             float dpt = 0.f;
 #pragma unroll 4
             for (int u0 = 0; u0 < n; u0 += G) {
@@ -616,23 +638,23 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_staged_kernel(
         const Coord c = load_coord(kc, rbase + j);
         StagedRow<T> vh;  // this lane's slice of the value row
         vh.hold(v + (rbase + j) * D + sub * V);
-        const ColEdges ce = col_edges(g, j);
+        const StagedList sl = col_list(g, col_edges(g, j), t);
         float adv[V];
 #pragma unroll
         for (int x = 0; x < V; ++x) adv[x] = 0.f;
         float gx = 0.f, gy = 0.f, gz = 0.f;
-        for (int64_t e0 = 0; e0 < ce.deg; e0 += 32) {
-            const int64_t e = e0 + lane;
+        for (int e0 = 0; e0 < sl.deg; e0 += 32) {
+            const int e = e0 + lane;
             int sr = t;  // lanes past the list: query j's own row (written), p = 0
             Coord a{0.f, 0.f, 0.f};
             float p = 0.f, Delta = 0.f;
-            if (e < ce.deg) {
-                sr = col_srow(g, ce, t, e);
+            if (e < sl.deg) {
+                sr = sl.row(e);
                 a = Coord{crd[3 * sr], crd[3 * sr + 1], crd[3 * sr + 2]};
                 p = ex2(dist_score(a, c, nscale2) - slse[sr]);
                 Delta = sdl[sr];
             }
-            const int n = ce.deg - e0 < 32 ? (int)(ce.deg - e0) : 32;
+            const int n = sl.deg - e0 < 32 ? sl.deg - e0 : 32;
             float dpt = 0.f;
 #pragma unroll 4
             for (int u0 = 0; u0 < n; u0 += G) {

@@ -386,6 +386,23 @@ __device__ __forceinline__ void stage_block(const GraphView &g, const int64_t *s
     __syncthreads();
 }
 
+// Shared-memory loads by 32-bit shared address (no generic-address math).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a));
+    return v;
+}
+
+__device__ __forceinline__ Coord lds_coord(uint32_t a) {
+    Coord c;
+    asm volatile("ld.shared.f32 %0, [%3];\n\tld.shared.f32 %1, [%3+4];\n\tld.shared.f32 %2, [%3+8];"
+                 : "=f"(c.x), "=f"(c.y), "=f"(c.z)
+                 : "r"(a));
+    return c;
+}
+
 // A lane's slice of a row held in registers (bf16: 4 words of bf16 pairs;
 // fp32: 4 floats), with the two row operations of phase 2 against a staged
 // slice: the partial dot product and p * row added to an accumulator.  bf16
@@ -401,8 +418,8 @@ struct StagedRow<__nv_bfloat16> {
         const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
         w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
     }
-    __device__ __forceinline__ void stage(const __nv_bfloat16 *p) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    __device__ __forceinline__ void stage(uint32_t a) {  // shared address
+        const uint4 u = lds128(a);
         w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
     }
     __device__ __forceinline__ float dot(const StagedRow &o) const {
@@ -431,9 +448,10 @@ struct StagedRow<float> {
         const float4 u = __ldg(reinterpret_cast<const float4 *>(p));
         f[0] = u.x, f[1] = u.y, f[2] = u.z, f[3] = u.w;
     }
-    __device__ __forceinline__ void stage(const float *p) {
-        const float4 u = *reinterpret_cast<const float4 *>(p);
-        f[0] = u.x, f[1] = u.y, f[2] = u.z, f[3] = u.w;
+    __device__ __forceinline__ void stage(uint32_t a) {  // shared address
+        const uint4 u = lds128(a);
+        f[0] = __uint_as_float(u.x), f[1] = __uint_as_float(u.y), f[2] = __uint_as_float(u.z),
+        f[3] = __uint_as_float(u.w);
     }
     __device__ __forceinline__ float dot(const StagedRow &o) const {
         return fmaf(f[0], o.f[0], fmaf(f[1], o.f[1], fmaf(f[2], o.f[2], f[3] * o.f[3])));
@@ -495,6 +513,9 @@ __global__ void __launch_bounds__(256, 4) dist_fwd_staged_kernel(
     float *crd = reinterpret_cast<float *>(dsm + (size_t)R * D * sizeof(T));
     stage_block<T, D, -1>(g, s_offs, rbase, b0, v, kc, nullptr, nullptr, rows, crd, nullptr,
                           nullptr);
+    constexpr uint32_t kRowBytes = D * sizeof(T);
+    const uint32_t rows_s = tc::smem_u32(rows) + 16 * sub;  // this lane's 16 bytes of row 0
+    const uint32_t crd_s = tc::smem_u32(crd);
     for (int t = warp; t < QB; t += kWarpsPerBlock) {
         const int64_t i = b0 + t;
         if (i >= T_) break;
@@ -509,7 +530,7 @@ __global__ void __launch_bounds__(256, 4) dist_fwd_staged_kernel(
             float s = -INFINITY;
             if (e < sl.deg) {
                 sr = sl.row(e);
-                s = dist_score(a, Coord{crd[3 * sr], crd[3 * sr + 1], crd[3 * sr + 2]}, nscale2);
+                s = dist_score(a, lds_coord(crd_s + 12 * sr), nscale2);
             }
             const float mn = fmaxf(m, warp_max(s));
             const float al = ex2(m - mn);
@@ -526,7 +547,7 @@ __global__ void __launch_bounds__(256, 4) dist_fwd_staged_kernel(
                 const int su = __shfl_sync(0xffffffffu, sr, u);
                 const float pu = __shfl_sync(0xffffffffu, p, u);
                 StagedRow<T> vr;
-                vr.stage(rows + (size_t)su * D + sub * V);
+                vr.stage(rows_s + (uint32_t)su * kRowBytes);
                 vr.axpy(pu, acc);
             }
         }
@@ -565,6 +586,9 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_da_staged_kernel(
     float *crd = reinterpret_cast<float *>(dsm + (size_t)R * D * sizeof(T));
     stage_block<T, D, -1>(g, s_offs, rbase, b0, v, kc, nullptr, nullptr, rows, crd, nullptr,
                           nullptr);
+    constexpr uint32_t kRowBytes = D * sizeof(T);
+    const uint32_t rows_s = tc::smem_u32(rows) + 16 * sub;  // this lane's 16 bytes of row 0
+    const uint32_t crd_s = tc::smem_u32(crd);
     for (int t = warp; t < QB; t += kWarpsPerBlock) {
         const int64_t i = b0 + t;
         if (i >= T_) break;
@@ -583,7 +607,7 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_da_staged_kernel(
             float p = 0.f;
             if (e < sl.deg) {
                 sr = sl.row(e);
-                c = Coord{crd[3 * sr], crd[3 * sr + 1], crd[3 * sr + 2]};
+                c = lds_coord(crd_s + 12 * sr);
                 p = ex2(dist_score(a, c, nscale2) - lse2);
             }
             const int n = sl.deg - e0 < 32 ? sl.deg - e0 : 32;
@@ -592,7 +616,7 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_da_staged_kernel(
             for (int u0 = 0; u0 < n; u0 += G) {
                 const int su = __shfl_sync(0xffffffffu, sr, u0 + grp);
                 StagedRow<T> vr;
-                vr.stage(rows + (size_t)su * D + sub * V);
+                vr.stage(rows_s + (uint32_t)su * kRowBytes);
                 take_dp<L, G>(group_sum<L>(dh.dot(vr)), u0, lane, dpt);
             }
             const float ds = p * (dpt - Delta);  // p = 0 past the list
@@ -632,6 +656,9 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_staged_kernel(
     float *crd = reinterpret_cast<float *>(dsm + (size_t)R * D * sizeof(T));
     float *slse = crd + 3 * R, *sdl = slse + R;
     stage_block<T, D, +1>(g, s_offs, rbase, b0, dout, qa, lse, delta, rows, crd, slse, sdl);
+    constexpr uint32_t kRowBytes = D * sizeof(T);
+    const uint32_t rows_s = tc::smem_u32(rows) + 16 * sub;  // this lane's 16 bytes of row 0
+    const uint32_t crd_s = tc::smem_u32(crd);
     for (int t = warp; t < QB; t += kWarpsPerBlock) {
         const int64_t j = b0 + t;
         if (j >= T_) break;
@@ -650,7 +677,7 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_staged_kernel(
             float p = 0.f, Delta = 0.f;
             if (e < sl.deg) {
                 sr = sl.row(e);
-                a = Coord{crd[3 * sr], crd[3 * sr + 1], crd[3 * sr + 2]};
+                a = lds_coord(crd_s + 12 * sr);
                 p = ex2(dist_score(a, c, nscale2) - slse[sr]);
                 Delta = sdl[sr];
             }
@@ -662,7 +689,7 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_staged_kernel(
                 const int su = __shfl_sync(0xffffffffu, sr, u);
                 const float pu = __shfl_sync(0xffffffffu, p, u);
                 StagedRow<T> dr;
-                dr.stage(rows + (size_t)su * D + sub * V);
+                dr.stage(rows_s + (uint32_t)su * kRowBytes);
                 dr.axpy(pu, adv);
                 take_dp<L, G>(group_sum<L>(vh.dot(dr)), u0, lane, dpt);
             }

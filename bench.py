@@ -225,9 +225,7 @@ def cpu_oracle_run(w: synth.Workload, seconds: float, seed_rows: int = 7):
         o.bwd(q, k, v, do, rp, local.astype(np.int32), w.scale, dtype=w.dtype)
         done_s += time.perf_counter() - t0
         done_edges += int(rp[-1])
-        n_rows = min(T, n_rows * 2)
-        if n_rows == T and done_s > seconds / 4:
-            break
+        n_rows = min(T, n_rows * 2)  # whole slices again once the sample reaches T rows
     desc = (f"fwd+bwd of {done_edges} edges: random query rows of slice 0 of {w.name}, "
             f"oracle single-threaded fp64 C")
     return done_edges / done_s, done_edges, done_s, desc

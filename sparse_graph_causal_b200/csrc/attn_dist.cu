@@ -516,10 +516,16 @@ __global__ void __launch_bounds__(256, 4) dist_fwd_staged_kernel(
     constexpr uint32_t kRowBytes = D * sizeof(T);
     const uint32_t rows_s = tc::smem_u32(rows) + 16 * sub;  // this lane's 16 bytes of row 0
     const uint32_t crd_s = tc::smem_u32(crd);
+    // each warp's rows are b0 + warp + 8 u; a row's own inputs are loaded one
+    // row ahead, so that their latency hides behind the previous row's work
+    Coord a_nx{0.f, 0.f, 0.f};
+    if (b0 + warp < T_) a_nx = load_coord(qa, rbase + b0 + warp);
     for (int t = warp; t < QB; t += kWarpsPerBlock) {
         const int64_t i = b0 + t;
         if (i >= T_) break;
-        const Coord a = load_coord(qa, rbase + i);
+        const Coord a = a_nx;
+        if (t + kWarpsPerBlock < QB && i + kWarpsPerBlock < T_)
+            a_nx = load_coord(qa, rbase + i + kWarpsPerBlock);
         const StagedList sl = fwd_list(g, row_edges(g, i), b0, t);
         float m = -INFINITY, lpart = 0.f, acc[V];
 #pragma unroll
@@ -589,15 +595,25 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_da_staged_kernel(
     constexpr uint32_t kRowBytes = D * sizeof(T);
     const uint32_t rows_s = tc::smem_u32(rows) + 16 * sub;  // this lane's 16 bytes of row 0
     const uint32_t crd_s = tc::smem_u32(crd);
+    // a row's own inputs one row ahead (as in the forward)
+    StagedRow<T> dh_nx, oh_nx;  // this lane's slices of the next row's dO and out
+    float lse_nx = 0.f;
+    Coord a_nx{0.f, 0.f, 0.f};
+    auto fetch = [&](int64_t ii) {
+        dh_nx.hold(dout + (rbase + ii) * D + sub * V);
+        oh_nx.hold(o + (rbase + ii) * D + sub * V);
+        lse_nx = __ldg(lse + rbase + ii);
+        a_nx = load_coord(qa, rbase + ii);
+    };
+    if (b0 + warp < T_) fetch(b0 + warp);
     for (int t = warp; t < QB; t += kWarpsPerBlock) {
         const int64_t i = b0 + t;
         if (i >= T_) break;
-        StagedRow<T> dh, oh;  // this lane's slices of the dO and out rows
-        dh.hold(dout + (rbase + i) * D + sub * V);
-        oh.hold(o + (rbase + i) * D + sub * V);
-        const float Delta = group_sum<L>(dh.dot(oh));
-        const float lse2 = lse[rbase + i] * kLog2e;
-        const Coord a = load_coord(qa, rbase + i);
+        const StagedRow<T> dh = dh_nx;
+        const float Delta = group_sum<L>(dh.dot(oh_nx));
+        const float lse2 = lse_nx * kLog2e;
+        const Coord a = a_nx;
+        if (t + kWarpsPerBlock < QB && i + kWarpsPerBlock < T_) fetch(i + kWarpsPerBlock);
         const StagedList sl = fwd_list(g, row_edges(g, i), b0, t);
         float gx = 0.f, gy = 0.f, gz = 0.f;
         for (int e0 = 0; e0 < sl.deg; e0 += 32) {

@@ -34,7 +34,7 @@
 namespace {
 
 constexpr int BM = 128;        // queries per tile
-constexpr int kDS = 3;         // ring stages per warp
+constexpr int kDS = 2;         // ring stages per warp
 constexpr int kMinBlocks = 2;  // CTAs per SM the register budget must allow
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;

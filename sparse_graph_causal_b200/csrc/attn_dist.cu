@@ -473,6 +473,28 @@ struct StagedList {
     __device__ __forceinline__ int row(int e) const { return e < nsplit ? a + sa * e : b + sb * e; }
 };
 
+// Number of distances (s_offs, descending) for which pred(o) holds, counted
+// by the warp's lanes in two ballots (n_off <= 64).  Every lane must call it.
+template <typename Pred>
+__device__ __forceinline__ int count_offsets(const int64_t *s_offs, int n_off, int lane, Pred pred) {
+    const unsigned b0 = __ballot_sync(0xffffffffu, lane < n_off && pred(s_offs[lane]));
+    const unsigned b1 = __ballot_sync(0xffffffffu, lane + 32 < n_off && pred(s_offs[lane + 32]));
+    return __popc(b0) + __popc(b1);
+}
+
+// The transpose list of key j as col_edges gives it (structured graph), its
+// distances counted by the warp instead of a loop over all of them (the
+// forward lists keep row_edges: its loop stops at the first distance that
+// reaches the row, which for most rows is the first one).
+__device__ __forceinline__ ColEdges col_edges_warp(const GraphView &g, const int64_t *s_offs,
+                                                   int64_t j, int lane) {
+    ColEdges c;
+    c.nwin = g.T - j < g.W ? g.T - j : g.W;
+    c.deg = c.nwin + count_offsets(s_offs, g.n_off, lane, [&](int64_t o) { return j + o < g.T; });
+    c.start = 0;
+    return c;
+}
+
 __device__ __forceinline__ StagedList fwd_list(const GraphView &g, const RowEdges &r, int64_t b0,
                                                int t) {
     StagedList l;
@@ -681,7 +703,7 @@ __global__ void __launch_bounds__(256, 4) dist_bwd_dcdv_staged_kernel(
         const Coord c = load_coord(kc, rbase + j);
         StagedRow<T> vh;  // this lane's slice of the value row
         vh.hold(v + (rbase + j) * D + sub * V);
-        const StagedList sl = col_list(g, col_edges(g, j), t);
+        const StagedList sl = col_list(g, col_edges_warp(g, s_offs, j, lane), t);
         float adv[V];
 #pragma unroll
         for (int x = 0; x < V; ++x) adv[x] = 0.f;

@@ -37,6 +37,10 @@ CASES = [
     (_wl("dist_d64_bf16", 1, 2, 1000, 64, "bf16", 32, range(0, 10)), None),
     (_wl("dist_d32_fp32", 1, 2, 300, 32, "fp32", 8, range(0, 9)), None),
     (_wl("dist_d128_bf16", 2, 1, 333, 128, "bf16", 16, (4, 6, 8)), None),
+    # fewer rows than one staged block, and one block plus a row (fp32: at a
+    # handful of rows the bf16 out's rounding in Delta dominates da and dc)
+    (_wl("dist_t5_fp32", 1, 2, 5, 64, "fp32", 4, (0, 1, 2)), None),
+    (_wl("dist_t33_fp32", 1, 1, 33, 64, "fp32", 8, range(0, 6)), None),
     # a structured graph whose staged rows exceed the staged kernels' shared
     # memory (fp32, D = 128): the per-row kernels
     (_wl("dist_d128_fp32_unstaged", 1, 2, 700, 128, "fp32", 64, range(6, 10)), None),

@@ -668,9 +668,6 @@ def run_gpu(args, dist, rank, world):
     extra = {}
     if not args.no_extra:
         chosen = set(filter(None, args.extra.split(",")))
-        unknown = chosen - set(EXTRA_WORKLOADS)
-        if unknown:
-            raise SystemExit(f"--extra: unknown workloads {sorted(unknown)}")
         for name in EXTRA_WORKLOADS:
             if name == w.name or name not in chosen:
                 continue
@@ -817,6 +814,9 @@ def main():
                     help="long distance links in a second forward pass: the library's "
                          "automatic choice, always, or never (sparse_attn_set_link_pass)")
     args = ap.parse_args()
+    unknown = set(filter(None, args.extra.split(","))) - set(EXTRA_WORKLOADS)
+    if unknown:
+        ap.error(f"--extra: unknown workloads {sorted(unknown)}")
     dist, rank, world = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
